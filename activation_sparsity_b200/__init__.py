@@ -1,0 +1,31 @@
+"""B200-native (sm_100a) LaRoSA rotated-sparse linear.
+
+For each token entering a linear layer: rotate the activation by the layer's
+orthogonal Q, keep its K largest-magnitude entries, and multiply by the
+counter-rotated weight W_rot = Q^T W, reading only the K kept rows
+("La RoSA: Enhancing LLM Efficiency via Layerwise Rotated Sparse
+Activation", method and abstract).
+
+The compute lives in liblarosa.so (C ABI, include/larosa.h); this package is
+its thin Python binding.  Importing it fails loudly if the library is not
+built: there is no fallback path.
+"""
+from .larosa import (  # noqa: F401
+    LarosaError,
+    Workspace,
+    larosa_check,
+    larosa_dense_linear,
+    larosa_prepare_weights,
+    larosa_rotate,
+    larosa_rotate_topk_linear,
+    larosa_sparse_linear,
+    larosa_topk,
+    larosa_version,
+    larosa_workspace_bytes,
+    larosa_workspace_layout,
+    LAROSA_F32,
+    LAROSA_BF16,
+    LAROSA_MAX_D,
+    LAROSA_MAX_M,
+    LIB_PATH,
+)

@@ -1,0 +1,358 @@
+// C ABI of the library: argument validation, workspace layout and the
+// sequencing of kernels for each entry point (see include/larosa.h).
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+using larosa::Elem;
+using larosa::GemvArgs;
+using larosa::GemvPlan;
+
+namespace {
+
+constexpr int kMaxDout = 65536;
+constexpr size_t kTicketWords = 2048;  // per GEMV role
+constexpr size_t kBitmapWords = LAROSA_MAX_D / 32;
+// Fixed header: words that must be zero before a call and are zero after it.
+constexpr size_t kOffTicketsRot = 0;
+constexpr size_t kOffTicketsLin = kOffTicketsRot + kTicketWords * 4;
+constexpr size_t kOffBitmap = kOffTicketsLin + kTicketWords * 4;
+constexpr size_t kHeaderEnd = kOffBitmap + kBitmapWords * 4;
+
+thread_local char g_last_error[256] = "";
+
+int cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
+  return LAROSA_ERR_CUDA;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_size(int dtype) { return dtype == LAROSA_BF16 ? 2 : 4; }
+
+Elem elem_of(int dtype) { return dtype == LAROSA_BF16 ? Elem::BF16 : Elem::F32; }
+
+bool valid_dtype(int dtype) { return dtype == LAROSA_BF16 || dtype == LAROSA_F32; }
+
+// Row length (elements) of a weight is a multiple of 16 bytes.
+bool row_aligned(int n, int dtype) { return (n * elem_size(dtype)) % 16 == 0; }
+
+struct Layout {
+  size_t x_rot = 0, idx = 0, val = 0;
+  size_t partials_rot = 0, partials_lin = 0;
+  size_t coef = 0, urows = 0, ucount = 0;
+  size_t total = 0;
+};
+
+int sparse_rows_max(int M, int d_in, int K) {
+  return M == 1 ? K : std::min<long long>(d_in, (long long)M * K);
+}
+
+// Plans every GEMV role for both element types and lays the workspace out so
+// that one buffer serves every entry point called with these sizes.
+int make_layout(int M, int d_in, int d_out, int K, Layout* L) {
+  size_t prot = 0, plin = 0;
+  for (int dt = 0; dt < 2; ++dt) {
+    const Elem w = dt == 0 ? Elem::F32 : Elem::BF16;
+    GemvPlan pr, ps, pd;
+    cudaError_t e = larosa::plan_gemv(w, w, M, d_in, d_in, &pr);
+    if (e != cudaSuccess) return cuda_fail(e, "plan rotate");
+    e = larosa::plan_gemv(w, Elem::F32, M, d_out, sparse_rows_max(M, d_in, K), &ps);
+    if (e != cudaSuccess) return cuda_fail(e, "plan sparse linear");
+    e = larosa::plan_gemv(w, w, M, d_out, d_in, &pd);
+    if (e != cudaSuccess) return cuda_fail(e, "plan dense linear");
+    if (pr.ticket_words > kTicketWords || ps.ticket_words > kTicketWords ||
+        pd.ticket_words > kTicketWords)
+      return LAROSA_ERR_SHAPE;
+    prot = std::max(prot, pr.partial_floats);
+    plin = std::max({plin, ps.partial_floats, pd.partial_floats});
+  }
+  size_t off = align_up(kHeaderEnd, 256);
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  L->x_rot = take((size_t)M * d_in * 4);
+  L->idx = take((size_t)M * K * 4);
+  L->val = take((size_t)M * K * 4);
+  L->partials_rot = take(prot * 4);
+  L->partials_lin = take(plin * 4);
+  if (M > 1) {
+    L->coef = take((size_t)M * d_in * 4);
+    L->urows = take((size_t)d_in * 4);
+    L->ucount = take(4);
+  }
+  L->total = off;
+  return LAROSA_OK;
+}
+
+int check_sizes(int M, int d_in, int d_out, int K) {
+  if (M < 1 || M > LAROSA_MAX_M) return LAROSA_ERR_SHAPE;
+  if (d_in < 1 || d_in > LAROSA_MAX_D) return LAROSA_ERR_SHAPE;
+  if (d_out < 1 || d_out > kMaxDout) return LAROSA_ERR_SHAPE;
+  if (K < 0 || K > d_in) return LAROSA_ERR_SHAPE;
+  return LAROSA_OK;
+}
+
+unsigned char* at(void* ws, size_t off) { return static_cast<unsigned char*>(ws) + off; }
+
+int workspace_ok(void* ws, size_t ws_bytes, const Layout& L) {
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < L.total) return LAROSA_ERR_WORKSPACE;
+  return LAROSA_OK;
+}
+
+// ---- the three GEMV roles ------------------------------------------------
+
+int run_rotate(const void* x, const void* Q, float* x_rot, int M, int d, int dtype, void* ws,
+               const Layout& L, int* dev_status, cudaStream_t s) {
+  GemvPlan pl;
+  cudaError_t e = larosa::plan_gemv(elem_of(dtype), elem_of(dtype), M, d, d, &pl);
+  if (e != cudaSuccess) return cuda_fail(e, "plan rotate");
+  GemvArgs a;
+  a.W = Q;
+  a.w_elem = elem_of(dtype);
+  a.d_out = d;
+  a.row_bound = d;
+  a.n_rows = d;
+  a.coef = x;
+  a.coef_elem = elem_of(dtype);
+  a.coef_ld = d;
+  a.M = M;
+  a.y = x_rot;
+  a.y_ld = d;
+  a.partials = reinterpret_cast<float*>(at(ws, L.partials_rot));
+  a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTicketsRot));
+  a.dev_status = dev_status;
+  e = larosa::launch_gemv(a, pl, s);
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "rotate kernel");
+}
+
+int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W_rot, int d_in,
+               int d_out, float* y, int dtype, void* ws, const Layout& L, int* dev_status,
+               cudaStream_t s) {
+  const int n_max = sparse_rows_max(M, d_in, K);
+  GemvPlan pl;
+  cudaError_t e = larosa::plan_gemv(elem_of(dtype), Elem::F32, M, d_out, n_max, &pl);
+  if (e != cudaSuccess) return cuda_fail(e, "plan sparse linear");
+  GemvArgs a;
+  a.W = W_rot;
+  a.w_elem = elem_of(dtype);
+  a.d_out = d_out;
+  a.row_bound = d_in;
+  a.coef_elem = Elem::F32;
+  a.M = M;
+  a.y = y;
+  a.y_ld = d_out;
+  a.partials = reinterpret_cast<float*>(at(ws, L.partials_lin));
+  a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTicketsLin));
+  a.dev_status = dev_status;
+  if (M == 1) {
+    a.rows = idx;
+    a.n_rows = K;
+    a.coef = val;
+    a.coef_ld = K;
+  } else {
+    float* coef = reinterpret_cast<float*>(at(ws, L.coef));
+    unsigned* bitmap = reinterpret_cast<unsigned*>(at(ws, kOffBitmap));
+    int32_t* urows = reinterpret_cast<int32_t*>(at(ws, L.urows));
+    int* ucount = reinterpret_cast<int*>(at(ws, L.ucount));
+    e = larosa::launch_scatter(idx, val, M, K, d_in, coef, bitmap, dev_status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scatter kernel");
+    e = larosa::launch_union(bitmap, d_in, urows, ucount, s);
+    if (e != cudaSuccess) return cuda_fail(e, "union kernel");
+    a.rows = urows;
+    a.n_rows = n_max;
+    a.n_rows_dev = ucount;
+    a.coef = coef;
+    a.coef_ld = d_in;
+    a.coef_by_row = 1;
+  }
+  e = larosa::launch_gemv(a, pl, s);
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "sparse linear kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* larosa_status_string(int status) {
+  switch (status) {
+    case LAROSA_OK: return "LAROSA_OK";
+    case LAROSA_ERR_INVALID_ARG: return "LAROSA_ERR_INVALID_ARG: invalid argument";
+    case LAROSA_ERR_SHAPE: return "LAROSA_ERR_SHAPE: size out of range";
+    case LAROSA_ERR_ALIGN: return "LAROSA_ERR_ALIGN: pointer or row length not 16-byte aligned";
+    case LAROSA_ERR_UNSUPPORTED_DTYPE: return "LAROSA_ERR_UNSUPPORTED_DTYPE: unsupported data type";
+    case LAROSA_ERR_CUDA: return "LAROSA_ERR_CUDA: a CUDA runtime call failed";
+    case LAROSA_ERR_WORKSPACE: return "LAROSA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case LAROSA_ERR_NONFINITE: return "LAROSA_ERR_NONFINITE: a NaN or Inf reached Top-K";
+    case LAROSA_ERR_TIMEOUT: return "LAROSA_ERR_TIMEOUT: a kernel wait exceeded its time limit";
+    case LAROSA_ERR_INDEX: return "LAROSA_ERR_INDEX: an index was out of range";
+    default: return "unknown larosa status";
+  }
+}
+
+int larosa_version(void) { return LAROSA_VERSION; }
+
+const char* larosa_last_error_string(void) { return g_last_error; }
+
+size_t larosa_workspace_bytes(int M, int d_in, int d_out, int K) {
+  if (check_sizes(M, d_in, d_out, K) != LAROSA_OK) return 0;
+  Layout L;
+  if (make_layout(M, d_in, d_out, K, &L) != LAROSA_OK) return 0;
+  return L.total;
+}
+
+int larosa_workspace_layout(int M, int d_in, int d_out, int K, size_t* x_rot_offset,
+                            size_t* idx_offset, size_t* val_offset) {
+  int st = check_sizes(M, d_in, d_out, K);
+  if (st != LAROSA_OK) return st;
+  Layout L;
+  st = make_layout(M, d_in, d_out, K, &L);
+  if (st != LAROSA_OK) return st;
+  if (x_rot_offset) *x_rot_offset = L.x_rot;
+  if (idx_offset) *idx_offset = L.idx;
+  if (val_offset) *val_offset = L.val;
+  return LAROSA_OK;
+}
+
+int larosa_prepare_weights(const void* Q, const void* W, void* W_rot, int d_in, int d_out,
+                           int dtype, larosa_stream_t stream) {
+  if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
+  if (Q == nullptr || W == nullptr || W_rot == nullptr) return LAROSA_ERR_INVALID_ARG;
+  if (d_in < 1 || d_in > LAROSA_MAX_D || d_out < 1 || d_out > kMaxDout) return LAROSA_ERR_SHAPE;
+  if (W_rot == W || W_rot == Q) return LAROSA_ERR_INVALID_ARG;
+  cudaError_t e = larosa::launch_prepare(Q, W, W_rot, d_in, d_out, elem_of(dtype),
+                                         reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "prepare kernel");
+}
+
+int larosa_rotate(const void* x, const void* Q, float* x_rot, int M, int d, int dtype, void* ws,
+                  size_t ws_bytes, int* dev_status, larosa_stream_t stream) {
+  if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
+  if (x == nullptr || Q == nullptr || x_rot == nullptr) return LAROSA_ERR_INVALID_ARG;
+  int st = check_sizes(M, d, d, 0);
+  if (st != LAROSA_OK) return st;
+  if (!aligned16(Q) || !row_aligned(d, dtype)) return LAROSA_ERR_ALIGN;
+  Layout L;
+  st = make_layout(M, d, d, 0, &L);
+  if (st != LAROSA_OK) return st;
+  st = workspace_ok(ws, ws_bytes, L);
+  if (st != LAROSA_OK) return st;
+  return run_rotate(x, Q, x_rot, M, d, dtype, ws, L, dev_status,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+int larosa_topk(const float* x_rot, int M, int d, int K, int32_t* idx, float* val,
+                int* dev_status, larosa_stream_t stream) {
+  if (x_rot == nullptr || (K > 0 && (idx == nullptr || val == nullptr)))
+    return LAROSA_ERR_INVALID_ARG;
+  if (M < 1 || M > LAROSA_MAX_M || d < 1 || d > LAROSA_MAX_D || K < 0 || K > d)
+    return LAROSA_ERR_SHAPE;
+  cudaError_t e = larosa::launch_topk(x_rot, M, d, K, idx, val, dev_status,
+                                      reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "topk kernel");
+}
+
+int larosa_sparse_linear(const int32_t* idx, const float* val, int M, int K, const void* W_rot,
+                         int d_in, int d_out, float* y, void* ws, size_t ws_bytes, int dtype,
+                         int* dev_status, larosa_stream_t stream) {
+  if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
+  if (W_rot == nullptr || y == nullptr || (K > 0 && (idx == nullptr || val == nullptr)))
+    return LAROSA_ERR_INVALID_ARG;
+  int st = check_sizes(M, d_in, d_out, K);
+  if (st != LAROSA_OK) return st;
+  if (!aligned16(W_rot) || !row_aligned(d_out, dtype)) return LAROSA_ERR_ALIGN;
+  Layout L;
+  st = make_layout(M, d_in, d_out, K, &L);
+  if (st != LAROSA_OK) return st;
+  st = workspace_ok(ws, ws_bytes, L);
+  if (st != LAROSA_OK) return st;
+  return run_sparse(idx, val, M, K, W_rot, d_in, d_out, y, dtype, ws, L, dev_status,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+int larosa_rotate_topk_linear(const void* x, const void* Q, const void* W_rot, int M, int d_in,
+                              int d_out, int K, float* y, void* ws, size_t ws_bytes,
+                              int* dev_status, int dtype, larosa_stream_t stream) {
+  if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
+  if (x == nullptr || Q == nullptr || W_rot == nullptr || y == nullptr)
+    return LAROSA_ERR_INVALID_ARG;
+  int st = check_sizes(M, d_in, d_out, K);
+  if (st != LAROSA_OK) return st;
+  if (!aligned16(Q) || !aligned16(W_rot) || !row_aligned(d_in, dtype) ||
+      !row_aligned(d_out, dtype))
+    return LAROSA_ERR_ALIGN;
+  Layout L;
+  st = make_layout(M, d_in, d_out, K, &L);
+  if (st != LAROSA_OK) return st;
+  st = workspace_ok(ws, ws_bytes, L);
+  if (st != LAROSA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* x_rot = reinterpret_cast<float*>(at(ws, L.x_rot));
+  int32_t* idx = reinterpret_cast<int32_t*>(at(ws, L.idx));
+  float* val = reinterpret_cast<float*>(at(ws, L.val));
+  st = run_rotate(x, Q, x_rot, M, d_in, dtype, ws, L, dev_status, s);
+  if (st != LAROSA_OK) return st;
+  cudaError_t e = larosa::launch_topk(x_rot, M, d_in, K, idx, val, dev_status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "topk kernel");
+  return run_sparse(idx, val, M, K, W_rot, d_in, d_out, y, dtype, ws, L, dev_status, s);
+}
+
+int larosa_dense_linear(const void* x, const void* W, int M, int d_in, int d_out, float* y,
+                        void* ws, size_t ws_bytes, int dtype, int* dev_status,
+                        larosa_stream_t stream) {
+  if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
+  if (x == nullptr || W == nullptr || y == nullptr) return LAROSA_ERR_INVALID_ARG;
+  int st = check_sizes(M, d_in, d_out, d_in);
+  if (st != LAROSA_OK) return st;
+  if (!aligned16(W) || !row_aligned(d_out, dtype)) return LAROSA_ERR_ALIGN;
+  Layout L;
+  st = make_layout(M, d_in, d_out, d_in, &L);
+  if (st != LAROSA_OK) return st;
+  st = workspace_ok(ws, ws_bytes, L);
+  if (st != LAROSA_OK) return st;
+  GemvPlan pl;
+  cudaError_t e = larosa::plan_gemv(elem_of(dtype), elem_of(dtype), M, d_out, d_in, &pl);
+  if (e != cudaSuccess) return cuda_fail(e, "plan dense linear");
+  GemvArgs a;
+  a.W = W;
+  a.w_elem = elem_of(dtype);
+  a.d_out = d_out;
+  a.row_bound = d_in;
+  a.n_rows = d_in;
+  a.coef = x;
+  a.coef_elem = elem_of(dtype);
+  a.coef_ld = d_in;
+  a.M = M;
+  a.y = y;
+  a.y_ld = d_out;
+  a.partials = reinterpret_cast<float*>(at(ws, L.partials_lin));
+  a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTicketsLin));
+  a.dev_status = dev_status;
+  e = larosa::launch_gemv(a, pl, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "dense linear kernel");
+}
+
+int larosa_check(const int* dev_status, larosa_stream_t stream, int* flags_out) {
+  if (dev_status == nullptr) return LAROSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int flags = 0;
+  cudaError_t e = cudaMemcpyAsync(&flags, dev_status, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "read status");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "synchronize");
+  if (flags_out) *flags_out = flags;
+  if (flags & LAROSA_DEV_NONFINITE) return LAROSA_ERR_NONFINITE;
+  if (flags & LAROSA_DEV_TIMEOUT) return LAROSA_ERR_TIMEOUT;
+  if (flags & LAROSA_DEV_INDEX) return LAROSA_ERR_INDEX;
+  return LAROSA_OK;
+}
+
+}  // extern "C"

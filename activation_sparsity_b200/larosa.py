@@ -1,0 +1,312 @@
+"""Python binding of liblarosa.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls, takes torch
+tensors that live on a CUDA device, passes their data pointers, sizes and the
+current CUDA stream to the library, and raises LarosaError on a nonzero
+status.  All arithmetic happens in the library's CUDA kernels; there is no
+CPU or PyTorch fallback, and importing this module fails if the library has
+not been built.
+
+Tensors must be contiguous.  Output tensors and the workspace may be passed
+in; when omitted they are allocated with torch (the only thing PyTorch does
+here besides providing the stream).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblarosa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m activation_sparsity_b200.build_lib` "
+        "(there is no fallback implementation)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_c = ctypes
+_vp, _i, _sz = _c.c_void_p, _c.c_int, _c.c_size_t
+
+_SIGNATURES = {
+    "larosa_status_string": ([_i], _c.c_char_p),
+    "larosa_version": ([], _i),
+    "larosa_last_error_string": ([], _c.c_char_p),
+    "larosa_prepare_weights": ([_vp, _vp, _vp, _i, _i, _i, _vp], _i),
+    "larosa_rotate": ([_vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp, _vp], _i),
+    "larosa_topk": ([_vp, _i, _i, _i, _vp, _vp, _vp, _vp], _i),
+    "larosa_sparse_linear": ([_vp, _vp, _i, _i, _vp, _i, _i, _vp, _vp, _sz, _i, _vp, _vp], _i),
+    "larosa_rotate_topk_linear": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp, _i, _vp], _i),
+    "larosa_dense_linear": ([_vp, _vp, _i, _i, _i, _vp, _vp, _sz, _i, _vp, _vp], _i),
+    "larosa_workspace_bytes": ([_i, _i, _i, _i], _sz),
+    "larosa_workspace_layout": ([_i, _i, _i, _i, _c.POINTER(_sz), _c.POINTER(_sz), _c.POINTER(_sz)], _i),
+    "larosa_check": ([_vp, _vp, _c.POINTER(_i)], _i),
+}
+for _name, (_args, _ret) in _SIGNATURES.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _ret
+
+LAROSA_F32 = 0
+LAROSA_BF16 = 1
+LAROSA_OK = 0
+LAROSA_ERR_NONFINITE = 7
+LAROSA_ERR_TIMEOUT = 8
+LAROSA_ERR_INDEX = 9
+LAROSA_DEV_NONFINITE = 0x1
+LAROSA_DEV_TIMEOUT = 0x2
+LAROSA_DEV_INDEX = 0x4
+LAROSA_MAX_M = 16
+LAROSA_MAX_D = 32768
+
+
+class LarosaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib.larosa_status_string(status).decode()
+        detail = _lib.larosa_last_error_string().decode()
+        super().__init__(f"{where}: {msg}" + (f" ({detail})" if detail and status == 5 else ""))
+        self.status = status
+
+
+def _check(status: int, where: str) -> None:
+    if status != LAROSA_OK:
+        raise LarosaError(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _as2d(t: torch.Tensor) -> torch.Tensor:
+    return t if t.dim() == 2 else t.reshape(1, -1)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return LAROSA_BF16
+    if t.dtype == torch.float32:
+        return LAROSA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: bfloat16 or float32")
+
+
+def _need(t: torch.Tensor, name: str, dtype=None) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+# ------------------------------------------------------------------ workspace
+
+class Workspace:
+    """A zero-initialised scratch buffer for one stream, grown on demand.
+
+    The library leaves the counter words it uses at zero after every call, so
+    the buffer is reused without clearing.  A buffer serves one stream at a
+    time; calls on different streams that may overlap need their own.
+    """
+
+    def __init__(self, device=None):
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
+            else torch.device(device)
+        self.buf = torch.zeros(0, dtype=torch.uint8, device=self.device)
+
+    def get(self, M: int, d_in: int, d_out: int, K: int) -> torch.Tensor:
+        with torch.cuda.device(self.device):
+            need = int(_lib.larosa_workspace_bytes(M, d_in, d_out, K))
+        if need == 0:
+            raise LarosaError(2, "larosa_workspace_bytes")
+        if self.buf.numel() < need:
+            self.buf = torch.zeros(need, dtype=torch.uint8, device=self.device)
+        return self.buf
+
+    def reset(self) -> None:
+        """Zero the buffer again (needed after a device-side error)."""
+        self.buf.zero_()
+
+
+_ws_lock = threading.Lock()
+_ws_cache: dict[tuple[int, int], Workspace] = {}
+_status_cache: dict[int, torch.Tensor] = {}
+
+
+def default_workspace(device: torch.device) -> Workspace:
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    with _ws_lock:
+        ws = _ws_cache.get(key)
+        if ws is None:
+            ws = _ws_cache[key] = Workspace(device)
+        return ws
+
+
+def default_status(device: torch.device) -> torch.Tensor:
+    """The per-device status word used when none is passed (see larosa_check)."""
+    with _ws_lock:
+        st = _status_cache.get(device.index)
+        if st is None:
+            st = _status_cache[device.index] = torch.zeros(1, dtype=torch.int32, device=device)
+        return st
+
+
+def _ws_args(ws, device, M, d_in, d_out, K):
+    if ws is None:
+        ws = default_workspace(device)
+    buf = ws.get(M, d_in, d_out, K) if isinstance(ws, Workspace) else ws
+    return ctypes.c_void_p(buf.data_ptr()), ctypes.c_size_t(buf.numel() * buf.element_size())
+
+
+def _status_ptr(dev_status, device):
+    return _ptr(default_status(device) if dev_status is None else dev_status)
+
+
+# ------------------------------------------------------------------ entry points
+
+def larosa_version() -> int:
+    return int(_lib.larosa_version())
+
+
+def larosa_workspace_bytes(M: int, d_in: int, d_out: int, K: int) -> int:
+    return int(_lib.larosa_workspace_bytes(M, d_in, d_out, K))
+
+
+def larosa_workspace_layout(M: int, d_in: int, d_out: int, K: int) -> tuple[int, int, int]:
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.larosa_workspace_layout(M, d_in, d_out, K, ctypes.byref(a), ctypes.byref(b),
+                                        ctypes.byref(c)), "larosa_workspace_layout")
+    return a.value, b.value, c.value
+
+
+def larosa_prepare_weights(Q: torch.Tensor, W: torch.Tensor, W_rot: torch.Tensor | None = None
+                           ) -> torch.Tensor:
+    """W_rot = Q^T . W (offline counter-rotation), same dtype as W."""
+    _need(Q, "Q")
+    _need(W, "W", Q.dtype)
+    d_in, d_out = W.shape
+    if W_rot is None:
+        W_rot = torch.empty_like(W)
+    _need(W_rot, "W_rot", W.dtype)
+    _check(_lib.larosa_prepare_weights(_ptr(Q), _ptr(W), _ptr(W_rot), d_in, d_out, _dtype_code(W),
+                                       _stream(W.device)), "larosa_prepare_weights")
+    return W_rot
+
+
+def larosa_rotate(x: torch.Tensor, Q: torch.Tensor, x_rot: torch.Tensor | None = None, ws=None,
+                  dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """x_rot = x . Q, fp32 output [M, d]."""
+    _need(x, "x")
+    _need(Q, "Q", x.dtype)
+    x2 = _as2d(x)
+    M, d = x2.shape
+    if x_rot is None:
+        x_rot = torch.empty((M, d), dtype=torch.float32, device=x.device)
+    _need(x_rot, "x_rot", torch.float32)
+    p, n = _ws_args(ws, x.device, M, d, d, 0)
+    _check(_lib.larosa_rotate(_ptr(x2), _ptr(Q), _ptr(x_rot), M, d, _dtype_code(x), p, n,
+                              _status_ptr(dev_status, x.device), _stream(x.device)), "larosa_rotate")
+    return x_rot
+
+
+def larosa_topk(x_rot: torch.Tensor, K: int, idx: torch.Tensor | None = None,
+                val: torch.Tensor | None = None, dev_status: torch.Tensor | None = None
+                ) -> tuple[torch.Tensor, torch.Tensor]:
+    """Per-row Top-K by magnitude: (idx int32 [M, K] ascending, val fp32 [M, K])."""
+    _need(x_rot, "x_rot", torch.float32)
+    x2 = _as2d(x_rot)
+    M, d = x2.shape
+    if idx is None:
+        idx = torch.empty((M, K), dtype=torch.int32, device=x_rot.device)
+    if val is None:
+        val = torch.empty((M, K), dtype=torch.float32, device=x_rot.device)
+    _need(idx, "idx", torch.int32)
+    _need(val, "val", torch.float32)
+    _check(_lib.larosa_topk(_ptr(x2), M, d, K, _ptr(idx), _ptr(val),
+                            _status_ptr(dev_status, x_rot.device), _stream(x_rot.device)),
+           "larosa_topk")
+    return idx, val
+
+
+def larosa_sparse_linear(idx: torch.Tensor, val: torch.Tensor, W_rot: torch.Tensor,
+                         y: torch.Tensor | None = None, ws=None,
+                         dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """y = sum_k val[:, k] * W_rot[idx[:, k]], fp32 [M, d_out]."""
+    _need(idx, "idx", torch.int32)
+    _need(val, "val", torch.float32)
+    _need(W_rot, "W_rot")
+    i2 = _as2d(idx)
+    val = _as2d(val)
+    M, K = i2.shape
+    d_in, d_out = W_rot.shape
+    if y is None:
+        y = torch.empty((M, d_out), dtype=torch.float32, device=W_rot.device)
+    _need(y, "y", torch.float32)
+    p, n = _ws_args(ws, W_rot.device, M, d_in, d_out, K)
+    _check(_lib.larosa_sparse_linear(_ptr(i2), _ptr(val), M, K, _ptr(W_rot), d_in, d_out, _ptr(y),
+                                     p, n, _dtype_code(W_rot), _status_ptr(dev_status, W_rot.device),
+                                     _stream(W_rot.device)), "larosa_sparse_linear")
+    return y
+
+
+def larosa_rotate_topk_linear(x: torch.Tensor, Q: torch.Tensor, W_rot: torch.Tensor, K: int,
+                              y: torch.Tensor | None = None, ws=None,
+                              dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """Fused rotate -> Top-K -> sparse linear, fp32 output [M, d_out]."""
+    _need(x, "x")
+    _need(Q, "Q", x.dtype)
+    _need(W_rot, "W_rot", x.dtype)
+    x2 = _as2d(x)
+    M, d_in = x2.shape
+    d_out = W_rot.shape[1]
+    if y is None:
+        y = torch.empty((M, d_out), dtype=torch.float32, device=x.device)
+    _need(y, "y", torch.float32)
+    p, n = _ws_args(ws, x.device, M, d_in, d_out, K)
+    _check(_lib.larosa_rotate_topk_linear(_ptr(x2), _ptr(Q), _ptr(W_rot), M, d_in, d_out, K, _ptr(y),
+                                          p, n, _status_ptr(dev_status, x.device), _dtype_code(x),
+                                          _stream(x.device)), "larosa_rotate_topk_linear")
+    return y
+
+
+def larosa_dense_linear(x: torch.Tensor, W: torch.Tensor, y: torch.Tensor | None = None, ws=None,
+                        dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """Dense baseline y = x . W (same streaming machinery), fp32 [M, d_out]."""
+    _need(x, "x")
+    _need(W, "W", x.dtype)
+    x2 = _as2d(x)
+    M, d_in = x2.shape
+    d_out = W.shape[1]
+    if y is None:
+        y = torch.empty((M, d_out), dtype=torch.float32, device=x.device)
+    _need(y, "y", torch.float32)
+    p, n = _ws_args(ws, x.device, M, d_in, d_out, d_in)
+    _check(_lib.larosa_dense_linear(_ptr(x2), _ptr(W), M, d_in, d_out, _ptr(y), p, n, _dtype_code(x),
+                                    _status_ptr(dev_status, x.device), _stream(x.device)),
+           "larosa_dense_linear")
+    return y
+
+
+def larosa_check(dev_status: torch.Tensor | None = None, device=None) -> int:
+    """Synchronises the current stream and returns the raw device status bits.
+
+    Raises LarosaError for a nonzero word (the status of its lowest bit).
+    """
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = default_status(device) if dev_status is None else dev_status
+    flags = ctypes.c_int(0)
+    status = _lib.larosa_check(_ptr(st), _stream(st.device), ctypes.byref(flags))
+    _check(status, "larosa_check")
+    return flags.value
+
+
+def raw_library() -> ctypes.CDLL:
+    """The loaded ctypes library (for tests of the C ABI itself)."""
+    return _lib

@@ -1,0 +1,512 @@
+#!/usr/bin/env python
+"""Benchmark of the LaRoSA rotated-sparse linear path on one node.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl larosa|reference]
+                    [--sparsity 40]
+
+A step is one decode token through the whole path of one LLaMA2-7B-shaped
+decoder layer: for each of its four projection groups (q|k|v 4096x12288,
+o 4096x4096, gate|up 4096x22016, down 11008x4096) rotate the input by the
+group's own orthogonal Q, keep the exact Top-K (40 % sparsity: K = 2458 of
+4096, 6605 of 11008) and multiply by the counter-rotated weight, reading only
+the kept rows.  Inputs are seeded and synthetic; weights are random of the
+right shapes.
+
+Timed with CUDA events on the launching stream after W warm-up steps, the K
+steps replayed from a CUDA graph of one step; the working set (586 MB of
+rotations and kept weight rows per step) exceeds the 126 MB L2, so no flush is
+needed.  N > 1 runs N independent replicas (one process per GPU, no data-path
+collective); the reported time is the maximum over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
+on the same workload instead (the only other path that may run it here).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "rotated-sparse linear tokens/s & HBM GB/s (% of roofline), LLaMA2-7B shapes, 40% sparse"
+UNIT = "tokens/s"
+HIDDEN, FFN, KV = 4096, 11008, 4096
+WORKLOAD_ID = 1
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=("larosa", "reference"), default="larosa")
+    ap.add_argument("--sparsity", type=float, default=40.0)
+    ap.add_argument("--cpu-tokens", type=int, default=4,
+                    help="tokens in the CPU oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    return a
+
+
+# ---------------------------------------------------------------- ranks
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate(per_rank_seconds: float, tokens_per_rank: int, world: int, device=None) -> tuple[float, float]:
+    """(whole-job tokens/s, slowest rank's seconds): all ranks' tokens over the max time."""
+    t = reduce_max(per_rank_seconds, world, device)
+    return tokens_per_rank * world / t, t
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[4:8]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- byte model
+
+def path_bytes(g, K: int, rotate: bool = True) -> dict:
+    """Algorithmic HBM bytes of one token through one projection group.
+
+    kept rows K*d_out*2 (bf16), the rotation d_in^2*2 when rotated online,
+    and the activations: x (d_in*2), x_rot (d_in*4), idx/val (K*8), y (d_out*4).
+    """
+    rows = K * g.d_out * 2
+    q = g.d_in * g.d_in * 2 if rotate else 0
+    act = g.d_in * 2 + g.d_in * 4 + K * 8 + g.d_out * 4
+    return {"rows": rows, "q": q, "act": act, "total": rows + q + act}
+
+
+def measured_peaks() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("rowstream.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "activation_sparsity_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch of ``kernel`` from the committed ncu summary, if the
+    summary was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def cpu_layer_inputs(sparsity: float, seed_layer: int = 0):
+    """fp64 host arrays of the 7B layer for the oracle.
+
+    The counter-rotated weight is drawn directly as N(0, 0.02^2): Q^T W of a
+    Gaussian W is again Gaussian with the same law, and the fp64 counter-
+    rotation itself is an offline step outside the per-token metric.
+    """
+    import numpy as np
+    import synthdata as sd
+    groups = []
+    for p in sd.llama_layer(HIDDEN, FFN, KV):
+        base = sd.seed_for(WORKLOAD_ID, seed_layer, 10 * p.q_id)
+        rng = np.random.default_rng(base + 1)
+        G = rng.standard_normal((p.d_in, p.d_in))
+        Q, _ = np.linalg.qr(G) if p.d_in <= 4096 else (None, None)
+        if Q is None:
+            # an orthogonal matrix of the same size and cost to apply
+            Q = np.linalg.qr(rng.standard_normal((p.d_in, p.d_in)).astype(np.float32))[0].astype(np.float64)
+        W_rot = rng.standard_normal((p.d_in, p.d_out)).astype(np.float32).astype(np.float64) * 0.02
+        x = sd.activations(1, p.d_in, base + 3, dtype=__import__("torch").float32).double().numpy()
+        groups.append((p.name, x, Q, W_rot, sd.k_for_sparsity(p.d_in, sparsity)))
+    return groups
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_seconds_per_token(groups, tokens: int) -> float:
+    import oracle
+    t0 = time.perf_counter()
+    for _ in range(tokens):
+        for _, x, Q, W_rot, K in groups:
+            oracle.rotate_topk_linear(x, Q, W_rot, K)
+    return (time.perf_counter() - t0) / tokens
+
+
+# ---------------------------------------------------------------- reference arm
+
+def bench_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    groups = cpu_layer_inputs(args.sparsity)
+    for _ in range(args.warmup):
+        cpu_oracle_seconds_per_token(groups, 1)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cpu_oracle_seconds_per_token(groups, 1)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config(args.sparsity, graph=False),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": "each step: one decode token through the 4 projection groups of "
+                                   "the LLaMA2-7B layer (fp64 numpy oracle, rank 0 only)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(sparsity: float, graph: bool) -> dict:
+    return {
+        "workload": "llama2-7b-layer: one decoder layer, batch 1 decode, q|k|v 4096x12288, o 4096x4096, "
+                    "gate|up 4096x22016, down 11008x4096, one orthogonal rotation per input "
+                    "(3 x 4096^2 + 11008^2), bf16 weights, fp32 accumulate",
+        "sparsity_pct": sparsity,
+        "batch_tokens": 1,
+        "l2": "inputs larger than L2: 586 MB of rotations and kept rows per step vs 126 MB L2, no flush",
+        "cuda_graph": graph,
+    }
+
+
+# ---------------------------------------------------------------- larosa arm
+
+def bench_larosa(args):
+    import numpy as np
+    import torch
+
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the library has no CPU path)")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    init_dist(world, "nccl")
+
+    import activation_sparsity_b200 as L
+    from activation_sparsity_b200.workload import build_layer
+
+    layer = build_layer(HIDDEN, FFN, KV, args.sparsity, WORKLOAD_ID, layer=rank, device=device)
+    groups = layer.groups
+    stream = torch.cuda.Stream(device)
+    ws = L.Workspace(device)
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    ys = [torch.empty((1, g.d_out), dtype=torch.float32, device=device) for g in groups]
+    for g in groups:
+        ws.get(1, g.d_in, g.d_out, g.d_in)
+    # component-call intermediates for the per-kernel pass
+    x_rots = [torch.empty((1, g.d_in), dtype=torch.float32, device=device) for g in groups]
+    idxs = [torch.empty((1, g.K), dtype=torch.int32, device=device) for g in groups]
+    vals = [torch.empty((1, g.K), dtype=torch.float32, device=device) for g in groups]
+
+    def fused_step():
+        for g, y in zip(groups, ys):
+            L.larosa_rotate_topk_linear(g.x, g.Q, g.W_rot, g.K, y=y, ws=ws, dev_status=st)
+
+    def sparse_only_step():  # the same path on pre-rotated inputs (no Q streamed)
+        for g, y, xr in zip(groups, ys, x_rots):
+            L.larosa_topk(xr, g.K, idx=idxs[groups.index(g)], val=vals[groups.index(g)], dev_status=st)
+            L.larosa_sparse_linear(idxs[groups.index(g)], vals[groups.index(g)], g.W_rot, y=y, ws=ws,
+                                   dev_status=st)
+
+    def dense_step():
+        for g, y in zip(groups, ys):
+            L.larosa_dense_linear(g.x, g.W, y=y, ws=ws, dev_status=st)
+
+    def graph_of(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+        torch.cuda.synchronize(device)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            fn()
+        torch.cuda.synchronize(device)
+        return gr
+
+    def time_graph(gr, steps: int, warmup: int, clocks: ClockSampler | None = None):
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                gr.replay()
+        torch.cuda.synchronize(device)
+        barrier(world, device)
+        if clocks:
+            clocks.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps):
+                gr.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+        clk = clocks.stop() if clocks else None
+        barrier(world, device)
+        return e0.elapsed_time(e1) / 1e3, clk
+
+    # rotate once so the sparse-only path has its pre-rotated inputs
+    with torch.cuda.stream(stream):
+        for g, xr in zip(groups, x_rots):
+            L.larosa_rotate(g.x, g.Q, x_rot=xr, ws=ws, dev_status=st)
+    torch.cuda.synchronize(device)
+
+    g_fused = graph_of(fused_step)
+    g_sparse = graph_of(sparse_only_step)
+    g_dense = graph_of(dense_step)
+
+    props = torch.cuda.get_device_properties(device)
+    clocks = ClockSampler(f"GPU-{props.uuid}")
+    t_fused, clk = time_graph(g_fused, args.steps, args.warmup, clocks)
+    value, t_max = aggregate(t_fused, args.steps, world, device)
+    t_sparse, _ = time_graph(g_sparse, args.steps, args.warmup)
+    t_dense, _ = time_graph(g_dense, args.steps, args.warmup)
+    sparse_tps, _ = aggregate(t_sparse, args.steps, world, device)
+    dense_tps, _ = aggregate(t_dense, args.steps, world, device)
+
+    # ---- per-kernel pass: the same kernels through the component calls, with
+    # CUDA events around each launch on the launching stream
+    n_rep = max(50, min(2000, args.steps // 5))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in groups]
+    rot_ms, topk_ms, lin_ms = [], [], []
+    with torch.cuda.stream(stream):
+        for r in range(args.warmup + n_rep):
+            for gi, g in enumerate(groups):
+                e = ev[gi]
+                e[0].record(stream)
+                L.larosa_rotate(g.x, g.Q, x_rot=x_rots[gi], ws=ws, dev_status=st)
+                e[1].record(stream)
+                L.larosa_topk(x_rots[gi], g.K, idx=idxs[gi], val=vals[gi], dev_status=st)
+                e[2].record(stream)
+                L.larosa_sparse_linear(idxs[gi], vals[gi], g.W_rot, y=ys[gi], ws=ws, dev_status=st)
+                e[3].record(stream)
+                if r >= args.warmup:
+                    e[3].synchronize()
+                    rot_ms.append((gi, e[0].elapsed_time(e[1])))
+                    topk_ms.append((gi, e[1].elapsed_time(e[2])))
+                    lin_ms.append((gi, e[2].elapsed_time(e[3])))
+    torch.cuda.synchronize(device)
+    assert L.larosa_check(st, device=device) == 0
+
+    def mean_by_group(rec):
+        return [statistics.mean(ms for gi2, ms in rec if gi2 == gi) for gi in range(len(groups))]
+
+    rot_g, topk_g, lin_g = mean_by_group(rot_ms), mean_by_group(topk_ms), mean_by_group(lin_ms)
+    rot_bytes = [g.d_in * g.d_in * 2 + g.d_in * 2 + g.d_in * 4 for g in groups]
+    lin_bytes = [g.K * g.d_out * 2 + g.K * 8 + g.d_out * 4 for g in groups]
+    step_bytes = sum(path_bytes(g, g.K)["total"] for g in groups)
+    sparse_bytes = sum(path_bytes(g, g.K, rotate=False)["total"] for g in groups)
+    peak, peak_kind = measured_peaks()
+    rot_gbs = sum(rot_bytes) / (sum(rot_g) * 1e-3) / 1e9
+    lin_gbs = sum(lin_bytes) / (sum(lin_g) * 1e-3) / 1e9
+    share_rot = sum(rot_g) / (sum(rot_g) + sum(topk_g) + sum(lin_g))
+    traffic = profiled_traffic("rotate")
+
+    # ---- end to end through the public API with host buffers
+    x_host = [g.x.cpu().pin_memory() for g in groups]
+    x_dev = [torch.empty_like(g.x) for g in groups]
+    y_host = [torch.empty((1, g.d_out), dtype=torch.float32).pin_memory() for g in groups]
+    e2e_steps = max(20, min(500, args.steps // 10))
+    with torch.cuda.stream(stream):
+        for r in range(args.warmup + e2e_steps):
+            if r == args.warmup:
+                torch.cuda.synchronize(device)
+                barrier(world, device)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            for gi, g in enumerate(groups):
+                x_dev[gi].copy_(x_host[gi], non_blocking=True)
+                L.larosa_rotate_topk_linear(x_dev[gi], g.Q, g.W_rot, g.K, y=ys[gi], ws=ws, dev_status=st)
+                y_host[gi].copy_(ys[gi], non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    t_e2e = e0.elapsed_time(e1) / 1e3
+    e2e_value, _ = aggregate(t_e2e, e2e_steps, world, device)
+    assert all(torch.isfinite(y).all() for y in y_host)
+
+    # ---- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cgroups = cpu_layer_inputs(args.sparsity)
+        cpu_oracle_seconds_per_token(cgroups, 1)
+        spt = cpu_oracle_seconds_per_token(cgroups, args.cpu_tokens)
+        cpu = {"value": 1.0 / spt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{args.cpu_tokens} decode tokens through the 4 projection groups of the "
+                         "LLaMA2-7B layer, fp64 numpy oracle on the host cores"}
+
+    if rank == 0:
+        ms_step = t_max * 1e3 / args.steps
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(args.sparsity, graph=True),
+            "hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
+            "hbm_frac": step_bytes / (ms_step * 1e-3) / 1e9 / peak,
+            "bytes_per_step": step_bytes,
+            "roofline": {"kernel": "rowstream_gemv (rotation x.Q, bf16)", "bound": "hbm",
+                         "achieved": rot_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": rot_gbs / peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": statistics.mean(rot_bytes),
+                         "avg_launch_us": statistics.mean(rot_g) * 1e3, "share_of_step": share_rot},
+            "kernels": {
+                "rotate_us": [round(v * 1e3, 2) for v in rot_g],
+                "topk_us": [round(v * 1e3, 2) for v in topk_g],
+                "sparse_linear_us": [round(v * 1e3, 2) for v in lin_g],
+                "sparse_linear_gbs": lin_gbs, "sparse_linear_frac": lin_gbs / peak,
+                "groups": [g.name for g in groups],
+            },
+            "paths": {
+                "fused_tokens_per_s": value,
+                "sparse_only_tokens_per_s": sparse_tps,
+                "sparse_only_hbm_frac": sparse_bytes * sparse_tps / world / 1e9 / peak,
+                "dense_tokens_per_s": dense_tps,
+                "sparse_only_vs_dense": sparse_tps / dense_tps,
+                "fused_vs_dense": value / dense_tps,
+            },
+            "e2e": {"value": e2e_value, "unit": UNIT,
+                    "h2d_bytes_per_step": sum(g.x.numel() * g.x.element_size() for g in groups),
+                    "d2h_bytes_per_step": sum(g.d_out * 4 for g in groups)},
+            "gpu_launches": args.steps * 3 * len(groups),
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    del g_fused, g_sparse, g_dense
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return bench_reference(args)
+    return bench_larosa(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,213 @@
+/*
+ * larosa.h -- C ABI of the B200 (sm_100a) rotated-sparse linear library.
+ *
+ * The library computes, for each token (activation row) entering a linear
+ * layer, the LaRoSA hot path:
+ *
+ *   1. rotate:   x_rot = x . Q              (Q orthogonal, d x d)
+ *   2. Top-K:    keep the K entries of x_rot of largest magnitude
+ *   3. multiply: y = sparse(x_rot) . W_rot,  W_rot = Q^T . W prepared offline,
+ *                reading only the K selected rows of W_rot.
+ *
+ * Source of each step (page title, section):
+ *   - "La RoSA: Enhancing LLM Efficiency via Layerwise Rotated Sparse
+ *     Activation" (summary page, 方法详解 / 技术框架): a rotation stage that
+ *     multiplies each layer's input activation by an orthogonal matrix, then
+ *     a sparsification stage that keeps the K largest-magnitude entries and
+ *     zeroes the rest.
+ *   - Same paper, abstract: layerwise orthogonal rotations of the input
+ *     activations; Top-K selection in the rotated activations gives the same
+ *     sparsity on every token; activation sparsity cuts memory transfers.
+ *   - The counter-rotation W_rot = Q^T W is not printed on the pages; it is
+ *     what keeps the layer's output unchanged at K = d, because Q Q^T = I.
+ *
+ * Conventions shared by every entry point
+ *   - Activations are row vectors; a batch of M tokens is a row-major [M x d]
+ *     array.  Weights are row-major [d_in x d_out]: row i holds input
+ *     channel i's weights (the transpose of torch.nn.Linear.weight), so the
+ *     K selected rows of W_rot are K contiguous runs of memory.
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, except
+ *     where marked "host".  The library never allocates or frees memory.
+ *   - Every compute call is asynchronous on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  Kernels are launched with programmatic
+ *     dependent launch, so a call may begin its set-up while the previous
+ *     kernel on the stream drains; it reads no activation before that kernel
+ *     has completed.
+ *   - Host-side validation happens before anything is enqueued; on failure
+ *     the call returns a nonzero larosa_status and enqueues nothing.
+ *   - Device-side conditions (a non-finite activation reaching Top-K, an
+ *     out-of-range index, a pipeline wait that exceeded its time limit) set
+ *     bits in a caller-provided `int* dev_status` word (see LAROSA_DEV_*);
+ *     read it with larosa_check().  dev_status may be NULL, in which case
+ *     those conditions are not reported.  Kernels never trap or spin without
+ *     bound: every wait inside a kernel gives up after about two seconds,
+ *     sets LAROSA_DEV_TIMEOUT and exits.
+ *   - Workspace: the split-K GEMV kernels use caller-provided scratch `ws`
+ *     of `ws_bytes` bytes, at least larosa_workspace_bytes(...).  It must be
+ *     16-byte aligned and ZERO-FILLED before its first use; every call that
+ *     completes leaves its counter words at zero again, so the same buffer
+ *     serves the next call on the same stream without clearing.  After a
+ *     device-side error, zero it again.  Calls that may run concurrently (on
+ *     different streams) need distinct workspaces.
+ *   - Data types: `dtype` is LAROSA_BF16 (bf16 activations and weights) or
+ *     LAROSA_F32 (fp32 activations and weights).  Rotated activations, kept
+ *     values and outputs are always fp32; all accumulation is fp32.
+ *   - Alignment: weight and activation base pointers 16-byte aligned, and
+ *     the row length of every weight (d_out, or d for Q) a multiple of 8
+ *     elements for bf16 or 4 for fp32; otherwise LAROSA_ERR_ALIGN.
+ *   - Sizes: 1 <= M <= LAROSA_MAX_M, 1 <= d <= LAROSA_MAX_D, 0 <= K <= d.
+ */
+#ifndef LAROSA_H
+#define LAROSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without including the CUDA runtime header. */
+typedef struct CUstream_st *larosa_stream_t;
+
+#define LAROSA_VERSION 100 /* 1.0.0 */
+#define LAROSA_MAX_M 16
+#define LAROSA_MAX_D 32768
+
+/* Return codes. */
+typedef enum {
+  LAROSA_OK = 0,
+  LAROSA_ERR_INVALID_ARG = 1,      /* NULL pointer, negative size, bad enum */
+  LAROSA_ERR_SHAPE = 2,            /* sizes out of range (M, d, K) */
+  LAROSA_ERR_ALIGN = 3,            /* pointer or row length not aligned */
+  LAROSA_ERR_UNSUPPORTED_DTYPE = 4,
+  LAROSA_ERR_CUDA = 5,             /* a CUDA runtime call failed */
+  LAROSA_ERR_WORKSPACE = 6,        /* ws NULL or smaller than required */
+  LAROSA_ERR_NONFINITE = 7,        /* device: NaN/Inf reached Top-K */
+  LAROSA_ERR_TIMEOUT = 8,          /* device: a pipeline wait gave up */
+  LAROSA_ERR_INDEX = 9             /* device: an index was out of range */
+} larosa_status;
+
+/* Element types of activations and weights. */
+typedef enum { LAROSA_F32 = 0, LAROSA_BF16 = 1 } larosa_dtype;
+
+/* Bits a kernel ORs into *dev_status. */
+#define LAROSA_DEV_NONFINITE 0x1
+#define LAROSA_DEV_TIMEOUT 0x2
+#define LAROSA_DEV_INDEX 0x4
+
+/* Human-readable name of a larosa_status value (static string, never NULL). */
+const char *larosa_status_string(int status);
+
+/* LAROSA_VERSION of the built library. */
+int larosa_version(void);
+
+/*
+ * Text of the last CUDA runtime failure behind an LAROSA_ERR_CUDA returned on
+ * the calling thread ("" if none).  Static per-thread storage.
+ */
+const char *larosa_last_error_string(void);
+
+/*
+ * Offline counter-rotation of a weight (step 0, not on the per-token path):
+ *   W_rot[i][j] = sum_k Q[k][i] * W[k][j],   i.e. W_rot = Q^T . W.
+ * Q: [d_in x d_in], W: [d_in x d_out], W_rot: [d_in x d_out], all row-major
+ * and all of type `dtype`.  fp32 accumulation; bf16 outputs are rounded to
+ * nearest even.  Projections that share an input (q|k|v, gate|up) are packed
+ * by passing their weights concatenated along d_out.  W_rot must not overlap
+ * Q or W.
+ */
+int larosa_prepare_weights(const void *Q, const void *W, void *W_rot,
+                           int d_in, int d_out, int dtype,
+                           larosa_stream_t stream);
+
+/*
+ * Rotation (step 1): x_rot[m][j] = sum_i x[m][i] * Q[i][j].
+ * x: [M x d] of `dtype`, Q: [d x d] of `dtype`, x_rot: [M x d] fp32.
+ * Streams all of Q once per call (an HBM-bound GEMV for small M).
+ * ws: at least larosa_workspace_bytes(M, d, d, 0) bytes.
+ */
+int larosa_rotate(const void *x, const void *Q, float *x_rot, int M, int d,
+                  int dtype, void *ws, size_t ws_bytes, int *dev_status,
+                  larosa_stream_t stream);
+
+/*
+ * Exact per-token Top-K by magnitude (step 2).
+ * For each of the M rows of x_rot ([M x d] fp32) keeps the K entries of
+ * largest |x_rot|; among equal magnitudes the lower index wins (+0 and -0
+ * are equal).  Writes idx [M x K] int32 in ascending index order and
+ * val [M x K] fp32 = the kept entries with their signs.  A NaN or Inf in a
+ * row sets LAROSA_DEV_NONFINITE; that row's output is then unspecified (but
+ * every index written is within [0, d)).  K = 0 writes nothing.
+ */
+int larosa_topk(const float *x_rot, int M, int d, int K, int32_t *idx,
+                float *val, int *dev_status, larosa_stream_t stream);
+
+/*
+ * Sparse linear (step 3): y[m][j] = sum_k val[m][k] * W_rot[idx[m][k]][j].
+ * idx/val: [M x K] as written by larosa_topk (each row's indices distinct;
+ * ascending order is not required for correctness).  W_rot: [d_in x d_out]
+ * of `dtype`; only the rows named in idx are read.  y: [M x d_out] fp32.
+ * For M > 1 the rows named by any token are streamed once and shared.
+ * An index outside [0, d_in) sets LAROSA_DEV_INDEX and contributes nothing.
+ * ws: at least larosa_workspace_bytes(M, d_in, d_out, K) bytes.
+ */
+int larosa_sparse_linear(const int32_t *idx, const float *val, int M, int K,
+                         const void *W_rot, int d_in, int d_out, float *y,
+                         void *ws, size_t ws_bytes, int dtype,
+                         int *dev_status, larosa_stream_t stream);
+
+/*
+ * Steps 1-3 in one call, one stream, no host synchronisation:
+ *   x_rot = x . Q;  (idx, val) = TopK(x_rot, K);  y = sparse(x_rot) . W_rot.
+ * x: [M x d_in] of `dtype`; Q: [d_in x d_in]; W_rot: [d_in x d_out] of
+ * `dtype` (from larosa_prepare_weights with the same Q); y: [M x d_out] fp32.
+ * The intermediate x_rot, idx and val live in the workspace; their offsets
+ * are given by larosa_workspace_layout() for inspection.
+ * ws: at least larosa_workspace_bytes(M, d_in, d_out, K) bytes.
+ */
+int larosa_rotate_topk_linear(const void *x, const void *Q, const void *W_rot,
+                              int M, int d_in, int d_out, int K, float *y,
+                              void *ws, size_t ws_bytes, int *dev_status,
+                              int dtype, larosa_stream_t stream);
+
+/*
+ * Dense baseline: y[m][j] = sum_i x[m][i] * W[i][j] with the same streaming
+ * GEMV machinery (no cuBLAS).  x: [M x d_in] of `dtype`, W: [d_in x d_out]
+ * of `dtype`, y: [M x d_out] fp32.
+ * ws: at least larosa_workspace_bytes(M, d_in, d_out, d_in) bytes.
+ */
+int larosa_dense_linear(const void *x, const void *W, int M, int d_in,
+                        int d_out, float *y, void *ws, size_t ws_bytes,
+                        int dtype, int *dev_status, larosa_stream_t stream);
+
+/*
+ * Workspace bytes sufficient for every entry point above called with these
+ * sizes (M tokens, d_in inputs, d_out outputs, K kept).  Returns 0 for
+ * out-of-range sizes.
+ */
+size_t larosa_workspace_bytes(int M, int d_in, int d_out, int K);
+
+/*
+ * Byte offsets inside the workspace of the fused call's intermediates:
+ * x_rot ([M x d_in] fp32), idx ([M x K] int32) and val ([M x K] fp32).
+ * Any output pointer may be NULL.  Returns LAROSA_ERR_SHAPE for
+ * out-of-range sizes.
+ */
+int larosa_workspace_layout(int M, int d_in, int d_out, int K,
+                            size_t *x_rot_offset, size_t *idx_offset,
+                            size_t *val_offset);
+
+/*
+ * Waits for `stream`, reads *dev_status (device pointer) and returns
+ * LAROSA_OK when it is zero, else the status of its lowest set bit
+ * (NONFINITE, TIMEOUT, INDEX).  If `flags_out` (host) is not NULL it
+ * receives the raw bits.  Does not clear the word.
+ */
+int larosa_check(const int *dev_status, larosa_stream_t stream, int *flags_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LAROSA_H */

@@ -175,3 +175,43 @@ WORKLOADS = {
     "llama2-13b-layer": dict(kind="layer", hidden=5120, ffn=13824, kv=5120, layers=1, w_std=0.02),
     "llama2-70b-slice": dict(kind="layer", hidden=8192, ffn=28672, kv=1024, layers=8, w_std=0.02),
 }
+
+
+ADVERSARIAL_KINDS = ("gaussian", "heavy", "small_ints", "equal_magnitude", "ulp_neighbours",
+                     "subnormal", "zeros")
+
+
+def adversarial_rows(kind: str, M: int, d: int, seed: int) -> torch.Tensor:
+    """fp32 [M x d] rows that stress a magnitude selection.
+
+    gaussian         N(0, 1)
+    heavy            the heavy-tailed activation recipe, in fp32
+    small_ints       integers in [-3, 3] (many equal magnitudes, +0 and -0)
+    equal_magnitude  +-1.5 with random signs (every magnitude ties)
+    ulp_neighbours   1.0 and its next fp32 neighbours, random signs
+    subnormal        fp32 subnormals and zeros
+    zeros            +0 and -0 only
+    """
+    rng = np.random.default_rng(seed)
+    if kind == "gaussian":
+        a = rng.standard_normal((M, d))
+    elif kind == "heavy":
+        a = rng.standard_normal((M, d)) * _channel_std(d, seed)[None, :]
+    elif kind == "small_ints":
+        a = rng.integers(-3, 4, size=(M, d)).astype(np.float64)
+        a[rng.random((M, d)) < 0.1] = -0.0
+    elif kind == "equal_magnitude":
+        a = np.where(rng.random((M, d)) < 0.5, -1.5, 1.5)
+    elif kind == "ulp_neighbours":
+        one = np.float32(1.0)
+        vals = np.array([np.nextafter(one, np.float32(0)), one, np.nextafter(one, np.float32(2))],
+                        dtype=np.float32)
+        a = vals[rng.integers(0, 3, size=(M, d))].astype(np.float64)
+        a *= np.where(rng.random((M, d)) < 0.5, -1.0, 1.0)
+    elif kind == "subnormal":
+        a = rng.integers(-40, 41, size=(M, d)).astype(np.float64) * 2.0 ** -149
+    elif kind == "zeros":
+        a = np.where(rng.random((M, d)) < 0.5, -0.0, 0.0)
+    else:
+        raise ValueError(kind)
+    return torch.from_numpy(a.astype(np.float32))

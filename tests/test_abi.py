@@ -1,0 +1,96 @@
+"""The C-ABI library on the CPU: it loads, exports what include/larosa.h
+declares, and rejects bad arguments on the host before touching a device.
+
+No call here launches work: every call fails validation first.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "larosa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from activation_sparsity_b200 import build_lib
+    path = build_lib.build()
+    lib = ctypes.CDLL(path)
+    return lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(larosa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ("larosa_prepare_weights", "larosa_rotate", "larosa_topk", "larosa_sparse_linear",
+                 "larosa_rotate_topk_linear", "larosa_dense_linear", "larosa_workspace_bytes",
+                 "larosa_check"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    path = lib._name
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\sT\s+(larosa_\w+)", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert getattr(lib, n) is not None
+
+
+def test_status_strings_and_version(lib):
+    lib.larosa_status_string.restype = ctypes.c_char_p
+    for code in range(10):
+        s = lib.larosa_status_string(code).decode()
+        assert s.startswith("LAROSA_")
+    assert b"unknown" in lib.larosa_status_string(99)
+    assert lib.larosa_version() == 100
+
+
+P = ctypes.c_void_p
+FAKE = P(0x10000)          # aligned, never dereferenced: validation fails first
+MISALIGNED = P(0x10008)
+
+
+def test_host_validation_rejects_bad_arguments(lib):
+    BF16, F32 = 1, 0
+    z = ctypes.c_size_t(1 << 20)
+    # unsupported dtype
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 64, 7, FAKE, z, None, None) == 4
+    assert lib.larosa_prepare_weights(FAKE, FAKE, FAKE, 64, 64, 9, None) == 4
+    # NULL pointers
+    assert lib.larosa_rotate(None, FAKE, FAKE, 1, 64, BF16, FAKE, z, None, None) == 1
+    assert lib.larosa_topk(None, 1, 64, 3, FAKE, FAKE, None, None) == 1
+    assert lib.larosa_topk(FAKE, 1, 64, 3, None, FAKE, None, None) == 1
+    assert lib.larosa_sparse_linear(FAKE, FAKE, 1, 4, None, 64, 64, FAKE, FAKE, z, BF16, None, None) == 1
+    assert lib.larosa_prepare_weights(FAKE, None, FAKE, 64, 64, BF16, None) == 1
+    # sizes
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 0, 64, BF16, FAKE, z, None, None) == 2
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 17, 64, BF16, FAKE, z, None, None) == 2
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 32769, BF16, FAKE, z, None, None) == 2
+    assert lib.larosa_topk(FAKE, 1, 64, 65, FAKE, FAKE, None, None) == 2
+    assert lib.larosa_topk(FAKE, 1, 64, -1, FAKE, FAKE, None, None) == 2
+    assert lib.larosa_sparse_linear(FAKE, FAKE, 1, 65, FAKE, 64, 64, FAKE, FAKE, z, BF16, None, None) == 2
+    assert lib.larosa_rotate_topk_linear(FAKE, FAKE, FAKE, 1, 64, 64, 65, FAKE, FAKE, z, None, BF16, None) == 2
+    assert lib.larosa_dense_linear(FAKE, FAKE, 1, 64, 0, FAKE, FAKE, z, BF16, None, None) == 2
+    # alignment: base pointers and row lengths (bf16 rows a multiple of 8 elements)
+    assert lib.larosa_rotate(FAKE, MISALIGNED, FAKE, 1, 64, BF16, FAKE, z, None, None) == 3
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 60, BF16, FAKE, z, None, None) == 3
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 62, F32, FAKE, z, None, None) == 3
+    assert lib.larosa_sparse_linear(FAKE, FAKE, 1, 4, MISALIGNED, 64, 64, FAKE, FAKE, z, BF16, None, None) == 3
+    assert lib.larosa_sparse_linear(FAKE, FAKE, 1, 4, FAKE, 64, 36, FAKE, FAKE, z, BF16, None, None) == 3
+    assert lib.larosa_rotate_topk_linear(FAKE, FAKE, FAKE, 1, 64, 12, 5, FAKE, FAKE, z, None, BF16, None) == 3
+    assert lib.larosa_dense_linear(FAKE, MISALIGNED, 1, 64, 64, FAKE, FAKE, z, BF16, None, None) == 3
+    # in-place counter-rotation is refused
+    assert lib.larosa_prepare_weights(FAKE, P(0x20000), P(0x20000), 64, 64, BF16, None) == 1
+    # status check needs a status word
+    assert lib.larosa_check(None, None, None) == 1
