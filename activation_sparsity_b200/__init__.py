@@ -6,26 +6,23 @@ counter-rotated weight W_rot = Q^T W, reading only the K kept rows
 ("La RoSA: Enhancing LLM Efficiency via Layerwise Rotated Sparse
 Activation", method and abstract).
 
-The compute lives in liblarosa.so (C ABI, include/larosa.h); this package is
-its thin Python binding.  Importing it fails loudly if the library is not
-built: there is no fallback path.
+The compute lives in liblarosa.so (C ABI, include/larosa.h); the submodule
+``larosa`` is its thin Python binding and is loaded on first use of any name
+below.  Loading fails loudly if the library is not built: there is no
+fallback path.  (``build_lib`` builds the library without loading it.)
 """
-from .larosa import (  # noqa: F401
-    LarosaError,
-    Workspace,
-    larosa_check,
-    larosa_dense_linear,
-    larosa_prepare_weights,
-    larosa_rotate,
-    larosa_rotate_topk_linear,
-    larosa_sparse_linear,
-    larosa_topk,
-    larosa_version,
-    larosa_workspace_bytes,
-    larosa_workspace_layout,
-    LAROSA_F32,
-    LAROSA_BF16,
-    LAROSA_MAX_D,
-    LAROSA_MAX_M,
-    LIB_PATH,
+_EXPORTS = (
+    "LarosaError", "Workspace", "larosa_check", "larosa_dense_linear", "larosa_prepare_weights",
+    "larosa_rotate", "larosa_rotate_topk_linear", "larosa_sparse_linear",
+    "larosa_topk", "larosa_version", "larosa_workspace_bytes",
+    "larosa_workspace_layout", "LAROSA_F32", "LAROSA_BF16", "LAROSA_MAX_D", "LAROSA_MAX_M",
+    "LIB_PATH",
 )
+__all__ = list(_EXPORTS)
+
+
+def __getattr__(name):
+    if name in _EXPORTS:
+        from . import larosa
+        return getattr(larosa, name)
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")
