@@ -180,6 +180,12 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
 
 }  // namespace
 
+namespace larosa {
+// Lets other translation units of the library report a message through
+// larosa_last_error_string().
+void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+}  // namespace larosa
+
 extern "C" {
 
 const char* larosa_status_string(int status) {

@@ -1,0 +1,151 @@
+// Sparse linear for callers that cannot hand the library a workspace.
+//
+// Some callers cannot allocate device memory on the path where they call the
+// library: an operator slot in another runtime that passes only inputs and
+// outputs and owns every allocation itself, or a latency-critical loop in
+// which cudaMalloc and cudaFree are forbidden because they may synchronise
+// the device.  For them larosa_sparse_linear_noalloc computes exactly what
+// larosa_sparse_linear computes, with the same kernels and launch geometry,
+// but keeps the split-K partial sums, the reduction tickets and (for several
+// tokens) the shared-row bookkeeping in one file-scope device array of fixed
+// size instead of a caller workspace.
+//
+// That array exists once per GPU that loads this library and stays resident
+// until the process exits.  Every call on a device uses the same array, so
+// calls whose work may overlap on that GPU (different streams, or different
+// host threads) race with each other; serialise them.  The array keeps
+// whatever the last call left in it; the words that must start at zero are
+// cleared by each call with cudaMemsetAsync on the caller's stream.
+#include <stdio.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace larosa {
+void set_last_error(const char* msg);
+}
+
+namespace {
+
+constexpr size_t kScratchBytes = size_t(2) << 20;  // 2 MiB per device
+constexpr int kMaxDevices = 64;
+constexpr int kMaxDout = 65536;
+
+static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+
+std::mutex g_mu;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_scratch on the current device, looked up once per
+// device with that device current (host code cannot use the symbol itself).
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+size_t up256(size_t v) { return (v + 255) / 256 * 256; }
+
+int fail_cuda(cudaError_t e, const char* where) {
+  char buf[200];
+  snprintf(buf, sizeof(buf), "larosa_sparse_linear_noalloc: %s: %s", where, cudaGetErrorString(e));
+  larosa::set_last_error(buf);
+  return LAROSA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val, int M, int K,
+                                            const void* W_rot, int d_in, int d_out, float* y,
+                                            int dtype, int* dev_status, larosa_stream_t stream) {
+  if (dtype != LAROSA_BF16 && dtype != LAROSA_F32) return LAROSA_ERR_UNSUPPORTED_DTYPE;
+  if (W_rot == nullptr || y == nullptr || (K > 0 && (idx == nullptr || val == nullptr)))
+    return LAROSA_ERR_INVALID_ARG;
+  if (M < 1 || M > LAROSA_MAX_M || d_in < 1 || d_in > LAROSA_MAX_D || d_out < 1 ||
+      d_out > kMaxDout || K < 0 || K > d_in)
+    return LAROSA_ERR_SHAPE;
+  const int esz = dtype == LAROSA_BF16 ? 2 : 4;
+  if ((reinterpret_cast<uintptr_t>(W_rot) & 15u) != 0 || (d_out * esz) % 16 != 0)
+    return LAROSA_ERR_ALIGN;
+
+  const larosa::Elem w = dtype == LAROSA_BF16 ? larosa::Elem::BF16 : larosa::Elem::F32;
+  const int n_max = M == 1 ? K : (int)std::min<long long>(d_in, (long long)M * K);
+  larosa::GemvPlan pl;
+  cudaError_t e = larosa::plan_gemv(w, larosa::Elem::F32, M, d_out, n_max, &pl);
+  if (e != cudaSuccess) return fail_cuda(e, "plan");
+
+  // scratch layout: [tickets][bitmap][partials][coef][rows][count]
+  const size_t bitmap_words = M > 1 ? (size_t)(d_in + 31) / 32 : 0;
+  const size_t off_bitmap = up256(pl.ticket_words * 4);
+  const size_t zero_bytes = off_bitmap + bitmap_words * 4;  // cleared every call
+  const size_t off_partials = up256(zero_bytes);
+  const size_t off_coef = up256(off_partials + pl.partial_floats * 4);
+  const size_t off_rows = up256(off_coef + (M > 1 ? (size_t)M * d_in * 4 : 0));
+  const size_t off_count = up256(off_rows + (M > 1 ? (size_t)d_in * 4 : 0));
+  const size_t total = off_count + 4;
+  if (total > kScratchBytes) {
+    char buf[200];
+    snprintf(buf, sizeof(buf),
+             "larosa_sparse_linear_noalloc: these sizes need %zu bytes of scratch; the static "
+             "scratch holds %zu",
+             total, kScratchBytes);
+    larosa::set_last_error(buf);
+    return LAROSA_ERR_WORKSPACE;
+  }
+
+  unsigned char* base = nullptr;
+  e = scratch_address(reinterpret_cast<void**>(&base));
+  if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  e = cudaMemsetAsync(base, 0, zero_bytes, s);
+  if (e != cudaSuccess) return fail_cuda(e, "clear scratch");
+
+  larosa::GemvArgs a;
+  a.W = W_rot;
+  a.w_elem = w;
+  a.d_out = d_out;
+  a.row_bound = d_in;
+  a.coef_elem = larosa::Elem::F32;
+  a.M = M;
+  a.y = y;
+  a.y_ld = d_out;
+  a.partials = reinterpret_cast<float*>(base + off_partials);
+  a.tickets = reinterpret_cast<unsigned*>(base);
+  a.dev_status = dev_status;
+  if (M == 1) {
+    a.rows = idx;
+    a.n_rows = K;
+    a.coef = val;
+    a.coef_ld = K;
+  } else {
+    float* coef = reinterpret_cast<float*>(base + off_coef);
+    unsigned* bitmap = reinterpret_cast<unsigned*>(base + off_bitmap);
+    int32_t* rows = reinterpret_cast<int32_t*>(base + off_rows);
+    int* count = reinterpret_cast<int*>(base + off_count);
+    e = larosa::launch_scatter(idx, val, M, K, d_in, coef, bitmap, dev_status, s);
+    if (e != cudaSuccess) return fail_cuda(e, "scatter kernel");
+    e = larosa::launch_union(bitmap, d_in, rows, count, s);
+    if (e != cudaSuccess) return fail_cuda(e, "union kernel");
+    a.rows = rows;
+    a.n_rows = n_max;
+    a.n_rows_dev = count;
+    a.coef = coef;
+    a.coef_ld = d_in;
+    a.coef_by_row = 1;
+  }
+  e = larosa::launch_gemv(a, pl, s);
+  return e == cudaSuccess ? LAROSA_OK : fail_cuda(e, "sparse linear kernel");
+}

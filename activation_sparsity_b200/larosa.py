@@ -42,6 +42,7 @@ _SIGNATURES = {
     "larosa_sparse_linear": ([_vp, _vp, _i, _i, _vp, _i, _i, _vp, _vp, _sz, _i, _vp, _vp], _i),
     "larosa_rotate_topk_linear": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp, _i, _vp], _i),
     "larosa_dense_linear": ([_vp, _vp, _i, _i, _i, _vp, _vp, _sz, _i, _vp, _vp], _i),
+    "larosa_sparse_linear_noalloc": ([_vp, _vp, _i, _i, _vp, _i, _i, _vp, _i, _vp, _vp], _i),
     "larosa_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "larosa_workspace_layout": ([_i, _i, _i, _i, _c.POINTER(_sz), _c.POINTER(_sz), _c.POINTER(_sz)], _i),
     "larosa_check": ([_vp, _vp, _c.POINTER(_i)], _i),
@@ -253,6 +254,32 @@ def larosa_sparse_linear(idx: torch.Tensor, val: torch.Tensor, W_rot: torch.Tens
     _check(_lib.larosa_sparse_linear(_ptr(i2), _ptr(val), M, K, _ptr(W_rot), d_in, d_out, _ptr(y),
                                      p, n, _dtype_code(W_rot), _status_ptr(dev_status, W_rot.device),
                                      _stream(W_rot.device)), "larosa_sparse_linear")
+    return y
+
+
+def larosa_sparse_linear_noalloc(idx: torch.Tensor, val: torch.Tensor, W_rot: torch.Tensor,
+                                 y: torch.Tensor | None = None,
+                                 dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """larosa_sparse_linear with the library's fixed device scratch instead of a
+    workspace (for callers that cannot allocate); calls on one device must not
+    overlap."""
+    _need(idx, "idx", torch.int32)
+    _need(val, "val", torch.float32)
+    _need(W_rot, "W_rot")
+    i2 = _as2d(idx)
+    val = _as2d(val)
+    M, K = i2.shape
+    d_in, d_out = W_rot.shape
+    if y is None:
+        y = torch.empty((M, d_out), dtype=torch.float32, device=W_rot.device)
+    _need(y, "y", torch.float32)
+    status = _lib.larosa_sparse_linear_noalloc(_ptr(i2), _ptr(val), M, K, _ptr(W_rot), d_in, d_out,
+                                               _ptr(y), _dtype_code(W_rot),
+                                               _status_ptr(dev_status, W_rot.device),
+                                               _stream(W_rot.device))
+    if status != LAROSA_OK:
+        raise LarosaError(status, "larosa_sparse_linear_noalloc: "
+                          + _lib.larosa_last_error_string().decode())
     return y
 
 

@@ -182,6 +182,31 @@ int larosa_dense_linear(const void *x, const void *W, int M, int d_in,
                         int dtype, int *dev_status, larosa_stream_t stream);
 
 /*
+ * larosa_sparse_linear without a workspace, for callers that cannot allocate
+ * device memory where they call the library: an operator slot in another
+ * runtime that passes only inputs and outputs, or a latency-critical loop in
+ * which cudaMalloc/cudaFree (which may synchronise the device) are not
+ * allowed.  The LaRoSA pages have no counterpart: this is a deployment
+ * variant of step 3, computing the same y with the same kernels.
+ *
+ * Arguments as for larosa_sparse_linear, minus ws/ws_bytes.  The split-K
+ * scratch lives in a 2 MiB file-scope device array that every GPU loading
+ * the library holds until the process exits.  Sizes whose scratch would
+ * exceed it (in practice only large multi-token batches, e.g. M = 16 with
+ * d_in = 32768) return LAROSA_ERR_WORKSPACE with the byte counts in
+ * larosa_last_error_string().  The call allocates nothing; it clears the
+ * words that must start at zero with cudaMemsetAsync on `stream`.  All calls
+ * on one device share the array, so calls that may overlap on that GPU race:
+ * serialise them.  The first call on each device looks up the array's device
+ * address and sizes its kernels (host-side CUDA queries); make that first
+ * call before any stream capture.
+ */
+int larosa_sparse_linear_noalloc(const int32_t *idx, const float *val, int M,
+                                 int K, const void *W_rot, int d_in, int d_out,
+                                 float *y, int dtype, int *dev_status,
+                                 larosa_stream_t stream);
+
+/*
  * Workspace bytes sufficient for every entry point above called with these
  * sizes (M tokens, d_in inputs, d_out outputs, K kept).  Returns 0 for
  * out-of-range sizes.
