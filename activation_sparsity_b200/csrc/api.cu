@@ -1,9 +1,17 @@
 // C ABI of the library: argument validation, workspace layout and the
 // sequencing of kernels for each entry point (see include/larosa.h).
+//
+//   rotation, dense baseline   rowdot (onetoken.cu), any M <= 16
+//   Top-K alone                topk_kernel (topk.cu)
+//   sparse linear, M = 1       gather over idx/val (onetoken.cu)
+//   sparse linear, M > 1       scatter + union (union.cu) + rowstream (rowstream.cu)
+//   fused, M = 1               rowdot -> select-and-gather: two kernels
+//   fused, M > 1               rowdot -> topk -> scatter/union -> rowstream
 #include <stdio.h>
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -15,12 +23,11 @@ using larosa::GemvPlan;
 namespace {
 
 constexpr int kMaxDout = 65536;
-constexpr size_t kTicketWords = 2048;  // per GEMV role
+constexpr size_t kTicketWords = 2048;
 constexpr size_t kBitmapWords = LAROSA_MAX_D / 32;
 // Fixed header: words that must be zero before a call and are zero after it.
-constexpr size_t kOffTicketsRot = 0;
-constexpr size_t kOffTicketsLin = kOffTicketsRot + kTicketWords * 4;
-constexpr size_t kOffBitmap = kOffTicketsLin + kTicketWords * 4;
+constexpr size_t kOffTickets = 0;
+constexpr size_t kOffBitmap = kOffTickets + kTicketWords * 4;
 constexpr size_t kHeaderEnd = kOffBitmap + kBitmapWords * 4;
 
 thread_local char g_last_error[256] = "";
@@ -40,38 +47,74 @@ Elem elem_of(int dtype) { return dtype == LAROSA_BF16 ? Elem::BF16 : Elem::F32; 
 
 bool valid_dtype(int dtype) { return dtype == LAROSA_BF16 || dtype == LAROSA_F32; }
 
-// Row length (elements) of a weight is a multiple of 16 bytes.
+// Row length (elements) of a row-major weight is a multiple of 16 bytes.
 bool row_aligned(int n, int dtype) { return (n * elem_size(dtype)) % 16 == 0; }
 
 struct Layout {
   size_t x_rot = 0, idx = 0, val = 0;
-  size_t partials_rot = 0, partials_lin = 0;
+  size_t partials = 0;
   size_t coef = 0, urows = 0, ucount = 0;
   size_t total = 0;
 };
 
 int sparse_rows_max(int M, int d_in, int K) {
-  return M == 1 ? K : std::min<long long>(d_in, (long long)M * K);
+  return M == 1 ? K : (int)std::min<long long>(d_in, (long long)M * K);
 }
 
-// Plans every GEMV role for both element types and lays the workspace out so
-// that one buffer serves every entry point called with these sizes.
+int make_layout_uncached(int M, int d_in, int d_out, int K, Layout* L);
+
+// Layouts already computed, per device and sizes.
+struct LayoutEntry {
+  int dev, M, d_in, d_out, K;
+  Layout L;
+};
+std::mutex g_layout_mu;
+LayoutEntry g_layouts[256];
+int g_layout_n = 0;
+int g_layout_next = 0;
+
+// One workspace layout serves every entry point called with these sizes.
 int make_layout(int M, int d_in, int d_out, int K, Layout* L) {
-  size_t prot = 0, plin = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  {
+    std::lock_guard<std::mutex> lock(g_layout_mu);
+    for (int i = 0; i < g_layout_n; ++i) {
+      const LayoutEntry& en = g_layouts[i];
+      if (en.dev == dev && en.M == M && en.d_in == d_in && en.d_out == d_out && en.K == K) {
+        *L = en.L;
+        return LAROSA_OK;
+      }
+    }
+  }
+  const int st = make_layout_uncached(M, d_in, d_out, K, L);
+  if (st != LAROSA_OK) return st;
+  std::lock_guard<std::mutex> lock(g_layout_mu);
+  LayoutEntry& en = g_layouts[g_layout_n < 256 ? g_layout_n++ : (g_layout_next++ & 255)];
+  en = LayoutEntry{dev, M, d_in, d_out, K, *L};
+  return LAROSA_OK;
+}
+
+int make_layout_uncached(int M, int d_in, int d_out, int K, Layout* L) {
+  size_t partials = 0;
   for (int dt = 0; dt < 2; ++dt) {
     const Elem w = dt == 0 ? Elem::F32 : Elem::BF16;
-    GemvPlan pr, ps, pd;
-    cudaError_t e = larosa::plan_gemv(w, w, M, d_in, d_in, &pr);
-    if (e != cudaSuccess) return cuda_fail(e, "plan rotate");
-    e = larosa::plan_gemv(w, Elem::F32, M, d_out, sparse_rows_max(M, d_in, K), &ps);
+    if (M == 1) {
+      larosa::StreamPlan sp;
+      cudaError_t e = larosa::plan_gather(w, d_out, K, &sp);
+      if (e != cudaSuccess) return cuda_fail(e, "plan gather");
+      if (sp.ok) {
+        if (sp.ticket_words > kTicketWords) return LAROSA_ERR_SHAPE;
+        partials = std::max(partials, sp.partial_floats);
+        continue;
+      }
+    }
+    GemvPlan ps;
+    cudaError_t e = larosa::plan_gemv(w, Elem::F32, M, d_out, sparse_rows_max(M, d_in, K), &ps);
     if (e != cudaSuccess) return cuda_fail(e, "plan sparse linear");
-    e = larosa::plan_gemv(w, w, M, d_out, d_in, &pd);
-    if (e != cudaSuccess) return cuda_fail(e, "plan dense linear");
-    if (pr.ticket_words > kTicketWords || ps.ticket_words > kTicketWords ||
-        pd.ticket_words > kTicketWords)
-      return LAROSA_ERR_SHAPE;
-    prot = std::max(prot, pr.partial_floats);
-    plin = std::max({plin, ps.partial_floats, pd.partial_floats});
+    if (ps.ticket_words > kTicketWords) return LAROSA_ERR_SHAPE;
+    partials = std::max(partials, ps.partial_floats);
   }
   size_t off = align_up(kHeaderEnd, 256);
   auto take = [&](size_t bytes) {
@@ -82,8 +125,7 @@ int make_layout(int M, int d_in, int d_out, int K, Layout* L) {
   L->x_rot = take((size_t)M * d_in * 4);
   L->idx = take((size_t)M * K * 4);
   L->val = take((size_t)M * K * 4);
-  L->partials_rot = take(prot * 4);
-  L->partials_lin = take(plin * 4);
+  L->partials = take(partials * 4);
   if (M > 1) {
     L->coef = take((size_t)M * d_in * 4);
     L->urows = take((size_t)d_in * 4);
@@ -108,35 +150,40 @@ int workspace_ok(void* ws, size_t ws_bytes, const Layout& L) {
   return LAROSA_OK;
 }
 
-// ---- the three GEMV roles ------------------------------------------------
+// Row-dot operands: rows of n_in elements, n_in a multiple of 8.
+bool rowdot_aligned(const void* A, const void* x, int n_in) {
+  return aligned16(A) && aligned16(x) && (n_in % 8) == 0;
+}
 
-int run_rotate(const void* x, const void* Q, float* x_rot, int M, int d, int dtype, void* ws,
-               const Layout& L, int* dev_status, cudaStream_t s) {
-  GemvPlan pl;
-  cudaError_t e = larosa::plan_gemv(elem_of(dtype), elem_of(dtype), M, d, d, &pl);
-  if (e != cudaSuccess) return cuda_fail(e, "plan rotate");
-  GemvArgs a;
-  a.W = Q;
-  a.w_elem = elem_of(dtype);
-  a.d_out = d;
-  a.row_bound = d;
-  a.n_rows = d;
-  a.coef = x;
-  a.coef_elem = elem_of(dtype);
-  a.coef_ld = d;
-  a.M = M;
-  a.y = x_rot;
-  a.y_ld = d;
-  a.partials = reinterpret_cast<float*>(at(ws, L.partials_rot));
-  a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTicketsRot));
-  a.dev_status = dev_status;
-  e = larosa::launch_gemv(a, pl, s);
-  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "rotate kernel");
+int run_rowdot(const void* x, const void* A, float* y, int M, int n_in, int n_out, int dtype,
+               cudaStream_t s, const char* what) {
+  cudaError_t e = larosa::launch_rowdot(elem_of(dtype), A, x, y, M, n_in, n_out, s);
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, what);
 }
 
 int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W_rot, int d_in,
                int d_out, float* y, int dtype, void* ws, const Layout& L, int* dev_status,
                cudaStream_t s) {
+  if (M == 1) {
+    larosa::StreamPlan sp;
+    cudaError_t e = larosa::plan_gather(elem_of(dtype), d_out, K, &sp);
+    if (e != cudaSuccess) return cuda_fail(e, "plan gather");
+    if (sp.ok) {
+      larosa::GatherArgs a;
+      a.W = W_rot;
+      a.d_out = d_out;
+      a.row_bound = d_in;
+      a.n = K;
+      a.coef = val;
+      a.rows = idx;
+      a.y = y;
+      a.partials = reinterpret_cast<float*>(at(ws, L.partials));
+      a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTickets));
+      a.dev_status = dev_status;
+      e = larosa::launch_gather(larosa::kGatherList, elem_of(dtype), a, sp, s);
+      return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "gather kernel");
+    }
+  }
   const int n_max = sparse_rows_max(M, d_in, K);
   GemvPlan pl;
   cudaError_t e = larosa::plan_gemv(elem_of(dtype), Elem::F32, M, d_out, n_max, &pl);
@@ -150,8 +197,8 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
   a.M = M;
   a.y = y;
   a.y_ld = d_out;
-  a.partials = reinterpret_cast<float*>(at(ws, L.partials_lin));
-  a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTicketsLin));
+  a.partials = reinterpret_cast<float*>(at(ws, L.partials));
+  a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTickets));
   a.dev_status = dev_status;
   if (M == 1) {
     a.rows = idx;
@@ -228,31 +275,26 @@ int larosa_workspace_layout(int M, int d_in, int d_out, int K, size_t* x_rot_off
   return LAROSA_OK;
 }
 
-int larosa_prepare_weights(const void* Q, const void* W, void* W_rot, int d_in, int d_out,
+int larosa_prepare_weights(const void* Qt, const void* W, void* W_rot, int d_in, int d_out,
                            int dtype, larosa_stream_t stream) {
   if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
-  if (Q == nullptr || W == nullptr || W_rot == nullptr) return LAROSA_ERR_INVALID_ARG;
+  if (Qt == nullptr || W == nullptr || W_rot == nullptr) return LAROSA_ERR_INVALID_ARG;
   if (d_in < 1 || d_in > LAROSA_MAX_D || d_out < 1 || d_out > kMaxDout) return LAROSA_ERR_SHAPE;
-  if (W_rot == W || W_rot == Q) return LAROSA_ERR_INVALID_ARG;
-  cudaError_t e = larosa::launch_prepare(Q, W, W_rot, d_in, d_out, elem_of(dtype),
+  if (W_rot == W || W_rot == Qt) return LAROSA_ERR_INVALID_ARG;
+  cudaError_t e = larosa::launch_prepare(Qt, W, W_rot, d_in, d_out, elem_of(dtype),
                                          reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "prepare kernel");
 }
 
-int larosa_rotate(const void* x, const void* Q, float* x_rot, int M, int d, int dtype, void* ws,
-                  size_t ws_bytes, int* dev_status, larosa_stream_t stream) {
+int larosa_rotate(const void* x, const void* Qt, float* x_rot, int M, int d, int dtype,
+                  larosa_stream_t stream) {
   if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
-  if (x == nullptr || Q == nullptr || x_rot == nullptr) return LAROSA_ERR_INVALID_ARG;
-  int st = check_sizes(M, d, d, 0);
+  if (x == nullptr || Qt == nullptr || x_rot == nullptr) return LAROSA_ERR_INVALID_ARG;
+  const int st = check_sizes(M, d, d, 0);
   if (st != LAROSA_OK) return st;
-  if (!aligned16(Q) || !row_aligned(d, dtype)) return LAROSA_ERR_ALIGN;
-  Layout L;
-  st = make_layout(M, d, d, 0, &L);
-  if (st != LAROSA_OK) return st;
-  st = workspace_ok(ws, ws_bytes, L);
-  if (st != LAROSA_OK) return st;
-  return run_rotate(x, Q, x_rot, M, d, dtype, ws, L, dev_status,
-                    reinterpret_cast<cudaStream_t>(stream));
+  if (!rowdot_aligned(Qt, x, d)) return LAROSA_ERR_ALIGN;
+  return run_rowdot(x, Qt, x_rot, M, d, d, dtype, reinterpret_cast<cudaStream_t>(stream),
+                    "rotation kernel");
 }
 
 int larosa_topk(const float* x_rot, int M, int d, int K, int32_t* idx, float* val,
@@ -274,7 +316,7 @@ int larosa_sparse_linear(const int32_t* idx, const float* val, int M, int K, con
     return LAROSA_ERR_INVALID_ARG;
   int st = check_sizes(M, d_in, d_out, K);
   if (st != LAROSA_OK) return st;
-  if (!aligned16(W_rot) || !row_aligned(d_out, dtype)) return LAROSA_ERR_ALIGN;
+  if (!aligned16(W_rot) || !aligned16(y) || !row_aligned(d_out, dtype)) return LAROSA_ERR_ALIGN;
   Layout L;
   st = make_layout(M, d_in, d_out, K, &L);
   if (st != LAROSA_OK) return st;
@@ -284,15 +326,15 @@ int larosa_sparse_linear(const int32_t* idx, const float* val, int M, int K, con
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
-int larosa_rotate_topk_linear(const void* x, const void* Q, const void* W_rot, int M, int d_in,
+int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, int M, int d_in,
                               int d_out, int K, float* y, void* ws, size_t ws_bytes,
                               int* dev_status, int dtype, larosa_stream_t stream) {
   if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
-  if (x == nullptr || Q == nullptr || W_rot == nullptr || y == nullptr)
+  if (x == nullptr || Qt == nullptr || W_rot == nullptr || y == nullptr)
     return LAROSA_ERR_INVALID_ARG;
   int st = check_sizes(M, d_in, d_out, K);
   if (st != LAROSA_OK) return st;
-  if (!aligned16(Q) || !aligned16(W_rot) || !row_aligned(d_in, dtype) ||
+  if (!rowdot_aligned(Qt, x, d_in) || !aligned16(W_rot) || !aligned16(y) ||
       !row_aligned(d_out, dtype))
     return LAROSA_ERR_ALIGN;
   Layout L;
@@ -304,46 +346,44 @@ int larosa_rotate_topk_linear(const void* x, const void* Q, const void* W_rot, i
   float* x_rot = reinterpret_cast<float*>(at(ws, L.x_rot));
   int32_t* idx = reinterpret_cast<int32_t*>(at(ws, L.idx));
   float* val = reinterpret_cast<float*>(at(ws, L.val));
-  st = run_rotate(x, Q, x_rot, M, d_in, dtype, ws, L, dev_status, s);
+  st = run_rowdot(x, Qt, x_rot, M, d_in, d_in, dtype, s, "rotation kernel");
   if (st != LAROSA_OK) return st;
+  if (M == 1) {
+    // every CTA of the gather selects the Top-K of x_rot on its own
+    larosa::StreamPlan sp;
+    cudaError_t e = larosa::plan_gather(elem_of(dtype), d_out, K, &sp);
+    if (e != cudaSuccess) return cuda_fail(e, "plan gather");
+    if (sp.ok) {
+      larosa::GatherArgs a;
+      a.W = W_rot;
+      a.d_out = d_out;
+      a.row_bound = d_in;
+      a.n = K;
+      a.coef = x_rot;
+      a.y = y;
+      a.partials = reinterpret_cast<float*>(at(ws, L.partials));
+      a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTickets));
+      a.idx_out = idx;
+      a.val_out = val;
+      a.dev_status = dev_status;
+      e = larosa::launch_gather(larosa::kGatherSelect, elem_of(dtype), a, sp, s);
+      return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "select-gather kernel");
+    }
+  }
   cudaError_t e = larosa::launch_topk(x_rot, M, d_in, K, idx, val, dev_status, s);
   if (e != cudaSuccess) return cuda_fail(e, "topk kernel");
   return run_sparse(idx, val, M, K, W_rot, d_in, d_out, y, dtype, ws, L, dev_status, s);
 }
 
-int larosa_dense_linear(const void* x, const void* W, int M, int d_in, int d_out, float* y,
-                        void* ws, size_t ws_bytes, int dtype, int* dev_status,
-                        larosa_stream_t stream) {
+int larosa_dense_linear(const void* x, const void* Wt, int M, int d_in, int d_out, float* y,
+                        int dtype, larosa_stream_t stream) {
   if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
-  if (x == nullptr || W == nullptr || y == nullptr) return LAROSA_ERR_INVALID_ARG;
-  int st = check_sizes(M, d_in, d_out, d_in);
+  if (x == nullptr || Wt == nullptr || y == nullptr) return LAROSA_ERR_INVALID_ARG;
+  const int st = check_sizes(M, d_in, d_out, d_in);
   if (st != LAROSA_OK) return st;
-  if (!aligned16(W) || !row_aligned(d_out, dtype)) return LAROSA_ERR_ALIGN;
-  Layout L;
-  st = make_layout(M, d_in, d_out, d_in, &L);
-  if (st != LAROSA_OK) return st;
-  st = workspace_ok(ws, ws_bytes, L);
-  if (st != LAROSA_OK) return st;
-  GemvPlan pl;
-  cudaError_t e = larosa::plan_gemv(elem_of(dtype), elem_of(dtype), M, d_out, d_in, &pl);
-  if (e != cudaSuccess) return cuda_fail(e, "plan dense linear");
-  GemvArgs a;
-  a.W = W;
-  a.w_elem = elem_of(dtype);
-  a.d_out = d_out;
-  a.row_bound = d_in;
-  a.n_rows = d_in;
-  a.coef = x;
-  a.coef_elem = elem_of(dtype);
-  a.coef_ld = d_in;
-  a.M = M;
-  a.y = y;
-  a.y_ld = d_out;
-  a.partials = reinterpret_cast<float*>(at(ws, L.partials_lin));
-  a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTicketsLin));
-  a.dev_status = dev_status;
-  e = larosa::launch_gemv(a, pl, reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "dense linear kernel");
+  if (!rowdot_aligned(Wt, x, d_in)) return LAROSA_ERR_ALIGN;
+  return run_rowdot(x, Wt, y, M, d_in, d_out, dtype, reinterpret_cast<cudaStream_t>(stream),
+                    "dense kernel");
 }
 
 int larosa_check(const int* dev_status, larosa_stream_t stream, int* flags_out) {

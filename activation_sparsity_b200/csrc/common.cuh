@@ -8,7 +8,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/larosa.h"
+#include "larosa.h"
 
 namespace larosa {
 

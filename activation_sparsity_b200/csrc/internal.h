@@ -68,7 +68,49 @@ cudaError_t launch_scatter(const int32_t* idx, const float* val, int M, int K, i
 cudaError_t launch_union(unsigned* bitmap, int d_in, int32_t* rows, int* count,
                          cudaStream_t stream);
 
-// W_rot = Q^T W.
+// Geometry of the one-token gather (see onetoken.cu).
+struct StreamPlan {
+  bool ok = false;
+  int grid = 0;            // CTAs (one per SM, fewer for tiny problems)
+  int col_tile = 0;        // output columns per tile
+  int tpr = 0;             // threads per weight row
+  int n_tiles = 0;
+  int max_slots = 0;       // partial slots per tile
+  size_t partial_floats = 0;
+  size_t ticket_words = 0;
+};
+
+struct GatherArgs {
+  const void* W = nullptr;  // [d_in x d_out] row-major
+  int d_out = 0;
+  int row_bound = 0;        // d_in
+  int n = 0;                // list length K
+  const void* coef = nullptr;     // kGatherList: val[K]; kGatherSelect: x_rot[d_in]
+  const int32_t* rows = nullptr;  // kGatherList: idx[K]
+  float* y = nullptr;
+  float* partials = nullptr;
+  unsigned* tickets = nullptr;
+  int32_t* idx_out = nullptr;     // kGatherSelect: kept indices / values (optional)
+  float* val_out = nullptr;
+  int* dev_status = nullptr;
+};
+
+constexpr int kGatherList = 1;    // rows idx[], coefficients val[]
+constexpr int kGatherSelect = 2;  // select the top-K of x_rot, then gather
+
+// Plans a one-token gather over an n-row list and d_out columns; plan->ok is
+// false when the shape exceeds the kernel's limits.
+cudaError_t plan_gather(Elem w_elem, int d_out, int n, StreamPlan* plan);
+cudaError_t launch_gather(int mode, Elem w_elem, const GatherArgs& a, const StreamPlan& plan,
+                          cudaStream_t stream);
+
+// Row-dot GEMV y[m][j] = sum_i x[m][i] A[j][i] for M <= 16 tokens, A row-major
+// [n_out x n_in] (the rotation through Q^T, or a dense layer in
+// torch.nn.Linear layout).  n_in a multiple of 8; x and A 16-byte aligned.
+cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M, int n_in,
+                          int n_out, cudaStream_t stream);
+
+// W_rot = Qt . W with Qt = Q^T given row-major.
 cudaError_t launch_prepare(const void* Q, const void* W, void* W_rot, int d_in, int d_out,
                            Elem elem, cudaStream_t stream);
 

@@ -78,10 +78,48 @@ extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val
       d_out > kMaxDout || K < 0 || K > d_in)
     return LAROSA_ERR_SHAPE;
   const int esz = dtype == LAROSA_BF16 ? 2 : 4;
-  if ((reinterpret_cast<uintptr_t>(W_rot) & 15u) != 0 || (d_out * esz) % 16 != 0)
+  if ((reinterpret_cast<uintptr_t>(W_rot) & 15u) != 0 ||
+      (reinterpret_cast<uintptr_t>(y) & 15u) != 0 || (d_out * esz) % 16 != 0)
     return LAROSA_ERR_ALIGN;
 
   const larosa::Elem w = dtype == LAROSA_BF16 ? larosa::Elem::BF16 : larosa::Elem::F32;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (M == 1) {
+    larosa::StreamPlan sp;
+    cudaError_t e = larosa::plan_gather(w, d_out, K, &sp);
+    if (e != cudaSuccess) return fail_cuda(e, "plan");
+    if (sp.ok) {
+      const size_t off_partials = up256(sp.ticket_words * 4);
+      const size_t total = off_partials + sp.partial_floats * 4;
+      if (total > kScratchBytes) {
+        char buf[200];
+        snprintf(buf, sizeof(buf),
+                 "larosa_sparse_linear_noalloc: these sizes need %zu bytes of scratch; the "
+                 "static scratch holds %zu",
+                 total, kScratchBytes);
+        larosa::set_last_error(buf);
+        return LAROSA_ERR_WORKSPACE;
+      }
+      unsigned char* base = nullptr;
+      e = scratch_address(reinterpret_cast<void**>(&base));
+      if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress");
+      e = cudaMemsetAsync(base, 0, sp.ticket_words * 4, s);
+      if (e != cudaSuccess) return fail_cuda(e, "clear scratch");
+      larosa::GatherArgs a;
+      a.W = W_rot;
+      a.d_out = d_out;
+      a.row_bound = d_in;
+      a.n = K;
+      a.coef = val;
+      a.rows = idx;
+      a.y = y;
+      a.partials = reinterpret_cast<float*>(base + off_partials);
+      a.tickets = reinterpret_cast<unsigned*>(base);
+      a.dev_status = dev_status;
+      e = larosa::launch_gather(larosa::kGatherList, w, a, sp, s);
+      return e == cudaSuccess ? LAROSA_OK : fail_cuda(e, "sparse linear kernel");
+    }
+  }
   const int n_max = M == 1 ? K : (int)std::min<long long>(d_in, (long long)M * K);
   larosa::GemvPlan pl;
   cudaError_t e = larosa::plan_gemv(w, larosa::Elem::F32, M, d_out, n_max, &pl);
@@ -109,7 +147,6 @@ extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val
   unsigned char* base = nullptr;
   e = scratch_address(reinterpret_cast<void**>(&base));
   if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress");
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   e = cudaMemsetAsync(base, 0, zero_bytes, s);
   if (e != cudaSuccess) return fail_cuda(e, "clear scratch");
 

@@ -2,10 +2,11 @@
 //
 // The pages do not print this step: it is what keeps the layer's output
 // unchanged when the input is rotated, since x . W = (x . Q) . (Q^T . W) for
-// an orthogonal Q.  It runs once per projection group, off the per-token
-// path.  A 128 x 64 output tile per 256-thread CTA, k-steps of 16 staged in
-// shared memory, 8 x 4 fp32 register accumulators per thread; bf16 results
-// are rounded to nearest even.
+// an orthogonal Q.  The rotation is stored as Qt = Q^T (row-major), so this is
+// the plain product Qt . W.  It runs once per projection group, off the
+// per-token path.  A 128 x 64 output tile per 256-thread CTA, k-steps of 16
+// staged in shared memory, 8 x 4 fp32 register accumulators per thread; bf16
+// results are rounded to nearest even.
 #include "common.cuh"
 #include "internal.h"
 
@@ -26,13 +27,13 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
   return __float2bfloat16_rn(v);
 }
 
-// W_rot[i][j] = sum_k Q[k][i] * W[k][j]; Q is [d x d], W and W_rot [d x n].
+// W_rot[i][j] = sum_k Qt[i][k] * W[k][j]; Qt is [d x d], W and W_rot [d x n].
 template <typename T>
-__global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const T* __restrict__ Q,
+__global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const T* __restrict__ Qt,
                                                                const T* __restrict__ W,
                                                                T* __restrict__ W_rot, int d,
                                                                int n) {
-  __shared__ float As[BK][BM + 4];  // As[k][i] = Q[k0 + k][i0 + i]
+  __shared__ float As[BK][BM + 4];  // As[k][i] = Qt[i0 + i][k0 + k]
   __shared__ float Bs[BK][BN + 4];  // Bs[k][j] = W[k0 + k][j0 + j]
   const int tid = threadIdx.x;
   const int i0 = blockIdx.y * BM;
@@ -53,9 +54,9 @@ __global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const T* __restri
 #pragma unroll
     for (int q = 0; q < (BK * BM) / kPrepThreads; ++q) {
       const int e = tid + q * kPrepThreads;
-      const int kk = e / BM, ii = e % BM;
+      const int ii = e / BK, kk = e % BK;  // consecutive threads read along k
       const int k = k0 + kk, i = i0 + ii;
-      As[kk][ii] = (k < d && i < d) ? to_f32(Q[(size_t)k * d + i]) : 0.f;
+      As[kk][ii] = (k < d && i < d) ? to_f32(Qt[(size_t)i * d + k]) : 0.f;
     }
 #pragma unroll
     for (int q = 0; q < (BK * BN) / kPrepThreads; ++q) {

@@ -6,57 +6,27 @@
 // towards the lower index, +0 and -0 are equal, and the kept entries are
 // emitted in ascending index order.
 //
-// Method: the magnitude of an fp32 value orders exactly like its bit pattern
-// with the sign bit cleared, read as an unsigned integer.  A three-pass MSB
-// radix select over those 31-bit keys (digits of 11, 11 and 9 bits, shared
-// memory histograms) finds the K-th largest key T and how many keys equal to
-// T must be kept.  One block-wide scan of packed (#greater, #equal) counts
-// over contiguous per-thread chunks then gives every kept entry its output
-// position, which is ascending in the index by construction.  The whole
-// vector (d <= 32768 fp32) stays in shared memory; nothing but the input row
-// and the K outputs touches global memory.
+// The selection itself (select.cuh) is a radix select over the fp32 bit
+// patterns with the sign cleared; one packed block scan then gives every kept
+// entry its position, ascending in the index.  The whole vector (d <= 32768
+// fp32) stays in shared memory; nothing but the input row and the K outputs
+// touches global memory.
 #include "common.cuh"
 #include "internal.h"
+#include "select.cuh"
 
 namespace larosa {
 namespace {
 
 constexpr int kTopkThreads = 1024;
-constexpr int kMaxBins = 2048;
-
-// Inclusive prefix sum over the 1024 threads of the block.
-__device__ __forceinline__ uint32_t block_inclusive_scan(uint32_t v, uint32_t* warp_sums) {
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += n;
-  }
-  if (lane == 31) warp_sums[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t w = warp_sums[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t n = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += n;
-    }
-    warp_sums[lane] = w;
-  }
-  __syncthreads();
-  if (warp > 0) v += warp_sums[warp - 1];
-  __syncthreads();
-  return v;
-}
+constexpr int kTopkCand = 2048;
 
 __global__ void __launch_bounds__(kTopkThreads, 1)
     topk_kernel(const float* __restrict__ x_rot, int d, int K, int32_t* __restrict__ idx,
                 float* __restrict__ val, int* dev_status) {
   extern __shared__ __align__(16) uint32_t bits[];  // raw fp32 bits of the row
-  __shared__ uint32_t hist[kMaxBins];
-  __shared__ uint32_t warp_sums[32];
-  __shared__ uint32_t pick[2];
+  __shared__ SelectScratch sel;
+  __shared__ uint32_t cand[kTopkCand];
 
   const int tid = threadIdx.x;
   const int m = blockIdx.x;
@@ -74,14 +44,14 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
     for (int i = tid; i < (d >> 2); i += kTopkThreads) {
       const uint4 u = __ldcg(x4 + i);
       b4[i] = u;
-      nonfinite |= ((u.x & 0x7fffffffu) >= 0x7f800000u) | ((u.y & 0x7fffffffu) >= 0x7f800000u) |
-                   ((u.z & 0x7fffffffu) >= 0x7f800000u) | ((u.w & 0x7fffffffu) >= 0x7f800000u);
+      nonfinite |= ((u.x & kKeyMask) >= 0x7f800000u) | ((u.y & kKeyMask) >= 0x7f800000u) |
+                   ((u.z & kKeyMask) >= 0x7f800000u) | ((u.w & kKeyMask) >= 0x7f800000u);
     }
   } else {
     for (int i = tid; i < d; i += kTopkThreads) {
       const uint32_t u = __float_as_uint(__ldcg(x + i));
       bits[i] = u;
-      nonfinite |= (u & 0x7fffffffu) >= 0x7f800000u;
+      nonfinite |= (u & kKeyMask) >= 0x7f800000u;
     }
   }
   if (__syncthreads_or(nonfinite) && tid == 0) report(dev_status, LAROSA_DEV_NONFINITE);
@@ -95,63 +65,18 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
     return;
   }
 
-  // ---- radix select of the K-th largest key, most significant digit first
-  uint32_t prefix = 0, mask = 0;
-  uint32_t krem = static_cast<uint32_t>(K);  // keys still to take at/below the prefix
-#pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 20 : (pass == 1 ? 9 : 0);
-    const int nb = pass == 2 ? 512 : 2048;
-    for (int b = tid; b < nb; b += kTopkThreads) hist[b] = 0;
-    __syncthreads();
-    for (int i = tid; i < d; i += kTopkThreads) {
-      const uint32_t k = bits[i] & 0x7fffffffu;
-      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & (nb - 1)], 1u);
-    }
-    __syncthreads();
-    // thread t owns bins nb-1-2t and nb-2-2t: counts from the top
-    uint32_t h_hi = 0, h_lo = 0;
-    if (2 * tid < nb) {
-      h_hi = hist[nb - 1 - 2 * tid];
-      h_lo = hist[nb - 2 - 2 * tid];
-    }
-    const uint32_t own = h_hi + h_lo;
-    const uint32_t incl = block_inclusive_scan(own, warp_sums);
-    const uint32_t before = incl - own;
-    if (2 * tid < nb && before < krem && krem <= incl) {
-      if (before + h_hi >= krem) {
-        pick[0] = static_cast<uint32_t>(nb - 1 - 2 * tid);
-        pick[1] = before;
-      } else {
-        pick[0] = static_cast<uint32_t>(nb - 2 - 2 * tid);
-        pick[1] = before + h_hi;
-      }
-    }
-    __syncthreads();
-    prefix |= pick[0] << shift;
-    mask |= static_cast<uint32_t>(nb - 1) << shift;
-    krem -= pick[1];
-    __syncthreads();
-  }
-  const uint32_t T = prefix;  // the K-th largest key; krem keys equal to T are kept
+  uint32_t T = 0, krem = 0;
+  select_threshold<kTopkThreads>(bits, d, K, &sel, cand, kTopkCand, &T, &krem);
 
-  // ---- stable compaction: contiguous chunks, one packed scan of (#eq, #gt)
+  // ---- stable compaction over contiguous chunks
   const int chunk = (d + kTopkThreads - 1) / kTopkThreads;
   const int i0 = min(d, tid * chunk);
   const int i1 = min(d, i0 + chunk);
-  uint32_t gt = 0, eq = 0;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t k = bits[i] & 0x7fffffffu;
-    gt += k > T;
-    eq += k == T;
-  }
-  const uint32_t packed = (eq << 16) | gt;  // d < 65536: no carry between halves
-  const uint32_t excl = block_inclusive_scan(packed, warp_sums) - packed;
-  uint32_t gt_before = excl & 0xffffu;
-  uint32_t eq_before = excl >> 16;
+  uint32_t gt_before = 0, eq_before = 0;
+  kept_chunk_base<kTopkThreads>(bits, i0, i1, T, &sel, &gt_before, &eq_before);
   for (int i = i0; i < i1; ++i) {
     const uint32_t u = bits[i];
-    const uint32_t k = u & 0x7fffffffu;
+    const uint32_t k = u & kKeyMask;
     if (k > T) {
       const uint32_t pos = gt_before + min(eq_before, krem);
       if (pos < static_cast<uint32_t>(K)) {

@@ -37,11 +37,11 @@ _SIGNATURES = {
     "larosa_version": ([], _i),
     "larosa_last_error_string": ([], _c.c_char_p),
     "larosa_prepare_weights": ([_vp, _vp, _vp, _i, _i, _i, _vp], _i),
-    "larosa_rotate": ([_vp, _vp, _vp, _i, _i, _i, _vp, _sz, _vp, _vp], _i),
+    "larosa_rotate": ([_vp, _vp, _vp, _i, _i, _i, _vp], _i),
     "larosa_topk": ([_vp, _i, _i, _i, _vp, _vp, _vp, _vp], _i),
     "larosa_sparse_linear": ([_vp, _vp, _i, _i, _vp, _i, _i, _vp, _vp, _sz, _i, _vp, _vp], _i),
     "larosa_rotate_topk_linear": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp, _i, _vp], _i),
-    "larosa_dense_linear": ([_vp, _vp, _i, _i, _i, _vp, _vp, _sz, _i, _vp, _vp], _i),
+    "larosa_dense_linear": ([_vp, _vp, _i, _i, _i, _vp, _i, _vp], _i),
     "larosa_sparse_linear_noalloc": ([_vp, _vp, _i, _i, _vp, _i, _i, _vp, _i, _vp, _vp], _i),
     "larosa_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "larosa_workspace_layout": ([_i, _i, _i, _i, _c.POINTER(_sz), _c.POINTER(_sz), _c.POINTER(_sz)], _i),
@@ -121,12 +121,17 @@ class Workspace:
         self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
             else torch.device(device)
         self.buf = torch.zeros(0, dtype=torch.uint8, device=self.device)
+        self._need: dict[tuple[int, int, int, int], int] = {}
 
     def get(self, M: int, d_in: int, d_out: int, K: int) -> torch.Tensor:
-        with torch.cuda.device(self.device):
-            need = int(_lib.larosa_workspace_bytes(M, d_in, d_out, K))
-        if need == 0:
-            raise LarosaError(2, "larosa_workspace_bytes")
+        key = (M, d_in, d_out, K)
+        need = self._need.get(key)
+        if need is None:
+            with torch.cuda.device(self.device):
+                need = int(_lib.larosa_workspace_bytes(M, d_in, d_out, K))
+            if need == 0:
+                raise LarosaError(2, "larosa_workspace_bytes")
+            self._need[key] = need
         if self.buf.numel() < need:
             self.buf = torch.zeros(need, dtype=torch.uint8, device=self.device)
         return self.buf
@@ -187,33 +192,35 @@ def larosa_workspace_layout(M: int, d_in: int, d_out: int, K: int) -> tuple[int,
     return a.value, b.value, c.value
 
 
-def larosa_prepare_weights(Q: torch.Tensor, W: torch.Tensor, W_rot: torch.Tensor | None = None
+def larosa_prepare_weights(Qt: torch.Tensor, W: torch.Tensor, W_rot: torch.Tensor | None = None
                            ) -> torch.Tensor:
-    """W_rot = Q^T . W (offline counter-rotation), same dtype as W."""
-    _need(Q, "Q")
-    _need(W, "W", Q.dtype)
+    """W_rot = Q^T . W = Qt . W (offline counter-rotation), same dtype as W.
+
+    Qt is the rotation stored transposed (Qt = Q.T.contiguous() for x_rot = x @ Q).
+    """
+    _need(Qt, "Qt")
+    _need(W, "W", Qt.dtype)
     d_in, d_out = W.shape
     if W_rot is None:
         W_rot = torch.empty_like(W)
     _need(W_rot, "W_rot", W.dtype)
-    _check(_lib.larosa_prepare_weights(_ptr(Q), _ptr(W), _ptr(W_rot), d_in, d_out, _dtype_code(W),
+    _check(_lib.larosa_prepare_weights(_ptr(Qt), _ptr(W), _ptr(W_rot), d_in, d_out, _dtype_code(W),
                                        _stream(W.device)), "larosa_prepare_weights")
     return W_rot
 
 
-def larosa_rotate(x: torch.Tensor, Q: torch.Tensor, x_rot: torch.Tensor | None = None, ws=None,
-                  dev_status: torch.Tensor | None = None) -> torch.Tensor:
-    """x_rot = x . Q, fp32 output [M, d]."""
+def larosa_rotate(x: torch.Tensor, Qt: torch.Tensor, x_rot: torch.Tensor | None = None
+                  ) -> torch.Tensor:
+    """x_rot = x . Q with Qt = Q^T, fp32 output [M, d]."""
     _need(x, "x")
-    _need(Q, "Q", x.dtype)
+    _need(Qt, "Qt", x.dtype)
     x2 = _as2d(x)
     M, d = x2.shape
     if x_rot is None:
         x_rot = torch.empty((M, d), dtype=torch.float32, device=x.device)
     _need(x_rot, "x_rot", torch.float32)
-    p, n = _ws_args(ws, x.device, M, d, d, 0)
-    _check(_lib.larosa_rotate(_ptr(x2), _ptr(Q), _ptr(x_rot), M, d, _dtype_code(x), p, n,
-                              _status_ptr(dev_status, x.device), _stream(x.device)), "larosa_rotate")
+    _check(_lib.larosa_rotate(_ptr(x2), _ptr(Qt), _ptr(x_rot), M, d, _dtype_code(x),
+                              _stream(x.device)), "larosa_rotate")
     return x_rot
 
 
@@ -283,12 +290,12 @@ def larosa_sparse_linear_noalloc(idx: torch.Tensor, val: torch.Tensor, W_rot: to
     return y
 
 
-def larosa_rotate_topk_linear(x: torch.Tensor, Q: torch.Tensor, W_rot: torch.Tensor, K: int,
+def larosa_rotate_topk_linear(x: torch.Tensor, Qt: torch.Tensor, W_rot: torch.Tensor, K: int,
                               y: torch.Tensor | None = None, ws=None,
                               dev_status: torch.Tensor | None = None) -> torch.Tensor:
-    """Fused rotate -> Top-K -> sparse linear, fp32 output [M, d_out]."""
+    """Fused rotate -> Top-K -> sparse linear (Qt = Q^T), fp32 output [M, d_out]."""
     _need(x, "x")
-    _need(Q, "Q", x.dtype)
+    _need(Qt, "Qt", x.dtype)
     _need(W_rot, "W_rot", x.dtype)
     x2 = _as2d(x)
     M, d_in = x2.shape
@@ -297,27 +304,27 @@ def larosa_rotate_topk_linear(x: torch.Tensor, Q: torch.Tensor, W_rot: torch.Ten
         y = torch.empty((M, d_out), dtype=torch.float32, device=x.device)
     _need(y, "y", torch.float32)
     p, n = _ws_args(ws, x.device, M, d_in, d_out, K)
-    _check(_lib.larosa_rotate_topk_linear(_ptr(x2), _ptr(Q), _ptr(W_rot), M, d_in, d_out, K, _ptr(y),
+    _check(_lib.larosa_rotate_topk_linear(_ptr(x2), _ptr(Qt), _ptr(W_rot), M, d_in, d_out, K, _ptr(y),
                                           p, n, _status_ptr(dev_status, x.device), _dtype_code(x),
                                           _stream(x.device)), "larosa_rotate_topk_linear")
     return y
 
 
-def larosa_dense_linear(x: torch.Tensor, W: torch.Tensor, y: torch.Tensor | None = None, ws=None,
-                        dev_status: torch.Tensor | None = None) -> torch.Tensor:
-    """Dense baseline y = x . W (same streaming machinery), fp32 [M, d_out]."""
+def larosa_dense_linear(x: torch.Tensor, Wt: torch.Tensor, y: torch.Tensor | None = None
+                        ) -> torch.Tensor:
+    """Dense baseline y = x . W with Wt = W^T in torch.nn.Linear layout [d_out, d_in]."""
     _need(x, "x")
-    _need(W, "W", x.dtype)
+    _need(Wt, "Wt", x.dtype)
     x2 = _as2d(x)
     M, d_in = x2.shape
-    d_out = W.shape[1]
+    d_out = Wt.shape[0]
+    if Wt.shape[1] != d_in:
+        raise ValueError("Wt must be [d_out, d_in]")
     if y is None:
         y = torch.empty((M, d_out), dtype=torch.float32, device=x.device)
     _need(y, "y", torch.float32)
-    p, n = _ws_args(ws, x.device, M, d_in, d_out, d_in)
-    _check(_lib.larosa_dense_linear(_ptr(x2), _ptr(W), M, d_in, d_out, _ptr(y), p, n, _dtype_code(x),
-                                    _status_ptr(dev_status, x.device), _stream(x.device)),
-           "larosa_dense_linear")
+    _check(_lib.larosa_dense_linear(_ptr(x2), _ptr(Wt), M, d_in, d_out, _ptr(y), _dtype_code(x),
+                                    _stream(x.device)), "larosa_dense_linear")
     return y
 
 

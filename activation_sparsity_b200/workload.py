@@ -19,18 +19,23 @@ from .larosa import larosa_prepare_weights
 
 @dataclass
 class Group:
+    """One projection group.  Qt is the rotation stored transposed (Q^T); W is
+    the dense weight row-major [d_in, d_out], Wt the same in torch.nn.Linear
+    layout [d_out, d_in] (used by the dense baseline); W_rot = Q^T W."""
+
     name: str
     d_in: int
     d_out: int
     K: int
-    Q: torch.Tensor
+    Qt: torch.Tensor
     W: torch.Tensor | None
+    Wt: torch.Tensor | None
     W_rot: torch.Tensor
     x: torch.Tensor
 
     @property
     def rot_bytes(self) -> int:
-        return self.Q.numel() * self.Q.element_size()
+        return self.Qt.numel() * self.Qt.element_size()
 
     def row_bytes(self, rows: int) -> int:
         return rows * self.d_out * self.W_rot.element_size()
@@ -48,11 +53,13 @@ def build_layer(hidden: int, ffn: int, kv: int, sparsity_pct: float, workload_id
     out = Layer()
     for p in sd.llama_layer(hidden, ffn, kv):
         base = sd.seed_for(workload_id, layer, 10 * p.q_id)
-        Q = sd.orthogonal(p.d_in, base + 1, device=device).to(dtype)
+        Qt = sd.orthogonal(p.d_in, base + 1, device=device).to(dtype).t().contiguous()
         W = sd.weights(p.d_in, p.d_out, w_std, base + 2, dtype, device=device)
-        W_rot = larosa_prepare_weights(Q, W)
+        W_rot = larosa_prepare_weights(Qt, W)
         x = sd.activations(M, p.d_in, base + 3, dtype, device=device)
         K = sd.k_for_sparsity(p.d_in, sparsity_pct)
-        out.groups.append(Group(p.name, p.d_in, p.d_out, K, Q, W if keep_dense else None, W_rot, x))
+        Wt = W.t().contiguous() if keep_dense else None
+        out.groups.append(Group(p.name, p.d_in, p.d_out, K, Qt, W if keep_dense else None, Wt,
+                                W_rot, x))
     torch.cuda.synchronize(device)
     return out

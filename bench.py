@@ -187,7 +187,7 @@ def measured_peaks() -> tuple[float, str]:
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("rowstream.cu", "common.cuh"):
+    for name in ("onetoken.cu", "common.cuh"):
         with open(os.path.join(ROOT, "activation_sparsity_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -325,17 +325,27 @@ def bench_larosa(args):
 
     def fused_step():
         for g, y in zip(groups, ys):
-            L.larosa_rotate_topk_linear(g.x, g.Q, g.W_rot, g.K, y=y, ws=ws, dev_status=st)
+            L.larosa_rotate_topk_linear(g.x, g.Qt, g.W_rot, g.K, y=y, ws=ws, dev_status=st)
+
+    def rotate_step():
+        for g, xr in zip(groups, x_rots):
+            L.larosa_rotate(g.x, g.Qt, x_rot=xr)
+
+    def topk_step():
+        for gi, g in enumerate(groups):
+            L.larosa_topk(x_rots[gi], g.K, idx=idxs[gi], val=vals[gi], dev_status=st)
+
+    def gather_step():
+        for gi, g in enumerate(groups):
+            L.larosa_sparse_linear(idxs[gi], vals[gi], g.W_rot, y=ys[gi], ws=ws, dev_status=st)
 
     def sparse_only_step():  # the same path on pre-rotated inputs (no Q streamed)
-        for g, y, xr in zip(groups, ys, x_rots):
-            L.larosa_topk(xr, g.K, idx=idxs[groups.index(g)], val=vals[groups.index(g)], dev_status=st)
-            L.larosa_sparse_linear(idxs[groups.index(g)], vals[groups.index(g)], g.W_rot, y=y, ws=ws,
-                                   dev_status=st)
+        topk_step()
+        gather_step()
 
     def dense_step():
         for g, y in zip(groups, ys):
-            L.larosa_dense_linear(g.x, g.W, y=y, ws=ws, dev_status=st)
+            L.larosa_dense_linear(g.x, g.Wt, y=y)
 
     def graph_of(fn):
         with torch.cuda.stream(stream):
@@ -367,15 +377,18 @@ def bench_larosa(args):
         barrier(world, device)
         return e0.elapsed_time(e1) / 1e3, clk
 
-    # rotate once so the sparse-only path has its pre-rotated inputs
+    # rotate and select once so the component graphs have their inputs
     with torch.cuda.stream(stream):
-        for g, xr in zip(groups, x_rots):
-            L.larosa_rotate(g.x, g.Q, x_rot=xr, ws=ws, dev_status=st)
+        rotate_step()
+        topk_step()
     torch.cuda.synchronize(device)
 
     g_fused = graph_of(fused_step)
     g_sparse = graph_of(sparse_only_step)
     g_dense = graph_of(dense_step)
+    g_rot = graph_of(rotate_step)
+    g_topk = graph_of(topk_step)
+    g_gather = graph_of(gather_step)
 
     props = torch.cuda.get_device_properties(device)
     clocks = ClockSampler(f"GPU-{props.uuid}")
@@ -386,43 +399,28 @@ def bench_larosa(args):
     sparse_tps, _ = aggregate(t_sparse, args.steps, world, device)
     dense_tps, _ = aggregate(t_dense, args.steps, world, device)
 
-    # ---- per-kernel pass: the same kernels through the component calls, with
-    # CUDA events around each launch on the launching stream
-    n_rep = max(50, min(2000, args.steps // 5))
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in groups]
-    rot_ms, topk_ms, lin_ms = [], [], []
-    with torch.cuda.stream(stream):
-        for r in range(args.warmup + n_rep):
-            for gi, g in enumerate(groups):
-                e = ev[gi]
-                e[0].record(stream)
-                L.larosa_rotate(g.x, g.Q, x_rot=x_rots[gi], ws=ws, dev_status=st)
-                e[1].record(stream)
-                L.larosa_topk(x_rots[gi], g.K, idx=idxs[gi], val=vals[gi], dev_status=st)
-                e[2].record(stream)
-                L.larosa_sparse_linear(idxs[gi], vals[gi], g.W_rot, y=ys[gi], ws=ws, dev_status=st)
-                e[3].record(stream)
-                if r >= args.warmup:
-                    e[3].synchronize()
-                    rot_ms.append((gi, e[0].elapsed_time(e[1])))
-                    topk_ms.append((gi, e[1].elapsed_time(e[2])))
-                    lin_ms.append((gi, e[2].elapsed_time(e[3])))
-    torch.cuda.synchronize(device)
+    # ---- per-kernel pass: graphs holding one kernel type for the four groups,
+    # timed with CUDA events on the launching stream over the same steps
+    t_rot, _ = time_graph(g_rot, args.steps, args.warmup)
+    t_topk, _ = time_graph(g_topk, args.steps, args.warmup)
+    t_gather, _ = time_graph(g_gather, args.steps, args.warmup)
+    n_launch = args.steps * len(groups)
+    rot_us = t_rot / n_launch * 1e6
+    topk_us = t_topk / n_launch * 1e6
+    gather_us = t_gather / n_launch * 1e6
+    select_gather_us = (t_fused - t_rot) / n_launch * 1e6
     assert L.larosa_check(st, device=device) == 0
 
-    def mean_by_group(rec):
-        return [statistics.mean(ms for gi2, ms in rec if gi2 == gi) for gi in range(len(groups))]
-
-    rot_g, topk_g, lin_g = mean_by_group(rot_ms), mean_by_group(topk_ms), mean_by_group(lin_ms)
     rot_bytes = [g.d_in * g.d_in * 2 + g.d_in * 2 + g.d_in * 4 for g in groups]
     lin_bytes = [g.K * g.d_out * 2 + g.K * 8 + g.d_out * 4 for g in groups]
     step_bytes = sum(path_bytes(g, g.K)["total"] for g in groups)
     sparse_bytes = sum(path_bytes(g, g.K, rotate=False)["total"] for g in groups)
+    dense_bytes = sum(g.d_in * g.d_out * 2 + g.d_in * 2 + g.d_out * 4 for g in groups)
     peak, peak_kind = measured_peaks()
-    rot_gbs = sum(rot_bytes) / (sum(rot_g) * 1e-3) / 1e9
-    lin_gbs = sum(lin_bytes) / (sum(lin_g) * 1e-3) / 1e9
-    share_rot = sum(rot_g) / (sum(rot_g) + sum(topk_g) + sum(lin_g))
-    traffic = profiled_traffic("rotate")
+    rot_gbs = sum(rot_bytes) * args.steps / t_rot / 1e9
+    lin_gbs = sum(lin_bytes) * args.steps / t_gather / 1e9
+    share_rot = t_rot / t_fused
+    traffic = profiled_traffic("rowdot")
 
     # ---- end to end through the public API with host buffers
     x_host = [g.x.cpu().pin_memory() for g in groups]
@@ -438,7 +436,7 @@ def bench_larosa(args):
                 e0.record(stream)
             for gi, g in enumerate(groups):
                 x_dev[gi].copy_(x_host[gi], non_blocking=True)
-                L.larosa_rotate_topk_linear(x_dev[gi], g.Q, g.W_rot, g.K, y=ys[gi], ws=ws, dev_status=st)
+                L.larosa_rotate_topk_linear(x_dev[gi], g.Qt, g.W_rot, g.K, y=ys[gi], ws=ws, dev_status=st)
                 y_host[gi].copy_(ys[gi], non_blocking=True)
         e1.record(stream)
     torch.cuda.synchronize(device)
@@ -466,16 +464,17 @@ def bench_larosa(args):
             "hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
             "hbm_frac": step_bytes / (ms_step * 1e-3) / 1e9 / peak,
             "bytes_per_step": step_bytes,
-            "roofline": {"kernel": "rowstream_gemv (rotation x.Q, bf16)", "bound": "hbm",
+            "roofline": {"kernel": "rowdot_kernel (rotation x.Q through Q^T, bf16)", "bound": "hbm",
                          "achieved": rot_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": rot_gbs / peak, "traffic": traffic,
                          "algorithmic_bytes_per_launch": statistics.mean(rot_bytes),
-                         "avg_launch_us": statistics.mean(rot_g) * 1e3, "share_of_step": share_rot},
+                         "avg_launch_us": rot_us, "share_of_step": share_rot},
             "kernels": {
-                "rotate_us": [round(v * 1e3, 2) for v in rot_g],
-                "topk_us": [round(v * 1e3, 2) for v in topk_g],
-                "sparse_linear_us": [round(v * 1e3, 2) for v in lin_g],
-                "sparse_linear_gbs": lin_gbs, "sparse_linear_frac": lin_gbs / peak,
+                "rotate_us_per_launch": rot_us,
+                "select_gather_us_per_launch": select_gather_us,
+                "topk_us_per_launch": topk_us,
+                "gather_us_per_launch": gather_us,
+                "gather_gbs": lin_gbs, "gather_frac": lin_gbs / peak,
                 "groups": [g.name for g in groups],
             },
             "paths": {
@@ -483,18 +482,19 @@ def bench_larosa(args):
                 "sparse_only_tokens_per_s": sparse_tps,
                 "sparse_only_hbm_frac": sparse_bytes * sparse_tps / world / 1e9 / peak,
                 "dense_tokens_per_s": dense_tps,
+                "dense_hbm_frac": dense_bytes * dense_tps / world / 1e9 / peak,
                 "sparse_only_vs_dense": sparse_tps / dense_tps,
                 "fused_vs_dense": value / dense_tps,
             },
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": sum(g.x.numel() * g.x.element_size() for g in groups),
                     "d2h_bytes_per_step": sum(g.d_out * 4 for g in groups)},
-            "gpu_launches": args.steps * 3 * len(groups),
+            "gpu_launches": args.steps * 2 * len(groups),
             "clocks": clk,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    del g_fused, g_sparse, g_dense
+    del g_fused, g_sparse, g_dense, g_rot, g_topk, g_gather
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -42,7 +42,8 @@
  *     those conditions are not reported.  Kernels never trap or spin without
  *     bound: every wait inside a kernel gives up after about two seconds,
  *     sets LAROSA_DEV_TIMEOUT and exits.
- *   - Workspace: the split-K GEMV kernels use caller-provided scratch `ws`
+ *   - Workspace: the sparse linear and the fused call use caller-provided
+ *     scratch `ws`
  *     of `ws_bytes` bytes, at least larosa_workspace_bytes(...).  It must be
  *     16-byte aligned and ZERO-FILLED before its first use; every call that
  *     completes leaves its counter words at zero again, so the same buffer
@@ -52,9 +53,10 @@
  *   - Data types: `dtype` is LAROSA_BF16 (bf16 activations and weights) or
  *     LAROSA_F32 (fp32 activations and weights).  Rotated activations, kept
  *     values and outputs are always fp32; all accumulation is fp32.
- *   - Alignment: weight and activation base pointers 16-byte aligned, and
- *     the row length of every weight (d_out, or d for Q) a multiple of 8
- *     elements for bf16 or 4 for fp32; otherwise LAROSA_ERR_ALIGN.
+ *   - Alignment: weight, activation and output base pointers 16-byte
+ *     aligned, and the row length of every weight a multiple of 16 bytes
+ *     (rotations and dense weights: a multiple of 8 elements); otherwise
+ *     LAROSA_ERR_ALIGN.
  *   - Sizes: 1 <= M <= LAROSA_MAX_M, 1 <= d <= LAROSA_MAX_D, 0 <= K <= d.
  */
 #ifndef LAROSA_H
@@ -109,27 +111,36 @@ int larosa_version(void);
 const char *larosa_last_error_string(void);
 
 /*
+ * Rotation storage.  The orthogonal rotation Q of a layer input is stored as
+ * its transpose Qt = Q^T, row-major [d x d]: row j of Qt is column j of Q, so
+ * each rotated entry x_rot[j] = sum_i x[i] Q[i][j] is the dot product of x
+ * with one contiguous row, and the offline counter-rotation is the plain
+ * product Qt . W.  (In PyTorch terms: Qt = Q.T.contiguous() for
+ * x_rot = x @ Q.)
+ */
+
+/*
  * Offline counter-rotation of a weight (step 0, not on the per-token path):
- *   W_rot[i][j] = sum_k Q[k][i] * W[k][j],   i.e. W_rot = Q^T . W.
- * Q: [d_in x d_in], W: [d_in x d_out], W_rot: [d_in x d_out], all row-major
+ *   W_rot[i][j] = sum_k Qt[i][k] * W[k][j],   i.e. W_rot = Q^T . W.
+ * Qt: [d_in x d_in], W: [d_in x d_out], W_rot: [d_in x d_out], all row-major
  * and all of type `dtype`.  fp32 accumulation; bf16 outputs are rounded to
  * nearest even.  Projections that share an input (q|k|v, gate|up) are packed
  * by passing their weights concatenated along d_out.  W_rot must not overlap
- * Q or W.
+ * Qt or W.
  */
-int larosa_prepare_weights(const void *Q, const void *W, void *W_rot,
+int larosa_prepare_weights(const void *Qt, const void *W, void *W_rot,
                            int d_in, int d_out, int dtype,
                            larosa_stream_t stream);
 
 /*
- * Rotation (step 1): x_rot[m][j] = sum_i x[m][i] * Q[i][j].
- * x: [M x d] of `dtype`, Q: [d x d] of `dtype`, x_rot: [M x d] fp32.
- * Streams all of Q once per call (an HBM-bound GEMV for small M).
- * ws: at least larosa_workspace_bytes(M, d, d, 0) bytes.
+ * Rotation (step 1): x_rot[m][j] = sum_i x[m][i] * Q[i][j]
+ *                                = sum_i x[m][i] * Qt[j][i].
+ * x: [M x d] of `dtype`, Qt: [d x d] of `dtype`, x_rot: [M x d] fp32.
+ * Streams all of Qt once per call (an HBM-bound GEMV for small M).  Needs
+ * d a multiple of 8, and x and Qt 16-byte aligned.  Uses no workspace.
  */
-int larosa_rotate(const void *x, const void *Q, float *x_rot, int M, int d,
-                  int dtype, void *ws, size_t ws_bytes, int *dev_status,
-                  larosa_stream_t stream);
+int larosa_rotate(const void *x, const void *Qt, float *x_rot, int M, int d,
+                  int dtype, larosa_stream_t stream);
 
 /*
  * Exact per-token Top-K by magnitude (step 2).
@@ -160,26 +171,30 @@ int larosa_sparse_linear(const int32_t *idx, const float *val, int M, int K,
 /*
  * Steps 1-3 in one call, one stream, no host synchronisation:
  *   x_rot = x . Q;  (idx, val) = TopK(x_rot, K);  y = sparse(x_rot) . W_rot.
- * x: [M x d_in] of `dtype`; Q: [d_in x d_in]; W_rot: [d_in x d_out] of
- * `dtype` (from larosa_prepare_weights with the same Q); y: [M x d_out] fp32.
- * The intermediate x_rot, idx and val live in the workspace; their offsets
- * are given by larosa_workspace_layout() for inspection.
+ * x: [M x d_in] of `dtype`; Qt = Q^T: [d_in x d_in]; W_rot: [d_in x d_out] of
+ * `dtype` (from larosa_prepare_weights with the same Qt); y: [M x d_out] fp32.
+ * For one token this is two kernels: the rotation, then a gather in which
+ * every CTA selects the Top-K of x_rot itself.  The intermediate x_rot, idx
+ * and val live in the workspace at the offsets larosa_workspace_layout()
+ * gives.  d_in a multiple of 8; x, Qt, W_rot and y 16-byte aligned.
  * ws: at least larosa_workspace_bytes(M, d_in, d_out, K) bytes.
  */
-int larosa_rotate_topk_linear(const void *x, const void *Q, const void *W_rot,
+int larosa_rotate_topk_linear(const void *x, const void *Qt, const void *W_rot,
                               int M, int d_in, int d_out, int K, float *y,
                               void *ws, size_t ws_bytes, int *dev_status,
                               int dtype, larosa_stream_t stream);
 
 /*
- * Dense baseline: y[m][j] = sum_i x[m][i] * W[i][j] with the same streaming
- * GEMV machinery (no cuBLAS).  x: [M x d_in] of `dtype`, W: [d_in x d_out]
- * of `dtype`, y: [M x d_out] fp32.
- * ws: at least larosa_workspace_bytes(M, d_in, d_out, d_in) bytes.
+ * Dense baseline: y[m][j] = sum_i x[m][i] * Wt[j][i], i.e. y = x . W for the
+ * dense layer, with the weight in torch.nn.Linear layout Wt = W^T
+ * [d_out x d_in] (each output a dot product with one contiguous row), by the
+ * same streaming machinery as the rotation (no cuBLAS).  x: [M x d_in] of
+ * `dtype`, y: [M x d_out] fp32.  d_in a multiple of 8; x and Wt 16-byte
+ * aligned.  Uses no workspace.
  */
-int larosa_dense_linear(const void *x, const void *W, int M, int d_in,
-                        int d_out, float *y, void *ws, size_t ws_bytes,
-                        int dtype, int *dev_status, larosa_stream_t stream);
+int larosa_dense_linear(const void *x, const void *Wt, int M, int d_in,
+                        int d_out, float *y, int dtype,
+                        larosa_stream_t stream);
 
 /*
  * larosa_sparse_linear without a workspace, for callers that cannot allocate

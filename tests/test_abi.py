@@ -65,31 +65,34 @@ def test_host_validation_rejects_bad_arguments(lib):
     BF16, F32 = 1, 0
     z = ctypes.c_size_t(1 << 20)
     # unsupported dtype
-    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 64, 7, FAKE, z, None, None) == 4
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 64, 7, None) == 4
     assert lib.larosa_prepare_weights(FAKE, FAKE, FAKE, 64, 64, 9, None) == 4
     # NULL pointers
-    assert lib.larosa_rotate(None, FAKE, FAKE, 1, 64, BF16, FAKE, z, None, None) == 1
+    assert lib.larosa_rotate(None, FAKE, FAKE, 1, 64, BF16, None) == 1
     assert lib.larosa_topk(None, 1, 64, 3, FAKE, FAKE, None, None) == 1
     assert lib.larosa_topk(FAKE, 1, 64, 3, None, FAKE, None, None) == 1
     assert lib.larosa_sparse_linear(FAKE, FAKE, 1, 4, None, 64, 64, FAKE, FAKE, z, BF16, None, None) == 1
     assert lib.larosa_prepare_weights(FAKE, None, FAKE, 64, 64, BF16, None) == 1
     # sizes
-    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 0, 64, BF16, FAKE, z, None, None) == 2
-    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 17, 64, BF16, FAKE, z, None, None) == 2
-    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 32769, BF16, FAKE, z, None, None) == 2
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 0, 64, BF16, None) == 2
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 17, 64, BF16, None) == 2
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 32769, BF16, None) == 2
     assert lib.larosa_topk(FAKE, 1, 64, 65, FAKE, FAKE, None, None) == 2
     assert lib.larosa_topk(FAKE, 1, 64, -1, FAKE, FAKE, None, None) == 2
     assert lib.larosa_sparse_linear(FAKE, FAKE, 1, 65, FAKE, 64, 64, FAKE, FAKE, z, BF16, None, None) == 2
     assert lib.larosa_rotate_topk_linear(FAKE, FAKE, FAKE, 1, 64, 64, 65, FAKE, FAKE, z, None, BF16, None) == 2
-    assert lib.larosa_dense_linear(FAKE, FAKE, 1, 64, 0, FAKE, FAKE, z, BF16, None, None) == 2
+    assert lib.larosa_dense_linear(FAKE, FAKE, 1, 64, 0, FAKE, BF16, None) == 2
     # alignment: base pointers and row lengths (bf16 rows a multiple of 8 elements)
-    assert lib.larosa_rotate(FAKE, MISALIGNED, FAKE, 1, 64, BF16, FAKE, z, None, None) == 3
-    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 60, BF16, FAKE, z, None, None) == 3
-    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 62, F32, FAKE, z, None, None) == 3
+    assert lib.larosa_rotate(FAKE, MISALIGNED, FAKE, 1, 64, BF16, None) == 3
+    assert lib.larosa_rotate(MISALIGNED, FAKE, FAKE, 1, 64, BF16, None) == 3
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 60, BF16, None) == 3
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 62, F32, None) == 3
+    assert lib.larosa_rotate(FAKE, FAKE, FAKE, 1, 12, F32, None) == 3  # rows a multiple of 8
     assert lib.larosa_sparse_linear(FAKE, FAKE, 1, 4, MISALIGNED, 64, 64, FAKE, FAKE, z, BF16, None, None) == 3
     assert lib.larosa_sparse_linear(FAKE, FAKE, 1, 4, FAKE, 64, 36, FAKE, FAKE, z, BF16, None, None) == 3
     assert lib.larosa_rotate_topk_linear(FAKE, FAKE, FAKE, 1, 64, 12, 5, FAKE, FAKE, z, None, BF16, None) == 3
-    assert lib.larosa_dense_linear(FAKE, MISALIGNED, 1, 64, 64, FAKE, FAKE, z, BF16, None, None) == 3
+    assert lib.larosa_dense_linear(FAKE, MISALIGNED, 1, 64, 64, FAKE, BF16, None) == 3
+    assert lib.larosa_dense_linear(FAKE, FAKE, 1, 60, 64, FAKE, BF16, None) == 3
     # in-place counter-rotation is refused
     assert lib.larosa_prepare_weights(FAKE, P(0x20000), P(0x20000), 64, 64, BF16, None) == 1
     # status check needs a status word

@@ -78,7 +78,7 @@ def check_bf16_rounding(got: np.ndarray, exact: np.ndarray, gamma: np.ndarray) -
 def test_prepare_weights(L, dtype, d, n):
     Q = sd.orthogonal(d, 101).to(dtype)
     W = sd.weights(d, n, 0.02, 102, dtype)
-    W_rot = L.larosa_prepare_weights(Q.cuda(), W.cuda())
+    W_rot = L.larosa_prepare_weights(Q.t().contiguous().cuda(), W.cuda())
     torch.cuda.synchronize()
     exact = oracle.prepare_weights(f64(Q), f64(W))
     got = f64(W_rot)
@@ -100,6 +100,10 @@ def test_prepare_weights(L, dtype, d, n):
     (torch.bfloat16, 8, 2048),
     (torch.bfloat16, 1, 4096),
     (torch.bfloat16, 2, 11008),
+    (torch.bfloat16, 16, 4096),   # activations too large for shared memory
+    (torch.float32, 16, 2048),
+    (torch.bfloat16, 1, 28672),
+    (torch.bfloat16, 1, 8),
 ])
 def test_rotate(L, dtype, M, d):
     if d > 4096:
@@ -107,9 +111,7 @@ def test_rotate(L, dtype, M, d):
     else:
         Q = sd.orthogonal(d, 201).to(dtype).cuda()
     x = sd.activations(M, d, 202, dtype)
-    st = status()
-    got = f64(L.larosa_rotate(x.cuda(), Q, dev_status=st))
-    assert L.larosa_check(st) == 0
+    got = f64(L.larosa_rotate(x.cuda(), Q.t().contiguous()))
     xq, qq = f64(x), f64(Q)
     ref = oracle.rotate(xq, qq)
     bound = (d + 2) * U * (np.abs(xq) @ np.abs(qq))
@@ -171,6 +173,12 @@ SPARSE_CASES = [
     (torch.bfloat16, 8, 512, 1024, 100),
     (torch.bfloat16, 16, 512, 256, 300),
     (torch.float32, 3, 300, 100, 50),
+    # one-token stream-K edge shapes: fewer units than SMs, one tile, ragged tiles
+    (torch.bfloat16, 1, 64, 8, 1),
+    (torch.bfloat16, 1, 300, 40, 7),
+    (torch.bfloat16, 1, 4096, 8200, 100),
+    (torch.bfloat16, 1, 28672, 2048, 17204),
+    (torch.float32, 1, 1000, 1028, 999),
 ]
 
 
@@ -211,11 +219,15 @@ def test_sparse_linear_reports_bad_index(L):
     (torch.bfloat16, 1, 4096, 4096),
     (torch.bfloat16, 3, 1000, 1032),
     (torch.bfloat16, 16, 512, 512),
+    (torch.bfloat16, 1, 16, 8),
+    (torch.bfloat16, 1, 11008, 4096),
+    (torch.float32, 1, 336, 44),
+    (torch.bfloat16, 4, 4096, 12288),
 ])
 def test_dense_linear(L, dtype, M, d_in, d_out):
     x = sd.activations(M, d_in, 501, dtype)
     W = sd.weights(d_in, d_out, 0.02, 502, dtype)
-    got = f64(L.larosa_dense_linear(x.cuda(), W.cuda()))
+    got = f64(L.larosa_dense_linear(x.cuda(), W.t().contiguous().cuda()))
     xd, Wd = f64(x), f64(W)
     ref = oracle.dense_linear(xd, Wd)
     assert np.all(np.abs(got - ref) <= (d_in + 2) * U * (np.abs(xd) @ np.abs(Wd)) + 1e-30)
@@ -223,14 +235,14 @@ def test_dense_linear(L, dtype, M, d_in, d_out):
 
 # ---------------------------------------------------------------- fused
 
-def fused_outputs(L, x, Q, W_rot, K):
+def fused_outputs(L, x, Qt, W_rot, K):
     """Runs the fused call; returns y and the workspace copies of x_rot, idx, val."""
     M, d_in = x.shape
     d_out = W_rot.shape[1]
     ws = L.Workspace()
     buf = ws.get(M, d_in, d_out, K)
     st = status()
-    y = L.larosa_rotate_topk_linear(x, Q, W_rot, K, ws=ws, dev_status=st)
+    y = L.larosa_rotate_topk_linear(x, Qt, W_rot, K, ws=ws, dev_status=st)
     assert L.larosa_check(st) == 0
     o_x, o_i, o_v = L.larosa_workspace_layout(M, d_in, d_out, K)
     x_rot = buf[o_x:o_x + M * d_in * 4].view(torch.float32).view(M, d_in)
@@ -268,14 +280,18 @@ def check_selection(x_rot_ref, gamma, idx, K):
     (torch.bfloat16, 4, 1024, 1032, 40),
     (torch.bfloat16, 1, 4096, 4096, 50),
     (torch.bfloat16, 16, 512, 256, 25),
+    (torch.bfloat16, 1, 64, 8, 90),
+    (torch.bfloat16, 1, 200, 24, 50),
+    (torch.bfloat16, 1, 11008, 4096, 40),
 ])
 def test_fused(L, dtype, M, d_in, d_out, sparsity):
     K = sd.k_for_sparsity(d_in, sparsity)
-    Q = sd.orthogonal(d_in, 601).to(dtype)
+    Q = sd.orthogonal(d_in, 601, device="cuda" if d_in > 4096 else "cpu").to(dtype).cpu()
     W = sd.weights(d_in, d_out, 0.02 if dtype == torch.bfloat16 else 1 / 16, 602, dtype)
     x = sd.activations(M, d_in, 603, dtype)
-    W_rot = L.larosa_prepare_weights(Q.cuda(), W.cuda())
-    y, x_rot, idx, val = fused_outputs(L, x.cuda(), Q.cuda(), W_rot, K)
+    Qt = Q.t().contiguous().cuda()
+    W_rot = L.larosa_prepare_weights(Qt, W.cuda())
+    y, x_rot, idx, val = fused_outputs(L, x.cuda(), Qt, W_rot, K)
     xq, qq = f64(x), f64(Q)
     x_rot_ref = oracle.rotate(xq, qq)
     gamma = (d_in + 2) * U * (np.abs(xq) @ np.abs(qq))
@@ -297,18 +313,19 @@ def test_fused_dense_equivalence_at_full_k(L, dtype, tol):
     Q = sd.orthogonal(d_in, 701).to(dtype)
     W = sd.weights(d_in, d_out, 1 / 16, 702, dtype)
     x = sd.activations(1, d_in, 703, dtype)
-    W_rot = L.larosa_prepare_weights(Q.cuda(), W.cuda())
-    y = f64(L.larosa_rotate_topk_linear(x.cuda(), Q.cuda(), W_rot, d_in))
+    Qt = Q.t().contiguous().cuda()
+    W_rot = L.larosa_prepare_weights(Qt, W.cuda())
+    y = f64(L.larosa_rotate_topk_linear(x.cuda(), Qt, W_rot, d_in))
     ref = oracle.dense_linear(f64(x), f64(W))
     assert rel_inf(y, ref) <= tol
 
 
 def test_fused_is_deterministic(L):
     d_in, d_out, K = 4096, 4096, 2458
-    Q = sd.orthogonal(d_in, 801, device="cuda").to(torch.bfloat16)
+    Qt = sd.orthogonal(d_in, 801, device="cuda").to(torch.bfloat16).t().contiguous()
     W = sd.weights(d_in, d_out, 0.02, 802, torch.bfloat16, device="cuda")
     x = sd.activations(1, d_in, 803, torch.bfloat16).cuda()
-    W_rot = L.larosa_prepare_weights(Q, W)
-    y1 = L.larosa_rotate_topk_linear(x, Q, W_rot, K).clone()
-    y2 = L.larosa_rotate_topk_linear(x, Q, W_rot, K).clone()
+    W_rot = L.larosa_prepare_weights(Qt, W)
+    y1 = L.larosa_rotate_topk_linear(x, Qt, W_rot, K).clone()
+    y2 = L.larosa_rotate_topk_linear(x, Qt, W_rot, K).clone()
     assert torch.equal(y1, y2)

@@ -26,8 +26,8 @@ def layer():
 def test_llama2_7b_layer_group(layer, gi):
     import activation_sparsity_b200 as L
     g = layer.groups[gi]
-    y, x_rot, idx, val = fused_outputs(L, g.x, g.Q, g.W_rot, g.K)
-    xq, qq = f64(g.x), f64(g.Q)
+    y, x_rot, idx, val = fused_outputs(L, g.x, g.Qt, g.W_rot, g.K)
+    xq, qq = f64(g.x), f64(g.Qt).T
     x_rot_ref = oracle.rotate(xq, qq)
     gamma = (g.d_in + 2) * U * (np.abs(xq) @ np.abs(qq))
     assert np.all(np.abs(x_rot - x_rot_ref) <= gamma + 1e-30)
