@@ -3,7 +3,7 @@
 //
 //   rotation, dense baseline   rowdot (onetoken.cu), any M <= 16
 //   Top-K alone                topk_kernel (topk.cu)
-//   sparse linear, M = 1       gather over idx/val (onetoken.cu)
+//   sparse linear, M = 1       cluster gather over idx/val (onetoken.cu)
 //   sparse linear, M > 1       scatter + union (union.cu) + rowstream (rowstream.cu)
 //   fused, M = 1               rowdot -> select-and-gather: two kernels
 //   fused, M > 1               rowdot -> topk -> scatter/union -> rowstream
@@ -101,14 +101,11 @@ int make_layout_uncached(int M, int d_in, int d_out, int K, Layout* L) {
   for (int dt = 0; dt < 2; ++dt) {
     const Elem w = dt == 0 ? Elem::F32 : Elem::BF16;
     if (M == 1) {
-      larosa::StreamPlan sp;
-      cudaError_t e = larosa::plan_gather(w, d_out, K, &sp);
+      larosa::StreamPlan sl, ss;
+      cudaError_t e = larosa::plan_gather(larosa::kGatherList, w, d_in, d_out, K, &sl);
+      if (e == cudaSuccess) e = larosa::plan_gather(larosa::kGatherSelect, w, d_in, d_out, K, &ss);
       if (e != cudaSuccess) return cuda_fail(e, "plan gather");
-      if (sp.ok) {
-        if (sp.ticket_words > kTicketWords) return LAROSA_ERR_SHAPE;
-        partials = std::max(partials, sp.partial_floats);
-        continue;
-      }
+      if (sl.ok && ss.ok) continue;  // the cluster kernels need no partials
     }
     GemvPlan ps;
     cudaError_t e = larosa::plan_gemv(w, Elem::F32, M, d_out, sparse_rows_max(M, d_in, K), &ps);
@@ -166,7 +163,7 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
                cudaStream_t s) {
   if (M == 1) {
     larosa::StreamPlan sp;
-    cudaError_t e = larosa::plan_gather(elem_of(dtype), d_out, K, &sp);
+    cudaError_t e = larosa::plan_gather(larosa::kGatherList, elem_of(dtype), d_in, d_out, K, &sp);
     if (e != cudaSuccess) return cuda_fail(e, "plan gather");
     if (sp.ok) {
       larosa::GatherArgs a;
@@ -177,8 +174,6 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
       a.coef = val;
       a.rows = idx;
       a.y = y;
-      a.partials = reinterpret_cast<float*>(at(ws, L.partials));
-      a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTickets));
       a.dev_status = dev_status;
       e = larosa::launch_gather(larosa::kGatherList, elem_of(dtype), a, sp, s);
       return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "gather kernel");
@@ -351,7 +346,7 @@ int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, 
   if (M == 1) {
     // every CTA of the gather selects the Top-K of x_rot on its own
     larosa::StreamPlan sp;
-    cudaError_t e = larosa::plan_gather(elem_of(dtype), d_out, K, &sp);
+    cudaError_t e = larosa::plan_gather(larosa::kGatherSelect, elem_of(dtype), d_in, d_out, K, &sp);
     if (e != cudaSuccess) return cuda_fail(e, "plan gather");
     if (sp.ok) {
       larosa::GatherArgs a;
@@ -361,8 +356,6 @@ int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, 
       a.n = K;
       a.coef = x_rot;
       a.y = y;
-      a.partials = reinterpret_cast<float*>(at(ws, L.partials));
-      a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTickets));
       a.idx_out = idx;
       a.val_out = val;
       a.dev_status = dev_status;

@@ -68,16 +68,17 @@ cudaError_t launch_scatter(const int32_t* idx, const float* val, int M, int K, i
 cudaError_t launch_union(unsigned* bitmap, int d_in, int32_t* rows, int* count,
                          cudaStream_t stream);
 
-// Geometry of the one-token gather (see onetoken.cu).
+// Geometry of the one-token gather (see onetoken.cu): one cluster of
+// `cluster` CTAs per column tile of `col_tile` columns.
 struct StreamPlan {
   bool ok = false;
-  int grid = 0;            // CTAs (one per SM, fewer for tiny problems)
-  int col_tile = 0;        // output columns per tile
-  int tpr = 0;             // threads per weight row
+  int cluster = 0;
   int n_tiles = 0;
-  int max_slots = 0;       // partial slots per tile
-  size_t partial_floats = 0;
-  size_t ticket_words = 0;
+  int col_tile = 0;
+  int tpr = 0;             // threads per weight row
+  int list_cap = 0;        // kept entries per CTA
+  size_t smem = 0;         // dynamic shared memory of a launch
+  size_t smem_alloc = 0;   // the size the occupancy was computed for
 };
 
 struct GatherArgs {
@@ -88,8 +89,6 @@ struct GatherArgs {
   const void* coef = nullptr;     // kGatherList: val[K]; kGatherSelect: x_rot[d_in]
   const int32_t* rows = nullptr;  // kGatherList: idx[K]
   float* y = nullptr;
-  float* partials = nullptr;
-  unsigned* tickets = nullptr;
   int32_t* idx_out = nullptr;     // kGatherSelect: kept indices / values (optional)
   float* val_out = nullptr;
   int* dev_status = nullptr;
@@ -98,9 +97,9 @@ struct GatherArgs {
 constexpr int kGatherList = 1;    // rows idx[], coefficients val[]
 constexpr int kGatherSelect = 2;  // select the top-K of x_rot, then gather
 
-// Plans a one-token gather over an n-row list and d_out columns; plan->ok is
-// false when the shape exceeds the kernel's limits.
-cudaError_t plan_gather(Elem w_elem, int d_out, int n, StreamPlan* plan);
+// Plans a one-token gather (mode kGatherList or kGatherSelect) of K kept rows
+// of a [d_in x d_out] weight; plan->ok is false when the shape does not fit.
+cudaError_t plan_gather(int mode, Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan);
 cudaError_t launch_gather(int mode, Elem w_elem, const GatherArgs& a, const StreamPlan& plan,
                           cudaStream_t stream);
 

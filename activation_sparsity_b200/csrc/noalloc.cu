@@ -5,10 +5,11 @@
 // outputs and owns every allocation itself, or a latency-critical loop in
 // which cudaMalloc and cudaFree are forbidden because they may synchronise
 // the device.  For them larosa_sparse_linear_noalloc computes exactly what
-// larosa_sparse_linear computes, with the same kernels and launch geometry,
-// but keeps the split-K partial sums, the reduction tickets and (for several
-// tokens) the shared-row bookkeeping in one file-scope device array of fixed
-// size instead of a caller workspace.
+// larosa_sparse_linear computes, with the same kernels and launch geometry.
+// One token needs no scratch at all (the cluster gather adds its partial sums
+// in distributed shared memory); several tokens keep their split-K partial
+// sums, reduction tickets and shared-row bookkeeping in one file-scope device
+// array of fixed size instead of a caller workspace.
 //
 // That array exists once per GPU that loads this library and stays resident
 // until the process exits.  Every call on a device uses the same array, so
@@ -85,26 +86,12 @@ extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val
   const larosa::Elem w = dtype == LAROSA_BF16 ? larosa::Elem::BF16 : larosa::Elem::F32;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (M == 1) {
+    // one token: the cluster gather keeps its partial sums in distributed
+    // shared memory and needs no scratch at all
     larosa::StreamPlan sp;
-    cudaError_t e = larosa::plan_gather(w, d_out, K, &sp);
+    cudaError_t e = larosa::plan_gather(larosa::kGatherList, w, d_in, d_out, K, &sp);
     if (e != cudaSuccess) return fail_cuda(e, "plan");
     if (sp.ok) {
-      const size_t off_partials = up256(sp.ticket_words * 4);
-      const size_t total = off_partials + sp.partial_floats * 4;
-      if (total > kScratchBytes) {
-        char buf[200];
-        snprintf(buf, sizeof(buf),
-                 "larosa_sparse_linear_noalloc: these sizes need %zu bytes of scratch; the "
-                 "static scratch holds %zu",
-                 total, kScratchBytes);
-        larosa::set_last_error(buf);
-        return LAROSA_ERR_WORKSPACE;
-      }
-      unsigned char* base = nullptr;
-      e = scratch_address(reinterpret_cast<void**>(&base));
-      if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress");
-      e = cudaMemsetAsync(base, 0, sp.ticket_words * 4, s);
-      if (e != cudaSuccess) return fail_cuda(e, "clear scratch");
       larosa::GatherArgs a;
       a.W = W_rot;
       a.d_out = d_out;
@@ -113,8 +100,6 @@ extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val
       a.coef = val;
       a.rows = idx;
       a.y = y;
-      a.partials = reinterpret_cast<float*>(base + off_partials);
-      a.tickets = reinterpret_cast<unsigned*>(base);
       a.dev_status = dev_status;
       e = larosa::launch_gather(larosa::kGatherList, w, a, sp, s);
       return e == cudaSuccess ? LAROSA_OK : fail_cuda(e, "sparse linear kernel");

@@ -3,11 +3,12 @@
 // flop per byte), so the design goal is bytes in flight and one read of every
 // weight byte:
 //
-//   * one CTA of 512 threads per SM; every lane keeps eight independent
-//     16-byte loads in flight (ld.global.cs: streamed, evict-first), which a
-//     streaming probe on B200 measured at about 7 TB/s, the copy peak; TMA
-//     bulk copies into a shared ring reached only about 4.2 TB/s with one CTA
-//     per SM and were left out;
+//   * CTAs of 512 threads, two per SM where registers and shared memory
+//     allow; every lane keeps eight independent 16-byte loads in flight
+//     (ld.global.cs: streamed, evict-first).  Streaming probes on B200 put
+//     this at 5.7 (one CTA per SM) to 6.4 TB/s (two), the copy peak, even
+//     for row segments of 128-256 bytes; TMA bulk copies into a shared ring
+//     reached only about 4.2 TB/s with one CTA per SM and were left out;
 //   * a fixed reduction order everywhere, so results are bit-reproducible.
 //
 // rowdot  y[m][j] = sum_i x[m][i] * A[j][i], A row-major [n_out x n_in].
@@ -17,22 +18,28 @@
 //         reads W in torch.nn.Linear layout.  Each warp owns whole output rows:
 //         no cross-CTA reduction at all.
 //
-// gather  y[c] = sum_{p < n} coef(p) * W[row(p)][c], W row-major
+// gather  y[c] = sum_{p < K} coef(p) * W[row(p)][c], W row-major
 //         [d_in x d_out]: the sparse linear over the kept rows of the
 //         counter-rotated weight (abstract: activation sparsity reduces memory
-//         transfers).  Work = (column tile, list position) pairs, tile-major,
-//         cut into equal contiguous ranges, one per CTA (at most two tiles per
-//         range).  Partials of a tile are added in CTA order by the
-//         last-arriving contributor (atomic ticket, no waiting).
+//         transfers).  One thread-block cluster per column tile; the cluster's
+//         CTAs take equal consecutive parts of the kept list and add their
+//         partial sums through distributed shared memory in rank order, so
+//         nothing leaves the cluster but y.  The tile width is chosen so the
+//         clusters that fit on the GPU at once cover d_out.
 //           kGather  row(p) = idx[p], coef(p) = val[p]
 //           kSelect  every CTA first selects the K largest |x_rot| itself
 //                    (exact, ties to the lower index; no grid-wide handoff),
-//                    then gathers them.
+//                    then gathers its part of them.
+#include <cooperative_groups.h>
+
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace larosa {
 namespace {
@@ -88,7 +95,7 @@ struct RParams {
 // One warp, one output row, MT tokens.  Lane l handles the 8-element vectors
 // l, l+32, l+64, ... of the row; kU of them are loaded before any is used.
 template <typename T, int MT>
-__global__ void __launch_bounds__(kT, 1) rowdot_kernel(const RParams p) {
+__global__ void __launch_bounds__(kT, (MT <= 2 && sizeof(T) == 2 ? 2 : 1)) rowdot_kernel(const RParams p) {
   extern __shared__ __align__(16) unsigned char xs_raw[];
   const T* xs = reinterpret_cast<const T*>(xs_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -158,168 +165,272 @@ __global__ void __launch_bounds__(kT, 1) rowdot_kernel(const RParams p) {
 
 constexpr int kModeGather = 1;
 constexpr int kModeSelect = 2;
-constexpr int kMaxUnits = 4096;   // list positions a CTA holds
-constexpr int kCandCap = 2048;
-constexpr int kXrotMax = 32768;   // selection buffer (fp32 words)
+constexpr int kCandCap = 1024;
 
 struct GParams {
   const void* W;         // [d_in x d_out] row-major
   int d_out;
-  int row_bound;         // d_in (also the length of x_rot)
-  int n;                 // list length (K)
-  const void* coef;      // gather: val; select: x_rot
-  const int32_t* rows;   // gather: idx
+  int d_in;              // row bound; also the length of x_rot
+  int K;                 // kept entries
+  const void* coef;      // gather: val[K]; select: x_rot[d_in]
+  const int32_t* rows;   // gather: idx[K]
   float* y;
-  float* partials;
-  unsigned* tickets;
   int col_tile;
-  int n_tiles;
   int tpr;
-  int max_slots;
+  int list_cap;          // list entries a CTA holds: ceil(K / cluster)
   int32_t* idx_out;      // select: kept indices/values (optional)
   float* val_out;
   int* dev_status;
 };
 
-struct GSmem {
-  SelectScratch sel;
-  int flags[4];
-  int32_t rows[kMaxUnits];
-  float coefs[kMaxUnits];
-  uint32_t cand[kCandCap];
-  float red[kT * 8];     // row groups x column tile (<= 4096 floats of 8 per thread)
+// Shared memory of one CTA, laid out from sizes known at launch.
+struct GLayout {
+  size_t sel, merged, xchg, keys, rows, vals, part, red, total;
 };
 
-__device__ __forceinline__ void tile_contributors(long long U, int G, int n, int t, int* first,
-                                                  int* last) {
-  const long long a = ((long long)t * n + 1) * G - 1;
-  const long long b = ((long long)(t + 1) * n) * G - 1;
-  *first = (int)max(0LL, a / U);
-  *last = (int)min((long long)G - 1, b / U);
+__host__ __device__ inline size_t al16(size_t v) { return (v + 15) & ~size_t(15); }
+
+// list_cap: list entries a CTA holds (kept positions of its part, or kept
+// entries of its index range); key_cap: rotated entries a CTA owns (select).
+__host__ __device__ inline GLayout glayout(int mode, int key_cap, int list_cap, int col_tile,
+                                           int cpt) {
+  GLayout L;
+  size_t o = 0;
+  const bool sel = mode == kModeSelect;
+  L.sel = o;      o = al16(o + (sel ? sizeof(SelectScratch) : 64));
+  L.merged = o;   o = al16(o + (sel ? kSelBins * 4 : 0));
+  L.xchg = o;     o = al16(o + (sel ? 64 * 4 : 0));
+  L.keys = o;     o = al16(o + (sel ? (size_t)key_cap * 4 : 0));
+  L.rows = o;     o = al16(o + (size_t)list_cap * 4);
+  L.vals = o;     o = al16(o + (size_t)list_cap * 4);
+  L.part = o;     o = al16(o + (size_t)col_tile * 4);
+  L.red = o;      o = al16(o + (size_t)kT * cpt * 4);
+  L.total = o;
+  return L;
 }
 
+// One radix pass of a selection spread over a cluster: histogram this CTA's
+// keys that match `prefix` under `mask` on digit (key >> shift) & (nb-1),
+// add the cluster's histograms (rank r adds bins [r*nb/C, (r+1)*nb/C) and
+// writes the sums into every CTA's `merged`), then find the bin holding the
+// krem-th largest counted key.  Writes bin, keys above it, keys in it to
+// pick[0], pick[1], pick[3].  `hist` (both copies) must be zero on entry and
+// is zero again on return.
+template <int NT>
+__device__ __forceinline__ void cluster_radix_pass(cg::cluster_group& cl, int C, int rank,
+                                                   const uint32_t* keys, int n_mine,
+                                                   uint32_t prefix, uint32_t mask, int shift,
+                                                   int nb, uint32_t krem, SelectScratch* s,
+                                                   uint32_t* merged) {
+  const int tid = threadIdx.x;
+  uint32_t* h = s->hist + (tid & 1) * kSelBins;
+  for (int i = tid; i < n_mine; i += NT) {
+    const uint32_t k = keys[i] & kKeyMask;
+    if ((k & mask) == prefix) atomicAdd(&h[(k >> shift) & static_cast<uint32_t>(nb - 1)], 1u);
+  }
+  __syncthreads();
+  for (int b = tid; b < nb; b += NT) {
+    s->hist[b] += s->hist[kSelBins + b];
+    s->hist[kSelBins + b] = 0u;
+  }
+  cl.sync();  // every CTA's histogram is final
+  const int b0 = (int)((long long)nb * rank / C), b1 = (int)((long long)nb * (rank + 1) / C);
+  for (int b = b0 + tid; b < b1; b += NT) {
+    uint32_t sum = 0;
+    for (int q = 0; q < C; ++q) sum += cl.map_shared_rank(s->hist, q)[b];
+    for (int q = 0; q < C; ++q) cl.map_shared_rank(merged, q)[b] = sum;
+  }
+  cl.sync();  // merged everywhere; no CTA still reads another's `hist`
+  for (int b = tid; b < nb; b += NT) s->hist[b] = 0u;
+  // boundary bin, counting from the top: thread t owns ranks [t*per, t*per+per)
+  constexpr int kPer = (kSelBins + NT - 1) / NT;
+  const int per = (nb + NT - 1) / NT;
+  uint32_t cnt[kPer];
+  uint32_t own = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int k = tid * per + j;
+    cnt[j] = (j < per && k < nb) ? merged[nb - 1 - k] : 0u;
+    own += cnt[j];
+  }
+  uint32_t before = block_scan_excl_1s<NT>(own, s->warp_sums, nullptr);
+  if (before < krem && krem <= before + own) {
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (j < per && before < krem && krem <= before + cnt[j]) {
+        s->pick[0] = static_cast<uint32_t>(nb - 1 - (tid * per + j));
+        s->pick[1] = before;
+        s->pick[3] = cnt[j];
+      }
+      before += cnt[j];
+    }
+  }
+  __syncthreads();
+}
+
+// One cluster per column tile; the cluster's CTAs split the kept list in
+// rank order, and their partial sums meet in distributed shared memory.
 template <typename Tw, int MODE>
-__global__ void __launch_bounds__(kT, 1) gather_kernel(const GParams p) {
+__global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
   constexpr int CPT = 16 / sizeof(Tw);  // columns per thread per row
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  GSmem& S = *reinterpret_cast<GSmem*>(smem_raw);
-  uint32_t* bits = reinterpret_cast<uint32_t*>(smem_raw + sizeof(GSmem));  // select buffer
+  cg::cluster_group cl = cg::this_cluster();
+  const int C = static_cast<int>(cl.num_blocks());
+  const int rank = static_cast<int>(cl.block_rank());
+  const int key_cap = (p.d_in + C - 1) / C;
+  const GLayout L = glayout(MODE, key_cap, p.list_cap, p.col_tile, CPT);
+  SelectScratch* sel = reinterpret_cast<SelectScratch*>(smem_raw + L.sel);
+  int32_t* lrows = reinterpret_cast<int32_t*>(smem_raw + L.rows);
+  float* lvals = reinterpret_cast<float*>(smem_raw + L.vals);
+  float* part = reinterpret_cast<float*>(smem_raw + L.part);
+  float* red = reinterpret_cast<float*>(smem_raw + L.red);
 
   const int tid = threadIdx.x;
-  const int G = gridDim.x, cta = blockIdx.x;
+  const int tile = blockIdx.y;
+  const int c0 = tile * p.col_tile;
+  const int wc = min(p.col_tile, p.d_out - c0);
+  const int K = p.K;
+  int len = 0;  // rows this CTA streams
+
+  if constexpr (MODE == kModeSelect) {
+    for (int b = tid; b < 2 * kSelBins; b += kT) sel->hist[b] = 0u;
+  }
   pdl_wait();
   pdl_launch_dependents();
 
-  const int n = p.n;
-  if (n == 0) {  // nothing kept: y = 0
-    const int per = (p.d_out + G - 1) / G;
-    for (int i = cta * per + tid; i < min(p.d_out, (cta + 1) * per); i += kT) p.y[i] = 0.f;
-    return;
-  }
-
-  // ---- this CTA's (at most two) segments: tile t, positions [a, b), slot offset
-  const long long U = (long long)p.n_tiles * n;
-  const long long u0 = U * cta / G;
-  const long long u1 = U * (cta + 1) / G;
-  const int t0 = (int)(u0 / n);
-  const int s0a = (int)(u0 - (long long)t0 * n);
-  const int s0b = (int)min((long long)n, u1 - (long long)t0 * n);
-  const bool two = u1 > (long long)(t0 + 1) * n;
-  const int t1 = t0 + 1;
-  const int s1b = two ? (int)(u1 - (long long)t1 * n) : 0;
-  const int len0 = s0b - s0a;
-  const int len1 = s1b;  // segment 1 starts at position 0 of tile t1
-
   if constexpr (MODE == kModeGather) {
+    // rank r takes the kept positions [K*r/C, K*(r+1)/C)
+    const int p0 = (int)((long long)K * rank / C);
+    const int p1 = (int)((long long)K * (rank + 1) / C);
+    len = p1 - p0;
     bool bad = false;
-    for (int j = tid; j < len0 + len1; j += kT) {
-      const int pos = j < len0 ? s0a + j : j - len0;
-      const int row = p.rows[pos];
-      const bool ok = static_cast<unsigned>(row) < static_cast<unsigned>(p.row_bound);
+    for (int j = tid; j < len; j += kT) {
+      const int row = p.rows[p0 + j];
+      const bool ok = static_cast<unsigned>(row) < static_cast<unsigned>(p.d_in);
       bad |= !ok;
-      S.rows[j] = ok ? row : 0;
-      S.coefs[j] = ok ? static_cast<const float*>(p.coef)[pos] : 0.f;
+      lrows[j] = ok ? row : 0;
+      lvals[j] = ok ? static_cast<const float*>(p.coef)[p0 + j] : 0.f;
     }
     if (__syncthreads_or(bad) && tid == 0) report(p.dev_status, LAROSA_DEV_INDEX);
   } else {
-    const int d = p.row_bound;
+    // rank r owns the rotated entries [d*r/C, d*(r+1)/C) and gathers the kept
+    // ones among them; the threshold is found by radix passes whose
+    // histograms are added across the cluster
+    const int d = p.d_in;
+    const int i_lo = (int)((long long)d * rank / C);
+    const int n_mine = (int)((long long)d * (rank + 1) / C) - i_lo;
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + L.keys);
+    uint32_t* merged = reinterpret_cast<uint32_t*>(smem_raw + L.merged);
+    uint32_t* xchg = reinterpret_cast<uint32_t*>(smem_raw + L.xchg);  // [0,32) > T, [32,64) == T
     {
-      const uint4* src = static_cast<const uint4*>(p.coef);
-      const int nv = d >> 2;
+      const float* src = static_cast<const float*>(p.coef) + i_lo;
       bool nonfinite = false;
-#pragma unroll 4
-      for (int i = tid; i < nv; i += kT) {
-        const uint4 u = __ldcg(src + i);
-        reinterpret_cast<uint4*>(bits)[i] = u;
-        nonfinite |= ((u.x & kKeyMask) >= 0x7f800000u) | ((u.y & kKeyMask) >= 0x7f800000u) |
-                     ((u.z & kKeyMask) >= 0x7f800000u) | ((u.w & kKeyMask) >= 0x7f800000u);
+      for (int i = tid; i < n_mine; i += kT) {
+        const uint32_t u = __float_as_uint(__ldcg(src + i));
+        keys[i] = u;
+        nonfinite |= (u & kKeyMask) >= 0x7f800000u;
       }
-      if (__syncthreads_or(nonfinite) && tid == 0 && cta == 0)
+      if (__syncthreads_or(nonfinite) && tid == 0 && tile == 0)
         report(p.dev_status, LAROSA_DEV_NONFINITE);
     }
-    const int K = n;
-    const bool all = K >= d;
     uint32_t T = 0, krem = 0;
-    if (!all) select_threshold<kT>(bits, d, K, &S.sel, S.cand, kCandCap, &T, &krem);
-    const int chunk = (d + kT - 1) / kT;
-    const int i0 = min(d, tid * chunk);
-    const int i1 = min(d, i0 + chunk);
+    const bool all = K >= d;
+    if (K > 0 && !all) {
+      uint32_t prefix = 0, mask = 0;
+      krem = static_cast<uint32_t>(K);
+#pragma unroll 1
+      for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 20 : (pass == 1 ? 9 : 0);
+        const int nb = pass == 2 ? 512 : 2048;
+        cluster_radix_pass<kT>(cl, C, rank, keys, n_mine, prefix, mask, shift, nb, krem, sel,
+                               merged);
+        prefix |= sel->pick[0] << shift;
+        mask |= static_cast<uint32_t>(nb - 1) << shift;
+        krem -= sel->pick[1];
+        __syncthreads();
+      }
+      T = prefix;  // krem keys equal to T are kept: the lowest-indexed ones
+    }
+    // this CTA's counts above / at the threshold, exchanged across the cluster
+    const int chunk = (n_mine + kT - 1) / kT;
+    const int j0 = min(n_mine, tid * chunk), j1 = min(n_mine, j0 + chunk);
     uint32_t gt = 0, eq = 0;
-    if (!all) kept_chunk_base<kT>(bits, i0, i1, T, &S.sel, &gt, &eq);
-    const bool write_out = p.idx_out != nullptr;
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t u = bits[i];
+    if (all) {
+      gt = (uint32_t)(j1 - j0);  // everything is kept
+    } else if (K > 0) {
+      for (int j = j0; j < j1; ++j) {
+        const uint32_t k = keys[j] & kKeyMask;
+        gt += k > T;
+        eq += k == T;
+      }
+    }
+    uint32_t tot = 0;
+    const uint32_t packed = block_scan_excl_1s<kT>((eq << 16) | gt, sel->warp_sums, &tot);
+    uint32_t gt_before = packed & 0xffffu, eq_before = packed >> 16;
+    const bool want_positions = tile == 0 && p.idx_out != nullptr;
+    if (tid == 0) {
+      for (int q = 0; q < C; ++q) {
+        cl.map_shared_rank(xchg, q)[rank] = tot & 0xffffu;
+        cl.map_shared_rank(xchg, q)[32 + rank] = tot >> 16;
+      }
+    }
+    cl.sync();  // every CTA's counts are in every CTA
+    uint32_t ties_before = 0, kept_before = 0;
+    for (int q = 0; q < rank; ++q) {
+      const uint32_t tq = xchg[32 + q];
+      kept_before += xchg[q] + min(tq, krem > ties_before ? krem - ties_before : 0u);
+      ties_before += tq;
+    }
+    // kept entries of this CTA before j0; the chunk's kept entries follow in
+    // index order
+    uint32_t pos_local = gt_before + min(eq_before, krem > ties_before ? krem - ties_before : 0u);
+    uint32_t eqc = eq_before;
+    for (int j = j0; j < j1; ++j) {
+      const uint32_t u = keys[j];
       const uint32_t k = u & kKeyMask;
-      int pos;
-      if (all) {
-        pos = i;
-      } else if (k > T) {
-        pos = (int)(gt + min(eq, krem));
-        ++gt;
-      } else if (k == T && eq < krem) {
-        pos = (int)(gt + eq);
-        ++eq;
+      bool kept;
+      if (K == 0) {
+        kept = false;
+      } else if (all || k > T) {
+        kept = true;
+      } else if (k == T) {
+        kept = eqc + ties_before < krem;
+        ++eqc;
       } else {
-        if (k == T) ++eq;
-        continue;
+        kept = false;
       }
-      const float val = __uint_as_float(u);
-      if (pos >= s0a && pos < s0b) {
-        S.rows[pos - s0a] = i;
-        S.coefs[pos - s0a] = val;
-        if (t0 == 0 && write_out) {
-          p.idx_out[pos] = i;
-          p.val_out[pos] = val;
+      if (kept) {
+        const float v = __uint_as_float(u);
+        lrows[pos_local] = i_lo + j;
+        lvals[pos_local] = v;
+        if (want_positions) {
+          p.idx_out[kept_before + pos_local] = i_lo + j;
+          p.val_out[kept_before + pos_local] = v;
         }
+        ++pos_local;
       }
-      if (pos < s1b) {
-        S.rows[len0 + pos] = i;
-        S.coefs[len0 + pos] = val;
-      }
+    }
+    // rows this CTA streams
+    {
+      const uint32_t gt_all = tot & 0xffffu, eq_all = tot >> 16;
+      len = (int)(K == 0 ? 0u
+                  : all ? (uint32_t)n_mine
+                        : gt_all + min(eq_all, krem > ties_before ? krem - ties_before : 0u));
     }
     __syncthreads();
   }
 
-  // ---- stream the rows: thread (g, col) reads 16 bytes of rows g, g+ng, ...
+  // ---- stream the kept rows of this tile: thread (g, col) reads 16 bytes
+  // of rows g, g+ng, ..., with kU loads in flight
   const int tpr = p.tpr;
-  const int g = tid / tpr;
   const int ng = kT / tpr;
-  const int col = (tid % tpr) * CPT;
-  float acc[2][CPT];
+  const int g = tid / tpr;
+  const int col = (tid - g * tpr) * CPT;
+  const bool active = g < ng && col < wc;
+  float acc[CPT];
 #pragma unroll
-  for (int s = 0; s < 2; ++s)
-#pragma unroll
-    for (int v = 0; v < CPT; ++v) acc[s][v] = 0.f;
-
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    const int t = s == 0 ? t0 : t1;
-    const int len = s == 0 ? len0 : len1;
-    const int off = s == 0 ? 0 : len0;
-    if (len == 0) continue;
-    const int c0 = t * p.col_tile;
-    const int wc = min(p.col_tile, p.d_out - c0);
-    if (col >= wc) continue;
+  for (int v = 0; v < CPT; ++v) acc[v] = 0.f;
+  if (active) {
     const unsigned char* wbase = static_cast<const unsigned char*>(p.W) + ((size_t)c0 + col) * sizeof(Tw);
     const size_t pitch = (size_t)p.d_out * sizeof(Tw);
     for (int r0 = g; r0 < len; r0 += ng * kU) {
@@ -327,79 +438,49 @@ __global__ void __launch_bounds__(kT, 1) gather_kernel(const GParams p) {
 #pragma unroll
       for (int k = 0; k < kU; ++k) {
         const int r = r0 + k * ng;
-        u[k] = r < len ? ld_stream(wbase + (size_t)S.rows[off + r] * pitch) : make_uint4(0, 0, 0, 0);
+        u[k] = r < len ? ld_stream(wbase + (size_t)lrows[r] * pitch) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int k = 0; k < kU; ++k) {
         const int r = r0 + k * ng;
-        if (r < len) {
-          const float cf = S.coefs[off + r];
-          if constexpr (CPT == 8) {
-            float w[8];
-            Vec8<__nv_bfloat16>::cvt(&u[k], w);
+        const float cf = r < len ? lvals[r] : 0.f;
+        if constexpr (CPT == 8) {
+          float w[8];
+          Vec8<__nv_bfloat16>::cvt(&u[k], w);
 #pragma unroll
-            for (int v = 0; v < 8; ++v) acc[s][v] = fmaf(cf, w[v], acc[s][v]);
-          } else {
-            acc[s][0] = fmaf(cf, __uint_as_float(u[k].x), acc[s][0]);
-            acc[s][1] = fmaf(cf, __uint_as_float(u[k].y), acc[s][1]);
-            acc[s][2] = fmaf(cf, __uint_as_float(u[k].z), acc[s][2]);
-            acc[s][3] = fmaf(cf, __uint_as_float(u[k].w), acc[s][3]);
-          }
+          for (int v = 0; v < 8; ++v) acc[v] = fmaf(cf, w[v], acc[v]);
+        } else {
+          acc[0] = fmaf(cf, __uint_as_float(u[k].x), acc[0]);
+          acc[1] = fmaf(cf, __uint_as_float(u[k].y), acc[1]);
+          acc[2] = fmaf(cf, __uint_as_float(u[k].z), acc[2]);
+          acc[3] = fmaf(cf, __uint_as_float(u[k].w), acc[3]);
         }
       }
     }
   }
 
-  // ---- per segment: row groups -> CTA partial -> tile result
+  // ---- row groups -> this CTA's partial, in shared memory
+  if (active) {
 #pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    const int t = s == 0 ? t0 : t1;
-    const int len = s == 0 ? len0 : len1;
-    if (len == 0) continue;  // uniform across the CTA
-    const int c0 = t * p.col_tile;
-    const int wc = min(p.col_tile, p.d_out - c0);
-    __syncthreads();  // S.red free
-    if (col < wc) {
-#pragma unroll
-      for (int v = 0; v < CPT; ++v) S.red[g * p.col_tile + col + v] = acc[s][v];
-    }
-    __syncthreads();
-    int first = 0, last = 0;
-    tile_contributors(U, G, n, t, &first, &last);
-    const int n_contrib = last - first + 1;
-    float* mine = p.partials + ((size_t)t * p.max_slots + (cta - first)) * p.col_tile;
-    for (int e = tid; e < wc; e += kT) {
-      float sum = 0.f;
-      for (int gg = 0; gg < ng; ++gg) sum += S.red[gg * p.col_tile + e];
-      if (n_contrib == 1)
-        p.y[c0 + e] = sum;
-      else
-        mine[e] = sum;
-    }
-    if (n_contrib > 1) {
-      __threadfence();
-      __syncthreads();
-      if (tid == 0) S.flags[0] = static_cast<int>(atomicAdd(&p.tickets[t], 1u));
-      __syncthreads();
-      if (S.flags[0] == n_contrib - 1) {
-        __threadfence();
-        const float* all = p.partials + (size_t)t * p.max_slots * p.col_tile;
-        for (int e4 = tid * 4; e4 < wc; e4 += kT * 4) {
-          float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int q = 0; q < n_contrib; ++q) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(all + (size_t)q * p.col_tile + e4));
-            acc4.x += v.x; acc4.y += v.y; acc4.z += v.z; acc4.w += v.w;
-          }
-          *reinterpret_cast<float4*>(p.y + c0 + e4) = acc4;
-        }
-        if (tid == 0) atomicExch(&p.tickets[t], 0u);
-      }
-    }
+    for (int v = 0; v < CPT; ++v) red[g * p.col_tile + col + v] = acc[v];
   }
+  __syncthreads();
+  for (int e = tid; e < wc; e += kT) {
+    float sum = 0.f;
+    for (int gg = 0; gg < ng; ++gg) sum += red[gg * p.col_tile + e];
+    part[e] = sum;
+  }
+  // ---- the cluster's partials -> y: rank r adds its column slice in rank order
+  cl.sync();
+  const int sl = (wc + C - 1) / C;
+  const int e0 = rank * sl, e1 = min(wc, e0 + sl);
+  for (int e = e0 + tid; e < e1; e += kT) {
+    float sum = 0.f;
+    for (int q = 0; q < C; ++q) sum += cl.map_shared_rank(part, q)[e];
+    p.y[c0 + e] = sum;
+  }
+  cl.sync();  // no CTA leaves while another may still read its partial
 }
-
-constexpr size_t kGatherSmem = sizeof(GSmem);
-constexpr size_t kSelectSmem = sizeof(GSmem) + (size_t)kXrotMax * 4;
 
 struct DevState {
   int sms = 0;
@@ -483,88 +564,151 @@ cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M,
   p.n_out = n_out;
   p.M = M;
   p.x_in_smem = in_smem ? 1 : 0;
-  const int grid = std::max(1, std::min(ds->sms, n_out));
+  const int per_sm = (MT <= 2 && e == Elem::BF16) ? 2 : 1;
+  const int grid = std::max(1, std::min(ds->sms * per_sm, n_out));
   return launch(fn, grid, in_smem ? xbytes : 0, &p, stream);
 }
 
-cudaError_t plan_gather(Elem w_elem, int d_out, int n, StreamPlan* plan) {
-  DevState* ds = nullptr;
-  cudaError_t e = dev_state(&ds);
-  if (e != cudaSuccess) return e;
-  const int G = ds->sms;
-  const int cpt = w_elem == Elem::BF16 ? 8 : 4;
-  StreamPlan best, fallback;
-  // the widest column tile whose last-contributor reduction stays small
-  for (int tpr = kT; tpr >= 32; tpr /= 2) {
-    const int wc = tpr * cpt;
-    if (tpr > 32 && wc / 2 >= d_out) continue;  // mostly idle threads
-    const int n_tiles = (d_out + wc - 1) / wc;
-    if (n_tiles > G) continue;
-    const long long U = (long long)n_tiles * n;
-    const int grid = (int)std::max(1LL, std::min<long long>(G, U));
-    if ((U + grid - 1) / grid > kMaxUnits) continue;
-    int max_slots = 1;
-    for (int t = 0; n > 0 && t < n_tiles; ++t) {
-      const long long a = ((long long)t * n + 1) * grid - 1;
-      const long long b = ((long long)(t + 1) * n) * grid - 1;
-      const int first = (int)std::max(0LL, a / U);
-      const int last = (int)std::min((long long)grid - 1, b / U);
-      max_slots = std::max(max_slots, last - first + 1);
-    }
-    StreamPlan pl;
-    pl.ok = true;
-    pl.grid = grid;
-    pl.col_tile = wc;
-    pl.tpr = tpr;
-    pl.n_tiles = n_tiles;
-    pl.max_slots = max_slots;
-    pl.partial_floats = (size_t)n_tiles * max_slots * wc;
-    pl.ticket_words = n_tiles;
-    fallback = pl;
-    if ((size_t)max_slots * wc * 4 <= 64 * 1024) {
-      best = pl;
-      break;
+namespace {
+
+// Largest number of co-resident clusters of C CTAs for a kernel and shared
+// memory size, cached per device.
+struct ClusterOcc {
+  void* fn;
+  size_t smem;
+  int C;
+  int clusters;
+};
+std::mutex g_occ_mu;
+ClusterOcc g_occ[64][64];
+int g_occ_n[64] = {0};
+
+cudaError_t max_clusters(int dev, void* fn, size_t smem, int C, int* out) {
+  {
+    std::lock_guard<std::mutex> lock(g_occ_mu);
+    for (int i = 0; i < g_occ_n[dev]; ++i) {
+      const ClusterOcc& o = g_occ[dev][i];
+      if (o.fn == fn && o.smem == smem && o.C == C) {
+        *out = o.clusters;
+        return cudaSuccess;
+      }
     }
   }
-  *plan = best.ok ? best : fallback;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C, 64, 1);
+  cfg.blockDim = dim3(kT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, fn, &cfg);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  std::lock_guard<std::mutex> lock(g_occ_mu);
+  if (g_occ_n[dev] < 64) g_occ[dev][g_occ_n[dev]++] = ClusterOcc{fn, smem, C, n};
+  *out = n;
+  return cudaSuccess;
+}
+
+void* gather_fn(Elem w, int mode) {
+  if (w == Elem::BF16)
+    return mode == kGatherSelect ? reinterpret_cast<void*>(&gather_kernel<__nv_bfloat16, kModeSelect>)
+                                 : reinterpret_cast<void*>(&gather_kernel<__nv_bfloat16, kModeGather>);
+  return mode == kGatherSelect ? reinterpret_cast<void*>(&gather_kernel<float, kModeSelect>)
+                               : reinterpret_cast<void*>(&gather_kernel<float, kModeGather>);
+}
+
+}  // namespace
+
+cudaError_t plan_gather(int mode, Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const int cpt = w_elem == Elem::BF16 ? 8 : 4;
+  const int kmode = mode == kGatherSelect ? kModeSelect : kModeGather;
+  void* fn = gather_fn(w_elem, mode);
+  StreamPlan best;
+  long long best_ctas = -1;
+  for (int C = 8; C >= 2; C /= 2) {
+    const int key_cap = (d_in + C - 1) / C;
+    // list mode: the rank's share of the kept list; select mode: the kept
+    // entries of the rank's index range
+    const int list_cap = std::max(1, kmode == kModeSelect ? key_cap : (K + C - 1) / C);
+    // column tile: fill the co-resident clusters, at least 64 columns wide
+    // (128 bytes of bf16) and at most one 16-byte vector per thread
+    const int wc_max = kT * cpt;
+    const size_t smem_probe = glayout(kmode, key_cap, list_cap, wc_max, cpt).total;
+    if (smem_probe > 227 * 1024) continue;
+    int clusters = 0;
+    e = max_clusters(dev, fn, smem_probe, C, &clusters);
+    if (e != cudaSuccess) return e;
+    if (clusters <= 0) continue;
+    int wc = (d_out + clusters - 1) / clusters;
+    wc = std::max(wc, std::min(64, d_out));
+    wc = (wc + cpt - 1) / cpt * cpt;
+    wc = std::min(wc, wc_max);
+    const int n_tiles = (d_out + wc - 1) / wc;
+    const long long ctas = (long long)std::min(n_tiles, clusters) * C;
+    if (ctas > best_ctas) {
+      best_ctas = ctas;
+      best.ok = true;
+      best.cluster = C;
+      best.n_tiles = n_tiles;
+      best.col_tile = wc;
+      best.tpr = wc / cpt;
+      best.list_cap = list_cap;
+      best.smem = glayout(kmode, key_cap, list_cap, wc, cpt).total;
+      best.smem_alloc = smem_probe;
+    }
+  }
+  *plan = best;
   return cudaSuccess;
 }
 
 cudaError_t launch_gather(int mode, Elem w_elem, const GatherArgs& a, const StreamPlan& pl,
                           cudaStream_t stream) {
   if (!pl.ok) return cudaErrorInvalidValue;
-  DevState* ds = nullptr;
-  cudaError_t e = dev_state(&ds);
-  if (e != cudaSuccess) return e;
-  const bool sel = mode == kGatherSelect;
-  void* fn;
-  if (w_elem == Elem::BF16)
-    fn = sel ? reinterpret_cast<void*>(&gather_kernel<__nv_bfloat16, kModeSelect>)
-             : reinterpret_cast<void*>(&gather_kernel<__nv_bfloat16, kModeGather>);
-  else
-    fn = sel ? reinterpret_cast<void*>(&gather_kernel<float, kModeSelect>)
-             : reinterpret_cast<void*>(&gather_kernel<float, kModeGather>);
-  const size_t smem = sel ? kSelectSmem : kGatherSmem;
-  e = configure(ds, 10 + (w_elem == Elem::BF16 ? 2 : 0) + (sel ? 1 : 0), fn, smem);
-  if (e != cudaSuccess) return e;
+  void* fn = gather_fn(w_elem, mode);
   GParams p;
   p.W = a.W;
   p.d_out = a.d_out;
-  p.row_bound = a.row_bound;
-  p.n = a.n;
+  p.d_in = a.row_bound;
+  p.K = a.n;
   p.coef = a.coef;
   p.rows = a.rows;
   p.y = a.y;
-  p.partials = a.partials;
-  p.tickets = a.tickets;
   p.col_tile = pl.col_tile;
-  p.n_tiles = pl.n_tiles;
   p.tpr = pl.tpr;
-  p.max_slots = pl.max_slots;
+  p.list_cap = pl.list_cap;
   p.idx_out = a.idx_out;
   p.val_out = a.val_out;
   p.dev_status = a.dev_status;
-  return launch(fn, pl.grid, smem, &p, stream);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.cluster, pl.n_tiles, 1);
+  cfg.blockDim = dim3(kT, 1, 1);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = pl.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  void* args[] = {&p};
+  return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
 }  // namespace larosa

@@ -38,7 +38,7 @@ constexpr uint32_t kKeyMask = 0x7fffffffu;
 struct SelectScratch {
   uint32_t hist[2 * kSelBins];  // two interleaved copies during counting
   uint32_t warp_sums[32];
-  uint32_t pick[4];             // boundary bin, keys above it, candidate count
+  uint32_t pick[8];  // [0] bin [1] keys above [2] candidates [3] bin count [4] ties kept [5] T
 };
 
 // Inclusive prefix sum of v over the NT threads of the block.  Contains
@@ -202,6 +202,173 @@ __device__ __forceinline__ void kept_chunk_base(const uint32_t* bits, int i0, in
   }
   const uint32_t packed = (eq << 16) | gt;  // d < 65536: no carry between halves
   const uint32_t excl = block_scan_incl<NT>(packed, s->warp_sums) - packed;
+  *gt_before = excl & 0xffffu;
+  *eq_before = excl >> 16;
+}
+
+// Exclusive prefix sum of v over the NT threads with a single barrier.  The
+// caller must place a barrier between two uses of warp_sums.
+template <int NT>
+__device__ __forceinline__ uint32_t block_scan_excl_1s(uint32_t v, uint32_t* warp_sums,
+                                                       uint32_t* total) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  uint32_t inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) warp_sums[warp] = inc;
+  __syncthreads();
+  uint32_t base = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const uint32_t ws = warp_sums[w];
+    base += w < warp ? ws : 0u;
+    all += ws;
+  }
+  if (total != nullptr) *total = all;
+  return base + inc - v;
+}
+
+// Same result as select_threshold, with fewer barriers: after the pass-1
+// histogram the keys of the boundary bin (at most cand_cap of them) are ranked
+// against each other directly -- larger key first, lower index first among
+// equal keys -- instead of two more radix passes.  Falls back to
+// select_threshold when the boundary bin holds more than cand_cap keys.
+// cand_key / cand_idx: shared arrays of cand_cap entries.  Requires
+// 1 <= K < d; s->hist must be zero on entry (both copies, all 2048 bins) and
+// the first barrier after that must come before this call's counting, which
+// the caller provides.
+template <int NT>
+__device__ __forceinline__ void select_threshold_fast(const uint32_t* bits, int d, int K,
+                                                      SelectScratch* s, uint32_t* cand_key,
+                                                      uint32_t* cand_idx, int cand_cap,
+                                                      uint32_t* T_out, uint32_t* krem_out) {
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  constexpr int NW = NT / 32;
+  uint32_t* h = s->hist + (lane & 1) * kSelBins;
+
+  // ---- pass 1: bits 30..20 over all keys
+#pragma unroll 4
+  for (int i = tid; i < d; i += NT) atomicAdd(&h[(bits[i] & kKeyMask) >> 20], 1u);
+  if (tid == 0) {
+    s->pick[2] = 0;
+    s->pick[4] = 0;
+  }
+  __syncthreads();
+
+  // ---- boundary bin with one barrier: thread t owns ranks [t*per, t*per+per)
+  constexpr int kPer = (kSelBins + NT - 1) / NT;
+  uint32_t cnt[kPer];
+  uint32_t own = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int k = tid * kPer + j;  // rank from the top
+    const int b = kSelBins - 1 - k;
+    cnt[j] = k < kSelBins ? s->hist[b] + s->hist[kSelBins + b] : 0u;
+    own += cnt[j];
+  }
+  const uint32_t before0 = block_scan_excl_1s<NT>(own, s->warp_sums, nullptr);
+  {
+    uint32_t before = before0;
+    const uint32_t krem = static_cast<uint32_t>(K);
+    if (before < krem && krem <= before + own) {
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        if (before < krem && krem <= before + cnt[j]) {
+          s->pick[0] = static_cast<uint32_t>(kSelBins - 1 - (tid * kPer + j));
+          s->pick[1] = before;
+          s->pick[3] = cnt[j];
+        }
+        before += cnt[j];
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t b1 = s->pick[0];
+  const uint32_t n1 = s->pick[3];
+  const uint32_t krem1 = static_cast<uint32_t>(K) - s->pick[1];  // to take from bin b1
+  constexpr int kMaxOwn = 4;  // candidates ranked per thread
+  if (n1 > static_cast<uint32_t>(cand_cap) || n1 > static_cast<uint32_t>(kMaxOwn * NT)) {
+    // too many keys share the boundary bin: exact radix passes instead
+    __syncthreads();
+    select_threshold<NT>(bits, d, K, s, cand_key, cand_cap, T_out, krem_out);
+    return;
+  }
+
+  // ---- the boundary bin's keys, with their indices
+  for (int i0 = 0; i0 < d; i0 += NT) {
+    const int i = i0 + tid;
+    const uint32_t k = i < d ? (bits[i] & kKeyMask) : 0u;
+    const bool hit = i < d && (k >> 20) == b1;
+    const uint32_t lanes = __ballot_sync(0xffffffffu, hit);
+    uint32_t base = 0;
+    if (lane == 0 && lanes) base = atomicAdd(&s->pick[2], __popc(lanes));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (hit) {
+      const uint32_t slot = base + __popc(lanes & ((1u << lane) - 1u));
+      cand_key[slot] = k;
+      cand_idx[slot] = static_cast<uint32_t>(i);
+    }
+  }
+  __syncthreads();
+
+  // ---- rank every candidate (larger key first, then lower index); the one
+  // ranked krem1-1 holds the K-th largest key overall
+  const int nc = static_cast<int>(n1);
+  uint32_t my_key[kMaxOwn], my_rank[kMaxOwn];
+#pragma unroll
+  for (int q = 0; q < kMaxOwn; ++q) {
+    const int c = tid + q * NT;
+    my_key[q] = 0;
+    my_rank[q] = 0xffffffffu;
+    if (c < nc) {
+      const uint32_t kc = cand_key[c], ic = cand_idx[c];
+      uint32_t rank = 0;
+      for (int j = 0; j < nc; ++j) {
+        const uint32_t kj = cand_key[j];
+        rank += (kj > kc) | ((kj == kc) & (cand_idx[j] < ic));
+      }
+      my_key[q] = kc;
+      my_rank[q] = rank;
+      if (rank == krem1 - 1) s->pick[5] = kc;  // ranks are unique
+    }
+  }
+  __syncthreads();
+  const uint32_t T = s->pick[5];
+  // keys equal to T that are kept = those ranked below krem1
+  uint32_t eq_kept = 0;
+#pragma unroll
+  for (int q = 0; q < kMaxOwn; ++q) eq_kept += (my_rank[q] < krem1) & (my_key[q] == T);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) eq_kept += __shfl_xor_sync(0xffffffffu, eq_kept, o);
+  if (lane == 0 && eq_kept) atomicAdd(&s->pick[4], eq_kept);
+  __syncthreads();
+  *T_out = T;
+  *krem_out = s->pick[4];
+  (void)warp;
+  (void)NW;
+}
+
+// kept_chunk_base with a single-barrier scan; also returns the CTA total of
+// kept entries would-be positions are relative to 0.  All threads call it.
+template <int NT>
+__device__ __forceinline__ void kept_chunk_base_1s(const uint32_t* bits, int i0, int i1,
+                                                   uint32_t T, SelectScratch* s,
+                                                   uint32_t* gt_before, uint32_t* eq_before) {
+  uint32_t gt = 0, eq = 0;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t k = bits[i] & kKeyMask;
+    gt += k > T;
+    eq += k == T;
+  }
+  const uint32_t packed = (eq << 16) | gt;  // d < 65536: no carry between halves
+  const uint32_t excl = block_scan_excl_1s<NT>(packed, s->warp_sums, nullptr);
   *gt_before = excl & 0xffffu;
   *eq_before = excl >> 16;
 }

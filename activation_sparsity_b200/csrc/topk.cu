@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
                 float* __restrict__ val, int* dev_status) {
   extern __shared__ __align__(16) uint32_t bits[];  // raw fp32 bits of the row
   __shared__ SelectScratch sel;
-  __shared__ uint32_t cand[kTopkCand];
+  __shared__ uint32_t cand[2 * kTopkCand];  // keys, then indices
 
   const int tid = threadIdx.x;
   const int m = blockIdx.x;
@@ -34,6 +34,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   int32_t* out_i = idx + (size_t)m * K;
   float* out_v = val + (size_t)m * K;
 
+  for (int b = tid; b < 2 * kSelBins; b += kTopkThreads) sel.hist[b] = 0u;
   pdl_wait();
   pdl_launch_dependents();
 
@@ -66,14 +67,15 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   }
 
   uint32_t T = 0, krem = 0;
-  select_threshold<kTopkThreads>(bits, d, K, &sel, cand, kTopkCand, &T, &krem);
+  select_threshold_fast<kTopkThreads>(bits, d, K, &sel, cand, cand + kTopkCand, kTopkCand, &T,
+                                      &krem);
 
   // ---- stable compaction over contiguous chunks
   const int chunk = (d + kTopkThreads - 1) / kTopkThreads;
   const int i0 = min(d, tid * chunk);
   const int i1 = min(d, i0 + chunk);
   uint32_t gt_before = 0, eq_before = 0;
-  kept_chunk_base<kTopkThreads>(bits, i0, i1, T, &sel, &gt_before, &eq_before);
+  kept_chunk_base_1s<kTopkThreads>(bits, i0, i1, T, &sel, &gt_before, &eq_before);
   for (int i = i0; i < i1; ++i) {
     const uint32_t u = bits[i];
     const uint32_t k = u & kKeyMask;

@@ -204,9 +204,11 @@ int larosa_dense_linear(const void *x, const void *Wt, int M, int d_in,
  * allowed.  The LaRoSA pages have no counterpart: this is a deployment
  * variant of step 3, computing the same y with the same kernels.
  *
- * Arguments as for larosa_sparse_linear, minus ws/ws_bytes.  The split-K
- * scratch lives in a 2 MiB file-scope device array that every GPU loading
- * the library holds until the process exits.  Sizes whose scratch would
+ * Arguments as for larosa_sparse_linear, minus ws/ws_bytes.  One token
+ * needs no scratch (its partial sums stay in distributed shared memory);
+ * several tokens keep their split-K partials and row bookkeeping in a 2 MiB
+ * file-scope device array that every GPU loading the library holds until
+ * the process exits.  Sizes whose scratch would
  * exceed it (in practice only large multi-token batches, e.g. M = 16 with
  * d_in = 32768) return LAROSA_ERR_WORKSPACE with the byte counts in
  * larosa_last_error_string().  The call allocates nothing; it clears the
