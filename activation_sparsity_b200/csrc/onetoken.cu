@@ -100,7 +100,6 @@ __global__ void __launch_bounds__(kT, (MT <= 2 && sizeof(T) == 2 ? 2 : 1)) rowdo
   const T* xs = reinterpret_cast<const T*>(xs_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_wait();
-  pdl_launch_dependents();
   const T* xg = static_cast<const T*>(p.x);
   if (p.x_in_smem) {
     const int nv = p.M * p.n_in * (int)sizeof(T) / 16;
@@ -159,12 +158,17 @@ __global__ void __launch_bounds__(kT, (MT <= 2 && sizeof(T) == 2 ? 2 : 1)) rowdo
       if (lane == 0 && m < p.M) p.y[(size_t)m * p.n_out + row] = s;
     }
   }
+  // No early trigger: the next kernel is often a cluster launch that needs
+  // whole GPCs, and placing its clusters around this grid's retiring CTAs
+  // left some of them for a second wave.  It launches when this grid ends.
 }
 
 // ================================================================ gather
 
 constexpr int kModeGather = 1;
 constexpr int kModeSelect = 2;
+constexpr int kC = 8;  // CTAs per cluster (one column tile)
+constexpr int kGatherSmemCeiling = 227 * 1024;
 constexpr int kCandCap = 1024;
 
 struct GParams {
@@ -211,13 +215,13 @@ __host__ __device__ inline GLayout glayout(int mode, int key_cap, int list_cap, 
 
 // One radix pass of a selection spread over a cluster: histogram this CTA's
 // keys that match `prefix` under `mask` on digit (key >> shift) & (nb-1),
-// add the cluster's histograms (rank r adds bins [r*nb/C, (r+1)*nb/C) and
+// add the cluster's histograms (rank r adds bins [r*nb/kC, (r+1)*nb/kC) and
 // writes the sums into every CTA's `merged`), then find the bin holding the
 // krem-th largest counted key.  Writes bin, keys above it, keys in it to
 // pick[0], pick[1], pick[3].  `hist` (both copies) must be zero on entry and
 // is zero again on return.
 template <int NT>
-__device__ __forceinline__ void cluster_radix_pass(cg::cluster_group& cl, int C, int rank,
+__device__ __forceinline__ void cluster_radix_pass(cg::cluster_group& cl, int rank,
                                                    const uint32_t* keys, int n_mine,
                                                    uint32_t prefix, uint32_t mask, int shift,
                                                    int nb, uint32_t krem, SelectScratch* s,
@@ -234,11 +238,16 @@ __device__ __forceinline__ void cluster_radix_pass(cg::cluster_group& cl, int C,
     s->hist[kSelBins + b] = 0u;
   }
   cl.sync();  // every CTA's histogram is final
-  const int b0 = (int)((long long)nb * rank / C), b1 = (int)((long long)nb * (rank + 1) / C);
+  const int b0 = nb * rank / kC, b1 = nb * (rank + 1) / kC;
   for (int b = b0 + tid; b < b1; b += NT) {
+    uint32_t v[kC];
+#pragma unroll
+    for (int q = 0; q < kC; ++q) v[q] = cl.map_shared_rank(s->hist, q)[b];  // all in flight
     uint32_t sum = 0;
-    for (int q = 0; q < C; ++q) sum += cl.map_shared_rank(s->hist, q)[b];
-    for (int q = 0; q < C; ++q) cl.map_shared_rank(merged, q)[b] = sum;
+#pragma unroll
+    for (int q = 0; q < kC; ++q) sum += v[q];
+#pragma unroll
+    for (int q = 0; q < kC; ++q) cl.map_shared_rank(merged, q)[b] = sum;
   }
   cl.sync();  // merged everywhere; no CTA still reads another's `hist`
   for (int b = tid; b < nb; b += NT) s->hist[b] = 0u;
@@ -275,7 +284,7 @@ __global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
   constexpr int CPT = 16 / sizeof(Tw);  // columns per thread per row
   extern __shared__ __align__(16) unsigned char smem_raw[];
   cg::cluster_group cl = cg::this_cluster();
-  const int C = static_cast<int>(cl.num_blocks());
+  constexpr int C = kC;
   const int rank = static_cast<int>(cl.block_rank());
   const int key_cap = (p.d_in + C - 1) / C;
   const GLayout L = glayout(MODE, key_cap, p.list_cap, p.col_tile, CPT);
@@ -342,8 +351,7 @@ __global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
       for (int pass = 0; pass < 3; ++pass) {
         const int shift = pass == 0 ? 20 : (pass == 1 ? 9 : 0);
         const int nb = pass == 2 ? 512 : 2048;
-        cluster_radix_pass<kT>(cl, C, rank, keys, n_mine, prefix, mask, shift, nb, krem, sel,
-                               merged);
+        cluster_radix_pass<kT>(cl, rank, keys, n_mine, prefix, mask, shift, nb, krem, sel, merged);
         prefix |= sel->pick[0] << shift;
         mask |= static_cast<uint32_t>(nb - 1) << shift;
         krem -= sel->pick[1];
@@ -368,11 +376,9 @@ __global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
     const uint32_t packed = block_scan_excl_1s<kT>((eq << 16) | gt, sel->warp_sums, &tot);
     uint32_t gt_before = packed & 0xffffu, eq_before = packed >> 16;
     const bool want_positions = tile == 0 && p.idx_out != nullptr;
-    if (tid == 0) {
-      for (int q = 0; q < C; ++q) {
-        cl.map_shared_rank(xchg, q)[rank] = tot & 0xffffu;
-        cl.map_shared_rank(xchg, q)[32 + rank] = tot >> 16;
-      }
+    if (tid < C) {  // one remote store pair per destination rank
+      cl.map_shared_rank(xchg, tid)[rank] = tot & 0xffffu;
+      cl.map_shared_rank(xchg, tid)[32 + rank] = tot >> 16;
     }
     cl.sync();  // every CTA's counts are in every CTA
     uint32_t ties_before = 0, kept_before = 0;
@@ -475,8 +481,12 @@ __global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
   const int sl = (wc + C - 1) / C;
   const int e0 = rank * sl, e1 = min(wc, e0 + sl);
   for (int e = e0 + tid; e < e1; e += kT) {
+    float v[C];
+#pragma unroll
+    for (int q = 0; q < C; ++q) v[q] = cl.map_shared_rank(part, q)[e];  // all in flight
     float sum = 0.f;
-    for (int q = 0; q < C; ++q) sum += cl.map_shared_rank(part, q)[e];
+#pragma unroll
+    for (int q = 0; q < C; ++q) sum += v[q];
     p.y[c0 + e] = sum;
   }
   cl.sync();  // no CTA leaves while another may still read its partial
@@ -594,7 +604,10 @@ cudaError_t max_clusters(int dev, void* fn, size_t smem, int C, int* out) {
       }
     }
   }
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // the attribute is a ceiling for every launch of fn: set it to the largest
+  // size a launch may use, not to the size probed here
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kGatherSmemCeiling);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, 64, 1);
@@ -639,7 +652,7 @@ cudaError_t plan_gather(int mode, Elem w_elem, int d_in, int d_out, int K, Strea
   void* fn = gather_fn(w_elem, mode);
   StreamPlan best;
   long long best_ctas = -1;
-  for (int C = 8; C >= 2; C /= 2) {
+  for (int C = kC; C == kC; C = 0) {
     const int key_cap = (d_in + C - 1) / C;
     // list mode: the rank's share of the kept list; select mode: the kept
     // entries of the rank's index range
@@ -648,7 +661,7 @@ cudaError_t plan_gather(int mode, Elem w_elem, int d_in, int d_out, int K, Strea
     // (128 bytes of bf16) and at most one 16-byte vector per thread
     const int wc_max = kT * cpt;
     const size_t smem_probe = glayout(kmode, key_cap, list_cap, wc_max, cpt).total;
-    if (smem_probe > 227 * 1024) continue;
+    if (smem_probe > (size_t)kGatherSmemCeiling) continue;
     int clusters = 0;
     e = max_clusters(dev, fn, smem_probe, C, &clusters);
     if (e != cudaSuccess) return e;
