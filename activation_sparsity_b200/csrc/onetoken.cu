@@ -27,9 +27,10 @@
 //         nothing leaves the cluster but y.  The tile width is chosen so the
 //         clusters that fit on the GPU at once cover d_out.
 //           kGather  row(p) = idx[p], coef(p) = val[p]
-//           kSelect  every CTA first selects the K largest |x_rot| itself
-//                    (exact, ties to the lower index; no grid-wide handoff),
-//                    then gathers its part of them.
+//           kSelect  each cluster first selects the K largest |x_rot| itself
+//                    (exact, ties to the lower index; no grid-wide handoff)
+//                    and starts streaming the rows it is sure of before the
+//                    last places are decided.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -169,7 +170,8 @@ constexpr int kModeGather = 1;
 constexpr int kModeSelect = 2;
 constexpr int kC = 8;  // CTAs per cluster (one column tile)
 constexpr int kGatherSmemCeiling = 227 * 1024;
-constexpr int kCandCap = 1024;
+// Boundary-bin candidates ranked directly; a fuller bin takes radix passes.
+constexpr int kRankCap = kT;
 
 struct GParams {
   const void* W;         // [d_in x d_out] row-major
@@ -189,7 +191,7 @@ struct GParams {
 
 // Shared memory of one CTA, laid out from sizes known at launch.
 struct GLayout {
-  size_t sel, merged, xchg, keys, rows, vals, part, red, total;
+  size_t sel, merged, xchg, keys, kflag, cand, call, cflag, rows, vals, part, red, total;
 };
 
 __host__ __device__ inline size_t al16(size_t v) { return (v + 15) & ~size_t(15); }
@@ -203,8 +205,12 @@ __host__ __device__ inline GLayout glayout(int mode, int key_cap, int list_cap, 
   const bool sel = mode == kModeSelect;
   L.sel = o;      o = al16(o + (sel ? sizeof(SelectScratch) : 64));
   L.merged = o;   o = al16(o + (sel ? kSelBins * 4 : 0));
-  L.xchg = o;     o = al16(o + (sel ? 64 * 4 : 0));
+  L.xchg = o;     o = al16(o + (sel ? 4 * 32 * 4 : 0));
   L.keys = o;     o = al16(o + (sel ? (size_t)key_cap * 4 : 0));
+  L.kflag = o;    o = al16(o + (sel ? (size_t)key_cap : 0));
+  L.cand = o;     o = al16(o + (sel ? (size_t)kRankCap * 8 : 0));
+  L.call = o;     o = al16(o + (sel ? (size_t)kRankCap * 8 : 0));
+  L.cflag = o;    o = al16(o + (sel ? (size_t)kRankCap : 0));
   L.rows = o;     o = al16(o + (size_t)list_cap * 4);
   L.vals = o;     o = al16(o + (size_t)list_cap * 4);
   L.part = o;     o = al16(o + (size_t)col_tile * 4);
@@ -213,13 +219,55 @@ __host__ __device__ inline GLayout glayout(int mode, int key_cap, int list_cap, 
   return L;
 }
 
+// Split cluster barrier: arrive publishes this thread's earlier writes
+// (shared and distributed shared memory) to every CTA of the cluster; wait
+// returns once all threads of the cluster have arrived.
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// The bin holding the krem-th largest counted key, scanning counts[nb] from
+// the top: writes bin, keys above it, keys in it to pick[0], pick[1],
+// pick[3].  Ends with a barrier.
+template <int NT>
+__device__ __forceinline__ void boundary_from_top(const uint32_t* counts, int nb, uint32_t krem,
+                                                  SelectScratch* s) {
+  const int tid = threadIdx.x;
+  // thread t owns ranks [t*per, t*per+per) counted from the top
+  constexpr int kPer = (kSelBins + NT - 1) / NT;
+  const int per = (nb + NT - 1) / NT;
+  uint32_t cnt[kPer];
+  uint32_t own = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int k = tid * per + j;
+    cnt[j] = (j < per && k < nb) ? counts[nb - 1 - k] : 0u;
+    own += cnt[j];
+  }
+  uint32_t before = block_scan_excl_1s<NT>(own, s->warp_sums, nullptr);
+  if (before < krem && krem <= before + own) {
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (j < per && before < krem && krem <= before + cnt[j]) {
+        s->pick[0] = static_cast<uint32_t>(nb - 1 - (tid * per + j));
+        s->pick[1] = before;
+        s->pick[3] = cnt[j];
+      }
+      before += cnt[j];
+    }
+  }
+  __syncthreads();
+}
+
 // One radix pass of a selection spread over a cluster: histogram this CTA's
 // keys that match `prefix` under `mask` on digit (key >> shift) & (nb-1),
 // add the cluster's histograms (rank r adds bins [r*nb/kC, (r+1)*nb/kC) and
-// writes the sums into every CTA's `merged`), then find the bin holding the
-// krem-th largest counted key.  Writes bin, keys above it, keys in it to
-// pick[0], pick[1], pick[3].  `hist` (both copies) must be zero on entry and
-// is zero again on return.
+// writes the sums into every CTA's `merged`), then find the boundary bin as
+// boundary_from_top does.  `hist` (both copies) must be zero on entry and is
+// zero again on return.
 template <int NT>
 __device__ __forceinline__ void cluster_radix_pass(cg::cluster_group& cl, int rank,
                                                    const uint32_t* keys, int n_mine,
@@ -251,34 +299,26 @@ __device__ __forceinline__ void cluster_radix_pass(cg::cluster_group& cl, int ra
   }
   cl.sync();  // merged everywhere; no CTA still reads another's `hist`
   for (int b = tid; b < nb; b += NT) s->hist[b] = 0u;
-  // boundary bin, counting from the top: thread t owns ranks [t*per, t*per+per)
-  constexpr int kPer = (kSelBins + NT - 1) / NT;
-  const int per = (nb + NT - 1) / NT;
-  uint32_t cnt[kPer];
-  uint32_t own = 0;
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int k = tid * per + j;
-    cnt[j] = (j < per && k < nb) ? merged[nb - 1 - k] : 0u;
-    own += cnt[j];
-  }
-  uint32_t before = block_scan_excl_1s<NT>(own, s->warp_sums, nullptr);
-  if (before < krem && krem <= before + own) {
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      if (j < per && before < krem && krem <= before + cnt[j]) {
-        s->pick[0] = static_cast<uint32_t>(nb - 1 - (tid * per + j));
-        s->pick[1] = before;
-        s->pick[3] = cnt[j];
-      }
-      before += cnt[j];
-    }
-  }
-  __syncthreads();
+  boundary_from_top<NT>(merged, nb, krem, s);
+}
+
+// Rank of a boundary-bin key: larger |x| first, then the lower index.
+__device__ __forceinline__ unsigned long long cand_order(uint32_t key, int idx) {
+  return (static_cast<unsigned long long>(key & kKeyMask) << 32) |
+         static_cast<uint32_t>(~static_cast<uint32_t>(idx));
 }
 
 // One cluster per column tile; the cluster's CTAs split the kept list in
 // rank order, and their partial sums meet in distributed shared memory.
+//
+// Select mode.  Rank r owns the rotated entries [d*r/C, d*(r+1)/C).  Every
+// CTA histograms all d keys on bits 30..20 (sign cleared) and finds the bin
+// B holding the K-th largest: keys above B are kept for certain, keys in B
+// are candidates for the remaining krem places.  Each CTA then streams its
+// certain rows while the cluster trades candidate lists (split barrier),
+// ranks the candidates exactly, and streams its kept candidates last.  The
+// order of the sum over rows is a function of the data only, so results
+// repeat bit for bit.
 template <typename Tw, int MODE>
 __global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
   constexpr int CPT = 16 / sizeof(Tw);  // columns per thread per row
@@ -295,139 +335,14 @@ __global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
   float* red = reinterpret_cast<float*>(smem_raw + L.red);
 
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.y;
   const int c0 = tile * p.col_tile;
   const int wc = min(p.col_tile, p.d_out - c0);
   const int K = p.K;
-  int len = 0;  // rows this CTA streams
 
-  if constexpr (MODE == kModeSelect) {
-    for (int b = tid; b < 2 * kSelBins; b += kT) sel->hist[b] = 0u;
-  }
-  pdl_wait();
-  pdl_launch_dependents();
-
-  if constexpr (MODE == kModeGather) {
-    // rank r takes the kept positions [K*r/C, K*(r+1)/C)
-    const int p0 = (int)((long long)K * rank / C);
-    const int p1 = (int)((long long)K * (rank + 1) / C);
-    len = p1 - p0;
-    bool bad = false;
-    for (int j = tid; j < len; j += kT) {
-      const int row = p.rows[p0 + j];
-      const bool ok = static_cast<unsigned>(row) < static_cast<unsigned>(p.d_in);
-      bad |= !ok;
-      lrows[j] = ok ? row : 0;
-      lvals[j] = ok ? static_cast<const float*>(p.coef)[p0 + j] : 0.f;
-    }
-    if (__syncthreads_or(bad) && tid == 0) report(p.dev_status, LAROSA_DEV_INDEX);
-  } else {
-    // rank r owns the rotated entries [d*r/C, d*(r+1)/C) and gathers the kept
-    // ones among them; the threshold is found by radix passes whose
-    // histograms are added across the cluster
-    const int d = p.d_in;
-    const int i_lo = (int)((long long)d * rank / C);
-    const int n_mine = (int)((long long)d * (rank + 1) / C) - i_lo;
-    uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + L.keys);
-    uint32_t* merged = reinterpret_cast<uint32_t*>(smem_raw + L.merged);
-    uint32_t* xchg = reinterpret_cast<uint32_t*>(smem_raw + L.xchg);  // [0,32) > T, [32,64) == T
-    {
-      const float* src = static_cast<const float*>(p.coef) + i_lo;
-      bool nonfinite = false;
-      for (int i = tid; i < n_mine; i += kT) {
-        const uint32_t u = __float_as_uint(__ldcg(src + i));
-        keys[i] = u;
-        nonfinite |= (u & kKeyMask) >= 0x7f800000u;
-      }
-      if (__syncthreads_or(nonfinite) && tid == 0 && tile == 0)
-        report(p.dev_status, LAROSA_DEV_NONFINITE);
-    }
-    uint32_t T = 0, krem = 0;
-    const bool all = K >= d;
-    if (K > 0 && !all) {
-      uint32_t prefix = 0, mask = 0;
-      krem = static_cast<uint32_t>(K);
-#pragma unroll 1
-      for (int pass = 0; pass < 3; ++pass) {
-        const int shift = pass == 0 ? 20 : (pass == 1 ? 9 : 0);
-        const int nb = pass == 2 ? 512 : 2048;
-        cluster_radix_pass<kT>(cl, rank, keys, n_mine, prefix, mask, shift, nb, krem, sel, merged);
-        prefix |= sel->pick[0] << shift;
-        mask |= static_cast<uint32_t>(nb - 1) << shift;
-        krem -= sel->pick[1];
-        __syncthreads();
-      }
-      T = prefix;  // krem keys equal to T are kept: the lowest-indexed ones
-    }
-    // this CTA's counts above / at the threshold, exchanged across the cluster
-    const int chunk = (n_mine + kT - 1) / kT;
-    const int j0 = min(n_mine, tid * chunk), j1 = min(n_mine, j0 + chunk);
-    uint32_t gt = 0, eq = 0;
-    if (all) {
-      gt = (uint32_t)(j1 - j0);  // everything is kept
-    } else if (K > 0) {
-      for (int j = j0; j < j1; ++j) {
-        const uint32_t k = keys[j] & kKeyMask;
-        gt += k > T;
-        eq += k == T;
-      }
-    }
-    uint32_t tot = 0;
-    const uint32_t packed = block_scan_excl_1s<kT>((eq << 16) | gt, sel->warp_sums, &tot);
-    uint32_t gt_before = packed & 0xffffu, eq_before = packed >> 16;
-    const bool want_positions = tile == 0 && p.idx_out != nullptr;
-    if (tid < C) {  // one remote store pair per destination rank
-      cl.map_shared_rank(xchg, tid)[rank] = tot & 0xffffu;
-      cl.map_shared_rank(xchg, tid)[32 + rank] = tot >> 16;
-    }
-    cl.sync();  // every CTA's counts are in every CTA
-    uint32_t ties_before = 0, kept_before = 0;
-    for (int q = 0; q < rank; ++q) {
-      const uint32_t tq = xchg[32 + q];
-      kept_before += xchg[q] + min(tq, krem > ties_before ? krem - ties_before : 0u);
-      ties_before += tq;
-    }
-    // kept entries of this CTA before j0; the chunk's kept entries follow in
-    // index order
-    uint32_t pos_local = gt_before + min(eq_before, krem > ties_before ? krem - ties_before : 0u);
-    uint32_t eqc = eq_before;
-    for (int j = j0; j < j1; ++j) {
-      const uint32_t u = keys[j];
-      const uint32_t k = u & kKeyMask;
-      bool kept;
-      if (K == 0) {
-        kept = false;
-      } else if (all || k > T) {
-        kept = true;
-      } else if (k == T) {
-        kept = eqc + ties_before < krem;
-        ++eqc;
-      } else {
-        kept = false;
-      }
-      if (kept) {
-        const float v = __uint_as_float(u);
-        lrows[pos_local] = i_lo + j;
-        lvals[pos_local] = v;
-        if (want_positions) {
-          p.idx_out[kept_before + pos_local] = i_lo + j;
-          p.val_out[kept_before + pos_local] = v;
-        }
-        ++pos_local;
-      }
-    }
-    // rows this CTA streams
-    {
-      const uint32_t gt_all = tot & 0xffffu, eq_all = tot >> 16;
-      len = (int)(K == 0 ? 0u
-                  : all ? (uint32_t)n_mine
-                        : gt_all + min(eq_all, krem > ties_before ? krem - ties_before : 0u));
-    }
-    __syncthreads();
-  }
-
-  // ---- stream the kept rows of this tile: thread (g, col) reads 16 bytes
-  // of rows g, g+ng, ..., with kU loads in flight
+  // ---- streaming: thread (g, col) reads 16 bytes of list rows lo+g,
+  // lo+g+ng, ... < hi, with kU loads in flight, into acc
   const int tpr = p.tpr;
   const int ng = kT / tpr;
   const int g = tid / tpr;
@@ -436,20 +351,21 @@ __global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
   float acc[CPT];
 #pragma unroll
   for (int v = 0; v < CPT; ++v) acc[v] = 0.f;
-  if (active) {
-    const unsigned char* wbase = static_cast<const unsigned char*>(p.W) + ((size_t)c0 + col) * sizeof(Tw);
-    const size_t pitch = (size_t)p.d_out * sizeof(Tw);
-    for (int r0 = g; r0 < len; r0 += ng * kU) {
+  const unsigned char* wbase = static_cast<const unsigned char*>(p.W) + ((size_t)c0 + col) * sizeof(Tw);
+  const size_t pitch = (size_t)p.d_out * sizeof(Tw);
+  auto stream_rows = [&](int lo, int hi) {
+    if (!active) return;
+    for (int r0 = lo + g; r0 < hi; r0 += ng * kU) {
       uint4 u[kU];
 #pragma unroll
       for (int k = 0; k < kU; ++k) {
         const int r = r0 + k * ng;
-        u[k] = r < len ? ld_stream(wbase + (size_t)lrows[r] * pitch) : make_uint4(0, 0, 0, 0);
+        u[k] = r < hi ? ld_stream(wbase + (size_t)lrows[r] * pitch) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int k = 0; k < kU; ++k) {
         const int r = r0 + k * ng;
-        const float cf = r < len ? lvals[r] : 0.f;
+        const float cf = r < hi ? lvals[r] : 0.f;
         if constexpr (CPT == 8) {
           float w[8];
           Vec8<__nv_bfloat16>::cvt(&u[k], w);
@@ -463,6 +379,234 @@ __global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
         }
       }
     }
+  };
+
+  if constexpr (MODE == kModeSelect) {
+    for (int b = tid; b < 2 * kSelBins; b += kT) sel->hist[b] = 0u;
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+
+  if constexpr (MODE == kModeGather) {
+    // rank r takes the kept positions [K*r/C, K*(r+1)/C)
+    const int p0 = (int)((long long)K * rank / C);
+    const int p1 = (int)((long long)K * (rank + 1) / C);
+    const int len = p1 - p0;
+    bool bad = false;
+    for (int j = tid; j < len; j += kT) {
+      const int row = p.rows[p0 + j];
+      const bool ok = static_cast<unsigned>(row) < static_cast<unsigned>(p.d_in);
+      bad |= !ok;
+      lrows[j] = ok ? row : 0;
+      lvals[j] = ok ? static_cast<const float*>(p.coef)[p0 + j] : 0.f;
+    }
+    if (__syncthreads_or(bad) && tid == 0) report(p.dev_status, LAROSA_DEV_INDEX);
+    stream_rows(0, len);
+  }
+
+  // select mode state kept for the index/value output at the end
+  const int d = p.d_in;
+  const int i_lo = (int)((long long)d * rank / C);
+  const int n_mine = (int)((long long)d * (rank + 1) / C) - i_lo;
+  const bool all = K >= d;
+  uint32_t B = 0;            // boundary bin (bits 30..20)
+  uint32_t kept_low = 0;     // kept entries owned by lower ranks
+  if constexpr (MODE == kModeSelect) {
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + L.keys);
+    uint8_t* kflag = reinterpret_cast<uint8_t*>(smem_raw + L.kflag);  // kept candidate
+    uint32_t* merged = reinterpret_cast<uint32_t*>(smem_raw + L.merged);
+    // xchg[q]: certain rows of rank q; [32+q]: its candidates; [64+q] and
+    // [96+q]: above / at the threshold (radix fallback)
+    uint32_t* xchg = reinterpret_cast<uint32_t*>(smem_raw + L.xchg);
+    unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem_raw + L.cand);
+    unsigned long long* call = reinterpret_cast<unsigned long long*>(smem_raw + L.call);
+    uint8_t* cflag = reinterpret_cast<uint8_t*>(smem_raw + L.cflag);
+
+    // ---- all d keys -> histogram on bits 30..20; own keys -> `keys`
+    {
+      uint32_t* h = sel->hist + (lane & 1) * kSelBins;
+      const uint4* src = static_cast<const uint4*>(p.coef);  // d is a multiple of 8
+      bool nonfinite = false;
+      for (int v = tid; v < d / 4; v += kT) {
+        const uint4 u4 = __ldcg(src + v);
+        const uint32_t u[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t k = u[e] & kKeyMask;
+          nonfinite |= k >= 0x7f800000u;
+          atomicAdd(&h[k >> 20], 1u);
+          const int j = 4 * v + e - i_lo;
+          if (j >= 0 && j < n_mine) {
+            keys[j] = u[e];
+            kflag[j] = 0;
+          }
+        }
+      }
+      if (__syncthreads_or(nonfinite) && tid == 0 && tile == 0 && rank == 0)
+        report(p.dev_status, LAROSA_DEV_NONFINITE);
+      for (int b = tid; b < kSelBins; b += kT) {
+        merged[b] = sel->hist[b] + sel->hist[kSelBins + b];
+        sel->hist[b] = 0u;
+        sel->hist[kSelBins + b] = 0u;
+      }
+      __syncthreads();
+    }
+    uint32_t krem = 0;  // candidates to keep
+    uint32_t nB = 0;    // keys in the boundary bin, cluster-wide
+    if (K > 0 && !all) {
+      boundary_from_top<kT>(merged, kSelBins, static_cast<uint32_t>(K), sel);
+      B = sel->pick[0];
+      krem = static_cast<uint32_t>(K) - sel->pick[1];
+      nB = sel->pick[3];
+    }
+    const bool ranked = nB <= static_cast<uint32_t>(kRankCap);  // same in every CTA
+
+    // ---- certain rows -> the list; candidates -> `cand` (ranked case)
+    const int chunk = (n_mine + kT - 1) / kT;
+    const int j0 = min(n_mine, tid * chunk), j1 = min(n_mine, j0 + chunk);
+    auto certain = [&](uint32_t k) { return K > 0 && (all || (k >> 20) > B); };
+    auto in_bin = [&](uint32_t k) { return K > 0 && !all && (k >> 20) == B; };
+    uint32_t n_def = 0, n_cand = 0;
+    {
+      uint32_t dc = 0, cc = 0;
+      for (int j = j0; j < j1; ++j) {
+        const uint32_t k = keys[j] & kKeyMask;
+        dc += certain(k);
+        cc += in_bin(k);
+      }
+      uint32_t tot = 0;
+      const uint32_t packed = block_scan_excl_1s<kT>((cc << 16) | dc, sel->warp_sums, &tot);
+      uint32_t dp = packed & 0xffffu, cp = packed >> 16;
+      n_def = tot & 0xffffu;
+      n_cand = tot >> 16;
+      for (int j = j0; j < j1; ++j) {
+        const uint32_t u = keys[j];
+        const uint32_t k = u & kKeyMask;
+        if (certain(k)) {
+          lrows[dp] = i_lo + j;
+          lvals[dp] = __uint_as_float(u);
+          ++dp;
+        } else if (ranked && in_bin(k)) {
+          cand[cp++] = cand_order(k, i_lo + j);
+        }
+      }
+      if (tid < C) {  // one remote store pair per destination rank
+        cl.map_shared_rank(xchg, tid)[rank] = n_def;
+        cl.map_shared_rank(xchg, tid)[32 + rank] = n_cand;
+      }
+      __syncthreads();  // the list is complete before it is streamed
+    }
+    cluster_arrive_release();
+    stream_rows(0, (int)n_def);
+    cluster_wait_acquire();  // every rank's counts and candidates are visible
+
+    const bool want_positions = tile == 0 && p.idx_out != nullptr;
+    int len = (int)n_def;
+    for (int q = 0; q < rank; ++q) kept_low += xchg[q];
+    if (ranked) {
+      // ---- the cluster's candidates in index order (rank, then position)
+      uint32_t run = 0, src_base = 0, lo_r = 0, hi_r = 0;
+      int src = 0;
+#pragma unroll
+      for (int q = 0; q < C; ++q) {
+        const uint32_t cq = xchg[32 + q];
+        if (static_cast<uint32_t>(tid) >= run) {  // the last rank starting at or below tid
+          src = q;
+          src_base = run;
+        }
+        if (q == rank) {
+          lo_r = run;
+          hi_r = run + cq;
+        }
+        run += cq;
+      }
+      const int n_all = (int)run;
+      if (tid < n_all) call[tid] = cl.map_shared_rank(cand, src)[tid - src_base];
+      __syncthreads();
+      // a warp per candidate: kept iff fewer than krem candidates outrank it
+      const int c_lo = want_positions ? 0 : (int)lo_r;
+      const int c_hi = (int)hi_r;
+      for (int c = c_lo + warp; c < c_hi; c += kWarps) {
+        const unsigned long long me = call[c];
+        uint32_t above = 0;
+        for (int i = lane; i < n_all; i += 32) above += call[i] > me;
+        above = __reduce_add_sync(0xffffffffu, above);
+        if (lane == 0) cflag[c] = above < krem;
+      }
+      __syncthreads();
+      const bool f = tid >= c_lo && tid < c_hi && cflag[tid];
+      const bool own = f && tid >= (int)lo_r;
+      uint32_t tot = 0;
+      const uint32_t packed = block_scan_excl_1s<kT>(((uint32_t)(f && !own) << 16) | own,
+                                                     sel->warp_sums, &tot);
+      if (own) {
+        const int idx = (int)~static_cast<uint32_t>(call[tid]);
+        const int pos = (int)n_def + (int)(packed & 0xffffu);
+        lrows[pos] = idx;
+        lvals[pos] = __uint_as_float(keys[idx - i_lo]);
+        kflag[idx - i_lo] = 1;
+      }
+      len += (int)(tot & 0xffffu);
+      kept_low += tot >> 16;
+    } else {
+      // ---- too many keys share bin B: two more radix passes inside it,
+      // with histograms added across the cluster, give the exact threshold
+      // T; ties at T go to the lowest indices across the cluster
+      uint32_t prefix = B << 20, mask = 0x7ffu << 20;
+#pragma unroll 1
+      for (int pass = 1; pass < 3; ++pass) {
+        const int shift = pass == 1 ? 9 : 0;
+        const int nb = pass == 1 ? 2048 : 512;
+        cluster_radix_pass<kT>(cl, rank, keys, n_mine, prefix, mask, shift, nb, krem, sel, merged);
+        prefix |= sel->pick[0] << shift;
+        mask |= static_cast<uint32_t>(nb - 1) << shift;
+        krem -= sel->pick[1];
+        __syncthreads();
+      }
+      const uint32_t T = prefix;  // krem keys equal to T are kept
+      uint32_t gt = 0, eq = 0;
+      for (int j = j0; j < j1; ++j) {
+        const uint32_t k = keys[j] & kKeyMask;
+        gt += (k >> 20) == B && k > T;
+        eq += k == T;
+      }
+      uint32_t tot = 0;
+      const uint32_t packed = block_scan_excl_1s<kT>((eq << 16) | gt, sel->warp_sums, &tot);
+      if (tid < C) {
+        cl.map_shared_rank(xchg, tid)[64 + rank] = tot & 0xffffu;
+        cl.map_shared_rank(xchg, tid)[96 + rank] = tot >> 16;
+      }
+      cl.sync();  // every CTA's counts are in every CTA
+      uint32_t ties_before = 0;
+      for (int q = 0; q < rank; ++q) {
+        const uint32_t tq = xchg[96 + q];
+        kept_low += xchg[64 + q] + min(tq, krem > ties_before ? krem - ties_before : 0u);
+        ties_before += tq;
+      }
+      const uint32_t ties_left = krem > ties_before ? krem - ties_before : 0u;
+      uint32_t eqc = packed >> 16;
+      uint32_t pos = n_def + (packed & 0xffffu) + min(eqc, ties_left);
+      for (int j = j0; j < j1; ++j) {
+        const uint32_t u = keys[j];
+        const uint32_t k = u & kKeyMask;
+        bool kept = false;
+        if ((k >> 20) == B && k > T) {
+          kept = true;
+        } else if (k == T) {
+          kept = eqc < ties_left;
+          ++eqc;
+        }
+        if (kept) {
+          lrows[pos] = i_lo + j;
+          lvals[pos] = __uint_as_float(u);
+          kflag[j] = 1;
+          ++pos;
+        }
+      }
+      len += (int)((tot & 0xffffu) + min(tot >> 16, ties_left));
+    }
+    __syncthreads();
+    stream_rows((int)n_def, len);
   }
 
   // ---- row groups -> this CTA's partial, in shared memory
@@ -490,6 +634,29 @@ __global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
     p.y[c0 + e] = sum;
   }
   cl.sync();  // no CTA leaves while another may still read its partial
+
+  // ---- the kept indices and values in ascending index order (one cluster)
+  if constexpr (MODE == kModeSelect) {
+    if (tile == 0 && p.idx_out != nullptr) {
+      const uint32_t* keys = reinterpret_cast<const uint32_t*>(smem_raw + L.keys);
+      const uint8_t* kflag = reinterpret_cast<const uint8_t*>(smem_raw + L.kflag);
+      const int chunk = (n_mine + kT - 1) / kT;
+      const int j0 = min(n_mine, tid * chunk), j1 = min(n_mine, j0 + chunk);
+      auto kept = [&](int j) {
+        return K > 0 && (all || ((keys[j] & kKeyMask) >> 20) > B || kflag[j] != 0);
+      };
+      uint32_t n = 0;
+      for (int j = j0; j < j1; ++j) n += kept(j);
+      uint32_t pos = kept_low + block_scan_excl_1s<kT>(n, sel->warp_sums, nullptr);
+      for (int j = j0; j < j1; ++j) {
+        if (kept(j)) {
+          p.idx_out[pos] = i_lo + j;
+          p.val_out[pos] = __uint_as_float(keys[j]);
+          ++pos;
+        }
+      }
+    }
+  }
 }
 
 struct DevState {

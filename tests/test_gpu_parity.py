@@ -329,3 +329,26 @@ def test_fused_is_deterministic(L):
     y1 = L.larosa_rotate_topk_linear(x, Qt, W_rot, K).clone()
     y2 = L.larosa_rotate_topk_linear(x, Qt, W_rot, K).clone()
     assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("kind", sd.ADVERSARIAL_KINDS)
+@pytest.mark.parametrize("d", [8, 200, 1024, 4096, 11008])
+def test_fused_selection_bit_exact_under_identity_rotation(L, kind, d):
+    """Q = I is orthogonal and makes the fused rotation exact (x_rot = x), so the
+    selection inside the fused kernel can be compared bit for bit with the
+    oracle's Top-K of x on rows full of ties, signed zeros and subnormals."""
+    d_out = 72
+    x = sd.adversarial_rows(kind, 1, d, 900 + d)
+    Qt = torch.eye(d, dtype=torch.float32, device="cuda")
+    W_rot = sd.weights(d, d_out, 1 / 16, 901, torch.float32).cuda()
+    xd = f64(x)
+    for K in sorted({1, max(1, d // 3), sd.k_for_sparsity(d, 40), d - 1}):
+        y, x_rot, idx, val = fused_outputs(L, x.cuda(), Qt, W_rot, K)
+        # x_rot equals x up to the sign of zero
+        assert np.array_equal(np.abs(x_rot), np.abs(xd)), (kind, d, K)
+        want_i, want_v = oracle.topk(xd, K)
+        assert np.array_equal(idx.reshape(-1), want_i.reshape(-1)), (kind, d, K)
+        assert np.array_equal(np.abs(val.reshape(-1)), np.abs(want_v.reshape(-1)).astype(np.float32))
+        ref = oracle.sparse_linear(want_i.reshape(-1), xd[0, want_i.reshape(-1)], f64(W_rot))
+        got, bound = y.reshape(-1), (K + 2) * U * (np.abs(xd[0, want_i.reshape(-1)]) @ np.abs(f64(W_rot)[want_i.reshape(-1)]))
+        assert np.all(np.abs(got - ref) <= bound + 1e-37), (kind, d, K)
