@@ -13,7 +13,7 @@ fallback path.  (``build_lib`` builds the library without loading it.)
 """
 _EXPORTS = (
     "LarosaError", "Workspace", "larosa_check", "larosa_dense_linear", "larosa_prepare_weights",
-    "larosa_rotate", "larosa_rotate_topk_linear", "larosa_sparse_linear",
+    "larosa_rotate", "larosa_rotate_topk", "larosa_rotate_topk_linear", "larosa_sparse_linear",
     "larosa_sparse_linear_noalloc", "larosa_topk", "larosa_version", "larosa_workspace_bytes",
     "larosa_workspace_layout", "LAROSA_F32", "LAROSA_BF16", "LAROSA_MAX_D", "LAROSA_MAX_M",
     "LIB_PATH",

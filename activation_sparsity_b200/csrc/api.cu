@@ -5,7 +5,9 @@
 //   Top-K alone                topk_kernel (topk.cu)
 //   sparse linear, M = 1       cluster gather over idx/val (onetoken.cu)
 //   sparse linear, M > 1       scatter + union (union.cu) + rowstream (rowstream.cu)
-//   fused, M = 1               rowdot -> select-and-gather: two kernels
+//   rotation + Top-K, M = 1    rotsel (onetoken.cu): its last CTA selects
+//   fused, M = 1               fused_kernel (onetoken.cu): one cooperative launch;
+//                              where it does not fit, rotsel -> list gather
 //   fused, M > 1               rowdot -> topk -> scatter/union -> rowstream
 #include <stdio.h>
 #include <string.h>
@@ -24,6 +26,12 @@ namespace {
 
 constexpr int kMaxDout = 65536;
 constexpr size_t kTicketWords = 2048;
+// The last 16 ticket words belong to the one-token kernels: 8 synchronisation
+// words of the fused kernel, and the rotate + select kernel's ticket.  The
+// multi-token split-K tickets use the words below them.
+constexpr size_t kSplitKTicketWords = kTicketWords - 16;
+constexpr size_t kFusedSync = kTicketWords - 16;
+constexpr size_t kRotSelTicket = kTicketWords - 1;
 constexpr size_t kBitmapWords = LAROSA_MAX_D / 32;
 // Fixed header: words that must be zero before a call and are zero after it.
 constexpr size_t kOffTickets = 0;
@@ -101,16 +109,15 @@ int make_layout_uncached(int M, int d_in, int d_out, int K, Layout* L) {
   for (int dt = 0; dt < 2; ++dt) {
     const Elem w = dt == 0 ? Elem::F32 : Elem::BF16;
     if (M == 1) {
-      larosa::StreamPlan sl, ss;
-      cudaError_t e = larosa::plan_gather(larosa::kGatherList, w, d_in, d_out, K, &sl);
-      if (e == cudaSuccess) e = larosa::plan_gather(larosa::kGatherSelect, w, d_in, d_out, K, &ss);
+      larosa::StreamPlan sl;
+      cudaError_t e = larosa::plan_gather(w, d_out, K, &sl);
       if (e != cudaSuccess) return cuda_fail(e, "plan gather");
-      if (sl.ok && ss.ok) continue;  // the cluster kernels need no partials
+      if (sl.ok) continue;  // the cluster kernel needs no partials
     }
     GemvPlan ps;
     cudaError_t e = larosa::plan_gemv(w, Elem::F32, M, d_out, sparse_rows_max(M, d_in, K), &ps);
     if (e != cudaSuccess) return cuda_fail(e, "plan sparse linear");
-    if (ps.ticket_words > kTicketWords) return LAROSA_ERR_SHAPE;
+    if (ps.ticket_words > kSplitKTicketWords) return LAROSA_ERR_SHAPE;
     partials = std::max(partials, ps.partial_floats);
   }
   size_t off = align_up(kHeaderEnd, 256);
@@ -163,7 +170,7 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
                cudaStream_t s) {
   if (M == 1) {
     larosa::StreamPlan sp;
-    cudaError_t e = larosa::plan_gather(larosa::kGatherList, elem_of(dtype), d_in, d_out, K, &sp);
+    cudaError_t e = larosa::plan_gather(elem_of(dtype), d_out, K, &sp);
     if (e != cudaSuccess) return cuda_fail(e, "plan gather");
     if (sp.ok) {
       larosa::GatherArgs a;
@@ -175,7 +182,7 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
       a.rows = idx;
       a.y = y;
       a.dev_status = dev_status;
-      e = larosa::launch_gather(larosa::kGatherList, elem_of(dtype), a, sp, s);
+      e = larosa::launch_gather(elem_of(dtype), a, sp, s);
       return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "gather kernel");
     }
   }
@@ -303,6 +310,35 @@ int larosa_topk(const float* x_rot, int M, int d, int K, int32_t* idx, float* va
   return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "topk kernel");
 }
 
+int larosa_rotate_topk(const void* x, const void* Qt, float* x_rot, int32_t* idx, float* val, int d,
+                       int K, void* ws, size_t ws_bytes, int* dev_status, int dtype,
+                       larosa_stream_t stream) {
+  if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
+  if (x == nullptr || Qt == nullptr || x_rot == nullptr || (K > 0 && (idx == nullptr || val == nullptr)))
+    return LAROSA_ERR_INVALID_ARG;
+  int st = check_sizes(1, d, 1, K);
+  if (st != LAROSA_OK) return st;
+  if (!rowdot_aligned(Qt, x, d) || !aligned16(x_rot)) return LAROSA_ERR_ALIGN;
+  if (!larosa::rotsel_fits(elem_of(dtype), d)) return LAROSA_ERR_SHAPE;
+  Layout L;
+  st = make_layout(1, d, 1, K, &L);
+  if (st != LAROSA_OK) return st;
+  st = workspace_ok(ws, ws_bytes, L);
+  if (st != LAROSA_OK) return st;
+  larosa::RotSelArgs r;
+  r.x = x;
+  r.Qt = Qt;
+  r.x_rot = x_rot;
+  r.idx = idx;
+  r.val = val;
+  r.ticket = reinterpret_cast<unsigned*>(at(ws, kOffTickets + kRotSelTicket * 4));
+  r.d = d;
+  r.K = K;
+  r.dev_status = dev_status;
+  cudaError_t e = larosa::launch_rotsel(elem_of(dtype), r, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "rotate-select kernel");
+}
+
 int larosa_sparse_linear(const int32_t* idx, const float* val, int M, int K, const void* W_rot,
                          int d_in, int d_out, float* y, void* ws, size_t ws_bytes, int dtype,
                          int* dev_status, larosa_stream_t stream) {
@@ -341,28 +377,62 @@ int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, 
   float* x_rot = reinterpret_cast<float*>(at(ws, L.x_rot));
   int32_t* idx = reinterpret_cast<int32_t*>(at(ws, L.idx));
   float* val = reinterpret_cast<float*>(at(ws, L.val));
-  st = run_rowdot(x, Qt, x_rot, M, d_in, d_in, dtype, s, "rotation kernel");
-  if (st != LAROSA_OK) return st;
   if (M == 1) {
-    // every CTA of the gather selects the Top-K of x_rot on its own
+    // one cooperative kernel: rotation, selection, gather
+    larosa::StreamPlan fp;
+    cudaError_t e = larosa::plan_fused(elem_of(dtype), d_in, d_out, K, &fp);
+    if (e != cudaSuccess) return cuda_fail(e, "plan fused");
+    if (fp.ok) {
+      larosa::FusedArgs f;
+      f.x = x;
+      f.Qt = Qt;
+      f.W = W_rot;
+      f.x_rot = x_rot;
+      f.idx = idx;
+      f.val = val;
+      f.y = y;
+      f.sync = reinterpret_cast<unsigned*>(at(ws, kOffTickets + kFusedSync * 4));
+      f.d_in = d_in;
+      f.d_out = d_out;
+      f.K = K;
+      f.dev_status = dev_status;
+      e = larosa::launch_fused(elem_of(dtype), f, fp, s);
+      return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "fused kernel");
+    }
+  }
+  if (M == 1 && larosa::rotsel_fits(elem_of(dtype), d_in)) {
+    // rotation whose last CTA writes the kept list, then the list-mode gather
     larosa::StreamPlan sp;
-    cudaError_t e = larosa::plan_gather(larosa::kGatherSelect, elem_of(dtype), d_in, d_out, K, &sp);
+    cudaError_t e = larosa::plan_gather(elem_of(dtype), d_out, K, &sp);
     if (e != cudaSuccess) return cuda_fail(e, "plan gather");
     if (sp.ok) {
+      larosa::RotSelArgs r;
+      r.x = x;
+      r.Qt = Qt;
+      r.x_rot = x_rot;
+      r.idx = idx;
+      r.val = val;
+      r.ticket = reinterpret_cast<unsigned*>(at(ws, kOffTickets + kRotSelTicket * 4));
+      r.d = d_in;
+      r.K = K;
+      r.dev_status = dev_status;
+      e = larosa::launch_rotsel(elem_of(dtype), r, s);
+      if (e != cudaSuccess) return cuda_fail(e, "rotate-select kernel");
       larosa::GatherArgs a;
       a.W = W_rot;
       a.d_out = d_out;
       a.row_bound = d_in;
       a.n = K;
-      a.coef = x_rot;
+      a.coef = val;
+      a.rows = idx;
       a.y = y;
-      a.idx_out = idx;
-      a.val_out = val;
       a.dev_status = dev_status;
-      e = larosa::launch_gather(larosa::kGatherSelect, elem_of(dtype), a, sp, s);
-      return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "select-gather kernel");
+      e = larosa::launch_gather(elem_of(dtype), a, sp, s);
+      return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "gather kernel");
     }
   }
+  st = run_rowdot(x, Qt, x_rot, M, d_in, d_in, dtype, s, "rotation kernel");
+  if (st != LAROSA_OK) return st;
   cudaError_t e = larosa::launch_topk(x_rot, M, d_in, K, idx, val, dev_status, s);
   if (e != cudaSuccess) return cuda_fail(e, "topk kernel");
   return run_sparse(idx, val, M, K, W_rot, d_in, d_out, y, dtype, ws, L, dev_status, s);

@@ -86,21 +86,16 @@ struct GatherArgs {
   int d_out = 0;
   int row_bound = 0;        // d_in
   int n = 0;                // list length K
-  const void* coef = nullptr;     // kGatherList: val[K]; kGatherSelect: x_rot[d_in]
-  const int32_t* rows = nullptr;  // kGatherList: idx[K]
+  const void* coef = nullptr;     // val[K]
+  const int32_t* rows = nullptr;  // idx[K]
   float* y = nullptr;
-  int32_t* idx_out = nullptr;     // kGatherSelect: kept indices / values (optional)
-  float* val_out = nullptr;
   int* dev_status = nullptr;
 };
 
-constexpr int kGatherList = 1;    // rows idx[], coefficients val[]
-constexpr int kGatherSelect = 2;  // select the top-K of x_rot, then gather
-
-// Plans a one-token gather (mode kGatherList or kGatherSelect) of K kept rows
-// of a [d_in x d_out] weight; plan->ok is false when the shape does not fit.
-cudaError_t plan_gather(int mode, Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan);
-cudaError_t launch_gather(int mode, Elem w_elem, const GatherArgs& a, const StreamPlan& plan,
+// Plans a one-token gather of K kept rows (indices idx[], coefficients val[])
+// of a row-major [* x d_out] weight; plan->ok is false when it does not fit.
+cudaError_t plan_gather(Elem w_elem, int d_out, int K, StreamPlan* plan);
+cudaError_t launch_gather(Elem w_elem, const GatherArgs& a, const StreamPlan& plan,
                           cudaStream_t stream);
 
 // Row-dot GEMV y[m][j] = sum_i x[m][i] A[j][i] for M <= 16 tokens, A row-major
@@ -108,6 +103,50 @@ cudaError_t launch_gather(int mode, Elem w_elem, const GatherArgs& a, const Stre
 // torch.nn.Linear layout).  n_in a multiple of 8; x and A 16-byte aligned.
 cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M, int n_in,
                           int n_out, cudaStream_t stream);
+
+// One token: x_rot = x . Q (through Qt = Q^T), then the last CTA to finish
+// writes the kept list (idx, val: the K largest |x_rot|, ties to the lower
+// index, ascending) for a list-mode gather launched right after it.
+// `ticket` must be zero before the call and is zero again after it.
+struct RotSelArgs {
+  const void* x = nullptr;
+  const void* Qt = nullptr;
+  float* x_rot = nullptr;
+  int32_t* idx = nullptr;
+  float* val = nullptr;
+  unsigned* ticket = nullptr;
+  int d = 0;
+  int K = 0;
+  int* dev_status = nullptr;
+};
+
+// True when d is a multiple of 8 and the selection fits in shared memory.
+bool rotsel_fits(Elem e, int d);
+cudaError_t launch_rotsel(Elem e, const RotSelArgs& a, cudaStream_t stream);
+
+// One token, one cooperative launch: rotation, Top-K by a selector CTA, and
+// the gather of the kept rows (onetoken.cu, fused_kernel).  `sync` points to
+// 8 words of the caller's workspace, zero before the first call; calls that
+// share them must not overlap on the GPU.
+struct FusedArgs {
+  const void* x = nullptr;
+  const void* Qt = nullptr;
+  const void* W = nullptr;
+  float* x_rot = nullptr;
+  int32_t* idx = nullptr;
+  float* val = nullptr;
+  float* y = nullptr;
+  unsigned* sync = nullptr;
+  int d_in = 0;
+  int d_out = 0;
+  int K = 0;
+  int* dev_status = nullptr;
+};
+
+// plan->ok is false when the shape does not fit (then use the two-kernel path).
+cudaError_t plan_fused(Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan);
+cudaError_t launch_fused(Elem w_elem, const FusedArgs& a, const StreamPlan& plan,
+                         cudaStream_t stream);
 
 // W_rot = Qt . W with Qt = Q^T given row-major.
 cudaError_t launch_prepare(const void* Q, const void* W, void* W_rot, int d_in, int d_out,

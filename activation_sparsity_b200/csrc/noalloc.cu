@@ -89,7 +89,7 @@ extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val
     // one token: the cluster gather keeps its partial sums in distributed
     // shared memory and needs no scratch at all
     larosa::StreamPlan sp;
-    cudaError_t e = larosa::plan_gather(larosa::kGatherList, w, d_in, d_out, K, &sp);
+    cudaError_t e = larosa::plan_gather(w, d_out, K, &sp);
     if (e != cudaSuccess) return fail_cuda(e, "plan");
     if (sp.ok) {
       larosa::GatherArgs a;
@@ -101,7 +101,7 @@ extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val
       a.rows = idx;
       a.y = y;
       a.dev_status = dev_status;
-      e = larosa::launch_gather(larosa::kGatherList, w, a, sp, s);
+      e = larosa::launch_gather(w, a, sp, s);
       return e == cudaSuccess ? LAROSA_OK : fail_cuda(e, "sparse linear kernel");
     }
   }

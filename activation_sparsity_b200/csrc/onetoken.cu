@@ -27,10 +27,10 @@
 //         nothing leaves the cluster but y.  The tile width is chosen so the
 //         clusters that fit on the GPU at once cover d_out.
 //           kGather  row(p) = idx[p], coef(p) = val[p]
-//           kSelect  each cluster first selects the K largest |x_rot| itself
-//                    (exact, ties to the lower index; no grid-wide handoff)
-//                    and starts streaming the rows it is sure of before the
-//                    last places are decided.
+//           kSelect  every CTA first selects the K largest |x_rot| itself
+//                    (exact, ties to the lower index; no grid-wide handoff
+//                    and no exchange inside the cluster), then takes its
+//                    part of the kept list.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -166,461 +166,106 @@ __global__ void __launch_bounds__(kT, (MT <= 2 && sizeof(T) == 2 ? 2 : 1)) rowdo
 
 // ================================================================ gather
 
-constexpr int kModeGather = 1;
-constexpr int kModeSelect = 2;
-constexpr int kC = 8;  // CTAs per cluster (one column tile)
 constexpr int kGatherSmemCeiling = 227 * 1024;
-// Boundary-bin candidates ranked directly; a fuller bin takes radix passes.
-constexpr int kRankCap = kT;
+constexpr int kCandCap = 1024;  // boundary-bin keys ranked directly
 
 struct GParams {
   const void* W;         // [d_in x d_out] row-major
   int d_out;
   int d_in;              // row bound; also the length of x_rot
   int K;                 // kept entries
-  const void* coef;      // gather: val[K]; select: x_rot[d_in]
-  const int32_t* rows;   // gather: idx[K]
+  const void* coef;      // val[K]
+  const int32_t* rows;   // idx[K]
   float* y;
   int col_tile;
   int tpr;
   int list_cap;          // list entries a CTA holds: ceil(K / cluster)
-  int32_t* idx_out;      // select: kept indices/values (optional)
-  float* val_out;
   int* dev_status;
 };
 
 // Shared memory of one CTA, laid out from sizes known at launch.
 struct GLayout {
-  size_t sel, merged, xchg, keys, kflag, cand, call, cflag, rows, vals, part, red, total;
+  size_t red, rows, vals, part, total;
 };
 
 __host__ __device__ inline size_t al16(size_t v) { return (v + 15) & ~size_t(15); }
 
-// list_cap: list entries a CTA holds (kept positions of its part, or kept
-// entries of its index range); key_cap: rotated entries a CTA owns (select).
-__host__ __device__ inline GLayout glayout(int mode, int key_cap, int list_cap, int col_tile,
-                                           int cpt) {
-  GLayout L;
+__host__ __device__ inline GLayout glayout(int list_cap, int col_tile, int cpt) {
+  GLayout L{};
   size_t o = 0;
-  const bool sel = mode == kModeSelect;
-  L.sel = o;      o = al16(o + (sel ? sizeof(SelectScratch) : 64));
-  L.merged = o;   o = al16(o + (sel ? kSelBins * 4 : 0));
-  L.xchg = o;     o = al16(o + (sel ? 4 * 32 * 4 : 0));
-  L.keys = o;     o = al16(o + (sel ? (size_t)key_cap * 4 : 0));
-  L.kflag = o;    o = al16(o + (sel ? (size_t)key_cap : 0));
-  L.cand = o;     o = al16(o + (sel ? (size_t)kRankCap * 8 : 0));
-  L.call = o;     o = al16(o + (sel ? (size_t)kRankCap * 8 : 0));
-  L.cflag = o;    o = al16(o + (sel ? (size_t)kRankCap : 0));
-  L.rows = o;     o = al16(o + (size_t)list_cap * 4);
-  L.vals = o;     o = al16(o + (size_t)list_cap * 4);
-  L.part = o;     o = al16(o + (size_t)col_tile * 4);
-  L.red = o;      o = al16(o + (size_t)kT * cpt * 4);
+  L.red = o;   o = al16(o + (size_t)(kT / (col_tile / cpt)) * col_tile * 4);
+  L.rows = o;  o = al16(o + (size_t)list_cap * 4);
+  L.vals = o;  o = al16(o + (size_t)list_cap * 4);
+  L.part = o;  o = al16(o + (size_t)col_tile * 4);
   L.total = o;
   return L;
 }
 
-// Split cluster barrier: arrive publishes this thread's earlier writes
-// (shared and distributed shared memory) to every CTA of the cluster; wait
-// returns once all threads of the cluster have arrived.
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// The bin holding the krem-th largest counted key, scanning counts[nb] from
-// the top: writes bin, keys above it, keys in it to pick[0], pick[1],
-// pick[3].  Ends with a barrier.
-template <int NT>
-__device__ __forceinline__ void boundary_from_top(const uint32_t* counts, int nb, uint32_t krem,
-                                                  SelectScratch* s) {
+// Streams rows lrows[lo, hi) of one column tile (columns [c0, c0 + wc) of a
+// row-major [* x d_out] weight), scaled by lvals, into this thread's acc.
+// Thread (g, col) reads 16 bytes of rows lo + g, lo + g + ng, ... with kU
+// loads in flight.
+template <typename Tw>
+__device__ __forceinline__ void accumulate_rows(const void* W, int d_out, int c0, int wc, int tpr,
+                                                const int32_t* lrows, const float* lvals, int lo,
+                                                int hi, float (&acc)[16 / sizeof(Tw)]) {
+  constexpr int CPT = 16 / sizeof(Tw);
   const int tid = threadIdx.x;
-  // thread t owns ranks [t*per, t*per+per) counted from the top
-  constexpr int kPer = (kSelBins + NT - 1) / NT;
-  const int per = (nb + NT - 1) / NT;
-  uint32_t cnt[kPer];
-  uint32_t own = 0;
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int k = tid * per + j;
-    cnt[j] = (j < per && k < nb) ? counts[nb - 1 - k] : 0u;
-    own += cnt[j];
-  }
-  uint32_t before = block_scan_excl_1s<NT>(own, s->warp_sums, nullptr);
-  if (before < krem && krem <= before + own) {
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      if (j < per && before < krem && krem <= before + cnt[j]) {
-        s->pick[0] = static_cast<uint32_t>(nb - 1 - (tid * per + j));
-        s->pick[1] = before;
-        s->pick[3] = cnt[j];
-      }
-      before += cnt[j];
-    }
-  }
-  __syncthreads();
-}
-
-// One radix pass of a selection spread over a cluster: histogram this CTA's
-// keys that match `prefix` under `mask` on digit (key >> shift) & (nb-1),
-// add the cluster's histograms (rank r adds bins [r*nb/kC, (r+1)*nb/kC) and
-// writes the sums into every CTA's `merged`), then find the boundary bin as
-// boundary_from_top does.  `hist` (both copies) must be zero on entry and is
-// zero again on return.
-template <int NT>
-__device__ __forceinline__ void cluster_radix_pass(cg::cluster_group& cl, int rank,
-                                                   const uint32_t* keys, int n_mine,
-                                                   uint32_t prefix, uint32_t mask, int shift,
-                                                   int nb, uint32_t krem, SelectScratch* s,
-                                                   uint32_t* merged) {
-  const int tid = threadIdx.x;
-  uint32_t* h = s->hist + (tid & 1) * kSelBins;
-  for (int i = tid; i < n_mine; i += NT) {
-    const uint32_t k = keys[i] & kKeyMask;
-    if ((k & mask) == prefix) atomicAdd(&h[(k >> shift) & static_cast<uint32_t>(nb - 1)], 1u);
-  }
-  __syncthreads();
-  for (int b = tid; b < nb; b += NT) {
-    s->hist[b] += s->hist[kSelBins + b];
-    s->hist[kSelBins + b] = 0u;
-  }
-  cl.sync();  // every CTA's histogram is final
-  const int b0 = nb * rank / kC, b1 = nb * (rank + 1) / kC;
-  for (int b = b0 + tid; b < b1; b += NT) {
-    uint32_t v[kC];
-#pragma unroll
-    for (int q = 0; q < kC; ++q) v[q] = cl.map_shared_rank(s->hist, q)[b];  // all in flight
-    uint32_t sum = 0;
-#pragma unroll
-    for (int q = 0; q < kC; ++q) sum += v[q];
-#pragma unroll
-    for (int q = 0; q < kC; ++q) cl.map_shared_rank(merged, q)[b] = sum;
-  }
-  cl.sync();  // merged everywhere; no CTA still reads another's `hist`
-  for (int b = tid; b < nb; b += NT) s->hist[b] = 0u;
-  boundary_from_top<NT>(merged, nb, krem, s);
-}
-
-// Rank of a boundary-bin key: larger |x| first, then the lower index.
-__device__ __forceinline__ unsigned long long cand_order(uint32_t key, int idx) {
-  return (static_cast<unsigned long long>(key & kKeyMask) << 32) |
-         static_cast<uint32_t>(~static_cast<uint32_t>(idx));
-}
-
-// One cluster per column tile; the cluster's CTAs split the kept list in
-// rank order, and their partial sums meet in distributed shared memory.
-//
-// Select mode.  Rank r owns the rotated entries [d*r/C, d*(r+1)/C).  Every
-// CTA histograms all d keys on bits 30..20 (sign cleared) and finds the bin
-// B holding the K-th largest: keys above B are kept for certain, keys in B
-// are candidates for the remaining krem places.  Each CTA then streams its
-// certain rows while the cluster trades candidate lists (split barrier),
-// ranks the candidates exactly, and streams its kept candidates last.  The
-// order of the sum over rows is a function of the data only, so results
-// repeat bit for bit.
-template <typename Tw, int MODE>
-__global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
-  constexpr int CPT = 16 / sizeof(Tw);  // columns per thread per row
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  cg::cluster_group cl = cg::this_cluster();
-  constexpr int C = kC;
-  const int rank = static_cast<int>(cl.block_rank());
-  const int key_cap = (p.d_in + C - 1) / C;
-  const GLayout L = glayout(MODE, key_cap, p.list_cap, p.col_tile, CPT);
-  SelectScratch* sel = reinterpret_cast<SelectScratch*>(smem_raw + L.sel);
-  int32_t* lrows = reinterpret_cast<int32_t*>(smem_raw + L.rows);
-  float* lvals = reinterpret_cast<float*>(smem_raw + L.vals);
-  float* part = reinterpret_cast<float*>(smem_raw + L.part);
-  float* red = reinterpret_cast<float*>(smem_raw + L.red);
-
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int tile = blockIdx.y;
-  const int c0 = tile * p.col_tile;
-  const int wc = min(p.col_tile, p.d_out - c0);
-  const int K = p.K;
-
-  // ---- streaming: thread (g, col) reads 16 bytes of list rows lo+g,
-  // lo+g+ng, ... < hi, with kU loads in flight, into acc
-  const int tpr = p.tpr;
   const int ng = kT / tpr;
   const int g = tid / tpr;
   const int col = (tid - g * tpr) * CPT;
-  const bool active = g < ng && col < wc;
-  float acc[CPT];
+  if (g >= ng || col >= wc) return;
+  const unsigned char* wbase = static_cast<const unsigned char*>(W) + ((size_t)c0 + col) * sizeof(Tw);
+  const size_t pitch = (size_t)d_out * sizeof(Tw);
+  for (int r0 = lo + g; r0 < hi; r0 += ng * kU) {
+    uint4 u[kU];
 #pragma unroll
-  for (int v = 0; v < CPT; ++v) acc[v] = 0.f;
-  const unsigned char* wbase = static_cast<const unsigned char*>(p.W) + ((size_t)c0 + col) * sizeof(Tw);
-  const size_t pitch = (size_t)p.d_out * sizeof(Tw);
-  auto stream_rows = [&](int lo, int hi) {
-    if (!active) return;
-    for (int r0 = lo + g; r0 < hi; r0 += ng * kU) {
-      uint4 u[kU];
+    for (int k = 0; k < kU; ++k) {
+      const int r = r0 + k * ng;
+      u[k] = r < hi ? ld_stream(wbase + (size_t)lrows[r] * pitch) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-      for (int k = 0; k < kU; ++k) {
-        const int r = r0 + k * ng;
-        u[k] = r < hi ? ld_stream(wbase + (size_t)lrows[r] * pitch) : make_uint4(0, 0, 0, 0);
-      }
+    for (int k = 0; k < kU; ++k) {
+      const int r = r0 + k * ng;
+      const float cf = r < hi ? lvals[r] : 0.f;
+      if constexpr (CPT == 8) {
+        float w[8];
+        Vec8<__nv_bfloat16>::cvt(&u[k], w);
 #pragma unroll
-      for (int k = 0; k < kU; ++k) {
-        const int r = r0 + k * ng;
-        const float cf = r < hi ? lvals[r] : 0.f;
-        if constexpr (CPT == 8) {
-          float w[8];
-          Vec8<__nv_bfloat16>::cvt(&u[k], w);
-#pragma unroll
-          for (int v = 0; v < 8; ++v) acc[v] = fmaf(cf, w[v], acc[v]);
-        } else {
-          acc[0] = fmaf(cf, __uint_as_float(u[k].x), acc[0]);
-          acc[1] = fmaf(cf, __uint_as_float(u[k].y), acc[1]);
-          acc[2] = fmaf(cf, __uint_as_float(u[k].z), acc[2]);
-          acc[3] = fmaf(cf, __uint_as_float(u[k].w), acc[3]);
-        }
+        for (int v = 0; v < 8; ++v) acc[v] = fmaf(cf, w[v], acc[v]);
+      } else {
+        acc[0] = fmaf(cf, __uint_as_float(u[k].x), acc[0]);
+        acc[1] = fmaf(cf, __uint_as_float(u[k].y), acc[1]);
+        acc[2] = fmaf(cf, __uint_as_float(u[k].z), acc[2]);
+        acc[3] = fmaf(cf, __uint_as_float(u[k].w), acc[3]);
       }
     }
-  };
-
-  if constexpr (MODE == kModeSelect) {
-    for (int b = tid; b < 2 * kSelBins; b += kT) sel->hist[b] = 0u;
   }
-  pdl_wait();
-  pdl_launch_dependents();
+}
 
-  if constexpr (MODE == kModeGather) {
-    // rank r takes the kept positions [K*r/C, K*(r+1)/C)
-    const int p0 = (int)((long long)K * rank / C);
-    const int p1 = (int)((long long)K * (rank + 1) / C);
-    const int len = p1 - p0;
-    bool bad = false;
-    for (int j = tid; j < len; j += kT) {
-      const int row = p.rows[p0 + j];
-      const bool ok = static_cast<unsigned>(row) < static_cast<unsigned>(p.d_in);
-      bad |= !ok;
-      lrows[j] = ok ? row : 0;
-      lvals[j] = ok ? static_cast<const float*>(p.coef)[p0 + j] : 0.f;
-    }
-    if (__syncthreads_or(bad) && tid == 0) report(p.dev_status, LAROSA_DEV_INDEX);
-    stream_rows(0, len);
-  }
-
-  // select mode state kept for the index/value output at the end
-  const int d = p.d_in;
-  const int i_lo = (int)((long long)d * rank / C);
-  const int n_mine = (int)((long long)d * (rank + 1) / C) - i_lo;
-  const bool all = K >= d;
-  uint32_t B = 0;            // boundary bin (bits 30..20)
-  uint32_t kept_low = 0;     // kept entries owned by lower ranks
-  if constexpr (MODE == kModeSelect) {
-    uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + L.keys);
-    uint8_t* kflag = reinterpret_cast<uint8_t*>(smem_raw + L.kflag);  // kept candidate
-    uint32_t* merged = reinterpret_cast<uint32_t*>(smem_raw + L.merged);
-    // xchg[q]: certain rows of rank q; [32+q]: its candidates; [64+q] and
-    // [96+q]: above / at the threshold (radix fallback)
-    uint32_t* xchg = reinterpret_cast<uint32_t*>(smem_raw + L.xchg);
-    unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem_raw + L.cand);
-    unsigned long long* call = reinterpret_cast<unsigned long long*>(smem_raw + L.call);
-    uint8_t* cflag = reinterpret_cast<uint8_t*>(smem_raw + L.cflag);
-
-    // ---- all d keys -> histogram on bits 30..20; own keys -> `keys`
-    {
-      uint32_t* h = sel->hist + (lane & 1) * kSelBins;
-      const uint4* src = static_cast<const uint4*>(p.coef);  // d is a multiple of 8
-      bool nonfinite = false;
-      for (int v = tid; v < d / 4; v += kT) {
-        const uint4 u4 = __ldcg(src + v);
-        const uint32_t u[4] = {u4.x, u4.y, u4.z, u4.w};
+// Adds the threads' acc of one column tile into y[c0, c0 + wc): the row
+// groups meet in `red`, the CTA's partial in `part`, and rank r of the
+// cluster adds its slice of the tile over the C partials in rank order.
+// Every CTA of the cluster calls it (it holds two cluster barriers).
+template <typename Tw, int C>
+__device__ __forceinline__ void reduce_tile(cg::cluster_group& cl, int rank, int c0, int wc,
+                                            int col_tile, int tpr, const float (&acc)[16 / sizeof(Tw)],
+                                            float* red, float* part, float* y) {
+  constexpr int CPT = 16 / sizeof(Tw);
+  const int tid = threadIdx.x;
+  const int ng = kT / tpr;
+  const int g = tid / tpr;
+  const int col = (tid - g * tpr) * CPT;
+  if (g < ng && col < wc) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t k = u[e] & kKeyMask;
-          nonfinite |= k >= 0x7f800000u;
-          atomicAdd(&h[k >> 20], 1u);
-          const int j = 4 * v + e - i_lo;
-          if (j >= 0 && j < n_mine) {
-            keys[j] = u[e];
-            kflag[j] = 0;
-          }
-        }
-      }
-      if (__syncthreads_or(nonfinite) && tid == 0 && tile == 0 && rank == 0)
-        report(p.dev_status, LAROSA_DEV_NONFINITE);
-      for (int b = tid; b < kSelBins; b += kT) {
-        merged[b] = sel->hist[b] + sel->hist[kSelBins + b];
-        sel->hist[b] = 0u;
-        sel->hist[kSelBins + b] = 0u;
-      }
-      __syncthreads();
-    }
-    uint32_t krem = 0;  // candidates to keep
-    uint32_t nB = 0;    // keys in the boundary bin, cluster-wide
-    if (K > 0 && !all) {
-      boundary_from_top<kT>(merged, kSelBins, static_cast<uint32_t>(K), sel);
-      B = sel->pick[0];
-      krem = static_cast<uint32_t>(K) - sel->pick[1];
-      nB = sel->pick[3];
-    }
-    const bool ranked = nB <= static_cast<uint32_t>(kRankCap);  // same in every CTA
-
-    // ---- certain rows -> the list; candidates -> `cand` (ranked case)
-    const int chunk = (n_mine + kT - 1) / kT;
-    const int j0 = min(n_mine, tid * chunk), j1 = min(n_mine, j0 + chunk);
-    auto certain = [&](uint32_t k) { return K > 0 && (all || (k >> 20) > B); };
-    auto in_bin = [&](uint32_t k) { return K > 0 && !all && (k >> 20) == B; };
-    uint32_t n_def = 0, n_cand = 0;
-    {
-      uint32_t dc = 0, cc = 0;
-      for (int j = j0; j < j1; ++j) {
-        const uint32_t k = keys[j] & kKeyMask;
-        dc += certain(k);
-        cc += in_bin(k);
-      }
-      uint32_t tot = 0;
-      const uint32_t packed = block_scan_excl_1s<kT>((cc << 16) | dc, sel->warp_sums, &tot);
-      uint32_t dp = packed & 0xffffu, cp = packed >> 16;
-      n_def = tot & 0xffffu;
-      n_cand = tot >> 16;
-      for (int j = j0; j < j1; ++j) {
-        const uint32_t u = keys[j];
-        const uint32_t k = u & kKeyMask;
-        if (certain(k)) {
-          lrows[dp] = i_lo + j;
-          lvals[dp] = __uint_as_float(u);
-          ++dp;
-        } else if (ranked && in_bin(k)) {
-          cand[cp++] = cand_order(k, i_lo + j);
-        }
-      }
-      if (tid < C) {  // one remote store pair per destination rank
-        cl.map_shared_rank(xchg, tid)[rank] = n_def;
-        cl.map_shared_rank(xchg, tid)[32 + rank] = n_cand;
-      }
-      __syncthreads();  // the list is complete before it is streamed
-    }
-    cluster_arrive_release();
-    stream_rows(0, (int)n_def);
-    cluster_wait_acquire();  // every rank's counts and candidates are visible
-
-    const bool want_positions = tile == 0 && p.idx_out != nullptr;
-    int len = (int)n_def;
-    for (int q = 0; q < rank; ++q) kept_low += xchg[q];
-    if (ranked) {
-      // ---- the cluster's candidates in index order (rank, then position)
-      uint32_t run = 0, src_base = 0, lo_r = 0, hi_r = 0;
-      int src = 0;
-#pragma unroll
-      for (int q = 0; q < C; ++q) {
-        const uint32_t cq = xchg[32 + q];
-        if (static_cast<uint32_t>(tid) >= run) {  // the last rank starting at or below tid
-          src = q;
-          src_base = run;
-        }
-        if (q == rank) {
-          lo_r = run;
-          hi_r = run + cq;
-        }
-        run += cq;
-      }
-      const int n_all = (int)run;
-      if (tid < n_all) call[tid] = cl.map_shared_rank(cand, src)[tid - src_base];
-      __syncthreads();
-      // a warp per candidate: kept iff fewer than krem candidates outrank it
-      const int c_lo = want_positions ? 0 : (int)lo_r;
-      const int c_hi = (int)hi_r;
-      for (int c = c_lo + warp; c < c_hi; c += kWarps) {
-        const unsigned long long me = call[c];
-        uint32_t above = 0;
-        for (int i = lane; i < n_all; i += 32) above += call[i] > me;
-        above = __reduce_add_sync(0xffffffffu, above);
-        if (lane == 0) cflag[c] = above < krem;
-      }
-      __syncthreads();
-      const bool f = tid >= c_lo && tid < c_hi && cflag[tid];
-      const bool own = f && tid >= (int)lo_r;
-      uint32_t tot = 0;
-      const uint32_t packed = block_scan_excl_1s<kT>(((uint32_t)(f && !own) << 16) | own,
-                                                     sel->warp_sums, &tot);
-      if (own) {
-        const int idx = (int)~static_cast<uint32_t>(call[tid]);
-        const int pos = (int)n_def + (int)(packed & 0xffffu);
-        lrows[pos] = idx;
-        lvals[pos] = __uint_as_float(keys[idx - i_lo]);
-        kflag[idx - i_lo] = 1;
-      }
-      len += (int)(tot & 0xffffu);
-      kept_low += tot >> 16;
-    } else {
-      // ---- too many keys share bin B: two more radix passes inside it,
-      // with histograms added across the cluster, give the exact threshold
-      // T; ties at T go to the lowest indices across the cluster
-      uint32_t prefix = B << 20, mask = 0x7ffu << 20;
-#pragma unroll 1
-      for (int pass = 1; pass < 3; ++pass) {
-        const int shift = pass == 1 ? 9 : 0;
-        const int nb = pass == 1 ? 2048 : 512;
-        cluster_radix_pass<kT>(cl, rank, keys, n_mine, prefix, mask, shift, nb, krem, sel, merged);
-        prefix |= sel->pick[0] << shift;
-        mask |= static_cast<uint32_t>(nb - 1) << shift;
-        krem -= sel->pick[1];
-        __syncthreads();
-      }
-      const uint32_t T = prefix;  // krem keys equal to T are kept
-      uint32_t gt = 0, eq = 0;
-      for (int j = j0; j < j1; ++j) {
-        const uint32_t k = keys[j] & kKeyMask;
-        gt += (k >> 20) == B && k > T;
-        eq += k == T;
-      }
-      uint32_t tot = 0;
-      const uint32_t packed = block_scan_excl_1s<kT>((eq << 16) | gt, sel->warp_sums, &tot);
-      if (tid < C) {
-        cl.map_shared_rank(xchg, tid)[64 + rank] = tot & 0xffffu;
-        cl.map_shared_rank(xchg, tid)[96 + rank] = tot >> 16;
-      }
-      cl.sync();  // every CTA's counts are in every CTA
-      uint32_t ties_before = 0;
-      for (int q = 0; q < rank; ++q) {
-        const uint32_t tq = xchg[96 + q];
-        kept_low += xchg[64 + q] + min(tq, krem > ties_before ? krem - ties_before : 0u);
-        ties_before += tq;
-      }
-      const uint32_t ties_left = krem > ties_before ? krem - ties_before : 0u;
-      uint32_t eqc = packed >> 16;
-      uint32_t pos = n_def + (packed & 0xffffu) + min(eqc, ties_left);
-      for (int j = j0; j < j1; ++j) {
-        const uint32_t u = keys[j];
-        const uint32_t k = u & kKeyMask;
-        bool kept = false;
-        if ((k >> 20) == B && k > T) {
-          kept = true;
-        } else if (k == T) {
-          kept = eqc < ties_left;
-          ++eqc;
-        }
-        if (kept) {
-          lrows[pos] = i_lo + j;
-          lvals[pos] = __uint_as_float(u);
-          kflag[j] = 1;
-          ++pos;
-        }
-      }
-      len += (int)((tot & 0xffffu) + min(tot >> 16, ties_left));
-    }
-    __syncthreads();
-    stream_rows((int)n_def, len);
-  }
-
-  // ---- row groups -> this CTA's partial, in shared memory
-  if (active) {
-#pragma unroll
-    for (int v = 0; v < CPT; ++v) red[g * p.col_tile + col + v] = acc[v];
+    for (int v = 0; v < CPT; ++v) red[g * col_tile + col + v] = acc[v];
   }
   __syncthreads();
   for (int e = tid; e < wc; e += kT) {
     float sum = 0.f;
-    for (int gg = 0; gg < ng; ++gg) sum += red[gg * p.col_tile + e];
+    for (int gg = 0; gg < ng; ++gg) sum += red[gg * col_tile + e];
     part[e] = sum;
   }
-  // ---- the cluster's partials -> y: rank r adds its column slice in rank order
   cl.sync();
   const int sl = (wc + C - 1) / C;
   const int e0 = rank * sl, e1 = min(wc, e0 + sl);
@@ -631,37 +276,603 @@ __global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
     float sum = 0.f;
 #pragma unroll
     for (int q = 0; q < C; ++q) sum += v[q];
-    p.y[c0 + e] = sum;
+    y[c0 + e] = sum;
   }
   cl.sync();  // no CTA leaves while another may still read its partial
+}
 
-  // ---- the kept indices and values in ascending index order (one cluster)
-  if constexpr (MODE == kModeSelect) {
-    if (tile == 0 && p.idx_out != nullptr) {
-      const uint32_t* keys = reinterpret_cast<const uint32_t*>(smem_raw + L.keys);
-      const uint8_t* kflag = reinterpret_cast<const uint8_t*>(smem_raw + L.kflag);
-      const int chunk = (n_mine + kT - 1) / kT;
-      const int j0 = min(n_mine, tid * chunk), j1 = min(n_mine, j0 + chunk);
-      auto kept = [&](int j) {
-        return K > 0 && (all || ((keys[j] & kKeyMask) >> 20) > B || kflag[j] != 0);
-      };
-      uint32_t n = 0;
-      for (int j = j0; j < j1; ++j) n += kept(j);
-      uint32_t pos = kept_low + block_scan_excl_1s<kT>(n, sel->warp_sums, nullptr);
-      for (int j = j0; j < j1; ++j) {
-        if (kept(j)) {
-          p.idx_out[pos] = i_lo + j;
-          p.val_out[pos] = __uint_as_float(keys[j]);
-          ++pos;
+// Streams rows lrows[0, len) of one column tile and adds the cluster's
+// partial sums into y (accumulate_rows, then reduce_tile).
+template <typename Tw, int C>
+__device__ __forceinline__ void gather_tile(cg::cluster_group& cl, int rank, const void* W, int d_out,
+                                            int c0, int wc, int col_tile, int tpr,
+                                            const int32_t* lrows, const float* lvals, int len,
+                                            float* red, float* part, float* y) {
+  float acc[16 / sizeof(Tw)];
+#pragma unroll
+  for (int v = 0; v < 16 / (int)sizeof(Tw); ++v) acc[v] = 0.f;
+  accumulate_rows<Tw>(W, d_out, c0, wc, tpr, lrows, lvals, 0, len, acc);
+  reduce_tile<Tw, C>(cl, rank, c0, wc, col_tile, tpr, acc, red, part, y);
+}
+
+// One cluster of C CTAs per column tile.  The cluster's CTAs take equal
+// consecutive parts of the kept list (in ascending row order), stream those
+// rows of the tile, and add their partial sums through distributed shared
+// memory in rank order.
+//
+// Select mode: every CTA reads all d rotated entries and selects the K
+// largest magnitudes itself (exact; ties to the lower index), so no CTA
+// waits on another before streaming.  The same integer-only selection runs
+// in every CTA, so all of them derive the same kept list.
+template <typename Tw, int C>
+__global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
+  constexpr int CPT = 16 / sizeof(Tw);  // columns per thread per row
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = static_cast<int>(cl.block_rank());
+  const GLayout L = glayout(p.list_cap, p.col_tile, CPT);
+  int32_t* lrows = reinterpret_cast<int32_t*>(smem_raw + L.rows);
+  float* lvals = reinterpret_cast<float*>(smem_raw + L.vals);
+  float* part = reinterpret_cast<float*>(smem_raw + L.part);
+  float* red = reinterpret_cast<float*>(smem_raw + L.red);
+
+  const int tid = threadIdx.x;
+  const int tile = blockIdx.y;
+  const int c0 = tile * p.col_tile;
+  const int wc = min(p.col_tile, p.d_out - c0);
+  const int K = p.K;
+  // this CTA's part of the kept list: positions [p0, p1)
+  const int p0 = (int)((long long)K * rank / C);
+  const int p1 = (int)((long long)K * (rank + 1) / C);
+  const int len = p1 - p0;
+
+  pdl_wait();
+  pdl_launch_dependents();
+
+  {
+    bool bad = false;
+    for (int j = tid; j < len; j += kT) {
+      const int row = p.rows[p0 + j];
+      const bool ok = static_cast<unsigned>(row) < static_cast<unsigned>(p.d_in);
+      bad |= !ok;
+      lrows[j] = ok ? row : 0;
+      lvals[j] = ok ? static_cast<const float*>(p.coef)[p0 + j] : 0.f;
+    }
+    if (__syncthreads_or(bad) && tid == 0) report(p.dev_status, LAROSA_DEV_INDEX);
+  }
+  __syncthreads();  // the list is complete
+
+  gather_tile<Tw, C>(cl, rank, p.W, p.d_out, c0, wc, p.col_tile, p.tpr, lrows, lvals, len, red,
+                     part, p.y);
+}
+
+// ================================================================ rotate + select
+//
+// First kernel of the one-token fused path.  Every CTA computes an equal
+// share of the rotated rows x_rot[j] = x . Q^T[j] (as rowdot does) and then
+// arrives on a ticket; the last CTA to arrive reads the whole x_rot, selects
+// the K largest magnitudes (kept_list: exact, ties to the lower index) and
+// writes the kept list, in ascending index order, for the list-mode gather
+// that follows.  No CTA waits for another: the ticket only decides which CTA
+// does the selection.  The kernel lets its dependent launch at once, so the
+// gather's clusters are placed on the SMs that retiring CTAs free and wait
+// there (griddepcontrol.wait) until the selection is done.
+
+struct RSParams {
+  const void* x;     // [d] activation
+  const void* Qt;    // [d x d] rotation, stored transposed (row j = column j of Q)
+  float* x_rot;      // [d]
+  int32_t* idx;      // [K] kept list
+  float* val;        // [K]
+  unsigned* ticket;  // zero between calls
+  int d;
+  int K;
+  int* dev_status;
+};
+
+// Shared memory: the staged activation, later the last CTA's selection.
+struct RSLayout {
+  size_t sel, keys, cand, cand_idx, total;
+};
+
+__host__ __device__ inline RSLayout rslayout(int d, int elem_bytes) {
+  RSLayout L{};
+  size_t o = 0;
+  L.sel = o;   o = al16(o + sizeof(SelectScratch));
+  L.keys = o;  o = al16(o + (size_t)d * 4);
+  L.cand = o;  o = al16(o + (size_t)kCandCap * 4);
+  L.cand_idx = o; o = al16(o + (size_t)kCandCap * 4);
+  const size_t x_bytes = al16((size_t)d * elem_bytes);
+  L.total = o > x_bytes ? o : x_bytes;
+  return L;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kT, 2) rotsel_kernel(const RSParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ unsigned s_last;
+  const RSLayout L = rslayout(p.d, sizeof(T));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int d = p.d, K = p.K;
+
+  pdl_wait();
+  pdl_launch_dependents();
+
+  // ---- rotation rows [r0, r1) of this CTA
+  {
+    const int nvx = d * (int)sizeof(T) / 16;
+    const uint4* xg = static_cast<const uint4*>(p.x);
+    for (int i = tid; i < nvx; i += kT) reinterpret_cast<uint4*>(smem_raw)[i] = __ldg(xg + i);
+    __syncthreads();
+    const T* xs = reinterpret_cast<const T*>(smem_raw);
+    const int r0 = (int)((long long)d * cta / G);
+    const int r1 = (int)((long long)d * (cta + 1) / G);
+    const int nv = d / 8;  // 8-element vectors per row
+    constexpr int LD = Vec8<T>::kLoads;
+    constexpr int KU = kU / LD;  // the same bytes in flight for both element sizes
+    for (int row = r0 + warp; row < r1; row += kWarps) {
+      const unsigned char* arow = static_cast<const unsigned char*>(p.Qt) + (size_t)row * d * sizeof(T);
+      float acc = 0.f;
+      for (int v0 = lane; v0 < nv; v0 += 32 * KU) {
+        uint4 u[KU][LD];
+#pragma unroll
+        for (int k = 0; k < KU; ++k) {
+          const int v = v0 + 32 * k;
+#pragma unroll
+          for (int l = 0; l < LD; ++l)
+            u[k][l] = v < nv ? ld_stream(arow + (size_t)v * 8 * sizeof(T) + l * 16) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < KU; ++k) {
+          const int v = v0 + 32 * k;
+          if (v < nv) {
+            float w[8], xv[8];
+            Vec8<T>::cvt(u[k], w);
+            uint4 xu[LD];
+#pragma unroll
+            for (int l = 0; l < LD; ++l)
+              xu[l] = *reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(xs + (size_t)v * 8) + l * 16);
+            Vec8<T>::cvt(xu, xv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc = fmaf(w[e], xv[e], acc);
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) __stcg(p.x_rot + row, acc);
+    }
+    // lane 0 of each warp stored this CTA's rows: make them visible GPU-wide
+    // before the CTA arrives
+    if (lane == 0) __threadfence();
+  }
+  SelectScratch* sel = reinterpret_cast<SelectScratch*>(smem_raw + L.sel);
+  __syncthreads();  // the staged x is dead
+  for (int b = tid; b < kFineBins; b += kT) sel->hist[b] = 0u;  // for the selection, if last
+  if (tid == 0) {
+    const bool last = atomicAdd(p.ticket, 1u) == static_cast<unsigned>(G - 1);
+    if (last) __threadfence();  // every CTA's x_rot is visible after this
+    s_last = last;
+  }
+  __syncthreads();
+  if (!s_last) return;
+
+  // ---- the last CTA to arrive selects
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + L.keys);
+  uint32_t* cand = reinterpret_cast<uint32_t*>(smem_raw + L.cand);
+  uint32_t* cand_idx = reinterpret_cast<uint32_t*>(smem_raw + L.cand_idx);
+  const uint4* src = reinterpret_cast<const uint4*>(p.x_rot);  // d is a multiple of 8
+  uint4* dst = reinterpret_cast<uint4*>(keys);
+  const int nv = d / 4;
+  bool nonfinite = false;
+  for (int v0 = tid; v0 < nv; v0 += kT * kU) {
+    uint4 u[kU];
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      const int v = v0 + k * kT;
+      u[k] = v < nv ? __ldcg(src + v) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      const int v = v0 + k * kT;
+      if (v < nv) {
+        dst[v] = u[k];
+        const uint32_t w[4] = {u[k].x & kKeyMask, u[k].y & kKeyMask, u[k].z & kKeyMask,
+                               u[k].w & kKeyMask};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          nonfinite |= w[e] >= 0x7f800000u;
+          atomicAdd(&sel->hist[w[e] >> kFineShift], 1u);
         }
       }
     }
   }
+  if (__syncthreads_or(nonfinite) && tid == 0) report(p.dev_status, LAROSA_DEV_NONFINITE);
+  if (K > 0 && K < d) {
+    kept_list<kT>(keys, d, K, sel, cand, cand_idx, kCandCap, 0, K, p.idx, p.val);
+  } else if (K >= d) {
+    for (int i = tid; i < d; i += kT) {
+      p.idx[i] = i;
+      p.val[i] = __uint_as_float(keys[i]);
+    }
+  }
+  if (tid == 0) *p.ticket = 0u;  // zero again for the next call
+}
+
+// ================================================================ fused, one token
+//
+// rotate -> select -> gather in one cooperative launch of thread-block
+// clusters: gridDim.y = n_tiles + 1 clusters of C CTAs, all resident at once.
+//
+//   1. every CTA computes an equal share of x_rot[j] = x . Q^T[j] (as rowdot
+//      does), stores it and arrives on a ticket;
+//   2. the selector (rank 0 of the last cluster) waits for every arrival,
+//      loads x_rot, finds the histogram bin B that holds the K-th largest
+//      magnitude and publishes it (flag 0); it then ranks B's keys, publishes
+//      the K-th entry (T, I) (flag 1) and writes the kept list for callers;
+//   3. the gather CTAs (clusters 0 .. n_tiles-1, one column tile each; rank r
+//      owns the indices [d*r/C, d*(r+1)/C)) load their range of x_rot while
+//      the selector works, stream the rows that are certainly kept (bin
+//      above B) as soon as B is published, then the few kept rows of bin B
+//      once (T, I) is, and add their partial sums through distributed shared
+//      memory.
+//
+// Kept = the K largest |x_rot|, ties to the lower index: key > T, or
+// key == T and index <= I.  Every wait is bounded (kWaitLimitNs) and reports
+// LAROSA_DEV_TIMEOUT; the cooperative launch guarantees that every CTA is
+// resident, so no CTA waits on one that cannot run.
+//
+// Synchronisation words (sync[8], in the caller's workspace; all zero
+// initially): sync[3] is the number of the last call whose K-th entry was
+// published.  Every CTA reads it before it arrives, so all CTAs of a call
+// agree on its number n = sync[3] + 1 (calls that share the words must not
+// overlap).  Call n counts arrivals in sync[n & 1]; its selector clears the
+// other slot, which call n - 1 has finished with, so no counter is reset
+// while a CTA may still read it.  sync[2] and sync[3] become n when the
+// boundary bin and the K-th entry are published in sync[4..7].
+
+struct FParams {
+  const void* x;      // [d] activation
+  const void* Qt;     // [d x d] rotation, stored transposed
+  const void* W;      // [d x d_out] counter-rotated weight
+  float* x_rot;       // [d]
+  int32_t* idx;       // [K] kept list (for callers)
+  float* val;         // [K]
+  float* y;           // [d_out]
+  unsigned* sync;     // [0, 1] arrivals, [2] boundary / [3] K-th entry published,
+                      // [4] mode (0 none kept, 1 Top-K, 2 all kept), [5] B, [6] T, [7] I
+  int d;
+  int d_out;
+  int K;
+  int col_tile;
+  int tpr;
+  int range_cap;      // ceil(d / C): indices a gather CTA owns
+  int n_tiles;        // gather clusters; cluster n_tiles holds the selector
+  int* dev_status;
+};
+
+struct FLayout {
+  size_t sel, keys, cand, cand_idx, red, rows, vals, part, total;
+};
+
+// Region A (offset 0) holds, one after the other in time: the staged x; then
+// in the selector its scratch, all d keys and the boundary candidates, and in
+// a gather CTA its range of keys, then the row-group partials.
+__host__ __device__ inline FLayout flayout(int d, int elem_bytes, int range_cap, int col_tile,
+                                           int cpt) {
+  FLayout L{};
+  size_t o = 0;
+  L.sel = o;      o = al16(o + sizeof(SelectScratch));
+  L.keys = o;     o = al16(o + (size_t)d * 4);
+  L.cand = o;     o = al16(o + (size_t)kCandCap * 4);
+  L.cand_idx = o; o = al16(o + (size_t)kCandCap * 4);
+  const size_t x_bytes = al16((size_t)d * elem_bytes);
+  const size_t range_bytes = al16((size_t)range_cap * 4);
+  const size_t red_bytes = al16((size_t)(kT / (col_tile / cpt)) * col_tile * 4);
+  L.red = 0;
+  o = o > x_bytes ? o : x_bytes;
+  o = o > range_bytes ? o : range_bytes;
+  o = o > red_bytes ? o : red_bytes;
+  L.rows = o;  o = al16(o + (size_t)range_cap * 4);
+  L.vals = o;  o = al16(o + (size_t)range_cap * 4);
+  L.part = o;  o = al16(o + (size_t)col_tile * 4);
+  L.total = o;
+  return L;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Thread 0 waits until *ticket >= target; false after kWaitLimitNs.
+__device__ __forceinline__ bool wait_ticket(const unsigned* ticket, unsigned target) {
+  if (ld_acquire_gpu(ticket) >= target) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(ticket) >= target) return true;
+    if ((it & 31u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// Thread 0 waits until *flag == value; false after kWaitLimitNs.
+__device__ __forceinline__ bool wait_flag(const unsigned* flag, unsigned value) {
+  if (ld_acquire_gpu(flag) == value) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) == value) return true;
+    if ((it & 31u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// Appends to rows/vals (from position `base`) the indices i_lo + i of the
+// keys[0, n) that satisfy pred(key, i_lo + i), in ascending order, and
+// returns how many (the same value in every thread).  Warp segments and
+// ballots; all kT threads call it; it holds one barrier.
+template <typename Pred>
+__device__ __forceinline__ int compact_range(const uint32_t* keys, int n, int i_lo, Pred pred,
+                                             int32_t* rows, float* vals, int base,
+                                             uint32_t* warp_sums) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t below = (1u << lane) - 1u;
+  int s0, s1;
+  warp_segment<kT>(n, &s0, &s1);
+  uint32_t cnt = 0;
+  for (int i = s0 + lane; i < s1; i += 32) cnt += pred(keys[i] & kKeyMask, i_lo + i);
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  uint32_t total = 0;
+  uint32_t pos = __shfl_sync(0xffffffffu, block_scan_excl_1s<kT>(lane == 0 ? cnt : 0u, warp_sums, &total), 0);
+  if (cnt != 0u) {
+    pos += static_cast<uint32_t>(base);
+    for (int i0 = s0; i0 < s1; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t u = i < s1 ? keys[i] : 0u;
+      const bool hit = i < s1 && pred(u & kKeyMask, i_lo + i);
+      const uint32_t m = __ballot_sync(0xffffffffu, hit);
+      if (hit) {
+        rows[pos + __popc(m & below)] = i_lo + i;
+        vals[pos + __popc(m & below)] = __uint_as_float(u);
+      }
+      pos += __popc(m);
+    }
+  }
+  return static_cast<int>(total);
+}
+
+template <typename T, int C>
+__global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
+  constexpr int CPT = 16 / sizeof(T);
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ uint32_t s_gen;
+  __shared__ uint32_t s_word[8];
+  __shared__ uint32_t s_warp_sums[32];
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = static_cast<int>(cl.block_rank());
+  const FLayout L = flayout(p.d, sizeof(T), p.range_cap, p.col_tile, CPT);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.y;
+  const int G = C * static_cast<int>(gridDim.y);
+  const int cta = tile * C + rank;
+  const int d = p.d, K = p.K;
+
+  pdl_wait();
+  if (tid == 0) s_gen = ld_acquire_gpu(p.sync + 3) + 1u;  // this call's number, read before arriving
+
+  // ---- 1. rotation rows [r0, r1) of this CTA
+  {
+    const int nvx = d * (int)sizeof(T) / 16;
+    const uint4* xg = static_cast<const uint4*>(p.x);
+    for (int i = tid; i < nvx; i += kT) reinterpret_cast<uint4*>(smem_raw)[i] = __ldg(xg + i);
+    __syncthreads();
+    const T* xs = reinterpret_cast<const T*>(smem_raw);
+    const int r0 = (int)((long long)d * cta / G);
+    const int r1 = (int)((long long)d * (cta + 1) / G);
+    const int nv = d / 8;  // 8-element vectors per row
+    constexpr int LD = Vec8<T>::kLoads;
+    constexpr int KU = kU / LD;  // the same bytes in flight for both element sizes
+    for (int row = r0 + warp; row < r1; row += kWarps) {
+      const unsigned char* arow = static_cast<const unsigned char*>(p.Qt) + (size_t)row * d * sizeof(T);
+      float acc = 0.f;
+      for (int v0 = lane; v0 < nv; v0 += 32 * KU) {
+        uint4 u[KU][LD];
+#pragma unroll
+        for (int k = 0; k < KU; ++k) {
+          const int v = v0 + 32 * k;
+#pragma unroll
+          for (int l = 0; l < LD; ++l)
+            u[k][l] = v < nv ? ld_stream(arow + (size_t)v * 8 * sizeof(T) + l * 16) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < KU; ++k) {
+          const int v = v0 + 32 * k;
+          if (v < nv) {
+            float w[8], xv[8];
+            Vec8<T>::cvt(u[k], w);
+            uint4 xu[LD];
+#pragma unroll
+            for (int l = 0; l < LD; ++l)
+              xu[l] = *reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(xs + (size_t)v * 8) + l * 16);
+            Vec8<T>::cvt(xu, xv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc = fmaf(w[e], xv[e], acc);
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) __stcg(p.x_rot + row, acc);
+    }
+    if (lane == 0) __threadfence();  // this CTA's rows are visible GPU-wide before it arrives
+  }
+  __syncthreads();  // the staged x is dead
+  const unsigned gen = s_gen;
+  unsigned* ticket = p.sync + (gen & 1u);
+  if (tid == 0) atomicAdd(ticket, 1u);
+  const unsigned target = static_cast<unsigned>(G);
+
+  if (tile == p.n_tiles) {
+    if (rank != 0) return;  // the selector cluster's other CTAs only rotate
+    // ---- 2. the selector
+    SelectScratch* sel = reinterpret_cast<SelectScratch*>(smem_raw + L.sel);
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + L.keys);
+    uint32_t* cand = reinterpret_cast<uint32_t*>(smem_raw + L.cand);
+    uint32_t* cand_idx = reinterpret_cast<uint32_t*>(smem_raw + L.cand_idx);
+    for (int b = tid; b < kFineBins; b += kT) sel->hist[b] = 0u;
+    if (tid == 0) {
+      const bool ok = wait_ticket(ticket, target);
+      if (!ok) report(p.dev_status, LAROSA_DEV_TIMEOUT);
+      p.sync[(gen + 1u) & 1u] = 0u;  // the next call's counter (the previous call's is done)
+      s_word[0] = ok;
+    }
+    __syncthreads();
+    const bool ok = s_word[0] != 0u;
+    const uint32_t mode = !ok || K <= 0 ? 0u : (K >= d ? 2u : 1u);
+    if (ok) {
+      const uint4* src = reinterpret_cast<const uint4*>(p.x_rot);  // d is a multiple of 8
+      uint4* dst = reinterpret_cast<uint4*>(keys);
+      const int nv = d / 4;
+      bool nonfinite = false;
+      for (int v0 = tid; v0 < nv; v0 += kT * kU) {
+        uint4 u[kU];
+#pragma unroll
+        for (int k = 0; k < kU; ++k) {
+          const int v = v0 + k * kT;
+          u[k] = v < nv ? __ldcg(src + v) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < kU; ++k) {
+          const int v = v0 + k * kT;
+          if (v < nv) {
+            dst[v] = u[k];
+            const uint32_t w[4] = {u[k].x & kKeyMask, u[k].y & kKeyMask, u[k].z & kKeyMask,
+                                   u[k].w & kKeyMask};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              nonfinite |= w[e] >= 0x7f800000u;
+              atomicAdd(&sel->hist[w[e] >> kFineShift], 1u);
+            }
+          }
+        }
+      }
+      if (__syncthreads_or(nonfinite) && tid == 0) report(p.dev_status, LAROSA_DEV_NONFINITE);
+    }
+    uint32_t B = 0, above = 0, nB = 0;
+    if (mode == 1u) fine_boundary<kT>(sel, K, &B, &above, &nB);
+    if (tid == 0) {
+      p.sync[4] = mode;
+      p.sync[5] = B;
+      __threadfence();
+      st_release_gpu(p.sync + 2, gen);
+    }
+    KthEntry e{0u, -1};
+    if (mode == 1u) e = kth_entry<kT>(keys, d, K, B, static_cast<uint32_t>(K) - above, nB, sel, cand,
+                                      cand_idx, kCandCap);
+    if (tid == 0) {
+      p.sync[6] = e.T;
+      p.sync[7] = static_cast<uint32_t>(e.I);
+      __threadfence();
+      st_release_gpu(p.sync + 3, gen);
+    }
+    // the kept list for callers, off the gather's path
+    if (mode == 1u) {
+      write_kept<kT>(keys, d, e, 0, K, p.idx, p.val, sel);
+    } else if (mode == 2u) {
+      for (int i = tid; i < d; i += kT) {
+        p.idx[i] = i;
+        p.val[i] = __uint_as_float(keys[i]);
+      }
+    }
+    return;
+  }
+
+  // ---- 3. a gather CTA: rank r owns the indices [i_lo, i_hi)
+  uint32_t* rkeys = reinterpret_cast<uint32_t*>(smem_raw);  // region A: the range's keys
+  int32_t* lrows = reinterpret_cast<int32_t*>(smem_raw + L.rows);
+  float* lvals = reinterpret_cast<float*>(smem_raw + L.vals);
+  float* part = reinterpret_cast<float*>(smem_raw + L.part);
+  float* red = reinterpret_cast<float*>(smem_raw + L.red);
+  const int i_lo = (int)((long long)d * rank / C);
+  const int n_r = (int)((long long)d * (rank + 1) / C) - i_lo;
+  const int c0 = tile * p.col_tile;
+  const int wc = min(p.col_tile, p.d_out - c0);
+  float acc[CPT];
+#pragma unroll
+  for (int v = 0; v < CPT; ++v) acc[v] = 0.f;
+
+  // every CTA's x_rot is written: load this range while the selector works
+  if (tid == 0) {
+    const bool ok = wait_ticket(ticket, target);
+    if (!ok) report(p.dev_status, LAROSA_DEV_TIMEOUT);
+    s_word[0] = ok;
+  }
+  __syncthreads();
+  if (s_word[0] != 0u) {
+    for (int j0 = tid; j0 < n_r; j0 += kT * kU) {
+      uint32_t u[kU];
+#pragma unroll
+      for (int k = 0; k < kU; ++k) {
+        const int j = j0 + k * kT;
+        u[k] = j < n_r ? __float_as_uint(__ldcg(p.x_rot + i_lo + j)) : 0u;
+      }
+#pragma unroll
+      for (int k = 0; k < kU; ++k)
+        if (j0 + k * kT < n_r) rkeys[j0 + k * kT] = u[k];
+    }
+  }
+  // the boundary bin: rows above it are certainly kept
+  if (tid == 0) {
+    bool got = false;
+    if (s_word[0] != 0u) {
+      got = wait_flag(p.sync + 2, gen);
+      if (!got) report(p.dev_status, LAROSA_DEV_TIMEOUT);
+    }
+    s_word[1] = got ? __ldcg(p.sync + 4) : 0u;  // mode; 0 keeps nothing
+    s_word[2] = got ? __ldcg(p.sync + 5) : 0u;  // B
+  }
+  __syncthreads();
+  const uint32_t mode = s_word[1];
+  const uint32_t B = s_word[2];
+  const int n_certain = compact_range(
+      rkeys, n_r, i_lo,
+      [&](uint32_t k, int) { return mode == 2u || (mode == 1u && (k >> kFineShift) > B); },
+      lrows, lvals, 0, s_warp_sums);
+  __syncthreads();  // the certain list is in place
+  accumulate_rows<T>(p.W, p.d_out, c0, wc, p.tpr, lrows, lvals, 0, n_certain, acc);
+
+  // the K-th entry: the kept rows of bin B
+  if (tid == 0) {
+    bool got = false;
+    if (mode == 1u) {
+      got = wait_flag(p.sync + 3, gen);
+      if (!got) report(p.dev_status, LAROSA_DEV_TIMEOUT);
+    }
+    s_word[4] = got ? __ldcg(p.sync + 6) : 0u;  // T
+    s_word[5] = got ? __ldcg(p.sync + 7) : 0u;  // I
+    s_word[6] = got;
+  }
+  __syncthreads();
+  const bool have_kth = s_word[6] != 0u;
+  const KthEntry e{s_word[4], static_cast<int32_t>(s_word[5])};
+  const int n_more = compact_range(
+      rkeys, n_r, i_lo,
+      [&](uint32_t k, int i) { return have_kth && (k >> kFineShift) == B && is_kept(k, i, e); },
+      lrows, lvals, n_certain, s_warp_sums);
+  __syncthreads();  // the list is complete; the range's keys are dead
+  accumulate_rows<T>(p.W, p.d_out, c0, wc, p.tpr, lrows, lvals, n_certain, n_certain + n_more, acc);
+  reduce_tile<T, C>(cl, rank, c0, wc, p.col_tile, p.tpr, acc, red, part, p.y);
 }
 
 struct DevState {
   int sms = 0;
-  bool configured[16] = {};
+  bool configured[16] = {};  // kernel slots whose shared-memory ceiling is set
 };
 DevState g_state[64];
 
@@ -746,6 +957,47 @@ cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M,
   return launch(fn, grid, in_smem ? xbytes : 0, &p, stream);
 }
 
+// ---------------------------------------------------------------- rotate + select
+
+// The kernel also holds a few words of static shared memory; the dynamic
+// part stays below the per-block limit minus that.
+constexpr int kRotSelSmemCeiling = kGatherSmemCeiling - 1024;
+
+bool rotsel_fits(Elem e, int d) {
+  const int esz = e == Elem::BF16 ? 2 : 4;
+  return d >= 8 && d % 8 == 0 && rslayout(d, esz).total <= (size_t)kRotSelSmemCeiling;
+}
+
+cudaError_t launch_rotsel(Elem e, const RotSelArgs& a, cudaStream_t stream) {
+  if (!rotsel_fits(e, a.d) || a.K < 0 || a.K > a.d) return cudaErrorInvalidValue;
+  DevState* ds = nullptr;
+  cudaError_t err = dev_state(&ds);
+  if (err != cudaSuccess) return err;
+  const int esz = e == Elem::BF16 ? 2 : 4;
+  void* fn = e == Elem::BF16 ? reinterpret_cast<void*>(&rotsel_kernel<__nv_bfloat16>)
+                             : reinterpret_cast<void*>(&rotsel_kernel<float>);
+  // the attribute is a ceiling for every launch of fn
+  err = configure(ds, 10 + (e == Elem::BF16 ? 1 : 0), fn, kRotSelSmemCeiling);
+  if (err != cudaSuccess) return err;
+  const size_t smem = rslayout(a.d, esz).total;
+  int per_sm = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kT, smem);
+  if (err != cudaSuccess) return err;
+  per_sm = std::max(1, std::min(per_sm, 2));
+  RSParams p;
+  p.x = a.x;
+  p.Qt = a.Qt;
+  p.x_rot = a.x_rot;
+  p.idx = a.idx;
+  p.val = a.val;
+  p.ticket = a.ticket;
+  p.d = a.d;
+  p.K = a.K;
+  p.dev_status = a.dev_status;
+  const int grid = std::max(1, std::min(ds->sms * per_sm, a.d));
+  return launch(fn, grid, smem, &p, stream);
+}
+
 namespace {
 
 // Largest number of co-resident clusters of C CTAs for a kernel and shared
@@ -760,7 +1012,8 @@ std::mutex g_occ_mu;
 ClusterOcc g_occ[64][64];
 int g_occ_n[64] = {0};
 
-cudaError_t max_clusters(int dev, void* fn, size_t smem, int C, int* out) {
+cudaError_t max_clusters(int dev, void* fn, size_t smem, int C, int* out,
+                         int ceiling = kGatherSmemCeiling) {
   {
     std::lock_guard<std::mutex> lock(g_occ_mu);
     for (int i = 0; i < g_occ_n[dev]; ++i) {
@@ -773,8 +1026,7 @@ cudaError_t max_clusters(int dev, void* fn, size_t smem, int C, int* out) {
   }
   // the attribute is a ceiling for every launch of fn: set it to the largest
   // size a launch may use, not to the size probed here
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kGatherSmemCeiling);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, ceiling);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, 64, 1);
@@ -799,35 +1051,35 @@ cudaError_t max_clusters(int dev, void* fn, size_t smem, int C, int* out) {
   return cudaSuccess;
 }
 
-void* gather_fn(Elem w, int mode) {
-  if (w == Elem::BF16)
-    return mode == kGatherSelect ? reinterpret_cast<void*>(&gather_kernel<__nv_bfloat16, kModeSelect>)
-                                 : reinterpret_cast<void*>(&gather_kernel<__nv_bfloat16, kModeGather>);
-  return mode == kGatherSelect ? reinterpret_cast<void*>(&gather_kernel<float, kModeSelect>)
-                               : reinterpret_cast<void*>(&gather_kernel<float, kModeGather>);
+template <int C>
+void* gather_fn_c(Elem w) {
+  return w == Elem::BF16 ? reinterpret_cast<void*>(&gather_kernel<__nv_bfloat16, C>)
+                         : reinterpret_cast<void*>(&gather_kernel<float, C>);
 }
+
+void* gather_fn(Elem w, int C) { return C == 8 ? gather_fn_c<8>(w) : gather_fn_c<4>(w); }
 
 }  // namespace
 
-cudaError_t plan_gather(int mode, Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan) {
+cudaError_t plan_gather(Elem w_elem, int d_out, int K, StreamPlan* plan) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   const int cpt = w_elem == Elem::BF16 ? 8 : 4;
-  const int kmode = mode == kGatherSelect ? kModeSelect : kModeGather;
-  void* fn = gather_fn(w_elem, mode);
   StreamPlan best;
+  *plan = best;
   long long best_ctas = -1;
-  for (int C = kC; C == kC; C = 0) {
-    const int key_cap = (d_in + C - 1) / C;
-    // list mode: the rank's share of the kept list; select mode: the kept
-    // entries of the rank's index range
-    const int list_cap = std::max(1, kmode == kModeSelect ? key_cap : (K + C - 1) / C);
+  // Clusters of 8 give the widest column tiles; clusters of 4 pack the SMs
+  // more evenly (the GPU holds fewer 8-CTA clusters than its CTA slots allow).
+  // Take the size that keeps more CTAs streaming at once.
+  for (int C : {8, 4}) {
+    void* fn = gather_fn(w_elem, C);
+    const int list_cap = std::max(1, (K + C - 1) / C);
     // column tile: fill the co-resident clusters, at least 64 columns wide
     // (128 bytes of bf16) and at most one 16-byte vector per thread
     const int wc_max = kT * cpt;
-    const size_t smem_probe = glayout(kmode, key_cap, list_cap, wc_max, cpt).total;
+    const size_t smem_probe = glayout(list_cap, wc_max, cpt).total;
     if (smem_probe > (size_t)kGatherSmemCeiling) continue;
     int clusters = 0;
     e = max_clusters(dev, fn, smem_probe, C, &clusters);
@@ -847,7 +1099,7 @@ cudaError_t plan_gather(int mode, Elem w_elem, int d_in, int d_out, int K, Strea
       best.col_tile = wc;
       best.tpr = wc / cpt;
       best.list_cap = list_cap;
-      best.smem = glayout(kmode, key_cap, list_cap, wc, cpt).total;
+      best.smem = glayout(list_cap, wc, cpt).total;
       best.smem_alloc = smem_probe;
     }
   }
@@ -855,10 +1107,10 @@ cudaError_t plan_gather(int mode, Elem w_elem, int d_in, int d_out, int K, Strea
   return cudaSuccess;
 }
 
-cudaError_t launch_gather(int mode, Elem w_elem, const GatherArgs& a, const StreamPlan& pl,
+cudaError_t launch_gather(Elem w_elem, const GatherArgs& a, const StreamPlan& pl,
                           cudaStream_t stream) {
-  if (!pl.ok) return cudaErrorInvalidValue;
-  void* fn = gather_fn(w_elem, mode);
+  if (!pl.ok || (pl.cluster != 4 && pl.cluster != 8)) return cudaErrorInvalidValue;
+  void* fn = gather_fn(w_elem, pl.cluster);
   GParams p;
   p.W = a.W;
   p.d_out = a.d_out;
@@ -870,8 +1122,6 @@ cudaError_t launch_gather(int mode, Elem w_elem, const GatherArgs& a, const Stre
   p.col_tile = pl.col_tile;
   p.tpr = pl.tpr;
   p.list_cap = pl.list_cap;
-  p.idx_out = a.idx_out;
-  p.val_out = a.val_out;
   p.dev_status = a.dev_status;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.cluster, pl.n_tiles, 1);
@@ -885,6 +1135,106 @@ cudaError_t launch_gather(int mode, Elem w_elem, const GatherArgs& a, const Stre
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  void* args[] = {&p};
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+namespace {
+
+template <int C>
+void* fused_fn_c(Elem w) {
+  return w == Elem::BF16 ? reinterpret_cast<void*>(&fused_kernel<__nv_bfloat16, C>)
+                         : reinterpret_cast<void*>(&fused_kernel<float, C>);
+}
+
+void* fused_fn(Elem w, int C) { return C == 8 ? fused_fn_c<8>(w) : fused_fn_c<4>(w); }
+
+// The fused kernel also holds a few hundred bytes of static shared memory.
+constexpr int kFusedSmemCeiling = kGatherSmemCeiling - 1024;
+
+}  // namespace
+
+cudaError_t plan_fused(Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  StreamPlan best;
+  *plan = best;
+  if (d_in < 8 || d_in % 8 != 0 || K < 0 || K > d_in) return cudaSuccess;
+  const int cpt = w_elem == Elem::BF16 ? 8 : 4;
+  const int esz = w_elem == Elem::BF16 ? 2 : 4;
+  long long best_ctas = -1;
+  for (int C : {8, 4}) {
+    void* fn = fused_fn(w_elem, C);
+    const int range_cap = (d_in + C - 1) / C;
+    const int wc_max = kT * cpt;
+    const size_t smem_probe = flayout(d_in, esz, range_cap, wc_max, cpt).total;
+    if (smem_probe > (size_t)kFusedSmemCeiling) continue;
+    int clusters = 0;
+    e = max_clusters(dev, fn, smem_probe, C, &clusters, kFusedSmemCeiling);
+    if (e != cudaSuccess) return e;
+    if (clusters < 2) continue;
+    const int gather = clusters - 1;  // one cluster holds the selector
+    int wc = (d_out + gather - 1) / gather;
+    wc = std::max(wc, std::min(64, d_out));
+    wc = (wc + cpt - 1) / cpt * cpt;
+    wc = std::min(wc, wc_max);
+    const int n_tiles = (d_out + wc - 1) / wc;
+    if (n_tiles > gather) continue;
+    const long long ctas = (long long)n_tiles * C;
+    if (ctas > best_ctas) {
+      best_ctas = ctas;
+      best.ok = true;
+      best.cluster = C;
+      best.n_tiles = n_tiles;
+      best.col_tile = wc;
+      best.tpr = wc / cpt;
+      best.list_cap = range_cap;
+      best.smem = flayout(d_in, esz, range_cap, wc, cpt).total;
+      best.smem_alloc = smem_probe;
+    }
+  }
+  *plan = best;
+  return cudaSuccess;
+}
+
+cudaError_t launch_fused(Elem w_elem, const FusedArgs& a, const StreamPlan& pl,
+                         cudaStream_t stream) {
+  if (!pl.ok || (pl.cluster != 4 && pl.cluster != 8)) return cudaErrorInvalidValue;
+  void* fn = fused_fn(w_elem, pl.cluster);
+  FParams p;
+  p.x = a.x;
+  p.Qt = a.Qt;
+  p.W = a.W;
+  p.x_rot = a.x_rot;
+  p.idx = a.idx;
+  p.val = a.val;
+  p.y = a.y;
+  p.sync = a.sync;
+  p.d = a.d_in;
+  p.d_out = a.d_out;
+  p.K = a.K;
+  p.col_tile = pl.col_tile;
+  p.tpr = pl.tpr;
+  p.range_cap = pl.list_cap;
+  p.n_tiles = pl.n_tiles;
+  p.dev_status = a.dev_status;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.cluster, pl.n_tiles + 1, 1);
+  cfg.blockDim = dim3(kT, 1, 1);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = pl.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  // every CTA must be resident at once: the gather CTAs wait on the selector
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   void* args[] = {&p};

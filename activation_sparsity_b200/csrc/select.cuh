@@ -7,21 +7,21 @@
 // and +0 / -0 are equal.
 //
 // An fp32 magnitude orders exactly like its bit pattern with the sign bit
-// cleared, read as an unsigned integer (a 31-bit "key").  select_threshold()
-// finds the K-th largest key T and how many keys equal to T are kept (the
-// lowest-indexed ones) with an MSB-first radix select:
+// cleared, read as an unsigned integer (a 31-bit "key"), so the selection is
+// integer work only and bit-exact.
 //
-//   pass 1   histogram of bits 30..20 over all d keys (shared-memory atomics
-//            on two lane-interleaved copies of the histogram, which halves
-//            same-address contention within a warp),
-//   compact  the keys of the boundary bin into a candidate list (when it is
-//            small; otherwise passes 2-3 scan all keys with a prefix test),
-//   pass 2,3 histograms of bits 19..9 and 8..0 over the candidates.
-//
-// Every pass finds its boundary bin with one block-wide scan of the bin
-// counts taken from the top.  kept_chunk_base() then gives each kept entry
-// its rank in ascending index order from one packed (#greater, #equal) scan
-// over contiguous per-thread chunks.
+//   kept_list()         the path every kernel takes (its steps are also used
+//                       on their own): a 4096-bin histogram of bits 30..19
+//                       (counted by the caller as it loads the vector), one
+//                       scan for the boundary bin, the boundary bin's keys
+//                       ranked against each other to find the K-th entry, and
+//                       one scan that places every kept entry in ascending
+//                       index order.
+//   select_threshold()  its fallback when the boundary bin holds too many keys
+//                       (heavy ties): an MSB-first radix select over bits
+//                       30..20, 19..9 and 8..0 that yields the K-th largest
+//                       key T and how many keys equal to T are kept (the
+//                       lowest-indexed ones).
 //
 // All buffers are shared memory passed by pointer; the functions are inlined
 // into their kernels so the compiler keeps shared-memory addressing.
@@ -188,24 +188,6 @@ __device__ __forceinline__ void select_threshold(const uint32_t* bits, int d, in
   *krem_out = krem;
 }
 
-// For the chunk [i0, i1) of this thread: the numbers of keys greater than T
-// and equal to T before i0 (exclusive block scan).  All threads call it.
-template <int NT>
-__device__ __forceinline__ void kept_chunk_base(const uint32_t* bits, int i0, int i1, uint32_t T,
-                                                SelectScratch* s, uint32_t* gt_before,
-                                                uint32_t* eq_before) {
-  uint32_t gt = 0, eq = 0;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t k = bits[i] & kKeyMask;
-    gt += k > T;
-    eq += k == T;
-  }
-  const uint32_t packed = (eq << 16) | gt;  // d < 65536: no carry between halves
-  const uint32_t excl = block_scan_incl<NT>(packed, s->warp_sums) - packed;
-  *gt_before = excl & 0xffffu;
-  *eq_before = excl >> 16;
-}
-
 // Exclusive prefix sum of v over the NT threads with a single barrier.  The
 // caller must place a barrier between two uses of warp_sums.
 template <int NT>
@@ -233,144 +215,222 @@ __device__ __forceinline__ uint32_t block_scan_excl_1s(uint32_t v, uint32_t* war
   return base + inc - v;
 }
 
-// Same result as select_threshold, with fewer barriers: after the pass-1
-// histogram the keys of the boundary bin (at most cand_cap of them) are ranked
-// against each other directly -- larger key first, lower index first among
-// equal keys -- instead of two more radix passes.  Falls back to
-// select_threshold when the boundary bin holds more than cand_cap keys.
-// cand_key / cand_idx: shared arrays of cand_cap entries.  Requires
-// 1 <= K < d; s->hist must be zero on entry (both copies, all 2048 bins) and
-// the first barrier after that must come before this call's counting, which
-// the caller provides.
-template <int NT>
-__device__ __forceinline__ void select_threshold_fast(const uint32_t* bits, int d, int K,
-                                                      SelectScratch* s, uint32_t* cand_key,
-                                                      uint32_t* cand_idx, int cand_cap,
-                                                      uint32_t* T_out, uint32_t* krem_out) {
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  constexpr int NW = NT / 32;
-  uint32_t* h = s->hist + (lane & 1) * kSelBins;
+// ---------------------------------------------------------------- kept list
+//
+// The K kept entries of one vector -- the K largest keys, ties to the lower
+// index -- are exactly those that come no later than the K-th entry (T, I)
+// in the order (key descending, index ascending): every key above T, and the
+// keys equal to T at indices <= I.  Finding (T, I):
+//
+//   1. the caller counts bits 30..19 of every key into kFineBins bins
+//      (s->hist read as one array of kFineBins words);
+//   2. fine_boundary(): one block scan over the bins from the top finds the
+//      bin B holding the K-th largest key, the number of keys above B and in B;
+//   3. kth_entry(): B's keys are listed in ascending index order and each is
+//      ranked against the others; the one ranked krem - 1 is (T, I).  When B
+//      holds more than cand_cap keys (heavy ties), select_threshold() gives T
+//      and one more scan finds I.
+//
+// write_kept() then places the kept entries at their positions.  Steps 3 and
+// write_kept walk warp segments: warp w owns the indices [w*seg, (w+1)*seg),
+// seg a multiple of 32, lane l reads index w*seg + 32*j + l, and ballots
+// order 32 consecutive indices at a time, so shared-memory reads are
+// conflict-free and every store instruction writes one contiguous run.
+constexpr int kFineBins = 4096;
+constexpr int kFineShift = 19;
+static_assert(2 * kSelBins >= kFineBins, "the fine histogram lives in SelectScratch::hist");
 
-  // ---- pass 1: bits 30..20 over all keys
-#pragma unroll 4
-  for (int i = tid; i < d; i += NT) atomicAdd(&h[(bits[i] & kKeyMask) >> 20], 1u);
-  if (tid == 0) {
-    s->pick[2] = 0;
-    s->pick[4] = 0;
-  }
-  __syncthreads();
+struct KthEntry {
+  uint32_t T;  // key of the K-th entry
+  int32_t I;   // its index
+};
 
-  // ---- boundary bin with one barrier: thread t owns ranks [t*per, t*per+per)
-  constexpr int kPer = (kSelBins + NT - 1) / NT;
-  uint32_t cnt[kPer];
-  uint32_t own = 0;
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int k = tid * kPer + j;  // rank from the top
-    const int b = kSelBins - 1 - k;
-    cnt[j] = k < kSelBins ? s->hist[b] + s->hist[kSelBins + b] : 0u;
-    own += cnt[j];
-  }
-  const uint32_t before0 = block_scan_excl_1s<NT>(own, s->warp_sums, nullptr);
-  {
-    uint32_t before = before0;
-    const uint32_t krem = static_cast<uint32_t>(K);
-    if (before < krem && krem <= before + own) {
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        if (before < krem && krem <= before + cnt[j]) {
-          s->pick[0] = static_cast<uint32_t>(kSelBins - 1 - (tid * kPer + j));
-          s->pick[1] = before;
-          s->pick[3] = cnt[j];
-        }
-        before += cnt[j];
-      }
-    }
-  }
-  __syncthreads();
-  const uint32_t b1 = s->pick[0];
-  const uint32_t n1 = s->pick[3];
-  const uint32_t krem1 = static_cast<uint32_t>(K) - s->pick[1];  // to take from bin b1
-  constexpr int kMaxOwn = 4;  // candidates ranked per thread
-  if (n1 > static_cast<uint32_t>(cand_cap) || n1 > static_cast<uint32_t>(kMaxOwn * NT)) {
-    // too many keys share the boundary bin: exact radix passes instead
-    __syncthreads();
-    select_threshold<NT>(bits, d, K, s, cand_key, cand_cap, T_out, krem_out);
-    return;
-  }
-
-  // ---- the boundary bin's keys, with their indices
-  for (int i0 = 0; i0 < d; i0 += NT) {
-    const int i = i0 + tid;
-    const uint32_t k = i < d ? (bits[i] & kKeyMask) : 0u;
-    const bool hit = i < d && (k >> 20) == b1;
-    const uint32_t lanes = __ballot_sync(0xffffffffu, hit);
-    uint32_t base = 0;
-    if (lane == 0 && lanes) base = atomicAdd(&s->pick[2], __popc(lanes));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    if (hit) {
-      const uint32_t slot = base + __popc(lanes & ((1u << lane) - 1u));
-      cand_key[slot] = k;
-      cand_idx[slot] = static_cast<uint32_t>(i);
-    }
-  }
-  __syncthreads();
-
-  // ---- rank every candidate (larger key first, then lower index); the one
-  // ranked krem1-1 holds the K-th largest key overall
-  const int nc = static_cast<int>(n1);
-  uint32_t my_key[kMaxOwn], my_rank[kMaxOwn];
-#pragma unroll
-  for (int q = 0; q < kMaxOwn; ++q) {
-    const int c = tid + q * NT;
-    my_key[q] = 0;
-    my_rank[q] = 0xffffffffu;
-    if (c < nc) {
-      const uint32_t kc = cand_key[c], ic = cand_idx[c];
-      uint32_t rank = 0;
-      for (int j = 0; j < nc; ++j) {
-        const uint32_t kj = cand_key[j];
-        rank += (kj > kc) | ((kj == kc) & (cand_idx[j] < ic));
-      }
-      my_key[q] = kc;
-      my_rank[q] = rank;
-      if (rank == krem1 - 1) s->pick[5] = kc;  // ranks are unique
-    }
-  }
-  __syncthreads();
-  const uint32_t T = s->pick[5];
-  // keys equal to T that are kept = those ranked below krem1
-  uint32_t eq_kept = 0;
-#pragma unroll
-  for (int q = 0; q < kMaxOwn; ++q) eq_kept += (my_rank[q] < krem1) & (my_key[q] == T);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) eq_kept += __shfl_xor_sync(0xffffffffu, eq_kept, o);
-  if (lane == 0 && eq_kept) atomicAdd(&s->pick[4], eq_kept);
-  __syncthreads();
-  *T_out = T;
-  *krem_out = s->pick[4];
-  (void)warp;
-  (void)NW;
+__device__ __forceinline__ bool is_kept(uint32_t key, int i, KthEntry e) {
+  return key > e.T || (key == e.T && i <= e.I);
 }
 
-// kept_chunk_base with a single-barrier scan; also returns the CTA total of
-// kept entries would-be positions are relative to 0.  All threads call it.
+// Step 2.  Requires 1 <= K <= (keys counted).  Ends with a barrier.
 template <int NT>
-__device__ __forceinline__ void kept_chunk_base_1s(const uint32_t* bits, int i0, int i1,
-                                                   uint32_t T, SelectScratch* s,
-                                                   uint32_t* gt_before, uint32_t* eq_before) {
-  uint32_t gt = 0, eq = 0;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t k = bits[i] & kKeyMask;
-    gt += k > T;
-    eq += k == T;
+__device__ __forceinline__ void fine_boundary(SelectScratch* s, int K, uint32_t* B, uint32_t* above,
+                                              uint32_t* nB) {
+  static_assert(kFineBins % (4 * NT) == 0, "each thread owns whole 4-bin vectors");
+  constexpr int kPer = kFineBins / NT;
+  const int tid = threadIdx.x;
+  // thread t owns ranks [t*kPer, t*kPer+kPer) counted from the top
+  uint32_t cnt[kPer];
+  uint32_t own = 0;
+  {
+    const uint4* hv = reinterpret_cast<const uint4*>(s->hist + kFineBins - kPer * (tid + 1));
+#pragma unroll
+    for (int q = 0; q < kPer / 4; ++q) {
+      const uint4 v = hv[q];
+      cnt[kPer - 1 - 4 * q] = v.x;
+      cnt[kPer - 2 - 4 * q] = v.y;
+      cnt[kPer - 3 - 4 * q] = v.z;
+      cnt[kPer - 4 - 4 * q] = v.w;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) own += cnt[j];
   }
-  const uint32_t packed = (eq << 16) | gt;  // d < 65536: no carry between halves
-  const uint32_t excl = block_scan_excl_1s<NT>(packed, s->warp_sums, nullptr);
-  *gt_before = excl & 0xffffu;
-  *eq_before = excl >> 16;
+  uint32_t before = block_scan_excl_1s<NT>(own, s->warp_sums, nullptr);
+  const uint32_t k = static_cast<uint32_t>(K);
+  if (before < k && k <= before + own) {
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (before < k && k <= before + cnt[j]) {
+        s->pick[0] = static_cast<uint32_t>(kFineBins - 1 - (kPer * tid + j));
+        s->pick[1] = before;
+        s->pick[3] = cnt[j];
+      }
+      before += cnt[j];
+    }
+  }
+  __syncthreads();
+  *B = s->pick[0];
+  *above = s->pick[1];
+  *nB = s->pick[3];
+}
+
+// Warp segment [s0, s1) of the indices [0, d) for the calling warp.
+template <int NT>
+__device__ __forceinline__ void warp_segment(int d, int* s0, int* s1) {
+  constexpr int NW = NT / 32;
+  const int seg = ((d + NW - 1) / NW + 31) & ~31;
+  *s0 = min(d, (static_cast<int>(threadIdx.x) >> 5) * seg);
+  *s1 = min(d, *s0 + seg);
+}
+
+// Step 3: the K-th entry of the d keys in `bits`, given step 2's boundary
+// (B, krem = K - above, nB).  Requires 1 <= K < d.  All NT threads call it;
+// it begins and ends with a barrier.  cand_key / cand_idx: cand_cap entries
+// of shared memory, cand_key 16-byte aligned.
+template <int NT>
+__device__ __forceinline__ KthEntry kth_entry(const uint32_t* bits, int d, int K, uint32_t B,
+                                              uint32_t krem, uint32_t nB, SelectScratch* s,
+                                              uint32_t* cand_key, uint32_t* cand_idx,
+                                              int cand_cap) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t below = (1u << lane) - 1u;  // lanes before this one
+  int s0, s1;
+  warp_segment<NT>(d, &s0, &s1);
+  __syncthreads();  // pick[] of step 2 has been read by every thread
+
+  if (nB > static_cast<uint32_t>(cand_cap)) {
+    // ---- heavy ties: exact threshold T by radix passes; then I = the index
+    // of the krem2-th key equal to T in ascending order
+    uint32_t T = 0, krem2 = 0;
+    select_threshold<NT>(bits, d, K, s, cand_key, cand_cap, &T, &krem2);
+    uint32_t n_eq = 0;
+    for (int i = s0 + lane; i < s1; i += 32) n_eq += (bits[i] & kKeyMask) == T;
+    n_eq = __reduce_add_sync(0xffffffffu, n_eq);
+    uint32_t base = __shfl_sync(
+        0xffffffffu, block_scan_excl_1s<NT>(lane == 0 ? n_eq : 0u, s->warp_sums, nullptr), 0);
+    if (base < krem2 && krem2 <= base + n_eq) {  // this warp holds it
+      for (int i0 = s0; i0 < s1; i0 += 32) {
+        const int i = i0 + lane;
+        const bool eq = i < s1 && (bits[i] & kKeyMask) == T;
+        const uint32_t m = __ballot_sync(0xffffffffu, eq);
+        if (eq && base + __popc(m & below) + 1u == krem2) s->pick[6] = static_cast<uint32_t>(i);
+        base += __popc(m);
+        if (base >= krem2) break;
+      }
+    }
+    __syncthreads();
+    return KthEntry{T, static_cast<int32_t>(s->pick[6])};
+  }
+
+  // ---- B's keys, with their indices, in ascending index order
+  uint32_t n_cand = 0;
+  for (int i = s0 + lane; i < s1; i += 32) n_cand += ((bits[i] & kKeyMask) >> kFineShift) == B;
+  n_cand = __reduce_add_sync(0xffffffffu, n_cand);
+  const uint32_t cbase = __shfl_sync(
+      0xffffffffu, block_scan_excl_1s<NT>(lane == 0 ? n_cand : 0u, s->warp_sums, nullptr), 0);
+  if (n_cand != 0u) {  // warp-uniform
+    uint32_t slot = cbase;
+    for (int i0 = s0; i0 < s1; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t k = i < s1 ? (bits[i] & kKeyMask) : 0u;
+      const bool hit = i < s1 && (k >> kFineShift) == B;
+      const uint32_t m = __ballot_sync(0xffffffffu, hit);
+      if (hit) {
+        cand_key[slot + __popc(m & below)] = k;
+        cand_idx[slot + __popc(m & below)] = static_cast<uint32_t>(i);
+      }
+      slot += __popc(m);
+    }
+  }
+  __syncthreads();
+
+  // ---- rank each candidate (larger key first, then lower index, which is
+  // the lower slot); the one ranked krem - 1 is the K-th entry
+  const int nc = static_cast<int>(nB);
+  for (int c = tid; c < nc; c += NT) {
+    const uint32_t kc = cand_key[c];
+    uint32_t r = 0;
+    int j = 0;
+    for (; j + 4 <= nc; j += 4) {
+      const uint4 q = *reinterpret_cast<const uint4*>(cand_key + j);
+      r += (q.x > kc) | ((q.x == kc) & (j < c));
+      r += (q.y > kc) | ((q.y == kc) & (j + 1 < c));
+      r += (q.z > kc) | ((q.z == kc) & (j + 2 < c));
+      r += (q.w > kc) | ((q.w == kc) & (j + 3 < c));
+    }
+    for (; j < nc; ++j) {
+      const uint32_t kj = cand_key[j];
+      r += (kj > kc) | ((kj == kc) & (j < c));
+    }
+    if (r == krem - 1u) {  // ranks are unique
+      s->pick[5] = kc;
+      s->pick[6] = cand_idx[c];
+    }
+  }
+  __syncthreads();
+  return KthEntry{s->pick[5], static_cast<int32_t>(s->pick[6])};
+}
+
+// Kept entries of the d keys in `bits` at positions [p0, p1) of the kept
+// list (ascending index order): rows[pos - p0] = index, vals[pos - p0] = the
+// raw fp32 value.  All NT threads call it; it holds one barrier.
+template <int NT>
+__device__ __forceinline__ void write_kept(const uint32_t* bits, int d, KthEntry e, int p0, int p1,
+                                           int32_t* rows, float* vals, SelectScratch* s) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t below = (1u << lane) - 1u;
+  int s0, s1;
+  warp_segment<NT>(d, &s0, &s1);
+  uint32_t n_kept = 0;
+  for (int i = s0 + lane; i < s1; i += 32) n_kept += is_kept(bits[i] & kKeyMask, i, e);
+  n_kept = __reduce_add_sync(0xffffffffu, n_kept);
+  uint32_t pos = __shfl_sync(
+      0xffffffffu, block_scan_excl_1s<NT>(lane == 0 ? n_kept : 0u, s->warp_sums, nullptr), 0);
+  if (pos < static_cast<uint32_t>(p1) && pos + n_kept > static_cast<uint32_t>(p0)) {
+    for (int i0 = s0; i0 < s1 && pos < static_cast<uint32_t>(p1); i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t u = i < s1 ? bits[i] : 0u;
+      const bool kept = i < s1 && is_kept(u & kKeyMask, i, e);
+      const uint32_t m = __ballot_sync(0xffffffffu, kept);
+      const uint32_t at = pos + __popc(m & below);
+      if (kept && at >= static_cast<uint32_t>(p0) && at < static_cast<uint32_t>(p1)) {
+        rows[at - p0] = i;
+        vals[at - p0] = __uint_as_float(u);
+      }
+      pos += __popc(m);
+    }
+  }
+}
+
+// Positions [p0, p1) of the kept list of the d keys in `bits`, whose bits
+// 30..19 the caller has counted into s->hist (then a barrier).  Requires
+// 1 <= K < d.  All NT threads call it.
+template <int NT>
+__device__ __forceinline__ void kept_list(const uint32_t* bits, int d, int K, SelectScratch* s,
+                                          uint32_t* cand_key, uint32_t* cand_idx, int cand_cap,
+                                          int p0, int p1, int32_t* rows, float* vals) {
+  uint32_t B, above, nB;
+  fine_boundary<NT>(s, K, &B, &above, &nB);
+  const KthEntry e = kth_entry<NT>(bits, d, K, B, static_cast<uint32_t>(K) - above, nB, s, cand_key,
+                                   cand_idx, cand_cap);
+  write_kept<NT>(bits, d, e, p0, p1, rows, vals, s);
 }
 
 }  // namespace larosa

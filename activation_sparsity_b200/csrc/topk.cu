@@ -6,11 +6,12 @@
 // towards the lower index, +0 and -0 are equal, and the kept entries are
 // emitted in ascending index order.
 //
-// The selection itself (select.cuh) is a radix select over the fp32 bit
-// patterns with the sign cleared; one packed block scan then gives every kept
-// entry its position, ascending in the index.  The whole vector (d <= 32768
-// fp32) stays in shared memory; nothing but the input row and the K outputs
-// touches global memory.
+// The selection itself is kept_list() (select.cuh): a 4096-bin histogram of
+// the top 12 bits of every magnitude, counted while the row is loaded, one
+// scan for the boundary bin, the boundary bin's keys ranked directly, and one
+// scan that places every kept entry, ascending in the index.  The whole
+// vector (d <= 32768 fp32) stays in shared memory; nothing but the input row
+// and the K outputs touches global memory.
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
@@ -20,21 +21,28 @@ namespace {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkCand = 2048;
+constexpr int kTopkU = 8;  // 16-byte loads in flight per thread
 
 __global__ void __launch_bounds__(kTopkThreads, 1)
     topk_kernel(const float* __restrict__ x_rot, int d, int K, int32_t* __restrict__ idx,
                 float* __restrict__ val, int* dev_status) {
-  extern __shared__ __align__(16) uint32_t bits[];  // raw fp32 bits of the row
+  // raw fp32 bits of the row, padded with zero keys to a multiple of 4: a
+  // zero key at an index >= d loses every tie, so padding is never kept
+  extern __shared__ __align__(16) uint32_t bits[];
   __shared__ SelectScratch sel;
-  __shared__ uint32_t cand[2 * kTopkCand];  // keys, then indices
+  __shared__ __align__(16) uint32_t cand[kTopkCand];
+  __shared__ uint32_t cand_idx[kTopkCand];
 
   const int tid = threadIdx.x;
   const int m = blockIdx.x;
+  const int d4 = (d + 3) & ~3;
   const float* x = x_rot + (size_t)m * d;
   int32_t* out_i = idx + (size_t)m * K;
   float* out_v = val + (size_t)m * K;
 
-  for (int b = tid; b < 2 * kSelBins; b += kTopkThreads) sel.hist[b] = 0u;
+  for (int b = tid; b < kFineBins; b += kTopkThreads) sel.hist[b] = 0u;
+  for (int i = d + tid; i < d4; i += kTopkThreads) bits[i] = 0u;
+  __syncthreads();
   pdl_wait();
   pdl_launch_dependents();
 
@@ -42,19 +50,37 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   if ((d & 3) == 0 && (reinterpret_cast<uintptr_t>(x) & 15u) == 0) {
     const uint4* x4 = reinterpret_cast<const uint4*>(x);
     uint4* b4 = reinterpret_cast<uint4*>(bits);
-    for (int i = tid; i < (d >> 2); i += kTopkThreads) {
-      const uint4 u = __ldcg(x4 + i);
-      b4[i] = u;
-      nonfinite |= ((u.x & kKeyMask) >= 0x7f800000u) | ((u.y & kKeyMask) >= 0x7f800000u) |
-                   ((u.z & kKeyMask) >= 0x7f800000u) | ((u.w & kKeyMask) >= 0x7f800000u);
+    const int nv = d >> 2;
+    for (int v0 = tid; v0 < nv; v0 += kTopkThreads * kTopkU) {
+      uint4 u[kTopkU];
+#pragma unroll
+      for (int k = 0; k < kTopkU; ++k) {
+        const int v = v0 + k * kTopkThreads;
+        u[k] = v < nv ? __ldcg(x4 + v) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int k = 0; k < kTopkU; ++k) {
+        if (v0 + k * kTopkThreads < nv) {
+          b4[v0 + k * kTopkThreads] = u[k];
+          const uint32_t w[4] = {u[k].x & kKeyMask, u[k].y & kKeyMask, u[k].z & kKeyMask,
+                                 u[k].w & kKeyMask};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            nonfinite |= w[e] >= 0x7f800000u;
+            atomicAdd(&sel.hist[w[e] >> kFineShift], 1u);
+          }
+        }
+      }
     }
   } else {
     for (int i = tid; i < d; i += kTopkThreads) {
       const uint32_t u = __float_as_uint(__ldcg(x + i));
       bits[i] = u;
       nonfinite |= (u & kKeyMask) >= 0x7f800000u;
+      atomicAdd(&sel.hist[(u & kKeyMask) >> kFineShift], 1u);
     }
   }
+  if (tid == 0 && d4 > d) atomicAdd(&sel.hist[0], static_cast<uint32_t>(d4 - d));
   if (__syncthreads_or(nonfinite) && tid == 0) report(dev_status, LAROSA_DEV_NONFINITE);
 
   if (K == 0) return;
@@ -65,43 +91,14 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
     }
     return;
   }
-
-  uint32_t T = 0, krem = 0;
-  select_threshold_fast<kTopkThreads>(bits, d, K, &sel, cand, cand + kTopkCand, kTopkCand, &T,
-                                      &krem);
-
-  // ---- stable compaction over contiguous chunks
-  const int chunk = (d + kTopkThreads - 1) / kTopkThreads;
-  const int i0 = min(d, tid * chunk);
-  const int i1 = min(d, i0 + chunk);
-  uint32_t gt_before = 0, eq_before = 0;
-  kept_chunk_base_1s<kTopkThreads>(bits, i0, i1, T, &sel, &gt_before, &eq_before);
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t u = bits[i];
-    const uint32_t k = u & kKeyMask;
-    if (k > T) {
-      const uint32_t pos = gt_before + min(eq_before, krem);
-      if (pos < static_cast<uint32_t>(K)) {
-        out_i[pos] = i;
-        out_v[pos] = __uint_as_float(u);
-      }
-      ++gt_before;
-    } else if (k == T) {
-      if (eq_before < krem && gt_before + eq_before < static_cast<uint32_t>(K)) {
-        const uint32_t pos = gt_before + eq_before;
-        out_i[pos] = i;
-        out_v[pos] = __uint_as_float(u);
-      }
-      ++eq_before;
-    }
-  }
+  kept_list<kTopkThreads>(bits, d4, K, &sel, cand, cand_idx, kTopkCand, 0, K, out_i, out_v);
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const float* x_rot, int M, int d, int K, int32_t* idx, float* val,
                         int* dev_status, cudaStream_t stream) {
-  const size_t smem = (size_t)d * sizeof(uint32_t);
+  const size_t smem = (size_t)((d + 3) & ~3) * sizeof(uint32_t);
   static int configured[64] = {0};  // per device: dynamic shared memory limit raised
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

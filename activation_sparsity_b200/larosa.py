@@ -39,6 +39,7 @@ _SIGNATURES = {
     "larosa_prepare_weights": ([_vp, _vp, _vp, _i, _i, _i, _vp], _i),
     "larosa_rotate": ([_vp, _vp, _vp, _i, _i, _i, _vp], _i),
     "larosa_topk": ([_vp, _i, _i, _i, _vp, _vp, _vp, _vp], _i),
+    "larosa_rotate_topk": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _sz, _vp, _i, _vp], _i),
     "larosa_sparse_linear": ([_vp, _vp, _i, _i, _vp, _i, _i, _vp, _vp, _sz, _i, _vp, _vp], _i),
     "larosa_rotate_topk_linear": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp, _i, _vp], _i),
     "larosa_dense_linear": ([_vp, _vp, _i, _i, _i, _vp, _i, _vp], _i),
@@ -241,6 +242,34 @@ def larosa_topk(x_rot: torch.Tensor, K: int, idx: torch.Tensor | None = None,
                             _status_ptr(dev_status, x_rot.device), _stream(x_rot.device)),
            "larosa_topk")
     return idx, val
+
+
+def larosa_rotate_topk(x: torch.Tensor, Qt: torch.Tensor, K: int, x_rot: torch.Tensor | None = None,
+                       idx: torch.Tensor | None = None, val: torch.Tensor | None = None, ws=None,
+                       dev_status: torch.Tensor | None = None
+                       ) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """One token: x_rot = x @ Q (Qt = Q^T) and its Top-K by magnitude in one
+    kernel; returns (x_rot fp32 [1, d], idx int32 [1, K] ascending, val fp32 [1, K])."""
+    _need(x, "x")
+    _need(Qt, "Qt", x.dtype)
+    x2 = _as2d(x)
+    M, d = x2.shape
+    if M != 1:
+        raise LarosaError(2, "larosa_rotate_topk: one token only")
+    if x_rot is None:
+        x_rot = torch.empty((1, d), dtype=torch.float32, device=x.device)
+    if idx is None:
+        idx = torch.empty((1, K), dtype=torch.int32, device=x.device)
+    if val is None:
+        val = torch.empty((1, K), dtype=torch.float32, device=x.device)
+    _need(x_rot, "x_rot", torch.float32)
+    _need(idx, "idx", torch.int32)
+    _need(val, "val", torch.float32)
+    p, n = _ws_args(ws, x.device, 1, d, 1, K)
+    _check(_lib.larosa_rotate_topk(_ptr(x2), _ptr(Qt), _ptr(x_rot), _ptr(idx), _ptr(val), d, K, p, n,
+                                   _status_ptr(dev_status, x.device), _dtype_code(x),
+                                   _stream(x.device)), "larosa_rotate_topk")
+    return x_rot, idx, val
 
 
 def larosa_sparse_linear(idx: torch.Tensor, val: torch.Tensor, W_rot: torch.Tensor,

@@ -187,7 +187,7 @@ def measured_peaks() -> tuple[float, str]:
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("onetoken.cu", "common.cuh"):
+    for name in ("onetoken.cu", "common.cuh", "select.cuh"):
         with open(os.path.join(ROOT, "activation_sparsity_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -331,6 +331,11 @@ def bench_larosa(args):
         for g, xr in zip(groups, x_rots):
             L.larosa_rotate(g.x, g.Qt, x_rot=xr)
 
+    def rotate_topk_step():  # the fused path's first kernel: rotation, then Top-K by its last CTA
+        for gi, g in enumerate(groups):
+            L.larosa_rotate_topk(g.x, g.Qt, g.K, x_rot=x_rots[gi], idx=idxs[gi], val=vals[gi], ws=ws,
+                                 dev_status=st)
+
     def topk_step():
         for gi, g in enumerate(groups):
             L.larosa_topk(x_rots[gi], g.K, idx=idxs[gi], val=vals[gi], dev_status=st)
@@ -387,6 +392,7 @@ def bench_larosa(args):
     g_sparse = graph_of(sparse_only_step)
     g_dense = graph_of(dense_step)
     g_rot = graph_of(rotate_step)
+    g_rotsel = graph_of(rotate_topk_step)
     g_topk = graph_of(topk_step)
     g_gather = graph_of(gather_step)
 
@@ -402,25 +408,29 @@ def bench_larosa(args):
     # ---- per-kernel pass: graphs holding one kernel type for the four groups,
     # timed with CUDA events on the launching stream over the same steps
     t_rot, _ = time_graph(g_rot, args.steps, args.warmup)
+    t_rotsel, _ = time_graph(g_rotsel, args.steps, args.warmup)
     t_topk, _ = time_graph(g_topk, args.steps, args.warmup)
     t_gather, _ = time_graph(g_gather, args.steps, args.warmup)
     n_launch = args.steps * len(groups)
     rot_us = t_rot / n_launch * 1e6
+    rotsel_us = t_rotsel / n_launch * 1e6
     topk_us = t_topk / n_launch * 1e6
     gather_us = t_gather / n_launch * 1e6
-    select_gather_us = (t_fused - t_rot) / n_launch * 1e6
     assert L.larosa_check(st, device=device) == 0
 
     rot_bytes = [g.d_in * g.d_in * 2 + g.d_in * 2 + g.d_in * 4 for g in groups]
+    # rotation + Top-K: Q, x, x_rot written and read back once, idx/val written
+    rotsel_bytes = [g.d_in * g.d_in * 2 + g.d_in * 2 + 2 * g.d_in * 4 + g.K * 8 for g in groups]
     lin_bytes = [g.K * g.d_out * 2 + g.K * 8 + g.d_out * 4 for g in groups]
     step_bytes = sum(path_bytes(g, g.K)["total"] for g in groups)
     sparse_bytes = sum(path_bytes(g, g.K, rotate=False)["total"] for g in groups)
     dense_bytes = sum(g.d_in * g.d_out * 2 + g.d_in * 2 + g.d_out * 4 for g in groups)
     peak, peak_kind = measured_peaks()
     rot_gbs = sum(rot_bytes) * args.steps / t_rot / 1e9
+    rotsel_gbs = sum(rotsel_bytes) * args.steps / t_rotsel / 1e9
     lin_gbs = sum(lin_bytes) * args.steps / t_gather / 1e9
-    share_rot = t_rot / t_fused
-    traffic = profiled_traffic("rowdot")
+    share_rotsel = t_rotsel / t_fused
+    traffic = profiled_traffic("rotsel")
 
     # ---- end to end through the public API with host buffers
     x_host = [g.x.cpu().pin_memory() for g in groups]
@@ -464,17 +474,18 @@ def bench_larosa(args):
             "hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
             "hbm_frac": step_bytes / (ms_step * 1e-3) / 1e9 / peak,
             "bytes_per_step": step_bytes,
-            "roofline": {"kernel": "rowdot_kernel (rotation x.Q through Q^T, bf16)", "bound": "hbm",
-                         "achieved": rot_gbs, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": rot_gbs / peak, "traffic": traffic,
-                         "algorithmic_bytes_per_launch": statistics.mean(rot_bytes),
-                         "avg_launch_us": rot_us, "share_of_step": share_rot},
+            "roofline": {"kernel": "rotsel_kernel (rotation x.Q through Q^T, then Top-K by the last CTA; bf16)",
+                         "bound": "hbm", "achieved": rotsel_gbs, "peak": peak, "peak_kind": peak_kind,
+                         "unit": "GB/s", "frac": rotsel_gbs / peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": statistics.mean(rotsel_bytes),
+                         "avg_launch_us": rotsel_us, "share_of_step": share_rotsel},
             "kernels": {
-                "rotate_us_per_launch": rot_us,
-                "select_gather_us_per_launch": select_gather_us,
-                "topk_us_per_launch": topk_us,
+                "rotate_topk_us_per_launch": rotsel_us,
+                "rotate_topk_gbs": rotsel_gbs,
+                "rotate_only_us_per_launch": rot_us, "rotate_only_gbs": rot_gbs,
                 "gather_us_per_launch": gather_us,
                 "gather_gbs": lin_gbs, "gather_frac": lin_gbs / peak,
+                "topk_us_per_launch": topk_us,
                 "groups": [g.name for g in groups],
             },
             "paths": {
@@ -484,6 +495,9 @@ def bench_larosa(args):
                 "dense_tokens_per_s": dense_tps,
                 "dense_hbm_frac": dense_bytes * dense_tps / world / 1e9 / peak,
                 "sparse_only_vs_dense": sparse_tps / dense_tps,
+                # the sparse linear alone on given kept lists (no Q, no Top-K)
+                "gather_only_tokens_per_s": args.steps / t_gather * world,
+                "gather_only_vs_dense": (args.steps / t_gather * world) / dense_tps,
                 "fused_vs_dense": value / dense_tps,
             },
             "e2e": {"value": e2e_value, "unit": UNIT,
@@ -494,7 +508,7 @@ def bench_larosa(args):
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    del g_fused, g_sparse, g_dense, g_rot, g_topk, g_gather
+    del g_fused, g_sparse, g_dense, g_rot, g_rotsel, g_topk, g_gather
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

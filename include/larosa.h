@@ -155,6 +155,24 @@ int larosa_topk(const float *x_rot, int M, int d, int K, int32_t *idx,
                 float *val, int *dev_status, larosa_stream_t stream);
 
 /*
+ * Steps 1 and 2 for one token (La RoSA summary, 方法详解 / 技术框架: rotate the
+ * layer input by its orthogonal matrix, then keep the K largest magnitudes;
+ * abstract: Top-K gives the same sparsity on every token):
+ *   x_rot = x . Q;  (idx, val) = TopK(x_rot, K)  with larosa_topk's rule.
+ * x: [d] of `dtype`, Qt = Q^T: [d x d] of `dtype`, x_rot: [d] fp32,
+ * idx: [K] int32 ascending, val: [K] fp32.  One kernel: every CTA computes a
+ * share of x_rot and the last one to finish selects.  d a multiple of 8;
+ * x, Qt and x_rot 16-byte aligned.  ws: at least
+ * larosa_workspace_bytes(1, d, 1, K) bytes; it holds a counter that is zero
+ * between calls, so calls sharing a workspace must not overlap.  A NaN or
+ * Inf in x_rot sets LAROSA_DEV_NONFINITE.
+ */
+int larosa_rotate_topk(const void *x, const void *Qt, float *x_rot,
+                       int32_t *idx, float *val, int d, int K, void *ws,
+                       size_t ws_bytes, int *dev_status, int dtype,
+                       larosa_stream_t stream);
+
+/*
  * Sparse linear (step 3): y[m][j] = sum_k val[m][k] * W_rot[idx[m][k]][j].
  * idx/val: [M x K] as written by larosa_topk (each row's indices distinct;
  * ascending order is not required for correctness).  W_rot: [d_in x d_out]
@@ -173,8 +191,8 @@ int larosa_sparse_linear(const int32_t *idx, const float *val, int M, int K,
  *   x_rot = x . Q;  (idx, val) = TopK(x_rot, K);  y = sparse(x_rot) . W_rot.
  * x: [M x d_in] of `dtype`; Qt = Q^T: [d_in x d_in]; W_rot: [d_in x d_out] of
  * `dtype` (from larosa_prepare_weights with the same Qt); y: [M x d_out] fp32.
- * For one token this is two kernels: the rotation, then a gather in which
- * every CTA selects the Top-K of x_rot itself.  The intermediate x_rot, idx
+ * For one token this is two kernels: larosa_rotate_topk's kernel, then the
+ * one-token gather of the kept rows.  The intermediate x_rot, idx
  * and val live in the workspace at the offsets larosa_workspace_layout()
  * gives.  d_in a multiple of 8; x, Qt, W_rot and y 16-byte aligned.
  * ws: at least larosa_workspace_bytes(M, d_in, d_out, K) bytes.

@@ -30,7 +30,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for must in ("larosa_prepare_weights", "larosa_rotate", "larosa_topk", "larosa_sparse_linear",
+    for must in ("larosa_prepare_weights", "larosa_rotate", "larosa_topk", "larosa_rotate_topk",
+                 "larosa_sparse_linear",
                  "larosa_rotate_topk_linear", "larosa_dense_linear", "larosa_workspace_bytes",
                  "larosa_check"):
         assert must in names
@@ -93,6 +94,14 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.larosa_rotate_topk_linear(FAKE, FAKE, FAKE, 1, 64, 12, 5, FAKE, FAKE, z, None, BF16, None) == 3
     assert lib.larosa_dense_linear(FAKE, MISALIGNED, 1, 64, 64, FAKE, BF16, None) == 3
     assert lib.larosa_dense_linear(FAKE, FAKE, 1, 60, 64, FAKE, BF16, None) == 3
+    # rotation + Top-K for one token
+    assert lib.larosa_rotate_topk(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 3, FAKE, z, None, 7, None) == 4
+    assert lib.larosa_rotate_topk(None, FAKE, FAKE, FAKE, FAKE, 64, 3, FAKE, z, None, BF16, None) == 1
+    assert lib.larosa_rotate_topk(FAKE, FAKE, FAKE, None, FAKE, 64, 3, FAKE, z, None, BF16, None) == 1
+    assert lib.larosa_rotate_topk(FAKE, FAKE, FAKE, FAKE, FAKE, 64, 65, FAKE, z, None, BF16, None) == 2
+    assert lib.larosa_rotate_topk(FAKE, FAKE, FAKE, FAKE, FAKE, 32776, 3, FAKE, z, None, BF16, None) == 2
+    assert lib.larosa_rotate_topk(FAKE, FAKE, MISALIGNED, FAKE, FAKE, 64, 3, FAKE, z, None, BF16, None) == 3
+    assert lib.larosa_rotate_topk(FAKE, FAKE, FAKE, FAKE, FAKE, 60, 3, FAKE, z, None, BF16, None) == 3
     # in-place counter-rotation is refused
     assert lib.larosa_prepare_weights(FAKE, P(0x20000), P(0x20000), 64, 64, BF16, None) == 1
     # status check needs a status word

@@ -352,3 +352,39 @@ def test_fused_selection_bit_exact_under_identity_rotation(L, kind, d):
         ref = oracle.sparse_linear(want_i.reshape(-1), xd[0, want_i.reshape(-1)], f64(W_rot))
         got, bound = y.reshape(-1), (K + 2) * U * (np.abs(xd[0, want_i.reshape(-1)]) @ np.abs(f64(W_rot)[want_i.reshape(-1)]))
         assert np.all(np.abs(got - ref) <= bound + 1e-37), (kind, d, K)
+
+
+@pytest.mark.parametrize("dtype,d,sparsity", [
+    (torch.float32, 256, 40), (torch.bfloat16, 1024, 40), (torch.bfloat16, 4096, 40),
+    (torch.bfloat16, 11008, 40), (torch.bfloat16, 4096, 0), (torch.bfloat16, 4096, 100),
+    (torch.bfloat16, 8, 50), (torch.bfloat16, 32768, 50),
+])
+def test_rotate_topk(L, dtype, d, sparsity):
+    """Rotation and Top-K in one kernel: x_rot within the summation bound, the
+    kept set a valid Top-K of the exact rotation, and (idx, val) exactly the
+    Top-K of the kernel's own fp32 x_rot."""
+    K = sd.k_for_sparsity(d, sparsity)
+    Q = sd.orthogonal(d, 1001 + d, device="cuda" if d > 4096 else "cpu").to(dtype).cpu()
+    x = sd.activations(1, d, 1002 + d, dtype)
+    st = status()
+    x_rot, idx, val = L.larosa_rotate_topk(x.cuda(), Q.t().contiguous().cuda(), K, dev_status=st)
+    assert L.larosa_check(st) == 0
+    xq, qq = f64(x), f64(Q)
+    x_rot_ref = oracle.rotate(xq, qq)
+    gamma = (d + 2) * U * (np.abs(xq) @ np.abs(qq))
+    got = f64(x_rot)
+    assert np.all(np.abs(got - x_rot_ref) <= gamma + 1e-30)
+    idx = idx.cpu().numpy().astype(np.int64)
+    check_selection(x_rot_ref, gamma, idx, K)
+    # selection rule on the kernel's fp32 values: every kept magnitude is
+    # >= every dropped one, and equal magnitudes favour the lower index
+    mags = np.abs(got[0]).astype(np.float32)
+    kept = np.zeros(d, dtype=bool)
+    kept[idx[0]] = True
+    if 0 < K < d:
+        thr = mags[kept].min()
+        assert np.all(mags[~kept] <= thr)
+        tied_out = np.nonzero(~kept & (mags == thr))[0]
+        tied_in = np.nonzero(kept & (mags == thr))[0]
+        assert len(tied_out) == 0 or tied_in.max() < tied_out.min()
+    assert np.array_equal(f64(val)[0], got[0, idx[0]])
