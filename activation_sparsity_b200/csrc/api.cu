@@ -109,10 +109,12 @@ int make_layout_uncached(int M, int d_in, int d_out, int K, Layout* L) {
   for (int dt = 0; dt < 2; ++dt) {
     const Elem w = dt == 0 ? Elem::F32 : Elem::BF16;
     if (M == 1) {
-      larosa::StreamPlan sl;
+      larosa::StreamPlan sl, sf;
       cudaError_t e = larosa::plan_gather(w, d_out, K, &sl);
+      if (e == cudaSuccess) e = larosa::plan_fused(w, d_in, d_out, K, &sf);
       if (e != cudaSuccess) return cuda_fail(e, "plan gather");
-      if (sl.ok) continue;  // the cluster kernel needs no partials
+      if (sf.ok) partials = std::max(partials, sf.partial_floats);
+      if (sl.ok) continue;  // the list-mode gather needs no partials
     }
     GemvPlan ps;
     cudaError_t e = larosa::plan_gemv(w, Elem::F32, M, d_out, sparse_rows_max(M, d_in, K), &ps);
@@ -391,6 +393,7 @@ int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, 
       f.idx = idx;
       f.val = val;
       f.y = y;
+      f.partials = reinterpret_cast<float*>(at(ws, L.partials));
       f.sync = reinterpret_cast<unsigned*>(at(ws, kOffTickets + kFusedSync * 4));
       f.d_in = d_in;
       f.d_out = d_out;

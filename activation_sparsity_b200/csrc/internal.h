@@ -79,6 +79,7 @@ struct StreamPlan {
   int list_cap = 0;        // kept entries per CTA
   size_t smem = 0;         // dynamic shared memory of a launch
   size_t smem_alloc = 0;   // the size the occupancy was computed for
+  size_t partial_floats = 0;  // workspace floats for per-CTA partials (fused kernel)
 };
 
 struct GatherArgs {
@@ -136,6 +137,7 @@ struct FusedArgs {
   int32_t* idx = nullptr;
   float* val = nullptr;
   float* y = nullptr;
+  float* partials = nullptr;  // plan.partial_floats floats of workspace
   unsigned* sync = nullptr;
   int d_in = 0;
   int d_out = 0;

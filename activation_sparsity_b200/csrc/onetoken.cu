@@ -281,6 +281,47 @@ __device__ __forceinline__ void reduce_tile(cg::cluster_group& cl, int rank, int
   cl.sync();  // no CTA leaves while another may still read its partial
 }
 
+// reduce_tile with the CTAs' partials exchanged through global memory (L2)
+// instead of distributed shared memory: each CTA writes its partial of the
+// tile to gpart[rank * col_tile, ...), one cluster barrier (release/acquire
+// at cluster scope, which covers global memory) makes them visible, and rank
+// r adds its slice over the C partials in rank order.  Used by the
+// cooperative fused kernel; profilers could not launch that kernel while it
+// read peers' shared memory.  Every CTA of the cluster calls it.
+template <typename Tw, int C>
+__device__ __forceinline__ void reduce_tile_l2(cg::cluster_group& cl, int rank, int c0, int wc,
+                                               int col_tile, int tpr,
+                                               const float (&acc)[16 / sizeof(Tw)], float* red,
+                                               float* gpart, float* y) {
+  constexpr int CPT = 16 / sizeof(Tw);
+  const int tid = threadIdx.x;
+  const int ng = kT / tpr;
+  const int g = tid / tpr;
+  const int col = (tid - g * tpr) * CPT;
+  if (g < ng && col < wc) {
+#pragma unroll
+    for (int v = 0; v < CPT; ++v) red[g * col_tile + col + v] = acc[v];
+  }
+  __syncthreads();
+  for (int e = tid; e < wc; e += kT) {
+    float sum = 0.f;
+    for (int gg = 0; gg < ng; ++gg) sum += red[gg * col_tile + e];
+    __stcg(gpart + (size_t)rank * col_tile + e, sum);
+  }
+  cl.sync();
+  const int sl = (wc + C - 1) / C;
+  const int e0 = rank * sl, e1 = min(wc, e0 + sl);
+  for (int e = e0 + tid; e < e1; e += kT) {
+    float v[C];
+#pragma unroll
+    for (int q = 0; q < C; ++q) v[q] = __ldcg(gpart + (size_t)q * col_tile + e);  // all in flight
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < C; ++q) sum += v[q];
+    y[c0 + e] = sum;
+  }
+}
+
 // Streams rows lrows[0, len) of one column tile and adds the cluster's
 // partial sums into y (accumulate_rows, then reduce_tile).
 template <typename Tw, int C>
@@ -540,6 +581,7 @@ struct FParams {
   int32_t* idx;       // [K] kept list (for callers)
   float* val;         // [K]
   float* y;           // [d_out]
+  float* partials;    // [n_tiles x C x col_tile] per-CTA partial sums of each column tile
   unsigned* sync;     // [0, 1] arrivals, [2] boundary / [3] K-th entry published,
                       // [4] mode (0 none kept, 1 Top-K, 2 all kept), [5] B, [6] T, [7] I
   int d;
@@ -553,7 +595,7 @@ struct FParams {
 };
 
 struct FLayout {
-  size_t sel, keys, cand, cand_idx, red, rows, vals, part, total;
+  size_t sel, keys, cand, cand_idx, red, rows, vals, total;
 };
 
 // Region A (offset 0) holds, one after the other in time: the staged x; then
@@ -576,7 +618,6 @@ __host__ __device__ inline FLayout flayout(int d, int elem_bytes, int range_cap,
   o = o > red_bytes ? o : red_bytes;
   L.rows = o;  o = al16(o + (size_t)range_cap * 4);
   L.vals = o;  o = al16(o + (size_t)range_cap * 4);
-  L.part = o;  o = al16(o + (size_t)col_tile * 4);
   L.total = o;
   return L;
 }
@@ -663,7 +704,8 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   const int cta = tile * C + rank;
   const int d = p.d, K = p.K;
 
-  pdl_wait();
+  // launched in ordinary stream order (not as a programmatic dependent), so
+  // everything earlier on the stream is complete and visible here
   if (tid == 0) s_gen = ld_acquire_gpu(p.sync + 3) + 1u;  // this call's number, read before arriving
 
   // ---- 1. rotation rows [r0, r1) of this CTA
@@ -797,7 +839,6 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   uint32_t* rkeys = reinterpret_cast<uint32_t*>(smem_raw);  // region A: the range's keys
   int32_t* lrows = reinterpret_cast<int32_t*>(smem_raw + L.rows);
   float* lvals = reinterpret_cast<float*>(smem_raw + L.vals);
-  float* part = reinterpret_cast<float*>(smem_raw + L.part);
   float* red = reinterpret_cast<float*>(smem_raw + L.red);
   const int i_lo = (int)((long long)d * rank / C);
   const int n_r = (int)((long long)d * (rank + 1) / C) - i_lo;
@@ -867,7 +908,8 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
       lrows, lvals, n_certain, s_warp_sums);
   __syncthreads();  // the list is complete; the range's keys are dead
   accumulate_rows<T>(p.W, p.d_out, c0, wc, p.tpr, lrows, lvals, n_certain, n_certain + n_more, acc);
-  reduce_tile<T, C>(cl, rank, c0, wc, p.col_tile, p.tpr, acc, red, part, p.y);
+  reduce_tile_l2<T, C>(cl, rank, c0, wc, p.col_tile, p.tpr, acc, red,
+                       p.partials + (size_t)tile * C * p.col_tile, p.y);
 }
 
 struct DevState {
@@ -1195,6 +1237,7 @@ cudaError_t plan_fused(Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan
       best.list_cap = range_cap;
       best.smem = flayout(d_in, esz, range_cap, wc, cpt).total;
       best.smem_alloc = smem_probe;
+      best.partial_floats = (size_t)n_tiles * C * wc;
     }
   }
   *plan = best;
@@ -1213,6 +1256,7 @@ cudaError_t launch_fused(Elem w_elem, const FusedArgs& a, const StreamPlan& pl,
   p.idx = a.idx;
   p.val = a.val;
   p.y = a.y;
+  p.partials = a.partials;
   p.sync = a.sync;
   p.d = a.d_in;
   p.d_out = a.d_out;

@@ -1,15 +1,16 @@
 """A small, fixed workload for kernel profilers (ncu): one LLaMA2-7B-shaped
 projection group, batch 1, run a few times through each decode entry point.
 
-    python -m activation_sparsity_b200.profile_case [--group gate_up] [--iters 3]
-                                                    [--sparsity 40]
+    python -m activation_sparsity_b200.profile_case [--group gate_up|all] [--iters 3]
+                                                    [--sparsity 40] [--fused-only]
 
-Each iteration launches, in this order: the fused call (rotation kernel, then
-the select-and-gather kernel), the sparse linear on a fixed kept list (list
-gather kernel) and the dense baseline (rotation kernel on W in nn.Linear
-layout).  The group's tensors take 0.2-0.5 GB of device memory, more than the
-126 MB L2, and ncu flushes the caches before every replayed launch, so DRAM
-counters describe cold-cache launches.  Prints "ok" and exits 0 on success.
+For each group (``all``: q|k|v, o, gate|up, down in that order) each
+iteration launches: the fused call (one fused_kernel), the sparse linear on a
+fixed kept list (gather_kernel) and the dense baseline (rowdot_kernel on W in
+nn.Linear layout); ``--fused-only`` launches only the fused call.  One group
+takes 0.2-0.5 GB of device memory, more than the 126 MB L2, and ncu flushes
+the caches before every replayed launch, so DRAM counters describe
+cold-cache launches.  Prints "ok" and exits 0 on success.
 """
 from __future__ import annotations
 
@@ -33,36 +34,45 @@ GROUPS = {p.name: p for p in sd.llama_layer(4096, 11008, 4096)}
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__,
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--group", choices=sorted(GROUPS), default="gate_up")
+    ap.add_argument("--group", choices=sorted(GROUPS) + ["all"], default="gate_up")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--sparsity", type=float, default=40.0)
+    ap.add_argument("--fused-only", action="store_true")
     a = ap.parse_args(argv)
     if not torch.cuda.is_available():
         raise SystemExit("profile_case: no CUDA device (the library has no CPU path)")
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    p = GROUPS[a.group]
-    base = sd.seed_for(1, 0, 10 * p.q_id)
-    Qt = sd.orthogonal(p.d_in, base + 1, device=dev).to(torch.bfloat16).t().contiguous()
-    W = sd.weights(p.d_in, p.d_out, 0.02, base + 2, torch.bfloat16, device=dev)
-    W_rot = L.larosa_prepare_weights(Qt, W)
-    Wt = W.t().contiguous()
-    del W
-    x = sd.activations(1, p.d_in, base + 3, torch.bfloat16, device=dev)
-    K = sd.k_for_sparsity(p.d_in, a.sparsity)
-    ws = L.Workspace(dev)
+    names = [p.name for p in sd.llama_layer(4096, 11008, 4096)] if a.group == "all" else [a.group]
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    y = torch.empty((1, p.d_out), dtype=torch.float32, device=dev)
-    x_rot = L.larosa_rotate(x, Qt)
-    idx, val = L.larosa_topk(x_rot, K, dev_status=st)
+    ws = L.Workspace(dev)
+    cases = []
+    for name in names:
+        p = GROUPS[name]
+        base = sd.seed_for(1, 0, 10 * p.q_id)
+        Qt = sd.orthogonal(p.d_in, base + 1, device=dev).to(torch.bfloat16).t().contiguous()
+        W = sd.weights(p.d_in, p.d_out, 0.02, base + 2, torch.bfloat16, device=dev)
+        W_rot = L.larosa_prepare_weights(Qt, W)
+        Wt = None if a.fused_only else W.t().contiguous()
+        del W
+        x = sd.activations(1, p.d_in, base + 3, torch.bfloat16, device=dev)
+        K = sd.k_for_sparsity(p.d_in, a.sparsity)
+        y = torch.empty((1, p.d_out), dtype=torch.float32, device=dev)
+        idx = val = None
+        if not a.fused_only:
+            x_rot = L.larosa_rotate(x, Qt)
+            idx, val = L.larosa_topk(x_rot, K, dev_status=st)
+        cases.append((p, Qt, W_rot, Wt, x, K, y, idx, val))
     for _ in range(a.iters):
-        L.larosa_rotate_topk_linear(x, Qt, W_rot, K, y=y, ws=ws, dev_status=st)
-        L.larosa_sparse_linear(idx, val, W_rot, y=y, ws=ws, dev_status=st)
-        L.larosa_dense_linear(x, Wt, y=y)
+        for p, Qt, W_rot, Wt, x, K, y, idx, val in cases:
+            L.larosa_rotate_topk_linear(x, Qt, W_rot, K, y=y, ws=ws, dev_status=st)
+            if not a.fused_only:
+                L.larosa_sparse_linear(idx, val, W_rot, y=y, ws=ws, dev_status=st)
+                L.larosa_dense_linear(x, Wt, y=y)
     torch.cuda.synchronize(dev)
     if L.larosa_check(st, device=dev) != 0:
         raise SystemExit("profile_case: the library reported a device status")
-    print(f"ok: {a.group} d_in={p.d_in} d_out={p.d_out} K={K} iters={a.iters}")
+    print(f"ok: groups {','.join(names)} sparsity {a.sparsity}% iters {a.iters}")
     return 0
 
 

@@ -429,8 +429,9 @@ def bench_larosa(args):
     rot_gbs = sum(rot_bytes) * args.steps / t_rot / 1e9
     rotsel_gbs = sum(rotsel_bytes) * args.steps / t_rotsel / 1e9
     lin_gbs = sum(lin_bytes) * args.steps / t_gather / 1e9
-    share_rotsel = t_rotsel / t_fused
-    traffic = profiled_traffic("rotsel")
+    fused_us = t_fused / n_launch * 1e6  # one fused kernel per group
+    fused_gbs = step_bytes * args.steps / t_fused / 1e9
+    traffic = profiled_traffic("fused")
 
     # ---- end to end through the public API with host buffers
     x_host = [g.x.cpu().pin_memory() for g in groups]
@@ -474,12 +475,14 @@ def bench_larosa(args):
             "hbm_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
             "hbm_frac": step_bytes / (ms_step * 1e-3) / 1e9 / peak,
             "bytes_per_step": step_bytes,
-            "roofline": {"kernel": "rotsel_kernel (rotation x.Q through Q^T, then Top-K by the last CTA; bf16)",
-                         "bound": "hbm", "achieved": rotsel_gbs, "peak": peak, "peak_kind": peak_kind,
-                         "unit": "GB/s", "frac": rotsel_gbs / peak, "traffic": traffic,
-                         "algorithmic_bytes_per_launch": statistics.mean(rotsel_bytes),
-                         "avg_launch_us": rotsel_us, "share_of_step": share_rotsel},
+            "roofline": {"kernel": "fused_kernel (rotation, Top-K and gather of one projection group "
+                                   "in one cooperative launch; bf16)",
+                         "bound": "hbm", "achieved": fused_gbs, "peak": peak, "peak_kind": peak_kind,
+                         "unit": "GB/s", "frac": fused_gbs / peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": step_bytes / len(groups),
+                         "avg_launch_us": fused_us, "share_of_step": 1.0},
             "kernels": {
+                "fused_us_per_launch": fused_us,
                 "rotate_topk_us_per_launch": rotsel_us,
                 "rotate_topk_gbs": rotsel_gbs,
                 "rotate_only_us_per_launch": rot_us, "rotate_only_gbs": rot_gbs,
