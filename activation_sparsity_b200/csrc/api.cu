@@ -26,11 +26,9 @@ namespace {
 
 constexpr int kMaxDout = 65536;
 constexpr size_t kTicketWords = 2048;
-// The last 16 ticket words belong to the one-token kernels: 8 synchronisation
-// words of the fused kernel, and the rotate + select kernel's ticket.  The
-// multi-token split-K tickets use the words below them.
-constexpr size_t kSplitKTicketWords = kTicketWords - 16;
-constexpr size_t kFusedSync = kTicketWords - 16;
+// The last ticket word belongs to the one-token rotate + select kernel; the
+// multi-token split-K tickets use the words below it.
+constexpr size_t kSplitKTicketWords = kTicketWords - 1;
 constexpr size_t kRotSelTicket = kTicketWords - 1;
 constexpr size_t kBitmapWords = LAROSA_MAX_D / 32;
 // Fixed header: words that must be zero before a call and are zero after it.
@@ -59,6 +57,7 @@ bool valid_dtype(int dtype) { return dtype == LAROSA_BF16 || dtype == LAROSA_F32
 bool row_aligned(int n, int dtype) { return (n * elem_size(dtype)) % 16 == 0; }
 
 struct Layout {
+  size_t fused_sync = 0;  // the fused kernel's synchronisation block (M = 1)
   size_t x_rot = 0, idx = 0, val = 0;
   size_t partials = 0;
   size_t coef = 0, urows = 0, ucount = 0;
@@ -128,6 +127,7 @@ int make_layout_uncached(int M, int d_in, int d_out, int K, Layout* L) {
     off = align_up(off + bytes, 256);
     return at;
   };
+  if (M == 1) L->fused_sync = take(larosa::kFusedSyncBytes);
   L->x_rot = take((size_t)M * d_in * 4);
   L->idx = take((size_t)M * K * 4);
   L->val = take((size_t)M * K * 4);
@@ -394,7 +394,7 @@ int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, 
       f.val = val;
       f.y = y;
       f.partials = reinterpret_cast<float*>(at(ws, L.partials));
-      f.sync = reinterpret_cast<unsigned*>(at(ws, kOffTickets + kFusedSync * 4));
+      f.sync = reinterpret_cast<unsigned*>(at(ws, L.fused_sync));
       f.d_in = d_in;
       f.d_out = d_out;
       f.K = K;

@@ -68,8 +68,9 @@ cudaError_t launch_scatter(const int32_t* idx, const float* val, int M, int K, i
 cudaError_t launch_union(unsigned* bitmap, int d_in, int32_t* rows, int* count,
                          cudaStream_t stream);
 
-// Geometry of the one-token gather (see onetoken.cu): one cluster of
-// `cluster` CTAs per column tile of `col_tile` columns.
+// Geometry of the one-token gather (see onetoken.cu): `cluster` CTAs per
+// column tile of `col_tile` columns (a thread-block cluster in the list-mode
+// gather; plain CTAs in the fused kernel).
 struct StreamPlan {
   bool ok = false;
   int cluster = 0;
@@ -127,8 +128,12 @@ cudaError_t launch_rotsel(Elem e, const RotSelArgs& a, cudaStream_t stream);
 
 // One token, one cooperative launch: rotation, Top-K by a selector CTA, and
 // the gather of the kept rows (onetoken.cu, fused_kernel).  `sync` points to
-// 8 words of the caller's workspace, zero before the first call; calls that
-// share them must not overlap on the GPU.
+// kFusedSyncBytes of the caller's workspace, zero before the first call and
+// kept consistent by every call after it; calls that share it must not
+// overlap on the GPU.
+constexpr int kFusedSyncWords = 8;
+constexpr int kFusedMaxTiles = 512;
+constexpr size_t kFusedSyncBytes = (kFusedSyncWords + 2 * kFusedMaxTiles) * 4;
 struct FusedArgs {
   const void* x = nullptr;
   const void* Qt = nullptr;

@@ -281,19 +281,18 @@ __device__ __forceinline__ void reduce_tile(cg::cluster_group& cl, int rank, int
   cl.sync();  // no CTA leaves while another may still read its partial
 }
 
-// reduce_tile with the CTAs' partials exchanged through global memory (L2)
-// instead of distributed shared memory: each CTA writes its partial of the
-// tile to gpart[rank * col_tile, ...), one cluster barrier (release/acquire
-// at cluster scope, which covers global memory) makes them visible, and rank
-// r adds its slice over the C partials in rank order.  Used by the
-// cooperative fused kernel; profilers could not launch that kernel while it
-// read peers' shared memory.  Every CTA of the cluster calls it.
+// Adds the C CTAs' partial sums of one column tile without any CTA waiting
+// for another: each CTA writes its partial of the tile (row groups added in
+// shared memory) to gpart[rank * col_tile, ...) and arrives on the tile's
+// counter; the CTA that arrives last adds the C partials in rank order and
+// writes y[c0, c0 + wc).  The counter must be zero beforehand and is left at
+// C.  All kT threads of the CTA call it.
 template <typename Tw, int C>
-__device__ __forceinline__ void reduce_tile_l2(cg::cluster_group& cl, int rank, int c0, int wc,
-                                               int col_tile, int tpr,
-                                               const float (&acc)[16 / sizeof(Tw)], float* red,
-                                               float* gpart, float* y) {
+__device__ __forceinline__ void reduce_tile_last(int rank, int c0, int wc, int col_tile, int tpr,
+                                                 const float (&acc)[16 / sizeof(Tw)], float* red,
+                                                 float* gpart, unsigned* counter, float* y) {
   constexpr int CPT = 16 / sizeof(Tw);
+  __shared__ unsigned s_last_of_tile;
   const int tid = threadIdx.x;
   const int ng = kT / tpr;
   const int g = tid / tpr;
@@ -303,15 +302,23 @@ __device__ __forceinline__ void reduce_tile_l2(cg::cluster_group& cl, int rank, 
     for (int v = 0; v < CPT; ++v) red[g * col_tile + col + v] = acc[v];
   }
   __syncthreads();
+  bool wrote = false;
   for (int e = tid; e < wc; e += kT) {
     float sum = 0.f;
     for (int gg = 0; gg < ng; ++gg) sum += red[gg * col_tile + e];
     __stcg(gpart + (size_t)rank * col_tile + e, sum);
+    wrote = true;
   }
-  cl.sync();
-  const int sl = (wc + C - 1) / C;
-  const int e0 = rank * sl, e1 = min(wc, e0 + sl);
-  for (int e = e0 + tid; e < e1; e += kT) {
+  if (wrote) __threadfence();  // this thread's part of the partial is visible GPU-wide
+  __syncthreads();
+  if (tid == 0) {
+    const bool last = atomicAdd(counter, 1u) == static_cast<unsigned>(C - 1);
+    if (last) __threadfence();  // the other CTAs' partials are visible after this
+    s_last_of_tile = last;
+  }
+  __syncthreads();
+  if (!s_last_of_tile) return;
+  for (int e = tid; e < wc; e += kT) {
     float v[C];
 #pragma unroll
     for (int q = 0; q < C; ++q) v[q] = __ldcg(gpart + (size_t)q * col_tile + e);  // all in flight
@@ -543,21 +550,20 @@ __global__ void __launch_bounds__(kT, 2) rotsel_kernel(const RSParams p) {
 
 // ================================================================ fused, one token
 //
-// rotate -> select -> gather in one cooperative launch of thread-block
-// clusters: gridDim.y = n_tiles + 1 clusters of C CTAs, all resident at once.
+// rotate -> select -> gather in one cooperative launch of n_tiles * C + 1 CTAs,
+// all resident at once: C CTAs per column tile of the output, and a selector.
 //
 //   1. every CTA computes an equal share of x_rot[j] = x . Q^T[j] (as rowdot
 //      does), stores it and arrives on a ticket;
-//   2. the selector (rank 0 of the last cluster) waits for every arrival,
+//   2. the selector (the last CTA) waits for every arrival,
 //      loads x_rot, finds the histogram bin B that holds the K-th largest
 //      magnitude and publishes it (flag 0); it then ranks B's keys, publishes
 //      the K-th entry (T, I) (flag 1) and writes the kept list for callers;
-//   3. the gather CTAs (clusters 0 .. n_tiles-1, one column tile each; rank r
-//      owns the indices [d*r/C, d*(r+1)/C)) load their range of x_rot while
-//      the selector works, stream the rows that are certainly kept (bin
-//      above B) as soon as B is published, then the few kept rows of bin B
-//      once (T, I) is, and add their partial sums through distributed shared
-//      memory.
+//   3. the gather CTAs (CTA tile*C + r takes column tile `tile` and owns the
+//      indices [d*r/C, d*(r+1)/C)) load their range of x_rot while the
+//      selector works, stream the rows that are certainly kept (bin above B)
+//      as soon as B is published, then the few kept rows of bin B once (T, I)
+//      is; the last CTA of each tile to finish adds the tile's C partial sums.
 //
 // Kept = the K largest |x_rot|, ties to the lower index: key > T, or
 // key == T and index <= I.  Every wait is bounded (kWaitLimitNs) and reports
@@ -571,7 +577,9 @@ __global__ void __launch_bounds__(kT, 2) rotsel_kernel(const RSParams p) {
 // overlap).  Call n counts arrivals in sync[n & 1]; its selector clears the
 // other slot, which call n - 1 has finished with, so no counter is reset
 // while a CTA may still read it.  sync[2] and sync[3] become n when the
-// boundary bin and the K-th entry are published in sync[4..7].
+// boundary bin and the K-th entry are published in sync[4..7].  The column
+// tiles' completion counters follow (two slots of kFusedMaxTiles words, used
+// and cleared the same way).
 
 struct FParams {
   const void* x;      // [d] activation
@@ -583,14 +591,15 @@ struct FParams {
   float* y;           // [d_out]
   float* partials;    // [n_tiles x C x col_tile] per-CTA partial sums of each column tile
   unsigned* sync;     // [0, 1] arrivals, [2] boundary / [3] K-th entry published,
-                      // [4] mode (0 none kept, 1 Top-K, 2 all kept), [5] B, [6] T, [7] I
+                      // [4] mode (0 none kept, 1 Top-K, 2 all kept), [5] B, [6] T, [7] I,
+                      // then 2 x kFusedMaxTiles tile counters
   int d;
   int d_out;
   int K;
   int col_tile;
   int tpr;
   int range_cap;      // ceil(d / C): indices a gather CTA owns
-  int n_tiles;        // gather clusters; cluster n_tiles holds the selector
+  int n_tiles;        // column tiles (C gather CTAs each)
   int* dev_status;
 };
 
@@ -695,13 +704,11 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   __shared__ uint32_t s_gen;
   __shared__ uint32_t s_word[8];
   __shared__ uint32_t s_warp_sums[32];
-  cg::cluster_group cl = cg::this_cluster();
-  const int rank = static_cast<int>(cl.block_rank());
   const FLayout L = flayout(p.d, sizeof(T), p.range_cap, p.col_tile, CPT);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = blockIdx.y;
-  const int G = C * static_cast<int>(gridDim.y);
-  const int cta = tile * C + rank;
+  const int G = static_cast<int>(gridDim.x);  // n_tiles * C gather CTAs + the selector
+  const int cta = blockIdx.x;
+  const int tile = cta / C, rank = cta - tile * C;
   const int d = p.d, K = p.K;
 
   // launched in ordinary stream order (not as a programmatic dependent), so
@@ -760,8 +767,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   if (tid == 0) atomicAdd(ticket, 1u);
   const unsigned target = static_cast<unsigned>(G);
 
-  if (tile == p.n_tiles) {
-    if (rank != 0) return;  // the selector cluster's other CTAs only rotate
+  if (cta == G - 1) {
     // ---- 2. the selector
     SelectScratch* sel = reinterpret_cast<SelectScratch*>(smem_raw + L.sel);
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + L.keys);
@@ -771,7 +777,10 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
     if (tid == 0) {
       const bool ok = wait_ticket(ticket, target);
       if (!ok) report(p.dev_status, LAROSA_DEV_TIMEOUT);
-      p.sync[(gen + 1u) & 1u] = 0u;  // the next call's counter (the previous call's is done)
+      // the next call's counters (the previous call, which used them, is done)
+      p.sync[(gen + 1u) & 1u] = 0u;
+      unsigned* tiles_next = p.sync + kFusedSyncWords + ((gen + 1u) & 1u) * kFusedMaxTiles;
+      for (int t = 0; t < p.n_tiles; ++t) tiles_next[t] = 0u;
       s_word[0] = ok;
     }
     __syncthreads();
@@ -908,8 +917,9 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
       lrows, lvals, n_certain, s_warp_sums);
   __syncthreads();  // the list is complete; the range's keys are dead
   accumulate_rows<T>(p.W, p.d_out, c0, wc, p.tpr, lrows, lvals, n_certain, n_certain + n_more, acc);
-  reduce_tile_l2<T, C>(cl, rank, c0, wc, p.col_tile, p.tpr, acc, red,
-                       p.partials + (size_t)tile * C * p.col_tile, p.y);
+  reduce_tile_last<T, C>(rank, c0, wc, p.col_tile, p.tpr, acc, red,
+                         p.partials + (size_t)tile * C * p.col_tile,
+                         p.sync + kFusedSyncWords + (gen & 1u) * kFusedMaxTiles + tile, p.y);
 }
 
 struct DevState {
@@ -1199,10 +1209,9 @@ constexpr int kFusedSmemCeiling = kGatherSmemCeiling - 1024;
 }  // namespace
 
 cudaError_t plan_fused(Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  DevState* ds = nullptr;
+  cudaError_t e = dev_state(&ds);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   StreamPlan best;
   *plan = best;
   if (d_in < 8 || d_in % 8 != 0 || K < 0 || K > d_in) return cudaSuccess;
@@ -1215,17 +1224,21 @@ cudaError_t plan_fused(Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan
     const int wc_max = kT * cpt;
     const size_t smem_probe = flayout(d_in, esz, range_cap, wc_max, cpt).total;
     if (smem_probe > (size_t)kFusedSmemCeiling) continue;
-    int clusters = 0;
-    e = max_clusters(dev, fn, smem_probe, C, &clusters, kFusedSmemCeiling);
+    // the attribute is a ceiling for every launch of fn
+    e = configure(ds, 12 + (w_elem == Elem::BF16 ? 2 : 0) + (C == 8 ? 1 : 0), fn, kFusedSmemCeiling);
     if (e != cudaSuccess) return e;
-    if (clusters < 2) continue;
-    const int gather = clusters - 1;  // one cluster holds the selector
-    int wc = (d_out + gather - 1) / gather;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kT, smem_probe);
+    if (e != cudaSuccess) return e;
+    const int gather_ctas = ds->sms * per_sm - 1;  // every CTA resident; one selects
+    const int tiles = std::min(gather_ctas / C, kFusedMaxTiles);
+    if (tiles < 1) continue;
+    int wc = (d_out + tiles - 1) / tiles;
     wc = std::max(wc, std::min(64, d_out));
     wc = (wc + cpt - 1) / cpt * cpt;
     wc = std::min(wc, wc_max);
     const int n_tiles = (d_out + wc - 1) / wc;
-    if (n_tiles > gather) continue;
+    if (n_tiles > tiles) continue;
     const long long ctas = (long long)n_tiles * C;
     if (ctas > best_ctas) {
       best_ctas = ctas;
@@ -1246,7 +1259,8 @@ cudaError_t plan_fused(Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan
 
 cudaError_t launch_fused(Elem w_elem, const FusedArgs& a, const StreamPlan& pl,
                          cudaStream_t stream) {
-  if (!pl.ok || (pl.cluster != 4 && pl.cluster != 8)) return cudaErrorInvalidValue;
+  if (!pl.ok || (pl.cluster != 4 && pl.cluster != 8) || pl.n_tiles > kFusedMaxTiles)
+    return cudaErrorInvalidValue;
   void* fn = fused_fn(w_elem, pl.cluster);
   FParams p;
   p.x = a.x;
@@ -1267,20 +1281,16 @@ cudaError_t launch_fused(Elem w_elem, const FusedArgs& a, const StreamPlan& pl,
   p.n_tiles = pl.n_tiles;
   p.dev_status = a.dev_status;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.cluster, pl.n_tiles + 1, 1);
+  cfg.gridDim = dim3(pl.n_tiles * pl.cluster + 1, 1, 1);
   cfg.blockDim = dim3(kT, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = pl.cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
   // every CTA must be resident at once: the gather CTAs wait on the selector
-  attr[1].id = cudaLaunchAttributeCooperative;
-  attr[1].val.cooperative = 1;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 1;
   void* args[] = {&p};
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
