@@ -302,19 +302,15 @@ __device__ __forceinline__ void reduce_tile_last(int rank, int c0, int wc, int c
     for (int v = 0; v < CPT; ++v) red[g * col_tile + col + v] = acc[v];
   }
   __syncthreads();
-  bool wrote = false;
   for (int e = tid; e < wc; e += kT) {
     float sum = 0.f;
     for (int gg = 0; gg < ng; ++gg) sum += red[gg * col_tile + e];
     __stcg(gpart + (size_t)rank * col_tile + e, sum);
-    wrote = true;
   }
-  if (wrote) __threadfence();  // this thread's part of the partial is visible GPU-wide
-  __syncthreads();
+  __syncthreads();  // the CTA's partial is written
   if (tid == 0) {
-    const bool last = atomicAdd(counter, 1u) == static_cast<unsigned>(C - 1);
-    if (last) __threadfence();  // the other CTAs' partials are visible after this
-    s_last_of_tile = last;
+    // release this CTA's partial; the last to arrive also acquires the others'
+    s_last_of_tile = atomic_add_acq_rel_gpu(counter, 1u) == static_cast<unsigned>(C - 1);
   }
   __syncthreads();
   if (!s_last_of_tile) return;
@@ -491,17 +487,13 @@ __global__ void __launch_bounds__(kT, 2) rotsel_kernel(const RSParams p) {
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (lane == 0) __stcg(p.x_rot + row, acc);
     }
-    // lane 0 of each warp stored this CTA's rows: make them visible GPU-wide
-    // before the CTA arrives
-    if (lane == 0) __threadfence();
   }
   SelectScratch* sel = reinterpret_cast<SelectScratch*>(smem_raw + L.sel);
-  __syncthreads();  // the staged x is dead
+  __syncthreads();  // the staged x is dead; this CTA's rows are written
   for (int b = tid; b < kFineBins; b += kT) sel->hist[b] = 0u;  // for the selection, if last
   if (tid == 0) {
-    const bool last = atomicAdd(p.ticket, 1u) == static_cast<unsigned>(G - 1);
-    if (last) __threadfence();  // every CTA's x_rot is visible after this
-    s_last = last;
+    // release this CTA's rows; the last to arrive also acquires every CTA's
+    s_last = atomic_add_acq_rel_gpu(p.ticket, 1u) == static_cast<unsigned>(G - 1);
   }
   __syncthreads();
   if (!s_last) return;
@@ -679,7 +671,7 @@ __device__ __forceinline__ int compact_range(const uint32_t* keys, int n, int i_
   for (int i = s0 + lane; i < s1; i += 32) cnt += pred(keys[i] & kKeyMask, i_lo + i);
   cnt = __reduce_add_sync(0xffffffffu, cnt);
   uint32_t total = 0;
-  uint32_t pos = __shfl_sync(0xffffffffu, block_scan_excl_1s<kT>(lane == 0 ? cnt : 0u, warp_sums, &total), 0);
+  uint32_t pos = warp_base<kT>(cnt, warp_sums, &total);
   if (cnt != 0u) {
     pos += static_cast<uint32_t>(base);
     for (int i0 = s0; i0 < s1; i0 += 32) {
@@ -759,12 +751,11 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (lane == 0) __stcg(p.x_rot + row, acc);
     }
-    if (lane == 0) __threadfence();  // this CTA's rows are visible GPU-wide before it arrives
   }
-  __syncthreads();  // the staged x is dead
+  __syncthreads();  // the staged x is dead; this CTA's rows are written
   const unsigned gen = s_gen;
   unsigned* ticket = p.sync + (gen & 1u);
-  if (tid == 0) atomicAdd(ticket, 1u);
+  if (tid == 0) atomic_add_release_gpu(ticket, 1u);  // publishes the CTA's rows with its arrival
   const unsigned target = static_cast<unsigned>(G);
 
   if (cta == G - 1) {
@@ -820,8 +811,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
     if (tid == 0) {
       p.sync[4] = mode;
       p.sync[5] = B;
-      __threadfence();
-      st_release_gpu(p.sync + 2, gen);
+      st_release_gpu(p.sync + 2, gen);  // orders the two words above before the flag
     }
     KthEntry e{0u, -1};
     if (mode == 1u) e = kth_entry<kT>(keys, d, K, B, static_cast<uint32_t>(K) - above, nB, sel, cand,
@@ -829,7 +819,6 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
     if (tid == 0) {
       p.sync[6] = e.T;
       p.sync[7] = static_cast<uint32_t>(e.I);
-      __threadfence();
       st_release_gpu(p.sync + 3, gen);
     }
     // the kept list for callers, off the gather's path

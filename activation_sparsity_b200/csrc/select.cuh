@@ -215,6 +215,23 @@ __device__ __forceinline__ uint32_t block_scan_excl_1s(uint32_t v, uint32_t* war
   return base + inc - v;
 }
 
+// Exclusive prefix over warps: every lane of warp w passes the same count c_w
+// and receives c_0 + ... + c_{w-1}; *total (if not null) receives the sum
+// over all warps.  One barrier; the caller must place a barrier between two
+// uses of warp_sums.
+template <int NT>
+__device__ __forceinline__ uint32_t warp_base(uint32_t warp_count, uint32_t* warp_sums,
+                                              uint32_t* total) {
+  constexpr int NW = NT / 32;
+  static_assert(NW <= 32, "one lane per warp");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) warp_sums[warp] = warp_count;
+  __syncthreads();
+  const uint32_t c = lane < NW ? warp_sums[lane] : 0u;
+  if (total != nullptr) *total = __reduce_add_sync(0xffffffffu, c);
+  return __reduce_add_sync(0xffffffffu, lane < warp ? c : 0u);
+}
+
 // ---------------------------------------------------------------- kept list
 //
 // The K kept entries of one vector -- the K largest keys, ties to the lower
@@ -323,8 +340,7 @@ __device__ __forceinline__ KthEntry kth_entry(const uint32_t* bits, int d, int K
     uint32_t n_eq = 0;
     for (int i = s0 + lane; i < s1; i += 32) n_eq += (bits[i] & kKeyMask) == T;
     n_eq = __reduce_add_sync(0xffffffffu, n_eq);
-    uint32_t base = __shfl_sync(
-        0xffffffffu, block_scan_excl_1s<NT>(lane == 0 ? n_eq : 0u, s->warp_sums, nullptr), 0);
+    uint32_t base = warp_base<NT>(n_eq, s->warp_sums, nullptr);
     if (base < krem2 && krem2 <= base + n_eq) {  // this warp holds it
       for (int i0 = s0; i0 < s1; i0 += 32) {
         const int i = i0 + lane;
@@ -343,8 +359,7 @@ __device__ __forceinline__ KthEntry kth_entry(const uint32_t* bits, int d, int K
   uint32_t n_cand = 0;
   for (int i = s0 + lane; i < s1; i += 32) n_cand += ((bits[i] & kKeyMask) >> kFineShift) == B;
   n_cand = __reduce_add_sync(0xffffffffu, n_cand);
-  const uint32_t cbase = __shfl_sync(
-      0xffffffffu, block_scan_excl_1s<NT>(lane == 0 ? n_cand : 0u, s->warp_sums, nullptr), 0);
+  const uint32_t cbase = warp_base<NT>(n_cand, s->warp_sums, nullptr);
   if (n_cand != 0u) {  // warp-uniform
     uint32_t slot = cbase;
     for (int i0 = s0; i0 < s1; i0 += 32) {
@@ -401,8 +416,7 @@ __device__ __forceinline__ void write_kept(const uint32_t* bits, int d, KthEntry
   uint32_t n_kept = 0;
   for (int i = s0 + lane; i < s1; i += 32) n_kept += is_kept(bits[i] & kKeyMask, i, e);
   n_kept = __reduce_add_sync(0xffffffffu, n_kept);
-  uint32_t pos = __shfl_sync(
-      0xffffffffu, block_scan_excl_1s<NT>(lane == 0 ? n_kept : 0u, s->warp_sums, nullptr), 0);
+  uint32_t pos = warp_base<NT>(n_kept, s->warp_sums, nullptr);
   if (pos < static_cast<uint32_t>(p1) && pos + n_kept > static_cast<uint32_t>(p0)) {
     for (int i0 = s0; i0 < s1 && pos < static_cast<uint32_t>(p1); i0 += 32) {
       const int i = i0 + lane;
