@@ -133,7 +133,9 @@ cudaError_t launch_rotsel(Elem e, const RotSelArgs& a, cudaStream_t stream);
 // overlap on the GPU.
 constexpr int kFusedSyncWords = 8;
 constexpr int kFusedMaxTiles = 512;
-constexpr size_t kFusedSyncBytes = (kFusedSyncWords + 2 * kFusedMaxTiles) * 4;
+constexpr int kFusedHistBins = 4096;  // bits 30..19 of |x_rot|
+constexpr size_t kFusedSyncBytes =
+    (kFusedSyncWords + 2 * kFusedMaxTiles + 2 * kFusedHistBins) * 4;
 struct FusedArgs {
   const void* x = nullptr;
   const void* Qt = nullptr;

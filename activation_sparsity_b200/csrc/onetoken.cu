@@ -596,7 +596,7 @@ struct FParams {
 };
 
 struct FLayout {
-  size_t sel, keys, cand, cand_idx, red, rows, vals, total;
+  size_t sel, keys, cand, cand_idx, range, red, rows, vals, total;
 };
 
 // Region A (offset 0) holds, one after the other in time: the staged x; then
@@ -611,7 +611,8 @@ __host__ __device__ inline FLayout flayout(int d, int elem_bytes, int range_cap,
   L.cand = o;     o = al16(o + (size_t)kCandCap * 4);
   L.cand_idx = o; o = al16(o + (size_t)kCandCap * 4);
   const size_t x_bytes = al16((size_t)d * elem_bytes);
-  const size_t range_bytes = al16((size_t)range_cap * 4);
+  L.range = L.keys;  // a gather CTA's keys follow its selection scratch
+  const size_t range_bytes = L.range + al16((size_t)range_cap * 4);
   const size_t red_bytes = al16((size_t)(kT / (col_tile / cpt)) * col_tile * 4);
   L.red = 0;
   o = o > x_bytes ? o : x_bytes;
@@ -622,6 +623,8 @@ __host__ __device__ inline FLayout flayout(int d, int elem_bytes, int range_cap,
   L.total = o;
   return L;
 }
+
+constexpr int kRowKeys = 256;  // rotated rows per CTA whose keys are aggregated in shared memory
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
@@ -696,6 +699,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   __shared__ uint32_t s_gen;
   __shared__ uint32_t s_word[8];
   __shared__ uint32_t s_warp_sums[32];
+  __shared__ uint32_t s_rowkey[kRowKeys];  // keys of this CTA's rotated rows
   const FLayout L = flayout(p.d, sizeof(T), p.range_cap, p.col_tile, CPT);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = static_cast<int>(gridDim.x);  // n_tiles * C gather CTAs + the selector
@@ -708,14 +712,14 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   if (tid == 0) s_gen = ld_acquire_gpu(p.sync + 3) + 1u;  // this call's number, read before arriving
 
   // ---- 1. rotation rows [r0, r1) of this CTA
+  const int r0 = (int)((long long)d * cta / G);
+  const int r1 = (int)((long long)d * (cta + 1) / G);
   {
     const int nvx = d * (int)sizeof(T) / 16;
     const uint4* xg = static_cast<const uint4*>(p.x);
     for (int i = tid; i < nvx; i += kT) reinterpret_cast<uint4*>(smem_raw)[i] = __ldg(xg + i);
     __syncthreads();
     const T* xs = reinterpret_cast<const T*>(smem_raw);
-    const int r0 = (int)((long long)d * cta / G);
-    const int r1 = (int)((long long)d * (cta + 1) / G);
     const int nv = d / 8;  // 8-element vectors per row
     constexpr int LD = Vec8<T>::kLoads;
     constexpr int KU = kU / LD;  // the same bytes in flight for both element sizes
@@ -749,12 +753,33 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) __stcg(p.x_rot + row, acc);
+      if (lane == 0) {
+        __stcg(p.x_rot + row, acc);
+        const uint32_t key = __float_as_uint(acc) & kKeyMask;
+        if (row - r0 < kRowKeys)
+          s_rowkey[row - r0] = key;
+        else  // more rows than the buffer holds (very small grids): count directly
+          atomicAdd(p.sync + kFusedSyncWords + 2 * kFusedMaxTiles + (s_gen & 1u) * kFusedHistBins +
+                        (key >> kFineShift), 1u);
+      }
     }
   }
   __syncthreads();  // the staged x is dead; this CTA's rows are written
   const unsigned gen = s_gen;
   unsigned* ticket = p.sync + (gen & 1u);
+  unsigned* ghist = p.sync + kFusedSyncWords + 2 * kFusedMaxTiles + (gen & 1u) * kFusedHistBins;
+  if (warp == 0) {
+    // this CTA's rows into the call's histogram of bits 30..19 of |x_rot|:
+    // equal bins among 32 rows are added once
+    const int nk = min(r1 - r0, kRowKeys);
+    for (int i0 = 0; i0 < nk; i0 += 32) {
+      const bool has = i0 + lane < nk;
+      const uint32_t bin = has ? s_rowkey[i0 + lane] >> kFineShift : 0xffffffffu;
+      const uint32_t same = __match_any_sync(0xffffffffu, bin);
+      if (has && lane == __ffs(same) - 1) atomicAdd(ghist + bin, static_cast<unsigned>(__popc(same)));
+    }
+  }
+  __syncthreads();  // the histogram adds come before the arrival
   if (tid == 0) atomic_add_release_gpu(ticket, 1u);  // publishes the CTA's rows with its arrival
   const unsigned target = static_cast<unsigned>(G);
 
@@ -764,7 +789,12 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
     uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + L.keys);
     uint32_t* cand = reinterpret_cast<uint32_t*>(smem_raw + L.cand);
     uint32_t* cand_idx = reinterpret_cast<uint32_t*>(smem_raw + L.cand_idx);
-    for (int b = tid; b < kFineBins; b += kT) sel->hist[b] = 0u;
+    // the next call's histogram (the previous call, which used it, is done)
+    {
+      uint4* hn = reinterpret_cast<uint4*>(p.sync + kFusedSyncWords + 2 * kFusedMaxTiles +
+                                           ((gen + 1u) & 1u) * kFusedHistBins);
+      for (int i = tid; i < kFusedHistBins / 4; i += kT) hn[i] = make_uint4(0, 0, 0, 0);
+    }
     if (tid == 0) {
       const bool ok = wait_ticket(ticket, target);
       if (!ok) report(p.dev_status, LAROSA_DEV_TIMEOUT);
@@ -777,7 +807,9 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
     __syncthreads();
     const bool ok = s_word[0] != 0u;
     const uint32_t mode = !ok || K <= 0 ? 0u : (K >= d ? 2u : 1u);
-    if (ok) {
+    if (ok) {  // the call's histogram and all d rotated entries -> shared memory
+      const uint4* hsrc = reinterpret_cast<const uint4*>(ghist);
+      for (int i = tid; i < kFusedHistBins / 4; i += kT) reinterpret_cast<uint4*>(sel->hist)[i] = __ldcg(hsrc + i);
       const uint4* src = reinterpret_cast<const uint4*>(p.x_rot);  // d is a multiple of 8
       uint4* dst = reinterpret_cast<uint4*>(keys);
       const int nv = d / 4;
@@ -794,13 +826,8 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
           const int v = v0 + k * kT;
           if (v < nv) {
             dst[v] = u[k];
-            const uint32_t w[4] = {u[k].x & kKeyMask, u[k].y & kKeyMask, u[k].z & kKeyMask,
-                                   u[k].w & kKeyMask};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              nonfinite |= w[e] >= 0x7f800000u;
-              atomicAdd(&sel->hist[w[e] >> kFineShift], 1u);
-            }
+            nonfinite |= (u[k].x & kKeyMask) >= 0x7f800000u || (u[k].y & kKeyMask) >= 0x7f800000u ||
+                         (u[k].z & kKeyMask) >= 0x7f800000u || (u[k].w & kKeyMask) >= 0x7f800000u;
           }
         }
       }
@@ -808,12 +835,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
     }
     uint32_t B = 0, above = 0, nB = 0;
     if (mode == 1u) fine_boundary<kT>(sel, K, &B, &above, &nB);
-    if (tid == 0) {
-      p.sync[4] = mode;
-      p.sync[5] = B;
-      st_release_gpu(p.sync + 2, gen);  // orders the two words above before the flag
-    }
-    KthEntry e{0u, -1};
+    KthEntry e{0xffffffffu, -1};  // after a timeout: no bin-B row is kept
     if (mode == 1u) e = kth_entry<kT>(keys, d, K, B, static_cast<uint32_t>(K) - above, nB, sel, cand,
                                       cand_idx, kCandCap);
     if (tid == 0) {
@@ -834,7 +856,10 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   }
 
   // ---- 3. a gather CTA: rank r owns the indices [i_lo, i_hi)
-  uint32_t* rkeys = reinterpret_cast<uint32_t*>(smem_raw);  // region A: the range's keys
+  // region A: the selection scratch (with the call's histogram), then the
+  // range's keys; later the row-group partials
+  SelectScratch* gsel = reinterpret_cast<SelectScratch*>(smem_raw);
+  uint32_t* rkeys = reinterpret_cast<uint32_t*>(smem_raw + L.range);
   int32_t* lrows = reinterpret_cast<int32_t*>(smem_raw + L.rows);
   float* lvals = reinterpret_cast<float*>(smem_raw + L.vals);
   float* red = reinterpret_cast<float*>(smem_raw + L.red);
@@ -846,14 +871,21 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
 #pragma unroll
   for (int v = 0; v < CPT; ++v) acc[v] = 0.f;
 
-  // every CTA's x_rot is written: load this range while the selector works
+  // every CTA's x_rot is written and counted: load this range and the
+  // histogram while the selector works
   if (tid == 0) {
     const bool ok = wait_ticket(ticket, target);
     if (!ok) report(p.dev_status, LAROSA_DEV_TIMEOUT);
     s_word[0] = ok;
   }
   __syncthreads();
-  if (s_word[0] != 0u) {
+  const bool arrived = s_word[0] != 0u;
+  const uint32_t mode = !arrived || K <= 0 ? 0u : (K >= d ? 2u : 1u);  // 0 keeps nothing
+  if (mode == 1u) {
+    const uint4* hsrc = reinterpret_cast<const uint4*>(ghist);
+    for (int i = tid; i < kFusedHistBins / 4; i += kT) reinterpret_cast<uint4*>(gsel->hist)[i] = __ldcg(hsrc + i);
+  }
+  if (arrived) {
     for (int j0 = tid; j0 < n_r; j0 += kT * kU) {
       uint32_t u[kU];
 #pragma unroll
@@ -866,19 +898,14 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
         if (j0 + k * kT < n_r) rkeys[j0 + k * kT] = u[k];
     }
   }
-  // the boundary bin: rows above it are certainly kept
-  if (tid == 0) {
-    bool got = false;
-    if (s_word[0] != 0u) {
-      got = wait_flag(p.sync + 2, gen);
-      if (!got) report(p.dev_status, LAROSA_DEV_TIMEOUT);
-    }
-    s_word[1] = got ? __ldcg(p.sync + 4) : 0u;  // mode; 0 keeps nothing
-    s_word[2] = got ? __ldcg(p.sync + 5) : 0u;  // B
+  // the boundary bin, from the histogram: rows above it are certainly kept
+  uint32_t B = 0, above = 0, nB = 0;
+  if (mode == 1u) {
+    __syncthreads();  // the histogram is in shared memory
+    fine_boundary<kT>(gsel, K, &B, &above, &nB);
+  } else {
+    __syncthreads();  // the range's keys are in shared memory
   }
-  __syncthreads();
-  const uint32_t mode = s_word[1];
-  const uint32_t B = s_word[2];
   const int n_certain = compact_range(
       rkeys, n_r, i_lo,
       [&](uint32_t k, int) { return mode == 2u || (mode == 1u && (k >> kFineShift) > B); },
@@ -1192,8 +1219,8 @@ void* fused_fn_c(Elem w) {
 
 void* fused_fn(Elem w, int C) { return C == 8 ? fused_fn_c<8>(w) : fused_fn_c<4>(w); }
 
-// The fused kernel also holds a few hundred bytes of static shared memory.
-constexpr int kFusedSmemCeiling = kGatherSmemCeiling - 1024;
+// The fused kernel also holds about 1.2 KB of static shared memory.
+constexpr int kFusedSmemCeiling = kGatherSmemCeiling - 4096;
 
 }  // namespace
 
