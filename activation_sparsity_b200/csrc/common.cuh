@@ -138,6 +138,13 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst_smem, const void* src, u
       : "memory");
 }
 
+// Asks the TMA unit to bring `bytes` of global memory at `src` into L2.  A
+// hint: nothing waits for it and it changes no result.  src 16-byte aligned,
+// bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------- conversions
 
 template <typename T>

@@ -911,6 +911,17 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
       [&](uint32_t k, int) { return mode == 2u || (mode == 1u && (k >> kFineShift) > B); },
       lrows, lvals, 0, s_warp_sums);
   __syncthreads();  // the certain list is in place
+  if (mode == 1u) {
+    // Some rows of bin B are kept too; which ones is known only once the
+    // selector has ranked them.  Their segments of this column tile are few
+    // (about nB / C per CTA): have them brought into L2 now, so that reading
+    // the kept ones later costs an L2 rather than an HBM round trip.
+    const unsigned char* wtile = static_cast<const unsigned char*>(p.W) + (size_t)c0 * sizeof(T);
+    const size_t pitch = (size_t)p.d_out * sizeof(T);
+    for (int j = tid; j < n_r; j += kT)
+      if (((rkeys[j] & kKeyMask) >> kFineShift) == B)
+        bulk_prefetch_l2(wtile + (size_t)(i_lo + j) * pitch, static_cast<uint32_t>(wc * sizeof(T)));
+  }
   accumulate_rows<T>(p.W, p.d_out, c0, wc, p.tpr, lrows, lvals, 0, n_certain, acc);
 
   // the K-th entry: the kept rows of bin B
