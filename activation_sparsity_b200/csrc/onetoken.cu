@@ -596,23 +596,24 @@ struct FParams {
 };
 
 struct FLayout {
-  size_t sel, keys, cand, cand_idx, range, red, rows, vals, total;
+  size_t bins, cand, cand_idx, red, rows, vals, total;
 };
 
+constexpr int kFusedCandCap = 512;  // boundary-bin keys the selector ranks directly
+
 // Region A (offset 0) holds, one after the other in time: the staged x; then
-// in the selector its scratch, all d keys and the boundary candidates, and in
-// a gather CTA its range of keys, then the row-group partials.
+// in the selector the bin numbers of all d entries and the boundary
+// candidates, and in a gather CTA its range of keys, then the row-group
+// partials.
 __host__ __device__ inline FLayout flayout(int d, int elem_bytes, int range_cap, int col_tile,
                                            int cpt) {
   FLayout L{};
   size_t o = 0;
-  L.sel = o;      o = al16(o + sizeof(SelectScratch));
-  L.keys = o;     o = al16(o + (size_t)d * 4);
-  L.cand = o;     o = al16(o + (size_t)kCandCap * 4);
-  L.cand_idx = o; o = al16(o + (size_t)kCandCap * 4);
+  L.bins = o;     o = al16(o + (size_t)d * 2);
+  L.cand = o;     o = al16(o + (size_t)kFusedCandCap * 4);
+  L.cand_idx = o; o = al16(o + (size_t)kFusedCandCap * 4);
   const size_t x_bytes = al16((size_t)d * elem_bytes);
-  L.range = L.keys;  // a gather CTA's keys follow its selection scratch
-  const size_t range_bytes = L.range + al16((size_t)range_cap * 4);
+  const size_t range_bytes = al16((size_t)range_cap * 4);
   const size_t red_bytes = al16((size_t)(kT / (col_tile / cpt)) * col_tile * 4);
   L.red = 0;
   o = o > x_bytes ? o : x_bytes;
@@ -692,6 +693,194 @@ __device__ __forceinline__ int compact_range(const uint32_t* keys, int n, int i_
   return static_cast<int>(total);
 }
 
+// ---- the selector's steps, on 16-bit bin numbers in shared memory and the
+// full keys in global memory (x_rot, read through L2)
+
+// Number of keys >= t among xkeys[0, d); the same value in every thread.
+__device__ __forceinline__ uint32_t count_keys_ge(const uint32_t* xkeys, int d, uint32_t t,
+                                                  uint32_t* warp_sums) {
+  uint32_t c = 0;
+  for (int i0 = threadIdx.x; i0 < d; i0 += kT * kU) {
+    uint32_t u[kU];
+#pragma unroll
+    for (int k = 0; k < kU; ++k) u[k] = i0 + k * kT < d ? __ldcg(xkeys + i0 + k * kT) & kKeyMask : 0u;
+#pragma unroll
+    for (int k = 0; k < kU; ++k) c += (i0 + k * kT < d) && u[k] >= t;
+  }
+  c = __reduce_add_sync(0xffffffffu, c);
+  uint32_t total = 0;
+  (void)warp_base<kT>(c, warp_sums, &total);
+  __syncthreads();  // warp_sums may be reused
+  return total;
+}
+
+// The K-th entry (key T, index I) in the order (key descending, index
+// ascending) of the d keys, given the boundary bin B of the K-th largest
+// key, the krem = K - (keys above B) entries to take from B and the nB keys
+// in B.  bins: bits 30..19 of every key (shared memory); xkeys: the raw
+// fp32 words (global).  Requires 1 <= K < d.  All kT threads call it.
+__device__ __forceinline__ KthEntry fused_kth(const uint32_t* xkeys, const uint16_t* bins, int d, int K,
+                                              uint32_t B, uint32_t krem, uint32_t nB,
+                                              uint32_t* cand_key, uint32_t* cand_idx,
+                                              uint32_t* warp_sums, uint32_t* pick) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t below = (1u << lane) - 1u;
+  int s0, s1;
+  warp_segment<kT>(d, &s0, &s1);
+  __syncthreads();  // pick[] of the boundary has been read by every thread
+
+  if (nB > static_cast<uint32_t>(kFusedCandCap)) {
+    // heavy ties: T = the largest t with count(key >= t) >= K, by bisection
+    // over the 31-bit keys; then I = the index of the krem2-th key equal to
+    // T in ascending order
+    uint32_t lo = 0u, hi = kKeyMask;
+    while (lo < hi) {
+      const uint32_t mid = lo + (hi - lo + 1u) / 2u;
+      if (count_keys_ge(xkeys, d, mid, warp_sums) >= static_cast<uint32_t>(K))
+        lo = mid;
+      else
+        hi = mid - 1u;
+    }
+    const uint32_t T = lo;
+    const uint32_t n_gt = T < kKeyMask ? count_keys_ge(xkeys, d, T + 1u, warp_sums) : 0u;
+    const uint32_t krem2 = static_cast<uint32_t>(K) - n_gt;
+    uint32_t n_eq = 0;
+    for (int i = s0 + lane; i < s1; i += 32) n_eq += (__ldcg(xkeys + i) & kKeyMask) == T;
+    n_eq = __reduce_add_sync(0xffffffffu, n_eq);
+    uint32_t base = warp_base<kT>(n_eq, warp_sums, nullptr);
+    if (base < krem2 && krem2 <= base + n_eq) {  // this warp holds it
+      for (int i0 = s0; i0 < s1; i0 += 32) {
+        const int i = i0 + lane;
+        const bool eq = i < s1 && (__ldcg(xkeys + i) & kKeyMask) == T;
+        const uint32_t m = __ballot_sync(0xffffffffu, eq);
+        if (eq && base + __popc(m & below) + 1u == krem2) pick[1] = static_cast<uint32_t>(i);
+        base += __popc(m);
+        if (base >= krem2) break;
+      }
+    }
+    __syncthreads();
+    return KthEntry{T, static_cast<int32_t>(pick[1])};
+  }
+
+  // B's keys, with their indices, in ascending index order
+  uint32_t n_cand = 0;
+  for (int i = s0 + lane; i < s1; i += 32) n_cand += bins[i] == B;
+  n_cand = __reduce_add_sync(0xffffffffu, n_cand);
+  const uint32_t cbase = warp_base<kT>(n_cand, warp_sums, nullptr);
+  if (n_cand != 0u) {  // warp-uniform; the full keys of 8 x 32 entries in flight at a time
+    uint32_t slot = cbase;
+    for (int i0 = s0; i0 < s1; i0 += 32 * kU) {
+      uint32_t key[kU];
+#pragma unroll
+      for (int k = 0; k < kU; ++k) {
+        const int i = i0 + 32 * k + lane;
+        key[k] = i < s1 && bins[i] == B ? __ldcg(xkeys + i) & kKeyMask : 0u;
+      }
+#pragma unroll
+      for (int k = 0; k < kU; ++k) {
+        const int i = i0 + 32 * k + lane;
+        const bool hit = i < s1 && bins[i] == B;
+        const uint32_t m = __ballot_sync(0xffffffffu, hit);
+        if (hit) {
+          cand_key[slot + __popc(m & below)] = key[k];
+          cand_idx[slot + __popc(m & below)] = static_cast<uint32_t>(i);
+        }
+        slot += __popc(m);
+      }
+    }
+  }
+  __syncthreads();
+  // rank each candidate (larger key first, then lower index, which is the
+  // lower slot); the one ranked krem - 1 is the K-th entry
+  const int nc = static_cast<int>(nB);
+  for (int c = tid; c < nc; c += kT) {
+    const uint32_t kc = cand_key[c];
+    uint32_t r = 0;
+    int j = 0;
+    for (; j + 4 <= nc; j += 4) {
+      const uint4 q = *reinterpret_cast<const uint4*>(cand_key + j);
+      r += (q.x > kc) | ((q.x == kc) & (j < c));
+      r += (q.y > kc) | ((q.y == kc) & (j + 1 < c));
+      r += (q.z > kc) | ((q.z == kc) & (j + 2 < c));
+      r += (q.w > kc) | ((q.w == kc) & (j + 3 < c));
+    }
+    for (; j < nc; ++j) {
+      const uint32_t kj = cand_key[j];
+      r += (kj > kc) | ((kj == kc) & (j < c));
+    }
+    if (r == krem - 1u) {  // ranks are unique
+      pick[0] = kc;
+      pick[1] = cand_idx[c];
+    }
+  }
+  __syncthreads();
+  return KthEntry{pick[0], static_cast<int32_t>(pick[1])};
+}
+
+// The kept list (idx, val: the K entries up to the K-th entry e, ascending
+// index) of the d keys: bin above B, or bin B and up to e.  When B's keys
+// were listed (cand_key, in ascending index order, i.e. in the order the
+// warp segments meet them) they decide; otherwise the full key is read from
+// global memory.  Warp segments and ballots, so stores are contiguous runs;
+// values are read from global memory 8 x 32 at a time.  All kT threads
+// call it.
+__device__ __forceinline__ void fused_export(const uint32_t* xkeys, const uint16_t* bins, int d,
+                                             uint32_t B, KthEntry e, bool listed,
+                                             const uint32_t* cand_key, int32_t* idx, float* val,
+                                             uint32_t* warp_sums) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t below = (1u << lane) - 1u;
+  int s0, s1;
+  warp_segment<kT>(d, &s0, &s1);
+  // bin-B entries of earlier warps (their slots in cand_key)
+  uint32_t n_b = 0;
+  for (int i = s0 + lane; i < s1; i += 32) n_b += bins[i] == B;
+  n_b = __reduce_add_sync(0xffffffffu, n_b);
+  const uint32_t slot = warp_base<kT>(n_b, warp_sums, nullptr);
+  __syncthreads();  // warp_sums is used again below
+  // kept count of this warp's segment
+  uint32_t n_kept = 0;
+  {
+    uint32_t sl = slot;
+    for (int i0 = s0; i0 < s1; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t b = i < s1 ? bins[i] : 0u;
+      const bool inb = i < s1 && b == B;
+      const uint32_t mb = __ballot_sync(0xffffffffu, inb);
+      bool k = i < s1 && b > B;
+      if (inb) {
+        const uint32_t key = listed ? cand_key[sl + __popc(mb & below)] : (__ldcg(xkeys + i) & kKeyMask);
+        k = is_kept(key, i, e);
+      }
+      n_kept += __popc(__ballot_sync(0xffffffffu, k));
+      sl += __popc(mb);
+    }
+  }
+  uint32_t pos = warp_base<kT>(n_kept, warp_sums, nullptr);
+  if (n_kept == 0u) return;
+  for (int i0 = s0; i0 < s1; i0 += 32 * kU) {
+    uint32_t u[kU];
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      const int i = i0 + 32 * k + lane;
+      u[k] = i < s1 ? __ldcg(xkeys + i) : 0u;
+    }
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      const int i = i0 + 32 * k + lane;
+      const uint32_t b = i < s1 ? bins[i] : 0u;
+      bool kept = i < s1 && b > B;
+      if (i < s1 && b == B) kept = is_kept(u[k] & kKeyMask, i, e);
+      const uint32_t m = __ballot_sync(0xffffffffu, kept);
+      if (kept) {
+        idx[pos + __popc(m & below)] = i;
+        val[pos + __popc(m & below)] = __uint_as_float(u[k]);
+      }
+      pos += __popc(m);
+    }
+  }
+}
+
 template <typename T, int C>
 __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   constexpr int CPT = 16 / sizeof(T);
@@ -699,6 +888,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   __shared__ uint32_t s_gen;
   __shared__ uint32_t s_word[8];
   __shared__ uint32_t s_warp_sums[32];
+  __shared__ uint32_t s_pick[4];
   __shared__ uint32_t s_rowkey[kRowKeys];  // keys of this CTA's rotated rows
   const FLayout L = flayout(p.d, sizeof(T), p.range_cap, p.col_tile, CPT);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -784,11 +974,12 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   const unsigned target = static_cast<unsigned>(G);
 
   if (cta == G - 1) {
-    // ---- 2. the selector
-    SelectScratch* sel = reinterpret_cast<SelectScratch*>(smem_raw + L.sel);
-    uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + L.keys);
+    // ---- 2. the selector: 16-bit bin numbers of all d entries in shared
+    // memory, full keys read from x_rot in L2 where a bin does not decide
+    uint16_t* bins = reinterpret_cast<uint16_t*>(smem_raw + L.bins);
     uint32_t* cand = reinterpret_cast<uint32_t*>(smem_raw + L.cand);
     uint32_t* cand_idx = reinterpret_cast<uint32_t*>(smem_raw + L.cand_idx);
+    const uint32_t* xkeys = reinterpret_cast<const uint32_t*>(p.x_rot);
     // the next call's histogram (the previous call, which used it, is done)
     {
       uint4* hn = reinterpret_cast<uint4*>(p.sync + kFusedSyncWords + 2 * kFusedMaxTiles +
@@ -807,11 +998,8 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
     __syncthreads();
     const bool ok = s_word[0] != 0u;
     const uint32_t mode = !ok || K <= 0 ? 0u : (K >= d ? 2u : 1u);
-    if (ok) {  // the call's histogram and all d rotated entries -> shared memory
-      const uint4* hsrc = reinterpret_cast<const uint4*>(ghist);
-      for (int i = tid; i < kFusedHistBins / 4; i += kT) reinterpret_cast<uint4*>(sel->hist)[i] = __ldcg(hsrc + i);
+    if (ok) {
       const uint4* src = reinterpret_cast<const uint4*>(p.x_rot);  // d is a multiple of 8
-      uint4* dst = reinterpret_cast<uint4*>(keys);
       const int nv = d / 4;
       bool nonfinite = false;
       for (int v0 = tid; v0 < nv; v0 += kT * kU) {
@@ -825,19 +1013,25 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
         for (int k = 0; k < kU; ++k) {
           const int v = v0 + k * kT;
           if (v < nv) {
-            dst[v] = u[k];
-            nonfinite |= (u[k].x & kKeyMask) >= 0x7f800000u || (u[k].y & kKeyMask) >= 0x7f800000u ||
-                         (u[k].z & kKeyMask) >= 0x7f800000u || (u[k].w & kKeyMask) >= 0x7f800000u;
+            const uint32_t w[4] = {u[k].x & kKeyMask, u[k].y & kKeyMask, u[k].z & kKeyMask,
+                                   u[k].w & kKeyMask};
+            nonfinite |= w[0] >= 0x7f800000u || w[1] >= 0x7f800000u || w[2] >= 0x7f800000u ||
+                         w[3] >= 0x7f800000u;
+            uint2 packed;
+            packed.x = (w[0] >> kFineShift) | ((w[1] >> kFineShift) << 16);
+            packed.y = (w[2] >> kFineShift) | ((w[3] >> kFineShift) << 16);
+            reinterpret_cast<uint2*>(bins)[v] = packed;
           }
         }
       }
       if (__syncthreads_or(nonfinite) && tid == 0) report(p.dev_status, LAROSA_DEV_NONFINITE);
     }
     uint32_t B = 0, above = 0, nB = 0;
-    if (mode == 1u) fine_boundary<kT>(sel, K, &B, &above, &nB);
+    if (mode == 1u) fine_boundary_at<kT, true>(ghist, K, s_warp_sums, s_pick, &B, &above, &nB);
     KthEntry e{0xffffffffu, -1};  // after a timeout: no bin-B row is kept
-    if (mode == 1u) e = kth_entry<kT>(keys, d, K, B, static_cast<uint32_t>(K) - above, nB, sel, cand,
-                                      cand_idx, kCandCap);
+    if (mode == 1u)
+      e = fused_kth(xkeys, bins, d, K, B, static_cast<uint32_t>(K) - above, nB, cand, cand_idx,
+                    s_warp_sums, s_pick);
     if (tid == 0) {
       p.sync[6] = e.T;
       p.sync[7] = static_cast<uint32_t>(e.I);
@@ -845,21 +1039,21 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
     }
     // the kept list for callers, off the gather's path
     if (mode == 1u) {
-      write_kept<kT>(keys, d, e, 0, K, p.idx, p.val, sel);
+      __syncthreads();  // warp_sums may be reused
+      fused_export(xkeys, bins, d, B, e, nB <= static_cast<uint32_t>(kFusedCandCap), cand, p.idx, p.val,
+                   s_warp_sums);
     } else if (mode == 2u) {
       for (int i = tid; i < d; i += kT) {
         p.idx[i] = i;
-        p.val[i] = __uint_as_float(keys[i]);
+        p.val[i] = __uint_as_float(__ldcg(xkeys + i));
       }
     }
     return;
   }
 
   // ---- 3. a gather CTA: rank r owns the indices [i_lo, i_hi)
-  // region A: the selection scratch (with the call's histogram), then the
-  // range's keys; later the row-group partials
-  SelectScratch* gsel = reinterpret_cast<SelectScratch*>(smem_raw);
-  uint32_t* rkeys = reinterpret_cast<uint32_t*>(smem_raw + L.range);
+  // region A: the range's keys, later the row-group partials
+  uint32_t* rkeys = reinterpret_cast<uint32_t*>(smem_raw);
   int32_t* lrows = reinterpret_cast<int32_t*>(smem_raw + L.rows);
   float* lvals = reinterpret_cast<float*>(smem_raw + L.vals);
   float* red = reinterpret_cast<float*>(smem_raw + L.red);
@@ -871,8 +1065,8 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
 #pragma unroll
   for (int v = 0; v < CPT; ++v) acc[v] = 0.f;
 
-  // every CTA's x_rot is written and counted: load this range and the
-  // histogram while the selector works
+  // every CTA's x_rot is written and counted: load this range while the
+  // selector works
   if (tid == 0) {
     const bool ok = wait_ticket(ticket, target);
     if (!ok) report(p.dev_status, LAROSA_DEV_TIMEOUT);
@@ -881,10 +1075,8 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   __syncthreads();
   const bool arrived = s_word[0] != 0u;
   const uint32_t mode = !arrived || K <= 0 ? 0u : (K >= d ? 2u : 1u);  // 0 keeps nothing
-  if (mode == 1u) {
-    const uint4* hsrc = reinterpret_cast<const uint4*>(ghist);
-    for (int i = tid; i < kFusedHistBins / 4; i += kT) reinterpret_cast<uint4*>(gsel->hist)[i] = __ldcg(hsrc + i);
-  }
+  uint32_t hcnt[kHistShare<kT>];  // this thread's share of the call's histogram
+  if (mode == 1u) hist_share<kT, true>(ghist, hcnt);
   if (arrived) {
     for (int j0 = tid; j0 < n_r; j0 += kT * kU) {
       uint32_t u[kU];
@@ -898,11 +1090,11 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
         if (j0 + k * kT < n_r) rkeys[j0 + k * kT] = u[k];
     }
   }
-  // the boundary bin, from the histogram: rows above it are certainly kept
+  // the boundary bin, from the call's histogram (read from L2): rows above
+  // it are certainly kept
   uint32_t B = 0, above = 0, nB = 0;
   if (mode == 1u) {
-    __syncthreads();  // the histogram is in shared memory
-    fine_boundary<kT>(gsel, K, &B, &above, &nB);
+    boundary_from_share<kT>(hcnt, K, s_warp_sums, s_pick, &B, &above, &nB);
   } else {
     __syncthreads();  // the range's keys are in shared memory
   }

@@ -266,46 +266,78 @@ __device__ __forceinline__ bool is_kept(uint32_t key, int i, KthEntry e) {
   return key > e.T || (key == e.T && i <= e.I);
 }
 
-// Step 2.  Requires 1 <= K <= (keys counted).  Ends with a barrier.
+// Step 2 split in two, so the caller can overlap the histogram read with
+// other loads: hist_share() reads this thread's kFineBins / NT counters,
+// ranks [t*kPer, t*kPer+kPer) counted from the top, from global memory (through
+// L2) or shared memory; boundary_from_share() finds the bin B holding the K-th
+// largest counted key, the keys above B and the keys in B.  Requires
+// 1 <= K <= (keys counted).  warp_sums (32 words) and pick (4 words) are
+// shared memory.  boundary_from_share ends with a barrier.
 template <int NT>
-__device__ __forceinline__ void fine_boundary(SelectScratch* s, int K, uint32_t* B, uint32_t* above,
-                                              uint32_t* nB) {
+constexpr int kHistShare = kFineBins / NT;
+
+template <int NT, bool kGlobal>
+__device__ __forceinline__ void hist_share(const uint32_t* hist, uint32_t (&cnt)[kHistShare<NT>]) {
   static_assert(kFineBins % (4 * NT) == 0, "each thread owns whole 4-bin vectors");
-  constexpr int kPer = kFineBins / NT;
-  const int tid = threadIdx.x;
-  // thread t owns ranks [t*kPer, t*kPer+kPer) counted from the top
-  uint32_t cnt[kPer];
-  uint32_t own = 0;
-  {
-    const uint4* hv = reinterpret_cast<const uint4*>(s->hist + kFineBins - kPer * (tid + 1));
+  constexpr int kPer = kHistShare<NT>;
+  const uint4* hv = reinterpret_cast<const uint4*>(hist + kFineBins - kPer * (threadIdx.x + 1));
 #pragma unroll
-    for (int q = 0; q < kPer / 4; ++q) {
-      const uint4 v = hv[q];
-      cnt[kPer - 1 - 4 * q] = v.x;
-      cnt[kPer - 2 - 4 * q] = v.y;
-      cnt[kPer - 3 - 4 * q] = v.z;
-      cnt[kPer - 4 - 4 * q] = v.w;
+  for (int q = 0; q < kPer / 4; ++q) {
+    uint4 v;
+    if constexpr (kGlobal) {
+      v = __ldcg(hv + q);
+    } else {
+      v = hv[q];
     }
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) own += cnt[j];
+    cnt[kPer - 1 - 4 * q] = v.x;
+    cnt[kPer - 2 - 4 * q] = v.y;
+    cnt[kPer - 3 - 4 * q] = v.z;
+    cnt[kPer - 4 - 4 * q] = v.w;
   }
-  uint32_t before = block_scan_excl_1s<NT>(own, s->warp_sums, nullptr);
+}
+
+template <int NT>
+__device__ __forceinline__ void boundary_from_share(const uint32_t (&cnt)[kHistShare<NT>], int K,
+                                                    uint32_t* warp_sums, uint32_t* pick,
+                                                    uint32_t* B, uint32_t* above, uint32_t* nB) {
+  constexpr int kPer = kHistShare<NT>;
+  const int tid = threadIdx.x;
+  uint32_t own = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) own += cnt[j];
+  uint32_t before = block_scan_excl_1s<NT>(own, warp_sums, nullptr);
   const uint32_t k = static_cast<uint32_t>(K);
   if (before < k && k <= before + own) {
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
       if (before < k && k <= before + cnt[j]) {
-        s->pick[0] = static_cast<uint32_t>(kFineBins - 1 - (kPer * tid + j));
-        s->pick[1] = before;
-        s->pick[3] = cnt[j];
+        pick[0] = static_cast<uint32_t>(kFineBins - 1 - (kPer * tid + j));
+        pick[1] = before;
+        pick[3] = cnt[j];
       }
       before += cnt[j];
     }
   }
   __syncthreads();
-  *B = s->pick[0];
-  *above = s->pick[1];
-  *nB = s->pick[3];
+  *B = pick[0];
+  *above = pick[1];
+  *nB = pick[3];
+}
+
+template <int NT, bool kGlobal>
+__device__ __forceinline__ void fine_boundary_at(const uint32_t* hist, int K, uint32_t* warp_sums,
+                                                 uint32_t* pick, uint32_t* B, uint32_t* above,
+                                                 uint32_t* nB) {
+  uint32_t cnt[kHistShare<NT>];
+  hist_share<NT, kGlobal>(hist, cnt);
+  boundary_from_share<NT>(cnt, K, warp_sums, pick, B, above, nB);
+}
+
+// Step 2 on the histogram in s->hist (shared memory).
+template <int NT>
+__device__ __forceinline__ void fine_boundary(SelectScratch* s, int K, uint32_t* B, uint32_t* above,
+                                              uint32_t* nB) {
+  fine_boundary_at<NT, false>(s->hist, K, s->warp_sums, s->pick, B, above, nB);
 }
 
 // Warp segment [s0, s1) of the indices [0, d) for the calling warp.
