@@ -546,32 +546,37 @@ __global__ void __launch_bounds__(kT, 2) rotsel_kernel(const RSParams p) {
 // all resident at once: C CTAs per column tile of the output, and a selector.
 //
 //   1. every CTA computes an equal share of x_rot[j] = x . Q^T[j] (as rowdot
-//      does), stores it and arrives on a ticket;
-//   2. the selector (the last CTA) waits for every arrival,
-//      loads x_rot, finds the histogram bin B that holds the K-th largest
-//      magnitude and publishes it (flag 0); it then ranks B's keys, publishes
-//      the K-th entry (T, I) (flag 1) and writes the kept list for callers;
+//      does), stores it, adds the keys (bits 30..19 of |x_rot|) to the call's
+//      histogram and arrives on a ticket;
+//   2. the selector (the last CTA) waits for every arrival, finds from the
+//      histogram the bin B that holds the K-th largest magnitude, lists B's
+//      keys in one pass over x_rot and ranks them in shared memory: the one
+//      ranked K - (keys above B) - 1 is the K-th entry (T, I), which it
+//      publishes.  Its L2 reads are made right after the arrivals, before the
+//      gather CTAs stream weight rows, while an L2 round trip is still short.
+//      It then writes the kept list for callers and clears the next call's
+//      counters;
 //   3. the gather CTAs (CTA tile*C + r takes column tile `tile` and owns the
-//      indices [d*r/C, d*(r+1)/C)) load their range of x_rot while the
-//      selector works, stream the rows that are certainly kept (bin above B)
-//      as soon as B is published, then the few kept rows of bin B once (T, I)
-//      is; the last CTA of each tile to finish adds the tile's C partial sums.
+//      indices [d*r/C, d*(r+1)/C)) read the histogram and their range of
+//      x_rot, find B themselves and stream the rows that are certainly kept
+//      (bin above B), then the few kept rows of bin B once (T, I) is
+//      published; the last CTA of each tile to finish adds the tile's C
+//      partial sums.
 //
 // Kept = the K largest |x_rot|, ties to the lower index: key > T, or
 // key == T and index <= I.  Every wait is bounded (kWaitLimitNs) and reports
 // LAROSA_DEV_TIMEOUT; the cooperative launch guarantees that every CTA is
 // resident, so no CTA waits on one that cannot run.
 //
-// Synchronisation words (sync[8], in the caller's workspace; all zero
-// initially): sync[3] is the number of the last call whose K-th entry was
-// published.  Every CTA reads it before it arrives, so all CTAs of a call
-// agree on its number n = sync[3] + 1 (calls that share the words must not
-// overlap).  Call n counts arrivals in sync[n & 1]; its selector clears the
-// other slot, which call n - 1 has finished with, so no counter is reset
-// while a CTA may still read it.  sync[2] and sync[3] become n when the
-// boundary bin and the K-th entry are published in sync[4..7].  The column
-// tiles' completion counters follow (two slots of kFusedMaxTiles words, used
-// and cleared the same way).
+// Synchronisation words (in the caller's workspace; all zero initially):
+// sync[3] is the number of the last call whose K-th entry was published.
+// Every CTA reads it before it arrives, so all CTAs of a call agree on its
+// number n = sync[3] + 1 (calls that share the words must not overlap).
+// Call n counts arrivals in sync[n & 1], its histogram in slot n & 1 of
+// 2 x kFusedHistBins counters and its tiles' completions in slot n & 1 of
+// 2 x kFusedMaxTiles counters; its selector clears the other slots, which
+// call n - 1 has finished with, so no counter is reset while a CTA may still
+// read it.  sync[3] becomes n when the K-th entry is published in sync[6..7].
 
 struct FParams {
   const void* x;      // [d] activation
@@ -582,9 +587,8 @@ struct FParams {
   float* val;         // [K]
   float* y;           // [d_out]
   float* partials;    // [n_tiles x C x col_tile] per-CTA partial sums of each column tile
-  unsigned* sync;     // [0, 1] arrivals, [2] boundary / [3] K-th entry published,
-                      // [4] mode (0 none kept, 1 Top-K, 2 all kept), [5] B, [6] T, [7] I,
-                      // then 2 x kFusedMaxTiles tile counters
+  unsigned* sync;     // [0, 1] arrivals, [3] K-th entry published, [6] T, [7] I; then
+                      // 2 x kFusedMaxTiles tile counters, 2 x kFusedHistBins histogram bins
   int d;
   int d_out;
   int K;
@@ -714,104 +718,154 @@ __device__ __forceinline__ uint32_t count_keys_ge(const uint32_t* xkeys, int d, 
   return total;
 }
 
-// The K-th entry (key T, index I) in the order (key descending, index
-// ascending) of the d keys, given the boundary bin B of the K-th largest
-// key, the krem = K - (keys above B) entries to take from B and the nB keys
-// in B.  bins: bits 30..19 of every key (shared memory); xkeys: the raw
-// fp32 words (global).  Requires 1 <= K < d.  All kT threads call it.
-__device__ __forceinline__ KthEntry fused_kth(const uint32_t* xkeys, const uint16_t* bins, int d, int K,
-                                              uint32_t B, uint32_t krem, uint32_t nB,
-                                              uint32_t* cand_key, uint32_t* cand_idx,
-                                              uint32_t* warp_sums, uint32_t* pick) {
-  const int tid = threadIdx.x, lane = tid & 31;
+// The K-th entry when the boundary bin holds more than kFusedCandCap keys
+// (heavy ties): T = the largest t with count(key >= t) >= K, by bisection
+// over the 31-bit keys, then I = the index of the (K - count(key > T))-th
+// key equal to T in ascending index order.  Requires 1 <= K < d.  All kT
+// threads call it.
+__device__ __noinline__ KthEntry kth_by_bisection(const uint32_t* xkeys, int d, int K,
+                                                  uint32_t* warp_sums, uint32_t* pick) {
+  const int lane = threadIdx.x & 31;
   const uint32_t below = (1u << lane) - 1u;
   int s0, s1;
   warp_segment<kT>(d, &s0, &s1);
-  __syncthreads();  // pick[] of the boundary has been read by every thread
-
-  if (nB > static_cast<uint32_t>(kFusedCandCap)) {
-    // heavy ties: T = the largest t with count(key >= t) >= K, by bisection
-    // over the 31-bit keys; then I = the index of the krem2-th key equal to
-    // T in ascending order
-    uint32_t lo = 0u, hi = kKeyMask;
-    while (lo < hi) {
-      const uint32_t mid = lo + (hi - lo + 1u) / 2u;
-      if (count_keys_ge(xkeys, d, mid, warp_sums) >= static_cast<uint32_t>(K))
-        lo = mid;
-      else
-        hi = mid - 1u;
-    }
-    const uint32_t T = lo;
-    const uint32_t n_gt = T < kKeyMask ? count_keys_ge(xkeys, d, T + 1u, warp_sums) : 0u;
-    const uint32_t krem2 = static_cast<uint32_t>(K) - n_gt;
-    uint32_t n_eq = 0;
-    for (int i = s0 + lane; i < s1; i += 32) n_eq += (__ldcg(xkeys + i) & kKeyMask) == T;
-    n_eq = __reduce_add_sync(0xffffffffu, n_eq);
-    uint32_t base = warp_base<kT>(n_eq, warp_sums, nullptr);
-    if (base < krem2 && krem2 <= base + n_eq) {  // this warp holds it
-      for (int i0 = s0; i0 < s1; i0 += 32) {
-        const int i = i0 + lane;
-        const bool eq = i < s1 && (__ldcg(xkeys + i) & kKeyMask) == T;
-        const uint32_t m = __ballot_sync(0xffffffffu, eq);
-        if (eq && base + __popc(m & below) + 1u == krem2) pick[1] = static_cast<uint32_t>(i);
-        base += __popc(m);
-        if (base >= krem2) break;
-      }
-    }
-    __syncthreads();
-    return KthEntry{T, static_cast<int32_t>(pick[1])};
+  uint32_t lo = 0u, hi = kKeyMask;
+  while (lo < hi) {
+    const uint32_t mid = lo + (hi - lo + 1u) / 2u;
+    if (count_keys_ge(xkeys, d, mid, warp_sums) >= static_cast<uint32_t>(K))
+      lo = mid;
+    else
+      hi = mid - 1u;
   }
-
-  // B's keys, with their indices, in ascending index order
-  uint32_t n_cand = 0;
-  for (int i = s0 + lane; i < s1; i += 32) n_cand += bins[i] == B;
-  n_cand = __reduce_add_sync(0xffffffffu, n_cand);
-  const uint32_t cbase = warp_base<kT>(n_cand, warp_sums, nullptr);
-  if (n_cand != 0u) {  // warp-uniform; the full keys of 8 x 32 entries in flight at a time
-    uint32_t slot = cbase;
-    for (int i0 = s0; i0 < s1; i0 += 32 * kU) {
-      uint32_t key[kU];
-#pragma unroll
-      for (int k = 0; k < kU; ++k) {
-        const int i = i0 + 32 * k + lane;
-        key[k] = i < s1 && bins[i] == B ? __ldcg(xkeys + i) & kKeyMask : 0u;
-      }
-#pragma unroll
-      for (int k = 0; k < kU; ++k) {
-        const int i = i0 + 32 * k + lane;
-        const bool hit = i < s1 && bins[i] == B;
-        const uint32_t m = __ballot_sync(0xffffffffu, hit);
-        if (hit) {
-          cand_key[slot + __popc(m & below)] = key[k];
-          cand_idx[slot + __popc(m & below)] = static_cast<uint32_t>(i);
-        }
-        slot += __popc(m);
-      }
+  const uint32_t T = lo;
+  const uint32_t n_gt = T < kKeyMask ? count_keys_ge(xkeys, d, T + 1u, warp_sums) : 0u;
+  const uint32_t krem = static_cast<uint32_t>(K) - n_gt;
+  uint32_t n_eq = 0;
+  for (int i = s0 + lane; i < s1; i += 32) n_eq += (__ldcg(xkeys + i) & kKeyMask) == T;
+  n_eq = __reduce_add_sync(0xffffffffu, n_eq);
+  uint32_t base = warp_base<kT>(n_eq, warp_sums, nullptr);
+  if (base < krem && krem <= base + n_eq) {  // this warp holds it
+    for (int i0 = s0; i0 < s1; i0 += 32) {
+      const int i = i0 + lane;
+      const bool eq = i < s1 && (__ldcg(xkeys + i) & kKeyMask) == T;
+      const uint32_t m = __ballot_sync(0xffffffffu, eq);
+      if (eq && base + __popc(m & below) + 1u == krem) pick[1] = static_cast<uint32_t>(i);
+      base += __popc(m);
+      if (base >= krem) break;
     }
   }
   __syncthreads();
-  // rank each candidate (larger key first, then lower index, which is the
-  // lower slot); the one ranked krem - 1 is the K-th entry
-  const int nc = static_cast<int>(nB);
-  for (int c = tid; c < nc; c += kT) {
-    const uint32_t kc = cand_key[c];
-    uint32_t r = 0;
-    int j = 0;
-    for (; j + 4 <= nc; j += 4) {
-      const uint4 q = *reinterpret_cast<const uint4*>(cand_key + j);
-      r += (q.x > kc) | ((q.x == kc) & (j < c));
-      r += (q.y > kc) | ((q.y == kc) & (j + 1 < c));
-      r += (q.z > kc) | ((q.z == kc) & (j + 2 < c));
-      r += (q.w > kc) | ((q.w == kc) & (j + 3 < c));
+  return KthEntry{T, static_cast<int32_t>(pick[1])};
+}
+
+constexpr int kPre = 6;  // 16-byte vectors of x_rot per thread read with the histogram
+
+// The selector's pass over x_rot once the boundary bin B is known: writes
+// the bin number (bits 30..19) of every key to bins (shared memory), lists
+// B's keys with their indices in cand_key / cand_idx (in no particular
+// order: each warp reserves its slots with one atomic), ranks each against
+// the others (larger key first, then lower index) and returns the one
+// ranked krem - 1, i.e. the K-th entry (T, I).  Requires
+// 1 <= krem <= nB <= kFusedCandCap.  pre[k] holds the 16-byte vector
+// tid + k * kT of xkeys, read ahead by the caller.  The kFusedCandCap slots
+// of cand_key / cand_idx (16-byte aligned) hold key 0 and index 0xffffffff
+// on entry; cnt: a word of shared memory, zero on entry.  Sets *nonfinite
+// in a thread that met a NaN or Inf.  All kT threads call it; it begins
+// after and ends with a barrier.
+__device__ __forceinline__ KthEntry select_kth(const uint32_t* xkeys, int d, uint32_t B,
+                                               uint32_t krem, const uint4 (&pre)[kPre],
+                                               uint16_t* bins, uint32_t* cand_key,
+                                               uint32_t* cand_idx, uint32_t* cnt, uint32_t* pick,
+                                               bool* nonfinite) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int nv = d / 4;  // d is a multiple of 8
+  bool bad = false;
+  auto list_batch = [&](const uint4 (&u)[kPre], int vb) {
+    uint32_t hits = 0;
+#pragma unroll
+    for (int k = 0; k < kPre; ++k) {
+      const int v = vb + tid + k * kT;
+      const uint32_t w[4] = {u[k].x & kKeyMask, u[k].y & kKeyMask, u[k].z & kKeyMask, u[k].w & kKeyMask};
+      if (v < nv) {
+        uint2 packed;
+        packed.x = (w[0] >> kFineShift) | ((w[1] >> kFineShift) << 16);
+        packed.y = (w[2] >> kFineShift) | ((w[3] >> kFineShift) << 16);
+        reinterpret_cast<uint2*>(bins)[v] = packed;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        hits += v < nv && (w[e] >> kFineShift) == B;
+        bad |= v < nv && w[e] >= 0x7f800000u;
+      }
     }
-    for (; j < nc; ++j) {
-      const uint32_t kj = cand_key[j];
-      r += (kj > kc) | ((kj == kc) & (j < c));
+    uint32_t inc = hits;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += n;
     }
-    if (r == krem - 1u) {  // ranks are unique
-      pick[0] = kc;
-      pick[1] = cand_idx[c];
+    const uint32_t wtot = __shfl_sync(0xffffffffu, inc, 31);
+    if (wtot == 0u) return;  // warp-uniform
+    uint32_t base = 0;
+    if (lane == 31) base = atomicAdd(cnt, wtot);
+    uint32_t slot = __shfl_sync(0xffffffffu, base, 31) + inc - hits;
+    if (hits == 0u) return;
+#pragma unroll
+    for (int k = 0; k < kPre; ++k) {
+      const int v = vb + tid + k * kT;
+      const uint32_t w[4] = {u[k].x & kKeyMask, u[k].y & kKeyMask, u[k].z & kKeyMask, u[k].w & kKeyMask};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (v < nv && (w[e] >> kFineShift) == B) {
+          if (slot < static_cast<uint32_t>(kFusedCandCap)) {
+            cand_key[slot] = w[e];
+            cand_idx[slot] = static_cast<uint32_t>(4 * v + e);
+          }
+          ++slot;
+        }
+      }
     }
+  };
+  list_batch(pre, 0);
+  for (int v0 = kPre * kT; v0 < nv; v0 += kPre * kT) {
+    uint4 u[kPre];
+#pragma unroll
+    for (int k = 0; k < kPre; ++k) {
+      const int v = v0 + tid + k * kT;
+      u[k] = v < nv ? __ldcg(reinterpret_cast<const uint4*>(xkeys) + v) : make_uint4(0, 0, 0, 0);
+    }
+    list_batch(u, v0);
+  }
+  *nonfinite = bad;
+  __syncthreads();
+  // g threads per candidate (a power of two, within one warp): thread
+  // c * g + s compares candidate c with the 16-byte vectors s, s + g, ... of
+  // the list; the slots after the last candidate hold key 0 and index
+  // 0xffffffff, which never rank above a candidate
+  const int nc = static_cast<int>(min(*cnt, static_cast<uint32_t>(kFusedCandCap)));  // nB
+  const int nq = (nc + 3) / 4;
+  int g = 32;
+  while (g > 1 && nc * g > kT) g >>= 1;
+  const int c = tid / g, s = tid - c * g;
+  uint32_t kc = 0, ic = 0, r = 0;
+  if (c < nc) {
+    kc = cand_key[c];
+    ic = cand_idx[c];
+    const uint4* kq = reinterpret_cast<const uint4*>(cand_key);
+    const uint4* iq = reinterpret_cast<const uint4*>(cand_idx);
+#pragma unroll 2
+    for (int q = s; q < nq; q += g) {
+      const uint4 a = kq[q], b = iq[q];
+      r += (a.x > kc) | ((a.x == kc) & (b.x < ic));
+      r += (a.y > kc) | ((a.y == kc) & (b.y < ic));
+      r += (a.z > kc) | ((a.z == kc) & (b.z < ic));
+      r += (a.w > kc) | ((a.w == kc) & (b.w < ic));
+    }
+  }
+  for (int o = 1; o < g; o <<= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+  if (c < nc && s == 0 && r == krem - 1u) {  // ranks are unique
+    pick[0] = kc;
+    pick[1] = ic;
   }
   __syncthreads();
   return KthEntry{pick[0], static_cast<int32_t>(pick[1])};
@@ -980,73 +1034,83 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
     uint32_t* cand = reinterpret_cast<uint32_t*>(smem_raw + L.cand);
     uint32_t* cand_idx = reinterpret_cast<uint32_t*>(smem_raw + L.cand_idx);
     const uint32_t* xkeys = reinterpret_cast<const uint32_t*>(p.x_rot);
-    // the next call's histogram (the previous call, which used it, is done)
-    {
-      uint4* hn = reinterpret_cast<uint4*>(p.sync + kFusedSyncWords + 2 * kFusedMaxTiles +
-                                           ((gen + 1u) & 1u) * kFusedHistBins);
-      for (int i = tid; i < kFusedHistBins / 4; i += kT) hn[i] = make_uint4(0, 0, 0, 0);
+    for (int j = tid; j < kFusedCandCap; j += kT) {  // empty candidate slots (see select_kth)
+      cand[j] = 0u;
+      cand_idx[j] = 0xffffffffu;
     }
     if (tid == 0) {
       const bool ok = wait_ticket(ticket, target);
       if (!ok) report(p.dev_status, LAROSA_DEV_TIMEOUT);
-      // the next call's counters (the previous call, which used them, is done)
-      p.sync[(gen + 1u) & 1u] = 0u;
-      unsigned* tiles_next = p.sync + kFusedSyncWords + ((gen + 1u) & 1u) * kFusedMaxTiles;
-      for (int t = 0; t < p.n_tiles; ++t) tiles_next[t] = 0u;
       s_word[0] = ok;
+      s_word[1] = 0u;  // boundary candidates listed
     }
     __syncthreads();
     const bool ok = s_word[0] != 0u;
     const uint32_t mode = !ok || K <= 0 ? 0u : (K >= d ? 2u : 1u);
-    if (ok) {
-      const uint4* src = reinterpret_cast<const uint4*>(p.x_rot);  // d is a multiple of 8
-      const int nv = d / 4;
-      bool nonfinite = false;
-      for (int v0 = tid; v0 < nv; v0 += kT * kU) {
-        uint4 u[kU];
+    // one batch of L2 reads, made while the gather CTAs find the boundary
+    // and before they stream: this thread's share of the call's histogram
+    // and the first kPre vectors of x_rot
+    uint32_t hcnt[kHistShare<kT>];
+    uint4 pre[kPre];
+    if (mode == 1u) {
+      hist_share<kT, true>(ghist, hcnt);
 #pragma unroll
-        for (int k = 0; k < kU; ++k) {
-          const int v = v0 + k * kT;
-          u[k] = v < nv ? __ldcg(src + v) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int k = 0; k < kU; ++k) {
-          const int v = v0 + k * kT;
-          if (v < nv) {
-            const uint32_t w[4] = {u[k].x & kKeyMask, u[k].y & kKeyMask, u[k].z & kKeyMask,
-                                   u[k].w & kKeyMask};
-            nonfinite |= w[0] >= 0x7f800000u || w[1] >= 0x7f800000u || w[2] >= 0x7f800000u ||
-                         w[3] >= 0x7f800000u;
-            uint2 packed;
-            packed.x = (w[0] >> kFineShift) | ((w[1] >> kFineShift) << 16);
-            packed.y = (w[2] >> kFineShift) | ((w[3] >> kFineShift) << 16);
-            reinterpret_cast<uint2*>(bins)[v] = packed;
-          }
-        }
+      for (int k = 0; k < kPre; ++k) {
+        const int v = tid + k * kT;
+        pre[k] = v < d / 4 ? __ldcg(reinterpret_cast<const uint4*>(xkeys) + v) : make_uint4(0, 0, 0, 0);
       }
-      if (__syncthreads_or(nonfinite) && tid == 0) report(p.dev_status, LAROSA_DEV_NONFINITE);
     }
     uint32_t B = 0, above = 0, nB = 0;
-    if (mode == 1u) fine_boundary_at<kT, true>(ghist, K, s_warp_sums, s_pick, &B, &above, &nB);
     KthEntry e{0xffffffffu, -1};  // after a timeout: no bin-B row is kept
-    if (mode == 1u)
-      e = fused_kth(xkeys, bins, d, K, B, static_cast<uint32_t>(K) - above, nB, cand, cand_idx,
-                    s_warp_sums, s_pick);
+    bool nonfinite = false;
+    if (mode == 1u) {
+      boundary_from_share<kT>(hcnt, K, s_warp_sums, s_pick, &B, &above, &nB);
+      if (nB <= static_cast<uint32_t>(kFusedCandCap)) {
+        e = select_kth(xkeys, d, B, static_cast<uint32_t>(K) - above, pre, bins, cand, cand_idx, s_word + 1,
+                       s_pick, &nonfinite);
+      } else {
+        const uint4* src = reinterpret_cast<const uint4*>(xkeys);
+        for (int v = tid; v < d / 4; v += kT) {
+          const uint4 u = __ldcg(src + v);
+          const uint32_t w[4] = {u.x & kKeyMask, u.y & kKeyMask, u.z & kKeyMask, u.w & kKeyMask};
+          nonfinite |= w[0] >= 0x7f800000u || w[1] >= 0x7f800000u || w[2] >= 0x7f800000u ||
+                       w[3] >= 0x7f800000u;
+          uint2 packed;
+          packed.x = (w[0] >> kFineShift) | ((w[1] >> kFineShift) << 16);
+          packed.y = (w[2] >> kFineShift) | ((w[3] >> kFineShift) << 16);
+          reinterpret_cast<uint2*>(bins)[v] = packed;
+        }
+        e = kth_by_bisection(xkeys, d, K, s_warp_sums, s_pick);
+      }
+    }
     if (tid == 0) {
       p.sync[6] = e.T;
       p.sync[7] = static_cast<uint32_t>(e.I);
       st_release_gpu(p.sync + 3, gen);
     }
+    if (nonfinite) report(p.dev_status, LAROSA_DEV_NONFINITE);
     // the kept list for callers, off the gather's path
     if (mode == 1u) {
       __syncthreads();  // warp_sums may be reused
-      fused_export(xkeys, bins, d, B, e, nB <= static_cast<uint32_t>(kFusedCandCap), cand, p.idx, p.val,
-                   s_warp_sums);
+      fused_export(xkeys, bins, d, B, e, false, cand, p.idx, p.val, s_warp_sums);
     } else if (mode == 2u) {
       for (int i = tid; i < d; i += kT) {
+        const uint32_t u = __ldcg(xkeys + i);
+        if ((u & kKeyMask) >= 0x7f800000u) report(p.dev_status, LAROSA_DEV_NONFINITE);
         p.idx[i] = i;
-        p.val[i] = __uint_as_float(__ldcg(xkeys + i));
+        p.val[i] = __uint_as_float(u);
       }
+    }
+    // the next call's counters and histogram (call n - 1, which used them,
+    // is done); last, so that these stores do not queue ahead of the
+    // selection's loads
+    {
+      uint4* hn = reinterpret_cast<uint4*>(p.sync + kFusedSyncWords + 2 * kFusedMaxTiles +
+                                           ((gen + 1u) & 1u) * kFusedHistBins);
+      for (int i = tid; i < kFusedHistBins / 4; i += kT) hn[i] = make_uint4(0, 0, 0, 0);
+      unsigned* tiles_next = p.sync + kFusedSyncWords + ((gen + 1u) & 1u) * kFusedMaxTiles;
+      for (int t = tid; t < p.n_tiles; t += kT) tiles_next[t] = 0u;
+      if (tid == 0) p.sync[(gen + 1u) & 1u] = 0u;
     }
     return;
   }
