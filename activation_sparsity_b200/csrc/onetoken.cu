@@ -630,6 +630,7 @@ __host__ __device__ inline FLayout flayout(int d, int elem_bytes, int range_cap,
 }
 
 constexpr int kRowKeys = 256;  // rotated rows per CTA whose keys are aggregated in shared memory
+constexpr size_t kQPrefetchBytes = 32 << 10;  // rows of Q per CTA requested into L2 before the wait
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
@@ -951,13 +952,25 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   const int tile = cta / C, rank = cta - tile * C;
   const int d = p.d, K = p.K;
 
-  // launched in ordinary stream order (not as a programmatic dependent), so
-  // everything earlier on the stream is complete and visible here
-  if (tid == 0) s_gen = ld_acquire_gpu(p.sync + 3) + 1u;  // this call's number, read before arriving
-
   // ---- 1. rotation rows [r0, r1) of this CTA
   const int r0 = (int)((long long)d * cta / G);
   const int r1 = (int)((long long)d * (cta + 1) / G);
+  // Launched as a programmatic dependent of the previous kernel on the
+  // stream: until griddepcontrol.wait returns, that kernel may still be
+  // running, and nothing it writes may be read.  Q is a weight that no
+  // kernel on the stream writes, so this CTA's first rows of it are
+  // requested into L2 now, while the previous kernel's last CTAs leave HBM
+  // idle.
+  if (warp == 0) {
+    const size_t row_bytes = (size_t)d * sizeof(T);
+    const int n_pf = min(r1 - r0, static_cast<int>(kQPrefetchBytes / row_bytes) + 1);
+    for (int j = lane; j < n_pf; j += 32)
+      bulk_prefetch_l2(static_cast<const unsigned char*>(p.Qt) + (size_t)(r0 + j) * row_bytes,
+                       static_cast<uint32_t>(row_bytes));
+  }
+  pdl_wait();
+  pdl_launch_dependents();  // the next call may start its own prefetch as CTAs of this one finish
+  if (tid == 0) s_gen = ld_acquire_gpu(p.sync + 3) + 1u;  // this call's number, read before arriving
   {
     const int nvx = d * (int)sizeof(T) / 16;
     const uint4* xg = static_cast<const uint4*>(p.x);
@@ -1568,12 +1581,16 @@ cudaError_t launch_fused(Elem w_elem, const FusedArgs& a, const StreamPlan& pl,
   cfg.blockDim = dim3(kT, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = stream;
-  // every CTA must be resident at once: the gather CTAs wait on the selector
-  cudaLaunchAttribute attr[1];
+  // every CTA must be resident at once: the gather CTAs wait on the selector.
+  // As a programmatic dependent the launch may begin before the previous
+  // kernel on the stream ends (the kernel waits before reading its inputs).
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   void* args[] = {&p};
   return cudaLaunchKernelExC(&cfg, fn, args);
 }

@@ -55,15 +55,20 @@ def bf16_ulp(v: np.ndarray) -> np.ndarray:
     return np.ldexp(1.0, e - 8)
 
 
-def check_bf16_rounding(got: np.ndarray, exact: np.ndarray, gamma: np.ndarray) -> None:
+def check_bf16_rounding(got: np.ndarray, exact: np.ndarray, gamma: np.ndarray,
+                        min_same: float = 0.999) -> None:
     """got is the bf16 rounding of an fp32-accumulated value within gamma of exact.
 
-    At least 99.9 % must equal the round-to-nearest-even of the exact product;
-    every element must lie within gamma plus half a bf16 ulp of it.
+    Every element must lie within gamma plus half a bf16 ulp of the exact
+    product.  At least min_same of them must equal its round-to-nearest-even
+    (a wrong rounding mode would miss about half): the fp32 sum lands on the
+    other side of a bf16 rounding midpoint only when the exact value lies
+    within the accumulation error of one, which grows with the length of the
+    sum.
     """
     want = oracle.round_to_bf16(exact)
     same = got == want
-    assert same.mean() >= 0.999, same.mean()
+    assert same.mean() >= min_same, same.mean()
     assert np.all(np.abs(got - exact) <= gamma + 0.5 * bf16_ulp(got) + 1e-30)
 
 
