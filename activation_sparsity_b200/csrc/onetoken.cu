@@ -957,10 +957,10 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   const int r1 = (int)((long long)d * (cta + 1) / G);
   // Launched as a programmatic dependent of the previous kernel on the
   // stream: until griddepcontrol.wait returns, that kernel may still be
-  // running, and nothing it writes may be read.  Q is a weight that no
-  // kernel on the stream writes, so this CTA's first rows of it are
-  // requested into L2 now, while the previous kernel's last CTAs leave HBM
-  // idle.
+  // running, and nothing it writes may be read.  This CTA's first rows of Q
+  // are asked into L2 now, while the previous kernel's last CTAs leave HBM
+  // idle; a prefetch into L2 (the point of coherence) only moves a read
+  // earlier and never changes what a later load returns.
   if (warp == 0) {
     const size_t row_bytes = (size_t)d * sizeof(T);
     const int n_pf = min(r1 - r0, static_cast<int>(kQPrefetchBytes / row_bytes) + 1);

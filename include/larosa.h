@@ -191,11 +191,20 @@ int larosa_sparse_linear(const int32_t *idx, const float *val, int M, int K,
  *   x_rot = x . Q;  (idx, val) = TopK(x_rot, K);  y = sparse(x_rot) . W_rot.
  * x: [M x d_in] of `dtype`; Qt = Q^T: [d_in x d_in]; W_rot: [d_in x d_out] of
  * `dtype` (from larosa_prepare_weights with the same Qt); y: [M x d_out] fp32.
- * For one token this is two kernels: larosa_rotate_topk's kernel, then the
- * one-token gather of the kept rows.  The intermediate x_rot, idx
- * and val live in the workspace at the offsets larosa_workspace_layout()
- * gives.  d_in a multiple of 8; x, Qt, W_rot and y 16-byte aligned.
- * ws: at least larosa_workspace_bytes(M, d_in, d_out, K) bytes.
+ * For one token this is one cooperative kernel: every CTA rotates a share
+ * of x, a selector CTA finds the K-th entry, and the rest stream the kept
+ * rows of W_rot by column tiles (when the grid cannot be made resident it
+ * falls back to larosa_rotate_topk's kernel followed by the one-token
+ * gather).  That kernel is launched as a programmatic dependent of the
+ * previous kernel on the stream: before the previous kernel has finished it
+ * only asks for its first rows of Qt to be brought into L2, a hint that does
+ * not change what is read later.  For M > 1 the steps run as
+ * separate kernels.  The intermediate x_rot, idx and val live in the
+ * workspace at the offsets larosa_workspace_layout() gives (the kept list
+ * in ascending index order).  d_in a multiple of 8; x, Qt, W_rot and y
+ * 16-byte aligned.  ws: at least larosa_workspace_bytes(M, d_in, d_out, K)
+ * bytes; for M = 1 it holds counters that are zero between calls, so calls
+ * sharing a workspace must not overlap.
  */
 int larosa_rotate_topk_linear(const void *x, const void *Qt, const void *W_rot,
                               int M, int d_in, int d_out, int K, float *y,
