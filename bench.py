@@ -445,9 +445,12 @@ def bench_larosa(args):
                 barrier(world, device)
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            for gi, g in enumerate(groups):
+            # the step's inputs in, the four groups back to back, the outputs out
+            for gi in range(len(groups)):
                 x_dev[gi].copy_(x_host[gi], non_blocking=True)
+            for gi, g in enumerate(groups):
                 L.larosa_rotate_topk_linear(x_dev[gi], g.Qt, g.W_rot, g.K, y=ys[gi], ws=ws, dev_status=st)
+            for gi in range(len(groups)):
                 y_host[gi].copy_(ys[gi], non_blocking=True)
         e1.record(stream)
     torch.cuda.synchronize(device)
