@@ -4,7 +4,10 @@ For each token entering a linear layer: rotate the activation by the layer's
 orthogonal Q, keep its K largest-magnitude entries, and multiply by the
 counter-rotated weight W_rot = Q^T W, reading only the K kept rows
 ("La RoSA: Enhancing LLM Efficiency via Layerwise Rotated Sparse
-Activation", method and abstract).
+Activation", method and abstract).  The same path also runs with the
+identity rotation (no Q: fixed-K magnitude sparsity) and with a threshold
+|x_rot| >= t in place of the Top-K (the threshold function of the R-Sparse
+report).
 
 The compute lives in liblarosa.so (C ABI, include/larosa.h); the submodule
 ``larosa`` is its thin Python binding and is loaded on first use of any name
@@ -15,7 +18,8 @@ _EXPORTS = (
     "LarosaError", "Workspace", "larosa_check", "larosa_dense_linear", "larosa_prepare_weights",
     "larosa_rotate", "larosa_rotate_topk", "larosa_rotate_topk_linear", "larosa_sparse_linear",
     "larosa_sparse_linear_noalloc", "larosa_topk", "larosa_version", "larosa_workspace_bytes",
-    "larosa_workspace_layout", "LAROSA_F32", "LAROSA_BF16", "LAROSA_MAX_D", "LAROSA_MAX_M",
+    "larosa_workspace_layout", "larosa_workspace_nnz_offset", "larosa_threshold",
+    "larosa_rotate_threshold_linear", "LAROSA_F32", "LAROSA_BF16", "LAROSA_MAX_D", "LAROSA_MAX_M",
     "LIB_PATH",
 )
 __all__ = list(_EXPORTS)

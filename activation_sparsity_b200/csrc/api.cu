@@ -9,6 +9,11 @@
 //   fused, M = 1               fused_kernel (onetoken.cu): one cooperative launch;
 //                              where it does not fit, rotsel -> list gather
 //   fused, M > 1               rowdot -> topk -> scatter/union -> rowstream
+//   threshold, M = 1           fused_kernel in threshold mode; where it does not
+//                              fit, rowdot -> threshold -> rowstream over the list
+//   threshold, M > 1           rowdot -> threshold (writes the coefficient rows
+//                              and the bitmap) -> union -> rowstream
+//   no Qt (identity rotation)  as above with widen in place of rowdot
 #include <stdio.h>
 #include <string.h>
 
@@ -58,10 +63,11 @@ bool row_aligned(int n, int dtype) { return (n * elem_size(dtype)) % 16 == 0; }
 
 struct Layout {
   size_t fused_sync = 0;  // the fused kernel's synchronisation block (M = 1)
-  size_t x_rot = 0, idx = 0, val = 0;
+  size_t x_rot = 0, idx = 0, val = 0, nnz = 0;
   size_t partials = 0;
   size_t coef = 0, urows = 0, ucount = 0;
   size_t total = 0;
+  bool list_gemv = false;  // M = 1: the row-streaming GEMV over a list of up to d_in rows fits
 };
 
 int sparse_rows_max(int M, int d_in, int K) {
@@ -105,6 +111,7 @@ int make_layout(int M, int d_in, int d_out, int K, Layout* L) {
 
 int make_layout_uncached(int M, int d_in, int d_out, int K, Layout* L) {
   size_t partials = 0;
+  L->list_gemv = M == 1;
   for (int dt = 0; dt < 2; ++dt) {
     const Elem w = dt == 0 ? Elem::F32 : Elem::BF16;
     if (M == 1) {
@@ -113,6 +120,14 @@ int make_layout_uncached(int M, int d_in, int d_out, int K, Layout* L) {
       if (e == cudaSuccess) e = larosa::plan_fused(w, d_in, d_out, K, &sf);
       if (e != cudaSuccess) return cuda_fail(e, "plan gather");
       if (sf.ok) partials = std::max(partials, sf.partial_floats);
+      // the threshold path's fallback streams a list of up to d_in rows
+      GemvPlan pt;
+      e = larosa::plan_gemv(w, Elem::F32, 1, d_out, d_in, &pt);
+      if (e != cudaSuccess) return cuda_fail(e, "plan sparse linear");
+      if (pt.ticket_words <= kSplitKTicketWords)
+        partials = std::max(partials, pt.partial_floats);
+      else
+        L->list_gemv = false;
       if (sl.ok) continue;  // the list-mode gather needs no partials
     }
     GemvPlan ps;
@@ -131,6 +146,7 @@ int make_layout_uncached(int M, int d_in, int d_out, int K, Layout* L) {
   L->x_rot = take((size_t)M * d_in * 4);
   L->idx = take((size_t)M * K * 4);
   L->val = take((size_t)M * K * 4);
+  L->nnz = take((size_t)M * 4);
   L->partials = take(partials * 4);
   if (M > 1) {
     L->coef = take((size_t)M * d_in * 4);
@@ -161,10 +177,32 @@ bool rowdot_aligned(const void* A, const void* x, int n_in) {
   return aligned16(A) && aligned16(x) && (n_in % 8) == 0;
 }
 
+// The rotation's operands, Qt null meaning the identity rotation.
+bool rotation_aligned(const void* Qt, const void* x, int d) {
+  return (Qt == nullptr || aligned16(Qt)) && aligned16(x) && (d % 8) == 0;
+}
+
 int run_rowdot(const void* x, const void* A, float* y, int M, int n_in, int n_out, int dtype,
                cudaStream_t s, const char* what) {
   cudaError_t e = larosa::launch_rowdot(elem_of(dtype), A, x, y, M, n_in, n_out, s);
   return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, what);
+}
+
+// x_rot = x . Q, or x widened when Qt is null (the identity rotation).
+int run_rotation(const void* x, const void* Qt, float* x_rot, int M, int d, int dtype,
+                 cudaStream_t s) {
+  if (Qt != nullptr) return run_rowdot(x, Qt, x_rot, M, d, d, dtype, s, "rotation kernel");
+  cudaError_t e = larosa::launch_widen(x, x_rot, M * d, elem_of(dtype), s);
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "widen kernel");
+}
+
+// Threshold t >= 0 as the key it is compared with (sign-cleared fp32 bits);
+// t <= 0 keeps everything.
+uint32_t threshold_key(float t) {
+  if (!(t > 0.f)) return 0u;
+  uint32_t k;
+  memcpy(&k, &t, sizeof(k));
+  return k;
 }
 
 int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W_rot, int d_in,
@@ -279,6 +317,16 @@ int larosa_workspace_layout(int M, int d_in, int d_out, int K, size_t* x_rot_off
   return LAROSA_OK;
 }
 
+int larosa_workspace_nnz_offset(int M, int d_in, int d_out, int K, size_t* nnz_offset) {
+  int st = check_sizes(M, d_in, d_out, K);
+  if (st != LAROSA_OK) return st;
+  Layout L;
+  st = make_layout(M, d_in, d_out, K, &L);
+  if (st != LAROSA_OK) return st;
+  if (nnz_offset) *nnz_offset = L.nnz;
+  return LAROSA_OK;
+}
+
 int larosa_prepare_weights(const void* Qt, const void* W, void* W_rot, int d_in, int d_out,
                            int dtype, larosa_stream_t stream) {
   if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
@@ -363,11 +411,10 @@ int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, 
                               int d_out, int K, float* y, void* ws, size_t ws_bytes,
                               int* dev_status, int dtype, larosa_stream_t stream) {
   if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
-  if (x == nullptr || Qt == nullptr || W_rot == nullptr || y == nullptr)
-    return LAROSA_ERR_INVALID_ARG;
+  if (x == nullptr || W_rot == nullptr || y == nullptr) return LAROSA_ERR_INVALID_ARG;
   int st = check_sizes(M, d_in, d_out, K);
   if (st != LAROSA_OK) return st;
-  if (!rowdot_aligned(Qt, x, d_in) || !aligned16(W_rot) || !aligned16(y) ||
+  if (!rotation_aligned(Qt, x, d_in) || !aligned16(W_rot) || !aligned16(y) ||
       !row_aligned(d_out, dtype))
     return LAROSA_ERR_ALIGN;
   Layout L;
@@ -403,7 +450,7 @@ int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, 
       return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "fused kernel");
     }
   }
-  if (M == 1 && larosa::rotsel_fits(elem_of(dtype), d_in)) {
+  if (M == 1 && Qt != nullptr && larosa::rotsel_fits(elem_of(dtype), d_in)) {
     // rotation whose last CTA writes the kept list, then the list-mode gather
     larosa::StreamPlan sp;
     cudaError_t e = larosa::plan_gather(elem_of(dtype), d_out, K, &sp);
@@ -434,11 +481,120 @@ int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, 
       return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "gather kernel");
     }
   }
-  st = run_rowdot(x, Qt, x_rot, M, d_in, d_in, dtype, s, "rotation kernel");
+  st = run_rotation(x, Qt, x_rot, M, d_in, dtype, s);
   if (st != LAROSA_OK) return st;
   cudaError_t e = larosa::launch_topk(x_rot, M, d_in, K, idx, val, dev_status, s);
   if (e != cudaSuccess) return cuda_fail(e, "topk kernel");
   return run_sparse(idx, val, M, K, W_rot, d_in, d_out, y, dtype, ws, L, dev_status, s);
+}
+
+int larosa_threshold(const float* x_rot, int M, int d, float t, int32_t* idx, float* val,
+                     int32_t* nnz, int* dev_status, larosa_stream_t stream) {
+  if (x_rot == nullptr || idx == nullptr || val == nullptr || nnz == nullptr || t != t)
+    return LAROSA_ERR_INVALID_ARG;
+  if (M < 1 || M > LAROSA_MAX_M || d < 1 || d > LAROSA_MAX_D) return LAROSA_ERR_SHAPE;
+  cudaError_t e = larosa::launch_threshold(x_rot, M, d, threshold_key(t), idx, val, nnz, nullptr,
+                                           nullptr, dev_status,
+                                           reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "threshold kernel");
+}
+
+int larosa_rotate_threshold_linear(const void* x, const void* Qt, const void* W_rot, int M,
+                                   int d_in, int d_out, float t, float* y, void* ws,
+                                   size_t ws_bytes, int* dev_status, int dtype,
+                                   larosa_stream_t stream) {
+  if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
+  if (x == nullptr || W_rot == nullptr || y == nullptr || t != t) return LAROSA_ERR_INVALID_ARG;
+  int st = check_sizes(M, d_in, d_out, d_in);
+  if (st != LAROSA_OK) return st;
+  if (!rotation_aligned(Qt, x, d_in) || !aligned16(W_rot) || !aligned16(y) ||
+      !row_aligned(d_out, dtype))
+    return LAROSA_ERR_ALIGN;
+  Layout L;
+  st = make_layout(M, d_in, d_out, d_in, &L);
+  if (st != LAROSA_OK) return st;
+  st = workspace_ok(ws, ws_bytes, L);
+  if (st != LAROSA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* x_rot = reinterpret_cast<float*>(at(ws, L.x_rot));
+  int32_t* idx = reinterpret_cast<int32_t*>(at(ws, L.idx));
+  float* val = reinterpret_cast<float*>(at(ws, L.val));
+  int32_t* nnz = reinterpret_cast<int32_t*>(at(ws, L.nnz));
+  const uint32_t t_key = threshold_key(t);
+  cudaError_t e;
+  if (M == 1) {
+    // one cooperative kernel: rotation, threshold, gather
+    larosa::StreamPlan fp;
+    e = larosa::plan_fused(elem_of(dtype), d_in, d_out, d_in, &fp);
+    if (e != cudaSuccess) return cuda_fail(e, "plan fused");
+    if (fp.ok) {
+      larosa::FusedArgs f;
+      f.x = x;
+      f.Qt = Qt;
+      f.W = W_rot;
+      f.x_rot = x_rot;
+      f.idx = idx;
+      f.val = val;
+      f.y = y;
+      f.partials = reinterpret_cast<float*>(at(ws, L.partials));
+      f.sync = reinterpret_cast<unsigned*>(at(ws, L.fused_sync));
+      f.d_in = d_in;
+      f.d_out = d_out;
+      f.K = d_in;
+      f.dev_status = dev_status;
+      f.threshold = true;
+      f.t_key = t_key;
+      f.nnz = nnz;
+      e = larosa::launch_fused(elem_of(dtype), f, fp, s);
+      return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "fused kernel");
+    }
+    if (!L.list_gemv) return LAROSA_ERR_SHAPE;
+  }
+  st = run_rotation(x, Qt, x_rot, M, d_in, dtype, s);
+  if (st != LAROSA_OK) return st;
+  GemvPlan pl;
+  e = larosa::plan_gemv(elem_of(dtype), Elem::F32, M, d_out, d_in, &pl);
+  if (e != cudaSuccess) return cuda_fail(e, "plan sparse linear");
+  GemvArgs a;
+  a.W = W_rot;
+  a.w_elem = elem_of(dtype);
+  a.d_out = d_out;
+  a.row_bound = d_in;
+  a.coef_elem = Elem::F32;
+  a.M = M;
+  a.y = y;
+  a.y_ld = d_out;
+  a.partials = reinterpret_cast<float*>(at(ws, L.partials));
+  a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTickets));
+  a.dev_status = dev_status;
+  a.n_rows = d_in;
+  if (M == 1) {
+    // the kept list and its length, read on the device
+    e = larosa::launch_threshold(x_rot, 1, d_in, t_key, idx, val, nnz, nullptr, nullptr,
+                                 dev_status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "threshold kernel");
+    a.rows = idx;
+    a.n_rows_dev = nnz;
+    a.coef = val;
+    a.coef_ld = d_in;
+  } else {
+    // every token's coefficient row and the union of the kept rows
+    float* coef = reinterpret_cast<float*>(at(ws, L.coef));
+    unsigned* bitmap = reinterpret_cast<unsigned*>(at(ws, kOffBitmap));
+    int32_t* urows = reinterpret_cast<int32_t*>(at(ws, L.urows));
+    int* ucount = reinterpret_cast<int*>(at(ws, L.ucount));
+    e = larosa::launch_threshold(x_rot, M, d_in, t_key, idx, val, nnz, coef, bitmap, dev_status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "threshold kernel");
+    e = larosa::launch_union(bitmap, d_in, urows, ucount, s);
+    if (e != cudaSuccess) return cuda_fail(e, "union kernel");
+    a.rows = urows;
+    a.n_rows_dev = ucount;
+    a.coef = coef;
+    a.coef_ld = d_in;
+    a.coef_by_row = 1;
+  }
+  e = larosa::launch_gemv(a, pl, s);
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "sparse linear kernel");
 }
 
 int larosa_dense_linear(const void* x, const void* Wt, int M, int d_in, int d_out, float* y,

@@ -58,6 +58,18 @@ cudaError_t launch_gemv(const GemvArgs& a, const GemvPlan& plan, cudaStream_t st
 cudaError_t launch_topk(const float* x_rot, int M, int d, int K, int32_t* idx, float* val,
                         int* dev_status, cudaStream_t stream);
 
+// Threshold selection: one 1024-thread CTA per token keeps |x_rot| >= t
+// (t_key: bit pattern of t, 0 for t <= 0), writes the kept (idx, val) in
+// ascending order into rows of length d and the count to nnz[m]; with coef
+// != nullptr also the coefficient row (x where kept, else 0) and the bitmap
+// of kept rows, as launch_scatter does.
+cudaError_t launch_threshold(const float* x_rot, int M, int d, uint32_t t_key, int32_t* idx,
+                             float* val, int32_t* nnz, float* coef, unsigned* bitmap,
+                             int* dev_status, cudaStream_t stream);
+
+// x_rot[i] = x[i] widened to fp32 (the identity rotation), n elements.
+cudaError_t launch_widen(const void* x, float* x_rot, int n, Elem elem, cudaStream_t stream);
+
 // M > 1: scatter each token's (idx, val) into a dense zero-filled coefficient
 // row and mark the rows used by any token in `bitmap` (d_in bits).
 cudaError_t launch_scatter(const int32_t* idx, const float* val, int M, int K, int d_in,
@@ -150,7 +162,11 @@ struct FusedArgs {
   int d_out = 0;
   int K = 0;
   int* dev_status = nullptr;
+  bool threshold = false;  // keep |x_rot| >= t (t_key) instead of the Top-K
+  uint32_t t_key = 0;
+  int32_t* nnz = nullptr;  // threshold mode: the kept count
 };
+// With Qt == nullptr the rotation is the identity (x_rot = x widened).
 
 // plan->ok is false when the shape does not fit (then use the two-kernel path).
 cudaError_t plan_fused(Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan);

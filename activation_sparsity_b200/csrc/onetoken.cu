@@ -580,7 +580,7 @@ __global__ void __launch_bounds__(kT, 2) rotsel_kernel(const RSParams p) {
 
 struct FParams {
   const void* x;      // [d] activation
-  const void* Qt;     // [d x d] rotation, stored transposed
+  const void* Qt;     // [d x d] rotation, stored transposed (unused when !rotate)
   const void* W;      // [d x d_out] counter-rotated weight
   float* x_rot;       // [d]
   int32_t* idx;       // [K] kept list (for callers)
@@ -597,6 +597,10 @@ struct FParams {
   int range_cap;      // ceil(d / C): indices a gather CTA owns
   int n_tiles;        // column tiles (C gather CTAs each)
   int* dev_status;
+  int rotate;         // 0: the identity rotation, x_rot = x
+  int thresh;         // 1: keep |x_rot| >= t (key >= t_key) instead of the Top-K
+  uint32_t t_key;
+  int32_t* nnz;       // threshold mode: the kept count (for callers)
 };
 
 struct FLayout {
@@ -936,6 +940,62 @@ __device__ __forceinline__ void fused_export(const uint32_t* xkeys, const uint16
   }
 }
 
+// Threshold mode's kept list for callers: the indices whose key (sign-
+// cleared bits of x_rot, read through L2) is >= t_key, in ascending order,
+// with their values; returns their number (the same in every thread) and
+// sets *nonfinite in a thread that met a NaN or Inf.  Warp segments, keys
+// read kU x 32 at a time, ballots; all kT threads call it.
+__device__ __noinline__ uint32_t export_threshold(const uint32_t* xkeys, int d, uint32_t t_key,
+                                                  int32_t* idx, float* val, uint32_t* warp_sums,
+                                                  bool* nonfinite) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t below = (1u << lane) - 1u;
+  int s0, s1;
+  warp_segment<kT>(d, &s0, &s1);
+  uint32_t n = 0;
+  bool bad = false;
+  for (int i0 = s0; i0 < s1; i0 += 32 * kU) {
+    uint32_t u[kU];
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      const int i = i0 + 32 * k + lane;
+      u[k] = i < s1 ? __ldcg(xkeys + i) & kKeyMask : 0u;
+    }
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      const int i = i0 + 32 * k + lane;
+      n += i < s1 && u[k] >= t_key;
+      bad |= u[k] >= 0x7f800000u;
+    }
+  }
+  *nonfinite = bad;
+  n = __reduce_add_sync(0xffffffffu, n);
+  uint32_t total = 0;
+  uint32_t pos = warp_base<kT>(n, warp_sums, &total);
+  if (n != 0u) {  // warp-uniform
+    for (int i0 = s0; i0 < s1; i0 += 32 * kU) {
+      uint32_t u[kU];
+#pragma unroll
+      for (int k = 0; k < kU; ++k) {
+        const int i = i0 + 32 * k + lane;
+        u[k] = i < s1 ? __ldcg(xkeys + i) : 0u;
+      }
+#pragma unroll
+      for (int k = 0; k < kU; ++k) {
+        const int i = i0 + 32 * k + lane;
+        const bool kept = i < s1 && (u[k] & kKeyMask) >= t_key;
+        const uint32_t m = __ballot_sync(0xffffffffu, kept);
+        if (kept) {
+          idx[pos + __popc(m & below)] = i;
+          val[pos + __popc(m & below)] = __uint_as_float(u[k]);
+        }
+        pos += __popc(m);
+      }
+    }
+  }
+  return total;
+}
+
 template <typename T, int C>
 __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   constexpr int CPT = 16 / sizeof(T);
@@ -961,7 +1021,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   // are asked into L2 now, while the previous kernel's last CTAs leave HBM
   // idle; a prefetch into L2 (the point of coherence) only moves a read
   // earlier and never changes what a later load returns.
-  if (warp == 0) {
+  if (warp == 0 && p.rotate) {
     const size_t row_bytes = (size_t)d * sizeof(T);
     const int n_pf = min(r1 - r0, static_cast<int>(kQPrefetchBytes / row_bytes) + 1);
     for (int j = lane; j < n_pf; j += 32)
@@ -971,7 +1031,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   pdl_wait();
   pdl_launch_dependents();  // the next call may start its own prefetch as CTAs of this one finish
   if (tid == 0) s_gen = ld_acquire_gpu(p.sync + 3) + 1u;  // this call's number, read before arriving
-  {
+  if (p.rotate) {
     const int nvx = d * (int)sizeof(T) / 16;
     const uint4* xg = static_cast<const uint4*>(p.x);
     for (int i = tid; i < nvx; i += kT) reinterpret_cast<uint4*>(smem_raw)[i] = __ldg(xg + i);
@@ -1020,12 +1080,26 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
                         (key >> kFineShift), 1u);
       }
     }
+  } else {
+    // the identity rotation (no Q): x_rot = x widened to fp32
+    __syncthreads();  // s_gen
+    const T* xv = static_cast<const T*>(p.x);
+    for (int row = r0 + tid; row < r1; row += kT) {
+      const float v = to_f32(xv[row]);
+      __stcg(p.x_rot + row, v);
+      const uint32_t key = __float_as_uint(v) & kKeyMask;
+      if (row - r0 < kRowKeys)
+        s_rowkey[row - r0] = key;
+      else
+        atomicAdd(p.sync + kFusedSyncWords + 2 * kFusedMaxTiles + (s_gen & 1u) * kFusedHistBins +
+                      (key >> kFineShift), 1u);
+    }
   }
   __syncthreads();  // the staged x is dead; this CTA's rows are written
   const unsigned gen = s_gen;
   unsigned* ticket = p.sync + (gen & 1u);
   unsigned* ghist = p.sync + kFusedSyncWords + 2 * kFusedMaxTiles + (gen & 1u) * kFusedHistBins;
-  if (warp == 0) {
+  if (warp == 0 && !p.thresh) {
     // this CTA's rows into the call's histogram of bits 30..19 of |x_rot|:
     // equal bins among 32 rows are added once
     const int nk = min(r1 - r0, kRowKeys);
@@ -1059,7 +1133,8 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
     }
     __syncthreads();
     const bool ok = s_word[0] != 0u;
-    const uint32_t mode = !ok || K <= 0 ? 0u : (K >= d ? 2u : 1u);
+    // 0 keeps nothing, 1 Top-K, 2 keeps all, 3 threshold
+    const uint32_t mode = !ok ? 0u : p.thresh ? 3u : (K <= 0 ? 0u : (K >= d ? 2u : 1u));
     // one batch of L2 reads, made while the gather CTAs find the boundary
     // and before they stream: this thread's share of the call's histogram
     // and the first kPre vectors of x_rot
@@ -1113,6 +1188,13 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
         p.idx[i] = i;
         p.val[i] = __uint_as_float(u);
       }
+    } else if (mode == 3u) {
+      bool bad = false;
+      const uint32_t n = export_threshold(xkeys, d, p.t_key, p.idx, p.val, s_warp_sums, &bad);
+      if (bad) report(p.dev_status, LAROSA_DEV_NONFINITE);
+      if (tid == 0) p.nnz[0] = static_cast<int32_t>(n);
+    } else if (p.thresh && tid == 0) {
+      p.nnz[0] = 0;  // after a timeout
     }
     // the next call's counters and histogram (call n - 1, which used them,
     // is done); last, so that these stores do not queue ahead of the
@@ -1151,7 +1233,8 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   }
   __syncthreads();
   const bool arrived = s_word[0] != 0u;
-  const uint32_t mode = !arrived || K <= 0 ? 0u : (K >= d ? 2u : 1u);  // 0 keeps nothing
+  // 0 keeps nothing, 1 Top-K, 2 keeps all, 3 threshold
+  const uint32_t mode = !arrived ? 0u : p.thresh ? 3u : (K <= 0 ? 0u : (K >= d ? 2u : 1u));
   uint32_t hcnt[kHistShare<kT>];  // this thread's share of the call's histogram
   if (mode == 1u) hist_share<kT, true>(ghist, hcnt);
   if (arrived) {
@@ -1177,7 +1260,9 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   }
   const int n_certain = compact_range(
       rkeys, n_r, i_lo,
-      [&](uint32_t k, int) { return mode == 2u || (mode == 1u && (k >> kFineShift) > B); },
+      [&](uint32_t k, int) {
+        return mode == 2u || (mode == 3u && k >= p.t_key) || (mode == 1u && (k >> kFineShift) > B);
+      },
       lrows, lvals, 0, s_warp_sums);
   __syncthreads();  // the certain list is in place
   if (mode == 1u) {
@@ -1277,6 +1362,15 @@ int round_up_mt(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 
 
 }  // namespace
 
+// The identity rotation for the composed paths: x_rot = x widened to fp32.
+template <typename T>
+__global__ void __launch_bounds__(kT) widen_kernel(const T* __restrict__ x, float* __restrict__ x_rot,
+                                                   int n) {
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int i = blockIdx.x * kT + threadIdx.x; i < n; i += gridDim.x * kT) x_rot[i] = to_f32(x[i]);
+}
+
 // ---------------------------------------------------------------- host API
 
 cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M, int n_in,
@@ -1303,6 +1397,31 @@ cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M,
   const int per_sm = (MT <= 2 && e == Elem::BF16) ? 2 : 1;
   const int grid = std::max(1, std::min(ds->sms * per_sm, n_out));
   return launch(fn, grid, in_smem ? xbytes : 0, &p, stream);
+}
+
+cudaError_t launch_widen(const void* x, float* x_rot, int n, Elem elem, cudaStream_t stream) {
+  DevState* ds = nullptr;
+  cudaError_t e = dev_state(&ds);
+  if (e != cudaSuccess) return e;
+  const int grid = std::max(1, std::min((n + kT - 1) / kT, 2 * ds->sms));
+  void* fn = elem == Elem::BF16 ? reinterpret_cast<void*>(&widen_kernel<__nv_bfloat16>)
+                                : reinterpret_cast<void*>(&widen_kernel<float>);
+  struct {
+    const void* x;
+    float* x_rot;
+    int n;
+  } a{x, x_rot, n};
+  void* args[] = {&a.x, &a.x_rot, &a.n};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kT, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
 // ---------------------------------------------------------------- rotate + select
@@ -1576,6 +1695,10 @@ cudaError_t launch_fused(Elem w_elem, const FusedArgs& a, const StreamPlan& pl,
   p.range_cap = pl.list_cap;
   p.n_tiles = pl.n_tiles;
   p.dev_status = a.dev_status;
+  p.rotate = a.Qt != nullptr;
+  p.thresh = a.threshold;
+  p.t_key = a.t_key;
+  p.nnz = a.nnz;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.n_tiles * pl.cluster + 1, 1, 1);
   cfg.blockDim = dim3(kT, 1, 1);

@@ -94,7 +94,81 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   kept_list<kTopkThreads>(bits, d4, K, &sel, cand, cand_idx, kTopkCand, 0, K, out_i, out_v);
 }
 
+// ---------------------------------------------------------------- threshold
+//
+// Threshold selection (R-Sparse report, 研究流程与方法 / R-Sparse框架设计: the
+// inputs with |x_j| >= t are kept, the rest masked), one 1024-thread CTA per
+// token.  t_key is the bit pattern of t >= 0 (0 for t <= 0); magnitudes
+// compare as their sign-cleared bit patterns.  The kept entries are written
+// in ascending index order to idx/val [M x d] (positions beyond nnz[m] are
+// left as they were) and their count to nnz[m].  With coef != nullptr the
+// token's row of coef [M x d] also receives x where kept and 0 elsewhere,
+// and the kept rows are marked in `bitmap` (the multi-token sparse linear's
+// input, as the scatter kernel makes it).  Each warp walks its own segment
+// of the row twice: once to count, once to place its kept entries after the
+// earlier warps' ones.
+__global__ void __launch_bounds__(kTopkThreads, 1)
+    threshold_kernel(const float* __restrict__ x_rot, int d, uint32_t t_key, int32_t* __restrict__ idx,
+                     float* __restrict__ val, int32_t* __restrict__ nnz, float* __restrict__ coef,
+                     unsigned* bitmap, int* dev_status) {
+  __shared__ uint32_t warp_sums[32];
+  const int m = blockIdx.x;
+  const int lane = threadIdx.x & 31;
+  const uint32_t below = (1u << lane) - 1u;
+  const uint32_t* bits = reinterpret_cast<const uint32_t*>(x_rot + (size_t)m * d);
+  pdl_wait();
+  pdl_launch_dependents();
+  int s0, s1;
+  warp_segment<kTopkThreads>(d, &s0, &s1);
+  uint32_t n = 0;
+  bool bad = false;
+  for (int i = s0 + lane; i < s1; i += 32) {
+    const uint32_t key = bits[i] & kKeyMask;
+    n += key >= t_key;
+    bad |= key >= 0x7f800000u;
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) report(dev_status, LAROSA_DEV_NONFINITE);
+  n = __reduce_add_sync(0xffffffffu, n);
+  uint32_t total = 0;
+  uint32_t pos = warp_base<kTopkThreads>(n, warp_sums, &total);
+  int32_t* out_i = idx + (size_t)m * d;
+  float* out_v = val + (size_t)m * d;
+  float* crow = coef != nullptr ? coef + (size_t)m * d : nullptr;
+  for (int i0 = s0; i0 < s1; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t u = i < s1 ? bits[i] : 0u;
+    const bool kept = i < s1 && (u & kKeyMask) >= t_key;
+    const uint32_t mk = __ballot_sync(0xffffffffu, kept);
+    if (kept) {
+      out_i[pos + __popc(mk & below)] = i;
+      out_v[pos + __popc(mk & below)] = __uint_as_float(u);
+    }
+    if (crow != nullptr && i < s1) {
+      crow[i] = kept ? __uint_as_float(u) : 0.f;
+      if (kept) atomicOr(&bitmap[i >> 5], 1u << (i & 31));
+    }
+    pos += __popc(mk);
+  }
+  if (threadIdx.x == 0) nnz[m] = static_cast<int32_t>(total);
+}
+
 }  // namespace
+
+cudaError_t launch_threshold(const float* x_rot, int M, int d, uint32_t t_key, int32_t* idx,
+                             float* val, int32_t* nnz, float* coef, unsigned* bitmap,
+                             int* dev_status, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(M, 1, 1);
+  cfg.blockDim = dim3(kTopkThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, threshold_kernel, x_rot, d, t_key, idx, val, nnz, coef, bitmap,
+                            dev_status);
+}
 
 cudaError_t launch_topk(const float* x_rot, int M, int d, int K, int32_t* idx, float* val,
                         int* dev_status, cudaStream_t stream) {

@@ -42,10 +42,14 @@ _SIGNATURES = {
     "larosa_rotate_topk": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _sz, _vp, _i, _vp], _i),
     "larosa_sparse_linear": ([_vp, _vp, _i, _i, _vp, _i, _i, _vp, _vp, _sz, _i, _vp, _vp], _i),
     "larosa_rotate_topk_linear": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp, _i, _vp], _i),
+    "larosa_threshold": ([_vp, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _vp], _i),
+    "larosa_rotate_threshold_linear": ([_vp, _vp, _vp, _i, _i, _i, _c.c_float, _vp, _vp, _sz, _vp, _i,
+                                        _vp], _i),
     "larosa_dense_linear": ([_vp, _vp, _i, _i, _i, _vp, _i, _vp], _i),
     "larosa_sparse_linear_noalloc": ([_vp, _vp, _i, _i, _vp, _i, _i, _vp, _i, _vp, _vp], _i),
     "larosa_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "larosa_workspace_layout": ([_i, _i, _i, _i, _c.POINTER(_sz), _c.POINTER(_sz), _c.POINTER(_sz)], _i),
+    "larosa_workspace_nnz_offset": ([_i, _i, _i, _i, _c.POINTER(_sz)], _i),
     "larosa_check": ([_vp, _vp, _c.POINTER(_i)], _i),
 }
 for _name, (_args, _ret) in _SIGNATURES.items():
@@ -193,6 +197,13 @@ def larosa_workspace_layout(M: int, d_in: int, d_out: int, K: int) -> tuple[int,
     return a.value, b.value, c.value
 
 
+def larosa_workspace_nnz_offset(M: int, d_in: int, d_out: int, K: int) -> int:
+    a = ctypes.c_size_t()
+    _check(_lib.larosa_workspace_nnz_offset(M, d_in, d_out, K, ctypes.byref(a)),
+           "larosa_workspace_nnz_offset")
+    return a.value
+
+
 def larosa_prepare_weights(Qt: torch.Tensor, W: torch.Tensor, W_rot: torch.Tensor | None = None
                            ) -> torch.Tensor:
     """W_rot = Q^T . W = Qt . W (offline counter-rotation), same dtype as W.
@@ -319,12 +330,15 @@ def larosa_sparse_linear_noalloc(idx: torch.Tensor, val: torch.Tensor, W_rot: to
     return y
 
 
-def larosa_rotate_topk_linear(x: torch.Tensor, Qt: torch.Tensor, W_rot: torch.Tensor, K: int,
+def larosa_rotate_topk_linear(x: torch.Tensor, Qt: torch.Tensor | None, W_rot: torch.Tensor, K: int,
                               y: torch.Tensor | None = None, ws=None,
                               dev_status: torch.Tensor | None = None) -> torch.Tensor:
-    """Fused rotate -> Top-K -> sparse linear (Qt = Q^T), fp32 output [M, d_out]."""
+    """Fused rotate -> Top-K -> sparse linear (Qt = Q^T), fp32 output [M, d_out].
+
+    Qt = None is the identity rotation (the unrotated fixed-K mode)."""
     _need(x, "x")
-    _need(Qt, "Qt", x.dtype)
+    if Qt is not None:
+        _need(Qt, "Qt", x.dtype)
     _need(W_rot, "W_rot", x.dtype)
     x2 = _as2d(x)
     M, d_in = x2.shape
@@ -336,6 +350,55 @@ def larosa_rotate_topk_linear(x: torch.Tensor, Qt: torch.Tensor, W_rot: torch.Te
     _check(_lib.larosa_rotate_topk_linear(_ptr(x2), _ptr(Qt), _ptr(W_rot), M, d_in, d_out, K, _ptr(y),
                                           p, n, _status_ptr(dev_status, x.device), _dtype_code(x),
                                           _stream(x.device)), "larosa_rotate_topk_linear")
+    return y
+
+
+def larosa_threshold(x_rot: torch.Tensor, t: float, idx: torch.Tensor | None = None,
+                     val: torch.Tensor | None = None, nnz: torch.Tensor | None = None,
+                     dev_status: torch.Tensor | None = None
+                     ) -> tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Per-row threshold selection |x_rot| >= t: (idx int32 [M, d], val fp32 [M, d],
+    nnz int32 [M]); row m's first nnz[m] entries are the kept ones, ascending."""
+    _need(x_rot, "x_rot", torch.float32)
+    x2 = _as2d(x_rot)
+    M, d = x2.shape
+    dev = x_rot.device
+    if idx is None:
+        idx = torch.empty((M, d), dtype=torch.int32, device=dev)
+    if val is None:
+        val = torch.empty((M, d), dtype=torch.float32, device=dev)
+    if nnz is None:
+        nnz = torch.empty((M,), dtype=torch.int32, device=dev)
+    _need(idx, "idx", torch.int32)
+    _need(val, "val", torch.float32)
+    _need(nnz, "nnz", torch.int32)
+    _check(_lib.larosa_threshold(_ptr(x2), M, d, float(t), _ptr(idx), _ptr(val), _ptr(nnz),
+                                 _status_ptr(dev_status, dev), _stream(dev)), "larosa_threshold")
+    return idx, val, nnz
+
+
+def larosa_rotate_threshold_linear(x: torch.Tensor, Qt: torch.Tensor | None, W_rot: torch.Tensor,
+                                   t: float, y: torch.Tensor | None = None, ws=None,
+                                   dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """Fused rotate -> threshold |x_rot| >= t -> sparse linear, fp32 output [M, d_out].
+
+    Qt = None is the identity rotation.  The kept lists and counts stay in the
+    workspace (larosa_workspace_layout / larosa_workspace_nnz_offset with K = d_in)."""
+    _need(x, "x")
+    if Qt is not None:
+        _need(Qt, "Qt", x.dtype)
+    _need(W_rot, "W_rot", x.dtype)
+    x2 = _as2d(x)
+    M, d_in = x2.shape
+    d_out = W_rot.shape[1]
+    if y is None:
+        y = torch.empty((M, d_out), dtype=torch.float32, device=x.device)
+    _need(y, "y", torch.float32)
+    p, n = _ws_args(ws, x.device, M, d_in, d_out, d_in)
+    _check(_lib.larosa_rotate_threshold_linear(_ptr(x2), _ptr(Qt), _ptr(W_rot), M, d_in, d_out, float(t),
+                                               _ptr(y), p, n, _status_ptr(dev_status, x.device),
+                                               _dtype_code(x), _stream(x.device)),
+           "larosa_rotate_threshold_linear")
     return y
 
 

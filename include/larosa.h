@@ -191,7 +191,10 @@ int larosa_sparse_linear(const int32_t *idx, const float *val, int M, int K,
  *   x_rot = x . Q;  (idx, val) = TopK(x_rot, K);  y = sparse(x_rot) . W_rot.
  * x: [M x d_in] of `dtype`; Qt = Q^T: [d_in x d_in]; W_rot: [d_in x d_out] of
  * `dtype` (from larosa_prepare_weights with the same Qt); y: [M x d_out] fp32.
- * For one token this is one cooperative kernel: every CTA rotates a share
+ * Qt = NULL selects the identity rotation (x_rot = x widened to fp32, W_rot
+ * the plain weight): the unrotated fixed-K mode, for comparison with the
+ * magnitude-pruning methods the La RoSA abstract compares against (TEAL,
+ * CATS).  For one token this is one cooperative kernel: every CTA rotates a share
  * of x, a selector CTA finds the K-th entry, and the rest stream the kept
  * rows of W_rot by column tiles (when the grid cannot be made resident it
  * falls back to larosa_rotate_topk's kernel followed by the one-token
@@ -210,6 +213,44 @@ int larosa_rotate_topk_linear(const void *x, const void *Qt, const void *W_rot,
                               int M, int d_in, int d_out, int K, float *y,
                               void *ws, size_t ws_bytes, int *dev_status,
                               int dtype, larosa_stream_t stream);
+
+/*
+ * Threshold selection (R-Sparse report, 研究流程与方法 / R-Sparse框架设计: the
+ * input channels with |x_j| >= t are kept, the rest masked; the count kept
+ * varies from token to token):
+ *   nnz[m] = |S_m|,  S_m = { i : |x_rot[m][i]| >= t }.
+ * x_rot: [M x d] fp32.  idx/val: [M x d]; row m's first nnz[m] entries
+ * receive S_m in ascending index order and the kept values, the rest of the
+ * row is left as it was.  nnz: [M] int32.  Magnitudes are compared exactly
+ * (+0 and -0 are equal); t <= 0 keeps every entry, t = +Inf only infinite
+ * ones; t = NaN returns LAROSA_ERR_INVALID_ARG.  A NaN or Inf in x_rot sets
+ * LAROSA_DEV_NONFINITE.  One CTA per token.
+ */
+int larosa_threshold(const float *x_rot, int M, int d, float t, int32_t *idx,
+                     float *val, int32_t *nnz, int *dev_status,
+                     larosa_stream_t stream);
+
+/*
+ * Rotation, threshold selection and sparse linear in one call (the
+ * threshold function sigma_t of the R-Sparse report in place of the Top-K):
+ *   x_rot = x . Q;  S_m = { i : |x_rot[m][i]| >= t };
+ *   y[m] = sum_{i in S_m} x_rot[m][i] * W_rot[i].
+ * Arguments as for larosa_rotate_topk_linear, with t in place of K (Qt =
+ * NULL again selects the identity rotation, the TEAL/CATS-style mode).  For
+ * one token one cooperative kernel as for the Top-K (no selection step: the
+ * gather CTAs stream their kept rows as soon as every CTA has rotated);
+ * otherwise rotation, larosa_threshold's kernel and the row-streaming sparse
+ * linear over the kept rows (for M > 1 over the union of the tokens' sets).
+ * ws: at least larosa_workspace_bytes(M, d_in, d_out, d_in) bytes; x_rot,
+ * idx and val ([M x d_in] each, as larosa_threshold writes them) lie at the
+ * offsets larosa_workspace_layout(M, d_in, d_out, d_in, ...) gives and nnz
+ * at larosa_workspace_nnz_offset(M, d_in, d_out, d_in, ...).
+ */
+int larosa_rotate_threshold_linear(const void *x, const void *Qt,
+                                   const void *W_rot, int M, int d_in,
+                                   int d_out, float t, float *y, void *ws,
+                                   size_t ws_bytes, int *dev_status, int dtype,
+                                   larosa_stream_t stream);
 
 /*
  * Dense baseline: y[m][j] = sum_i x[m][i] * Wt[j][i], i.e. y = x . W for the
@@ -266,6 +307,13 @@ size_t larosa_workspace_bytes(int M, int d_in, int d_out, int K);
 int larosa_workspace_layout(int M, int d_in, int d_out, int K,
                             size_t *x_rot_offset, size_t *idx_offset,
                             size_t *val_offset);
+
+/*
+ * Byte offset inside the workspace of the threshold call's kept counts
+ * (nnz, [M] int32).  Returns LAROSA_ERR_SHAPE for out-of-range sizes.
+ */
+int larosa_workspace_nnz_offset(int M, int d_in, int d_out, int K,
+                                size_t *nnz_offset);
 
 /*
  * Waits for `stream`, reads *dev_status (device pointer) and returns

@@ -33,7 +33,7 @@ def test_header_declares_the_entry_points():
     for must in ("larosa_prepare_weights", "larosa_rotate", "larosa_topk", "larosa_rotate_topk",
                  "larosa_sparse_linear",
                  "larosa_rotate_topk_linear", "larosa_dense_linear", "larosa_workspace_bytes",
-                 "larosa_check"):
+                 "larosa_threshold", "larosa_rotate_threshold_linear", "larosa_check"):
         assert must in names
 
 
@@ -102,6 +102,27 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.larosa_rotate_topk(FAKE, FAKE, FAKE, FAKE, FAKE, 32776, 3, FAKE, z, None, BF16, None) == 2
     assert lib.larosa_rotate_topk(FAKE, FAKE, MISALIGNED, FAKE, FAKE, 64, 3, FAKE, z, None, BF16, None) == 3
     assert lib.larosa_rotate_topk(FAKE, FAKE, FAKE, FAKE, FAKE, 60, 3, FAKE, z, None, BF16, None) == 3
+    # threshold selection and the threshold path (t is a float; NaN is refused)
+    f = ctypes.c_float
+    nan = f(float("nan"))
+    assert lib.larosa_threshold(None, 1, 64, f(0.5), FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.larosa_threshold(FAKE, 1, 64, f(0.5), FAKE, FAKE, None, None, None) == 1
+    assert lib.larosa_threshold(FAKE, 1, 64, nan, FAKE, FAKE, FAKE, None, None) == 1
+    assert lib.larosa_threshold(FAKE, 0, 64, f(0.5), FAKE, FAKE, FAKE, None, None) == 2
+    assert lib.larosa_threshold(FAKE, 1, 32769, f(0.5), FAKE, FAKE, FAKE, None, None) == 2
+    rtl = lib.larosa_rotate_threshold_linear
+    assert rtl(FAKE, FAKE, FAKE, 1, 64, 64, f(0.5), FAKE, FAKE, z, None, 7, None) == 4
+    assert rtl(None, FAKE, FAKE, 1, 64, 64, f(0.5), FAKE, FAKE, z, None, BF16, None) == 1
+    assert rtl(FAKE, FAKE, FAKE, 1, 64, 64, nan, FAKE, FAKE, z, None, BF16, None) == 1
+    assert rtl(FAKE, FAKE, FAKE, 17, 64, 64, f(0.5), FAKE, FAKE, z, None, BF16, None) == 2
+    assert rtl(FAKE, FAKE, FAKE, 1, 64, 12, f(0.5), FAKE, FAKE, z, None, BF16, None) == 3
+    assert rtl(MISALIGNED, None, FAKE, 1, 64, 64, f(0.5), FAKE, FAKE, z, None, BF16, None) == 3
+    assert rtl(FAKE, None, FAKE, 1, 60, 64, f(0.5), FAKE, FAKE, z, None, BF16, None) == 3
+    # the identity rotation (no Qt) is checked like the rotated path
+    assert lib.larosa_rotate_topk_linear(MISALIGNED, None, FAKE, 1, 64, 64, 5, FAKE, FAKE, z, None, BF16, None) == 3
+    assert lib.larosa_rotate_topk_linear(FAKE, None, FAKE, 1, 64, 64, 65, FAKE, FAKE, z, None, BF16, None) == 2
+    off = ctypes.c_size_t()
+    assert lib.larosa_workspace_nnz_offset(1, 64, 64, 65, ctypes.byref(off)) == 2
     # in-place counter-rotation is refused
     assert lib.larosa_prepare_weights(FAKE, P(0x20000), P(0x20000), 64, 64, BF16, None) == 1
     # status check needs a status word

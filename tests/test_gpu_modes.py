@@ -1,0 +1,215 @@
+"""Parity of the comparison modes with the fp64 oracle, through the C ABI:
+
+* threshold selection |x| >= t (R-Sparse report, R-Sparse框架设计): the kept
+  lists and counts bit-exact on given fp32 rows, including ties at t, +-0,
+  subnormals, t <= 0 and t = +Inf;
+* the fused rotate -> threshold -> sparse linear call (one token: the
+  cooperative kernel in threshold mode; several tokens: the composed path);
+* the identity rotation (no Q): fixed-K and threshold selection on x itself,
+  where the selection is exact because x_rot = x.
+
+Bars as in test_gpu_parity: x_rot within the fp32 summation bound of the
+exact rotation, the kept set exactly the selection of the path's own fp32
+x_rot and valid against the exact rotation outside a band of the bound's
+width around t, y within 2e-3 of the oracle's product on that set.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthdata as sd
+from tests.test_gpu_parity import U, Y_TOL, check_selection, f64, rel_inf, status
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def L():
+    from activation_sparsity_b200 import build_lib
+    build_lib.build()
+    import activation_sparsity_b200 as L
+    torch.cuda.init()
+    return L
+
+
+def f32(v: float) -> float:
+    return float(np.float32(v))
+
+
+# ---------------------------------------------------------------- threshold selection
+
+SIZES = [(1, 1), (3, 7), (2, 256), (4, 1000), (1, 4096), (2, 11008), (1, 32768), (16, 512)]
+
+
+def thresholds(x: np.ndarray) -> list[float]:
+    mag = np.abs(x[0])
+    srt = np.sort(mag)
+    mid = srt[len(srt) // 2]  # an exact magnitude of the row: a tie at t
+    return sorted({0.0, -1.0, f32(mid), f32(srt[-1]), f32(mid * 1.0000001), float("inf"), 1e-40, 1e30})
+
+
+@pytest.mark.parametrize("kind", sd.ADVERSARIAL_KINDS)
+@pytest.mark.parametrize("M,d", SIZES)
+def test_threshold_bit_exact(L, kind, M, d):
+    x = sd.adversarial_rows(kind, M, d, 700 + d)
+    xd = x.cuda()
+    xn = x.double().numpy()
+    for t in thresholds(xn):
+        st = status()
+        idx, val, nnz = L.larosa_threshold(xd, t, dev_status=st)
+        assert L.larosa_check(st) == 0
+        want = oracle.threshold_select(xn, f32(t))
+        n = nnz.cpu().numpy()
+        gi = idx.cpu().numpy()
+        gv = val.cpu().numpy()
+        for m in range(M):
+            wi, wv = want[m]
+            assert n[m] == len(wi), (kind, d, t)
+            assert np.array_equal(gi[m, :n[m]], wi), (kind, d, t)
+            assert np.array_equal(gv[m, :n[m]].view(np.uint32), wv.astype(np.float32).view(np.uint32))
+
+
+def test_threshold_reports_nonfinite(L):
+    x = sd.adversarial_rows("gaussian", 2, 300, 5)
+    x[1, 17] = float("nan")
+    st = status()
+    _, _, nnz = L.larosa_threshold(x.cuda(), 0.5, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & 0x1
+    assert 0 <= int(nnz[1].item()) <= 300
+
+
+# ---------------------------------------------------------------- fused threshold path
+
+def threshold_outputs(L, x, Qt, W, t):
+    M, d_in = x.shape
+    d_out = W.shape[1]
+    ws = L.Workspace()
+    buf = ws.get(M, d_in, d_out, d_in)
+    st = status()
+    y = L.larosa_rotate_threshold_linear(x, Qt, W, t, ws=ws, dev_status=st)
+    assert L.larosa_check(st) == 0
+    o_x, o_i, o_v = L.larosa_workspace_layout(M, d_in, d_out, d_in)
+    o_n = L.larosa_workspace_nnz_offset(M, d_in, d_out, d_in)
+    x_rot = buf[o_x:o_x + M * d_in * 4].view(torch.float32).view(M, d_in)
+    idx = buf[o_i:o_i + M * d_in * 4].view(torch.int32).view(M, d_in)
+    val = buf[o_v:o_v + M * d_in * 4].view(torch.float32).view(M, d_in)
+    nnz = buf[o_n:o_n + M * 4].view(torch.int32)
+    return (f64(y), f64(x_rot), idx.cpu().numpy().astype(np.int64), val.cpu().numpy(),
+            nnz.cpu().numpy().astype(np.int64))
+
+
+def check_threshold_path(x_rot, x_rot_ref, gamma, idx, val, nnz, t):
+    M, d = x_rot.shape
+    for m in range(M):
+        # exactly the threshold selection of the path's own fp32 x_rot
+        (wi, wv), = oracle.threshold_select(x_rot[m], t)
+        assert nnz[m] == len(wi)
+        assert np.array_equal(idx[m, :nnz[m]], wi)
+        assert np.array_equal(val[m, :nnz[m]], wv.astype(np.float32))
+        # against the exact rotation: only entries within the bound of t may differ
+        kept = np.zeros(d, dtype=bool)
+        kept[wi] = True
+        mag = np.abs(x_rot_ref[m])
+        assert np.all(kept[mag >= t + gamma[m] + 1e-30])
+        assert not np.any(kept[mag < t - gamma[m] - 1e-30])
+
+
+@pytest.mark.parametrize("dtype,M,d_in,d_out,drop", [
+    (torch.float32, 1, 256, 512, 40),
+    (torch.bfloat16, 1, 1024, 1032, 40),
+    (torch.bfloat16, 1, 4096, 4096, 40),
+    (torch.bfloat16, 1, 11008, 4096, 50),
+    (torch.bfloat16, 1, 200, 24, 50),
+    (torch.bfloat16, 4, 1024, 1032, 40),
+    (torch.bfloat16, 16, 512, 256, 25),
+    (torch.bfloat16, 1, 1024, 1032, 0),
+    (torch.bfloat16, 1, 1024, 1032, 100),
+])
+def test_fused_threshold(L, dtype, M, d_in, d_out, drop):
+    Q = sd.orthogonal(d_in, 801, device="cuda" if d_in > 4096 else "cpu").to(dtype).cpu()
+    W = sd.weights(d_in, d_out, 0.02 if dtype == torch.bfloat16 else 1 / 16, 802, dtype)
+    x = sd.activations(M, d_in, 803, dtype)
+    Qt = Q.t().contiguous().cuda()
+    W_rot = L.larosa_prepare_weights(Qt, W.cuda())
+    xq, qq = f64(x), f64(Q)
+    x_rot_ref = oracle.rotate(xq, qq)
+    gamma = (d_in + 2) * U * (np.abs(xq) @ np.abs(qq))
+    # t drops about drop % of the first token's exact magnitudes (0: t = 0, 100: t = +Inf)
+    mag = np.sort(np.abs(x_rot_ref[0]))
+    t = 0.0 if drop == 0 else float("inf") if drop == 100 else f32(mag[int(len(mag) * drop / 100)])
+    y, x_rot, idx, val, nnz = threshold_outputs(L, x.cuda(), Qt, W_rot, t)
+    assert np.all(np.abs(x_rot - x_rot_ref) <= gamma + 1e-30)
+    check_threshold_path(x_rot, x_rot_ref, gamma, idx, val, nnz, t)
+    W_rot_ref = oracle.prepare_weights(qq, f64(W))
+    if dtype == torch.bfloat16:
+        W_rot_ref = oracle.round_to_bf16(W_rot_ref)
+    ref = np.stack([oracle.sparse_linear(idx[m, :nnz[m]], x_rot_ref[m, idx[m, :nnz[m]]], W_rot_ref)
+                    for m in range(M)])
+    if drop == 100:
+        assert np.all(y == 0.0) and np.all(nnz == 0)
+    else:
+        assert rel_inf(y, ref) <= Y_TOL
+
+
+# ---------------------------------------------------------------- the identity rotation
+
+@pytest.mark.parametrize("dtype,M,d_in,d_out,sparsity", [
+    (torch.float32, 1, 256, 512, 40),
+    (torch.bfloat16, 1, 200, 24, 50),
+    (torch.bfloat16, 1, 4096, 4096, 40),
+    (torch.bfloat16, 1, 11008, 4096, 40),
+    (torch.bfloat16, 4, 1024, 1032, 40),
+])
+def test_fused_identity_topk(L, dtype, M, d_in, d_out, sparsity):
+    K = sd.k_for_sparsity(d_in, sparsity)
+    W = sd.weights(d_in, d_out, 0.02 if dtype == torch.bfloat16 else 1 / 16, 902, dtype)
+    x = sd.activations(M, d_in, 903, dtype)
+    ws = L.Workspace()
+    buf = ws.get(M, d_in, d_out, K)
+    st = status()
+    y = L.larosa_rotate_topk_linear(x.cuda(), None, W.cuda(), K, ws=ws, dev_status=st)
+    assert L.larosa_check(st) == 0
+    o_x, o_i, o_v = L.larosa_workspace_layout(M, d_in, d_out, K)
+    x_rot = f64(buf[o_x:o_x + M * d_in * 4].view(torch.float32).view(M, d_in))
+    idx = buf[o_i:o_i + M * K * 4].view(torch.int32).view(M, K).cpu().numpy().astype(np.int64)
+    xq = f64(x)
+    # the identity rotation: x_rot is x itself, so the selection is exact
+    assert np.array_equal(x_rot, xq)
+    want_i, want_v = oracle.topk(xq, K)
+    assert np.array_equal(idx, want_i.reshape(M, K))
+    ref = np.stack([oracle.sparse_linear(want_i.reshape(M, K)[m], want_v.reshape(M, K)[m], f64(W))
+                    for m in range(M)])
+    assert rel_inf(f64(y), ref) <= Y_TOL
+
+
+@pytest.mark.parametrize("dtype,M,d_in,d_out", [
+    (torch.bfloat16, 1, 4096, 4096),
+    (torch.bfloat16, 1, 11008, 4096),
+    (torch.bfloat16, 4, 1024, 1032),
+])
+def test_fused_identity_threshold(L, dtype, M, d_in, d_out):
+    W = sd.weights(d_in, d_out, 0.02, 912, dtype)
+    x = sd.activations(M, d_in, 913, dtype)
+    xq = f64(x)
+    t = f32(np.sort(np.abs(xq[0]))[int(0.4 * d_in)])
+    y, x_rot, idx, val, nnz = threshold_outputs(L, x.cuda(), None, W.cuda(), t)
+    assert np.array_equal(x_rot, xq)
+    want = oracle.threshold_select(xq, t)
+    for m in range(M):
+        wi, wv = want[m]
+        assert nnz[m] == len(wi) and np.array_equal(idx[m, :nnz[m]], wi)
+    ref = np.stack([oracle.sparse_linear(want[m][0], want[m][1], f64(W)) for m in range(M)])
+    assert rel_inf(y, ref) <= Y_TOL
+
+
+def test_identity_topk_matches_rotated_path_with_identity_q(L):
+    """Qt = NULL and an explicit identity Qt select the same set and give the same y."""
+    d_in, d_out, K = 1024, 1032, 600
+    W = sd.weights(d_in, d_out, 0.02, 922, torch.bfloat16).cuda()
+    x = sd.activations(1, d_in, 923, torch.bfloat16).cuda()
+    eye = torch.eye(d_in, dtype=torch.bfloat16, device="cuda")
+    y0 = L.larosa_rotate_topk_linear(x, None, W, K)
+    y1 = L.larosa_rotate_topk_linear(x, eye, L.larosa_prepare_weights(eye, W), K)
+    assert rel_inf(f64(y0), f64(y1)) <= 1e-6
