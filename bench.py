@@ -308,6 +308,7 @@ def bench_larosa(args):
     init_dist(world, "nccl")
 
     import activation_sparsity_b200 as L
+    import synthdata as sd
     from activation_sparsity_b200.workload import build_layer
 
     layer = build_layer(HIDDEN, FFN, KV, args.sparsity, WORKLOAD_ID, layer=rank, device=device)
@@ -352,6 +353,21 @@ def bench_larosa(args):
         for g, y in zip(groups, ys):
             L.larosa_dense_linear(g.x, g.Wt, y=y)
 
+    # comparison modes: the unrotated fixed-K path (Q = I, plain weight) and the
+    # threshold selection |x_rot| >= t, rotated and unrotated, with t set per
+    # group from this token's own magnitudes so that the same share is dropped
+    def unrot_topk_step():
+        for g, y in zip(groups, ys):
+            L.larosa_rotate_topk_linear(g.x, None, g.W, g.K, y=y, ws=ws, dev_status=st)
+
+    def rot_thr_step():
+        for gi, (g, y) in enumerate(zip(groups, ys)):
+            L.larosa_rotate_threshold_linear(g.x, g.Qt, g.W_rot, t_rot[gi], y=y, ws=ws, dev_status=st)
+
+    def unrot_thr_step():
+        for gi, (g, y) in enumerate(zip(groups, ys)):
+            L.larosa_rotate_threshold_linear(g.x, None, g.W, t_x[gi], y=y, ws=ws, dev_status=st)
+
     def graph_of(fn):
         with torch.cuda.stream(stream):
             for _ in range(3):
@@ -388,6 +404,20 @@ def bench_larosa(args):
         topk_step()
     torch.cuda.synchronize(device)
 
+    def calibrate(mag: torch.Tensor, d: int) -> tuple[float, int]:
+        """t = the magnitude below which the sparsity's share of entries lies; kept count."""
+        srt = torch.sort(mag.flatten().float()).values
+        t = float(srt[d - sd.k_for_sparsity(d, args.sparsity)].item())
+        return t, int((mag >= t).sum().item())
+    t_rot, nnz_rot, t_x, nnz_x = [], [], [], []
+    for gi, g in enumerate(groups):
+        t, n = calibrate(x_rots[gi].abs(), g.d_in)
+        t_rot.append(t)
+        nnz_rot.append(n)
+        t, n = calibrate(g.x.float().abs(), g.d_in)
+        t_x.append(t)
+        nnz_x.append(n)
+
     g_fused = graph_of(fused_step)
     g_sparse = graph_of(sparse_only_step)
     g_dense = graph_of(dense_step)
@@ -395,6 +425,9 @@ def bench_larosa(args):
     g_rotsel = graph_of(rotate_topk_step)
     g_topk = graph_of(topk_step)
     g_gather = graph_of(gather_step)
+    g_unrot_topk = graph_of(unrot_topk_step)
+    g_rot_thr = graph_of(rot_thr_step)
+    g_unrot_thr = graph_of(unrot_thr_step)
 
     props = torch.cuda.get_device_properties(device)
     clocks = ClockSampler(f"GPU-{props.uuid}")
@@ -411,6 +444,9 @@ def bench_larosa(args):
     t_rotsel, _ = time_graph(g_rotsel, args.steps, args.warmup)
     t_topk, _ = time_graph(g_topk, args.steps, args.warmup)
     t_gather, _ = time_graph(g_gather, args.steps, args.warmup)
+    t_unrot_topk, _ = time_graph(g_unrot_topk, args.steps, args.warmup)
+    t_rot_thr, _ = time_graph(g_rot_thr, args.steps, args.warmup)
+    t_unrot_thr, _ = time_graph(g_unrot_thr, args.steps, args.warmup)
     n_launch = args.steps * len(groups)
     rot_us = t_rot / n_launch * 1e6
     rotsel_us = t_rotsel / n_launch * 1e6
@@ -425,6 +461,9 @@ def bench_larosa(args):
     step_bytes = sum(path_bytes(g, g.K)["total"] for g in groups)
     sparse_bytes = sum(path_bytes(g, g.K, rotate=False)["total"] for g in groups)
     dense_bytes = sum(g.d_in * g.d_out * 2 + g.d_in * 2 + g.d_out * 4 for g in groups)
+    unrot_topk_bytes = sum(path_bytes(g, g.K, rotate=False)["total"] for g in groups)
+    rot_thr_bytes = sum(path_bytes(g, n)["total"] for g, n in zip(groups, nnz_rot))
+    unrot_thr_bytes = sum(path_bytes(g, n, rotate=False)["total"] for g, n in zip(groups, nnz_x))
     peak, peak_kind = measured_peaks()
     rot_gbs = sum(rot_bytes) * args.steps / t_rot / 1e9
     rotsel_gbs = sum(rotsel_bytes) * args.steps / t_rotsel / 1e9
@@ -505,16 +544,25 @@ def bench_larosa(args):
                 "gather_only_tokens_per_s": args.steps / t_gather * world,
                 "gather_only_vs_dense": (args.steps / t_gather * world) / dense_tps,
                 "fused_vs_dense": value / dense_tps,
+                # comparison modes, each one call per group through the public API
+                "unrotated_topk_tokens_per_s": args.steps / t_unrot_topk * world,
+                "unrotated_topk_hbm_frac": unrot_topk_bytes * args.steps / t_unrot_topk / 1e9 / peak,
+                "rotated_threshold_tokens_per_s": args.steps / t_rot_thr * world,
+                "rotated_threshold_hbm_frac": rot_thr_bytes * args.steps / t_rot_thr / 1e9 / peak,
+                "rotated_threshold_kept_frac": sum(nnz_rot) / sum(g.d_in for g in groups),
+                "unrotated_threshold_tokens_per_s": args.steps / t_unrot_thr * world,
+                "unrotated_threshold_hbm_frac": unrot_thr_bytes * args.steps / t_unrot_thr / 1e9 / peak,
+                "unrotated_threshold_kept_frac": sum(nnz_x) / sum(g.d_in for g in groups),
             },
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": sum(g.x.numel() * g.x.element_size() for g in groups),
                     "d2h_bytes_per_step": sum(g.d_out * 4 for g in groups)},
-            "gpu_launches": args.steps * 2 * len(groups),
+            "gpu_launches": args.steps * len(groups),  # one fused_kernel per group and step
             "clocks": clk,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    del g_fused, g_sparse, g_dense, g_rot, g_rotsel, g_topk, g_gather
+    del g_fused, g_sparse, g_dense, g_rot, g_rotsel, g_topk, g_gather, g_unrot_topk, g_rot_thr, g_unrot_thr
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
