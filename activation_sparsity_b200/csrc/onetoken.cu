@@ -203,9 +203,9 @@ __host__ __device__ inline GLayout glayout(int list_cap, int col_tile, int cpt) 
 
 // Streams rows lrows[lo, hi) of one column tile (columns [c0, c0 + wc) of a
 // row-major [* x d_out] weight), scaled by lvals, into this thread's acc.
-// Thread (g, col) reads 16 bytes of rows lo + g, lo + g + ng, ... with kU
+// Thread (g, col) reads 16 bytes of rows lo + g, lo + g + ng, ... with NU
 // loads in flight.
-template <typename Tw>
+template <typename Tw, int NU = kU>
 __device__ __forceinline__ void accumulate_rows(const void* W, int d_out, int c0, int wc, int tpr,
                                                 const int32_t* lrows, const float* lvals, int lo,
                                                 int hi, float (&acc)[16 / sizeof(Tw)]) {
@@ -217,15 +217,15 @@ __device__ __forceinline__ void accumulate_rows(const void* W, int d_out, int c0
   if (g >= ng || col >= wc) return;
   const unsigned char* wbase = static_cast<const unsigned char*>(W) + ((size_t)c0 + col) * sizeof(Tw);
   const size_t pitch = (size_t)d_out * sizeof(Tw);
-  for (int r0 = lo + g; r0 < hi; r0 += ng * kU) {
-    uint4 u[kU];
+  for (int r0 = lo + g; r0 < hi; r0 += ng * NU) {
+    uint4 u[NU];
 #pragma unroll
-    for (int k = 0; k < kU; ++k) {
+    for (int k = 0; k < NU; ++k) {
       const int r = r0 + k * ng;
       u[k] = r < hi ? ld_stream(wbase + (size_t)lrows[r] * pitch) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int k = 0; k < kU; ++k) {
+    for (int k = 0; k < NU; ++k) {
       const int r = r0 + k * ng;
       const float cf = r < hi ? lvals[r] : 0.f;
       if constexpr (CPT == 8) {
@@ -635,6 +635,12 @@ __host__ __device__ inline FLayout flayout(int d, int elem_bytes, int range_cap,
 
 constexpr int kRowKeys = 256;  // rotated rows per CTA whose keys are aggregated in shared memory
 constexpr size_t kQPrefetchBytes = 32 << 10;  // rows of Q per CTA requested into L2 before the wait
+// Weight rows a gather thread of the fused kernel has in flight.  Fewer than
+// the kU of the standalone kernels: the fused kernel's critical path after
+// the arrivals is a chain of L2 round trips (the K-th entry, the tile
+// reduction) that wait behind every load queued on the SM, and four rows
+// per thread (128 KB per SM) already keep HBM streaming.
+constexpr int kFusedU = 4;
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
@@ -1276,7 +1282,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
       if (((rkeys[j] & kKeyMask) >> kFineShift) == B)
         bulk_prefetch_l2(wtile + (size_t)(i_lo + j) * pitch, static_cast<uint32_t>(wc * sizeof(T)));
   }
-  accumulate_rows<T>(p.W, p.d_out, c0, wc, p.tpr, lrows, lvals, 0, n_certain, acc);
+  accumulate_rows<T, kFusedU>(p.W, p.d_out, c0, wc, p.tpr, lrows, lvals, 0, n_certain, acc);
 
   // the K-th entry: the kept rows of bin B
   if (tid == 0) {
@@ -1297,7 +1303,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
       [&](uint32_t k, int i) { return have_kth && (k >> kFineShift) == B && is_kept(k, i, e); },
       lrows, lvals, n_certain, s_warp_sums);
   __syncthreads();  // the list is complete; the range's keys are dead
-  accumulate_rows<T>(p.W, p.d_out, c0, wc, p.tpr, lrows, lvals, n_certain, n_certain + n_more, acc);
+  accumulate_rows<T, kFusedU>(p.W, p.d_out, c0, wc, p.tpr, lrows, lvals, n_certain, n_certain + n_more, acc);
   reduce_tile_last<T, C>(rank, c0, wc, p.col_tile, p.tpr, acc, red,
                          p.partials + (size_t)tile * C * p.col_tile,
                          p.sync + kFusedSyncWords + (gen & 1u) * kFusedMaxTiles + tile, p.y);
