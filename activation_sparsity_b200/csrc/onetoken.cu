@@ -205,6 +205,10 @@ __host__ __device__ inline GLayout glayout(int list_cap, int col_tile, int cpt) 
 // row-major [* x d_out] weight), scaled by lvals, into this thread's acc.
 // Thread (g, col) reads 16 bytes of rows lo + g, lo + g + ng, ... with NU
 // loads in flight.
+// Weight rows a thread of the list-mode gather has in flight (6 measured
+// faster than 8 and 4 on the LLaMA2-7B groups).
+constexpr int kGatherU = 6;
+
 template <typename Tw, int NU = kU>
 __device__ __forceinline__ void accumulate_rows(const void* W, int d_out, int c0, int wc, int tpr,
                                                 const int32_t* lrows, const float* lvals, int lo,
@@ -335,7 +339,7 @@ __device__ __forceinline__ void gather_tile(cg::cluster_group& cl, int rank, con
   float acc[16 / sizeof(Tw)];
 #pragma unroll
   for (int v = 0; v < 16 / (int)sizeof(Tw); ++v) acc[v] = 0.f;
-  accumulate_rows<Tw>(W, d_out, c0, wc, tpr, lrows, lvals, 0, len, acc);
+  accumulate_rows<Tw, kGatherU>(W, d_out, c0, wc, tpr, lrows, lvals, 0, len, acc);
   reduce_tile<Tw, C>(cl, rank, c0, wc, col_tile, tpr, acc, red, part, y);
 }
 
