@@ -338,6 +338,13 @@ int larosa_prepare_weights(const void* Qt, const void* W, void* W_rot, int d_in,
   return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "prepare kernel");
 }
 
+int larosa_fold_rotation(const void* Qt, const void* Wt_prev, void* Wt_prev_rot, int d, int d_prev,
+                         int dtype, larosa_stream_t stream) {
+  // Q^T . Wt_prev is the counter-rotation of larosa_prepare_weights applied
+  // to the producer's [d x d_prev] weight
+  return larosa_prepare_weights(Qt, Wt_prev, Wt_prev_rot, d, d_prev, dtype, stream);
+}
+
 int larosa_rotate(const void* x, const void* Qt, float* x_rot, int M, int d, int dtype,
                   larosa_stream_t stream) {
   if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;

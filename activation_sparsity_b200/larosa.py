@@ -37,6 +37,7 @@ _SIGNATURES = {
     "larosa_version": ([], _i),
     "larosa_last_error_string": ([], _c.c_char_p),
     "larosa_prepare_weights": ([_vp, _vp, _vp, _i, _i, _i, _vp], _i),
+    "larosa_fold_rotation": ([_vp, _vp, _vp, _i, _i, _i, _vp], _i),
     "larosa_rotate": ([_vp, _vp, _vp, _i, _i, _i, _vp], _i),
     "larosa_topk": ([_vp, _i, _i, _i, _vp, _vp, _vp, _vp], _i),
     "larosa_rotate_topk": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _sz, _vp, _i, _vp], _i),
@@ -219,6 +220,21 @@ def larosa_prepare_weights(Qt: torch.Tensor, W: torch.Tensor, W_rot: torch.Tenso
     _check(_lib.larosa_prepare_weights(_ptr(Qt), _ptr(W), _ptr(W_rot), d_in, d_out, _dtype_code(W),
                                        _stream(W.device)), "larosa_prepare_weights")
     return W_rot
+
+
+def larosa_fold_rotation(Qt: torch.Tensor, Wt_prev: torch.Tensor, out: torch.Tensor | None = None
+                         ) -> torch.Tensor:
+    """Q^T . Wt_prev: the producer's nn.Linear weight [d, d_prev] after folding the
+    rotation into it, so that the producer outputs x . Q."""
+    _need(Qt, "Qt")
+    _need(Wt_prev, "Wt_prev", Qt.dtype)
+    d, d_prev = Wt_prev.shape
+    if out is None:
+        out = torch.empty_like(Wt_prev)
+    _need(out, "out", Wt_prev.dtype)
+    _check(_lib.larosa_fold_rotation(_ptr(Qt), _ptr(Wt_prev), _ptr(out), d, d_prev, _dtype_code(Wt_prev),
+                                     _stream(Wt_prev.device)), "larosa_fold_rotation")
+    return out
 
 
 def larosa_rotate(x: torch.Tensor, Qt: torch.Tensor, x_rot: torch.Tensor | None = None

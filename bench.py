@@ -368,6 +368,17 @@ def bench_larosa(args):
         for gi, (g, y) in enumerate(zip(groups, ys)):
             L.larosa_rotate_threshold_linear(g.x, None, g.W, t_x[gi], y=y, ws=ws, dev_status=st)
 
+    # the rotation folded into the producer: the input arrives rotated (as the
+    # producer's bf16 output x . Q) and the call runs with the identity rotation
+    def folded_topk_step():
+        for gi, (g, y) in enumerate(zip(groups, ys)):
+            L.larosa_rotate_topk_linear(x_folded[gi], None, g.W_rot, g.K, y=y, ws=ws, dev_status=st)
+
+    def folded_thr_step():
+        for gi, (g, y) in enumerate(zip(groups, ys)):
+            L.larosa_rotate_threshold_linear(x_folded[gi], None, g.W_rot, t_rot[gi], y=y, ws=ws,
+                                             dev_status=st)
+
     def graph_of(fn):
         with torch.cuda.stream(stream):
             for _ in range(3):
@@ -409,6 +420,7 @@ def bench_larosa(args):
         srt = torch.sort(mag.flatten().float()).values
         t = float(srt[d - sd.k_for_sparsity(d, args.sparsity)].item())
         return t, int((mag >= t).sum().item())
+    x_folded = [xr.to(torch.bfloat16) for xr in x_rots]
     t_rot, nnz_rot, t_x, nnz_x = [], [], [], []
     for gi, g in enumerate(groups):
         t, n = calibrate(x_rots[gi].abs(), g.d_in)
@@ -428,6 +440,8 @@ def bench_larosa(args):
     g_unrot_topk = graph_of(unrot_topk_step)
     g_rot_thr = graph_of(rot_thr_step)
     g_unrot_thr = graph_of(unrot_thr_step)
+    g_folded_topk = graph_of(folded_topk_step)
+    g_folded_thr = graph_of(folded_thr_step)
 
     props = torch.cuda.get_device_properties(device)
     clocks = ClockSampler(f"GPU-{props.uuid}")
@@ -447,6 +461,8 @@ def bench_larosa(args):
     t_unrot_topk, _ = time_graph(g_unrot_topk, args.steps, args.warmup)
     t_rot_thr, _ = time_graph(g_rot_thr, args.steps, args.warmup)
     t_unrot_thr, _ = time_graph(g_unrot_thr, args.steps, args.warmup)
+    t_folded_topk, _ = time_graph(g_folded_topk, args.steps, args.warmup)
+    t_folded_thr, _ = time_graph(g_folded_thr, args.steps, args.warmup)
     n_launch = args.steps * len(groups)
     rot_us = t_rot / n_launch * 1e6
     rotsel_us = t_rotsel / n_launch * 1e6
@@ -553,6 +569,12 @@ def bench_larosa(args):
                 "unrotated_threshold_tokens_per_s": args.steps / t_unrot_thr * world,
                 "unrotated_threshold_hbm_frac": unrot_thr_bytes * args.steps / t_unrot_thr / 1e9 / peak,
                 "unrotated_threshold_kept_frac": sum(nnz_x) / sum(g.d_in for g in groups),
+                # Q folded into the producer: no Q streamed per token
+                "folded_topk_tokens_per_s": args.steps / t_folded_topk * world,
+                "folded_topk_hbm_frac": sparse_bytes * args.steps / t_folded_topk / 1e9 / peak,
+                "folded_topk_vs_dense": (args.steps / t_folded_topk * world) / dense_tps,
+                "folded_threshold_tokens_per_s": args.steps / t_folded_thr * world,
+                "folded_threshold_vs_dense": (args.steps / t_folded_thr * world) / dense_tps,
             },
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": sum(g.x.numel() * g.x.element_size() for g in groups),
@@ -563,6 +585,7 @@ def bench_larosa(args):
         }
         print(json.dumps(line), flush=True)
     del g_fused, g_sparse, g_dense, g_rot, g_rotsel, g_topk, g_gather, g_unrot_topk, g_rot_thr, g_unrot_thr
+    del g_folded_topk, g_folded_thr
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -133,6 +133,25 @@ int larosa_prepare_weights(const void *Qt, const void *W, void *W_rot,
                            larosa_stream_t stream);
 
 /*
+ * Folded rotation (offline): moves the rotation of a layer's input into the
+ * layer that produces it, so that the producer outputs x_rot = x . Q and the
+ * per-token path runs with the identity rotation (larosa_rotate_topk_linear
+ * or larosa_rotate_threshold_linear with Qt = NULL) and without streaming Q.
+ * For a producer x = h . Wt_prev^T whose weight is given in torch.nn.Linear
+ * layout Wt_prev [d x d_prev] (one row per output channel):
+ *   Wt_prev_rot[i][j] = sum_k Qt[i][k] * Wt_prev[k][j],  i.e. Q^T . Wt_prev,
+ * which is the nn.Linear weight of the producer of x . Q, since
+ * h . (Q^T . Wt_prev)^T = (h . Wt_prev^T) . Q.  The pages leave open where
+ * the rotation is applied; folding is exact only where nothing nonlinear
+ * lies between the producer's product and the rotated input.  Same kernel
+ * and rounding as larosa_prepare_weights (fp32 accumulation, bf16 rounded
+ * to nearest even); Qt: [d x d], Wt_prev, Wt_prev_rot: [d x d_prev].
+ */
+int larosa_fold_rotation(const void *Qt, const void *Wt_prev,
+                         void *Wt_prev_rot, int d, int d_prev, int dtype,
+                         larosa_stream_t stream);
+
+/*
  * Rotation (step 1): x_rot[m][j] = sum_i x[m][i] * Q[i][j]
  *                                = sum_i x[m][i] * Qt[j][i].
  * x: [M x d] of `dtype`, Qt: [d x d] of `dtype`, x_rot: [M x d] fp32.

@@ -22,6 +22,9 @@ Functions and the passages they follow (page title, section):
                         from Q being orthogonal (x W = (x Q)(Q^T W)).
 * ``dense_linear``      y = x W, the dense layer the method replaces.
 * ``rotate_topk_linear`` the three steps above in the pages' order.
+* ``fold_rotation``     the rotation moved into the producing linear layer
+                        (x . Q delivered by the producer): a reading, since
+                        the pages do not say where Q is applied.
 * ``round_to_bf16``     round-to-nearest-even onto bfloat16 (storage format of
                         the prepared weights; not a step of the method).
 * ``threshold_select``  R-Sparse report, 研究流程与方法 / R-Sparse框架设计
@@ -49,6 +52,7 @@ from .larosa_ref import (  # noqa: F401
     dense_linear,
     prepare_weights,
     rotate_topk_linear,
+    fold_rotation,
     round_to_bf16,
     threshold_select,
     lowrank_factors,

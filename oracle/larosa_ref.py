@@ -114,6 +114,23 @@ def prepare_weights(Q, W) -> np.ndarray:
     return Q.T @ W
 
 
+def fold_rotation(Q, Wt_prev) -> np.ndarray:
+    """The producer's weight with the rotation folded into it.
+
+    Reading (the pages leave open where Q is applied): a layer whose input x
+    is produced by a linear map x = h . Wt_prev^T (Wt_prev [d, d_prev] in
+    torch.nn.Linear layout, one row per output channel) can receive x . Q
+    directly from a producer with weight Wt_fold = Q^T . Wt_prev, because
+    h . Wt_fold^T = h . Wt_prev^T . Q.  Returns Wt_fold [d, d_prev]:
+    Wt_fold[i, j] = sum_k Q[k, i] * Wt_prev[k, j].
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    Wt = np.asarray(Wt_prev, dtype=np.float64)
+    if Q.shape[0] != Q.shape[1] or Q.shape[0] != Wt.shape[0]:
+        raise ValueError("Q must be d x d and Wt_prev d x d_prev")
+    return Q.T @ Wt
+
+
 def rotate_topk_linear(x, Q, W_rot, K: int):
     """The three steps in the pages' order: rotate, keep the Top-K, multiply.
 

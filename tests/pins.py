@@ -203,6 +203,30 @@ def check_prepare_weights(prepare_weights, rotate) -> None:
     np.testing.assert_allclose(rotate(x, Q) @ prepare_weights(Q, W), x @ W, rtol=0, atol=1e-12)
 
 
+def check_fold_rotation(fold_rotation, rotate) -> None:
+    rng = np.random.default_rng(16)
+    d, d_prev = 24, 10
+    Wt = rng.standard_normal((d, d_prev))
+    # the identity rotation leaves the producer unchanged
+    assert np.array_equal(fold_rotation(np.eye(d), Wt), Wt)
+    # a permutation Q[p[i], i] = 1 moves output channel p[i] to position i
+    p = rng.permutation(d)
+    P = np.zeros((d, d))
+    P[p, np.arange(d)] = 1.0
+    assert np.array_equal(fold_rotation(P, Wt), Wt[p])
+    # the folded producer delivers the rotated input: h Wt_fold^T = (h Wt^T) Q
+    Q = haar(d, 22)
+    h = rng.standard_normal((3, d_prev))
+    np.testing.assert_allclose(h @ fold_rotation(Q, Wt).T, rotate(h @ Wt.T, Q), rtol=0, atol=1e-12)
+    # a 2 x 2 Givens rotation by hand: Q = [[c, -s], [s, c]] gives rows
+    # (c w0 + s w1, -s w0 + c w1)
+    c, sn = 0.6, 0.8
+    G = np.array([[c, -sn], [sn, c]])
+    w = np.array([[1.0, 2.0], [3.0, -1.0]])
+    np.testing.assert_allclose(fold_rotation(G, w), [[c * 1 + sn * 3, c * 2 + sn * -1],
+                                                      [-sn * 1 + c * 3, -sn * 2 + c * -1]], rtol=0, atol=1e-15)
+
+
 def check_round_to_bf16(round_to_bf16) -> None:
     import torch
     rng = np.random.default_rng(4)

@@ -123,6 +123,10 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.larosa_rotate_topk_linear(FAKE, None, FAKE, 1, 64, 64, 65, FAKE, FAKE, z, None, BF16, None) == 2
     off = ctypes.c_size_t()
     assert lib.larosa_workspace_nnz_offset(1, 64, 64, 65, ctypes.byref(off)) == 2
+    # folding the rotation into a producer is validated as the counter-rotation
+    assert lib.larosa_fold_rotation(FAKE, None, FAKE, 64, 64, BF16, None) == 1
+    assert lib.larosa_fold_rotation(FAKE, FAKE, FAKE, 64, 64, 9, None) == 4
+    assert lib.larosa_fold_rotation(FAKE, FAKE, FAKE, 0, 64, BF16, None) == 2
     # in-place counter-rotation is refused
     assert lib.larosa_prepare_weights(FAKE, P(0x20000), P(0x20000), 64, 64, BF16, None) == 1
     # status check needs a status word

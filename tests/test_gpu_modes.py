@@ -213,3 +213,44 @@ def test_identity_topk_matches_rotated_path_with_identity_q(L):
     y0 = L.larosa_rotate_topk_linear(x, None, W, K)
     y1 = L.larosa_rotate_topk_linear(x, eye, L.larosa_prepare_weights(eye, W), K)
     assert rel_inf(f64(y0), f64(y1)) <= 1e-6
+
+
+# ---------------------------------------------------------------- folded rotation
+
+@pytest.mark.parametrize("d_prev,d,d_out", [(1024, 4096, 4096), (4096, 11008, 4096)])
+def test_folded_rotation_path(L, d_prev, d, d_out):
+    """Q folded into the producing layer; the consumer runs with the identity rotation."""
+    from tests.test_gpu_parity import check_bf16_rounding
+    K = sd.k_for_sparsity(d, 40.0)
+    Q = sd.orthogonal(d, 951, device="cuda" if d > 4096 else "cpu").to(torch.bfloat16).cpu()
+    Qt = Q.t().contiguous().cuda()
+    Wt_prev = sd.weights(d, d_prev, 0.02, 952, torch.bfloat16)  # producer, nn.Linear layout [d, d_prev]
+    W = sd.weights(d, d_out, 0.02, 953, torch.bfloat16)
+    h = sd.activations(1, d_prev, 954, torch.bfloat16)
+    # offline: fold Q into the producer, counter-rotate the consumer
+    Wt_fold = L.larosa_fold_rotation(Qt, Wt_prev.cuda())
+    W_rot = L.larosa_prepare_weights(Qt, W.cuda())
+    qq, wp = f64(Q), f64(Wt_prev)
+    exact_fold = oracle.fold_rotation(qq, wp)
+    cols = np.random.default_rng(955).choice(d_prev, size=32, replace=False)
+    check_bf16_rounding(f64(Wt_fold)[:, cols], exact_fold[:, cols],
+                        (d + 2) * U * (np.abs(qq).T @ np.abs(wp[:, cols])))
+    # per token: the producer emits x . Q (rounded to bf16, as a layer output)
+    x_rot = L.larosa_dense_linear(h.cuda(), Wt_fold).to(torch.bfloat16)
+    ws = L.Workspace()
+    buf = ws.get(1, d, d_out, K)
+    st = status()
+    y = L.larosa_rotate_topk_linear(x_rot, None, W_rot, K, ws=ws, dev_status=st)
+    assert L.larosa_check(st) == 0
+    _, o_i, _ = L.larosa_workspace_layout(1, d, d_out, K)
+    idx = buf[o_i:o_i + K * 4].view(torch.int32).cpu().numpy().astype(np.int64)
+    xr = f64(x_rot)[0]
+    want_i, want_v = oracle.topk(xr, K)
+    assert np.array_equal(idx, want_i)
+    W_rot_ref = oracle.round_to_bf16(oracle.prepare_weights(qq, f64(W)))
+    assert rel_inf(f64(y)[0], oracle.sparse_linear(want_i, want_v, W_rot_ref)) <= Y_TOL
+    # the unfolded path on the exact values keeps nearly the same rows: only
+    # entries within the rounding of the fold and of the bf16 output differ
+    x_exact = oracle.rotate(f64(h) @ wp.T, qq)[0]
+    exact_i, _ = oracle.topk(x_exact, K)
+    assert len(np.intersect1d(idx, exact_i)) >= 0.95 * K

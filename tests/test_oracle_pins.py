@@ -30,6 +30,10 @@ def test_prepare_weights_pins():
     pins.check_prepare_weights(oracle.prepare_weights, oracle.rotate)
 
 
+def test_fold_rotation_pins():
+    pins.check_fold_rotation(oracle.fold_rotation, oracle.rotate)
+
+
 def test_round_to_bf16_pins():
     pins.check_round_to_bf16(oracle.round_to_bf16)
 
@@ -145,6 +149,10 @@ def _prepare_untransposed(Q, W):
     return np.asarray(Q, dtype=np.float64) @ np.asarray(W, dtype=np.float64)
 
 
+def _fold_untransposed(Q, Wt):
+    return np.asarray(Q, dtype=np.float64) @ np.asarray(Wt, dtype=np.float64)
+
+
 def _round_truncating(a):
     a = np.asarray(a, dtype=np.float64)
     m, e = np.frexp(a)
@@ -162,6 +170,7 @@ def _round_truncating(a):
     (pins.check_sparse_linear, _sparse_linear_drops_last),
     (lambda f: pins.check_prepare_weights(f, oracle.rotate), _prepare_untransposed),
     (pins.check_round_to_bf16, _round_truncating),
+    (lambda f: pins.check_fold_rotation(f, oracle.rotate), _fold_untransposed),
 ])
 def test_planted_mistake_is_caught(check, broken):
     with pytest.raises(AssertionError):
