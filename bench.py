@@ -315,6 +315,13 @@ def bench_larosa(args):
     groups = layer.groups
     stream = torch.cuda.Stream(device)
     ws = L.Workspace(device)
+    # size the workspace once for every call below (one token up to 16, Top-K
+    # and threshold), so that no captured graph holds a buffer that a later
+    # call would replace
+    for g in groups:
+        for M in (1, 2, 4, 8, 16):
+            ws.get(M, g.d_in, g.d_out, g.d_in)
+            ws.get(M, g.d_in, g.d_out, g.K)
     st = torch.zeros(1, dtype=torch.int32, device=device)
     ys = [torch.empty((1, g.d_out), dtype=torch.float32, device=device) for g in groups]
     for g in groups:
@@ -331,6 +338,31 @@ def bench_larosa(args):
     def rotate_step():
         for g, xr in zip(groups, x_rots):
             L.larosa_rotate(g.x, g.Qt, x_rot=xr)
+
+    # the other sparsities of the sweep (same layer, K from the sparsity) and
+    # batches of M tokens (each keeps its own Top-K; the rows kept by any
+    # token are streamed once)
+    sweep = (0.0, 25.0, 50.0)
+    batch_sizes = (2, 4, 8, 16)
+    x_batch = {M: [sd.activations(M, g.d_in, sd.seed_for(WORKLOAD_ID, 900 + M, 10 * gi + 3),
+                                  torch.bfloat16, device=device) for gi, g in enumerate(groups)]
+               for M in batch_sizes}
+    y_batch = {M: [torch.empty((M, g.d_out), dtype=torch.float32, device=device) for g in groups]
+               for M in batch_sizes}
+
+    def sparsity_step(sp):
+        Ks = [sd.k_for_sparsity(g.d_in, sp) for g in groups]
+
+        def step():
+            for g, y, K in zip(groups, ys, Ks):
+                L.larosa_rotate_topk_linear(g.x, g.Qt, g.W_rot, K, y=y, ws=ws, dev_status=st)
+        return step
+
+    def batch_step(M):
+        def step():
+            for g, x, y in zip(groups, x_batch[M], y_batch[M]):
+                L.larosa_rotate_topk_linear(x, g.Qt, g.W_rot, g.K, y=y, ws=ws, dev_status=st)
+        return step
 
     def rotate_topk_step():  # the fused path's first kernel: rotation, then Top-K by its last CTA
         for gi, g in enumerate(groups):
@@ -441,6 +473,8 @@ def bench_larosa(args):
     g_rot_thr = graph_of(rot_thr_step)
     g_unrot_thr = graph_of(unrot_thr_step)
     g_folded_topk = graph_of(folded_topk_step)
+    g_sweep = {sp: graph_of(sparsity_step(sp)) for sp in sweep}
+    g_batch = {M: graph_of(batch_step(M)) for M in batch_sizes}
     g_folded_thr = graph_of(folded_thr_step)
 
     props = torch.cuda.get_device_properties(device)
@@ -463,6 +497,19 @@ def bench_larosa(args):
     t_unrot_thr, _ = time_graph(g_unrot_thr, args.steps, args.warmup)
     t_folded_topk, _ = time_graph(g_folded_topk, args.steps, args.warmup)
     t_folded_thr, _ = time_graph(g_folded_thr, args.steps, args.warmup)
+    side_steps = max(1, args.steps // 4)
+    t_sweep = {sp: time_graph(gr, side_steps, args.warmup)[0] for sp, gr in g_sweep.items()}
+    t_batch = {M: time_graph(gr, side_steps, args.warmup)[0] for M, gr in g_batch.items()}
+    # rows streamed per batch step: the union of the tokens' kept rows (Q once per batch)
+    batch_bytes = {}
+    for M in batch_sizes:
+        tot = 0
+        for g, x in zip(groups, x_batch[M]):
+            xr = L.larosa_rotate(x, g.Qt)
+            idx, _ = L.larosa_topk(xr, g.K, dev_status=st)
+            rows = int(torch.unique(idx.flatten()).numel())
+            tot += rows * g.d_out * 2 + g.d_in * g.d_in * 2 + M * (g.d_in * 6 + g.K * 8 + g.d_out * 4)
+        batch_bytes[M] = tot
     n_launch = args.steps * len(groups)
     rot_us = t_rot / n_launch * 1e6
     rotsel_us = t_rotsel / n_launch * 1e6
@@ -576,6 +623,18 @@ def bench_larosa(args):
                 "folded_threshold_tokens_per_s": args.steps / t_folded_thr * world,
                 "folded_threshold_vs_dense": (args.steps / t_folded_thr * world) / dense_tps,
             },
+            # the fused path at the sweep's other sparsities, and with M tokens
+            # per call (tokens/s counts every token; bytes: Q once plus the
+            # union of the tokens' kept rows), each timed over steps/4
+            "sparsity_sweep": {
+                f"{sp:g}%": {"tokens_per_s": side_steps / t * world,
+                             "hbm_frac": sum(path_bytes(g, sd.k_for_sparsity(g.d_in, sp))["total"] for g in groups)
+                             * side_steps / t / 1e9 / peak}
+                for sp, t in t_sweep.items()},
+            "batch_sweep": {
+                f"M={M}": {"tokens_per_s": M * side_steps / t * world,
+                           "hbm_frac": batch_bytes[M] * side_steps / t / 1e9 / peak}
+                for M, t in t_batch.items()},
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": sum(g.x.numel() * g.x.element_size() for g in groups),
                     "d2h_bytes_per_step": sum(g.d_out * 4 for g in groups)},
@@ -585,7 +644,7 @@ def bench_larosa(args):
         }
         print(json.dumps(line), flush=True)
     del g_fused, g_sparse, g_dense, g_rot, g_rotsel, g_topk, g_gather, g_unrot_topk, g_rot_thr, g_unrot_thr
-    del g_folded_topk, g_folded_thr
+    del g_folded_topk, g_folded_thr, g_sweep, g_batch
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
