@@ -12,6 +12,7 @@ struct GemvPlan {
   int col_tile = 0;        // Wc: output columns per CTA
   int tpr = 0;             // consumer threads per weight row (Wc / columns per thread)
   int rows_per_stage = 0;  // weight rows per pipeline stage
+  int pitch = 0;           // bytes between two weight rows of a stage
   int n_col_tiles = 0;     // ceil(d_out / Wc)
   int splits = 0;          // CTAs along the row dimension (a multiple of cluster)
   int cluster = 1;         // CTAs per thread-block cluster (along the splits)

@@ -164,6 +164,102 @@ __global__ void __launch_bounds__(kT, (MT <= 2 && sizeof(T) == 2 ? 2 : 1)) rowdo
   // left some of them for a second wave.  It launches when this grid ends.
 }
 
+// ================================================================ rowmma
+//
+// y[m][j] = sum_k x[m][k] * A[j][k] for 3 to 16 bf16 tokens on the tensor
+// cores (mma.sync m16n8k16, bf16 inputs, fp32 accumulation).  From about
+// eight tokens on, the products per weight byte exceed what the FMA pipes
+// deliver at HBM speed, and the FMA kernel also reads every token's inputs
+// from shared memory once per weight vector.  The tokens are the MMA's 16
+// rows (zero beyond M), 8 consecutive output rows j its 8 columns, 16 inputs
+// k its reduction.  Lane (g, q) = (lane / 4, lane % 4) loads 16 bytes of
+// output row j0 + g of A and the same 8 inputs of tokens g and g + 8 per
+// block of 32 inputs; the order of the 32 inputs inside a block is permuted
+// the same way for x and for A (a sum does not depend on its order), so that
+// these loads are the fragments of two MMAs as they stand.  A CTA of
+// kMmaWarps warps owns 8 output rows; warp w adds up the input blocks
+// [nb*w/kMmaWarps, nb*(w+1)/kMmaWarps) and the warps' partial tiles are added
+// in warp order.  Needs n_in % 32 == 0 and n_out % 8 == 0.
+constexpr int kMmaWarps = 8;
+constexpr int kMmaU = 4;          // 32-input blocks in flight per lane
+constexpr int kMmaMinTokens = 3;  // from this many tokens on (bf16) the tensor-core kernel is used
+
+struct MParams {
+  const void* A;  // [n_out x n_in] bf16
+  const void* x;  // [M x n_in] bf16
+  float* y;       // [M x n_out]
+  int n_in;
+  int n_out;
+  int M;
+};
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <bool kTwoRows>  // tokens 8..15 present
+__global__ void __launch_bounds__(kMmaWarps * 32) rowmma_kernel(const MParams p) {
+  __shared__ float4 s_part[kMmaWarps][32];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, q = lane & 3;
+  const int j0 = blockIdx.x * 8;
+  pdl_wait();
+  const int nb = p.n_in / 32;
+  const int b0 = nb * warp / kMmaWarps, b1 = nb * (warp + 1) / kMmaWarps;
+  const unsigned char* arow =
+      static_cast<const unsigned char*>(p.A) + ((size_t)(j0 + g) * p.n_in + 8 * q) * 2;
+  const unsigned char* xr0 = static_cast<const unsigned char*>(p.x) + ((size_t)g * p.n_in + 8 * q) * 2;
+  const unsigned char* xr8 = xr0 + (size_t)8 * p.n_in * 2;
+  const bool has0 = g < p.M, has8 = kTwoRows && g + 8 < p.M;
+  const uint4 zero = make_uint4(0, 0, 0, 0);
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int b = b0; b < b1; b += kMmaU) {
+    uint4 w[kMmaU], u0[kMmaU], u8[kMmaU];
+#pragma unroll
+    for (int k = 0; k < kMmaU; ++k) {
+      const bool in = b + k < b1;
+      w[k] = in ? ld_stream(arow + (size_t)(b + k) * 64) : zero;
+      u0[k] = in && has0 ? __ldg(reinterpret_cast<const uint4*>(xr0 + (size_t)(b + k) * 64)) : zero;
+      u8[k] = kTwoRows && in && has8 ? __ldg(reinterpret_cast<const uint4*>(xr8 + (size_t)(b + k) * 64))
+                                     : zero;
+    }
+#pragma unroll
+    for (int k = 0; k < kMmaU; ++k) {
+      // step 0 takes the block's inputs 8q + 0..3, step 1 the inputs 8q + 4..7
+      mma_bf16_16816(d, u0[k].x, u8[k].x, u0[k].y, u8[k].y, w[k].x, w[k].y);
+      mma_bf16_16816(d, u0[k].z, u8[k].z, u0[k].w, u8[k].w, w[k].z, w[k].w);
+    }
+  }
+  s_part[warp][lane] = make_float4(d[0], d[1], d[2], d[3]);
+  __syncthreads();
+  if (warp == 0) {
+    float4 t = s_part[0][lane];
+#pragma unroll
+    for (int v = 1; v < kMmaWarps; ++v) {
+      const float4 o = s_part[v][lane];
+      t.x += o.x;
+      t.y += o.y;
+      t.z += o.z;
+      t.w += o.w;
+    }
+    // D[g][2q], D[g][2q + 1], D[g + 8][2q], D[g + 8][2q + 1]: tokens by rows
+    const int j = j0 + 2 * q;
+    if (g < p.M) {
+      p.y[(size_t)g * p.n_out + j] = t.x;
+      p.y[(size_t)g * p.n_out + j + 1] = t.y;
+    }
+    if (g + 8 < p.M) {
+      p.y[(size_t)(g + 8) * p.n_out + j] = t.z;
+      p.y[(size_t)(g + 8) * p.n_out + j + 1] = t.w;
+    }
+  }
+}
+
 // ================================================================ gather
 
 constexpr int kGatherSmemCeiling = 227 * 1024;
@@ -1388,6 +1484,28 @@ cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M,
   DevState* ds = nullptr;
   cudaError_t err = dev_state(&ds);
   if (err != cudaSuccess) return err;
+  if (e == Elem::BF16 && M >= kMmaMinTokens && n_in % 32 == 0 && n_out % 8 == 0) {
+    MParams p;
+    p.A = A;
+    p.x = x;
+    p.y = y;
+    p.n_in = n_in;
+    p.n_out = n_out;
+    p.M = M;
+    void* fn = M > 8 ? reinterpret_cast<void*>(&rowmma_kernel<true>)
+                     : reinterpret_cast<void*>(&rowmma_kernel<false>);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n_out / 8, 1, 1);
+    cfg.blockDim = dim3(kMmaWarps * 32, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {&p};
+    return cudaLaunchKernelExC(&cfg, fn, args);
+  }
   const int MT = round_up_mt(M);
   const int esz = e == Elem::BF16 ? 2 : 4;
   const size_t xbytes = (size_t)M * n_in * esz;

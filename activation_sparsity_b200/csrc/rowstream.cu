@@ -17,6 +17,14 @@
 //    TMA engine) completing on per-stage mbarriers; 8 consumer warps hold
 //    fp32 accumulators for CPT columns x MT tokens per thread and release
 //    each stage through an "empty" mbarrier.
+//  * From 8 tokens on (bf16 weights, fp32 coefficients) the consumers use
+//    the tensor cores instead (mma.sync m16n8k16): tokens are the MMA's
+//    rows, 8 output columns its columns, 16 weight rows its reduction.  A
+//    16 x 8 weight tile is read from the ring with ldmatrix.trans (ring rows
+//    padded by 16 bytes so that its 8-row reads do not share banks); each
+//    fp32 coefficient is split into a bf16 head and a bf16 tail, two MMAs
+//    per tile, so the products keep about 16 bits of the coefficient.
+//    Consumer warp w owns the 8-column blocks w, w + 8, ... of the tile.
 //  * Reduction order is fixed (rows in list order per thread, row groups in
 //    order, cluster ranks in order, cluster partials in order), so results
 //    are bitwise reproducible for a given launch geometry.
@@ -61,6 +69,7 @@ struct Params {
   int col_tile;
   int tpr;
   int rows_per_stage;
+  int pitch;  // bytes between two rows of a stage
   int max_rpc;
   int* dev_status;
 };
@@ -70,7 +79,39 @@ struct Acc {
   float v[MT][CPT];
 };
 
-template <typename Tw, typename Tc, int MT, int CPT>
+constexpr int kMmaBlocks = 8;                           // 8-column blocks per consumer warp
+constexpr int kMmaTile = 8 * kMmaBlocks * kConsumerWarps;  // columns of a tensor-core tile
+
+// bf16 pair {lo, hi} of two floats, round to nearest even
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// head (bf16 of c) and tail (bf16 of c - head) of two coefficients
+__device__ __forceinline__ void split_pair(float c0, float c1, uint32_t* head, uint32_t* tail) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(c0, c1);
+  const float2 hf = __bfloat1622float2(h);
+  *head = *reinterpret_cast<const uint32_t*>(&h);
+  *tail = pack_bf16x2(c0 - hf.x, c1 - hf.y);
+}
+
+__device__ __forceinline__ void ldmatrix_x2_trans(uint32_t* b0, uint32_t* b1, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(*b0), "=r"(*b1)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <typename Tw, typename Tc, int MT, int CPT, bool kMma>
 __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_kernel(const Params p) {
   extern __shared__ __align__(1024) unsigned char smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -135,13 +176,18 @@ __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_ke
   const int rstage = p.rows_per_stage;
   const int n_it = (nr + rstage - 1) / rstage;
   const uint32_t row_bytes = static_cast<uint32_t>(wc) * sizeof(Tw);
-  const int pitch = p.col_tile * static_cast<int>(sizeof(Tw));
+  const int pitch = p.pitch;
 
-  Acc<MT, CPT> acc;
+  Acc<MT, (kMma ? 1 : CPT)> acc;
 #pragma unroll
   for (int m = 0; m < MT; ++m)
 #pragma unroll
-    for (int v = 0; v < CPT; ++v) acc.v[m][v] = 0.f;
+    for (int v = 0; v < (kMma ? 1 : CPT); ++v) acc.v[m][v] = 0.f;
+  float dacc[kMmaBlocks][4];  // tensor-core variant: D tiles of this warp's column blocks
+#pragma unroll
+  for (int bi = 0; bi < kMmaBlocks; ++bi)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dacc[bi][e] = 0.f;
 
   const int g = tid / p.tpr;                 // row group of a consumer thread
   const int n_groups = kConsumers / p.tpr;   // row groups
@@ -187,7 +233,37 @@ __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_ke
         break;
       }
       const int rows_here = min(rstage, nr - it * rstage);
-      if (active) {
+      if constexpr (kMma) {
+        const unsigned char* base = stages + s * kStageBytes;
+        const float* cs = coef_s + it * rstage;
+        const int gq = lane >> 2, q = lane & 3;
+        const int nb8 = wc / 8;
+        for (int kb = 0; kb < rows_here; kb += 16) {
+          // A: coefficients of tokens gq, gq + 8 for rows kb + 2q + {0, 1}
+          // and kb + 2q + {8, 9}, as bf16 head + tail (zero past the rows)
+          auto cf = [&](int m, int r) {
+            return (m < MT && kb + r < rows_here) ? cs[m * p.max_rpc + kb + r] : 0.f;
+          };
+          uint32_t h0, t0, h1, t1, h2, t2, h3, t3;
+          split_pair(cf(gq, 2 * q), cf(gq, 2 * q + 1), &h0, &t0);
+          split_pair(cf(gq + 8, 2 * q), cf(gq + 8, 2 * q + 1), &h1, &t1);
+          split_pair(cf(gq, 2 * q + 8), cf(gq, 2 * q + 9), &h2, &t2);
+          split_pair(cf(gq + 8, 2 * q + 8), cf(gq + 8, 2 * q + 9), &h3, &t3);
+          // lanes 0..15 address the 16 weight rows of the tile (a row past
+          // the stage's last repeats it: its coefficient is zero)
+          const int rr = min(kb + (lane & 15), rows_here - 1);
+#pragma unroll
+          for (int bi = 0; bi < kMmaBlocks; ++bi) {
+            const int blk = warp + bi * kConsumerWarps;
+            if (blk < nb8) {  // warp-uniform
+              uint32_t b0, b1;
+              ldmatrix_x2_trans(&b0, &b1, smem_u32(base + rr * pitch + blk * 16));
+              mma_16816(dacc[bi], h0, h1, h2, h3, b0, b1);
+              mma_16816(dacc[bi], t0, t1, t2, t3, b0, b1);
+            }
+          }
+        }
+      } else if (active) {
         const unsigned char* base = stages + s * kStageBytes + col * sizeof(Tw);
         const float* cs = coef_s + it * rstage;
         for (int j = g; j < rows_here; j += n_groups) {
@@ -224,20 +300,43 @@ __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_ke
   // ---------------------------------------------------------------- epilogue
   // 1) row groups -> CTA partial, in shared memory (reusing the ring).
   float* red = reinterpret_cast<float*>(stages);
-  float* part = red + n_groups * MT * p.col_tile;
-  if (warp < kConsumerWarps && col < wc) {
+  // the CTA partial; the start of the ring later holds this rank's reduced
+  // slice (outs), which must not overlap a partial a peer may still read
+  float* part = red + (kMma ? 1 : n_groups) * MT * p.col_tile;
+  if constexpr (kMma) {
+    // D[token][column]: (gq, 2q), (gq, 2q + 1), (gq + 8, 2q), (gq + 8, 2q + 1)
+    const int gq = lane >> 2, q = lane & 3;
+    if (warp < kConsumerWarps) {
 #pragma unroll
-    for (int m = 0; m < MT; ++m)
+      for (int bi = 0; bi < kMmaBlocks; ++bi) {
+        const int c = (warp + bi * kConsumerWarps) * 8 + 2 * q;
+        if (c < wc) {
+          if (gq < MT) {
+            part[gq * p.col_tile + c] = dacc[bi][0];
+            part[gq * p.col_tile + c + 1] = dacc[bi][1];
+          }
+          if (gq + 8 < MT) {
+            part[(gq + 8) * p.col_tile + c] = dacc[bi][2];
+            part[(gq + 8) * p.col_tile + c + 1] = dacc[bi][3];
+          }
+        }
+      }
+    }
+  } else {
+    if (warp < kConsumerWarps && col < wc) {
 #pragma unroll
-      for (int v = 0; v < CPT; ++v) red[(g * MT + m) * p.col_tile + col + v] = acc.v[m][v];
-  }
-  __syncthreads();
-  for (int e = tid; e < MT * wc; e += kThreads) {
-    const int m = e / wc;
-    const int c = e - m * wc;
-    float s = 0.f;
-    for (int gg = 0; gg < n_groups; ++gg) s += red[(gg * MT + m) * p.col_tile + c];
-    part[m * p.col_tile + c] = s;
+      for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int v = 0; v < CPT; ++v) red[(g * MT + m) * p.col_tile + col + v] = acc.v[m][v];
+    }
+    __syncthreads();
+    for (int e = tid; e < MT * wc; e += kThreads) {
+      const int m = e / wc;
+      const int c = e - m * wc;
+      float s = 0.f;
+      for (int gg = 0; gg < n_groups; ++gg) s += red[(gg * MT + m) * p.col_tile + c];
+      part[m * p.col_tile + c] = s;
+    }
   }
 
   // 2) cluster ranks -> cluster partial: rank q owns columns [q*sl, q*sl+sl).
@@ -298,10 +397,15 @@ __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_ke
 
 // ------------------------------------------------------------------ host side
 
-template <typename Tw, typename Tc, int MT, int CPT>
+template <typename Tw, typename Tc, int MT, int CPT, bool kMma = false>
 struct Inst {
-  static void* fn() { return reinterpret_cast<void*>(&rowstream_gemv_kernel<Tw, Tc, MT, CPT>); }
+  static void* fn() { return reinterpret_cast<void*>(&rowstream_gemv_kernel<Tw, Tc, MT, CPT, kMma>); }
 };
+
+// bf16 weights and fp32 coefficients from 8 tokens on: the tensor-core
+// consumers (at 4 tokens the FMA consumers with their wider tiles measured
+// faster)
+bool uses_mma(Elem w, Elem c, int MT) { return w == Elem::BF16 && c == Elem::F32 && MT >= 8; }
 
 constexpr int cols_per_thread(Elem w, int MT) {
   // 16-byte shared-memory reads per row for MT <= 4; fewer columns per thread
@@ -322,6 +426,13 @@ void* kernel_for(Elem w, Elem c, int MT) {
     default: return nullptr;                                                   \
   }
   if (w == Elem::BF16 && c == Elem::BF16) { LAROSA_PICK(__nv_bfloat16, __nv_bfloat16) }
+  if (uses_mma(w, c, MT)) {
+    switch (MT) {
+      case 8: return Inst<__nv_bfloat16, float, 8, 8, true>::fn();
+      case 16: return Inst<__nv_bfloat16, float, 16, 8, true>::fn();
+      default: return nullptr;
+    }
+  }
   if (w == Elem::BF16 && c == Elem::F32) { LAROSA_PICK(__nv_bfloat16, float) }
   if (w == Elem::F32 && c == Elem::F32) { LAROSA_PICK(float, float) }
 #undef LAROSA_PICK
@@ -417,9 +528,11 @@ cudaError_t plan_gemv(Elem w_elem, Elem coef_elem, int M, int d_out, int n_rows_
   const int n_rows = std::max(0, n_rows_max);
 
   // Widest column tile that is not mostly idle threads.
+  const bool mma = uses_mma(w_elem, coef_elem, MT);
   int tpr = 256;
   while (tpr > 32 && (tpr / 2) * cpt >= d_out) tpr /= 2;
-  const int wc = tpr * cpt;
+  // the tensor-core tile: kMmaTile columns, fewer when d_out is smaller
+  const int wc = mma ? std::min(kMmaTile, (d_out + 7) / 8 * 8) : tpr * cpt;
   const int n_ct = (d_out + wc - 1) / wc;
 
   const int min_s = (n_rows + max_rpc - 1) / max_rpc;  // coefficient capacity
@@ -441,7 +554,8 @@ cudaError_t plan_gemv(Elem w_elem, Elem coef_elem, int M, int d_out, int n_rows_
   GemvPlan pl;
   pl.col_tile = wc;
   pl.tpr = tpr;
-  pl.rows_per_stage = kStageBytes / (wc * elem);
+  pl.pitch = mma ? wc * elem + 16 : wc * elem;
+  pl.rows_per_stage = kStageBytes / pl.pitch;
   pl.n_col_tiles = n_ct;
   pl.splits = best_s;
   pl.cluster = best_c;
@@ -477,6 +591,7 @@ cudaError_t launch_gemv(const GemvArgs& a, const GemvPlan& pl, cudaStream_t stre
   p.col_tile = pl.col_tile;
   p.tpr = pl.tpr;
   p.rows_per_stage = pl.rows_per_stage;
+  p.pitch = pl.pitch;
   p.max_rpc = pl.max_rows_per_cta;
   p.dev_status = a.dev_status;
 
