@@ -14,6 +14,9 @@
 //   threshold, M > 1           rowdot -> threshold (writes the coefficient rows
 //                              and the bitmap) -> union -> rowstream
 //   no Qt (identity rotation)  as above with widen in place of rowdot
+//   sparse + low rank          sparse linear on the kept list; dropped part
+//                              (lowrank.cu); two dense row-streaming GEMVs
+//                              through the factors; y += y_r
 #include <stdio.h>
 #include <string.h>
 
@@ -265,6 +268,68 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
   }
   e = larosa::launch_gemv(a, pl, s);
   return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "sparse linear kernel");
+}
+
+// Workspace of larosa_sparse_lowrank_linear: the sparse linear's layout, then
+// the dropped part of x, u = dropped . A_r, y_r = u . B_r and the split-K
+// partials of the two GEMVs through the factors.
+struct LowrankLayout {
+  Layout base;
+  size_t x_drop = 0, u = 0, y_r = 0, partials = 0, total = 0;
+};
+
+int make_lowrank_layout(int M, int d_in, int d_out, int K, int r, LowrankLayout* LL) {
+  int st = make_layout(M, d_in, d_out, K, &LL->base);
+  if (st != LAROSA_OK) return st;
+  size_t pf = 0;
+  for (int dt = 0; dt < 2; ++dt) {
+    const Elem w = dt == 0 ? Elem::F32 : Elem::BF16;
+    GemvPlan pa, pb;
+    cudaError_t e = larosa::plan_gemv(w, Elem::F32, M, r, d_in, &pa);
+    if (e == cudaSuccess) e = larosa::plan_gemv(w, Elem::F32, M, d_out, r, &pb);
+    if (e != cudaSuccess) return cuda_fail(e, "plan low-rank GEMV");
+    if (pa.ticket_words > kSplitKTicketWords || pb.ticket_words > kSplitKTicketWords)
+      return LAROSA_ERR_SHAPE;
+    pf = std::max(pf, std::max(pa.partial_floats, pb.partial_floats));
+  }
+  size_t off = align_up(LL->base.total, 256);
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  LL->x_drop = take((size_t)M * d_in * 4);
+  LL->u = take((size_t)M * r * 4);
+  LL->y_r = take((size_t)M * d_out * 4);
+  LL->partials = take(pf * 4);
+  LL->total = off;
+  return LAROSA_OK;
+}
+
+// out[M x cols] = coef[M x rows] . Wm[rows x cols] (all rows, fp32 coefficients).
+int run_dense_gemv(const void* Wm, int rows, int cols, const float* coef, int M, float* out,
+                   int dtype, void* ws, float* partials, int* dev_status, cudaStream_t s) {
+  GemvPlan pl;
+  cudaError_t e = larosa::plan_gemv(elem_of(dtype), Elem::F32, M, cols, rows, &pl);
+  if (e != cudaSuccess) return cuda_fail(e, "plan low-rank GEMV");
+  GemvArgs a;
+  a.W = Wm;
+  a.w_elem = elem_of(dtype);
+  a.d_out = cols;
+  a.row_bound = rows;
+  a.rows = nullptr;
+  a.n_rows = rows;
+  a.coef = coef;
+  a.coef_elem = Elem::F32;
+  a.coef_ld = rows;
+  a.M = M;
+  a.y = out;
+  a.y_ld = cols;
+  a.partials = partials;
+  a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTickets));
+  a.dev_status = dev_status;
+  e = larosa::launch_gemv(a, pl, s);
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "low-rank GEMV kernel");
 }
 
 }  // namespace
@@ -602,6 +667,50 @@ int larosa_rotate_threshold_linear(const void* x, const void* Qt, const void* W_
   }
   e = larosa::launch_gemv(a, pl, s);
   return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "sparse linear kernel");
+}
+
+size_t larosa_lowrank_workspace_bytes(int M, int d_in, int d_out, int K, int r) {
+  if (check_sizes(M, d_in, d_out, K) != LAROSA_OK || r < 1 || r > kMaxDout) return 0;
+  LowrankLayout LL;
+  if (make_lowrank_layout(M, d_in, d_out, K, r, &LL) != LAROSA_OK) return 0;
+  return LL.total;
+}
+
+int larosa_sparse_lowrank_linear(const float* x, const int32_t* idx, const float* val, int M, int K,
+                                 const void* W, const void* A_r, const void* B_r, int d_in,
+                                 int d_out, int r, float* y, void* ws, size_t ws_bytes, int dtype,
+                                 int* dev_status, larosa_stream_t stream) {
+  if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
+  if (x == nullptr || W == nullptr || A_r == nullptr || B_r == nullptr || y == nullptr ||
+      (K > 0 && (idx == nullptr || val == nullptr)))
+    return LAROSA_ERR_INVALID_ARG;
+  int st = check_sizes(M, d_in, d_out, K);
+  if (st != LAROSA_OK) return st;
+  if (r < 1 || r > kMaxDout) return LAROSA_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(W) || !aligned16(A_r) || !aligned16(B_r) || !aligned16(y) ||
+      !row_aligned(d_out, dtype) || !row_aligned(r, dtype))
+    return LAROSA_ERR_ALIGN;
+  LowrankLayout LL;
+  st = make_lowrank_layout(M, d_in, d_out, K, r, &LL);
+  if (st != LAROSA_OK) return st;
+  if (ws == nullptr || !aligned16(ws) || ws_bytes < LL.total) return LAROSA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* x_drop = reinterpret_cast<float*>(at(ws, LL.x_drop));
+  float* u = reinterpret_cast<float*>(at(ws, LL.u));
+  float* y_r = reinterpret_cast<float*>(at(ws, LL.y_r));
+  float* part = reinterpret_cast<float*>(at(ws, LL.partials));
+  // y_s: the kept rows of W
+  st = run_sparse(idx, val, M, K, W, d_in, d_out, y, dtype, ws, LL.base, dev_status, s);
+  if (st != LAROSA_OK) return st;
+  // y_r = ((x - sigma(x)) . A_r) . B_r, then y = y_s + y_r
+  cudaError_t e = larosa::launch_dropped(x, idx, M, K, d_in, x_drop, dev_status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "dropped-part kernel");
+  st = run_dense_gemv(A_r, d_in, r, x_drop, M, u, dtype, ws, part, dev_status, s);
+  if (st != LAROSA_OK) return st;
+  st = run_dense_gemv(B_r, r, d_out, u, M, y_r, dtype, ws, part, dev_status, s);
+  if (st != LAROSA_OK) return st;
+  e = larosa::launch_add(y, y_r, M * d_out, s);
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "add kernel");
 }
 
 int larosa_dense_linear(const void* x, const void* Wt, int M, int d_in, int d_out, float* y,

@@ -47,6 +47,9 @@ _SIGNATURES = {
     "larosa_rotate_threshold_linear": ([_vp, _vp, _vp, _i, _i, _i, _c.c_float, _vp, _vp, _sz, _vp, _i,
                                         _vp], _i),
     "larosa_dense_linear": ([_vp, _vp, _i, _i, _i, _vp, _i, _vp], _i),
+    "larosa_sparse_lowrank_linear": ([_vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _sz, _i, _vp,
+                                      _vp], _i),
+    "larosa_lowrank_workspace_bytes": ([_i, _i, _i, _i, _i], _sz),
     "larosa_sparse_linear_noalloc": ([_vp, _vp, _i, _i, _vp, _i, _i, _vp, _i, _vp, _vp], _i),
     "larosa_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "larosa_workspace_layout": ([_i, _i, _i, _i, _c.POINTER(_sz), _c.POINTER(_sz), _c.POINTER(_sz)], _i),
@@ -189,6 +192,10 @@ def larosa_version() -> int:
 
 def larosa_workspace_bytes(M: int, d_in: int, d_out: int, K: int) -> int:
     return int(_lib.larosa_workspace_bytes(M, d_in, d_out, K))
+
+
+def larosa_lowrank_workspace_bytes(M: int, d_in: int, d_out: int, K: int, r: int) -> int:
+    return int(_lib.larosa_lowrank_workspace_bytes(M, d_in, d_out, K, r))
 
 
 def larosa_workspace_layout(M: int, d_in: int, d_out: int, K: int) -> tuple[int, int, int]:
@@ -415,6 +422,38 @@ def larosa_rotate_threshold_linear(x: torch.Tensor, Qt: torch.Tensor | None, W_r
                                                _ptr(y), p, n, _status_ptr(dev_status, x.device),
                                                _dtype_code(x), _stream(x.device)),
            "larosa_rotate_threshold_linear")
+    return y
+
+
+def larosa_sparse_lowrank_linear(x: torch.Tensor, idx: torch.Tensor, val: torch.Tensor, W: torch.Tensor,
+                                 A_r: torch.Tensor, B_r: torch.Tensor, y: torch.Tensor | None = None,
+                                 ws: torch.Tensor | None = None, dev_status: torch.Tensor | None = None
+                                 ) -> torch.Tensor:
+    """y = sparse(x) . W + ((x - sparse(x)) . A_r) . B_r for the kept lists idx/val of x (fp32)."""
+    _need(x, "x", torch.float32)
+    _need(W, "W")
+    _need(A_r, "A_r", W.dtype)
+    _need(B_r, "B_r", W.dtype)
+    x2 = _as2d(x)
+    M, d_in = x2.shape
+    d_out, r = W.shape[1], A_r.shape[1]
+    idx2, val2 = _as2d(idx), _as2d(val)
+    K = idx2.shape[1]
+    _need(idx2, "idx", torch.int32)
+    _need(val2, "val", torch.float32)
+    if y is None:
+        y = torch.empty((M, d_out), dtype=torch.float32, device=x.device)
+    _need(y, "y", torch.float32)
+    nb = int(_lib.larosa_lowrank_workspace_bytes(M, d_in, d_out, K, r))
+    if nb == 0:
+        raise LarosaError(2, "larosa_lowrank_workspace_bytes")
+    if ws is None or ws.numel() * ws.element_size() < nb:
+        ws = torch.zeros(nb, dtype=torch.uint8, device=x.device)
+    _check(_lib.larosa_sparse_lowrank_linear(_ptr(x2), _ptr(idx2), _ptr(val2), M, K, _ptr(W), _ptr(A_r),
+                                             _ptr(B_r), d_in, d_out, r, _ptr(y), _ptr(ws),
+                                             ws.numel() * ws.element_size(), _dtype_code(W),
+                                             _status_ptr(dev_status, x.device), _stream(x.device)),
+           "larosa_sparse_lowrank_linear")
     return y
 
 

@@ -406,6 +406,21 @@ def bench_larosa(args):
         for gi, (g, y) in enumerate(zip(groups, ys)):
             L.larosa_rotate_topk_linear(x_folded[gi], None, g.W_rot, g.K, y=y, ws=ws, dev_status=st)
 
+    # sparse + low-rank compensation of the dropped entries (rank-256
+    # factors of each group's weight, random here: the time depends on shapes)
+    LR = 256
+    lr_A = [sd.weights(g.d_in, LR, 0.02, sd.seed_for(WORKLOAD_ID, 950, 10 * gi + 1), torch.bfloat16, device=device)
+            for gi, g in enumerate(groups)]
+    lr_B = [sd.weights(LR, g.d_out, 0.02, sd.seed_for(WORKLOAD_ID, 950, 10 * gi + 2), torch.bfloat16, device=device)
+            for gi, g in enumerate(groups)]
+    lr_ws = [torch.zeros(L.larosa_lowrank_workspace_bytes(1, g.d_in, g.d_out, g.K, LR), dtype=torch.uint8,
+                         device=device) for g in groups]
+
+    def lowrank_step():
+        for gi, (g, y) in enumerate(zip(groups, ys)):
+            L.larosa_sparse_lowrank_linear(x_rots[gi], idxs[gi], vals[gi], g.W_rot, lr_A[gi], lr_B[gi], y=y,
+                                           ws=lr_ws[gi], dev_status=st)
+
     def folded_thr_step():
         for gi, (g, y) in enumerate(zip(groups, ys)):
             L.larosa_rotate_threshold_linear(x_folded[gi], None, g.W_rot, t_rot[gi], y=y, ws=ws,
@@ -476,6 +491,7 @@ def bench_larosa(args):
     g_sweep = {sp: graph_of(sparsity_step(sp)) for sp in sweep}
     g_batch = {M: graph_of(batch_step(M)) for M in batch_sizes}
     g_folded_thr = graph_of(folded_thr_step)
+    g_lowrank = graph_of(lowrank_step)
 
     props = torch.cuda.get_device_properties(device)
     clocks = ClockSampler(f"GPU-{props.uuid}")
@@ -497,6 +513,7 @@ def bench_larosa(args):
     t_unrot_thr, _ = time_graph(g_unrot_thr, args.steps, args.warmup)
     t_folded_topk, _ = time_graph(g_folded_topk, args.steps, args.warmup)
     t_folded_thr, _ = time_graph(g_folded_thr, args.steps, args.warmup)
+    t_lowrank, _ = time_graph(g_lowrank, args.steps, args.warmup)
     side_steps = max(1, args.steps // 4)
     t_sweep = {sp: time_graph(gr, side_steps, args.warmup)[0] for sp, gr in g_sweep.items()}
     t_batch = {M: time_graph(gr, side_steps, args.warmup)[0] for M, gr in g_batch.items()}
@@ -523,6 +540,7 @@ def bench_larosa(args):
     lin_bytes = [g.K * g.d_out * 2 + g.K * 8 + g.d_out * 4 for g in groups]
     step_bytes = sum(path_bytes(g, g.K)["total"] for g in groups)
     sparse_bytes = sum(path_bytes(g, g.K, rotate=False)["total"] for g in groups)
+    lowrank_bytes = sparse_bytes + sum((g.d_in + g.d_out) * LR * 2 + g.d_in * 4 for g in groups)
     dense_bytes = sum(g.d_in * g.d_out * 2 + g.d_in * 2 + g.d_out * 4 for g in groups)
     unrot_topk_bytes = sum(path_bytes(g, g.K, rotate=False)["total"] for g in groups)
     rot_thr_bytes = sum(path_bytes(g, n)["total"] for g, n in zip(groups, nnz_rot))
@@ -622,6 +640,10 @@ def bench_larosa(args):
                 "folded_topk_vs_dense": (args.steps / t_folded_topk * world) / dense_tps,
                 "folded_threshold_tokens_per_s": args.steps / t_folded_thr * world,
                 "folded_threshold_vs_dense": (args.steps / t_folded_thr * world) / dense_tps,
+                # kept rows plus rank-256 compensation of the dropped entries, on
+                # the pre-rotated input (Q not streamed)
+                "sparse_lowrank_r256_tokens_per_s": args.steps / t_lowrank * world,
+                "sparse_lowrank_r256_hbm_frac": lowrank_bytes * args.steps / t_lowrank / 1e9 / peak,
             },
             # the fused path at the sweep's other sparsities, and with M tokens
             # per call (tokens/s counts every token; bytes: Q once plus the
@@ -644,7 +666,7 @@ def bench_larosa(args):
         }
         print(json.dumps(line), flush=True)
     del g_fused, g_sparse, g_dense, g_rot, g_rotsel, g_topk, g_gather, g_unrot_topk, g_rot_thr, g_unrot_thr
-    del g_folded_topk, g_folded_thr, g_sweep, g_batch
+    del g_folded_topk, g_folded_thr, g_sweep, g_batch, g_lowrank
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

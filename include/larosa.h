@@ -272,6 +272,32 @@ int larosa_rotate_threshold_linear(const void *x, const void *Qt,
                                    larosa_stream_t stream);
 
 /*
+ * Sparse + low-rank linear (R-Sparse report, 研究流程与方法 / R-Sparse框架设计,
+ * hybrid computation): the entries a selection drops are sent through
+ * rank-r factors of the weight instead of being discarded:
+ *   y[m] = sum_k val[m][k] * W[idx[m][k]]  +  ((x[m] - sigma(x[m])) . A_r) . B_r,
+ * where sigma(x[m]) is x[m] with every entry outside idx[m] set to zero.
+ * x: [M x d_in] fp32, the vector the selection was made on (x_rot for the
+ * rotated path; idx/val then come from larosa_topk or larosa_threshold on
+ * it, val = x at idx).  W: [d_in x d_out], A_r: [d_in x r], B_r: [r x d_out],
+ * all of `dtype` (the factors of an offline SVD W ~ U S V^T: A_r = U_r
+ * S_r^1/2, B_r = S_r^1/2 V_r^T); y: [M x d_out] fp32.  d_out and r rows of
+ * 16 bytes; x, W, A_r, B_r, y 16-byte aligned.  Kernels: the sparse linear
+ * on the kept list, the dropped part of x, u = dropped . A_r and y_r = u . B_r
+ * by the row-streaming GEMV with fp32 coefficients, and y += y_r.
+ * ws: at least larosa_lowrank_workspace_bytes(M, d_in, d_out, K, r) bytes.
+ */
+int larosa_sparse_lowrank_linear(const float *x, const int32_t *idx,
+                                 const float *val, int M, int K, const void *W,
+                                 const void *A_r, const void *B_r, int d_in,
+                                 int d_out, int r, float *y, void *ws,
+                                 size_t ws_bytes, int dtype, int *dev_status,
+                                 larosa_stream_t stream);
+
+/* Workspace bytes of larosa_sparse_lowrank_linear (0 for out-of-range sizes). */
+size_t larosa_lowrank_workspace_bytes(int M, int d_in, int d_out, int K, int r);
+
+/*
  * Dense baseline: y[m][j] = sum_i x[m][i] * Wt[j][i], i.e. y = x . W for the
  * dense layer, with the weight in torch.nn.Linear layout Wt = W^T
  * [d_out x d_in] (each output a dot product with one contiguous row), by the

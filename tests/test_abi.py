@@ -33,7 +33,8 @@ def test_header_declares_the_entry_points():
     for must in ("larosa_prepare_weights", "larosa_rotate", "larosa_topk", "larosa_rotate_topk",
                  "larosa_sparse_linear",
                  "larosa_rotate_topk_linear", "larosa_dense_linear", "larosa_workspace_bytes",
-                 "larosa_threshold", "larosa_rotate_threshold_linear", "larosa_check"):
+                 "larosa_threshold", "larosa_rotate_threshold_linear", "larosa_fold_rotation",
+                 "larosa_sparse_lowrank_linear", "larosa_check"):
         assert must in names
 
 
@@ -127,6 +128,15 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.larosa_fold_rotation(FAKE, None, FAKE, 64, 64, BF16, None) == 1
     assert lib.larosa_fold_rotation(FAKE, FAKE, FAKE, 64, 64, 9, None) == 4
     assert lib.larosa_fold_rotation(FAKE, FAKE, FAKE, 0, 64, BF16, None) == 2
+    # sparse + low rank
+    slr = lib.larosa_sparse_lowrank_linear
+    assert slr(None, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, 64, 64, 16, FAKE, FAKE, z, BF16, None, None) == 1
+    assert slr(FAKE, FAKE, FAKE, 1, 4, FAKE, None, FAKE, 64, 64, 16, FAKE, FAKE, z, BF16, None, None) == 1
+    assert slr(FAKE, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, 64, 64, 0, FAKE, FAKE, z, BF16, None, None) == 2
+    assert slr(FAKE, FAKE, FAKE, 1, 65, FAKE, FAKE, FAKE, 64, 64, 16, FAKE, FAKE, z, BF16, None, None) == 2
+    assert slr(FAKE, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, 64, 64, 12, FAKE, FAKE, z, BF16, None, None) == 3
+    assert slr(FAKE, FAKE, FAKE, 1, 4, FAKE, MISALIGNED, FAKE, 64, 64, 16, FAKE, FAKE, z, BF16, None, None) == 3
+    assert slr(FAKE, FAKE, FAKE, 1, 4, FAKE, FAKE, FAKE, 64, 64, 16, FAKE, FAKE, z, 7, None, None) == 4
     # in-place counter-rotation is refused
     assert lib.larosa_prepare_weights(FAKE, P(0x20000), P(0x20000), 64, 64, BF16, None) == 1
     # status check needs a status word

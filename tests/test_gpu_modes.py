@@ -254,3 +254,33 @@ def test_folded_rotation_path(L, d_prev, d, d_out):
     x_exact = oracle.rotate(f64(h) @ wp.T, qq)[0]
     exact_i, _ = oracle.topk(x_exact, K)
     assert len(np.intersect1d(idx, exact_i)) >= 0.95 * K
+
+
+# ---------------------------------------------------------------- sparse + low rank
+
+@pytest.mark.parametrize("dtype,M,d_in,d_out,r,sparsity", [
+    (torch.float32, 1, 256, 512, 32, 40),
+    (torch.bfloat16, 1, 512, 256, 64, 40),
+    (torch.bfloat16, 4, 1024, 1032, 128, 50),
+    (torch.bfloat16, 16, 512, 256, 64, 40),
+    (torch.bfloat16, 1, 4096, 4096, 256, 40),
+    (torch.bfloat16, 2, 200, 24, 16, 0),
+])
+def test_sparse_lowrank_linear(L, dtype, M, d_in, d_out, r, sparsity):
+    """y = y_s + (x - sigma(x)) A_r B_r against the oracle on the same factors."""
+    K = sd.k_for_sparsity(d_in, sparsity)
+    W = sd.weights(d_in, d_out, 0.02 if dtype == torch.bfloat16 else 1 / 16, 1002, dtype)
+    A64, B64 = oracle.lowrank_factors(f64(W), r)
+    A = torch.from_numpy(A64).to(dtype)
+    B = torch.from_numpy(B64).to(dtype)
+    x = sd.activations(M, d_in, 1003, torch.float32)
+    xq = f64(x)
+    idx, val = oracle.topk(xq, K)
+    idx, val = idx.reshape(M, K), val.reshape(M, K)
+    st = status()
+    y = L.larosa_sparse_lowrank_linear(x.cuda(), torch.from_numpy(idx.astype(np.int32)).cuda(),
+                                       torch.from_numpy(val.astype(np.float32)).cuda(), W.cuda(),
+                                       A.cuda(), B.cuda(), dev_status=st)
+    assert L.larosa_check(st) == 0
+    ref = np.stack([oracle.sparse_lowrank_linear(xq[m], f64(W), f64(A), f64(B), idx[m]) for m in range(M)])
+    assert rel_inf(f64(y), ref) <= Y_TOL
