@@ -159,6 +159,25 @@ def _round_truncating(a):
     return np.ldexp(np.trunc(m * 256.0), e - 8)
 
 
+def _lowrank_full_spectrum(W, r):
+    U, S, Vt = np.linalg.svd(np.asarray(W, dtype=np.float64), full_matrices=False)
+    return U[:, :r] * S[None, :r], Vt[:r, :]
+
+
+def _lowrank_subtracts(x, W, A_r, B_r, idx):
+    x = np.asarray(x, dtype=np.float64)
+    kept = np.zeros_like(x)
+    kept[idx] = x[idx]
+    return kept @ W - (x - kept) @ A_r @ B_r
+
+
+def _lowrank_whole_input(x, W, A_r, B_r, idx):
+    x = np.asarray(x, dtype=np.float64)
+    kept = np.zeros_like(x)
+    kept[idx] = x[idx]
+    return kept @ W + x @ A_r @ B_r
+
+
 @pytest.mark.parametrize("check, broken", [
     (pins.check_rotate, _rotate_transposed),
     (pins.check_rotate, _rotate_dropped_term),
@@ -171,6 +190,9 @@ def _round_truncating(a):
     (lambda f: pins.check_prepare_weights(f, oracle.rotate), _prepare_untransposed),
     (pins.check_round_to_bf16, _round_truncating),
     (lambda f: pins.check_fold_rotation(f, oracle.rotate), _fold_untransposed),
+    (lambda f: pins.check_lowrank(f, oracle.sparse_lowrank_linear), _lowrank_full_spectrum),
+    (lambda f: pins.check_lowrank(oracle.lowrank_factors, f), _lowrank_subtracts),
+    (lambda f: pins.check_lowrank(oracle.lowrank_factors, f), _lowrank_whole_input),
 ])
 def test_planted_mistake_is_caught(check, broken):
     with pytest.raises(AssertionError):
