@@ -439,13 +439,9 @@ void* kernel_for(Elem w, Elem c, int MT) {
   return nullptr;
 }
 
-// Rows (and their coefficients) a CTA keeps in shared memory.  MT <= 4 stays
-// small enough for two CTAs per SM next to the 96 KB ring; MT = 8 and 16 run
-// one CTA per SM anyway, so they take enough rows that a batch's union of
-// kept rows (up to all 11008 inputs of a down projection) fits in one wave.
-int max_rows_per_cta(int MT) {
-  return MT <= 2 ? 1024 : (MT == 4 ? 512 : (MT == 8 ? 2048 : 1024));
-}
+// Rows (and their coefficients) a CTA keeps in shared memory; sized so that
+// MT <= 2 fits two CTAs per SM next to the 96 KB ring.
+int max_rows_per_cta(int MT) { return MT <= 2 ? 1024 : (MT <= 8 ? 512 : 256); }
 
 size_t smem_bytes_for(int MT) {
   const size_t pre = kHeaderBytes + (size_t)max_rows_per_cta(MT) * 4 * (1 + MT);
