@@ -870,21 +870,108 @@ __device__ __noinline__ KthEntry kth_by_bisection(const uint32_t* xkeys, int d, 
 }
 
 constexpr int kPre = 6;  // 16-byte vectors of x_rot per thread read with the histogram
+constexpr int kSubBits = 8;  // key bits below the bin that refine_boundary resolves
+static_assert(kRowKeys >= (1 << kSubBits), "the sub-bin histogram reuses s_rowkey");
+
+// When the boundary bin B holds more keys than the candidate slots (large d,
+// where a bin of bits 30..19 spans hundreds of entries): a histogram of the
+// next kSubBits key bits of B's keys, in shared memory (sub, 2^kSubBits
+// words), gives the sub-bin holding the krem-th largest of them (*B2), the
+// number of B's keys above it (*above2) and its own count (*n2).  Also writes
+// the bin numbers of all keys to bins and sets *nonfinite in a thread that
+// met a NaN or Inf, as select_kth does.  Requires 1 <= krem <= (keys in B).
+// All kT threads call it; it begins after and ends with a barrier.
+__device__ __forceinline__ void refine_boundary(const uint32_t* xkeys, int d, uint32_t B, uint32_t krem,
+                                             uint16_t* bins, uint32_t* sub, uint32_t* pick,
+                                             uint32_t* B2, uint32_t* above2, uint32_t* n2,
+                                             bool* nonfinite) {
+  constexpr int kSub = 1 << kSubBits;
+  constexpr int kLoads = 4;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int nv = d / 4;  // d is a multiple of 8
+  for (int j = tid; j < kSub; j += kT) sub[j] = 0u;
+  __syncthreads();
+  bool bad = false;
+  for (int v0 = tid; v0 < nv; v0 += kLoads * kT) {
+    uint4 u[kLoads];
+#pragma unroll
+    for (int k = 0; k < kLoads; ++k) {
+      const int v = v0 + k * kT;
+      u[k] = v < nv ? __ldcg(reinterpret_cast<const uint4*>(xkeys) + v) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int k = 0; k < kLoads; ++k) {
+      const int v = v0 + k * kT;
+      if (v < nv) {
+        const uint32_t w[4] = {u[k].x & kKeyMask, u[k].y & kKeyMask, u[k].z & kKeyMask, u[k].w & kKeyMask};
+        uint2 packed;
+        packed.x = (w[0] >> kFineShift) | ((w[1] >> kFineShift) << 16);
+        packed.y = (w[2] >> kFineShift) | ((w[3] >> kFineShift) << 16);
+        reinterpret_cast<uint2*>(bins)[v] = packed;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          bad |= w[e] >= 0x7f800000u;
+          if ((w[e] >> kFineShift) == B)
+            atomicAdd(sub + ((w[e] >> (kFineShift - kSubBits)) & (kSub - 1u)), 1u);
+        }
+      }
+    }
+  }
+  *nonfinite = bad;
+  __syncthreads();
+  if (tid < 32) {
+    // lane l holds the sub-bins hi, hi - 1, ..., hi - per + 1 (hi = kSub - 1 - per * l):
+    // counts from the top, the krem-th largest key lies in the first sub-bin
+    // where the running count reaches krem
+    constexpr int per = kSub / 32;
+    const int hi = kSub - 1 - per * lane;
+    uint32_t mine = 0;
+#pragma unroll
+    for (int j = 0; j < per; ++j) mine += sub[hi - j];
+    uint32_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    uint32_t run = incl - mine;
+    if (run < krem && krem <= incl) {  // exactly one lane
+      for (int j = 0; j < per; ++j) {
+        const uint32_t c = sub[hi - j];
+        if (run + c >= krem) {
+          pick[0] = static_cast<uint32_t>(hi - j);
+          pick[1] = run;
+          pick[2] = c;
+          break;
+        }
+        run += c;
+      }
+    }
+  }
+  __syncthreads();
+  *B2 = pick[0];
+  *above2 = pick[1];
+  *n2 = pick[2];
+  __syncthreads();  // pick may be written again
+}
 
 // The selector's pass over x_rot once the boundary bin B is known: writes
 // the bin number (bits 30..19) of every key to bins (shared memory), lists
-// B's keys with their indices in cand_key / cand_idx (in no particular
-// order: each warp reserves its slots with one atomic), ranks each against
-// the others (larger key first, then lower index) and returns the one
-// ranked krem - 1, i.e. the K-th entry (T, I).  Requires
-// 1 <= krem <= nB <= kFusedCandCap.  pre[k] holds the 16-byte vector
-// tid + k * kT of xkeys, read ahead by the caller.  The kFusedCandCap slots
+// the keys whose top bits (key >> shift) equal target -- B's keys, or after
+// refine_boundary those of one sub-bin of B -- with their indices in
+// cand_key / cand_idx (in no particular order: each warp reserves its slots
+// with one atomic), ranks each against the others (larger key first, then
+// lower index) and returns the one ranked krem - 1, i.e. the K-th entry
+// (T, I).  Requires 1 <= krem <= (keys listed) <= kFusedCandCap.  With
+// kHavePre, pre[k] holds the 16-byte vector tid + k * kT of xkeys, read
+// ahead by the caller; without, pre is not read.  The kFusedCandCap slots
 // of cand_key / cand_idx (16-byte aligned) hold key 0 and index 0xffffffff
 // on entry; cnt: a word of shared memory, zero on entry.  Sets *nonfinite
 // in a thread that met a NaN or Inf.  All kT threads call it; it begins
 // after and ends with a barrier.
-__device__ __forceinline__ KthEntry select_kth(const uint32_t* xkeys, int d, uint32_t B,
-                                               uint32_t krem, const uint4 (&pre)[kPre],
+template <bool kHavePre>
+__device__ __forceinline__ KthEntry select_kth(const uint32_t* xkeys, int d, int shift,
+                                               uint32_t target, uint32_t krem, const uint4 (&pre)[kPre],
                                                uint16_t* bins, uint32_t* cand_key,
                                                uint32_t* cand_idx, uint32_t* cnt, uint32_t* pick,
                                                bool* nonfinite) {
@@ -905,7 +992,7 @@ __device__ __forceinline__ KthEntry select_kth(const uint32_t* xkeys, int d, uin
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        hits += v < nv && (w[e] >> kFineShift) == B;
+        hits += v < nv && (w[e] >> shift) == target;
         bad |= v < nv && w[e] >= 0x7f800000u;
       }
     }
@@ -927,7 +1014,7 @@ __device__ __forceinline__ KthEntry select_kth(const uint32_t* xkeys, int d, uin
       const uint32_t w[4] = {u[k].x & kKeyMask, u[k].y & kKeyMask, u[k].z & kKeyMask, u[k].w & kKeyMask};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        if (v < nv && (w[e] >> kFineShift) == B) {
+        if (v < nv && (w[e] >> shift) == target) {
           if (slot < static_cast<uint32_t>(kFusedCandCap)) {
             cand_key[slot] = w[e];
             cand_idx[slot] = static_cast<uint32_t>(4 * v + e);
@@ -937,8 +1024,8 @@ __device__ __forceinline__ KthEntry select_kth(const uint32_t* xkeys, int d, uin
       }
     }
   };
-  list_batch(pre, 0);
-  for (int v0 = kPre * kT; v0 < nv; v0 += kPre * kT) {
+  if constexpr (kHavePre) list_batch(pre, 0);
+  for (int v0 = kHavePre ? kPre * kT : 0; v0 < nv; v0 += kPre * kT) {
     uint4 u[kPre];
 #pragma unroll
     for (int k = 0; k < kPre; ++k) {
@@ -980,6 +1067,28 @@ __device__ __forceinline__ KthEntry select_kth(const uint32_t* xkeys, int d, uin
   }
   __syncthreads();
   return KthEntry{pick[0], static_cast<int32_t>(pick[1])};
+}
+
+// The K-th entry where B holds more than kFusedCandCap keys: refine_boundary
+// narrows the candidates to one sub-bin of B; only when that too overflows
+// (heavy ties) does the bisection over all keys decide.  Out of line, so the
+// common path keeps its registers and code.  Arguments as for select_kth and
+// refine_boundary; sub: 2^kSubBits words of shared memory.
+__device__ __noinline__ KthEntry select_crowded(const uint32_t* xkeys, int d, int K, uint32_t B,
+                                                uint32_t krem, uint16_t* bins, uint32_t* sub,
+                                                uint32_t* cand_key, uint32_t* cand_idx, uint32_t* cnt,
+                                                uint32_t* pick, uint32_t* warp_sums, bool* nonfinite) {
+  uint32_t B2 = 0, above2 = 0, n2 = 0;
+  refine_boundary(xkeys, d, B, krem, bins, sub, pick, &B2, &above2, &n2, nonfinite);
+  if (n2 <= static_cast<uint32_t>(kFusedCandCap)) {
+    const uint4 unused[kPre] = {};
+    bool bad = false;
+    const KthEntry e = select_kth<false>(xkeys, d, kFineShift - kSubBits, (B << kSubBits) | B2, krem - above2,
+                                         unused, bins, cand_key, cand_idx, cnt, pick, &bad);
+    *nonfinite |= bad;
+    return e;
+  }
+  return kth_by_bisection(xkeys, d, K, warp_sums, pick);
 }
 
 // The kept list (idx, val: the K entries up to the K-th entry e, ascending
@@ -1259,22 +1368,16 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
     bool nonfinite = false;
     if (mode == 1u) {
       boundary_from_share<kT>(hcnt, K, s_warp_sums, s_pick, &B, &above, &nB);
+      // list B's keys, or where B holds more than the slots, those of the
+      // sub-bin of B that holds the K-th entry; only when that too overflows
+      // (heavy ties) does the bisection over all keys decide
+      const uint32_t krem = static_cast<uint32_t>(K) - above;
       if (nB <= static_cast<uint32_t>(kFusedCandCap)) {
-        e = select_kth(xkeys, d, B, static_cast<uint32_t>(K) - above, pre, bins, cand, cand_idx, s_word + 1,
-                       s_pick, &nonfinite);
+        e = select_kth<true>(xkeys, d, kFineShift, B, krem, pre, bins, cand, cand_idx, s_word + 1, s_pick,
+                             &nonfinite);
       } else {
-        const uint4* src = reinterpret_cast<const uint4*>(xkeys);
-        for (int v = tid; v < d / 4; v += kT) {
-          const uint4 u = __ldcg(src + v);
-          const uint32_t w[4] = {u.x & kKeyMask, u.y & kKeyMask, u.z & kKeyMask, u.w & kKeyMask};
-          nonfinite |= w[0] >= 0x7f800000u || w[1] >= 0x7f800000u || w[2] >= 0x7f800000u ||
-                       w[3] >= 0x7f800000u;
-          uint2 packed;
-          packed.x = (w[0] >> kFineShift) | ((w[1] >> kFineShift) << 16);
-          packed.y = (w[2] >> kFineShift) | ((w[3] >> kFineShift) << 16);
-          reinterpret_cast<uint2*>(bins)[v] = packed;
-        }
-        e = kth_by_bisection(xkeys, d, K, s_warp_sums, s_pick);
+        e = select_crowded(xkeys, d, K, B, krem, bins, s_rowkey, cand, cand_idx, s_word + 1, s_pick, s_warp_sums,
+                           &nonfinite);
       }
     }
     if (tid == 0) {

@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-tokens", type=int, default=4,
                     help="tokens in the CPU oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-model-configs", action="store_true",
+                    help="skip the 32-layer 7B stack, the 13B batch sweep and the 70B slice")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -292,6 +294,234 @@ def workload_config(sparsity: float, graph: bool) -> dict:
         "l2": "inputs larger than L2: 586 MB of rotations and kept rows per step vs 126 MB L2, no flush",
         "cuda_graph": graph,
     }
+
+
+# ---------------------------------------------------------------- the other workloads
+
+class PerfGroup:
+    """One projection group of a perf-only layer (no dense weight kept)."""
+
+    def __init__(self, name, d_in, d_out, Qt, W_rot, x):
+        self.name, self.d_in, self.d_out = name, d_in, d_out
+        self.Qt, self.W_rot, self.x = Qt, W_rot, x
+
+
+def perf_layers(torch, sd, hidden: int, ffn: int, kv: int, n_layers: int, workload_id: int, M: int,
+                device) -> list:
+    """``n_layers`` decoder layers of distinct, device-resident tensors.
+
+    Rotations: one seeded Haar rotation per input width (fp32 QR on the
+    device, rounded to bf16), and for every layer and group a seeded signed
+    permutation of its rows, which is again orthogonal.  W_rot is drawn
+    directly as N(0, 0.02^2): for a Gaussian W, Q^T W has that distribution.
+    Activations are the heavy-tailed rows of the single-layer workload.
+    """
+    projs = sd.llama_layer(hidden, ffn, kv)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(sd.seed_for(workload_id, 999, 0))
+    base = {}
+    for p in projs:
+        if p.d_in not in base:
+            base[p.d_in] = sd.orthogonal(p.d_in, sd.seed_for(workload_id, 999, p.d_in % 997),
+                                         device=device).to(torch.bfloat16)
+    layers = []
+    for layer in range(n_layers):
+        gs = []
+        for p in projs:
+            perm = torch.randperm(p.d_in, generator=gen, device=device)
+            sign = torch.randint(0, 2, (p.d_in, 1), generator=gen, device=device).to(torch.bfloat16) * 2 - 1
+            Qt = (base[p.d_in][perm] * sign).contiguous()
+            W_rot = torch.randn((p.d_in, p.d_out), generator=gen, device=device, dtype=torch.float32)
+            W_rot = W_rot.mul_(0.02).to(torch.bfloat16)
+            x = sd.activations(M, p.d_in, sd.seed_for(workload_id, layer, 10 * p.q_id + 3), torch.bfloat16,
+                               device=device)
+            gs.append(PerfGroup(p.name, p.d_in, p.d_out, Qt, W_rot, x))
+        layers.append(gs)
+    del base
+    torch.cuda.synchronize(device)
+    return layers
+
+
+def bench_model_configs(args, torch, L, sd, device, stream, world, graph_of, time_graph, peak) -> dict:
+    """The other workloads of the path, each with its own device-resident tensors.
+
+    * llama2-7b-stack: 32 decoder layers (128 fused calls per token), at 0,
+      25, 40 and 50 % sparsity, from a CUDA graph and from eager launches;
+      the library's dense bf16 GEMV over the same stack; microseconds per
+      projection group (one group's 32 calls back to back);
+    * llama2-13b-layer: the fused path with M = 1, 2, 4, 8, 16 tokens per
+      call, each token its own Top-K (bytes: Q once plus the union of kept rows);
+    * llama2-70b-slice: 8 layers (q|k|v 8192x10240 with GQA, ffn 28672) at 40
+      and 50 %, and the dense GEMV.
+    Each is timed over a short run (inputs far larger than L2) and freed
+    before the next is built.
+    """
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    n = max(10, min(100, args.steps // 30))
+    out = {}
+    t0 = time.time()
+
+    def log(msg):
+        print(f"[bench] {msg}: {time.time() - t0:.1f} s", file=sys.stderr, flush=True)
+
+    def time_eager(fn, steps):
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                fn()
+        torch.cuda.synchronize(device)
+        barrier(world, device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps):
+                fn()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(world, device)
+        return e0.elapsed_time(e1) / 1e3
+
+    def rate(t, steps, tokens_per_step, step_bytes):
+        tps, t_max = aggregate(t, steps * tokens_per_step, world, device)
+        return {"tokens_per_s": tps, "ms_per_token": t_max * 1e3 / (steps * tokens_per_step),
+                "gb_per_token": step_bytes / tokens_per_step / 1e9,
+                "hbm_frac": step_bytes * steps / t_max / 1e9 / peak}
+
+    def fused_bytes(layers, sp):
+        return sum(path_bytes(g, sd.k_for_sparsity(g.d_in, sp))["total"] for gs in layers for g in gs)
+
+    def dense_bytes(layers):
+        return sum(g.d_in * g.d_out * 2 + g.d_in * 2 + g.d_out * 4 for gs in layers for g in gs)
+
+    def presize(ws, layers, Ms=(1,)):
+        for g in layers[0]:
+            for M in Ms:
+                ws.get(M, g.d_in, g.d_out, g.d_in)
+
+    # ---- 7B: 32-layer stack
+    layers = perf_layers(torch, sd, 4096, 11008, 4096, 32, 2, 1, device)
+    log("7B stack built")
+    ws = L.Workspace(device)
+    presize(ws, layers)
+    ys = {g.name: torch.empty((1, g.d_out), dtype=torch.float32, device=device) for g in layers[0]}
+
+    def stack_step(sp, only=None):
+        Ks = {g.name: sd.k_for_sparsity(g.d_in, sp) for g in layers[0]}
+
+        def step():
+            for gs in layers:
+                for g in gs:
+                    if only is None or g.name == only:
+                        L.larosa_rotate_topk_linear(g.x, g.Qt, g.W_rot, Ks[g.name], y=ys[g.name], ws=ws,
+                                                    dev_status=st)
+        return step
+
+    def dense_stack():
+        # the dense GEMV reads an nn.Linear-layout [d_out x d_in] weight: each
+        # layer's random W_rot buffer serves as one (same bytes, random values)
+        for gs in layers:
+            for g in gs:
+                L.larosa_dense_linear(g.x, g.W_rot.view(g.d_out, g.d_in), y=ys[g.name])
+
+    stack = {"layers": 32, "calls_per_token": 128, "fused": {}}
+    for sp in (0.0, 25.0, 40.0, 50.0):
+        gr = graph_of(stack_step(sp))
+        stack["fused"][f"{sp:g}%"] = rate(time_graph(gr, n, args.warmup)[0], n, 1, fused_bytes(layers, sp))
+        del gr
+    stack["fused_eager_40%"] = rate(time_eager(stack_step(40.0), n), n, 1, fused_bytes(layers, 40.0))
+    gr = graph_of(dense_stack)
+    stack["dense"] = rate(time_graph(gr, n, args.warmup)[0], n, 1, dense_bytes(layers))
+    del gr
+    stack["dense_eager"] = rate(time_eager(dense_stack, n), n, 1, dense_bytes(layers))
+    stack["fused_vs_dense_40%"] = stack["fused"]["40%"]["tokens_per_s"] / stack["dense"]["tokens_per_s"]
+    us = {}
+    for g in layers[0]:
+        gr = graph_of(stack_step(40.0, only=g.name))
+        t, _ = time_graph(gr, n, args.warmup)
+        us[g.name] = reduce_max(t, world, device) / (n * 32) * 1e6
+        del gr
+    stack["us_per_projection_40%"] = us
+    out["llama2-7b-stack"] = stack
+    log("7B stack timed")
+    del layers, ws, ys
+    torch.cuda.empty_cache()
+
+    # ---- 13B: one layer, M tokens per call
+    Ms = (1, 2, 4, 8, 16)
+    per_M = {M: perf_layers(torch, sd, 5120, 13824, 5120, 1, 3, M, device)[0] for M in Ms}
+    ws = L.Workspace(device)
+    presize(ws, [per_M[1]], Ms)
+    ysM = {M: {g.name: torch.empty((M, g.d_out), dtype=torch.float32, device=device) for g in per_M[M]}
+           for M in Ms}
+    sweep = {}
+    for M in Ms:
+        gs = per_M[M]
+        Ks = {g.name: sd.k_for_sparsity(g.d_in, 40.0) for g in gs}
+
+        def step(gs=gs, Ks=Ks, M=M):
+            for g in gs:
+                L.larosa_rotate_topk_linear(g.x, g.Qt, g.W_rot, Ks[g.name], y=ysM[M][g.name], ws=ws,
+                                            dev_status=st)
+        nbytes = 0
+        for g in gs:
+            idx, _ = L.larosa_topk(L.larosa_rotate(g.x, g.Qt), Ks[g.name], dev_status=st)
+            rows = int(torch.unique(idx.flatten()).numel())
+            nbytes += rows * g.d_out * 2 + g.d_in * g.d_in * 2 + M * (g.d_in * 6 + Ks[g.name] * 8 + g.d_out * 4)
+        gr = graph_of(step)
+        sweep[f"M={M}"] = rate(time_graph(gr, n, args.warmup)[0], n, M, nbytes)
+        del gr
+    out["llama2-13b-layer"] = {"batch_sweep_40%": sweep}
+    log("13B layer timed")
+    del per_M, ws, ysM
+    torch.cuda.empty_cache()
+
+    # ---- 70B: 8-layer slice
+    layers = perf_layers(torch, sd, 8192, 28672, 1024, 8, 4, 1, device)
+    log("70B slice built")
+    ws = L.Workspace(device)
+    presize(ws, layers)
+    ys = {g.name: torch.empty((1, g.d_out), dtype=torch.float32, device=device) for g in layers[0]}
+    slc = {"layers": 8, "fused": {}}
+    for sp in (40.0, 50.0):
+        gr = graph_of(stack_step(sp))
+        slc["fused"][f"{sp:g}%"] = rate(time_graph(gr, n, args.warmup)[0], n, 1, fused_bytes(layers, sp))
+        del gr
+    gr = graph_of(dense_stack)
+    slc["dense"] = rate(time_graph(gr, n, args.warmup)[0], n, 1, dense_bytes(layers))
+    del gr
+    out["llama2-70b-slice"] = slc
+    log("70B slice timed")
+    del layers, ws, ys
+    torch.cuda.empty_cache()
+    assert L.larosa_check(st, device=device) == 0
+    out["timed_steps"] = n
+    return out
+
+
+def read_probe(torch, L, device, stream, warmup: int) -> dict:
+    """Pure-read bandwidth: the library's dense GEMV over a 4 GiB bf16 weight
+    (one token: the weight is the whole traffic) and torch's sum of the same
+    buffer, each timed with CUDA events over 10 passes."""
+    d_in, d_out = 32768, 65536
+    W = torch.empty((d_out, d_in), dtype=torch.bfloat16, device=device).normal_()
+    x = torch.ones((1, d_in), dtype=torch.bfloat16, device=device)
+    y = torch.empty((1, d_out), dtype=torch.float32, device=device)
+    res = {}
+    for name, fn in (("dense_gemv_gbs", lambda: L.larosa_dense_linear(x, W, y=y)),
+                     ("torch_sum_gbs", lambda: torch.sum(W, dtype=torch.float32))):
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(10):
+                fn()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+        res[name] = W.numel() * 2 * 10 / (e0.elapsed_time(e1) / 1e3) / 1e9
+    del W
+    torch.cuda.empty_cache()
+    res["bytes"] = d_in * d_out * 2
+    return res
 
 
 # ---------------------------------------------------------------- larosa arm
@@ -578,6 +808,12 @@ def bench_larosa(args):
     e2e_value, _ = aggregate(t_e2e, e2e_steps, world, device)
     assert all(torch.isfinite(y).all() for y in y_host)
 
+    # ---- the other workloads and the pure-read probe
+    model_cfgs = None
+    if not args.no_model_configs:
+        model_cfgs = bench_model_configs(args, torch, L, sd, device, stream, world, graph_of, time_graph, peak)
+    probe = read_probe(torch, L, device, stream, args.warmup)
+
     # ---- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -602,6 +838,7 @@ def bench_larosa(args):
                                    "in one cooperative launch; bf16)",
                          "bound": "hbm", "achieved": fused_gbs, "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": fused_gbs / peak, "traffic": traffic,
+                         "frac_of_nominal_8tbs": fused_gbs / 8000.0,
                          "algorithmic_bytes_per_launch": step_bytes / len(groups),
                          "avg_launch_us": fused_us, "share_of_step": 1.0},
             "kernels": {
@@ -657,6 +894,8 @@ def bench_larosa(args):
                 f"M={M}": {"tokens_per_s": M * side_steps / t * world,
                            "hbm_frac": batch_bytes[M] * side_steps / t / 1e9 / peak}
                 for M, t in t_batch.items()},
+            "model_configs": model_cfgs,
+            "read_probe": probe,
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": sum(g.x.numel() * g.x.element_size() for g in groups),
                     "d2h_bytes_per_step": sum(g.d_out * 4 for g in groups)},

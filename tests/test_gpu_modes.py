@@ -184,6 +184,49 @@ def test_fused_identity_topk(L, dtype, M, d_in, d_out, sparsity):
     assert rel_inf(f64(y), ref) <= Y_TOL
 
 
+def crowded_row(d: int, n_high: int, n_bin: int, width: float, seed: int, dtype) -> np.ndarray:
+    """One row whose Top-K boundary falls inside a crowded 12-bit key bin.
+
+    n_high magnitudes in [2, 4) (certainly kept), n_bin in [1, 1 + width)
+    (one bin of bits 30..19 when width <= 1/16), the rest in [0, 0.5); random
+    signs and positions.  Rounded to ``dtype``, so bf16 rows carry ties.
+    """
+    rng = np.random.default_rng(seed)
+    mag = rng.uniform(0.0, 0.5, d)
+    pos = rng.permutation(d)
+    mag[pos[:n_high]] = rng.uniform(2.0, 4.0, n_high)
+    mag[pos[n_high:n_high + n_bin]] = 1.0 + rng.uniform(0.0, width, n_bin)
+    x = mag * rng.choice([-1.0, 1.0], d)
+    return torch.from_numpy(x[None, :]).to(dtype)
+
+
+@pytest.mark.parametrize("dtype,d,n_high,n_bin,width", [
+    (torch.float32, 4096, 500, 2000, 1 / 16),       # B holds 2000 keys: one sub-bin of ~8 is ranked
+    (torch.float32, 4096, 300, 1500, 1 / 4096),     # 1500 keys within one sub-bin: the bisection decides
+    (torch.bfloat16, 8192, 1000, 2400, 1 / 16),     # bf16: 8 distinct keys in B, hundreds of ties each
+    (torch.bfloat16, 28672, 2000, 3600, 1 / 16),    # the 70B down-projection width
+])
+def test_fused_identity_crowded_boundary_bin(L, dtype, d, n_high, n_bin, width):
+    """The selector where the boundary bin holds more keys than its candidate slots."""
+    d_out = 512
+    W = sd.weights(d, d_out, 0.02 if dtype == torch.bfloat16 else 1 / 16, 922, dtype)
+    x = crowded_row(d, n_high, n_bin, width, 923, dtype)
+    xq = f64(x)
+    for K in (n_high + 1, n_high + n_bin // 3, n_high + n_bin - 1):
+        ws = L.Workspace()
+        buf = ws.get(1, d, d_out, K)
+        st = status()
+        y = L.larosa_rotate_topk_linear(x.cuda(), None, W.cuda(), K, ws=ws, dev_status=st)
+        assert L.larosa_check(st) == 0
+        o_x, o_i, _ = L.larosa_workspace_layout(1, d, d_out, K)
+        assert np.array_equal(f64(buf[o_x:o_x + d * 4].view(torch.float32).view(1, d)), xq)
+        idx = buf[o_i:o_i + K * 4].view(torch.int32).cpu().numpy().astype(np.int64)
+        want_i, want_v = oracle.topk(xq, K)
+        assert np.array_equal(idx, want_i.reshape(K)), K
+        ref = oracle.sparse_linear(want_i.reshape(K), want_v.reshape(K), f64(W))
+        assert rel_inf(f64(y)[0], ref) <= Y_TOL
+
+
 @pytest.mark.parametrize("dtype,M,d_in,d_out", [
     (torch.bfloat16, 1, 4096, 4096),
     (torch.bfloat16, 1, 11008, 4096),
