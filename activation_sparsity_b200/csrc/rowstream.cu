@@ -64,6 +64,7 @@ struct Params {
   int M;
   float* y;
   int y_ld;
+  int accumulate;  // 1: y += the product (y was written by an earlier kernel)
   float* partials;
   unsigned* tickets;
   int col_tile;
@@ -364,7 +365,8 @@ __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_ke
     for (int e = tid; e < Mw * ns; e += kThreads) {
       const int m = e / ns;
       const int c = cs0 + (e - m * ns);
-      p.y[(size_t)m * p.y_ld + c0 + c] = outs[e];
+      float* yo = p.y + (size_t)m * p.y_ld + c0 + c;
+      *yo = p.accumulate ? *yo + outs[e] : outs[e];
     }
     return;
   }
@@ -390,7 +392,8 @@ __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_ke
     const int c = cs0 + (e - m * ns);
     float s = 0.f;
     for (int k = 0; k < n_clusters; ++k) s += __ldcg(all + ((size_t)k * Mw + m) * p.col_tile + c);
-    p.y[(size_t)m * p.y_ld + c0 + c] = s;
+    float* yo = p.y + (size_t)m * p.y_ld + c0 + c;
+    *yo = p.accumulate ? *yo + s : s;
   }
   if (tid == 0) atomicExch(ticket, 0u);
 }
@@ -586,6 +589,7 @@ cudaError_t launch_gemv(const GemvArgs& a, const GemvPlan& pl, cudaStream_t stre
   p.M = a.M;
   p.y = a.y;
   p.y_ld = a.y_ld;
+  p.accumulate = a.accumulate ? 1 : 0;
   p.partials = a.partials;
   p.tickets = a.tickets;
   p.col_tile = pl.col_tile;
