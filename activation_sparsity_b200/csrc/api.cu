@@ -275,7 +275,7 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
 // partials of the two GEMVs through the factors.
 struct LowrankLayout {
   Layout base;
-  size_t x_drop = 0, u = 0, partials = 0, total = 0;
+  size_t x_drop = 0, u = 0, y_r = 0, partials = 0, total = 0;
 };
 
 int make_lowrank_layout(int M, int d_in, int d_out, int K, int r, LowrankLayout* LL) {
@@ -300,16 +300,15 @@ int make_lowrank_layout(int M, int d_in, int d_out, int K, int r, LowrankLayout*
   };
   LL->x_drop = take((size_t)M * d_in * 4);
   LL->u = take((size_t)M * r * 4);
+  LL->y_r = take((size_t)M * d_out * 4);
   LL->partials = take(pf * 4);
   LL->total = off;
   return LAROSA_OK;
 }
 
-// out[M x cols] = coef[M x rows] . Wm[rows x cols] (all rows, fp32 coefficients);
-// with accumulate, out += that product instead.
+// out[M x cols] = coef[M x rows] . Wm[rows x cols] (all rows, fp32 coefficients).
 int run_dense_gemv(const void* Wm, int rows, int cols, const float* coef, int M, float* out,
-                   bool accumulate, int dtype, void* ws, float* partials, int* dev_status,
-                   cudaStream_t s) {
+                   int dtype, void* ws, float* partials, int* dev_status, cudaStream_t s) {
   GemvPlan pl;
   cudaError_t e = larosa::plan_gemv(elem_of(dtype), Elem::F32, M, cols, rows, &pl);
   if (e != cudaSuccess) return cuda_fail(e, "plan low-rank GEMV");
@@ -326,7 +325,6 @@ int run_dense_gemv(const void* Wm, int rows, int cols, const float* coef, int M,
   a.M = M;
   a.y = out;
   a.y_ld = cols;
-  a.accumulate = accumulate;
   a.partials = partials;
   a.tickets = reinterpret_cast<unsigned*>(at(ws, kOffTickets));
   a.dev_status = dev_status;
@@ -699,16 +697,20 @@ int larosa_sparse_lowrank_linear(const float* x, const int32_t* idx, const float
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* x_drop = reinterpret_cast<float*>(at(ws, LL.x_drop));
   float* u = reinterpret_cast<float*>(at(ws, LL.u));
+  float* y_r = reinterpret_cast<float*>(at(ws, LL.y_r));
   float* part = reinterpret_cast<float*>(at(ws, LL.partials));
   // y_s: the kept rows of W
   st = run_sparse(idx, val, M, K, W, d_in, d_out, y, dtype, ws, LL.base, dev_status, s);
   if (st != LAROSA_OK) return st;
-  // y_r = ((x - sigma(x)) . A_r) . B_r, added into y by the last GEMV
+  // y_r = ((x - sigma(x)) . A_r) . B_r, then y = y_s + y_r
   cudaError_t e = larosa::launch_dropped(x, idx, M, K, d_in, x_drop, dev_status, s);
   if (e != cudaSuccess) return cuda_fail(e, "dropped-part kernel");
-  st = run_dense_gemv(A_r, d_in, r, x_drop, M, u, false, dtype, ws, part, dev_status, s);
+  st = run_dense_gemv(A_r, d_in, r, x_drop, M, u, dtype, ws, part, dev_status, s);
   if (st != LAROSA_OK) return st;
-  return run_dense_gemv(B_r, r, d_out, u, M, y, true, dtype, ws, part, dev_status, s);
+  st = run_dense_gemv(B_r, r, d_out, u, M, y_r, dtype, ws, part, dev_status, s);
+  if (st != LAROSA_OK) return st;
+  e = larosa::launch_add(y, y_r, M * d_out, s);
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "add kernel");
 }
 
 int larosa_dense_linear(const void* x, const void* Wt, int M, int d_in, int d_out, float* y,

@@ -43,7 +43,6 @@ struct GemvArgs {
   int M = 1;
   float* y = nullptr;
   int y_ld = 0;
-  bool accumulate = false;  // y += the product instead of y = the product
   float* partials = nullptr;
   unsigned* tickets = nullptr;
   int* dev_status = nullptr;
@@ -69,9 +68,11 @@ cudaError_t launch_threshold(const float* x_rot, int M, int d, uint32_t t_key, i
                              float* val, int32_t* nnz, float* coef, unsigned* bitmap,
                              int* dev_status, cudaStream_t stream);
 
-// Low-rank compensation: x_drop = x with each token's kept entries zeroed.
+// Low-rank compensation: x_drop = x with each token's kept entries zeroed;
+// y += add (n elements).
 cudaError_t launch_dropped(const float* x, const int32_t* idx, int M, int K, int d, float* x_drop,
                            int* dev_status, cudaStream_t stream);
+cudaError_t launch_add(float* y, const float* add, int n, cudaStream_t stream);
 
 // x_rot[i] = x[i] widened to fp32 (the identity rotation), n elements.
 cudaError_t launch_widen(const void* x, float* x_rot, int n, Elem elem, cudaStream_t stream);

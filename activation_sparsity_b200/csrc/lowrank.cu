@@ -1,13 +1,14 @@
-// Low-rank compensation of the dropped entries (sm_100a): the kernel that
-// forms the dropped part ahead of the row-streaming GEMVs of
-// larosa_sparse_lowrank_linear.
+// Low-rank compensation of the dropped entries (sm_100a): the two small
+// kernels around the row-streaming GEMVs of larosa_sparse_lowrank_linear.
 //
 // R-Sparse report, 研究流程与方法 / R-Sparse框架设计 (hybrid computation): the
 // entries a selection drops are not discarded but sent through rank-r
 // factors of the weight, y = y_s + (x - sigma(x)) . A_r . B_r.  The dropped
 // part is x with the kept entries set to zero; the two products with the
-// factors and the sparse product are GEMVs of the library, the last of which
-// adds its result into y.
+// factors and the sparse product are GEMVs of the library; the sum is the
+// last step.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -40,6 +41,14 @@ __global__ void __launch_bounds__(kThreads) dropped_kernel(const float* __restri
   if (__syncthreads_or(bad) && threadIdx.x == 0) report(dev_status, LAROSA_DEV_INDEX);
 }
 
+// y[i] += add[i], n elements.
+__global__ void __launch_bounds__(kThreads) add_kernel(float* __restrict__ y,
+                                                       const float* __restrict__ add, int n) {
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int i = blockIdx.x * kThreads + threadIdx.x; i < n; i += gridDim.x * kThreads) y[i] += add[i];
+}
+
 cudaError_t launch_pdl(const void* fn, int grid, void** args, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
@@ -59,6 +68,12 @@ cudaError_t launch_dropped(const float* x, const int32_t* idx, int M, int K, int
                            int* dev_status, cudaStream_t stream) {
   void* args[] = {&x, &idx, &K, &d, &x_drop, &dev_status};
   return launch_pdl(reinterpret_cast<const void*>(&dropped_kernel), M, args, stream);
+}
+
+cudaError_t launch_add(float* y, const float* add, int n, cudaStream_t stream) {
+  const int grid = std::max(1, std::min((n + kThreads - 1) / kThreads, 296));
+  void* args[] = {&y, &add, &n};
+  return launch_pdl(reinterpret_cast<const void*>(&add_kernel), grid, args, stream);
 }
 
 }  // namespace larosa

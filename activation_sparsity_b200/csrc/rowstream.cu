@@ -64,7 +64,6 @@ struct Params {
   int M;
   float* y;
   int y_ld;
-  int accumulate;  // 1: y += the product (y was written by an earlier kernel)
   float* partials;
   unsigned* tickets;
   int col_tile;
@@ -365,8 +364,7 @@ __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_ke
     for (int e = tid; e < Mw * ns; e += kThreads) {
       const int m = e / ns;
       const int c = cs0 + (e - m * ns);
-      float* yo = p.y + (size_t)m * p.y_ld + c0 + c;
-      *yo = p.accumulate ? *yo + outs[e] : outs[e];
+      p.y[(size_t)m * p.y_ld + c0 + c] = outs[e];
     }
     return;
   }
@@ -392,8 +390,7 @@ __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_ke
     const int c = cs0 + (e - m * ns);
     float s = 0.f;
     for (int k = 0; k < n_clusters; ++k) s += __ldcg(all + ((size_t)k * Mw + m) * p.col_tile + c);
-    float* yo = p.y + (size_t)m * p.y_ld + c0 + c;
-    *yo = p.accumulate ? *yo + s : s;
+    p.y[(size_t)m * p.y_ld + c0 + c] = s;
   }
   if (tid == 0) atomicExch(ticket, 0u);
 }
@@ -589,7 +586,6 @@ cudaError_t launch_gemv(const GemvArgs& a, const GemvPlan& pl, cudaStream_t stre
   p.M = a.M;
   p.y = a.y;
   p.y_ld = a.y_ld;
-  p.accumulate = a.accumulate ? 1 : 0;
   p.partials = a.partials;
   p.tickets = a.tickets;
   p.col_tile = pl.col_tile;

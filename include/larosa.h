@@ -283,8 +283,8 @@ int larosa_rotate_threshold_linear(const void *x, const void *Qt,
  * all of `dtype` (the factors of an offline SVD W ~ U S V^T: A_r = U_r
  * S_r^1/2, B_r = S_r^1/2 V_r^T); y: [M x d_out] fp32.  d_out and r rows of
  * 16 bytes; x, W, A_r, B_r, y 16-byte aligned.  Kernels: the sparse linear
- * on the kept list, the dropped part of x, then u = dropped . A_r and
- * y += u . B_r by the row-streaming GEMV with fp32 coefficients.
+ * on the kept list, the dropped part of x, u = dropped . A_r and y_r = u . B_r
+ * by the row-streaming GEMV with fp32 coefficients, and y += y_r.
  * ws: at least larosa_lowrank_workspace_bytes(M, d_in, d_out, K, r) bytes.
  */
 int larosa_sparse_lowrank_linear(const float *x, const int32_t *idx,
