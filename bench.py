@@ -784,9 +784,17 @@ def bench_larosa(args):
     traffic = profiled_traffic("fused")
 
     # ---- end to end through the public API with host buffers
-    x_host = [g.x.cpu().pin_memory() for g in groups]
-    x_dev = [torch.empty_like(g.x) for g in groups]
-    y_host = [torch.empty((1, g.d_out), dtype=torch.float32).pin_memory() for g in groups]
+    # the four groups' inputs live in one pinned host buffer and one device
+    # buffer (and likewise the outputs), so a step moves them with one copy
+    # each way
+    x_sizes = [g.x.numel() for g in groups]
+    y_sizes = [g.d_out for g in groups]
+    x_host_all = torch.cat([g.x.flatten().cpu() for g in groups]).pin_memory()
+    x_dev_all = torch.empty_like(x_host_all, device=device)
+    x_dev = [v.view(1, -1) for v in torch.split(x_dev_all, x_sizes)]
+    y_dev_all = torch.empty(sum(y_sizes), dtype=torch.float32, device=device)
+    y_dev = [v.view(1, -1) for v in torch.split(y_dev_all, y_sizes)]
+    y_host_all = torch.empty(sum(y_sizes), dtype=torch.float32).pin_memory()
     e2e_steps = max(20, min(500, args.steps // 10))
     with torch.cuda.stream(stream):
         for r in range(args.warmup + e2e_steps):
@@ -796,17 +804,15 @@ def bench_larosa(args):
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
             # the step's inputs in, the four groups back to back, the outputs out
-            for gi in range(len(groups)):
-                x_dev[gi].copy_(x_host[gi], non_blocking=True)
+            x_dev_all.copy_(x_host_all, non_blocking=True)
             for gi, g in enumerate(groups):
-                L.larosa_rotate_topk_linear(x_dev[gi], g.Qt, g.W_rot, g.K, y=ys[gi], ws=ws, dev_status=st)
-            for gi in range(len(groups)):
-                y_host[gi].copy_(ys[gi], non_blocking=True)
+                L.larosa_rotate_topk_linear(x_dev[gi], g.Qt, g.W_rot, g.K, y=y_dev[gi], ws=ws, dev_status=st)
+            y_host_all.copy_(y_dev_all, non_blocking=True)
         e1.record(stream)
     torch.cuda.synchronize(device)
     t_e2e = e0.elapsed_time(e1) / 1e3
     e2e_value, _ = aggregate(t_e2e, e2e_steps, world, device)
-    assert all(torch.isfinite(y).all() for y in y_host)
+    assert torch.isfinite(y_host_all).all()
 
     # ---- the other workloads and the pure-read probe
     model_cfgs = None
