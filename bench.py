@@ -338,7 +338,8 @@ def perf_layers(torch, sd, hidden: int, ffn: int, kv: int, n_layers: int, worklo
             gs.append(PerfGroup(p.name, p.d_in, p.d_out, Qt, W_rot, x))
         layers.append(gs)
     del base
-    torch.cuda.synchronize(device)
+    if torch.device(device).type == "cuda":
+        torch.cuda.synchronize(device)
     return layers
 
 
