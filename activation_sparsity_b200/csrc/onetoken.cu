@@ -18,7 +18,7 @@
 //         reads W in torch.nn.Linear layout.  Each warp owns whole output rows:
 //         no cross-CTA reduction at all.
 //
-// gather  y[c] = sum_{p < K} coef(p) * W[row(p)][c], W row-major
+// gather  y[c] = sum_{p < K} val[p] * W[idx[p]][c], W row-major
 //         [d_in x d_out]: the sparse linear over the kept rows of the
 //         counter-rotated weight (abstract: activation sparsity reduces memory
 //         transfers).  One thread-block cluster per column tile; the cluster's
@@ -26,11 +26,11 @@
 //         partial sums through distributed shared memory in rank order, so
 //         nothing leaves the cluster but y.  The tile width is chosen so the
 //         clusters that fit on the GPU at once cover d_out.
-//           kGather  row(p) = idx[p], coef(p) = val[p]
-//           kSelect  every CTA first selects the K largest |x_rot| itself
-//                    (exact, ties to the lower index; no grid-wide handoff
-//                    and no exchange inside the cluster), then takes its
-//                    part of the kept list.
+//
+// rotsel  the rotation with the Top-K by the last CTA to arrive, and fused
+//         the whole one-token path in one cooperative launch (rotation,
+//         selection by one CTA, gather of the kept rows by the others); each
+//         is described at its kernel below.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -442,12 +442,8 @@ __device__ __forceinline__ void gather_tile(cg::cluster_group& cl, int rank, con
 // One cluster of C CTAs per column tile.  The cluster's CTAs take equal
 // consecutive parts of the kept list (in ascending row order), stream those
 // rows of the tile, and add their partial sums through distributed shared
-// memory in rank order.
-//
-// Select mode: every CTA reads all d rotated entries and selects the K
-// largest magnitudes itself (exact; ties to the lower index), so no CTA
-// waits on another before streaming.  The same integer-only selection runs
-// in every CTA, so all of them derive the same kept list.
+// memory in rank order.  An index outside [0, d_in) sets LAROSA_DEV_INDEX
+// and is read as row 0 with coefficient 0.
 template <typename Tw, int C>
 __global__ void __launch_bounds__(kT, 2) gather_kernel(const GParams p) {
   constexpr int CPT = 16 / sizeof(Tw);  // columns per thread per row

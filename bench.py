@@ -28,6 +28,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -187,11 +188,21 @@ def measured_peaks() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C++/CUDA source without its comments, blank lines and trailing spaces."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", line).rstrip() for line in text.splitlines())
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_source_hash() -> str:
+    """Hash of the fused kernel's code (onetoken.cu, common.cuh, select.cuh),
+    comments excluded: a stored ncu capture stays valid while only comments
+    change, and is dropped as soon as the code does."""
     h = hashlib.sha256()
     for name in ("onetoken.cu", "common.cuh", "select.cuh"):
-        with open(os.path.join(ROOT, "activation_sparsity_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "activation_sparsity_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
