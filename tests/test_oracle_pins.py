@@ -159,6 +159,22 @@ def _round_truncating(a):
     return np.ldexp(np.trunc(m * 256.0), e - 8)
 
 
+def _dense_drops_last_input(x, W):
+    x = np.asarray(x, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    return x[..., :-1] @ W[:-1]
+
+
+def _threshold_strict(x, t):
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    return [(np.nonzero(np.abs(r) > t)[0], r[np.abs(r) > t]) for r in x]
+
+
+def _threshold_signed(x, t):
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    return [(np.nonzero(r >= t)[0], r[r >= t]) for r in x]
+
+
 def _lowrank_full_spectrum(W, r):
     U, S, Vt = np.linalg.svd(np.asarray(W, dtype=np.float64), full_matrices=False)
     return U[:, :r] * S[None, :r], Vt[:r, :]
@@ -190,6 +206,9 @@ def _lowrank_whole_input(x, W, A_r, B_r, idx):
     (lambda f: pins.check_prepare_weights(f, oracle.rotate), _prepare_untransposed),
     (pins.check_round_to_bf16, _round_truncating),
     (lambda f: pins.check_fold_rotation(f, oracle.rotate), _fold_untransposed),
+    (pins.check_dense_linear, _dense_drops_last_input),
+    (lambda f: pins.check_threshold_select(f, oracle.topk), _threshold_strict),
+    (lambda f: pins.check_threshold_select(f, oracle.topk), _threshold_signed),
     (lambda f: pins.check_lowrank(f, oracle.sparse_lowrank_linear), _lowrank_full_spectrum),
     (lambda f: pins.check_lowrank(oracle.lowrank_factors, f), _lowrank_subtracts),
     (lambda f: pins.check_lowrank(oracle.lowrank_factors, f), _lowrank_whole_input),
