@@ -226,9 +226,13 @@ def profiled_traffic(kernel: str):
 def cpu_layer_inputs(sparsity: float, seed_layer: int = 0):
     """fp64 host arrays of the 7B layer for the oracle.
 
-    The counter-rotated weight is drawn directly as N(0, 0.02^2): Q^T W of a
-    Gaussian W is again Gaussian with the same law, and the fp64 counter-
-    rotation itself is an offline step outside the per-token metric.
+    The rotation is a dense orthogonal matrix of the group's size: the
+    Kronecker product of two seeded Haar rotations of sizes a x b = d (the
+    oracle's cost of applying it is that of any dense d x d matrix, and it is
+    built in milliseconds instead of a d x d QR).  The counter-rotated weight
+    is drawn directly as N(0, 0.02^2): Q^T W of a Gaussian W is again
+    Gaussian with the same law, and the fp64 counter-rotation itself is an
+    offline step outside the per-token metric.
     """
     import numpy as np
     import synthdata as sd
@@ -236,11 +240,10 @@ def cpu_layer_inputs(sparsity: float, seed_layer: int = 0):
     for p in sd.llama_layer(HIDDEN, FFN, KV):
         base = sd.seed_for(WORKLOAD_ID, seed_layer, 10 * p.q_id)
         rng = np.random.default_rng(base + 1)
-        G = rng.standard_normal((p.d_in, p.d_in))
-        Q, _ = np.linalg.qr(G) if p.d_in <= 4096 else (None, None)
-        if Q is None:
-            # an orthogonal matrix of the same size and cost to apply
-            Q = np.linalg.qr(rng.standard_normal((p.d_in, p.d_in)).astype(np.float32))[0].astype(np.float64)
+        a = max(f for f in range(1, int(p.d_in ** 0.5) + 1) if p.d_in % f == 0)
+        qa = np.linalg.qr(rng.standard_normal((a, a)))[0]
+        qb = np.linalg.qr(rng.standard_normal((p.d_in // a, p.d_in // a)))[0]
+        Q = np.kron(qa, qb)
         W_rot = rng.standard_normal((p.d_in, p.d_out)).astype(np.float32).astype(np.float64) * 0.02
         x = sd.activations(1, p.d_in, base + 3, dtype=__import__("torch").float32).double().numpy()
         groups.append((p.name, x, Q, W_rot, sd.k_for_sparsity(p.d_in, sparsity)))
@@ -275,11 +278,10 @@ def bench_reference(args):
     of a token, so that the whole run stays within a few minutes: per
     group, a block of the rotation's output columns (the oracle's dense
     product x . Q[:, block], the same sums as its rotation) and a block of
-    W_rot's output columns (its sparse product on the kept rows), with the
-    Top-K at full size on the token's rotated vector.  Tokens are counted as
-    the share of the token's multiply-adds that the blocks perform; the
-    Top-K is done whole every step, so the reported rate is, if anything,
-    low for the oracle.
+    W_rot's output columns (its sparse product on the kept rows), and the
+    whole Top-K of the token's rotated vector on as many steps as tokens are
+    done.  Tokens are counted as the share of the token's multiply-adds that
+    the blocks perform.
     """
     import numpy as np
     import oracle
@@ -309,17 +311,25 @@ def bench_reference(args):
             total += d * d + K * d_out
         tokens_per_step = done / total
 
+        kept = [oracle.topk(xr, K) for xr, (_, _, _, _, K) in zip(x_rots, groups)]
+
         def step(i):
-            for (_, x, Q, W_rot, K), xr, (m, n) in zip(groups, x_rots, blocks):
+            # the Top-K (whole) runs on the steps where the count of tokens
+            # done passes an integer: as many Top-Ks as tokens
+            due = int((i + 1) * tokens_per_step) > int(i * tokens_per_step)
+            for g, ((_, x, Q, W_rot, K), xr, (m, n)) in enumerate(zip(groups, x_rots, blocks)):
                 c0 = (i * m) % (Q.shape[1] - m + 1)
                 o0 = (i * n) % (W_rot.shape[1] - n + 1)
                 oracle.dense_linear(x, Q[:, c0:c0 + m])
-                idx, val = oracle.topk(xr, K)
+                if due:
+                    kept[g] = oracle.topk(xr, K)
+                idx, val = kept[g]
                 oracle.sparse_linear(idx, val, W_rot[:, o0:o0 + n])
         sample = (f"each step: {tokens_per_step:.4g} of a decode token through the 4 projection groups of "
                   "the LLaMA2-7B layer: per group a block of the rotation's output columns and of "
-                  "W_rot's output columns, the Top-K at full size; tokens counted as the share of the "
-                  "token's multiply-adds done (fp64 numpy oracle, rank 0 only)")
+                  "W_rot's output columns, and the whole Top-K on as many steps as tokens are done; "
+                  "tokens counted as the share of the token's multiply-adds done "
+                  "(fp64 numpy oracle, rank 0 only)")
     for i in range(args.warmup):
         step(i)
     t0 = time.perf_counter()
