@@ -141,3 +141,48 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.larosa_prepare_weights(FAKE, P(0x20000), P(0x20000), 64, 64, BF16, None) == 1
     # status check needs a status word
     assert lib.larosa_check(None, None, None) == 1
+
+
+def _prototypes():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//.*", "", text)
+    out = {}
+    for ret, name, args in re.findall(r"([A-Za-z_][\w \*]*?)\b(larosa_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text,
+                                      flags=re.S):
+        params = [a.strip() for a in args.replace("\n", " ").split(",")] if args.strip() not in ("", "void") else []
+        out[name] = (ret.strip(), params)
+    return out
+
+
+def _kind_of_c(decl: str) -> str:
+    """'ptr', 'int', 'size', 'float' or 'str' for one C parameter or return type."""
+    if decl.startswith("const char") and "*" in decl:
+        return "str"
+    if "*" in decl or decl.startswith("larosa_stream_t"):
+        return "ptr"
+    t = decl.split()[0] if not decl.startswith("const ") else decl.split()[1]
+    return {"int": "int", "size_t": "size", "float": "float"}[t]
+
+
+def _kind_of_ctypes(t) -> str:
+    if t is ctypes.c_char_p:
+        return "str"
+    if t is ctypes.c_void_p or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "ptr"
+    return {ctypes.c_int: "int", ctypes.c_size_t: "size", ctypes.c_float: "float"}[t]
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every entry point the binding calls has the header's arity and
+    argument kinds (pointer, int, size_t, float), so the marshalling cannot
+    drift from the C ABI unnoticed."""
+    from activation_sparsity_b200 import larosa as binding
+    protos = _prototypes()
+    for name, (args, ret) in binding._SIGNATURES.items():
+        assert name in protos, name
+        c_ret, c_params = protos[name]
+        assert [_kind_of_c(p) for p in c_params] == [_kind_of_ctypes(a) for a in args], name
+        assert _kind_of_c(c_ret) == _kind_of_ctypes(ret), name
+    # and the binding covers every declared entry point
+    assert set(protos) == set(binding._SIGNATURES)
