@@ -20,7 +20,8 @@ _EXPORTS = (
     "larosa_sparse_linear_noalloc", "larosa_topk", "larosa_version", "larosa_workspace_bytes",
     "larosa_workspace_layout", "larosa_workspace_nnz_offset", "larosa_threshold",
     "larosa_rotate_threshold_linear", "larosa_fold_rotation",
-    "larosa_sparse_lowrank_linear", "larosa_lowrank_workspace_bytes", "LAROSA_F32", "LAROSA_BF16", "LAROSA_MAX_D", "LAROSA_MAX_M",
+    "larosa_sparse_lowrank_linear", "larosa_lowrank_workspace_bytes", "larosa_sparse_linear_noalloc_bytes",
+    "larosa_workspace_sync_offset", "larosa_set_wait_limit_ns", "LAROSA_NOALLOC_SCRATCH_BYTES", "LAROSA_F32", "LAROSA_BF16", "LAROSA_MAX_D", "LAROSA_MAX_M",
     "LIB_PATH",
 )
 __all__ = list(_EXPORTS)

@@ -21,6 +21,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -338,6 +339,10 @@ namespace larosa {
 // Lets other translation units of the library report a message through
 // larosa_last_error_string().
 void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
+std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 }  // namespace larosa
 
 extern "C" {
@@ -389,6 +394,26 @@ int larosa_workspace_nnz_offset(int M, int d_in, int d_out, int K, size_t* nnz_o
   st = make_layout(M, d_in, d_out, K, &L);
   if (st != LAROSA_OK) return st;
   if (nnz_offset) *nnz_offset = L.nnz;
+  return LAROSA_OK;
+}
+
+int larosa_workspace_sync_offset(int M, int d_in, int d_out, int K, size_t* sync_offset) {
+  int st = check_sizes(M, d_in, d_out, K);
+  if (st != LAROSA_OK) return st;
+  if (M != 1) return LAROSA_ERR_SHAPE;
+  Layout L;
+  st = make_layout(M, d_in, d_out, K, &L);
+  if (st != LAROSA_OK) return st;
+  if (sync_offset) *sync_offset = L.fused_sync;
+  return LAROSA_OK;
+}
+
+int larosa_set_wait_limit_ns(uint64_t limit_ns, uint64_t* previous) {
+  if (limit_ns != 0 && (limit_ns < LAROSA_MIN_WAIT_LIMIT_NS || limit_ns > LAROSA_MAX_WAIT_LIMIT_NS))
+    return LAROSA_ERR_INVALID_ARG;
+  const unsigned long long v = limit_ns == 0 ? larosa::kDefaultWaitLimitNs : limit_ns;
+  const unsigned long long old = larosa::g_wait_limit_ns.exchange(v);
+  if (previous) *previous = old;
   return LAROSA_OK;
 }
 

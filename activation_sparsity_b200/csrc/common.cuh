@@ -12,9 +12,14 @@
 
 namespace larosa {
 
-// Every wait inside a kernel gives up after this many nanoseconds of
-// %globaltimer, reports LAROSA_DEV_TIMEOUT and lets the kernel exit.
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// Every wait inside a kernel gives up after a limit of %globaltimer
+// nanoseconds, reports LAROSA_DEV_TIMEOUT and lets the kernel exit.  The
+// limit is read on the host at each launch (larosa_set_wait_limit_ns) and
+// passed in the kernel's parameters; this is its default.
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
+
+// The wait limit for launches enqueued now (api.cu).
+unsigned long long wait_limit_ns();
 
 __device__ __forceinline__ unsigned long long global_timer_ns() {
   unsigned long long t;
@@ -101,17 +106,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for phase `parity` of `bar` to complete.  Returns false (without
-// reporting) if it did not within kWaitLimitNs, or as soon as *abort becomes
+// reporting) if it did not within limit_ns, or as soon as *abort becomes
 // nonzero.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort) {
+                                                  volatile int* abort, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+      if (global_timer_ns() - t0 > limit_ns) return false;
     }
   }
 }

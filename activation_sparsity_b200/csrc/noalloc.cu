@@ -6,10 +6,15 @@
 // which cudaMalloc and cudaFree are forbidden because they may synchronise
 // the device.  For them larosa_sparse_linear_noalloc computes exactly what
 // larosa_sparse_linear computes, with the same kernels and launch geometry.
-// One token needs no scratch at all (the cluster gather adds its partial sums
-// in distributed shared memory); several tokens keep their split-K partial
-// sums, reduction tickets and shared-row bookkeeping in one file-scope device
-// array of fixed size instead of a caller workspace.
+// One token needs no scratch when the cluster gather fits the GPU (its
+// partial sums meet in distributed shared memory; on B200 this holds for
+// every size the library accepts), and otherwise falls back to the
+// row-streaming GEMV, whose split-K partials use the array below.  Several
+// tokens keep their split-K partial sums, reduction tickets and shared-row
+// bookkeeping in one file-scope device array of fixed size instead of a
+// caller workspace.  larosa_sparse_linear_noalloc_bytes tells a caller,
+// without allocating or launching anything, how much of the array a size
+// needs, so that it can check a size before relying on it.
 //
 // That array exists once per GPU that loads this library and stays resident
 // until the process exits.  Every call on a device uses the same array, so
@@ -67,7 +72,58 @@ int fail_cuda(cudaError_t e, const char* where) {
   return LAROSA_ERR_CUDA;
 }
 
+// Where each piece of the multi-token (or fallback) scratch lies.
+struct ScratchLayout {
+  size_t off_bitmap = 0, zero_bytes = 0, off_partials = 0, off_coef = 0, off_rows = 0, off_count = 0;
+  size_t total = 0;  // 0: no scratch (the one-token cluster gather)
+};
+
+bool valid_sizes(int M, int d_in, int d_out, int K) {
+  return M >= 1 && M <= LAROSA_MAX_M && d_in >= 1 && d_in <= LAROSA_MAX_D && d_out >= 1 &&
+         d_out <= kMaxDout && K >= 0 && K <= d_in;
+}
+
+// Plans the call on the current device: *sp (one token) and *pl (otherwise)
+// and the scratch layout.
+cudaError_t plan_noalloc(larosa::Elem w, int M, int d_in, int d_out, int K, larosa::StreamPlan* sp,
+                         larosa::GemvPlan* pl, ScratchLayout* S) {
+  *S = ScratchLayout{};
+  if (M == 1) {
+    cudaError_t e = larosa::plan_gather(w, d_out, K, sp);
+    if (e != cudaSuccess) return e;
+    if (sp->ok) return cudaSuccess;
+  }
+  const int n_max = M == 1 ? K : (int)std::min<long long>(d_in, (long long)M * K);
+  cudaError_t e = larosa::plan_gemv(w, larosa::Elem::F32, M, d_out, n_max, pl);
+  if (e != cudaSuccess) return e;
+  // [tickets][bitmap][partials][coef][rows][count]
+  const size_t bitmap_words = M > 1 ? (size_t)(d_in + 31) / 32 : 0;
+  S->off_bitmap = up256(pl->ticket_words * 4);
+  S->zero_bytes = S->off_bitmap + bitmap_words * 4;  // cleared every call
+  S->off_partials = up256(S->zero_bytes);
+  S->off_coef = up256(S->off_partials + pl->partial_floats * 4);
+  S->off_rows = up256(S->off_coef + (M > 1 ? (size_t)M * d_in * 4 : 0));
+  S->off_count = up256(S->off_rows + (M > 1 ? (size_t)d_in * 4 : 0));
+  S->total = S->off_count + 4;
+  return cudaSuccess;
+}
+
 }  // namespace
+
+static_assert(kScratchBytes == LAROSA_NOALLOC_SCRATCH_BYTES, "the header states the scratch size");
+
+extern "C" size_t larosa_sparse_linear_noalloc_bytes(int M, int d_in, int d_out, int K, int dtype) {
+  if ((dtype != LAROSA_BF16 && dtype != LAROSA_F32) || !valid_sizes(M, d_in, d_out, K)) return 0;
+  larosa::StreamPlan sp;
+  larosa::GemvPlan pl;
+  ScratchLayout S;
+  const larosa::Elem w = dtype == LAROSA_BF16 ? larosa::Elem::BF16 : larosa::Elem::F32;
+  if (plan_noalloc(w, M, d_in, d_out, K, &sp, &pl, &S) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return S.total;
+}
 
 extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val, int M, int K,
                                             const void* W_rot, int d_in, int d_out, float* y,
@@ -85,40 +141,30 @@ extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val
 
   const larosa::Elem w = dtype == LAROSA_BF16 ? larosa::Elem::BF16 : larosa::Elem::F32;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (M == 1) {
+  larosa::StreamPlan sp;
+  larosa::GemvPlan pl;
+  ScratchLayout S;
+  cudaError_t e = plan_noalloc(w, M, d_in, d_out, K, &sp, &pl, &S);
+  if (e != cudaSuccess) return fail_cuda(e, "plan");
+  if (M == 1 && sp.ok) {
     // one token: the cluster gather keeps its partial sums in distributed
     // shared memory and needs no scratch at all
-    larosa::StreamPlan sp;
-    cudaError_t e = larosa::plan_gather(w, d_out, K, &sp);
-    if (e != cudaSuccess) return fail_cuda(e, "plan");
-    if (sp.ok) {
-      larosa::GatherArgs a;
-      a.W = W_rot;
-      a.d_out = d_out;
-      a.row_bound = d_in;
-      a.n = K;
-      a.coef = val;
-      a.rows = idx;
-      a.y = y;
-      a.dev_status = dev_status;
-      e = larosa::launch_gather(w, a, sp, s);
-      return e == cudaSuccess ? LAROSA_OK : fail_cuda(e, "sparse linear kernel");
-    }
+    larosa::GatherArgs a;
+    a.W = W_rot;
+    a.d_out = d_out;
+    a.row_bound = d_in;
+    a.n = K;
+    a.coef = val;
+    a.rows = idx;
+    a.y = y;
+    a.dev_status = dev_status;
+    e = larosa::launch_gather(w, a, sp, s);
+    return e == cudaSuccess ? LAROSA_OK : fail_cuda(e, "sparse linear kernel");
   }
   const int n_max = M == 1 ? K : (int)std::min<long long>(d_in, (long long)M * K);
-  larosa::GemvPlan pl;
-  cudaError_t e = larosa::plan_gemv(w, larosa::Elem::F32, M, d_out, n_max, &pl);
-  if (e != cudaSuccess) return fail_cuda(e, "plan");
-
-  // scratch layout: [tickets][bitmap][partials][coef][rows][count]
-  const size_t bitmap_words = M > 1 ? (size_t)(d_in + 31) / 32 : 0;
-  const size_t off_bitmap = up256(pl.ticket_words * 4);
-  const size_t zero_bytes = off_bitmap + bitmap_words * 4;  // cleared every call
-  const size_t off_partials = up256(zero_bytes);
-  const size_t off_coef = up256(off_partials + pl.partial_floats * 4);
-  const size_t off_rows = up256(off_coef + (M > 1 ? (size_t)M * d_in * 4 : 0));
-  const size_t off_count = up256(off_rows + (M > 1 ? (size_t)d_in * 4 : 0));
-  const size_t total = off_count + 4;
+  const size_t off_bitmap = S.off_bitmap, zero_bytes = S.zero_bytes, off_partials = S.off_partials;
+  const size_t off_coef = S.off_coef, off_rows = S.off_rows, off_count = S.off_count;
+  const size_t total = S.total;
   if (total > kScratchBytes) {
     char buf[200];
     snprintf(buf, sizeof(buf),

@@ -660,7 +660,7 @@ __global__ void __launch_bounds__(kT, 2) rotsel_kernel(const RSParams p) {
 //      partial sums.
 //
 // Kept = the K largest |x_rot|, ties to the lower index: key > T, or
-// key == T and index <= I.  Every wait is bounded (kWaitLimitNs) and reports
+// key == T and index <= I.  Every wait is bounded (FParams::wait_ns) and reports
 // LAROSA_DEV_TIMEOUT; the cooperative launch guarantees that every CTA is
 // resident, so no CTA waits on one that cannot run.
 //
@@ -697,6 +697,7 @@ struct FParams {
   int thresh;         // 1: keep |x_rot| >= t (key >= t_key) instead of the Top-K
   uint32_t t_key;
   int32_t* nnz;       // threshold mode: the kept count (for callers)
+  unsigned long long wait_ns;  // limit of every wait
 };
 
 struct FLayout {
@@ -748,25 +749,20 @@ __device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Thread 0 waits until *ticket >= target; false after kWaitLimitNs.
-__device__ __forceinline__ bool wait_ticket(const unsigned* ticket, unsigned target) {
-  if (ld_acquire_gpu(ticket) >= target) return true;
+// Thread 0 waits until *word == value; false after limit_ns.  An arrival
+// counter is waited on with its exact final count: it only grows during a
+// call and is cleared only after the call has completed, so every waiter
+// sees that value, and a counter left over from a call that gave up (it
+// starts above zero) can never reach it, so such a call times out instead
+// of reading a half-built selection.
+__device__ __forceinline__ bool wait_word(const unsigned* word, unsigned value,
+                                          unsigned long long limit_ns) {
+  if (ld_acquire_gpu(word) == value) return true;
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     __nanosleep(64);
-    if (ld_acquire_gpu(ticket) >= target) return true;
-    if ((it & 31u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
-  }
-}
-
-// Thread 0 waits until *flag == value; false after kWaitLimitNs.
-__device__ __forceinline__ bool wait_flag(const unsigned* flag, unsigned value) {
-  if (ld_acquire_gpu(flag) == value) return true;
-  const unsigned long long t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(64);
-    if (ld_acquire_gpu(flag) == value) return true;
-    if ((it & 31u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (ld_acquire_gpu(word) == value) return true;
+    if ((it & 31u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -1337,7 +1333,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
       cand_idx[j] = 0xffffffffu;
     }
     if (tid == 0) {
-      const bool ok = wait_ticket(ticket, target);
+      const bool ok = wait_word(ticket, target, p.wait_ns);
       if (!ok) report(p.dev_status, LAROSA_DEV_TIMEOUT);
       s_word[0] = ok;
       s_word[1] = 0u;  // boundary candidates listed
@@ -1432,7 +1428,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   // every CTA's x_rot is written and counted: load this range while the
   // selector works
   if (tid == 0) {
-    const bool ok = wait_ticket(ticket, target);
+    const bool ok = wait_word(ticket, target, p.wait_ns);
     if (!ok) report(p.dev_status, LAROSA_DEV_TIMEOUT);
     s_word[0] = ok;
   }
@@ -1487,7 +1483,7 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   if (tid == 0) {
     bool got = false;
     if (mode == 1u) {
-      got = wait_flag(p.sync + 3, gen);
+      got = wait_word(p.sync + 3, gen, p.wait_ns);
       if (!got) report(p.dev_status, LAROSA_DEV_TIMEOUT);
     }
     s_word[4] = got ? __ldcg(p.sync + 6) : 0u;  // T
@@ -1926,6 +1922,7 @@ cudaError_t launch_fused(Elem w_elem, const FusedArgs& a, const StreamPlan& pl,
   p.thresh = a.threshold;
   p.t_key = a.t_key;
   p.nnz = a.nnz;
+  p.wait_ns = wait_limit_ns();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.n_tiles * pl.cluster + 1, 1, 1);
   cfg.blockDim = dim3(kT, 1, 1);

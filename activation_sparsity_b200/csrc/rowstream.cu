@@ -72,6 +72,7 @@ struct Params {
   int pitch;  // bytes between two rows of a stage
   int max_rpc;
   int* dev_status;
+  unsigned long long wait_ns;  // limit of every mbarrier wait
 };
 
 template <int MT, int CPT>
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_ke
       const int s = it % kStages;
       if (it >= kStages) {
         int ok = 1;
-        if (lane == 0) ok = mbar_wait_bounded(&empty[s], ((it / kStages) - 1) & 1, abort_flag);
+        if (lane == 0) ok = mbar_wait_bounded(&empty[s], ((it / kStages) - 1) & 1, abort_flag, p.wait_ns);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) {
           if (lane == 0) *abort_flag = 1;
@@ -227,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_ke
       const int s = it % kStages;
       // every lane polls the barrier (acquiring the copied bytes); the warp
       // leaves together if any lane gave up
-      const bool ok = mbar_wait_bounded(&full[s], (it / kStages) & 1, abort_flag);
+      const bool ok = mbar_wait_bounded(&full[s], (it / kStages) & 1, abort_flag, p.wait_ns);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) *abort_flag = 1;
         break;
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, (MT <= 2 ? 2 : 1)) rowstream_gemv_ke
     // CTA's shared memory is released, then leave without writing outputs.
     if (warp == kConsumerWarps && lane == 0) {
       for (int it = max(0, issued - kStages); it < issued; ++it)
-        mbar_wait_bounded(&full[it % kStages], (it / kStages) & 1, nullptr);
+        mbar_wait_bounded(&full[it % kStages], (it / kStages) & 1, nullptr, p.wait_ns);
       report(p.dev_status, LAROSA_DEV_TIMEOUT);
     }
     __syncthreads();
@@ -594,6 +595,7 @@ cudaError_t launch_gemv(const GemvArgs& a, const GemvPlan& pl, cudaStream_t stre
   p.pitch = pl.pitch;
   p.max_rpc = pl.max_rows_per_cta;
   p.dev_status = a.dev_status;
+  p.wait_ns = wait_limit_ns();
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.splits, pl.n_col_tiles, 1);

@@ -51,6 +51,9 @@ _SIGNATURES = {
                                       _vp], _i),
     "larosa_lowrank_workspace_bytes": ([_i, _i, _i, _i, _i], _sz),
     "larosa_sparse_linear_noalloc": ([_vp, _vp, _i, _i, _vp, _i, _i, _vp, _i, _vp, _vp], _i),
+    "larosa_sparse_linear_noalloc_bytes": ([_i, _i, _i, _i, _i], _sz),
+    "larosa_workspace_sync_offset": ([_i, _i, _i, _i, _c.POINTER(_sz)], _i),
+    "larosa_set_wait_limit_ns": ([_c.c_uint64, _c.POINTER(_c.c_uint64)], _i),
     "larosa_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "larosa_workspace_layout": ([_i, _i, _i, _i, _c.POINTER(_sz), _c.POINTER(_sz), _c.POINTER(_sz)], _i),
     "larosa_workspace_nnz_offset": ([_i, _i, _i, _i, _c.POINTER(_sz)], _i),
@@ -72,6 +75,7 @@ LAROSA_DEV_TIMEOUT = 0x2
 LAROSA_DEV_INDEX = 0x4
 LAROSA_MAX_M = 16
 LAROSA_MAX_D = 32768
+LAROSA_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 
 class LarosaError(RuntimeError):
@@ -210,6 +214,27 @@ def larosa_workspace_nnz_offset(M: int, d_in: int, d_out: int, K: int) -> int:
     _check(_lib.larosa_workspace_nnz_offset(M, d_in, d_out, K, ctypes.byref(a)),
            "larosa_workspace_nnz_offset")
     return a.value
+
+
+def larosa_workspace_sync_offset(M: int, d_in: int, d_out: int, K: int) -> int:
+    a = ctypes.c_size_t()
+    _check(_lib.larosa_workspace_sync_offset(M, d_in, d_out, K, ctypes.byref(a)),
+           "larosa_workspace_sync_offset")
+    return a.value
+
+
+def larosa_set_wait_limit_ns(limit_ns: int) -> int:
+    """Sets the in-kernel wait limit for later launches (0: the default);
+    returns the previous limit."""
+    prev = ctypes.c_uint64(0)
+    _check(_lib.larosa_set_wait_limit_ns(int(limit_ns), ctypes.byref(prev)), "larosa_set_wait_limit_ns")
+    return prev.value
+
+
+def larosa_sparse_linear_noalloc_bytes(M: int, d_in: int, d_out: int, K: int,
+                                       dtype: torch.dtype = torch.bfloat16) -> int:
+    code = LAROSA_BF16 if dtype == torch.bfloat16 else LAROSA_F32
+    return int(_lib.larosa_sparse_linear_noalloc_bytes(M, d_in, d_out, K, code))
 
 
 def larosa_prepare_weights(Qt: torch.Tensor, W: torch.Tensor, W_rot: torch.Tensor | None = None

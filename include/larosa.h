@@ -40,8 +40,9 @@
  *     bits in a caller-provided `int* dev_status` word (see LAROSA_DEV_*);
  *     read it with larosa_check().  dev_status may be NULL, in which case
  *     those conditions are not reported.  Kernels never trap or spin without
- *     bound: every wait inside a kernel gives up after about two seconds,
- *     sets LAROSA_DEV_TIMEOUT and exits.
+ *     bound: every wait inside a kernel gives up after a time limit (two
+ *     seconds unless changed with larosa_set_wait_limit_ns), sets
+ *     LAROSA_DEV_TIMEOUT and exits.
  *   - Workspace: the sparse linear and the fused call use caller-provided
  *     scratch `ws`
  *     of `ws_bytes` bytes, at least larosa_workspace_bytes(...).  It must be
@@ -318,12 +319,15 @@ int larosa_dense_linear(const void *x, const void *Wt, int M, int d_in,
  * variant of step 3, computing the same y with the same kernels.
  *
  * Arguments as for larosa_sparse_linear, minus ws/ws_bytes.  One token
- * needs no scratch (its partial sums stay in distributed shared memory);
- * several tokens keep their split-K partials and row bookkeeping in a 2 MiB
- * file-scope device array that every GPU loading the library holds until
- * the process exits.  Sizes whose scratch would
- * exceed it (in practice only large multi-token batches, e.g. M = 16 with
- * d_in = 32768) return LAROSA_ERR_WORKSPACE with the byte counts in
+ * needs no scratch when the cluster gather fits the GPU (its partial sums
+ * stay in distributed shared memory; on B200 that holds for every accepted
+ * size); otherwise, and for several tokens, the split-K partials and row
+ * bookkeeping live in a file-scope device array of
+ * LAROSA_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds
+ * until the process exits.  larosa_sparse_linear_noalloc_bytes() gives the
+ * scratch a size needs.  Sizes whose scratch would exceed the array (in
+ * practice only large multi-token batches, e.g. M = 16 with d_in = 32768)
+ * return LAROSA_ERR_WORKSPACE with the byte counts in
  * larosa_last_error_string().  The call allocates nothing; it clears the
  * words that must start at zero with cudaMemsetAsync on `stream`.  All calls
  * on one device share the array, so calls that may overlap on that GPU race:
@@ -335,6 +339,19 @@ int larosa_sparse_linear_noalloc(const int32_t *idx, const float *val, int M,
                                  int K, const void *W_rot, int d_in, int d_out,
                                  float *y, int dtype, int *dev_status,
                                  larosa_stream_t stream);
+
+/* Size of the file-scope scratch array behind larosa_sparse_linear_noalloc. */
+#define LAROSA_NOALLOC_SCRATCH_BYTES (2u << 20)
+
+/*
+ * Bytes of that array larosa_sparse_linear_noalloc would use for these sizes
+ * on the current device (0: none, the one-token cluster gather).  A result
+ * above LAROSA_NOALLOC_SCRATCH_BYTES means the call would be refused with
+ * LAROSA_ERR_WORKSPACE.  Allocates and launches nothing (host-side device
+ * queries only).  Returns 0 for out-of-range sizes or an unknown dtype too.
+ */
+size_t larosa_sparse_linear_noalloc_bytes(int M, int d_in, int d_out, int K,
+                                          int dtype);
 
 /*
  * Workspace bytes sufficient for every entry point above called with these
@@ -359,6 +376,36 @@ int larosa_workspace_layout(int M, int d_in, int d_out, int K,
  */
 int larosa_workspace_nnz_offset(int M, int d_in, int d_out, int K,
                                 size_t *nnz_offset);
+
+/*
+ * Byte offset inside the workspace of the one-token fused call's
+ * synchronisation block (M = 1 only; LAROSA_ERR_SHAPE otherwise).  Its
+ * 32-bit words: [0] and [1] count the arrivals of even and odd calls, [3]
+ * is the number of the last call whose selection was published, [6] and [7]
+ * the K-th entry it published; then the per-tile completion counters and
+ * the magnitude histograms of the two call parities.  A caller never needs
+ * to touch it (it is zero between calls); it is exposed for diagnosis and
+ * for tests of the bounded waits: a call whose arrival counter does not
+ * start at zero can never see its exact count and gives up after the wait
+ * limit with LAROSA_DEV_TIMEOUT.
+ */
+int larosa_workspace_sync_offset(int M, int d_in, int d_out, int K,
+                                 size_t *sync_offset);
+
+/* Range accepted by larosa_set_wait_limit_ns (besides 0). */
+#define LAROSA_MIN_WAIT_LIMIT_NS 1000ull
+#define LAROSA_MAX_WAIT_LIMIT_NS 60000000000ull
+
+/*
+ * Sets the time after which every wait inside a kernel gives up (reporting
+ * LAROSA_DEV_TIMEOUT), for launches enqueued after this call; work already
+ * enqueued or captured in a CUDA graph keeps the limit it was launched
+ * with.  limit_ns = 0 restores the default (2 s); otherwise it must lie in
+ * [LAROSA_MIN_WAIT_LIMIT_NS, LAROSA_MAX_WAIT_LIMIT_NS], else
+ * LAROSA_ERR_INVALID_ARG and nothing changes.  Process-wide; `previous`
+ * (host, may be NULL) receives the limit in force before the call.
+ */
+int larosa_set_wait_limit_ns(uint64_t limit_ns, uint64_t *previous);
 
 /*
  * Waits for `stream`, reads *dev_status (device pointer) and returns

@@ -162,7 +162,9 @@ def _kind_of_c(decl: str) -> str:
     if "*" in decl or decl.startswith("larosa_stream_t"):
         return "ptr"
     t = decl.split()[0] if not decl.startswith("const ") else decl.split()[1]
-    return {"int": "int", "size_t": "size", "float": "float"}[t]
+    # uint64_t and size_t are the same 64-bit unsigned integer on this ABI
+    # (ctypes.c_uint64 is ctypes.c_size_t)
+    return {"int": "int", "size_t": "size", "uint64_t": "size", "float": "float"}[t]
 
 
 def _kind_of_ctypes(t) -> str:

@@ -303,6 +303,9 @@ def test_fused(L, dtype, M, d_in, d_out, sparsity):
     assert np.all(np.abs(x_rot - x_rot_ref) <= gamma + 1e-30)
     check_selection(x_rot_ref, gamma, idx, K)
     for m in range(M):
+        # exactly the oracle's Top-K of the path's own fp32 x_rot
+        want, _ = oracle.topk(x_rot[m], K)
+        assert np.array_equal(idx[m], want)
         assert np.array_equal(val[m], x_rot[m, idx[m]].astype(np.float32))
     W_rot_ref = oracle.prepare_weights(qq, f64(W))
     if dtype == torch.bfloat16:
@@ -392,4 +395,6 @@ def test_rotate_topk(L, dtype, d, sparsity):
         tied_out = np.nonzero(~kept & (mags == thr))[0]
         tied_in = np.nonzero(kept & (mags == thr))[0]
         assert len(tied_out) == 0 or tied_in.max() < tied_out.min()
+    want, _ = oracle.topk(got[0], K)
+    assert np.array_equal(idx[0], want)
     assert np.array_equal(f64(val)[0], got[0, idx[0]])

@@ -32,6 +32,10 @@ def test_llama2_7b_layer_group(layer, gi):
     gamma = (g.d_in + 2) * U * (np.abs(xq) @ np.abs(qq))
     assert np.all(np.abs(x_rot - x_rot_ref) <= gamma + 1e-30)
     check_selection(x_rot_ref, gamma, idx, g.K)
+    # the kept set is exactly the oracle's Top-K of the kernel's own fp32 x_rot
+    # (checked against the exact rotation just above), ties to the lower index
+    want, _ = oracle.topk(x_rot[0], g.K)
+    assert np.array_equal(idx[0], want)
     assert np.array_equal(val[0], x_rot[0, idx[0]].astype(np.float32))
     rng = np.random.default_rng(1000 + gi)
     cols = np.sort(rng.choice(g.d_out, size=96, replace=False))

@@ -1,10 +1,16 @@
-"""larosa_sparse_linear_noalloc against larosa_sparse_linear, through the C ABI.
+"""larosa_sparse_linear_noalloc through the C ABI, against the fp64 oracle and
+against larosa_sparse_linear.
 
 The no-allocation variant serves callers that cannot give the library a
 workspace (an operator slot that passes only inputs and outputs, or a loop in
-which cudaMalloc/cudaFree are not allowed).  It must return what the
-workspace entry point returns, on consecutive calls that reuse its fixed
-device scratch, and refuse sizes whose scratch would not fit.
+which cudaMalloc/cudaFree are not allowed).  It runs the same kernels with the
+same launch geometry as the workspace entry point, so its output must equal
+that entry point's bit for bit, and both must lie within the fp32 summation
+bound of the oracle's exact sum.  Two consecutive calls use different index
+sets, so a value left behind in the shared static scratch by the first call
+(coefficient rows, the row bitmap, the union list, split-K tickets) would
+change the second call's result.  Sizes whose scratch would not fit are
+refused, and larosa_sparse_linear_noalloc_bytes says so in advance.
 
 This file is collected last on purpose.  It must pass both alone in a fresh
 process and after the rest of the suite.
@@ -15,11 +21,14 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synthdata as sd
 
 pytestmark = pytest.mark.gpu
 
 Y_TOL = 2e-3  # the tolerance the parity tests use for y
+U = 2.0 ** -24  # unit roundoff of fp32
+SCRATCH = 2 << 20  # LAROSA_NOALLOC_SCRATCH_BYTES
 
 
 @pytest.fixture(scope="module")
@@ -27,7 +36,9 @@ def lib():
     from activation_sparsity_b200 import build_lib
     build_lib.build()
     from activation_sparsity_b200 import larosa
-    return larosa.raw_library()
+    lib = larosa.raw_library()
+    lib.larosa_last_error_string.restype = ctypes.c_char_p
+    return lib
 
 
 def _p(t):
@@ -42,43 +53,67 @@ def _call_noalloc(lib, idx, val, W, y, st):
                                             1 if W.dtype == torch.bfloat16 else 0, _p(st), stream)
 
 
-def _rel_inf(got, ref):
-    return float((got - ref).abs().max() / ref.abs().max())
+def _check_against_oracle(y, idx, val, W):
+    got = y.double().cpu().numpy()
+    Wd = W.double().cpu().numpy()
+    i64 = idx.cpu().numpy().astype(np.int64)
+    v64 = val.double().cpu().numpy()
+    M, K = i64.shape
+    for m in range(M):
+        ref = oracle.sparse_linear(i64[m], v64[m], Wd)
+        bound = (K + 2) * U * (np.abs(v64[m]) @ np.abs(Wd[i64[m]]))
+        assert np.all(np.abs(got[m] - ref) <= bound + 1e-30), m
+        assert np.max(np.abs(got[m] - ref)) <= Y_TOL * np.max(np.abs(ref)), m
 
 
 @pytest.mark.parametrize("M,d_in,d_out,K", [
     (1, 4096, 12288, 2458),   # LLaMA2-7B q|k|v at 40 % sparsity
     (1, 11008, 4096, 6605),   # LLaMA2-7B down at 40 % sparsity
     (4, 1024, 2048, 400),     # several tokens sharing streamed rows
+    (8, 2048, 1024, 1229),    # eight tokens: the scratch holds coefficient rows of all of them
 ])
-def test_noalloc_matches_workspace_entry_point_on_two_calls(lib, M, d_in, d_out, K):
+def test_noalloc_matches_oracle_and_workspace_entry_point_on_two_calls(lib, M, d_in, d_out, K):
     import activation_sparsity_b200 as L
-    idx, val = sd.index_values(M, d_in, K, 900 + M)
     W = sd.weights(d_in, d_out, 0.02, 901, torch.bfloat16, device="cuda")
-    idx, val = idx.cuda(), val.cuda()
-    ref = L.larosa_sparse_linear(idx, val, W)
-    torch.cuda.synchronize()
+    need = L.larosa_sparse_linear_noalloc_bytes(M, d_in, d_out, K)
+    assert need <= SCRATCH
+    if M == 1:
+        assert need == 0  # the one-token cluster gather uses no scratch on this GPU
     for call in range(2):
+        # a different index set on each call: few rows shared between them
+        idx, val = sd.index_values(M, d_in, K, 900 + 17 * call + M)
+        idx, val = idx.cuda(), val.cuda()
+        ref = L.larosa_sparse_linear(idx, val, W)
         y = torch.full((M, d_out), float("nan"), dtype=torch.float32, device="cuda")
         st = torch.zeros(1, dtype=torch.int32, device="cuda")
         rc = _call_noalloc(lib, idx, val, W, y, st)
         assert rc == 0, (call, rc)
         torch.cuda.synchronize()
         assert int(st.item()) == 0
-        assert torch.isfinite(y).all()
-        assert _rel_inf(y, ref) <= Y_TOL, call
+        # same kernels, same geometry: the same sums in the same order
+        assert torch.equal(y, ref), call
+        _check_against_oracle(y, idx, val, W)
 
 
 def test_noalloc_refuses_sizes_beyond_its_scratch(lib):
+    import activation_sparsity_b200 as L
     M, d_in, d_out, K = 16, 32768, 4096, 100   # dense per-token coefficients alone take 2 MiB
+    assert L.larosa_sparse_linear_noalloc_bytes(M, d_in, d_out, K) > SCRATCH
     idx = torch.zeros((M, K), dtype=torch.int32, device="cuda")
     val = torch.zeros((M, K), dtype=torch.float32, device="cuda")
     W = torch.zeros((d_in, d_out), dtype=torch.bfloat16, device="cuda")
     y = torch.zeros((M, d_out), dtype=torch.float32, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     assert _call_noalloc(lib, idx, val, W, y, st) == 6  # LAROSA_ERR_WORKSPACE
-    lib.larosa_last_error_string.restype = ctypes.c_char_p
     msg = lib.larosa_last_error_string().decode()
-    assert "scratch" in msg and str(2 << 20) in msg
+    assert "scratch" in msg and str(SCRATCH) in msg
     torch.cuda.synchronize()
     assert np.all(y.cpu().numpy() == 0)  # nothing was enqueued
+
+
+def test_noalloc_one_token_needs_no_scratch_at_the_largest_sizes(lib):
+    """One token never reaches the scratch-using fallback on this GPU: the
+    cluster gather plan fits every accepted size, up to d_in = K = 32768."""
+    import activation_sparsity_b200 as L
+    for d_in, d_out, K in [(32768, 8192, 32768), (32768, 65536, 16384), (8, 8, 1), (4096, 8, 0)]:
+        assert L.larosa_sparse_linear_noalloc_bytes(1, d_in, d_out, K) == 0, (d_in, d_out, K)
