@@ -40,10 +40,17 @@ constexpr size_t kTicketWords = 2048;
 constexpr size_t kSplitKTicketWords = kTicketWords - 1;
 constexpr size_t kRotSelTicket = kTicketWords - 1;
 constexpr size_t kBitmapWords = LAROSA_MAX_D / 32;
-// Fixed header: words that must be zero before a call and are zero after it.
+// Fixed header, at the same offsets in the layout of every size, so that
+// calls of different sizes may share one workspace: words that must be zero
+// before a call and are zero after it, then the one-token fused kernel's
+// synchronisation block, whose call number and alternating counters persist
+// from one call to the next (a call of another size that laid its own
+// intermediates over them would leave the next one-token call a counter that
+// can never reach its count).
 constexpr size_t kOffTickets = 0;
 constexpr size_t kOffBitmap = kOffTickets + kTicketWords * 4;
-constexpr size_t kHeaderEnd = kOffBitmap + kBitmapWords * 4;
+constexpr size_t kOffFusedSync = (kOffBitmap + kBitmapWords * 4 + 255) / 256 * 256;
+constexpr size_t kHeaderEnd = kOffFusedSync + larosa::kFusedSyncBytes;
 
 thread_local char g_last_error[256] = "";
 
@@ -66,10 +73,11 @@ bool valid_dtype(int dtype) { return dtype == LAROSA_BF16 || dtype == LAROSA_F32
 bool row_aligned(int n, int dtype) { return (n * elem_size(dtype)) % 16 == 0; }
 
 struct Layout {
-  size_t fused_sync = 0;  // the fused kernel's synchronisation block (M = 1)
+  size_t fused_sync = 0;  // the fused kernel's synchronisation block (M = 1; in the fixed header)
   size_t x_rot = 0, idx = 0, val = 0, nnz = 0;
   size_t partials = 0;
   size_t coef = 0, urows = 0, ucount = 0;
+  size_t coef_hl = 0;  // M >= 8: the coefficients' bf16 head and tail for the tensor-core GEMV
   size_t total = 0;
   bool list_gemv = false;  // M = 1: the row-streaming GEMV over a list of up to d_in rows fits
 };
@@ -146,7 +154,7 @@ int make_layout_uncached(int M, int d_in, int d_out, int K, Layout* L) {
     off = align_up(off + bytes, 256);
     return at;
   };
-  if (M == 1) L->fused_sync = take(larosa::kFusedSyncBytes);
+  L->fused_sync = kOffFusedSync;
   L->x_rot = take((size_t)M * d_in * 4);
   L->idx = take((size_t)M * K * 4);
   L->val = take((size_t)M * K * 4);
@@ -156,6 +164,7 @@ int make_layout_uncached(int M, int d_in, int d_out, int K, Layout* L) {
     L->coef = take((size_t)M * d_in * 4);
     L->urows = take((size_t)d_in * 4);
     L->ucount = take(4);
+    if (M >= 8) L->coef_hl = take((size_t)2 * M * d_in * 2);
   }
   L->total = off;
   return LAROSA_OK;
@@ -258,6 +267,18 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
     int* ucount = reinterpret_cast<int*>(at(ws, L.ucount));
     e = larosa::launch_scatter(idx, val, M, K, d_in, coef, bitmap, dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e, "scatter kernel");
+    if (dtype == LAROSA_BF16 && L.coef_hl != 0 && larosa::umma_gemv_applies(M, d_in, d_out)) {
+      // every row is kept by some token at this many tokens: the dense
+      // product with the per-token coefficients (zero where not kept)
+      int dev = 0, sms = 0;
+      e = cudaGetDevice(&dev);
+      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return cuda_fail(e, "device query");
+      __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(at(ws, L.coef_hl));
+      e = larosa::launch_umma_gemv(W_rot, coef, hi, hi + (size_t)M * d_in, bitmap, y, M, d_in, d_out, sms,
+                                   dev_status, s);
+      return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "tensor-core sparse linear kernel");
+    }
     e = larosa::launch_union(bitmap, d_in, urows, ucount, s);
     if (e != cudaSuccess) return cuda_fail(e, "union kernel");
     a.rows = urows;

@@ -125,6 +125,23 @@ cudaError_t launch_gather(Elem w_elem, const GatherArgs& a, const StreamPlan& pl
 cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M, int n_in,
                           int n_out, cudaStream_t stream);
 
+// The same row-dot product for 8 to 16 bf16 tokens on tcgen05 (TMEM
+// accumulator, TMA-fed shared-memory operands); rot_umma_applies tells
+// whether the shapes suit it (n_in a multiple of 64).
+bool rot_umma_applies(int M, int n_in, int n_out);
+cudaError_t launch_rot_umma(const void* A, const void* x, float* y, int M, int n_in, int n_out, int sms,
+                            int* dev_status, cudaStream_t stream);
+
+// The sparse linear of 8 to 16 tokens as a dense tensor-core product over
+// every row of W (bf16) with the per-token coefficient rows coef [M x d_in]
+// (zero where a token did not keep the row): splits coef into bf16 head and
+// tail (coef_hi, coef_lo: M x d_in each) and clears the row bitmap the
+// scatter kernel set, then y = coef . W on tcgen05.
+bool umma_gemv_applies(int M, int d_in, int d_out);
+cudaError_t launch_umma_gemv(const void* W, const float* coef, __nv_bfloat16* coef_hi, __nv_bfloat16* coef_lo,
+                             unsigned* bitmap, float* y, int M, int d_in, int d_out, int sms, int* dev_status,
+                             cudaStream_t stream);
+
 // One token: x_rot = x . Q (through Qt = Q^T), then the last CTA to finish
 // writes the kept list (idx, val: the K largest |x_rot|, ties to the lower
 // index, ascending) for a list-mode gather launched right after it.

@@ -74,7 +74,9 @@ int fail_cuda(cudaError_t e, const char* where) {
 
 // Where each piece of the multi-token (or fallback) scratch lies.
 struct ScratchLayout {
+  bool tensor_core = false;  // 8-16 bf16 tokens: the dense tcgen05 product, as larosa_sparse_linear
   size_t off_bitmap = 0, zero_bytes = 0, off_partials = 0, off_coef = 0, off_rows = 0, off_count = 0;
+  size_t off_coef_hl = 0;    // tensor_core: the coefficients' bf16 head and tail
   size_t total = 0;  // 0: no scratch (the one-token cluster gather)
 };
 
@@ -92,6 +94,15 @@ cudaError_t plan_noalloc(larosa::Elem w, int M, int d_in, int d_out, int K, laro
     cudaError_t e = larosa::plan_gather(w, d_out, K, sp);
     if (e != cudaSuccess) return e;
     if (sp->ok) return cudaSuccess;
+  }
+  if (M > 1 && w == larosa::Elem::BF16 && larosa::umma_gemv_applies(M, d_in, d_out)) {
+    // [bitmap][coef][coef head and tail]
+    S->tensor_core = true;
+    S->zero_bytes = (size_t)(d_in + 31) / 32 * 4;
+    S->off_coef = up256(S->zero_bytes);
+    S->off_coef_hl = up256(S->off_coef + (size_t)M * d_in * 4);
+    S->total = S->off_coef_hl + (size_t)2 * M * d_in * 2;
+    return cudaSuccess;
   }
   const int n_max = M == 1 ? K : (int)std::min<long long>(d_in, (long long)M * K);
   cudaError_t e = larosa::plan_gemv(w, larosa::Elem::F32, M, d_out, n_max, pl);
@@ -180,6 +191,22 @@ extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val
   if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress");
   e = cudaMemsetAsync(base, 0, zero_bytes, s);
   if (e != cudaSuccess) return fail_cuda(e, "clear scratch");
+
+  if (S.tensor_core) {
+    // the row bitmap the scatter sets is cleared again by the coefficient split
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return fail_cuda(e, "device query");
+    float* coef = reinterpret_cast<float*>(base + off_coef);
+    unsigned* bitmap = reinterpret_cast<unsigned*>(base);
+    __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(base + S.off_coef_hl);
+    e = larosa::launch_scatter(idx, val, M, K, d_in, coef, bitmap, dev_status, s);
+    if (e != cudaSuccess) return fail_cuda(e, "scatter kernel");
+    e = larosa::launch_umma_gemv(W_rot, coef, hi, hi + (size_t)M * d_in, bitmap, y, M, d_in, d_out, sms,
+                                 dev_status, s);
+    return e == cudaSuccess ? LAROSA_OK : fail_cuda(e, "tensor-core sparse linear kernel");
+  }
 
   larosa::GemvArgs a;
   a.W = W_rot;

@@ -1579,6 +1579,8 @@ cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M,
   DevState* ds = nullptr;
   cudaError_t err = dev_state(&ds);
   if (err != cudaSuccess) return err;
+  if (e == Elem::BF16 && rot_umma_applies(M, n_in, n_out))
+    return launch_rot_umma(A, x, y, M, n_in, n_out, ds->sms, nullptr, stream);
   if (e == Elem::BF16 && M >= kMmaMinTokens && n_in % 32 == 0 && n_out % 8 == 0) {
     MParams p;
     p.A = A;

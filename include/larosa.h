@@ -47,10 +47,12 @@
  *     scratch `ws`
  *     of `ws_bytes` bytes, at least larosa_workspace_bytes(...).  It must be
  *     16-byte aligned and ZERO-FILLED before its first use; every call that
- *     completes leaves its counter words at zero again, so the same buffer
- *     serves the next call on the same stream without clearing.  After a
- *     device-side error, zero it again.  Calls that may run concurrently (on
- *     different streams) need distinct workspaces.
+ *     completes leaves its counter words consistent again, so the same
+ *     buffer serves the next call on the same stream without clearing, also
+ *     when that call has other sizes (the persistent words sit at the same
+ *     offsets in the layout of every size).  After a device-side error, zero
+ *     it again.  Calls that may run concurrently (on different streams) need
+ *     distinct workspaces.
  *   - Data types: `dtype` is LAROSA_BF16 (bf16 activations and weights) or
  *     LAROSA_F32 (fp32 activations and weights).  Rotated activations, kept
  *     values and outputs are always fp32; all accumulation is fp32.

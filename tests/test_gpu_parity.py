@@ -398,3 +398,31 @@ def test_rotate_topk(L, dtype, d, sparsity):
     want, _ = oracle.topk(got[0], K)
     assert np.array_equal(idx[0], want)
     assert np.array_equal(f64(val)[0], got[0, idx[0]])
+
+
+def test_one_workspace_serves_calls_of_every_size(L):
+    """The one-token fused call keeps a call number and alternating counters
+    in the workspace from call to call; calls of other sizes (several tokens,
+    the threshold layout) on the same workspace must leave them intact.  A
+    one-token call after each of them returns exactly what it returns on a
+    workspace of its own, without a device error."""
+    d_in, d_out = 1024, 2048
+    K = sd.k_for_sparsity(d_in, 40)
+    dev = torch.device("cuda")
+    Qt = sd.orthogonal(d_in, 1301).to(torch.bfloat16).t().contiguous().to(dev)
+    W_rot = L.larosa_prepare_weights(Qt, sd.weights(d_in, d_out, 0.02, 1302, torch.bfloat16, device=dev))
+    x1 = sd.activations(1, d_in, 1303, torch.bfloat16).to(dev)
+    st = status()
+    y_alone = L.larosa_rotate_topk_linear(x1, Qt, W_rot, K, ws=L.Workspace(), dev_status=st).clone()
+    ws = L.Workspace()
+    for M in (1, 4, 16):
+        ws.get(M, d_in, d_out, d_in)
+        ws.get(M, d_in, d_out, K)
+    for M in (4, 16, 2):
+        xM = sd.activations(M, d_in, 1310 + M, torch.bfloat16).to(dev)
+        L.larosa_rotate_topk_linear(xM, Qt, W_rot, K, ws=ws, dev_status=st)
+        L.larosa_rotate_threshold_linear(xM, Qt, W_rot, 0.05, ws=ws, dev_status=st)
+        for _ in range(2):  # the call number alternates the counters' slots
+            y1 = L.larosa_rotate_topk_linear(x1, Qt, W_rot, K, ws=ws, dev_status=st)
+            assert L.larosa_check(st) == 0, M
+            assert torch.equal(y1, y_alone), M
