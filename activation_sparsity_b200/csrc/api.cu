@@ -218,6 +218,13 @@ uint32_t threshold_key(float t) {
   return k;
 }
 
+// 8 to 16 bf16 tokens: the union of their kept rows is (nearly) every row,
+// so the sparse linear is the dense tcgen05 product with each token's
+// coefficient row (zero where the token did not keep the row).
+bool tensor_core_gemv(int M, int d_in, int d_out, int dtype, const Layout& L) {
+  return dtype == LAROSA_BF16 && L.coef_hl != 0 && larosa::umma_gemv_applies(M, d_in, d_out);
+}
+
 int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W_rot, int d_in,
                int d_out, float* y, int dtype, void* ws, const Layout& L, int* dev_status,
                cudaStream_t s) {
@@ -261,24 +268,21 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
     a.coef = val;
     a.coef_ld = K;
   } else {
+    if (tensor_core_gemv(M, d_in, d_out, dtype, L)) {
+      // every row is kept by some token at this many tokens: the dense
+      // product with the per-token coefficients (zero where not kept)
+      __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(at(ws, L.coef_hl));
+      e = larosa::launch_coef_rows(idx, val, M, K, d_in, hl, dev_status, s);
+      if (e != cudaSuccess) return cuda_fail(e, "coefficient rows kernel");
+      e = larosa::launch_umma_gemv(W_rot, hl, y, M, d_in, d_out, dev_status, s);
+      return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "tensor-core sparse linear kernel");
+    }
     float* coef = reinterpret_cast<float*>(at(ws, L.coef));
     unsigned* bitmap = reinterpret_cast<unsigned*>(at(ws, kOffBitmap));
     int32_t* urows = reinterpret_cast<int32_t*>(at(ws, L.urows));
     int* ucount = reinterpret_cast<int*>(at(ws, L.ucount));
     e = larosa::launch_scatter(idx, val, M, K, d_in, coef, bitmap, dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e, "scatter kernel");
-    if (dtype == LAROSA_BF16 && L.coef_hl != 0 && larosa::umma_gemv_applies(M, d_in, d_out)) {
-      // every row is kept by some token at this many tokens: the dense
-      // product with the per-token coefficients (zero where not kept)
-      int dev = 0, sms = 0;
-      e = cudaGetDevice(&dev);
-      if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-      if (e != cudaSuccess) return cuda_fail(e, "device query");
-      __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(at(ws, L.coef_hl));
-      e = larosa::launch_umma_gemv(W_rot, coef, hi, hi + (size_t)M * d_in, bitmap, y, M, d_in, d_out, sms,
-                                   dev_status, s);
-      return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "tensor-core sparse linear kernel");
-    }
     e = larosa::launch_union(bitmap, d_in, urows, ucount, s);
     if (e != cudaSuccess) return cuda_fail(e, "union kernel");
     a.rows = urows;
@@ -601,6 +605,15 @@ int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, 
   }
   st = run_rotation(x, Qt, x_rot, M, d_in, dtype, s);
   if (st != LAROSA_OK) return st;
+  if (M > 1 && tensor_core_gemv(M, d_in, d_out, dtype, L)) {
+    // the Top-K kernel also writes the tokens' coefficient rows for the
+    // tensor-core product
+    __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(at(ws, L.coef_hl));
+    cudaError_t e = larosa::launch_topk(x_rot, M, d_in, K, idx, val, dev_status, s, hl);
+    if (e != cudaSuccess) return cuda_fail(e, "topk kernel");
+    e = larosa::launch_umma_gemv(W_rot, hl, y, M, d_in, d_out, dev_status, s);
+    return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "tensor-core sparse linear kernel");
+  }
   cudaError_t e = larosa::launch_topk(x_rot, M, d_in, K, idx, val, dev_status, s);
   if (e != cudaSuccess) return cuda_fail(e, "topk kernel");
   return run_sparse(idx, val, M, K, W_rot, d_in, d_out, y, dtype, ws, L, dev_status, s);

@@ -55,9 +55,16 @@ cudaError_t plan_gemv(Elem w_elem, Elem coef_elem, int M, int d_out, int n_rows_
 // Enqueues the GEMV with programmatic dependent launch on `stream`.
 cudaError_t launch_gemv(const GemvArgs& a, const GemvPlan& plan, cudaStream_t stream);
 
-// Top-K: one 1024-thread CTA per token.
+// Top-K: one 1024-thread CTA per token.  With hl != nullptr (d a multiple of
+// 8) it also writes the tokens' dense coefficient rows as bf16 head and tail
+// for the tensor-core sparse linear: hl[m][0, d) heads, hl[M + m][0, d) tails.
 cudaError_t launch_topk(const float* x_rot, int M, int d, int K, int32_t* idx, float* val,
-                        int* dev_status, cudaStream_t stream);
+                        int* dev_status, cudaStream_t stream, __nv_bfloat16* hl = nullptr);
+
+// The same dense head/tail coefficient rows from given kept lists (idx/val
+// [M x K], indices distinct within a row): one CTA per token.
+cudaError_t launch_coef_rows(const int32_t* idx, const float* val, int M, int K, int d, __nv_bfloat16* hl,
+                             int* dev_status, cudaStream_t stream);
 
 // Threshold selection: one 1024-thread CTA per token keeps |x_rot| >= t
 // (t_key: bit pattern of t, 0 for t <= 0), writes the kept (idx, val) in
@@ -129,18 +136,16 @@ cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M,
 // accumulator, TMA-fed shared-memory operands); rot_umma_applies tells
 // whether the shapes suit it (n_in a multiple of 64).
 bool rot_umma_applies(int M, int n_in, int n_out);
-cudaError_t launch_rot_umma(const void* A, const void* x, float* y, int M, int n_in, int n_out, int sms,
+cudaError_t launch_rot_umma(const void* A, const void* x, float* y, int M, int n_in, int n_out,
                             int* dev_status, cudaStream_t stream);
 
 // The sparse linear of 8 to 16 tokens as a dense tensor-core product over
-// every row of W (bf16) with the per-token coefficient rows coef [M x d_in]
-// (zero where a token did not keep the row): splits coef into bf16 head and
-// tail (coef_hi, coef_lo: M x d_in each) and clears the row bitmap the
-// scatter kernel set, then y = coef . W on tcgen05.
+// every row of W (bf16) with the per-token coefficient rows (zero where a
+// token did not keep the row), given as bf16 head and tail hl [2 x M x d_in]
+// (launch_topk or launch_coef_rows): y = (head + tail) . W on tcgen05.
 bool umma_gemv_applies(int M, int d_in, int d_out);
-cudaError_t launch_umma_gemv(const void* W, const float* coef, __nv_bfloat16* coef_hi, __nv_bfloat16* coef_lo,
-                             unsigned* bitmap, float* y, int M, int d_in, int d_out, int sms, int* dev_status,
-                             cudaStream_t stream);
+cudaError_t launch_umma_gemv(const void* W, const __nv_bfloat16* hl, float* y, int M, int d_in, int d_out,
+                             int* dev_status, cudaStream_t stream);
 
 // One token: x_rot = x . Q (through Qt = Q^T), then the last CTA to finish
 // writes the kept list (idx, val: the K largest |x_rot|, ties to the lower

@@ -96,12 +96,10 @@ cudaError_t plan_noalloc(larosa::Elem w, int M, int d_in, int d_out, int K, laro
     if (sp->ok) return cudaSuccess;
   }
   if (M > 1 && w == larosa::Elem::BF16 && larosa::umma_gemv_applies(M, d_in, d_out)) {
-    // [bitmap][coef][coef head and tail]
+    // [coefficient heads and tails]: every word is written by each call
     S->tensor_core = true;
-    S->zero_bytes = (size_t)(d_in + 31) / 32 * 4;
-    S->off_coef = up256(S->zero_bytes);
-    S->off_coef_hl = up256(S->off_coef + (size_t)M * d_in * 4);
-    S->total = S->off_coef_hl + (size_t)2 * M * d_in * 2;
+    S->off_coef_hl = 0;
+    S->total = (size_t)2 * M * d_in * 2;
     return cudaSuccess;
   }
   const int n_max = M == 1 ? K : (int)std::min<long long>(d_in, (long long)M * K);
@@ -189,24 +187,15 @@ extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val
   unsigned char* base = nullptr;
   e = scratch_address(reinterpret_cast<void**>(&base));
   if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress");
-  e = cudaMemsetAsync(base, 0, zero_bytes, s);
-  if (e != cudaSuccess) return fail_cuda(e, "clear scratch");
-
   if (S.tensor_core) {
-    // the row bitmap the scatter sets is cleared again by the coefficient split
-    int dev = 0, sms = 0;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return fail_cuda(e, "device query");
-    float* coef = reinterpret_cast<float*>(base + off_coef);
-    unsigned* bitmap = reinterpret_cast<unsigned*>(base);
-    __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(base + S.off_coef_hl);
-    e = larosa::launch_scatter(idx, val, M, K, d_in, coef, bitmap, dev_status, s);
-    if (e != cudaSuccess) return fail_cuda(e, "scatter kernel");
-    e = larosa::launch_umma_gemv(W_rot, coef, hi, hi + (size_t)M * d_in, bitmap, y, M, d_in, d_out, sms,
-                                 dev_status, s);
+    __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(base + S.off_coef_hl);
+    e = larosa::launch_coef_rows(idx, val, M, K, d_in, hl, dev_status, s);
+    if (e != cudaSuccess) return fail_cuda(e, "coefficient rows kernel");
+    e = larosa::launch_umma_gemv(W_rot, hl, y, M, d_in, d_out, dev_status, s);
     return e == cudaSuccess ? LAROSA_OK : fail_cuda(e, "tensor-core sparse linear kernel");
   }
+  e = cudaMemsetAsync(base, 0, zero_bytes, s);
+  if (e != cudaSuccess) return fail_cuda(e, "clear scratch");
 
   larosa::GemvArgs a;
   a.W = W_rot;

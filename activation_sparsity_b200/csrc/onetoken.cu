@@ -683,7 +683,8 @@ struct FParams {
   float* val;         // [K]
   float* y;           // [d_out]
   float* partials;    // [n_tiles x C x col_tile] per-CTA partial sums of each column tile
-  unsigned* sync;     // [0, 1] arrivals, [3] K-th entry published, [6] T, [7] I; then
+  unsigned* sync;     // [0, 1] arrivals, [3] the last call's number, [4, 5] the K-th entry
+                      // with its call's tag (one 64-bit word, see pack_kth); then
                       // 2 x kFusedMaxTiles tile counters, 2 x kFusedHistBins histogram bins
   int d;
   int d_out;
@@ -747,6 +748,46 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
 
 __device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// The K-th entry as one word: T in bits 0..31, I (16 bits; -1 as 0xffff) in
+// bits 32..47 and the call's tag (its number mod 2^16) in bits 48..63, so
+// that the one acquire load that sees the publication also returns the entry.
+__device__ __forceinline__ unsigned long long pack_kth(uint32_t T, int32_t I, unsigned gen) {
+  return (unsigned long long)T | ((unsigned long long)(static_cast<uint32_t>(I) & 0xffffu) << 32) |
+         ((unsigned long long)(gen & 0xffffu) << 48);
+}
+
+// Thread 0 waits until the word at kth carries the tag of call gen and
+// returns it in *w; false after limit_ns.
+__device__ __forceinline__ bool wait_kth(const unsigned long long* kth, unsigned gen, unsigned long long* w,
+                                         unsigned long long limit_ns) {
+  const unsigned long long tag = gen & 0xffffu;
+  unsigned long long v = ld_acquire_gpu_u64(kth);
+  if ((v >> 48) == tag) {
+    *w = v;
+    return true;
+  }
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    v = ld_acquire_gpu_u64(kth);
+    if ((v >> 48) == tag) {
+      *w = v;
+      return true;
+    }
+    if ((it & 31u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
+  }
 }
 
 // Thread 0 waits until *word == value; false after limit_ns.  An arrival
@@ -1373,9 +1414,10 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
       }
     }
     if (tid == 0) {
-      p.sync[6] = e.T;
-      p.sync[7] = static_cast<uint32_t>(e.I);
-      st_release_gpu(p.sync + 3, gen);
+      // the entry and this call's tag in one release store; the call number,
+      // read only by the next call once this one has completed, follows
+      st_release_gpu_u64(reinterpret_cast<unsigned long long*>(p.sync + 4), pack_kth(e.T, e.I, gen));
+      p.sync[3] = gen;
     }
     if (nonfinite) report(p.dev_status, LAROSA_DEV_NONFINITE);
     // the kept list for callers, off the gather's path
@@ -1482,12 +1524,14 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
   // the K-th entry: the kept rows of bin B
   if (tid == 0) {
     bool got = false;
+    unsigned long long w = 0;
     if (mode == 1u) {
-      got = wait_word(p.sync + 3, gen, p.wait_ns);
+      got = wait_kth(reinterpret_cast<const unsigned long long*>(p.sync + 4), gen, &w, p.wait_ns);
       if (!got) report(p.dev_status, LAROSA_DEV_TIMEOUT);
     }
-    s_word[4] = got ? __ldcg(p.sync + 6) : 0u;  // T
-    s_word[5] = got ? __ldcg(p.sync + 7) : 0u;  // I
+    s_word[4] = got ? static_cast<uint32_t>(w) : 0u;  // T
+    s_word[5] = got ? static_cast<uint32_t>(static_cast<int32_t>(static_cast<int16_t>((w >> 32) & 0xffffu)))
+                    : 0u;  // I, sign-extended
     s_word[6] = got;
   }
   __syncthreads();
@@ -1580,7 +1624,7 @@ cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M,
   cudaError_t err = dev_state(&ds);
   if (err != cudaSuccess) return err;
   if (e == Elem::BF16 && rot_umma_applies(M, n_in, n_out))
-    return launch_rot_umma(A, x, y, M, n_in, n_out, ds->sms, nullptr, stream);
+    return launch_rot_umma(A, x, y, M, n_in, n_out, nullptr, stream);
   if (e == Elem::BF16 && M >= kMmaMinTokens && n_in % 32 == 0 && n_out % 8 == 0) {
     MParams p;
     p.A = A;

@@ -41,8 +41,10 @@ __global__ void __launch_bounds__(kPrepThreads) prepare_kernel(const T* __restri
   const int tx = tid % 16;  // 4 columns each
   const int ty = tid / 16;  // 8 rows each
 
+  // No early trigger: the kernels of the decode path may read their weights
+  // as soon as the previous kernel lets them launch, so the kernel that
+  // writes a weight lets them launch only when it ends.
   pdl_wait();
-  pdl_launch_dependents();
 
   float acc[8][4];
 #pragma unroll

@@ -23,9 +23,40 @@ constexpr int kTopkThreads = 1024;
 constexpr int kTopkCand = 2048;
 constexpr int kTopkU = 8;  // 16-byte loads in flight per thread
 
+// The coefficient c of a kept entry (0 elsewhere) as the bf16 head and tail
+// the tensor cores multiply: head = bf16(c), tail = bf16(c - head), both
+// rounded to nearest even (about 16 significant bits of c kept in all).
+__device__ __forceinline__ void split_head_tail(float c, __nv_bfloat16* head, __nv_bfloat16* tail) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(c);
+  *head = h;
+  *tail = __float2bfloat16_rn(c - __bfloat162float(h));
+}
+
+// Writes the token's dense coefficient rows hi[0, d), lo[0, d): the head and
+// tail of x where kept(key, i), zero elsewhere.  d a multiple of 8, hi and lo
+// 16-byte aligned; 8 entries (one 16-byte store to each row) per step.
+template <typename Kept>
+__device__ __forceinline__ void write_head_tail(const uint32_t* bits, int d, Kept kept,
+                                                __nv_bfloat16* hi, __nv_bfloat16* lo) {
+  for (int v = threadIdx.x; v < d / 8; v += kTopkThreads) {
+    __align__(16) __nv_bfloat16 h[8], t[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = 8 * v + e;
+      const uint32_t u = bits[i];
+      split_head_tail(kept(u & kKeyMask, i) ? __uint_as_float(u) : 0.f, &h[e], &t[e]);
+    }
+    reinterpret_cast<uint4*>(hi)[v] = *reinterpret_cast<const uint4*>(h);
+    reinterpret_cast<uint4*>(lo)[v] = *reinterpret_cast<const uint4*>(t);
+  }
+}
+
+// With hl != nullptr the kernel also writes each token's dense coefficient
+// rows for the tensor-core product: hl[m][0, d) the heads, hl[M + m][0, d)
+// the tails (d a multiple of 8).
 __global__ void __launch_bounds__(kTopkThreads, 1)
     topk_kernel(const float* __restrict__ x_rot, int d, int K, int32_t* __restrict__ idx,
-                float* __restrict__ val, int* dev_status) {
+                float* __restrict__ val, int* dev_status, __nv_bfloat16* hl) {
   // raw fp32 bits of the row, padded with zero keys to a multiple of 4: a
   // zero key at an index >= d loses every tie, so padding is never kept
   extern __shared__ __align__(16) uint32_t bits[];
@@ -83,15 +114,55 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   if (tid == 0 && d4 > d) atomicAdd(&sel.hist[0], static_cast<uint32_t>(d4 - d));
   if (__syncthreads_or(nonfinite) && tid == 0) report(dev_status, LAROSA_DEV_NONFINITE);
 
-  if (K == 0) return;
+  // the K-th entry (T, I): K = 0 keeps nothing, K = d everything
+  KthEntry e{0xffffffffu, -1};
   if (K == d) {
+    e = KthEntry{0u, d};
     for (int i = tid; i < d; i += kTopkThreads) {
       out_i[i] = i;
       out_v[i] = __uint_as_float(bits[i]);
     }
-    return;
+  } else if (K > 0) {
+    uint32_t B, above, nB;
+    fine_boundary<kTopkThreads>(&sel, K, &B, &above, &nB);
+    e = kth_entry<kTopkThreads>(bits, d4, K, B, static_cast<uint32_t>(K) - above, nB, &sel, cand, cand_idx,
+                                kTopkCand);
+    write_kept<kTopkThreads>(bits, d4, e, 0, K, out_i, out_v, &sel);
   }
-  kept_list<kTopkThreads>(bits, d4, K, &sel, cand, cand_idx, kTopkCand, 0, K, out_i, out_v);
+  if (hl != nullptr) {
+    const size_t M = gridDim.x;
+    write_head_tail(bits, d, [&](uint32_t key, int i) { return is_kept(key, i, e); }, hl + (size_t)m * d,
+                    hl + (M + m) * d);
+  }
+}
+
+// The tokens' dense coefficient rows for the tensor-core sparse linear, from
+// given kept lists: hl[m][i] / hl[M + m][i] = head / tail of val[m][k] where
+// idx[m][k] = i, zero at rows no entry names.  One CTA per token builds the
+// row in shared memory (indices within a row are distinct, so no two threads
+// write one word) and stores it with 16-byte stores.  An index outside
+// [0, d) sets LAROSA_DEV_INDEX and is skipped.
+__global__ void __launch_bounds__(kTopkThreads, 1)
+    coef_rows_kernel(const int32_t* __restrict__ idx, const float* __restrict__ val, int K, int d,
+                     __nv_bfloat16* hl, int* dev_status) {
+  extern __shared__ __align__(16) uint32_t row[];  // [d] fp32 coefficients
+  const int m = blockIdx.x;
+  for (int i = threadIdx.x; i < d; i += kTopkThreads) row[i] = 0u;
+  __syncthreads();
+  pdl_wait();
+  pdl_launch_dependents();
+  bool bad = false;
+  for (int k = threadIdx.x; k < K; k += kTopkThreads) {
+    const int i = __ldg(idx + (size_t)m * K + k);
+    if (static_cast<unsigned>(i) < static_cast<unsigned>(d))
+      row[i] = __float_as_uint(__ldg(val + (size_t)m * K + k));
+    else
+      bad = true;
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) report(dev_status, LAROSA_DEV_INDEX);
+  const size_t M = gridDim.x;
+  // every word of the row is the coefficient itself (0 where not named)
+  write_head_tail(row, d, [](uint32_t, int) { return true; }, hl + (size_t)m * d, hl + (M + m) * d);
 }
 
 // ---------------------------------------------------------------- threshold
@@ -170,8 +241,36 @@ cudaError_t launch_threshold(const float* x_rot, int M, int d, uint32_t t_key, i
                             dev_status);
 }
 
+cudaError_t launch_coef_rows(const int32_t* idx, const float* val, int M, int K, int d, __nv_bfloat16* hl,
+                             int* dev_status, cudaStream_t stream) {
+  if (d % 8 != 0) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)d * sizeof(uint32_t);
+  static int configured[64] = {0};  // per device: dynamic shared memory limit raised
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !configured[dev]) {
+    e = cudaFuncSetAttribute(coef_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(LAROSA_MAX_D * sizeof(uint32_t)));
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) configured[dev] = 1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(M, 1, 1);
+  cfg.blockDim = dim3(kTopkThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, coef_rows_kernel, idx, val, K, d, hl, dev_status);
+}
+
 cudaError_t launch_topk(const float* x_rot, int M, int d, int K, int32_t* idx, float* val,
-                        int* dev_status, cudaStream_t stream) {
+                        int* dev_status, cudaStream_t stream, __nv_bfloat16* hl) {
+  if (hl != nullptr && d % 8 != 0) return cudaErrorInvalidValue;
   const size_t smem = (size_t)((d + 3) & ~3) * sizeof(uint32_t);
   static int configured[64] = {0};  // per device: dynamic shared memory limit raised
   int dev = 0;
@@ -193,7 +292,7 @@ cudaError_t launch_topk(const float* x_rot, int M, int d, int K, int32_t* idx, f
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, topk_kernel, x_rot, d, K, idx, val, dev_status);
+  return cudaLaunchKernelEx(&cfg, topk_kernel, x_rot, d, K, idx, val, dev_status, hl);
 }
 
 }  // namespace larosa

@@ -328,8 +328,8 @@ int larosa_dense_linear(const void *x, const void *Wt, int M, int d_in,
  * LAROSA_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds
  * until the process exits.  larosa_sparse_linear_noalloc_bytes() gives the
  * scratch a size needs.  Sizes whose scratch would exceed the array (in
- * practice only large multi-token batches, e.g. M = 16 with d_in = 32768)
- * return LAROSA_ERR_WORKSPACE with the byte counts in
+ * practice only large multi-token batches, e.g. 16 fp32 tokens with
+ * d_in = 32768) return LAROSA_ERR_WORKSPACE with the byte counts in
  * larosa_last_error_string().  The call allocates nothing; it clears the
  * words that must start at zero with cudaMemsetAsync on `stream`.  All calls
  * on one device share the array, so calls that may overlap on that GPU race:
