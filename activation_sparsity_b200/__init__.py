@@ -17,6 +17,7 @@ fallback path.  (``build_lib`` builds the library without loading it.)
 _EXPORTS = (
     "LarosaError", "Workspace", "larosa_check", "larosa_dense_linear", "larosa_prepare_weights",
     "larosa_rotate", "larosa_rotate_topk", "larosa_rotate_topk_linear", "larosa_sparse_linear",
+    "larosa_topk_linear",
     "larosa_sparse_linear_noalloc", "larosa_topk", "larosa_version", "larosa_workspace_bytes",
     "larosa_workspace_layout", "larosa_workspace_nnz_offset", "larosa_threshold",
     "larosa_rotate_threshold_linear", "larosa_fold_rotation",

@@ -619,6 +619,34 @@ int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, 
   return run_sparse(idx, val, M, K, W_rot, d_in, d_out, y, dtype, ws, L, dev_status, s);
 }
 
+int larosa_topk_linear(const float* x_rot, const void* W_rot, int M, int d_in, int d_out, int K, float* y,
+                       void* ws, size_t ws_bytes, int* dev_status, int dtype, larosa_stream_t stream) {
+  if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
+  if (x_rot == nullptr || W_rot == nullptr || y == nullptr) return LAROSA_ERR_INVALID_ARG;
+  int st = check_sizes(M, d_in, d_out, K);
+  if (st != LAROSA_OK) return st;
+  if (!aligned16(x_rot) || !aligned16(W_rot) || !aligned16(y) || !row_aligned(d_out, dtype))
+    return LAROSA_ERR_ALIGN;
+  Layout L;
+  st = make_layout(M, d_in, d_out, K, &L);
+  if (st != LAROSA_OK) return st;
+  st = workspace_ok(ws, ws_bytes, L);
+  if (st != LAROSA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* idx = reinterpret_cast<int32_t*>(at(ws, L.idx));
+  float* val = reinterpret_cast<float*>(at(ws, L.val));
+  if (M > 1 && tensor_core_gemv(M, d_in, d_out, dtype, L)) {
+    __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(at(ws, L.coef_hl));
+    cudaError_t e = larosa::launch_topk(x_rot, M, d_in, K, idx, val, dev_status, s, hl);
+    if (e != cudaSuccess) return cuda_fail(e, "topk kernel");
+    e = larosa::launch_umma_gemv(W_rot, hl, y, M, d_in, d_out, dev_status, s);
+    return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "tensor-core sparse linear kernel");
+  }
+  cudaError_t e = larosa::launch_topk(x_rot, M, d_in, K, idx, val, dev_status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "topk kernel");
+  return run_sparse(idx, val, M, K, W_rot, d_in, d_out, y, dtype, ws, L, dev_status, s);
+}
+
 int larosa_threshold(const float* x_rot, int M, int d, float t, int32_t* idx, float* val,
                      int32_t* nnz, int* dev_status, larosa_stream_t stream) {
   if (x_rot == nullptr || idx == nullptr || val == nullptr || nnz == nullptr || t != t)

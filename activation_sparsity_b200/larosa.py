@@ -43,6 +43,7 @@ _SIGNATURES = {
     "larosa_rotate_topk": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _vp, _sz, _vp, _i, _vp], _i),
     "larosa_sparse_linear": ([_vp, _vp, _i, _i, _vp, _i, _i, _vp, _vp, _sz, _i, _vp, _vp], _i),
     "larosa_rotate_topk_linear": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp, _i, _vp], _i),
+    "larosa_topk_linear": ([_vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp, _i, _vp], _i),
     "larosa_threshold": ([_vp, _i, _i, _c.c_float, _vp, _vp, _vp, _vp, _vp], _i),
     "larosa_rotate_threshold_linear": ([_vp, _vp, _vp, _i, _i, _i, _c.c_float, _vp, _vp, _sz, _vp, _i,
                                         _vp], _i),
@@ -398,6 +399,27 @@ def larosa_rotate_topk_linear(x: torch.Tensor, Qt: torch.Tensor | None, W_rot: t
     _check(_lib.larosa_rotate_topk_linear(_ptr(x2), _ptr(Qt), _ptr(W_rot), M, d_in, d_out, K, _ptr(y),
                                           p, n, _status_ptr(dev_status, x.device), _dtype_code(x),
                                           _stream(x.device)), "larosa_rotate_topk_linear")
+    return y
+
+
+def larosa_topk_linear(x_rot: torch.Tensor, W_rot: torch.Tensor, K: int, y: torch.Tensor | None = None,
+                       ws=None, dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """Top-K of an already rotated fp32 vector and the sparse linear over the kept
+    rows of W_rot, fp32 output [M, d_out] (the kept list stays in the workspace)."""
+    _need(x_rot, "x_rot", torch.float32)
+    _need(W_rot, "W_rot")
+    x2 = _as2d(x_rot)
+    M, d_in = x2.shape
+    d_out = W_rot.shape[1]
+    if W_rot.shape[0] != d_in:
+        raise ValueError("W_rot must be [d_in, d_out]")
+    if y is None:
+        y = torch.empty((M, d_out), dtype=torch.float32, device=x_rot.device)
+    _need(y, "y", torch.float32)
+    p, n = _ws_args(ws, x_rot.device, M, d_in, d_out, K)
+    _check(_lib.larosa_topk_linear(_ptr(x2), _ptr(W_rot), M, d_in, d_out, K, _ptr(y), p, n,
+                                   _status_ptr(dev_status, x_rot.device), _dtype_code(W_rot),
+                                   _stream(x_rot.device)), "larosa_topk_linear")
     return y
 
 

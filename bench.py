@@ -675,9 +675,9 @@ def bench_larosa(args):
         for gi, g in enumerate(groups):
             L.larosa_sparse_linear(idxs[gi], vals[gi], g.W_rot, y=ys[gi], ws=ws, dev_status=st)
 
-    def sparse_only_step():  # the same path on pre-rotated inputs (no Q streamed)
-        topk_step()
-        gather_step()
+    def sparse_only_step():  # the same path on pre-rotated inputs (no Q streamed): Top-K + sparse linear
+        for gi, g in enumerate(groups):
+            L.larosa_topk_linear(x_rots[gi], g.W_rot, g.K, y=ys[gi], ws=ws, dev_status=st)
 
     def dense_step():
         for g, y in zip(groups, ys):

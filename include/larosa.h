@@ -237,6 +237,27 @@ int larosa_rotate_topk_linear(const void *x, const void *Qt, const void *W_rot,
                               int dtype, larosa_stream_t stream);
 
 /*
+ * Steps 2 and 3 for a vector that is already rotated (La RoSA summary,
+ * 方法详解 / 技术框架: keep the K largest magnitudes of each rotated
+ * activation vector, then multiply by the counter-rotated weight):
+ *   (idx, val) = TopK(x_rot, K) with larosa_topk's rule;
+ *   y = sum_k val[k] * W_rot[idx[k]].
+ * x_rot: [M x d_in] fp32 (as larosa_rotate writes it, or the output of a
+ * producer whose weight was counter-rotated with larosa_fold_rotation);
+ * W_rot: [d_in x d_out] of `dtype`; y: [M x d_out] fp32.  larosa_topk's
+ * kernel, then the sparse linear on its kept lists (from 8 bf16 tokens on,
+ * the Top-K kernel also writes the coefficient rows of the tensor-core
+ * product, as in larosa_rotate_topk_linear).  The kept list
+ * (ascending) lies in the workspace at the offsets larosa_workspace_layout
+ * gives.  x_rot, W_rot and y 16-byte aligned, d_out rows of 16 bytes.
+ * ws: at least larosa_workspace_bytes(M, d_in, d_out, K) bytes.  A NaN or
+ * Inf in x_rot sets LAROSA_DEV_NONFINITE.
+ */
+int larosa_topk_linear(const float *x_rot, const void *W_rot, int M, int d_in,
+                       int d_out, int K, float *y, void *ws, size_t ws_bytes,
+                       int *dev_status, int dtype, larosa_stream_t stream);
+
+/*
  * Threshold selection (R-Sparse report, 研究流程与方法 / R-Sparse框架设计: the
  * input channels with |x_j| >= t are kept, the rest masked; the count kept
  * varies from token to token):

@@ -7,8 +7,9 @@ projection group, run a few times through each decode entry point.
 For each group (``all``: q|k|v, o, gate|up, down in that order) each
 iteration launches, for one token: the fused call (one fused_kernel), the
 Top-K of a pre-rotated input (topk_kernel), the sparse linear on a fixed kept
-list (gather_kernel) and the dense baseline (rowdot_kernel on W in nn.Linear
-layout); ``--fused-only`` launches only the fused call.  With ``--tokens M``
+list (gather_kernel), the dense baseline (rowdot_kernel on W in nn.Linear
+layout) and the Top-K + sparse linear of the pre-rotated input in one call
+(topk_kernel, gather_kernel); ``--fused-only`` launches only the fused call.  With ``--tokens M``
 (2 to 16) each iteration runs M tokens through the same entry points: the
 rotation, the Top-K, the multi-token sparse linear and the fused call (for
 8 to 16 tokens the tcgen05 kernels).  One group takes 0.2-0.5 GB of device
@@ -79,6 +80,7 @@ def main(argv=None) -> int:
                 L.larosa_topk(x_rot, K, idx=idx, val=val, dev_status=st)
                 L.larosa_sparse_linear(idx, val, W_rot, y=y, ws=ws, dev_status=st)
                 L.larosa_dense_linear(x, Wt, y=y)
+                L.larosa_topk_linear(x_rot, W_rot, K, y=y, ws=ws, dev_status=st)
     torch.cuda.synchronize(dev)
     if L.larosa_check(st, device=dev) != 0:
         raise SystemExit("profile_case: the library reported a device status")
