@@ -1,21 +1,38 @@
-"""A small, fixed workload for kernel profilers (ncu): one LLaMA2-7B-shaped
-projection group, run a few times through each decode entry point.
+"""A small, fixed workload for kernel profilers (ncu): LLaMA2-7B-shaped
+projection groups run a few times through the library's entry points.
 
     python profile_case.py [--group gate_up|all] [--iters 3] [--sparsity 40]
-                           [--fused-only] [--tokens M]
+                           [--tokens M] [--calls fused,topk,...] [--fused-only]
 
 For each group (``all``: q|k|v, o, gate|up, down in that order) each
-iteration launches, for one token: the fused call (one fused_kernel), the
-Top-K of a pre-rotated input (topk_kernel), the sparse linear on a fixed kept
-list (gather_kernel), the dense baseline (rowdot_kernel on W in nn.Linear
-layout) and the Top-K + sparse linear of the pre-rotated input in one call
-(topk_kernel, gather_kernel); ``--fused-only`` launches only the fused call.  With ``--tokens M``
-(2 to 16) each iteration runs M tokens through the same entry points: the
-rotation, the Top-K, the multi-token sparse linear and the fused call (for
-8 to 16 tokens the tcgen05 kernels).  One group takes 0.2-0.5 GB of device
-memory, more than the 126 MB L2, and ncu flushes the caches before every
-replayed launch, so DRAM counters describe cold-cache launches.  Prints "ok"
-and exits 0 on success.
+iteration makes the calls named in --calls, in this order (default: all of
+them), each on the same seeded inputs:
+
+  fused        larosa_rotate_topk_linear     one token: fused_kernel; several:
+                                             rotation, topk_kernel and the
+                                             multi-token sparse linear
+  identity     the same with Qt = NULL       one token: fused_kernel without
+                                             its rotation
+  thresh_fused larosa_rotate_threshold_linear fused_kernel in threshold mode
+  rotate       larosa_rotate                 rowdot_kernel (1-2 tokens),
+                                             rowmma_kernel (3-7), umma_kernel (8-16)
+  rotate_topk  larosa_rotate_topk            rotsel_kernel (one token)
+  topk         larosa_topk                   topk_kernel
+  threshold    larosa_threshold              threshold_kernel
+  sparse       larosa_sparse_linear          gather_kernel (one token);
+                                             scatter, union, rowstream_gemv
+                                             (2-7 tokens); coef_rows and
+                                             umma_kernel (8-16)
+  topk_linear  larosa_topk_linear            topk_kernel, then the sparse linear
+  dense        larosa_dense_linear           as rotate, on W in nn.Linear layout
+  lowrank      larosa_sparse_lowrank_linear  the sparse linear, dropped_kernel,
+                                             two rowstream GEMVs (r = 256), add_kernel
+
+--fused-only is --calls fused.  The set-up (weights, the counter-rotation by
+prepare_kernel, the reference kept lists) runs before the first call.  One
+group takes 0.2-0.5 GB of device memory, more than the 126 MB L2, and ncu
+flushes the caches before every replayed launch, so DRAM counters describe
+cold-cache launches.  Prints "ok" and exits 0 on success.
 """
 from __future__ import annotations
 
@@ -33,6 +50,9 @@ import synthdata as sd  # noqa: E402
 from activation_sparsity_b200 import larosa as L  # noqa: E402
 
 GROUPS = {p.name: p for p in sd.llama_layer(4096, 11008, 4096)}
+CALLS = ("fused", "identity", "thresh_fused", "rotate", "rotate_topk", "topk", "threshold", "sparse",
+         "topk_linear", "dense", "lowrank")
+RANK = 256  # low-rank factors of the lowrank call
 
 
 def main(argv=None) -> int:
@@ -41,11 +61,20 @@ def main(argv=None) -> int:
     ap.add_argument("--group", choices=sorted(GROUPS) + ["all"], default="gate_up")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--sparsity", type=float, default=40.0)
-    ap.add_argument("--fused-only", action="store_true")
     ap.add_argument("--tokens", type=int, default=1)
+    ap.add_argument("--calls", default=",".join(CALLS))
+    ap.add_argument("--fused-only", action="store_true")
     a = ap.parse_args(argv)
+    calls = ["fused"] if a.fused_only else [c for c in a.calls.split(",") if c]
+    bad = [c for c in calls if c not in CALLS]
+    if bad:
+        ap.error(f"unknown calls {bad}; choose from {CALLS}")
     if not 1 <= a.tokens <= 16:
         ap.error("--tokens must be 1 to 16")
+    M = a.tokens
+    one = M == 1
+    if not one:  # these entry points take one token
+        calls = [c for c in calls if c not in ("rotate_topk",)]
     if not torch.cuda.is_available():
         raise SystemExit("profile_case: no CUDA device (the library has no CPU path)")
     dev = torch.device("cuda", 0)
@@ -60,31 +89,61 @@ def main(argv=None) -> int:
         Qt = sd.orthogonal(p.d_in, base + 1, device=dev).to(torch.bfloat16).t().contiguous()
         W = sd.weights(p.d_in, p.d_out, 0.02, base + 2, torch.bfloat16, device=dev)
         W_rot = L.larosa_prepare_weights(Qt, W)
-        Wt = None if a.fused_only else W.t().contiguous()
-        del W
-        M = a.tokens
+        Wt = W.t().contiguous() if "dense" in calls else None
+        if "identity" not in calls:
+            W = None
         x = sd.activations(M, p.d_in, base + 3, torch.bfloat16, device=dev)
         K = sd.k_for_sparsity(p.d_in, a.sparsity)
         y = torch.empty((M, p.d_out), dtype=torch.float32, device=dev)
-        x_rot = idx = val = None
-        if not a.fused_only:
-            x_rot = L.larosa_rotate(x, Qt)
-            idx, val = L.larosa_topk(x_rot, K, dev_status=st)
-        cases.append((p, Qt, W_rot, Wt, x, K, y, x_rot, idx, val))
+        x_rot = L.larosa_rotate(x, Qt)
+        idx, val = L.larosa_topk(x_rot, K, dev_status=st)
+        t = float(torch.sort(x_rot.abs().flatten()).values[p.d_in - K].item())  # drops the same share
+        nnz = torch.empty((M,), dtype=torch.int32, device=dev)
+        thr = (torch.empty((M, p.d_in), dtype=torch.int32, device=dev),
+               torch.empty((M, p.d_in), dtype=torch.float32, device=dev))
+        lr = None
+        if "lowrank" in calls:
+            A_r = sd.weights(p.d_in, RANK, 0.02, base + 4, torch.bfloat16, device=dev)
+            B_r = sd.weights(RANK, p.d_out, 0.02, base + 5, torch.bfloat16, device=dev)
+            lr = (A_r, B_r, torch.zeros(L.larosa_lowrank_workspace_bytes(M, p.d_in, p.d_out, K, RANK),
+                                        dtype=torch.uint8, device=dev))
+        cases.append(dict(Qt=Qt, W=W, W_rot=W_rot, Wt=Wt, x=x, K=K, y=y, x_rot=x_rot, idx=idx, val=val,
+                          t=t, nnz=nnz, thr=thr, lr=lr))
     for _ in range(a.iters):
-        for p, Qt, W_rot, Wt, x, K, y, x_rot, idx, val in cases:
-            L.larosa_rotate_topk_linear(x, Qt, W_rot, K, y=y, ws=ws, dev_status=st)
-            if not a.fused_only:
-                if a.tokens > 1:
-                    L.larosa_rotate(x, Qt, x_rot=x_rot)
-                L.larosa_topk(x_rot, K, idx=idx, val=val, dev_status=st)
-                L.larosa_sparse_linear(idx, val, W_rot, y=y, ws=ws, dev_status=st)
-                L.larosa_dense_linear(x, Wt, y=y)
-                L.larosa_topk_linear(x_rot, W_rot, K, y=y, ws=ws, dev_status=st)
+        for c in cases:
+            for call in calls:
+                if call == "fused":
+                    L.larosa_rotate_topk_linear(c["x"], c["Qt"], c["W_rot"], c["K"], y=c["y"], ws=ws, dev_status=st)
+                elif call == "identity":
+                    L.larosa_rotate_topk_linear(c["x"], None, c["W"], c["K"], y=c["y"], ws=ws, dev_status=st)
+                elif call == "thresh_fused":
+                    L.larosa_rotate_threshold_linear(c["x"], c["Qt"], c["W_rot"], c["t"], y=c["y"], ws=ws,
+                                                     dev_status=st)
+                elif call == "rotate":
+                    L.larosa_rotate(c["x"], c["Qt"], x_rot=c["x_rot"])
+                elif call == "rotate_topk":
+                    L.larosa_rotate_topk(c["x"], c["Qt"], c["K"], x_rot=c["x_rot"], idx=c["idx"], val=c["val"],
+                                         ws=ws, dev_status=st)
+                elif call == "topk":
+                    L.larosa_topk(c["x_rot"], c["K"], idx=c["idx"], val=c["val"], dev_status=st)
+                elif call == "threshold":
+                    L.larosa_threshold(c["x_rot"], c["t"], idx=c["thr"][0], val=c["thr"][1], nnz=c["nnz"],
+                                       dev_status=st)
+                elif call == "sparse":
+                    L.larosa_sparse_linear(c["idx"], c["val"], c["W_rot"], y=c["y"], ws=ws, dev_status=st)
+                elif call == "topk_linear":
+                    L.larosa_topk_linear(c["x_rot"], c["W_rot"], c["K"], y=c["y"], ws=ws, dev_status=st)
+                elif call == "dense":
+                    L.larosa_dense_linear(c["x"], c["Wt"], y=c["y"])
+                elif call == "lowrank":
+                    A_r, B_r, lws = c["lr"]
+                    L.larosa_sparse_lowrank_linear(c["x_rot"], c["idx"], c["val"], c["W_rot"], A_r, B_r, y=c["y"],
+                                                   ws=lws, dev_status=st)
     torch.cuda.synchronize(dev)
     if L.larosa_check(st, device=dev) != 0:
         raise SystemExit("profile_case: the library reported a device status")
-    print(f"ok: groups {','.join(names)} tokens {a.tokens} sparsity {a.sparsity}% iters {a.iters}")
+    print(f"ok: groups {','.join(names)} tokens {M} calls {','.join(calls)} sparsity {a.sparsity}% "
+          f"iters {a.iters}")
     return 0
 
 
