@@ -132,14 +132,14 @@ cudaError_t launch_gather(Elem w_elem, const GatherArgs& a, const StreamPlan& pl
 cudaError_t launch_rowdot(Elem e, const void* A, const void* x, float* y, int M, int n_in,
                           int n_out, cudaStream_t stream);
 
-// The same row-dot product for 8 to 16 bf16 tokens on tcgen05 (TMEM
+// The same row-dot product for 2 to 16 bf16 tokens on tcgen05 (TMEM
 // accumulator, TMA-fed shared-memory operands); rot_umma_applies tells
 // whether the shapes suit it (n_in a multiple of 64).
 bool rot_umma_applies(int M, int n_in, int n_out);
 cudaError_t launch_rot_umma(const void* A, const void* x, float* y, int M, int n_in, int n_out,
                             int* dev_status, cudaStream_t stream);
 
-// The sparse linear of 8 to 16 tokens as a dense tensor-core product over
+// The sparse linear of 2 to 16 tokens as a dense tensor-core product over
 // every row of W (bf16) with the per-token coefficient rows (zero where a
 // token did not keep the row), given as bf16 head and tail hl [2 x M x d_in]
 // (launch_topk or launch_coef_rows): y = (head + tail) . W on tcgen05.

@@ -1,4 +1,4 @@
-// Products of 8 to 16 bf16 tokens on the fifth-generation tensor cores
+// Products of 2 to 16 bf16 tokens on the fifth-generation tensor cores
 // (sm_100a), both HBM-bound streams of a bf16 matrix:
 //
 //   row-dot  y[m][j] = sum_i x[m][i] * A[j][i], A row-major [n_out x n_in]:
@@ -9,9 +9,9 @@
 //   GEMV     y[m][c] = sum_r coef[m][r] * W[r][c], W row-major [d_in x d_out]:
 //            the sparse linear of several tokens over every row of the
 //            counter-rotated weight (abstract: activation sparsity reduces
-//            memory transfers; from 8 tokens on, the rows some token keeps
-//            are nearly all of them), each token's coefficient row zero
-//            where it did not keep the row.
+//            memory transfers; from a few tokens on, the rows some token
+//            keeps are nearly all of them), each token's coefficient row
+//            zero where it did not keep the row.
 //
 // One MMA tile is 128 output elements (M) by the token slots (N), over 16
 // inputs (K) per instruction; the accumulators live in TMEM.  A CTA owns
@@ -506,8 +506,15 @@ cudaError_t plan_umma(int n_in, int n_out, int* R, long long* t) {
 
 }  // namespace
 
+// From two tokens on the tensor-core kernels take the batch path: their cost
+// does not depend on the token count (16 slots, the unused ones zero), and
+// they stream faster than the CUDA-core kernels (the row-dot of 2 tokens,
+// mma.sync for 3-7, the row-streaming GEMV over the union of kept rows) even
+// where the union of two tokens' kept rows is only 84 % of the weight.
+constexpr int kUMinTokens = 2;
+
 bool rot_umma_applies(int M, int n_in, int n_out) {
-  return M >= 8 && M <= kUTokens && n_in % kUBox == 0 && n_out % 8 == 0 && n_in >= kUBox;
+  return M >= kUMinTokens && M <= kUTokens && n_in % kUBox == 0 && n_out % 8 == 0 && n_in >= kUBox;
 }
 
 cudaError_t launch_rot_umma(const void* A, const void* x, float* y, int M, int n_in, int n_out,
@@ -523,7 +530,7 @@ cudaError_t launch_rot_umma(const void* A, const void* x, float* y, int M, int n
 }
 
 bool umma_gemv_applies(int M, int d_in, int d_out) {
-  return M >= 8 && M <= kUTokens && d_in % 8 == 0 && d_out % 8 == 0 && d_in >= kUBox;
+  return M >= kUMinTokens && M <= kUTokens && d_in % 8 == 0 && d_out % 8 == 0 && d_in >= kUBox;
 }
 
 // Column tiles of 256 (two accumulators) read each weight row 512 contiguous

@@ -199,7 +199,11 @@ int larosa_rotate_topk(const void *x, const void *Qt, float *x_rot,
  * idx/val: [M x K] as written by larosa_topk (each row's indices distinct;
  * ascending order is not required for correctness).  W_rot: [d_in x d_out]
  * of `dtype`; only the rows named in idx are read.  y: [M x d_out] fp32.
- * For M > 1 the rows named by any token are streamed once and shared.
+ * For M > 1 the rows named by any token are streamed once and shared; with
+ * bf16 weights every row is, as a dense tensor-core product with each
+ * token's coefficient row (zero at the rows it did not keep), since the
+ * tokens' kept rows cover most rows (84 % at two tokens and 40 % sparsity,
+ * nearly all from four on).
  * An index outside [0, d_in) sets LAROSA_DEV_INDEX and contributes nothing.
  * ws: at least larosa_workspace_bytes(M, d_in, d_out, K) bytes.
  */
@@ -245,7 +249,7 @@ int larosa_rotate_topk_linear(const void *x, const void *Qt, const void *W_rot,
  * x_rot: [M x d_in] fp32 (as larosa_rotate writes it, or the output of a
  * producer whose weight was counter-rotated with larosa_fold_rotation);
  * W_rot: [d_in x d_out] of `dtype`; y: [M x d_out] fp32.  larosa_topk's
- * kernel, then the sparse linear on its kept lists (from 8 bf16 tokens on,
+ * kernel, then the sparse linear on its kept lists (from 2 bf16 tokens on,
  * the Top-K kernel also writes the coefficient rows of the tensor-core
  * product, as in larosa_rotate_topk_linear).  The kept list
  * (ascending) lies in the workspace at the offsets larosa_workspace_layout

@@ -1,7 +1,7 @@
-"""The tcgen05 kernels for 8 to 16 tokens against the fp64 oracle, smallest
-cases first: the rotation / dense row-dot product (one 128 x 16 MMA tile per
-CTA, split over a cluster) and the sparse linear as a dense product with the
-tokens' coefficients.  Bars as in test_gpu_parity: the fp32 summation bound
+"""The tcgen05 kernels for 2 to 16 tokens against the fp64 oracle, smallest
+cases first: the rotation / dense row-dot product (128 output rows x 16 token
+slots per CTA, split over a cluster) and the sparse linear as a dense product
+with the tokens' coefficients (256 output columns per CTA).  Bars as in test_gpu_parity: the fp32 summation bound
 per element; for the sparse linear also the coefficients' bf16 head + tail
 representation (2^-16 of each coefficient) and the 2e-3 norm bar.
 """
@@ -25,7 +25,8 @@ def L():
     return L
 
 
-@pytest.mark.parametrize("M,d", [(16, 64), (8, 128), (12, 256), (16, 1024), (16, 4096), (8, 11008)])
+@pytest.mark.parametrize("M,d", [(16, 64), (8, 128), (12, 256), (2, 512), (4, 1024), (5, 192), (16, 1024),
+                                 (16, 4096), (8, 11008), (3, 11008)])
 def test_rotate_tcgen05(L, M, d):
     Q = sd.orthogonal(d, 211, device="cuda" if d > 4096 else "cpu").to(torch.bfloat16)
     x = sd.activations(M, d, 212, torch.bfloat16)
@@ -36,7 +37,8 @@ def test_rotate_tcgen05(L, M, d):
     assert np.all(np.abs(got - ref) <= bound + 1e-30)
 
 
-@pytest.mark.parametrize("M,d_in,d_out", [(16, 64, 8), (8, 128, 136), (16, 512, 1000), (16, 4096, 4096)])
+@pytest.mark.parametrize("M,d_in,d_out", [(16, 64, 8), (8, 128, 136), (16, 512, 1000), (2, 4096, 4096),
+                                         (16, 4096, 4096)])
 def test_dense_tcgen05(L, M, d_in, d_out):
     x = sd.activations(M, d_in, 221, torch.bfloat16)
     W = sd.weights(d_in, d_out, 0.02, 222, torch.bfloat16)
@@ -47,7 +49,8 @@ def test_dense_tcgen05(L, M, d_in, d_out):
 
 
 @pytest.mark.parametrize("M,d_in,d_out,K", [(8, 64, 128, 20), (16, 512, 1032, 300), (16, 4096, 4096, 2458),
-                                            (12, 11008, 4096, 6605)])
+                                            (12, 11008, 4096, 6605), (2, 512, 264, 300), (4, 4096, 4096, 2458),
+                                            (7, 1000, 2056, 400)])
 def test_sparse_tcgen05(L, M, d_in, d_out, K):
     idx, val = sd.index_values(M, d_in, K, 230 + K)
     W = sd.weights(d_in, d_out, 0.02, 231, torch.bfloat16)

@@ -92,9 +92,9 @@ def test_topk_linear_several_tokens(L, M):
     x = sd.activations(M, d_in, 1420 + M, torch.float32).cuda()
     W = sd.weights(d_in, d_out, 0.02, 1421, torch.bfloat16, device="cuda")
     y, idx, val = run(L, x, W, K)
-    # from 8 bf16 tokens on the tensor cores multiply each coefficient as a
+    # from 2 bf16 tokens on the tensor cores multiply each coefficient as a
     # bf16 head and tail, within 2^-16 of its value
-    check(y, idx, val, x, W, K, rep=2.0 ** -16 if M >= 8 else 0.0)
+    check(y, idx, val, x, W, K, rep=2.0 ** -16)
 
 
 def test_topk_linear_is_deterministic_and_matches_the_two_calls(L):

@@ -59,9 +59,9 @@ def _check_against_oracle(y, idx, val, W):
     i64 = idx.cpu().numpy().astype(np.int64)
     v64 = val.double().cpu().numpy()
     M, K = i64.shape
-    # from 8 bf16 tokens on the tensor cores multiply each coefficient as a
+    # from 2 bf16 tokens on the tensor cores multiply each coefficient as a
     # bf16 head and tail, which keep it to within 2^-16 of its value
-    rep = 2.0 ** -16 if (M >= 8 and W.dtype == torch.bfloat16) else 0.0
+    rep = 2.0 ** -16 if (M >= 2 and W.dtype == torch.bfloat16) else 0.0
     for m in range(M):
         ref = oracle.sparse_linear(i64[m], v64[m], Wd)
         bound = ((K + 2) * U + rep) * (np.abs(v64[m]) @ np.abs(Wd[i64[m]]))
