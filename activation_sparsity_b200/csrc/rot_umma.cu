@@ -44,6 +44,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tcgen05.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -97,77 +98,6 @@ struct UParams {
   unsigned long long wait_ns;  // limit of every mbarrier wait
 };
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-      : "memory");
-}
-
-// Shared-memory matrix descriptor of a K-major tile in the 128-byte swizzled
-// layout: 8-row groups 1024 bytes apart (stride byte offset), leading byte
-// offset 1 (unused by swizzled K-major layouts), descriptor version 1,
-// layout type 2 (128-byte swizzle).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-// Shared-memory descriptor of an MN-major tile in the 128-byte swizzled
-// layout: atoms of 64 MN-elements x 8 K-rows (1024 bytes), K-atoms `sbo`
-// bytes apart, MN-atoms `lbo` bytes apart.
-__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B,
-// B K-major, M = 128, N = n; A MN-major when a_mn.
-constexpr uint32_t idesc(int n, bool a_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn ? (1u << 15) : 0u) | ((uint32_t)(n >> 3) << 17) |
-         ((uint32_t)(128 >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate,
-                                          uint32_t id) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
-      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(id), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u),
-      "r"(0u));
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// 16 consecutive fp32 accumulator columns of this thread's
-// TMEM lane into registers.  The whole warp issues it together.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-      "%14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int c = 0; c < 16; ++c) v[c] = __uint_as_float(r[c]);
-}
-
 // kGemv = false: y[m][j] = sum_i x[m][i] A[j][i] (A = map_a, K-major rows;
 // x = map_b0).  kGemv = true: y[m][c] = sum_r coef[m][r] W[r][c] (W = map_a,
 // read MN-major; the coefficients' bf16 heads map_b0 and tails map_b1).
@@ -178,7 +108,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
   using C = UCfg<kGemv, kNB>;
   using S = UShape<kGemv, kNB>;
   constexpr int kStages = C::kStages;
-  constexpr uint32_t kId = idesc(C::kN, kGemv);
+  constexpr uint32_t kId = tc::idesc(C::kN, kGemv);
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // the swizzled stages need 1024-byte alignment
   unsigned char* stages = reinterpret_cast<unsigned char*>(
@@ -210,9 +140,9 @@ __global__ void __launch_bounds__(kUThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  tmem_fence_before();
+  tc::tmem_fence_before();
   __syncthreads();
-  tmem_fence_after();
+  tc::tmem_fence_after();
   const uint32_t tmem = s_tmem;
   volatile int* abort_flag = &s_abort;
 
@@ -228,11 +158,11 @@ __global__ void __launch_bounds__(kUThreads, 1)
     if constexpr (kGemv) {
       // 64 rows of W (the reduction) x kCols columns, as 64-column boxes
 #pragma unroll
-      for (int j = 0; j < 2 * C::kNB; ++j) tma_load_2d(a_dst + j * 8192, &map_a, j0 + 64 * j, k, &full[s]);
+      for (int j = 0; j < 2 * C::kNB; ++j) tc::tma_load_2d(a_dst + j * 8192, &map_a, j0 + 64 * j, k, &full[s]);
     } else {
       // kKB boxes of 128 rows of A x 64 inputs
 #pragma unroll
-      for (int kb = 0; kb < C::kKB; ++kb) tma_load_2d(a_dst + kb * 16384, &map_a, k + kUBox * kb, j0, &full[s]);
+      for (int kb = 0; kb < C::kKB; ++kb) tc::tma_load_2d(a_dst + kb * 16384, &map_a, k + kUBox * kb, j0, &full[s]);
     }
   };
   auto load_b = [&](int it) {
@@ -240,12 +170,12 @@ __global__ void __launch_bounds__(kUThreads, 1)
     unsigned char* b_dst = stages + (size_t)s * S::kStage + S::kABytes;
     const int k = k0 + it * S::kChunk;
     if constexpr (kGemv) {
-      tma_load_2d(b_dst, &map_b0, k, 0, &full[s]);
-      tma_load_2d(b_dst + kUTokens * kUBox * 2, &map_b1, k, 0, &full[s]);
+      tc::tma_load_2d(b_dst, &map_b0, k, 0, &full[s]);
+      tc::tma_load_2d(b_dst + kUTokens * kUBox * 2, &map_b1, k, 0, &full[s]);
     } else {
 #pragma unroll
       for (int kb = 0; kb < C::kKB; ++kb)
-        tma_load_2d(b_dst + kb * (kUTokens * kUBox * 2), &map_b0, k + kUBox * kb, 0, &full[s]);
+        tc::tma_load_2d(b_dst + kb * (kUTokens * kUBox * 2), &map_b0, k + kUBox * kb, 0, &full[s]);
     }
   };
 
@@ -283,18 +213,18 @@ __global__ void __launch_bounds__(kUThreads, 1)
           *abort_flag = 1;
           break;
         }
-        tmem_fence_after();
+        tc::tmem_fence_after();
         const uint32_t a_addr = smem_u32(stages + (size_t)s * S::kStage);
         const uint32_t b_addr = a_addr + S::kABytes;
         if constexpr (kGemv) {
 #pragma unroll
           for (int kk = 0; kk < kUBox / 16; ++kk) {  // 16 rows of W per instruction: two 8-row atoms
-            const uint64_t bd = sw128_desc(b_addr + kk * 32);
+            const uint64_t bd = tc::sw128_desc(b_addr + kk * 32);
 #pragma unroll
             for (int nb = 0; nb < C::kNB; ++nb) {
               // columns 128 nb .. 128 nb + 127: two 64-column boxes 8 KB apart
-              const uint64_t ad = sw128_mn_desc(a_addr + nb * 16384 + kk * 2048, 8192, 1024);
-              umma_bf16(tmem + nb * C::kN, ad, bd, (it > 0 || kk > 0) ? 1u : 0u, kId);
+              const uint64_t ad = tc::sw128_mn_desc(a_addr + nb * 16384 + kk * 2048, 8192, 1024);
+              tc::umma_bf16(tmem + nb * C::kN, ad, bd, (it > 0 || kk > 0) ? 1u : 0u, kId);
             }
           }
         } else {
@@ -302,13 +232,13 @@ __global__ void __launch_bounds__(kUThreads, 1)
           for (int kb = 0; kb < C::kKB; ++kb)
 #pragma unroll
             for (int kk = 0; kk < kUBox / 16; ++kk)  // 16 inputs per instruction
-              umma_bf16(tmem, sw128_desc(a_addr + kb * 16384 + kk * 32),
-                        sw128_desc(b_addr + kb * (kUTokens * kUBox * 2) + kk * 32),
+              tc::umma_bf16(tmem, tc::sw128_desc(a_addr + kb * 16384 + kk * 32),
+                        tc::sw128_desc(b_addr + kb * (kUTokens * kUBox * 2) + kk * 32),
                         (it > 0 || kb > 0 || kk > 0) ? 1u : 0u, kId);
         }
-        umma_commit(&empty[s]);  // the stage is free once these MMAs have read it
+        tc::umma_commit(&empty[s]);  // the stage is free once these MMAs have read it
       }
-      umma_commit(&done);  // every MMA issued above has completed
+      tc::umma_commit(&done);  // every MMA issued above has completed
     }
   }
   __syncwarp();
@@ -316,7 +246,7 @@ __global__ void __launch_bounds__(kUThreads, 1)
   // ------------------------------------------------------------------ epilogue
   // all MMAs (and so all their shared-memory reads) are complete once `done` fires
   const bool ok = mbar_wait_bounded(&done, 0, nullptr, p.wait_ns);
-  tmem_fence_after();
+  tc::tmem_fence_after();
   __syncwarp();  // tcgen05.ld is .aligned: the whole warp issues it together
   if (!ok) *abort_flag = 1;
   __syncthreads();
@@ -335,20 +265,20 @@ __global__ void __launch_bounds__(kUThreads, 1)
 #pragma unroll
   for (int nb = 0; nb < C::kNB; ++nb) {
     float v[16];
-    tmem_ld16(lane_base + nb * C::kN, v);
+    tc::tmem_ld16(lane_base + nb * C::kN, v);
     if constexpr (kGemv) {
       float t[16];
-      tmem_ld16(lane_base + nb * C::kN + kUTokens, t);  // the tails' products
+      tc::tmem_ld16(lane_base + nb * C::kN + kUTokens, t);  // the tails' products
 #pragma unroll
       for (int c = 0; c < 16; ++c) v[c] += t[c];
     }
 #pragma unroll
     for (int c = 0; c < kUTokens; ++c) part[c * S::kCols + nb * 128 + tid] = n_it > 0 ? v[c] : 0.f;
   }
-  tmem_fence_before();
+  tc::tmem_fence_before();
   __syncthreads();
   if (warp == 2) {
-    tmem_fence_after();
+    tc::tmem_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(S::kTmemCols)
                  : "memory");
   }
@@ -369,39 +299,6 @@ __global__ void __launch_bounds__(kUThreads, 1)
     }
   }
   cluster.sync();  // no CTA leaves while another may still read its partial tile
-}
-
-// The driver's tensor-map encoder, looked up through the runtime so that the
-// library does not link against the driver library itself.
-using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encoder() {
-  static EncodeTiled fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiled>(p);
-  }
-  return fn;
-}
-
-// A 2-D bf16 tensor map of a row-major [rows x cols] matrix, box
-// [box_rows x 64 columns], 128-byte swizzle; elements past the matrix read
-// as zero.
-bool make_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
-  const EncodeTiled enc = encoder();
-  if (enc == nullptr) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kUBox, (cuuint32_t)box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Splits of the reduction per tile, for `slots` co-resident CTAs: the S in
@@ -520,7 +417,7 @@ bool rot_umma_applies(int M, int n_in, int n_out) {
 cudaError_t launch_rot_umma(const void* A, const void* x, float* y, int M, int n_in, int n_out,
                             int* dev_status, cudaStream_t stream) {
   CUtensorMap map_a, map_x;
-  if (!make_map(&map_a, A, n_out, n_in, 128) || !make_map(&map_x, x, M, n_in, kUTokens))
+  if (!tc::make_map(&map_a, A, n_out, n_in, 128) || !tc::make_map(&map_x, x, M, n_in, kUTokens))
     return cudaErrorInvalidValue;
   int R = 1;
   long long t = 0;
@@ -543,8 +440,8 @@ cudaError_t launch_umma_gemv(const void* W, const __nv_bfloat16* hl, float* y, i
                              int* dev_status, cudaStream_t stream) {
   CUtensorMap map_w, map_hi, map_lo;
   // W: d_in rows (the reduction) of d_out columns, boxes of 64 rows x 64 columns
-  if (!make_map(&map_w, W, d_in, d_out, kUBox) || !make_map(&map_hi, hl, M, d_in, kUTokens) ||
-      !make_map(&map_lo, hl + (size_t)M * d_in, M, d_in, kUTokens))
+  if (!tc::make_map(&map_w, W, d_in, d_out, kUBox) || !tc::make_map(&map_hi, hl, M, d_in, kUTokens) ||
+      !tc::make_map(&map_lo, hl + (size_t)M * d_in, M, d_in, kUTokens))
     return cudaErrorInvalidValue;
   int R1 = 1, R2 = 1;
   long long t1 = 0, t2 = 0;
