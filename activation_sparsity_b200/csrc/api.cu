@@ -303,6 +303,9 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
 struct LowrankLayout {
   Layout base;
   size_t x_drop = 0, u = 0, y_r = 0, partials = 0, total = 0;
+  // one token in one launch (lowrank_kernel): its u, partials and counters
+  bool one_launch = false;
+  size_t lr_u = 0, lr_partials = 0, lr_sync = 0;
 };
 
 int make_lowrank_layout(int M, int d_in, int d_out, int K, int r, LowrankLayout* LL) {
@@ -329,6 +332,24 @@ int make_lowrank_layout(int M, int d_in, int d_out, int K, int r, LowrankLayout*
   LL->u = take((size_t)M * r * 4);
   LL->y_r = take((size_t)M * d_out * 4);
   LL->partials = take(pf * 4);
+  if (M == 1) {
+    // the one-launch kernel, for either weight type
+    size_t lp = 0;
+    bool ok = true;
+    for (int dt = 0; dt < 2; ++dt) {
+      larosa::StreamPlan pl;
+      cudaError_t e = larosa::plan_lowrank(dt == 0 ? Elem::F32 : Elem::BF16, d_in, d_out, K, r, &pl);
+      if (e != cudaSuccess) return cuda_fail(e, "plan low-rank kernel");
+      ok = ok && pl.ok;
+      lp = std::max(lp, pl.partial_floats);
+    }
+    if (ok) {
+      LL->one_launch = true;
+      LL->lr_sync = take((2 + larosa::kFusedMaxTiles) * 4);
+      LL->lr_u = take((size_t)r * 4);
+      LL->lr_partials = take(lp * 4);
+    }
+  }
   LL->total = off;
   return LAROSA_OK;
 }
@@ -783,6 +804,32 @@ int larosa_sparse_lowrank_linear(const float* x, const int32_t* idx, const float
   if (st != LAROSA_OK) return st;
   if (ws == nullptr || !aligned16(ws) || ws_bytes < LL.total) return LAROSA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (M == 1 && LL.one_launch) {
+    // one cooperative launch: kept rows of W, x_drop . A_r, then u . B_r
+    larosa::StreamPlan pl;
+    cudaError_t e = larosa::plan_lowrank(elem_of(dtype), d_in, d_out, K, r, &pl);
+    if (e != cudaSuccess) return cuda_fail(e, "plan low-rank kernel");
+    if (pl.ok) {
+      larosa::LowrankArgs a;
+      a.x = x;
+      a.idx = idx;
+      a.val = val;
+      a.W = W;
+      a.A_r = A_r;
+      a.B_r = B_r;
+      a.y = y;
+      a.u = reinterpret_cast<float*>(at(ws, LL.lr_u));
+      a.partials = reinterpret_cast<float*>(at(ws, LL.lr_partials));
+      a.sync = reinterpret_cast<unsigned*>(at(ws, LL.lr_sync));
+      a.d_in = d_in;
+      a.d_out = d_out;
+      a.K = K;
+      a.r = r;
+      a.dev_status = dev_status;
+      e = larosa::launch_lowrank(elem_of(dtype), a, pl, s);
+      return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "low-rank kernel");
+    }
+  }
   float* x_drop = reinterpret_cast<float*>(at(ws, LL.x_drop));
   float* u = reinterpret_cast<float*>(at(ws, LL.u));
   float* y_r = reinterpret_cast<float*>(at(ws, LL.y_r));

@@ -202,6 +202,32 @@ cudaError_t plan_fused(Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan
 cudaError_t launch_fused(Elem w_elem, const FusedArgs& a, const StreamPlan& plan,
                          cudaStream_t stream);
 
+// Sparse + low rank for one token in one cooperative launch (onetoken.cu,
+// lowrank_kernel): y = sum_k val[k] W[idx[k]] + ((x - sigma(x)) . A_r) . B_r,
+// x fp32 [d_in], sigma(x) the kept entries of x.  Workspace: u (r floats),
+// partials (plan.partial_floats floats) and sync (2 + n_tiles words, zero
+// between calls).  plan->ok is false when the shape does not fit (d_in >
+// 16384, r > 2048, or the grid cannot be resident).
+struct LowrankArgs {
+  const float* x = nullptr;
+  const int32_t* idx = nullptr;
+  const float* val = nullptr;
+  const void* W = nullptr;
+  const void* A_r = nullptr;
+  const void* B_r = nullptr;
+  float* y = nullptr;
+  float* u = nullptr;
+  float* partials = nullptr;
+  unsigned* sync = nullptr;
+  int d_in = 0;
+  int d_out = 0;
+  int K = 0;
+  int r = 0;
+  int* dev_status = nullptr;
+};
+cudaError_t plan_lowrank(Elem w_elem, int d_in, int d_out, int K, int r, StreamPlan* plan);
+cudaError_t launch_lowrank(Elem w_elem, const LowrankArgs& a, const StreamPlan& plan, cudaStream_t stream);
+
 // W_rot = Qt . W with Qt = Q^T given row-major.
 cudaError_t launch_prepare(const void* Q, const void* W, void* W_rot, int d_in, int d_out,
                            Elem elem, cudaStream_t stream);

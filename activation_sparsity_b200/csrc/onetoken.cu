@@ -1548,9 +1548,220 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
                          p.sync + kFusedSyncWords + (gen & 1u) * kFusedMaxTiles + tile, p.y);
 }
 
+// ================================================================ sparse + low rank, one token
+//
+// R-Sparse report, 研究流程与方法 / R-Sparse框架设计 (hybrid computation): the
+// entries a selection drops go through rank-r factors of the weight instead
+// of being discarded, y = sum_{k} val[k] W[idx[k]] + ((x - sigma(x)) . A_r) . B_r.
+// One cooperative launch of n_tiles * C column-tile CTAs and U factor CTAs,
+// all resident at once:
+//   * factor CTA q stages x in shared memory with the kept entries zeroed
+//     (the dropped part) and computes u[j] = sum_i x_drop[i] A_r[i][j] for its
+//     32 columns j of A_r, loading only the rows with a nonzero coefficient;
+//     it writes its slice of u to the workspace and arrives on a counter;
+//   * column-tile CTA (tile, rank) streams positions [K rank / C,
+//     K (rank + 1) / C) of the kept list of W for its columns, then waits for
+//     every factor CTA, streams rows [r rank / C, r (rank + 1) / C) of B_r
+//     with the coefficients u into the same partial sums, and the last CTA of
+//     the tile adds the C partials in rank order (y = y_s + y_r).
+// Counter words in the workspace, all zero between calls: [0] factor CTAs
+// done, [1] column-tile CTAs that have seen them (the last resets both),
+// [2 + t] column tile t's CTAs done (its last CTA resets it).  A wait that
+// runs out reports LAROSA_DEV_TIMEOUT; the workspace must then be zeroed.
+
+struct LRParams {
+  const float* x;       // [d] the vector the selection was made on (fp32)
+  const int32_t* idx;   // [K] kept list
+  const float* val;     // [K]
+  const void* W;        // [d x d_out]
+  const void* A_r;      // [d x r]
+  const void* B_r;      // [r x d_out]
+  float* y;             // [d_out]
+  float* u;             // [r] workspace
+  float* partials;      // [n_tiles x C x col_tile] workspace
+  unsigned* sync;       // [2 + n_tiles] counters, workspace
+  int d;
+  int d_out;
+  int K;
+  int r;
+  int col_tile;
+  int tpr;
+  int list_cap;         // entries a column-tile CTA lists: max(ceil(K / C), ceil(r / C))
+  int n_tiles;
+  int u_ctas;           // factor CTAs, kLRUCols columns of A_r each
+  int* dev_status;
+  unsigned long long wait_ns;
+};
+
+constexpr int kLRUCols = 32;    // columns of A_r per factor CTA (64 bytes of bf16 per row)
+constexpr int kLRMaxD = 16384;  // x_drop staged in shared memory
+
+struct LRLayout {
+  size_t xs, red, rows, vals, total;
+};
+
+// Region A: the factor CTA's x_drop, or the column-tile CTA's row-group
+// partials (red); then the kept / factor-row lists.
+__host__ __device__ inline LRLayout lrlayout(int d, int list_cap, int col_tile, int cpt) {
+  LRLayout L{};
+  const size_t xs_bytes = al16((size_t)d * 4);
+  const size_t red_tile = al16((size_t)(kT / (col_tile / cpt)) * col_tile * 4);
+  const size_t red_u = al16((size_t)(kT / (kLRUCols / cpt)) * kLRUCols * 4);
+  L.xs = 0;
+  L.red = 0;
+  size_t o = xs_bytes;
+  o = o > red_tile ? o : red_tile;
+  o = o > xs_bytes + red_u ? o : xs_bytes + red_u;  // the factor CTA's partials follow its x_drop
+  L.rows = o;  o = al16(o + (size_t)list_cap * 4);
+  L.vals = o;  o = al16(o + (size_t)list_cap * 4);
+  L.total = o;
+  return L;
+}
+
+template <typename Tw, int C>
+__global__ void __launch_bounds__(kT, 2) lowrank_kernel(const LRParams p) {
+  constexpr int CPT = 16 / sizeof(Tw);
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ uint32_t s_word[2];
+  const LRLayout L = lrlayout(p.d, p.list_cap, p.col_tile, CPT);
+  int32_t* lrows = reinterpret_cast<int32_t*>(smem_raw + L.rows);
+  float* lvals = reinterpret_cast<float*>(smem_raw + L.vals);
+  const int tid = threadIdx.x;
+  const int n_tile_ctas = p.n_tiles * C;
+  const int cta = blockIdx.x;
+  const int d = p.d, K = p.K;
+  pdl_wait();
+  pdl_launch_dependents();
+
+  if (cta >= n_tile_ctas) {
+    // ---- factor CTA q: u[c0u .. c0u + wcu) = x_drop . A_r[:, c0u ..]
+    float* xs = reinterpret_cast<float*>(smem_raw + L.xs);
+    float* red = reinterpret_cast<float*>(smem_raw + al16((size_t)d * 4));
+    const int q = cta - n_tile_ctas;
+    const int c0u = q * kLRUCols;
+    const int wcu = min(kLRUCols, p.r - c0u);
+    for (int i = tid; i < d; i += kT) xs[i] = __ldg(p.x + i);
+    __syncthreads();
+    bool bad = false;
+    for (int k = tid; k < K; k += kT) {
+      const int i = __ldg(p.idx + k);
+      if (static_cast<unsigned>(i) < static_cast<unsigned>(d))
+        xs[i] = 0.f;  // kept: not part of the dropped vector
+      else
+        bad = true;
+    }
+    if (__syncthreads_or(bad) && tid == 0 && q == 0) report(p.dev_status, LAROSA_DEV_INDEX);
+    // thread (g, col) takes rows g, g + ng, ... of the slice, loading only
+    // the rows whose coefficient is nonzero
+    const int tpr = kLRUCols / CPT;
+    const int ng = kT / tpr;
+    const int g = tid / tpr;
+    const int col = (tid - g * tpr) * CPT;
+    float acc[CPT];
+#pragma unroll
+    for (int v = 0; v < CPT; ++v) acc[v] = 0.f;
+    if (col < wcu) {
+      const unsigned char* base = static_cast<const unsigned char*>(p.A_r) + ((size_t)c0u + col) * sizeof(Tw);
+      const size_t pitch = (size_t)p.r * sizeof(Tw);
+      constexpr int NU = 4;
+      for (int i0 = g; i0 < d; i0 += ng * NU) {
+        uint4 w[NU];
+        float cf[NU];
+#pragma unroll
+        for (int t = 0; t < NU; ++t) {
+          const int i = i0 + t * ng;
+          cf[t] = i < d ? xs[i] : 0.f;
+          w[t] = cf[t] != 0.f ? ld_stream(base + (size_t)i * pitch) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int t = 0; t < NU; ++t) {
+          if constexpr (CPT == 8) {
+            float wv[8];
+            Vec8<__nv_bfloat16>::cvt(&w[t], wv);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) acc[v] = fmaf(cf[t], wv[v], acc[v]);
+          } else {
+            acc[0] = fmaf(cf[t], __uint_as_float(w[t].x), acc[0]);
+            acc[1] = fmaf(cf[t], __uint_as_float(w[t].y), acc[1]);
+            acc[2] = fmaf(cf[t], __uint_as_float(w[t].z), acc[2]);
+            acc[3] = fmaf(cf[t], __uint_as_float(w[t].w), acc[3]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < CPT; ++v) red[g * kLRUCols + col + v] = acc[v];
+    __syncthreads();
+    for (int e = tid; e < wcu; e += kT) {
+      float s = 0.f;
+      for (int gg = 0; gg < ng; ++gg) s += red[gg * kLRUCols + e];  // row groups in order
+      __stcg(p.u + c0u + e, s);
+    }
+    __syncthreads();  // this CTA's slice of u is written
+    if (tid == 0) atomic_add_release_gpu(p.sync, 1u);
+    return;
+  }
+
+  // ---- column-tile CTA
+  const int tile = cta / C, rank = cta - tile * C;
+  const int c0 = tile * p.col_tile;
+  const int wc = min(p.col_tile, p.d_out - c0);
+  float acc[CPT];
+#pragma unroll
+  for (int v = 0; v < CPT; ++v) acc[v] = 0.f;
+  {
+    // y_s: positions [p0, p1) of the kept list
+    const int p0 = (int)((long long)K * rank / C), p1 = (int)((long long)K * (rank + 1) / C);
+    bool bad = false;
+    for (int j = tid; j < p1 - p0; j += kT) {
+      const int row = __ldg(p.idx + p0 + j);
+      const bool ok = static_cast<unsigned>(row) < static_cast<unsigned>(d);
+      bad |= !ok;
+      lrows[j] = ok ? row : 0;
+      lvals[j] = ok ? __ldg(p.val + p0 + j) : 0.f;
+    }
+    if (__syncthreads_or(bad) && tid == 0) report(p.dev_status, LAROSA_DEV_INDEX);
+    accumulate_rows<Tw, kFusedU>(p.W, p.d_out, c0, wc, p.tpr, lrows, lvals, 0, p1 - p0, acc);
+  }
+  // every factor CTA has written its slice of u
+  if (tid == 0) {
+    const bool ok = wait_word(p.sync, static_cast<unsigned>(p.u_ctas), p.wait_ns);
+    if (!ok) {
+      report(p.dev_status, LAROSA_DEV_TIMEOUT);
+    } else if (atomicAdd(p.sync + 1, 1u) == static_cast<unsigned>(n_tile_ctas - 1)) {
+      // the last column-tile CTA to see the factor CTAs: both counters back to zero
+      p.sync[0] = 0u;
+      p.sync[1] = 0u;
+    }
+    s_word[0] = ok;
+  }
+  __syncthreads();  // this CTA's kept rows are consumed: the lists are free
+  if (s_word[0] != 0u) {
+    // y_r: rows [q0, q1) of B_r, coefficients u
+    const int q0 = (int)((long long)p.r * rank / C), q1 = (int)((long long)p.r * (rank + 1) / C);
+    for (int j = tid; j < q1 - q0; j += kT) {
+      lrows[j] = q0 + j;
+      lvals[j] = __ldcg(p.u + q0 + j);
+    }
+    __syncthreads();
+    accumulate_rows<Tw, kFusedU>(p.B_r, p.d_out, c0, wc, p.tpr, lrows, lvals, 0, q1 - q0, acc);
+  }
+  float* red = reinterpret_cast<float*>(smem_raw + L.red);
+  reduce_tile_last<Tw, C>(rank, c0, wc, p.col_tile, p.tpr, acc, red, p.partials + (size_t)tile * C * p.col_tile,
+                          p.sync + 2 + tile, p.y);
+  // reduce_tile_last returns in every CTA; the counter of the tile now holds
+  // C, and only after its last CTA has read it: reset by that CTA (which
+  // saw C - 1 and is the only one still running this tile)
+  if (tid == 0 && ld_acquire_gpu(p.sync + 2 + tile) == static_cast<unsigned>(C)) {
+    // every CTA of the tile has arrived; the one that reduced may still be
+    // reading the partials, so only the counter is reset
+    atomicCAS(p.sync + 2 + tile, static_cast<unsigned>(C), 0u);
+  }
+}
+
 struct DevState {
   int sms = 0;
-  bool configured[16] = {};  // kernel slots whose shared-memory ceiling is set
+  bool configured[24] = {};  // kernel slots whose shared-memory ceiling is set
 };
 DevState g_state[64];
 
@@ -1977,6 +2188,107 @@ cudaError_t launch_fused(Elem w_elem, const FusedArgs& a, const StreamPlan& pl,
   // every CTA must be resident at once: the gather CTAs wait on the selector.
   // As a programmatic dependent the launch may begin before the previous
   // kernel on the stream ends (the kernel waits before reading its inputs).
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  void* args[] = {&p};
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+namespace {
+
+template <int C>
+void* lowrank_fn_c(Elem w) {
+  return w == Elem::BF16 ? reinterpret_cast<void*>(&lowrank_kernel<__nv_bfloat16, C>)
+                         : reinterpret_cast<void*>(&lowrank_kernel<float, C>);
+}
+
+void* lowrank_fn(Elem w, int C) { return C == 8 ? lowrank_fn_c<8>(w) : lowrank_fn_c<4>(w); }
+
+}  // namespace
+
+cudaError_t plan_lowrank(Elem w_elem, int d_in, int d_out, int K, int r, StreamPlan* plan) {
+  DevState* ds = nullptr;
+  cudaError_t e = dev_state(&ds);
+  if (e != cudaSuccess) return e;
+  StreamPlan best;
+  *plan = best;
+  const int u_ctas = (r + kLRUCols - 1) / kLRUCols;
+  if (d_in < 1 || d_in > kLRMaxD || K < 0 || K > d_in || r < 1 || u_ctas > 64) return cudaSuccess;
+  const int cpt = w_elem == Elem::BF16 ? 8 : 4;
+  long long best_ctas = -1;
+  for (int C : {8, 4}) {
+    void* fn = lowrank_fn(w_elem, C);
+    const int list_cap = std::max((K + C - 1) / C, (r + C - 1) / C);
+    const int wc_max = kT * cpt;
+    const size_t smem_probe = lrlayout(d_in, list_cap, wc_max, cpt).total;
+    if (smem_probe > (size_t)kFusedSmemCeiling) continue;
+    e = configure(ds, 12 + 4 + (w_elem == Elem::BF16 ? 1 : 0) * 2 + (C == 8 ? 1 : 0), fn, kFusedSmemCeiling);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kT, smem_probe);
+    if (e != cudaSuccess) return e;
+    const int tiles = std::min((ds->sms * per_sm - u_ctas) / C, kFusedMaxTiles);  // every CTA resident
+    if (tiles < 1) continue;
+    int wc = (d_out + tiles - 1) / tiles;
+    wc = std::max(wc, std::min(64, d_out));
+    wc = (wc + cpt - 1) / cpt * cpt;
+    wc = std::min(wc, wc_max);
+    const int n_tiles = (d_out + wc - 1) / wc;
+    if (n_tiles > tiles) continue;
+    const long long ctas = (long long)n_tiles * C;
+    if (ctas > best_ctas) {
+      best_ctas = ctas;
+      best.ok = true;
+      best.cluster = C;
+      best.n_tiles = n_tiles;
+      best.col_tile = wc;
+      best.tpr = wc / cpt;
+      best.list_cap = list_cap;
+      best.smem = lrlayout(d_in, list_cap, wc, cpt).total;
+      best.smem_alloc = smem_probe;
+      best.partial_floats = (size_t)n_tiles * C * wc;
+    }
+  }
+  *plan = best;
+  return cudaSuccess;
+}
+
+cudaError_t launch_lowrank(Elem w_elem, const LowrankArgs& a, const StreamPlan& pl, cudaStream_t stream) {
+  if (!pl.ok || (pl.cluster != 4 && pl.cluster != 8) || pl.n_tiles > kFusedMaxTiles) return cudaErrorInvalidValue;
+  void* fn = lowrank_fn(w_elem, pl.cluster);
+  LRParams p;
+  p.x = a.x;
+  p.idx = a.idx;
+  p.val = a.val;
+  p.W = a.W;
+  p.A_r = a.A_r;
+  p.B_r = a.B_r;
+  p.y = a.y;
+  p.u = a.u;
+  p.partials = a.partials;
+  p.sync = a.sync;
+  p.d = a.d_in;
+  p.d_out = a.d_out;
+  p.K = a.K;
+  p.r = a.r;
+  p.col_tile = pl.col_tile;
+  p.tpr = pl.tpr;
+  p.list_cap = pl.list_cap;
+  p.n_tiles = pl.n_tiles;
+  p.u_ctas = (a.r + kLRUCols - 1) / kLRUCols;
+  p.dev_status = a.dev_status;
+  p.wait_ns = wait_limit_ns();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pl.n_tiles * pl.cluster + p.u_ctas, 1, 1);
+  cfg.blockDim = dim3(kT, 1, 1);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  // every CTA must be resident at once: the column-tile CTAs wait on the factor CTAs
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;

@@ -308,6 +308,13 @@ def test_folded_rotation_path(L, d_prev, d, d_out):
     (torch.bfloat16, 16, 512, 256, 64, 40),
     (torch.bfloat16, 1, 4096, 4096, 256, 40),
     (torch.bfloat16, 2, 200, 24, 16, 0),
+    # one token, one launch: every entry dropped, none dropped, a rank that is
+    # not a multiple of the factor CTAs' 32 columns, the down projection's width
+    (torch.bfloat16, 1, 1024, 1032, 40, 100),
+    (torch.bfloat16, 1, 1024, 1032, 40, 0),
+    (torch.float32, 1, 1000, 264, 72, 50),
+    (torch.bfloat16, 1, 11008, 4096, 256, 40),
+    (torch.bfloat16, 1, 4096, 12288, 8, 40),
 ])
 def test_sparse_lowrank_linear(L, dtype, M, d_in, d_out, r, sparsity):
     """y = y_s + (x - sigma(x)) A_r B_r against the oracle on the same factors."""
@@ -327,3 +334,31 @@ def test_sparse_lowrank_linear(L, dtype, M, d_in, d_out, r, sparsity):
     assert L.larosa_check(st) == 0
     ref = np.stack([oracle.sparse_lowrank_linear(xq[m], f64(W), f64(A), f64(B), idx[m]) for m in range(M)])
     assert rel_inf(f64(y), ref) <= Y_TOL
+
+
+def test_sparse_lowrank_one_launch_repeats_on_one_workspace(L):
+    """The one-token kernel leaves its counters at zero: calls with different
+    kept lists on one workspace each match the oracle, and repeat bit for bit."""
+    d_in, d_out, r = 4096, 4096, 256
+    K = sd.k_for_sparsity(d_in, 40)
+    W = sd.weights(d_in, d_out, 0.02, 1012, torch.bfloat16)
+    A64, B64 = oracle.lowrank_factors(f64(W), r)
+    A, B = torch.from_numpy(A64).to(torch.bfloat16).cuda(), torch.from_numpy(B64).to(torch.bfloat16).cuda()
+    Wd = W.cuda()
+    ws = torch.zeros(L.larosa_lowrank_workspace_bytes(1, d_in, d_out, K, r), dtype=torch.uint8, device="cuda")
+    st = status()
+    first = None
+    for call in range(3):
+        x = sd.activations(1, d_in, 1013 + (call % 2), torch.float32)
+        xq = f64(x)
+        idx, val = oracle.topk(xq, K)
+        y = L.larosa_sparse_lowrank_linear(x.cuda(), torch.from_numpy(idx.reshape(1, K).astype(np.int32)).cuda(),
+                                           torch.from_numpy(val.reshape(1, K).astype(np.float32)).cuda(), Wd,
+                                           A, B, ws=ws, dev_status=st)
+        assert L.larosa_check(st) == 0
+        ref = oracle.sparse_lowrank_linear(xq[0], f64(W), f64(A), f64(B), idx.reshape(K))
+        assert rel_inf(f64(y)[0], ref) <= Y_TOL, call
+        if call == 0:
+            first = y.clone()
+        elif call == 2:
+            assert torch.equal(y, first)  # same inputs as call 0
