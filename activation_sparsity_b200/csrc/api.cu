@@ -346,7 +346,7 @@ int make_lowrank_layout(int M, int d_in, int d_out, int K, int r, LowrankLayout*
     if (ok) {
       LL->one_launch = true;
       LL->lr_sync = take((2 + larosa::kFusedMaxTiles) * 4);
-      LL->lr_u = take((size_t)r * 4);
+      LL->lr_u = take((size_t)larosa::kLowrankMaxFactorCtas * r * 4);
       LL->lr_partials = take(lp * 4);
     }
   }

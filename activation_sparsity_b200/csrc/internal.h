@@ -107,6 +107,8 @@ struct StreamPlan {
   size_t smem = 0;         // dynamic shared memory of a launch
   size_t smem_alloc = 0;   // the size the occupancy was computed for
   size_t partial_floats = 0;  // workspace floats for per-CTA partials (fused kernel)
+  int aux_ctas = 0;        // low-rank kernel: factor CTAs
+  int aux_len = 0;         // low-rank kernel: indices of x per factor CTA at most
 };
 
 struct GatherArgs {
@@ -225,6 +227,9 @@ struct LowrankArgs {
   int r = 0;
   int* dev_status = nullptr;
 };
+// u of the one-launch kernel: the factor CTAs' partials, [aux_ctas x r]
+// floats; at most kLowrankMaxFactorCtas x r.
+constexpr int kLowrankMaxFactorCtas = 64;
 cudaError_t plan_lowrank(Elem w_elem, int d_in, int d_out, int K, int r, StreamPlan* plan);
 cudaError_t launch_lowrank(Elem w_elem, const LowrankArgs& a, const StreamPlan& plan, cudaStream_t stream);
 

@@ -1553,21 +1553,28 @@ __global__ void __launch_bounds__(kT, 2) fused_kernel(const FParams p) {
 // R-Sparse report, 研究流程与方法 / R-Sparse框架设计 (hybrid computation): the
 // entries a selection drops go through rank-r factors of the weight instead
 // of being discarded, y = sum_{k} val[k] W[idx[k]] + ((x - sigma(x)) . A_r) . B_r.
-// One cooperative launch of n_tiles * C column-tile CTAs and U factor CTAs,
+// One cooperative launch of n_tiles * C column-tile CTAs and F factor CTAs,
 // all resident at once:
-//   * factor CTA q stages x in shared memory with the kept entries zeroed
-//     (the dropped part) and computes u[j] = sum_i x_drop[i] A_r[i][j] for its
-//     32 columns j of A_r, loading only the rows with a nonzero coefficient;
-//     it writes its slice of u to the workspace and arrives on a counter;
+//   * factor CTA q takes the indices [d q / F, d (q + 1) / F) of x, zeroes
+//     the kept ones (what is left is its share of the dropped vector), lists
+//     the nonzero entries in index order and streams only those rows of A_r,
+//     every column, into a partial u_q = x_drop[range] . A_r[range]; it writes
+//     u_q to the workspace and arrives on a counter.  F is chosen so that a
+//     factor CTA has about two batches of row loads, which keeps u off the
+//     critical path;
 //   * column-tile CTA (tile, rank) streams positions [K rank / C,
-//     K (rank + 1) / C) of the kept list of W for its columns, then waits for
-//     every factor CTA, streams rows [r rank / C, r (rank + 1) / C) of B_r
-//     with the coefficients u into the same partial sums, and the last CTA of
-//     the tile adds the C partials in rank order (y = y_s + y_r).
-// Counter words in the workspace, all zero between calls: [0] factor CTAs
-// done, [1] column-tile CTAs that have seen them (the last resets both),
-// [2 + t] column tile t's CTAs done (its last CTA resets it).  A wait that
-// runs out reports LAROSA_DEV_TIMEOUT; the workspace must then be zeroed.
+//     K (rank + 1) / C) of the kept list of W for its columns, waits for
+//     every factor CTA, adds the F partials of its entries [r rank / C,
+//     r (rank + 1) / C) of u in factor order, streams those rows of B_r with
+//     them as coefficients into the same partial sums, and the last CTA of
+//     the tile adds the C partials in rank order (y = y_s + y_r).  (Asking
+//     for the B_r rows to be brought into L2 before the kept rows was
+//     measured 1.6 % slower: the prefetches queue ahead of the kept rows.)
+// Every sum has a fixed order, so results repeat bit for bit.  Counter words
+// in the workspace, all zero between calls: [0] factor CTAs done, [1]
+// column-tile CTAs that have seen them (the last resets both), [2 + t]
+// column tile t's CTAs done (its last CTA resets it).  A wait that runs out
+// reports LAROSA_DEV_TIMEOUT; the workspace must then be zeroed.
 
 struct LRParams {
   const float* x;       // [d] the vector the selection was made on (fp32)
@@ -1577,7 +1584,7 @@ struct LRParams {
   const void* A_r;      // [d x r]
   const void* B_r;      // [r x d_out]
   float* y;             // [d_out]
-  float* u;             // [r] workspace
+  float* u;             // [F x r] workspace: the factor CTAs' partials of u
   float* partials;      // [n_tiles x C x col_tile] workspace
   unsigned* sync;       // [2 + n_tiles] counters, workspace
   int d;
@@ -1588,34 +1595,50 @@ struct LRParams {
   int tpr;
   int list_cap;         // entries a column-tile CTA lists: max(ceil(K / C), ceil(r / C))
   int n_tiles;
-  int u_ctas;           // factor CTAs, kLRUCols columns of A_r each
+  int f_ctas;           // factor CTAs F
+  int f_len;            // indices of x a factor CTA covers at most: ceil(d / F)
   int* dev_status;
   unsigned long long wait_ns;
 };
 
-constexpr int kLRUCols = 32;    // columns of A_r per factor CTA (64 bytes of bf16 per row)
-constexpr int kLRMaxD = 16384;  // x_drop staged in shared memory
+constexpr int kLRMaxF = kLowrankMaxFactorCtas;  // factor CTAs at most
+constexpr int kLRMaxRank = 2048;   // r: one A_r row per at most kT / 2 threads
+constexpr int kLRMaxLen = 4096;    // indices of x per factor CTA at most (shared memory)
+constexpr int kLRMaxD = kLRMaxF * kLRMaxLen;
 
 struct LRLayout {
-  size_t xs, red, rows, vals, total;
+  size_t keys, red, rows, vals, total;
 };
 
-// Region A: the factor CTA's x_drop, or the column-tile CTA's row-group
-// partials (red); then the kept / factor-row lists.
-__host__ __device__ inline LRLayout lrlayout(int d, int list_cap, int col_tile, int cpt) {
+// Column-tile CTA: its row-group partials (red), then the kept / B_r row
+// lists.  The partials' space also serves to add the factor partials of u.
+__host__ __device__ inline LRLayout lr_tile_layout(int list_cap, int col_tile, int cpt) {
   LRLayout L{};
-  const size_t xs_bytes = al16((size_t)d * 4);
-  const size_t red_tile = al16((size_t)(kT / (col_tile / cpt)) * col_tile * 4);
-  const size_t red_u = al16((size_t)(kT / (kLRUCols / cpt)) * kLRUCols * 4);
-  L.xs = 0;
+  const size_t red = al16((size_t)(kT / (col_tile / cpt)) * col_tile * 4);
+  L.keys = 0;
   L.red = 0;
-  size_t o = xs_bytes;
-  o = o > red_tile ? o : red_tile;
-  o = o > xs_bytes + red_u ? o : xs_bytes + red_u;  // the factor CTA's partials follow its x_drop
-  L.rows = o;  o = al16(o + (size_t)list_cap * 4);
-  L.vals = o;  o = al16(o + (size_t)list_cap * 4);
-  L.total = o;
+  L.rows = red;
+  L.vals = al16(L.rows + (size_t)list_cap * 4);
+  L.total = al16(L.vals + (size_t)list_cap * 4);
   return L;
+}
+
+// Factor CTA: the keys of its range of x, the row-group partials of u, its
+// list of dropped rows.
+__host__ __device__ inline LRLayout lr_factor_layout(int len, int cpt) {
+  LRLayout L{};
+  L.keys = 0;
+  L.red = al16((size_t)len * 4);
+  L.rows = al16(L.red + (size_t)kT * cpt * 4);
+  L.vals = al16(L.rows + (size_t)len * 4);
+  L.total = al16(L.vals + (size_t)len * 4);
+  return L;
+}
+
+// Floats of the column-tile CTA's partials space (used to add the factor
+// partials of u, F per entry).
+__host__ __device__ inline int lr_red_floats(int col_tile, int cpt) {
+  return (kT / (col_tile / cpt)) * col_tile;
 }
 
 template <typename Tw, int C>
@@ -1623,9 +1646,7 @@ __global__ void __launch_bounds__(kT, 2) lowrank_kernel(const LRParams p) {
   constexpr int CPT = 16 / sizeof(Tw);
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __shared__ uint32_t s_word[2];
-  const LRLayout L = lrlayout(p.d, p.list_cap, p.col_tile, CPT);
-  int32_t* lrows = reinterpret_cast<int32_t*>(smem_raw + L.rows);
-  float* lvals = reinterpret_cast<float*>(smem_raw + L.vals);
+  __shared__ uint32_t s_warp_sums[32];
   const int tid = threadIdx.x;
   const int n_tile_ctas = p.n_tiles * C;
   const int cta = blockIdx.x;
@@ -1634,78 +1655,63 @@ __global__ void __launch_bounds__(kT, 2) lowrank_kernel(const LRParams p) {
   pdl_launch_dependents();
 
   if (cta >= n_tile_ctas) {
-    // ---- factor CTA q: u[c0u .. c0u + wcu) = x_drop . A_r[:, c0u ..]
-    float* xs = reinterpret_cast<float*>(smem_raw + L.xs);
-    float* red = reinterpret_cast<float*>(smem_raw + al16((size_t)d * 4));
+    // ---- factor CTA q: u_q = x_drop[i_lo, i_hi) . A_r[i_lo, i_hi)
+    const LRLayout L = lr_factor_layout(p.f_len, CPT);
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + L.keys);
+    float* red = reinterpret_cast<float*>(smem_raw + L.red);
+    int32_t* frows = reinterpret_cast<int32_t*>(smem_raw + L.rows);
+    float* fvals = reinterpret_cast<float*>(smem_raw + L.vals);
     const int q = cta - n_tile_ctas;
-    const int c0u = q * kLRUCols;
-    const int wcu = min(kLRUCols, p.r - c0u);
-    for (int i = tid; i < d; i += kT) xs[i] = __ldg(p.x + i);
+    const int i_lo = (int)((long long)d * q / p.f_ctas), i_hi = (int)((long long)d * (q + 1) / p.f_ctas);
+    const int n = i_hi - i_lo;
+    for (int i = tid; i < n; i += kT) keys[i] = __float_as_uint(__ldg(p.x + i_lo + i));
     __syncthreads();
     bool bad = false;
     for (int k = tid; k < K; k += kT) {
       const int i = __ldg(p.idx + k);
-      if (static_cast<unsigned>(i) < static_cast<unsigned>(d))
-        xs[i] = 0.f;  // kept: not part of the dropped vector
-      else
+      if (static_cast<unsigned>(i) >= static_cast<unsigned>(d))
         bad = true;
+      else if (i >= i_lo && i < i_hi)
+        keys[i - i_lo] = 0u;  // kept: not part of the dropped vector
     }
     if (__syncthreads_or(bad) && tid == 0 && q == 0) report(p.dev_status, LAROSA_DEV_INDEX);
-    // thread (g, col) takes rows g, g + ng, ... of the slice, loading only
-    // the rows whose coefficient is nonzero
-    const int tpr = kLRUCols / CPT;
-    const int ng = kT / tpr;
-    const int g = tid / tpr;
-    const int col = (tid - g * tpr) * CPT;
+    // the dropped entries with a nonzero value, in index order
+    const int nd = compact_range(
+        keys, n, i_lo, [](uint32_t k, int) { return k != 0u; }, frows, fvals, 0, s_warp_sums);
+    __syncthreads();
+    const int tpr = p.r / CPT;  // r is a multiple of CPT
     float acc[CPT];
 #pragma unroll
     for (int v = 0; v < CPT; ++v) acc[v] = 0.f;
-    if (col < wcu) {
-      const unsigned char* base = static_cast<const unsigned char*>(p.A_r) + ((size_t)c0u + col) * sizeof(Tw);
-      const size_t pitch = (size_t)p.r * sizeof(Tw);
-      constexpr int NU = 4;
-      for (int i0 = g; i0 < d; i0 += ng * NU) {
-        uint4 w[NU];
-        float cf[NU];
+    accumulate_rows<Tw, kFusedU>(p.A_r, p.r, 0, p.r, tpr, frows, fvals, 0, nd, acc);
+    const int ng = kT / tpr;
+    const int g = tid / tpr;
+    const int col = (tid - g * tpr) * CPT;
+    if (g < ng) {
 #pragma unroll
-        for (int t = 0; t < NU; ++t) {
-          const int i = i0 + t * ng;
-          cf[t] = i < d ? xs[i] : 0.f;
-          w[t] = cf[t] != 0.f ? ld_stream(base + (size_t)i * pitch) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int t = 0; t < NU; ++t) {
-          if constexpr (CPT == 8) {
-            float wv[8];
-            Vec8<__nv_bfloat16>::cvt(&w[t], wv);
-#pragma unroll
-            for (int v = 0; v < 8; ++v) acc[v] = fmaf(cf[t], wv[v], acc[v]);
-          } else {
-            acc[0] = fmaf(cf[t], __uint_as_float(w[t].x), acc[0]);
-            acc[1] = fmaf(cf[t], __uint_as_float(w[t].y), acc[1]);
-            acc[2] = fmaf(cf[t], __uint_as_float(w[t].z), acc[2]);
-            acc[3] = fmaf(cf[t], __uint_as_float(w[t].w), acc[3]);
-          }
-        }
-      }
+      for (int v = 0; v < CPT; ++v) red[g * p.r + col + v] = acc[v];
     }
-#pragma unroll
-    for (int v = 0; v < CPT; ++v) red[g * kLRUCols + col + v] = acc[v];
     __syncthreads();
-    for (int e = tid; e < wcu; e += kT) {
+    float* uq = p.u + (size_t)q * p.r;
+    for (int e = tid; e < p.r; e += kT) {
       float s = 0.f;
-      for (int gg = 0; gg < ng; ++gg) s += red[gg * kLRUCols + e];  // row groups in order
-      __stcg(p.u + c0u + e, s);
+      for (int gg = 0; gg < ng; ++gg) s += red[gg * p.r + e];  // row groups in order
+      __stcg(uq + e, s);
     }
-    __syncthreads();  // this CTA's slice of u is written
+    __syncthreads();  // this CTA's partial of u is written
     if (tid == 0) atomic_add_release_gpu(p.sync, 1u);
     return;
   }
 
   // ---- column-tile CTA
+  const LRLayout L = lr_tile_layout(p.list_cap, p.col_tile, CPT);
+  int32_t* lrows = reinterpret_cast<int32_t*>(smem_raw + L.rows);
+  float* lvals = reinterpret_cast<float*>(smem_raw + L.vals);
+  float* red = reinterpret_cast<float*>(smem_raw + L.red);
   const int tile = cta / C, rank = cta - tile * C;
   const int c0 = tile * p.col_tile;
   const int wc = min(p.col_tile, p.d_out - c0);
+  const int q0 = (int)((long long)p.r * rank / C), q1 = (int)((long long)p.r * (rank + 1) / C);
   float acc[CPT];
 #pragma unroll
   for (int v = 0; v < CPT; ++v) acc[v] = 0.f;
@@ -1723,9 +1729,9 @@ __global__ void __launch_bounds__(kT, 2) lowrank_kernel(const LRParams p) {
     if (__syncthreads_or(bad) && tid == 0) report(p.dev_status, LAROSA_DEV_INDEX);
     accumulate_rows<Tw, kFusedU>(p.W, p.d_out, c0, wc, p.tpr, lrows, lvals, 0, p1 - p0, acc);
   }
-  // every factor CTA has written its slice of u
+  // every factor CTA has written its partial of u
   if (tid == 0) {
-    const bool ok = wait_word(p.sync, static_cast<unsigned>(p.u_ctas), p.wait_ns);
+    const bool ok = wait_word(p.sync, static_cast<unsigned>(p.f_ctas), p.wait_ns);
     if (!ok) {
       report(p.dev_status, LAROSA_DEV_TIMEOUT);
     } else if (atomicAdd(p.sync + 1, 1u) == static_cast<unsigned>(n_tile_ctas - 1)) {
@@ -1737,16 +1743,36 @@ __global__ void __launch_bounds__(kT, 2) lowrank_kernel(const LRParams p) {
   }
   __syncthreads();  // this CTA's kept rows are consumed: the lists are free
   if (s_word[0] != 0u) {
-    // y_r: rows [q0, q1) of B_r, coefficients u
-    const int q0 = (int)((long long)p.r * rank / C), q1 = (int)((long long)p.r * (rank + 1) / C);
-    for (int j = tid; j < q1 - q0; j += kT) {
-      lrows[j] = q0 + j;
-      lvals[j] = __ldcg(p.u + q0 + j);
+    // u[q0, q1): the F partials of each entry, added in factor order, a
+    // chunk of entries at a time through the partials space
+    const int F = p.f_ctas;
+    const int chunk = max(1, lr_red_floats(p.col_tile, CPT) / F);
+    for (int j0 = q0; j0 < q1; j0 += chunk) {
+      const int m = min(chunk, q1 - j0);
+      for (int t0 = tid; t0 < m * F; t0 += 4 * kT) {
+        float v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int t = t0 + k * kT;
+          const int f = t / m;
+          v[k] = t < m * F ? __ldcg(p.u + (size_t)f * p.r + j0 + (t - f * m)) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (t0 + k * kT < m * F) red[t0 + k * kT] = v[k];
+      }
+      __syncthreads();
+      for (int j = tid; j < m; j += kT) {
+        float s = 0.f;
+        for (int f = 0; f < F; ++f) s += red[f * m + j];
+        lrows[j0 - q0 + j] = j0 + j;
+        lvals[j0 - q0 + j] = s;
+      }
+      __syncthreads();
     }
-    __syncthreads();
+    // y_r: rows [q0, q1) of B_r, coefficients u
     accumulate_rows<Tw, kFusedU>(p.B_r, p.d_out, c0, wc, p.tpr, lrows, lvals, 0, q1 - q0, acc);
   }
-  float* red = reinterpret_cast<float*>(smem_raw + L.red);
   reduce_tile_last<Tw, C>(rank, c0, wc, p.col_tile, p.tpr, acc, red, p.partials + (size_t)tile * C * p.col_tile,
                           p.sync + 2 + tile, p.y);
   // reduce_tile_last returns in every CTA; the counter of the tile now holds
@@ -2217,22 +2243,32 @@ cudaError_t plan_lowrank(Elem w_elem, int d_in, int d_out, int K, int r, StreamP
   if (e != cudaSuccess) return e;
   StreamPlan best;
   *plan = best;
-  const int u_ctas = (r + kLRUCols - 1) / kLRUCols;
-  if (d_in < 1 || d_in > kLRMaxD || K < 0 || K > d_in || r < 1 || u_ctas > 64) return cudaSuccess;
   const int cpt = w_elem == Elem::BF16 ? 8 : 4;
+  if (d_in < 1 || d_in > kLRMaxD || K < 0 || K > d_in || r < cpt || r > kLRMaxRank || r % cpt != 0)
+    return cudaSuccess;
+  // factor CTAs: about two batches of A_r row loads each over the dropped
+  // entries, and at most kLRMaxLen indices of x each
+  const int rows_per_batch = (kT / (r / cpt)) * kFusedU;
+  const int dropped = d_in - K;
+  int F = (dropped + 2 * rows_per_batch - 1) / (2 * rows_per_batch);
+  F = std::max(F, (d_in + kLRMaxLen - 1) / kLRMaxLen);
+  F = std::max(1, std::min(F, kLRMaxF));
+  const int f_len = (d_in + F - 1) / F;
+  if (f_len > kLRMaxLen) return cudaSuccess;
+  const size_t f_smem = lr_factor_layout(f_len, cpt).total;
   long long best_ctas = -1;
   for (int C : {8, 4}) {
     void* fn = lowrank_fn(w_elem, C);
     const int list_cap = std::max((K + C - 1) / C, (r + C - 1) / C);
     const int wc_max = kT * cpt;
-    const size_t smem_probe = lrlayout(d_in, list_cap, wc_max, cpt).total;
+    const size_t smem_probe = std::max(lr_tile_layout(list_cap, wc_max, cpt).total, f_smem);
     if (smem_probe > (size_t)kFusedSmemCeiling) continue;
     e = configure(ds, 12 + 4 + (w_elem == Elem::BF16 ? 1 : 0) * 2 + (C == 8 ? 1 : 0), fn, kFusedSmemCeiling);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kT, smem_probe);
     if (e != cudaSuccess) return e;
-    const int tiles = std::min((ds->sms * per_sm - u_ctas) / C, kFusedMaxTiles);  // every CTA resident
+    const int tiles = std::min((ds->sms * per_sm - F) / C, kFusedMaxTiles);  // every CTA resident
     if (tiles < 1) continue;
     int wc = (d_out + tiles - 1) / tiles;
     wc = std::max(wc, std::min(64, d_out));
@@ -2249,7 +2285,9 @@ cudaError_t plan_lowrank(Elem w_elem, int d_in, int d_out, int K, int r, StreamP
       best.col_tile = wc;
       best.tpr = wc / cpt;
       best.list_cap = list_cap;
-      best.smem = lrlayout(d_in, list_cap, wc, cpt).total;
+      best.aux_ctas = F;
+      best.aux_len = f_len;
+      best.smem = std::max(lr_tile_layout(list_cap, wc, cpt).total, f_smem);
       best.smem_alloc = smem_probe;
       best.partial_floats = (size_t)n_tiles * C * wc;
     }
@@ -2259,7 +2297,9 @@ cudaError_t plan_lowrank(Elem w_elem, int d_in, int d_out, int K, int r, StreamP
 }
 
 cudaError_t launch_lowrank(Elem w_elem, const LowrankArgs& a, const StreamPlan& pl, cudaStream_t stream) {
-  if (!pl.ok || (pl.cluster != 4 && pl.cluster != 8) || pl.n_tiles > kFusedMaxTiles) return cudaErrorInvalidValue;
+  if (!pl.ok || (pl.cluster != 4 && pl.cluster != 8) || pl.n_tiles > kFusedMaxTiles || pl.aux_ctas < 1 ||
+      pl.aux_ctas > kLRMaxF)
+    return cudaErrorInvalidValue;
   void* fn = lowrank_fn(w_elem, pl.cluster);
   LRParams p;
   p.x = a.x;
@@ -2280,11 +2320,12 @@ cudaError_t launch_lowrank(Elem w_elem, const LowrankArgs& a, const StreamPlan& 
   p.tpr = pl.tpr;
   p.list_cap = pl.list_cap;
   p.n_tiles = pl.n_tiles;
-  p.u_ctas = (a.r + kLRUCols - 1) / kLRUCols;
+  p.f_ctas = pl.aux_ctas;
+  p.f_len = pl.aux_len;
   p.dev_status = a.dev_status;
   p.wait_ns = wait_limit_ns();
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(pl.n_tiles * pl.cluster + p.u_ctas, 1, 1);
+  cfg.gridDim = dim3(pl.n_tiles * pl.cluster + p.f_ctas, 1, 1);
   cfg.blockDim = dim3(kT, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = stream;

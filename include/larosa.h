@@ -310,11 +310,12 @@ int larosa_rotate_threshold_linear(const void *x, const void *Qt,
  * it, val = x at idx).  W: [d_in x d_out], A_r: [d_in x r], B_r: [r x d_out],
  * all of `dtype` (the factors of an offline SVD W ~ U S V^T: A_r = U_r
  * S_r^1/2, B_r = S_r^1/2 V_r^T); y: [M x d_out] fp32.  d_out and r rows of
- * 16 bytes; x, W, A_r, B_r, y 16-byte aligned.  One token (d_in <= 16384,
- * r <= 2048): one cooperative kernel, in which column-tile CTAs stream the
- * kept rows of W while factor CTAs compute u = dropped . A_r (reading only
- * the dropped rows of A_r), then the column-tile CTAs stream the rows of B_r
- * with the coefficients u into the same sums.  Otherwise: the sparse linear
+ * 16 bytes; x, W, A_r, B_r, y 16-byte aligned.  One token (r <= 2048):
+ * one cooperative kernel, in which column-tile CTAs stream the kept rows of
+ * W while factor CTAs, each over a range of x, compute partials of
+ * u = dropped . A_r (reading only the dropped rows of A_r), then the
+ * column-tile CTAs add the partials of their entries of u and stream the
+ * rows of B_r with those coefficients into the same sums.  Otherwise: the sparse linear
  * on the kept list, the dropped part of x, u = dropped . A_r and
  * y_r = u . B_r by the row-streaming GEMV with fp32 coefficients, and
  * y += y_r.  The workspace must be zero-filled before its first use (the

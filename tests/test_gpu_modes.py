@@ -308,13 +308,20 @@ def test_folded_rotation_path(L, d_prev, d, d_out):
     (torch.bfloat16, 16, 512, 256, 64, 40),
     (torch.bfloat16, 1, 4096, 4096, 256, 40),
     (torch.bfloat16, 2, 200, 24, 16, 0),
-    # one token, one launch: every entry dropped, none dropped, a rank that is
-    # not a multiple of the factor CTAs' 32 columns, the down projection's width
+    # one token, one launch: every entry dropped, none dropped, ranks that are
+    # not powers of two, the down projection's width, a width over 16384 (a
+    # factor CTA covers at most 4096 entries of x), every entry of the down
+    # width dropped (the factor CTAs at their cap of 64), the largest rank of
+    # the one-launch kernel in both weight types
     (torch.bfloat16, 1, 1024, 1032, 40, 100),
     (torch.bfloat16, 1, 1024, 1032, 40, 0),
     (torch.float32, 1, 1000, 264, 72, 50),
     (torch.bfloat16, 1, 11008, 4096, 256, 40),
     (torch.bfloat16, 1, 4096, 12288, 8, 40),
+    (torch.bfloat16, 1, 20000, 264, 64, 40),
+    (torch.bfloat16, 1, 11008, 1024, 256, 100),
+    (torch.bfloat16, 1, 2048, 2048, 2048, 40),
+    (torch.float32, 1, 2048, 2048, 2048, 50),
 ])
 def test_sparse_lowrank_linear(L, dtype, M, d_in, d_out, r, sparsity):
     """y = y_s + (x - sigma(x)) A_r B_r against the oracle on the same factors."""
