@@ -70,7 +70,12 @@ template <int NB>
 struct UCfg<true, NB> {
   static constexpr int kNB = NB;     // 128-column accumulators per CTA: 256 NB contiguous bytes per row
   static constexpr int kKB = 1;      // one 64-row box per stage
-  static constexpr int kStages = NB == 1 ? 5 : 3;  // 5 x 20 KB or 3 x 36 KB: two CTAs per SM
+  // 2 x 20 KB: four CTAs per SM, or 3 x 36 KB: two.  More CTAs issuing
+  // copies beat deeper rings: at 16 tokens on the LLaMA2-7B groups, 128
+  // columns with two stages (4 CTAs per SM) were 5 % faster than 256 columns
+  // with three (2 per SM), 128 with three (3 per SM) 1.5 %, 256 with two
+  // (3 per SM) 1.5 % slower.
+  static constexpr int kStages = NB == 1 ? 2 : 3;
   static constexpr int kN = 2 * kUTokens;          // heads, then tails
 };
 
@@ -430,11 +435,11 @@ bool umma_gemv_applies(int M, int d_in, int d_out) {
   return M >= kUMinTokens && M <= kUTokens && d_in % 8 == 0 && d_out % 8 == 0 && d_in >= kUBox;
 }
 
-// Column tiles of 256 (two accumulators) read each weight row 512 contiguous
-// bytes at a time.  Measured on the LLaMA2-7B groups at 8 and 16 tokens they
-// beat tiles of 128 on every group, the small ones (16 tiles) included, so
-// they are used throughout; 0 would choose per shape by the wave model.
-constexpr int kGemvNB = 2;
+// Column tiles of 128 (one accumulator) with the two-stage ring above, four
+// CTAs per SM: measured on the LLaMA2-7B groups at 2 to 16 tokens they beat
+// tiles of 256 at two CTAs per SM on every batch size; 0 would choose per
+// shape by the wave model.
+constexpr int kGemvNB = 1;
 
 cudaError_t launch_umma_gemv(const void* W, const __nv_bfloat16* hl, float* y, int M, int d_in, int d_out,
                              int* dev_status, cudaStream_t stream) {
