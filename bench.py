@@ -420,7 +420,9 @@ def bench_model_configs(args, torch, L, sd, device, stream, world, graph_of, tim
     * llama2-13b-layer: the fused path with M = 1, 2, 4, 8, 16 tokens per
       call, each token its own Top-K (bytes: Q once plus the union of kept rows);
     * llama2-70b-slice: 8 layers (q|k|v 8192x10240 with GQA, ffn 28672) at 40
-      and 50 %, and the dense GEMV.
+      and 50 %, with the rotation online and folded into the producer (the
+      identity rotation on an input that arrives rotated), and the dense GEMV.
+    The 7B stack also runs the folded path at 40 %.
     Each is timed over a short run (inputs far larger than L2) and freed
     before the next is built.
     """
@@ -454,8 +456,8 @@ def bench_model_configs(args, torch, L, sd, device, stream, world, graph_of, tim
                 "gb_per_token": step_bytes / tokens_per_step / 1e9,
                 "hbm_frac": step_bytes * steps / t_max / 1e9 / peak}
 
-    def fused_bytes(layers, sp):
-        return sum(path_bytes(g, sd.k_for_sparsity(g.d_in, sp))["total"] for gs in layers for g in gs)
+    def fused_bytes(layers, sp, rotate=True):
+        return sum(path_bytes(g, sd.k_for_sparsity(g.d_in, sp), rotate)["total"] for gs in layers for g in gs)
 
     def dense_bytes(layers):
         return sum(g.d_in * g.d_out * 2 + g.d_in * 2 + g.d_out * 4 for gs in layers for g in gs)
@@ -472,15 +474,17 @@ def bench_model_configs(args, torch, L, sd, device, stream, world, graph_of, tim
     presize(ws, layers)
     ys = {g.name: torch.empty((1, g.d_out), dtype=torch.float32, device=device) for g in layers[0]}
 
-    def stack_step(sp, only=None):
+    def stack_step(sp, only=None, folded=False):
+        # folded: the rotation folded into the producer, so the input arrives
+        # rotated and the call runs with the identity rotation (no Q read)
         Ks = {g.name: sd.k_for_sparsity(g.d_in, sp) for g in layers[0]}
 
         def step():
             for gs in layers:
                 for g in gs:
                     if only is None or g.name == only:
-                        L.larosa_rotate_topk_linear(g.x, g.Qt, g.W_rot, Ks[g.name], y=ys[g.name], ws=ws,
-                                                    dev_status=st)
+                        L.larosa_rotate_topk_linear(g.x, None if folded else g.Qt, g.W_rot, Ks[g.name],
+                                                    y=ys[g.name], ws=ws, dev_status=st)
         return step
 
     def dense_stack():
@@ -496,9 +500,13 @@ def bench_model_configs(args, torch, L, sd, device, stream, world, graph_of, tim
         stack["fused"][f"{sp:g}%"] = rate(time_graph(gr, n, args.warmup)[0], n, 1, fused_bytes(layers, sp))
         del gr
     stack["fused_eager_40%"] = rate(time_eager(stack_step(40.0), n), n, 1, fused_bytes(layers, 40.0))
+    gr = graph_of(stack_step(40.0, folded=True))
+    stack["folded_40%"] = rate(time_graph(gr, n, args.warmup)[0], n, 1, fused_bytes(layers, 40.0, rotate=False))
+    del gr
     gr = graph_of(dense_stack)
     stack["dense"] = rate(time_graph(gr, n, args.warmup)[0], n, 1, dense_bytes(layers))
     del gr
+    stack["folded_vs_dense_40%"] = stack["folded_40%"]["tokens_per_s"] / stack["dense"]["tokens_per_s"]
     stack["dense_eager"] = rate(time_eager(dense_stack, n), n, 1, dense_bytes(layers))
     stack["fused_vs_dense_40%"] = stack["fused"]["40%"]["tokens_per_s"] / stack["dense"]["tokens_per_s"]
     us = {}
@@ -548,14 +556,20 @@ def bench_model_configs(args, torch, L, sd, device, stream, world, graph_of, tim
     ws = L.Workspace(device)
     presize(ws, layers)
     ys = {g.name: torch.empty((1, g.d_out), dtype=torch.float32, device=device) for g in layers[0]}
-    slc = {"layers": 8, "fused": {}}
+    slc = {"layers": 8, "fused": {}, "folded": {}}
     for sp in (40.0, 50.0):
         gr = graph_of(stack_step(sp))
         slc["fused"][f"{sp:g}%"] = rate(time_graph(gr, n, args.warmup)[0], n, 1, fused_bytes(layers, sp))
         del gr
+        gr = graph_of(stack_step(sp, folded=True))
+        slc["folded"][f"{sp:g}%"] = rate(time_graph(gr, n, args.warmup)[0], n, 1,
+                                          fused_bytes(layers, sp, rotate=False))
+        del gr
     gr = graph_of(dense_stack)
     slc["dense"] = rate(time_graph(gr, n, args.warmup)[0], n, 1, dense_bytes(layers))
     del gr
+    for sp in ("40%", "50%"):
+        slc[f"folded_vs_dense_{sp}"] = slc["folded"][sp]["tokens_per_s"] / slc["dense"]["tokens_per_s"]
     out["llama2-70b-slice"] = slc
     log("70B slice timed")
     del layers, ws, ys
