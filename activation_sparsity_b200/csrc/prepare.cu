@@ -126,6 +126,10 @@ constexpr uint32_t kPStage = kPABytes + kPBBytes;
 constexpr size_t kPSmem = (size_t)kPStages * kPStage + 1024;
 constexpr int kPTmemCols = 2 * kPN;  // two segment buffers
 constexpr int kPThreads = 192;       // producer, MMA issuer, four epilogue warps
+// Tile order: groups of kPGroup row tiles, row tile fastest inside a group,
+// so that a wave of CTAs shares a few column blocks of W (and row blocks of
+// Qt) through L2 instead of each wave reading all of W once more.
+constexpr int kPGroup = 8;
 
 struct PParams {
   __nv_bfloat16* W_rot;
@@ -145,7 +149,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int j0 = blockIdx.x * kPN, i0 = blockIdx.y * kPM;
+  const int tiles_m = (p.d + kPM - 1) / kPM, tiles_n = (p.n + kPN - 1) / kPN;
+  const int group = static_cast<int>(blockIdx.x) / (kPGroup * tiles_n);
+  const int first_m = group * kPGroup;
+  const int gm = min(tiles_m - first_m, kPGroup);
+  const int in_group = static_cast<int>(blockIdx.x) - group * kPGroup * tiles_n;
+  const int j0 = (in_group / gm) * kPN, i0 = (first_m + in_group % gm) * kPM;
   const int n_it = (p.d + tc::kBox - 1) / tc::kBox;
   const int n_seg = (n_it + kPSeg - 1) / kPSeg;
   constexpr uint32_t kId = tc::idesc(kPN, false, true);
@@ -294,7 +303,7 @@ cudaError_t launch_prep_umma(const void* Qt, const void* W, void* W_rot, int d, 
   }
   PParams p{static_cast<__nv_bfloat16*>(W_rot), d, n, nullptr, wait_limit_ns()};
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((n + kPN - 1) / kPN, (d + kPM - 1) / kPM, 1);
+  cfg.gridDim = dim3(((n + kPN - 1) / kPN) * ((d + kPM - 1) / kPM), 1, 1);
   cfg.blockDim = dim3(kPThreads, 1, 1);
   cfg.dynamicSmemBytes = kPSmem;
   cfg.stream = stream;
