@@ -22,7 +22,10 @@ _EXPORTS = (
     "larosa_workspace_layout", "larosa_workspace_nnz_offset", "larosa_threshold",
     "larosa_rotate_threshold_linear", "larosa_fold_rotation",
     "larosa_sparse_lowrank_linear", "larosa_lowrank_workspace_bytes", "larosa_sparse_linear_noalloc_bytes",
-    "larosa_workspace_sync_offset", "larosa_set_wait_limit_ns", "LAROSA_NOALLOC_SCRATCH_BYTES", "LAROSA_F32", "LAROSA_BF16", "LAROSA_MAX_D", "LAROSA_MAX_M",
+    "larosa_workspace_sync_offset", "larosa_set_wait_limit_ns", "larosa_set_debug", "larosa_set_split_k",
+    "LAROSA_OK", "LAROSA_ERR_NONFINITE", "LAROSA_ERR_TIMEOUT", "LAROSA_ERR_INDEX", "LAROSA_ERR_LIST",
+    "LAROSA_DEV_NONFINITE", "LAROSA_DEV_TIMEOUT", "LAROSA_DEV_INDEX", "LAROSA_DEV_LIST", "LAROSA_MAX_SPLIT_K",
+    "LAROSA_NOALLOC_SCRATCH_BYTES", "LAROSA_F32", "LAROSA_BF16", "LAROSA_MAX_D", "LAROSA_MAX_M",
     "LIB_PATH",
 )
 __all__ = list(_EXPORTS)

@@ -22,6 +22,8 @@
 
 #include <algorithm>
 #include <atomic>
+#include <climits>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -390,7 +392,51 @@ void set_last_error(const char* msg) { snprintf(g_last_error, sizeof(g_last_erro
 std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
 
 unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
+namespace {
+// An integer environment variable, `fallback` when unset or not a number.
+int env_int(const char* name, int fallback) {
+  const char* v = getenv(name);
+  if (v == nullptr || *v == 0) return fallback;
+  char* end = nullptr;
+  const long x = strtol(v, &end, 10);
+  return (end != nullptr && *end == 0 && x >= INT_MIN && x <= INT_MAX) ? static_cast<int>(x) : fallback;
+}
+}  // namespace
+
+// -1 until the first use reads the environment
+std::atomic<int> g_debug{-1};
+std::atomic<int> g_split_k{-1};
+
+bool debug_checks() {
+  if (g_debug.load(std::memory_order_relaxed) < 0) {
+    int unset = -1;
+    g_debug.compare_exchange_strong(unset, env_int("LAROSA_DEBUG", 0) != 0 ? 1 : 0);
+  }
+  return g_debug.load(std::memory_order_relaxed) == 1;
+}
+
+int split_k_override() {
+  if (g_split_k.load(std::memory_order_relaxed) < 0) {
+    int v = env_int("LAROSA_SPLIT_K", 0);
+    if (v < 0 || v > LAROSA_MAX_SPLIT_K) v = 0;
+    int unset = -1;
+    g_split_k.compare_exchange_strong(unset, v);
+  }
+  return g_split_k.load(std::memory_order_relaxed);
+}
 }  // namespace larosa
+
+namespace {
+// With the debug checks on: the kept lists idx/val ([M x K]) checked on the
+// stream (see larosa_set_debug).
+int debug_check_lists(const int32_t* idx, const float* val, int M, int K, int d, bool ascending,
+                      int* dev_status, cudaStream_t s) {
+  if (!larosa::debug_checks()) return LAROSA_OK;
+  const cudaError_t e = larosa::launch_check_lists(idx, val, M, K, d, ascending, dev_status, s);
+  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "list check kernel");
+}
+}  // namespace
 
 extern "C" {
 
@@ -406,6 +452,7 @@ const char* larosa_status_string(int status) {
     case LAROSA_ERR_NONFINITE: return "LAROSA_ERR_NONFINITE: a NaN or Inf reached Top-K";
     case LAROSA_ERR_TIMEOUT: return "LAROSA_ERR_TIMEOUT: a kernel wait exceeded its time limit";
     case LAROSA_ERR_INDEX: return "LAROSA_ERR_INDEX: an index was out of range";
+    case LAROSA_ERR_LIST: return "LAROSA_ERR_LIST: a kept list repeats an index or is out of order";
     default: return "unknown larosa status";
   }
 }
@@ -464,6 +511,22 @@ int larosa_set_wait_limit_ns(uint64_t limit_ns, uint64_t* previous) {
   return LAROSA_OK;
 }
 
+int larosa_set_debug(int on, int* previous) {
+  if (on != 0 && on != 1) return LAROSA_ERR_INVALID_ARG;
+  (void)larosa::debug_checks();  // the environment's setting, if not read yet
+  const int old = larosa::g_debug.exchange(on);
+  if (previous) *previous = old;
+  return LAROSA_OK;
+}
+
+int larosa_set_split_k(int splits, int* previous) {
+  if (splits < 0 || splits > LAROSA_MAX_SPLIT_K) return LAROSA_ERR_INVALID_ARG;
+  (void)larosa::split_k_override();
+  const int old = larosa::g_split_k.exchange(splits);
+  if (previous) *previous = old;
+  return LAROSA_OK;
+}
+
 int larosa_prepare_weights(const void* Qt, const void* W, void* W_rot, int d_in, int d_out,
                            int dtype, larosa_stream_t stream) {
   if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
@@ -501,7 +564,8 @@ int larosa_topk(const float* x_rot, int M, int d, int K, int32_t* idx, float* va
     return LAROSA_ERR_SHAPE;
   cudaError_t e = larosa::launch_topk(x_rot, M, d, K, idx, val, dev_status,
                                       reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "topk kernel");
+  if (e != cudaSuccess) return cuda_fail(e, "topk kernel");
+  return debug_check_lists(idx, val, M, K, d, true, dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int larosa_rotate_topk(const void* x, const void* Qt, float* x_rot, int32_t* idx, float* val, int d,
@@ -530,7 +594,8 @@ int larosa_rotate_topk(const void* x, const void* Qt, float* x_rot, int32_t* idx
   r.K = K;
   r.dev_status = dev_status;
   cudaError_t e = larosa::launch_rotsel(elem_of(dtype), r, reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "rotate-select kernel");
+  if (e != cudaSuccess) return cuda_fail(e, "rotate-select kernel");
+  return debug_check_lists(idx, val, 1, K, d, true, dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int larosa_sparse_linear(const int32_t* idx, const float* val, int M, int K, const void* W_rot,
@@ -547,13 +612,15 @@ int larosa_sparse_linear(const int32_t* idx, const float* val, int M, int K, con
   if (st != LAROSA_OK) return st;
   st = workspace_ok(ws, ws_bytes, L);
   if (st != LAROSA_OK) return st;
+  st = debug_check_lists(idx, val, M, K, d_in, false, dev_status, reinterpret_cast<cudaStream_t>(stream));
+  if (st != LAROSA_OK) return st;
   return run_sparse(idx, val, M, K, W_rot, d_in, d_out, y, dtype, ws, L, dev_status,
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
-int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, int M, int d_in,
-                              int d_out, int K, float* y, void* ws, size_t ws_bytes,
-                              int* dev_status, int dtype, larosa_stream_t stream) {
+static int rotate_topk_linear_impl(const void* x, const void* Qt, const void* W_rot, int M, int d_in,
+                                   int d_out, int K, float* y, void* ws, size_t ws_bytes,
+                                   int* dev_status, int dtype, larosa_stream_t stream) {
   if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
   if (x == nullptr || W_rot == nullptr || y == nullptr) return LAROSA_ERR_INVALID_ARG;
   int st = check_sizes(M, d_in, d_out, K);
@@ -641,8 +708,30 @@ int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, 
   return run_sparse(idx, val, M, K, W_rot, d_in, d_out, y, dtype, ws, L, dev_status, s);
 }
 
-int larosa_topk_linear(const float* x_rot, const void* W_rot, int M, int d_in, int d_out, int K, float* y,
-                       void* ws, size_t ws_bytes, int* dev_status, int dtype, larosa_stream_t stream) {
+// The kept lists a successful call left in the workspace, checked when the
+// debug checks are on.
+static int check_workspace_lists(int M, int d_in, int d_out, int K, void* ws, int* dev_status,
+                                 larosa_stream_t stream) {
+  if (!larosa::debug_checks()) return LAROSA_OK;
+  Layout L;
+  const int st = make_layout(M, d_in, d_out, K, &L);
+  if (st != LAROSA_OK) return st;
+  return debug_check_lists(reinterpret_cast<const int32_t*>(at(ws, L.idx)),
+                           reinterpret_cast<const float*>(at(ws, L.val)), M, K, d_in, true, dev_status,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+int larosa_rotate_topk_linear(const void* x, const void* Qt, const void* W_rot, int M, int d_in,
+                              int d_out, int K, float* y, void* ws, size_t ws_bytes,
+                              int* dev_status, int dtype, larosa_stream_t stream) {
+  const int st = rotate_topk_linear_impl(x, Qt, W_rot, M, d_in, d_out, K, y, ws, ws_bytes, dev_status,
+                                         dtype, stream);
+  return st != LAROSA_OK ? st : check_workspace_lists(M, d_in, d_out, K, ws, dev_status, stream);
+}
+
+static int topk_linear_impl(const float* x_rot, const void* W_rot, int M, int d_in, int d_out, int K,
+                            float* y, void* ws, size_t ws_bytes, int* dev_status, int dtype,
+                            larosa_stream_t stream) {
   if (!valid_dtype(dtype)) return LAROSA_ERR_UNSUPPORTED_DTYPE;
   if (x_rot == nullptr || W_rot == nullptr || y == nullptr) return LAROSA_ERR_INVALID_ARG;
   int st = check_sizes(M, d_in, d_out, K);
@@ -667,6 +756,12 @@ int larosa_topk_linear(const float* x_rot, const void* W_rot, int M, int d_in, i
   cudaError_t e = larosa::launch_topk(x_rot, M, d_in, K, idx, val, dev_status, s);
   if (e != cudaSuccess) return cuda_fail(e, "topk kernel");
   return run_sparse(idx, val, M, K, W_rot, d_in, d_out, y, dtype, ws, L, dev_status, s);
+}
+
+int larosa_topk_linear(const float* x_rot, const void* W_rot, int M, int d_in, int d_out, int K, float* y,
+                       void* ws, size_t ws_bytes, int* dev_status, int dtype, larosa_stream_t stream) {
+  const int st = topk_linear_impl(x_rot, W_rot, M, d_in, d_out, K, y, ws, ws_bytes, dev_status, dtype, stream);
+  return st != LAROSA_OK ? st : check_workspace_lists(M, d_in, d_out, K, ws, dev_status, stream);
 }
 
 int larosa_threshold(const float* x_rot, int M, int d, float t, int32_t* idx, float* val,
@@ -804,6 +899,8 @@ int larosa_sparse_lowrank_linear(const float* x, const int32_t* idx, const float
   if (st != LAROSA_OK) return st;
   if (ws == nullptr || !aligned16(ws) || ws_bytes < LL.total) return LAROSA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = debug_check_lists(idx, val, M, K, d_in, false, dev_status, s);
+  if (st != LAROSA_OK) return st;
   if (M == 1 && LL.one_launch) {
     // one cooperative launch: kept rows of W, x_drop . A_r, then u . B_r
     larosa::StreamPlan pl;
@@ -871,6 +968,7 @@ int larosa_check(const int* dev_status, larosa_stream_t stream, int* flags_out) 
   if (flags & LAROSA_DEV_NONFINITE) return LAROSA_ERR_NONFINITE;
   if (flags & LAROSA_DEV_TIMEOUT) return LAROSA_ERR_TIMEOUT;
   if (flags & LAROSA_DEV_INDEX) return LAROSA_ERR_INDEX;
+  if (flags & LAROSA_DEV_LIST) return LAROSA_ERR_LIST;
   return LAROSA_OK;
 }
 

@@ -63,6 +63,17 @@ cudaError_t launch_topk(const float* x_rot, int M, int d, int K, int32_t* idx, f
 
 // The same dense head/tail coefficient rows from given kept lists (idx/val
 // [M x K], indices distinct within a row): one CTA per token.
+// Debug checks (debug.cu): each of the M rows of idx/val ([M x K]) has
+// distinct indices in [0, d), ascending where `ascending`, and finite values;
+// violations set LAROSA_DEV_INDEX, LAROSA_DEV_LIST or LAROSA_DEV_NONFINITE.
+// Launches nothing when dev_status is NULL or there is no entry.
+cudaError_t launch_check_lists(const int32_t* idx, const float* val, int M, int K, int d, bool ascending,
+                               int* dev_status, cudaStream_t stream);
+// Process-wide settings (api.cu): the debug checks, and the forced split
+// count of the tensor-core kernels of several tokens (0: chosen per shape).
+bool debug_checks();
+int split_k_override();
+
 cudaError_t launch_coef_rows(const int32_t* idx, const float* val, int M, int K, int d, __nv_bfloat16* hl,
                              int* dev_status, cudaStream_t stream);
 

@@ -155,6 +155,11 @@ extern "C" int larosa_sparse_linear_noalloc(const int32_t* idx, const float* val
   ScratchLayout S;
   cudaError_t e = plan_noalloc(w, M, d_in, d_out, K, &sp, &pl, &S);
   if (e != cudaSuccess) return fail_cuda(e, "plan");
+  if (larosa::debug_checks()) {
+    // the caller's lists, as larosa_sparse_linear checks them (larosa_set_debug)
+    e = larosa::launch_check_lists(idx, val, M, K, d_in, false, dev_status, s);
+    if (e != cudaSuccess) return fail_cuda(e, "list check kernel");
+  }
   if (M == 1 && sp.ok) {
     // one token: the cluster gather keeps its partial sums in distributed
     // shared memory and needs no scratch at all

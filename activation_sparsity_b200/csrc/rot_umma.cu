@@ -399,7 +399,8 @@ cudaError_t plan_umma(int n_in, int n_out, int* R, long long* t) {
   const int tiles = (n_out + S::kCols - 1) / S::kCols;
   const int chunks = (n_in + S::kChunk - 1) / S::kChunk;
   const int slots = d.sms * d.per_sm;
-  *R = pick_splits(tiles, chunks, slots);
+  const int forced = split_k_override();  // larosa_set_split_k
+  *R = forced > 0 ? std::min(forced, chunks) : pick_splits(tiles, chunks, slots);
   // bytes of the slowest wave's CTAs, in 64 x 128 bf16 units
   const long long ctas = (long long)tiles * *R;
   *t = (ctas + slots - 1) / slots * ((chunks + *R - 1) / *R) * S::kChunk / kUBox * kNB;

@@ -55,6 +55,8 @@ _SIGNATURES = {
     "larosa_sparse_linear_noalloc_bytes": ([_i, _i, _i, _i, _i], _sz),
     "larosa_workspace_sync_offset": ([_i, _i, _i, _i, _c.POINTER(_sz)], _i),
     "larosa_set_wait_limit_ns": ([_c.c_uint64, _c.POINTER(_c.c_uint64)], _i),
+    "larosa_set_debug": ([_i, _c.POINTER(_i)], _i),
+    "larosa_set_split_k": ([_i, _c.POINTER(_i)], _i),
     "larosa_workspace_bytes": ([_i, _i, _i, _i], _sz),
     "larosa_workspace_layout": ([_i, _i, _i, _i, _c.POINTER(_sz), _c.POINTER(_sz), _c.POINTER(_sz)], _i),
     "larosa_workspace_nnz_offset": ([_i, _i, _i, _i, _c.POINTER(_sz)], _i),
@@ -71,9 +73,12 @@ LAROSA_OK = 0
 LAROSA_ERR_NONFINITE = 7
 LAROSA_ERR_TIMEOUT = 8
 LAROSA_ERR_INDEX = 9
+LAROSA_ERR_LIST = 10
 LAROSA_DEV_NONFINITE = 0x1
 LAROSA_DEV_TIMEOUT = 0x2
 LAROSA_DEV_INDEX = 0x4
+LAROSA_DEV_LIST = 0x8
+LAROSA_MAX_SPLIT_K = 8
 LAROSA_MAX_M = 16
 LAROSA_MAX_D = 32768
 LAROSA_NOALLOC_SCRATCH_BYTES = 2 << 20
@@ -229,6 +234,22 @@ def larosa_set_wait_limit_ns(limit_ns: int) -> int:
     returns the previous limit."""
     prev = ctypes.c_uint64(0)
     _check(_lib.larosa_set_wait_limit_ns(int(limit_ns), ctypes.byref(prev)), "larosa_set_wait_limit_ns")
+    return prev.value
+
+
+def larosa_set_debug(on: bool) -> bool:
+    """Turns the library's debug checks of kept lists on or off for later
+    calls; returns the previous setting (see larosa_set_debug in the header)."""
+    prev = ctypes.c_int(0)
+    _check(_lib.larosa_set_debug(1 if on else 0, ctypes.byref(prev)), "larosa_set_debug")
+    return bool(prev.value)
+
+
+def larosa_set_split_k(splits: int) -> int:
+    """Forces the reduction split of the tensor-core kernels of 2 to 16 tokens
+    (0: chosen per shape); returns the previous setting."""
+    prev = ctypes.c_int(0)
+    _check(_lib.larosa_set_split_k(int(splits), ctypes.byref(prev)), "larosa_set_split_k")
     return prev.value
 
 

@@ -90,7 +90,10 @@ typedef enum {
   LAROSA_ERR_WORKSPACE = 6,        /* ws NULL or smaller than required */
   LAROSA_ERR_NONFINITE = 7,        /* device: NaN/Inf reached Top-K */
   LAROSA_ERR_TIMEOUT = 8,          /* device: a pipeline wait gave up */
-  LAROSA_ERR_INDEX = 9             /* device: an index was out of range */
+  LAROSA_ERR_INDEX = 9,            /* device: an index was out of range */
+  LAROSA_ERR_LIST = 10             /* device (debug checks): a kept list repeats an
+                                      index, or a list the library wrote is not
+                                      in ascending order */
 } larosa_status;
 
 /* Element types of activations and weights. */
@@ -100,6 +103,7 @@ typedef enum { LAROSA_F32 = 0, LAROSA_BF16 = 1 } larosa_dtype;
 #define LAROSA_DEV_NONFINITE 0x1
 #define LAROSA_DEV_TIMEOUT 0x2
 #define LAROSA_DEV_INDEX 0x4
+#define LAROSA_DEV_LIST 0x8 /* only with the debug checks on (larosa_set_debug) */
 
 /* Human-readable name of a larosa_status value (static string, never NULL). */
 const char *larosa_status_string(int status);
@@ -415,8 +419,9 @@ int larosa_workspace_nnz_offset(int M, int d_in, int d_out, int K,
  * Byte offset inside the workspace of the one-token fused call's
  * synchronisation block (M = 1 only; LAROSA_ERR_SHAPE otherwise).  Its
  * 32-bit words: [0] and [1] count the arrivals of even and odd calls, [3]
- * is the number of the last call whose selection was published, [6] and [7]
- * the K-th entry it published; then the per-tile completion counters and
+ * is the number of the last call whose selection was published, [4] and
+ * [5] (one 64-bit word) the K-th entry it published with the call's 16-bit
+ * tag; then the per-tile completion counters and
  * the magnitude histograms of the two call parities.  A caller never needs
  * to touch it (it is zero between calls); it is exposed for diagnosis and
  * for tests of the bounded waits: a call whose arrival counter does not
@@ -442,9 +447,45 @@ int larosa_workspace_sync_offset(int M, int d_in, int d_out, int K,
 int larosa_set_wait_limit_ns(uint64_t limit_ns, uint64_t *previous);
 
 /*
+ * Debug checks (off unless the environment variable LAROSA_DEBUG is set to
+ * a nonzero integer when the library is first used, or this call turns them
+ * on).  While on, every call that takes or writes kept lists also launches
+ * a check of them on the same stream, after (for lists the library writes:
+ * larosa_topk, larosa_rotate_topk, larosa_rotate_topk_linear,
+ * larosa_topk_linear) or before (for the caller's lists: larosa_sparse_linear,
+ * larosa_sparse_linear_noalloc, larosa_sparse_lowrank_linear) the compute:
+ * each row's indices must lie in [0, d_in) (else LAROSA_DEV_INDEX), be
+ * distinct and, where the library wrote them, ascending (else
+ * LAROSA_DEV_LIST), and the values finite (else LAROSA_DEV_NONFINITE).
+ * Results are unchanged; the check costs one small launch per call and
+ * reports only where dev_status is not NULL.  on = 0 turns them off, 1 on;
+ * anything else is LAROSA_ERR_INVALID_ARG.  Process-wide; `previous` (host,
+ * may be NULL) receives the setting in force before the call.
+ */
+int larosa_set_debug(int on, int *previous);
+
+/* Largest split count larosa_set_split_k accepts. */
+#define LAROSA_MAX_SPLIT_K 8
+
+/*
+ * Split of the reduction in the tensor-core kernels of 2 to 16 bf16 tokens
+ * (the rotation, the dense product and the sparse linear): splits = 0 lets
+ * the library choose (a wave model over the SMs, the default, also chosen
+ * by the environment variable LAROSA_SPLIT_K when the library is first
+ * used), 1 ... LAROSA_MAX_SPLIT_K forces that many CTAs per output tile
+ * (fewer where the reduction has fewer 64- or 128-input chunks).  The splits
+ * of a tile form a thread-block cluster and add their partials in rank
+ * order, so a fixed split gives results that repeat bit for bit; different
+ * splits round differently (each within the fp32 summation bound).  Other
+ * values are LAROSA_ERR_INVALID_ARG.  Process-wide, for calls made after
+ * it; `previous` (host, may be NULL) receives the setting before the call.
+ */
+int larosa_set_split_k(int splits, int *previous);
+
+/*
  * Waits for `stream`, reads *dev_status (device pointer) and returns
  * LAROSA_OK when it is zero, else the status of its lowest set bit
- * (NONFINITE, TIMEOUT, INDEX).  If `flags_out` (host) is not NULL it
+ * (NONFINITE, TIMEOUT, INDEX, LIST).  If `flags_out` (host) is not NULL it
  * receives the raw bits.  Does not clear the word.
  */
 int larosa_check(const int *dev_status, larosa_stream_t stream, int *flags_out);

@@ -7,6 +7,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -51,11 +52,45 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_status_strings_and_version(lib):
     lib.larosa_status_string.restype = ctypes.c_char_p
-    for code in range(10):
+    for code in range(11):
         s = lib.larosa_status_string(code).decode()
         assert s.startswith("LAROSA_")
     assert b"unknown" in lib.larosa_status_string(99)
     assert lib.larosa_version() == 100
+
+
+def test_debug_and_split_k_settings_validate_and_restore(lib):
+    """Host-only settings: out-of-range values change nothing; each setter
+    returns the setting it replaced."""
+    prev = ctypes.c_int(-7)
+    assert lib.larosa_set_debug(2, ctypes.byref(prev)) == 1 and prev.value == -7
+    assert lib.larosa_set_split_k(-1, None) == 1
+    assert lib.larosa_set_split_k(9, None) == 1
+    assert lib.larosa_set_split_k(3, ctypes.byref(prev)) == 0
+    first = prev.value
+    assert lib.larosa_set_split_k(first, ctypes.byref(prev)) == 0 and prev.value == 3
+    assert lib.larosa_set_debug(1, ctypes.byref(prev)) == 0
+    was = prev.value
+    assert lib.larosa_set_debug(was, ctypes.byref(prev)) == 0 and prev.value == 1
+
+
+@pytest.mark.parametrize("env,expect", [
+    ({"LAROSA_SPLIT_K": "5", "LAROSA_DEBUG": "1"}, (5, 1)),
+    ({"LAROSA_SPLIT_K": "12", "LAROSA_DEBUG": "0"}, (0, 0)),   # out of range: chosen per shape
+    ({"LAROSA_SPLIT_K": "x", "LAROSA_DEBUG": ""}, (0, 0)),
+])
+def test_settings_read_from_the_environment_at_first_use(lib, env, expect):
+    code = (
+        "import ctypes, sys; lib = ctypes.CDLL(sys.argv[1]); p = ctypes.c_int(-1); q = ctypes.c_int(-1);"
+        "lib.larosa_set_split_k(0, ctypes.byref(p)); lib.larosa_set_debug(0, ctypes.byref(q));"
+        "print(p.value, q.value)")
+    e = dict(os.environ)
+    e.pop("LAROSA_SPLIT_K", None)
+    e.pop("LAROSA_DEBUG", None)
+    e.update(env)
+    out = subprocess.run([sys.executable, "-c", code, lib._name], capture_output=True, text=True, env=e,
+                         check=True).stdout.split()
+    assert (int(out[0]), int(out[1])) == expect
 
 
 P = ctypes.c_void_p
