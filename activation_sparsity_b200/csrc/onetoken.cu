@@ -2043,7 +2043,43 @@ void* gather_fn(Elem w, int C) { return C == 8 ? gather_fn_c<8>(w) : gather_fn_c
 
 }  // namespace
 
-cudaError_t plan_gather(Elem w_elem, int d_out, int K, StreamPlan* plan) {
+// Launch plans already computed, per device, kernel and sizes: a plan costs
+// occupancy queries, and the one-token calls are made once per token.
+struct PlanKey {
+  int dev, kind, elem, a, b, c, r;
+  bool operator==(const PlanKey& o) const {
+    return dev == o.dev && kind == o.kind && elem == o.elem && a == o.a && b == o.b && c == o.c && r == o.r;
+  }
+};
+struct PlanEntry {
+  PlanKey key;
+  StreamPlan plan;
+};
+std::mutex g_plan_mu;
+PlanEntry g_plans[512];
+int g_plan_n = 0, g_plan_next = 0;
+
+template <typename F>
+cudaError_t cached_plan(PlanKey key, StreamPlan* plan, F compute) {
+  cudaError_t e = cudaGetDevice(&key.dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lock(g_plan_mu);
+    for (int i = 0; i < g_plan_n; ++i)
+      if (g_plans[i].key == key) {
+        *plan = g_plans[i].plan;
+        return cudaSuccess;
+      }
+  }
+  e = compute(plan);  // also sets the kernel's attributes on this device
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_plan_mu);
+  PlanEntry& en = g_plans[g_plan_n < 512 ? g_plan_n++ : (g_plan_next++ & 511)];
+  en = PlanEntry{key, *plan};
+  return cudaSuccess;
+}
+
+static cudaError_t plan_gather_uncached(Elem w_elem, int d_out, int K, StreamPlan* plan) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -2138,7 +2174,7 @@ constexpr int kFusedSmemCeiling = kGatherSmemCeiling - 4096;
 
 }  // namespace
 
-cudaError_t plan_fused(Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan) {
+static cudaError_t plan_fused_uncached(Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan) {
   DevState* ds = nullptr;
   cudaError_t e = dev_state(&ds);
   if (e != cudaSuccess) return e;
@@ -2246,7 +2282,7 @@ void* lowrank_fn(Elem w, int C) { return C == 8 ? lowrank_fn_c<8>(w) : lowrank_f
 
 }  // namespace
 
-cudaError_t plan_lowrank(Elem w_elem, int d_in, int d_out, int K, int r, StreamPlan* plan) {
+static cudaError_t plan_lowrank_uncached(Elem w_elem, int d_in, int d_out, int K, int r, StreamPlan* plan) {
   DevState* ds = nullptr;
   cudaError_t e = dev_state(&ds);
   if (e != cudaSuccess) return e;
@@ -2303,6 +2339,21 @@ cudaError_t plan_lowrank(Elem w_elem, int d_in, int d_out, int K, int r, StreamP
   }
   *plan = best;
   return cudaSuccess;
+}
+
+cudaError_t plan_gather(Elem w_elem, int d_out, int K, StreamPlan* plan) {
+  return cached_plan(PlanKey{0, 0, static_cast<int>(w_elem), 0, d_out, K, 0}, plan,
+                     [&](StreamPlan* p) { return plan_gather_uncached(w_elem, d_out, K, p); });
+}
+
+cudaError_t plan_fused(Elem w_elem, int d_in, int d_out, int K, StreamPlan* plan) {
+  return cached_plan(PlanKey{0, 1, static_cast<int>(w_elem), d_in, d_out, K, 0}, plan,
+                     [&](StreamPlan* p) { return plan_fused_uncached(w_elem, d_in, d_out, K, p); });
+}
+
+cudaError_t plan_lowrank(Elem w_elem, int d_in, int d_out, int K, int r, StreamPlan* plan) {
+  return cached_plan(PlanKey{0, 2, static_cast<int>(w_elem), d_in, d_out, K, r}, plan,
+                     [&](StreamPlan* p) { return plan_lowrank_uncached(w_elem, d_in, d_out, K, r, p); });
 }
 
 cudaError_t launch_lowrank(Elem w_elem, const LowrankArgs& a, const StreamPlan& pl, cudaStream_t stream) {

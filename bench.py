@@ -867,8 +867,9 @@ def bench_larosa(args):
 
     # ---- end to end through the public API with host buffers
     # the four groups' inputs live in one pinned host buffer and one device
-    # buffer (and likewise the outputs), so a step moves them with one copy
-    # each way
+    # buffer, so a step moves them in with one copy; each group's output is
+    # read back on a copy stream as soon as its call is done, while the next
+    # group computes, and the step ends when every output is on the host
     x_sizes = [g.x.numel() for g in groups]
     y_sizes = [g.d_out for g in groups]
     x_host_all = torch.cat([g.x.flatten().cpu() for g in groups]).pin_memory()
@@ -877,6 +878,9 @@ def bench_larosa(args):
     y_dev_all = torch.empty(sum(y_sizes), dtype=torch.float32, device=device)
     y_dev = [v.view(1, -1) for v in torch.split(y_dev_all, y_sizes)]
     y_host_all = torch.empty(sum(y_sizes), dtype=torch.float32).pin_memory()
+    y_host = list(torch.split(y_host_all, y_sizes))
+    copy_stream = torch.cuda.Stream(device)
+    done = [torch.cuda.Event() for _ in groups]
     e2e_steps = max(20, min(500, args.steps // 10))
     with torch.cuda.stream(stream):
         for r in range(args.warmup + e2e_steps):
@@ -885,11 +889,15 @@ def bench_larosa(args):
                 barrier(world, device)
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            # the step's inputs in, the four groups back to back, the outputs out
+            # the step's inputs in, the four groups back to back, each output out
             x_dev_all.copy_(x_host_all, non_blocking=True)
             for gi, g in enumerate(groups):
                 L.larosa_rotate_topk_linear(x_dev[gi], g.Qt, g.W_rot, g.K, y=y_dev[gi], ws=ws, dev_status=st)
-            y_host_all.copy_(y_dev_all, non_blocking=True)
+                done[gi].record(stream)
+                copy_stream.wait_event(done[gi])
+                with torch.cuda.stream(copy_stream):
+                    y_host[gi].copy_(y_dev[gi].view(-1), non_blocking=True)
+            stream.wait_stream(copy_stream)  # the step's outputs are on the host
         e1.record(stream)
     torch.cuda.synchronize(device)
     t_e2e = e0.elapsed_time(e1) / 1e3
