@@ -74,7 +74,7 @@ int fail_cuda(cudaError_t e, const char* where) {
 
 // Where each piece of the multi-token (or fallback) scratch lies.
 struct ScratchLayout {
-  bool tensor_core = false;  // 8-16 bf16 tokens: the dense tcgen05 product, as larosa_sparse_linear
+  bool tensor_core = false;  // 2-16 bf16 tokens: the dense tcgen05 product, as larosa_sparse_linear
   size_t off_bitmap = 0, zero_bytes = 0, off_partials = 0, off_coef = 0, off_rows = 0, off_count = 0;
   size_t off_coef_hl = 0;    // tensor_core: the coefficients' bf16 head and tail
   size_t total = 0;  // 0: no scratch (the one-token cluster gather)

@@ -166,11 +166,13 @@ __global__ void __launch_bounds__(kT, (MT <= 2 && sizeof(T) == 2 ? 2 : 1)) rowdo
 
 // ================================================================ rowmma
 //
-// y[m][j] = sum_k x[m][k] * A[j][k] for 3 to 16 bf16 tokens on the tensor
-// cores (mma.sync m16n8k16, bf16 inputs, fp32 accumulation).  From about
-// eight tokens on, the products per weight byte exceed what the FMA pipes
-// deliver at HBM speed, and the FMA kernel also reads every token's inputs
-// from shared memory once per weight vector.  The tokens are the MMA's 16
+// y[m][j] = sum_k x[m][k] * A[j][k] for 3 to 16 bf16 tokens on the legacy
+// tensor-core path (mma.sync m16n8k16, bf16 inputs, fp32 accumulation), for
+// the shapes the tcgen05 kernel (rot_umma.cu) does not take: n_in a
+// multiple of 32 but not of 64.  From about eight tokens on, the products
+// per weight byte exceed what the FMA pipes deliver at HBM speed, and the
+// FMA kernel also reads every token's inputs from shared memory once per
+// weight vector.  The tokens are the MMA's 16
 // rows (zero beyond M), 8 consecutive output rows j its 8 columns, 16 inputs
 // k its reduction.  Lane (g, q) = (lane / 4, lane % 4) loads 16 bytes of
 // output row j0 + g of A and the same 8 inputs of tokens g and g + 8 per

@@ -1,5 +1,9 @@
-// Row-streaming GEMV for sm_100a: the kernel behind the rotation (x . Q), the
-// sparse linear (sum over the kept rows of W_rot) and the dense baseline.
+// Row-streaming GEMV for sm_100a: the sparse linear of several tokens where
+// the tcgen05 product does not apply (fp32 weights, d_in < 64) and after a
+// threshold selection of several tokens (over the union of their kept
+// rows), the factor GEMVs of the sparse + low-rank mode for several tokens,
+// and the one-token fallbacks (a kept list longer than the cluster gather
+// holds, the no-allocation entry point when its gather plan does not fit).
 //
 //   y[m][c] = sum_r coef(m, r) * W[row(r)][c]
 //

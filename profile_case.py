@@ -14,19 +14,19 @@ them), each on the same seeded inputs:
   identity     the same with Qt = NULL       one token: fused_kernel without
                                              its rotation
   thresh_fused larosa_rotate_threshold_linear fused_kernel in threshold mode
-  rotate       larosa_rotate                 rowdot_kernel (1-2 tokens),
-                                             rowmma_kernel (3-7), umma_kernel (8-16)
+  rotate       larosa_rotate                 rowdot_kernel (one token),
+                                             umma_kernel (2-16)
   rotate_topk  larosa_rotate_topk            rotsel_kernel (one token)
   topk         larosa_topk                   topk_kernel
   threshold    larosa_threshold              threshold_kernel
   sparse       larosa_sparse_linear          gather_kernel (one token);
-                                             scatter, union, rowstream_gemv
-                                             (2-7 tokens); coef_rows and
-                                             umma_kernel (8-16)
+                                             coef_rows and umma_kernel (2-16)
   topk_linear  larosa_topk_linear            topk_kernel, then the sparse linear
   dense        larosa_dense_linear           as rotate, on W in nn.Linear layout
-  lowrank      larosa_sparse_lowrank_linear  the sparse linear, dropped_kernel,
-                                             two rowstream GEMVs (r = 256), add_kernel
+  lowrank      larosa_sparse_lowrank_linear  lowrank_kernel (one token, r = 256);
+                                             several: the sparse linear,
+                                             dropped_kernel, two rowstream
+                                             GEMVs, add_kernel
 
 --fused-only is --calls fused.  The set-up (weights, the counter-rotation by
 prepare_kernel, the reference kept lists) runs before the first call.  One
