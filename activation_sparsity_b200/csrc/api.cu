@@ -224,8 +224,8 @@ uint32_t threshold_key(float t) {
 // two tokens and 40 % sparsity, nearly all from four on), so the sparse
 // linear is the dense tcgen05 product with each token's coefficient row
 // (zero where the token did not keep the row).
-bool tensor_core_gemv(int M, int d_in, int d_out, int dtype, const Layout& L) {
-  return dtype == LAROSA_BF16 && L.coef_hl != 0 && larosa::umma_gemv_applies(M, d_in, d_out);
+bool tensor_core_gemv(int M, int d_in, int d_out, int K, int dtype, const Layout& L) {
+  return dtype == LAROSA_BF16 && L.coef_hl != 0 && larosa::umma_gemv_pays(M, d_in, d_out, K);
 }
 
 int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W_rot, int d_in,
@@ -271,7 +271,7 @@ int run_sparse(const int32_t* idx, const float* val, int M, int K, const void* W
     a.coef = val;
     a.coef_ld = K;
   } else {
-    if (tensor_core_gemv(M, d_in, d_out, dtype, L)) {
+    if (tensor_core_gemv(M, d_in, d_out, K, dtype, L)) {
       // every row is kept by some token at this many tokens: the dense
       // product with the per-token coefficients (zero where not kept)
       __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(at(ws, L.coef_hl));
@@ -694,7 +694,7 @@ static int rotate_topk_linear_impl(const void* x, const void* Qt, const void* W_
   }
   st = run_rotation(x, Qt, x_rot, M, d_in, dtype, s);
   if (st != LAROSA_OK) return st;
-  if (M > 1 && tensor_core_gemv(M, d_in, d_out, dtype, L)) {
+  if (M > 1 && tensor_core_gemv(M, d_in, d_out, K, dtype, L)) {
     // the Top-K kernel also writes the tokens' coefficient rows for the
     // tensor-core product
     __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(at(ws, L.coef_hl));
@@ -746,7 +746,7 @@ static int topk_linear_impl(const float* x_rot, const void* W_rot, int M, int d_
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int32_t* idx = reinterpret_cast<int32_t*>(at(ws, L.idx));
   float* val = reinterpret_cast<float*>(at(ws, L.val));
-  if (M > 1 && tensor_core_gemv(M, d_in, d_out, dtype, L)) {
+  if (M > 1 && tensor_core_gemv(M, d_in, d_out, K, dtype, L)) {
     __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(at(ws, L.coef_hl));
     cudaError_t e = larosa::launch_topk(x_rot, M, d_in, K, idx, val, dev_status, s, hl);
     if (e != cudaSuccess) return cuda_fail(e, "topk kernel");

@@ -157,6 +157,11 @@ cudaError_t launch_rot_umma(const void* A, const void* x, float* y, int M, int n
 // token did not keep the row), given as bf16 head and tail hl [2 x M x d_in]
 // (launch_topk or launch_coef_rows): y = (head + tail) . W on tcgen05.
 bool umma_gemv_applies(int M, int d_in, int d_out);
+// Whether the dense product pays for M tokens keeping K of d_in rows each:
+// umma_gemv_applies, unless few tokens keep so few rows that streaming only
+// their union (expected share 1 - (1 - K / d_in)^M for independent
+// selections: below 0.3 for 2 tokens, 0.2 for 3-4) is faster.
+bool umma_gemv_pays(int M, int d_in, int d_out, int K);
 cudaError_t launch_umma_gemv(const void* W, const __nv_bfloat16* hl, float* y, int M, int d_in, int d_out,
                              int* dev_status, cudaStream_t stream);
 

@@ -74,7 +74,7 @@ int fail_cuda(cudaError_t e, const char* where) {
 
 // Where each piece of the multi-token (or fallback) scratch lies.
 struct ScratchLayout {
-  bool tensor_core = false;  // 2-16 bf16 tokens: the dense tcgen05 product, as larosa_sparse_linear
+  bool tensor_core = false;  // 2-16 bf16 tokens: the dense tcgen05 product where larosa_sparse_linear takes it
   size_t off_bitmap = 0, zero_bytes = 0, off_partials = 0, off_coef = 0, off_rows = 0, off_count = 0;
   size_t off_coef_hl = 0;    // tensor_core: the coefficients' bf16 head and tail
   size_t total = 0;  // 0: no scratch (the one-token cluster gather)
@@ -95,7 +95,7 @@ cudaError_t plan_noalloc(larosa::Elem w, int M, int d_in, int d_out, int K, laro
     if (e != cudaSuccess) return e;
     if (sp->ok) return cudaSuccess;
   }
-  if (M > 1 && w == larosa::Elem::BF16 && larosa::umma_gemv_applies(M, d_in, d_out)) {
+  if (M > 1 && w == larosa::Elem::BF16 && larosa::umma_gemv_pays(M, d_in, d_out, K)) {
     // [coefficient heads and tails]: every word is written by each call
     S->tensor_core = true;
     S->off_coef_hl = 0;

@@ -41,6 +41,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cmath>
 
 #include "common.cuh"
 #include "internal.h"
@@ -434,6 +435,22 @@ cudaError_t launch_rot_umma(const void* A, const void* x, float* y, int M, int n
 
 bool umma_gemv_applies(int M, int d_in, int d_out) {
   return M >= kUMinTokens && M <= kUTokens && d_in % 8 == 0 && d_out % 8 == 0 && d_in >= kUBox;
+}
+
+// The dense product streams every row of W; the row-streaming GEMV only the
+// union of the kept rows, but with a fixed cost of about 20 us (coefficient
+// scatter, union, its own ramp) and a lower rate per byte, worse still with
+// the mma.sync consumers it uses from 8 tokens.  Measured on a 4096 x 22016
+// weight (us per call, dense / union): 2 tokens keeping 15 % 31.8 / 24.6,
+// 30 % 32.6 / 32.6 (the union then covers 51 %); 4 tokens keeping 5 %
+// 32.5 / 29.9, 10 % 32.5 / 35.4; 8 tokens keeping 3 % 33.0 / 39.8; 16 tokens
+// keeping 5 % 34.8 / 128.  So the union is streamed only where few tokens
+// keep few rows.
+bool umma_gemv_pays(int M, int d_in, int d_out, int K) {
+  if (!umma_gemv_applies(M, d_in, d_out) || K <= 0) return false;
+  const double kept = 1.0 - std::pow(1.0 - static_cast<double>(K) / d_in, M);
+  const double union_below = M <= 2 ? 0.3 : M <= 4 ? 0.2 : 0.0;
+  return kept >= union_below;
 }
 
 // Column tiles of 128 (one accumulator) with the two-stage ring above, four

@@ -74,6 +74,7 @@ def _check_against_oracle(y, idx, val, W):
     (1, 11008, 4096, 6605),   # LLaMA2-7B down at 40 % sparsity
     (4, 1024, 2048, 400),     # several tokens sharing streamed rows
     (8, 2048, 1024, 1229),    # eight tokens: the scratch holds coefficient rows of all of them
+    (2, 4096, 1024, 100),     # few rows per token: the union of the kept rows is streamed
 ])
 def test_noalloc_matches_oracle_and_workspace_entry_point_on_two_calls(lib, M, d_in, d_out, K):
     import activation_sparsity_b200 as L
