@@ -828,6 +828,16 @@ int larosa_rotate_threshold_linear(const void* x, const void* Qt, const void* W_
   }
   st = run_rotation(x, Qt, x_rot, M, d_in, dtype, s);
   if (st != LAROSA_OK) return st;
+  if (M > 1 && dtype == LAROSA_BF16 && L.coef_hl != 0 && larosa::umma_gemv_applies(M, d_in, d_out)) {
+    // how many rows the tokens keep is known only on the device: the dense
+    // tensor-core product with the coefficient rows the threshold kernel
+    // writes, as the Top-K path takes at the sparsities the method uses
+    __nv_bfloat16* hl = reinterpret_cast<__nv_bfloat16*>(at(ws, L.coef_hl));
+    e = larosa::launch_threshold(x_rot, M, d_in, t_key, idx, val, nnz, nullptr, nullptr, dev_status, s, hl);
+    if (e != cudaSuccess) return cuda_fail(e, "threshold kernel");
+    e = larosa::launch_umma_gemv(W_rot, hl, y, M, d_in, d_out, dev_status, s);
+    return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "tensor-core sparse linear kernel");
+  }
   GemvPlan pl;
   e = larosa::plan_gemv(elem_of(dtype), Elem::F32, M, d_out, d_in, &pl);
   if (e != cudaSuccess) return cuda_fail(e, "plan sparse linear");

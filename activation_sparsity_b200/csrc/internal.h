@@ -84,7 +84,7 @@ cudaError_t launch_coef_rows(const int32_t* idx, const float* val, int M, int K,
 // of kept rows, as launch_scatter does.
 cudaError_t launch_threshold(const float* x_rot, int M, int d, uint32_t t_key, int32_t* idx,
                              float* val, int32_t* nnz, float* coef, unsigned* bitmap,
-                             int* dev_status, cudaStream_t stream);
+                             int* dev_status, cudaStream_t stream, __nv_bfloat16* hl = nullptr);
 
 // Low-rank compensation: x_drop = x with each token's kept entries zeroed;
 // y += add (n elements).

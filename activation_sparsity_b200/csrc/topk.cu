@@ -175,13 +175,15 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
 // left as they were) and their count to nnz[m].  With coef != nullptr the
 // token's row of coef [M x d] also receives x where kept and 0 elsewhere,
 // and the kept rows are marked in `bitmap` (the multi-token sparse linear's
-// input, as the scatter kernel makes it).  Each warp walks its own segment
+// input, as the scatter kernel makes it); with hl != nullptr the token's
+// dense bf16 head and tail coefficient rows for the tensor-core product, as
+// the Top-K kernel writes them.  Each warp walks its own segment
 // of the row twice: once to count, once to place its kept entries after the
 // earlier warps' ones.
 __global__ void __launch_bounds__(kTopkThreads, 1)
     threshold_kernel(const float* __restrict__ x_rot, int d, uint32_t t_key, int32_t* __restrict__ idx,
                      float* __restrict__ val, int32_t* __restrict__ nnz, float* __restrict__ coef,
-                     unsigned* bitmap, int* dev_status) {
+                     unsigned* bitmap, int* dev_status, __nv_bfloat16* hl) {
   __shared__ uint32_t warp_sums[32];
   const int m = blockIdx.x;
   const int lane = threadIdx.x & 31;
@@ -221,13 +223,19 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
     pos += __popc(mk);
   }
   if (threadIdx.x == 0) nnz[m] = static_cast<int32_t>(total);
+  if (hl != nullptr) {
+    const size_t M = gridDim.x;
+    write_head_tail(bits, d, [&](uint32_t key, int) { return key >= t_key; }, hl + (size_t)m * d,
+                    hl + (M + m) * d);
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_threshold(const float* x_rot, int M, int d, uint32_t t_key, int32_t* idx,
                              float* val, int32_t* nnz, float* coef, unsigned* bitmap,
-                             int* dev_status, cudaStream_t stream) {
+                             int* dev_status, cudaStream_t stream, __nv_bfloat16* hl) {
+  if (hl != nullptr && d % 8 != 0) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(M, 1, 1);
   cfg.blockDim = dim3(kTopkThreads, 1, 1);
@@ -238,7 +246,7 @@ cudaError_t launch_threshold(const float* x_rot, int M, int d, uint32_t t_key, i
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, threshold_kernel, x_rot, d, t_key, idx, val, nnz, coef, bitmap,
-                            dev_status);
+                            dev_status, hl);
 }
 
 cudaError_t launch_coef_rows(const int32_t* idx, const float* val, int M, int K, int d, __nv_bfloat16* hl,

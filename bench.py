@@ -708,6 +708,10 @@ def bench_larosa(args):
         for gi, (g, y) in enumerate(zip(groups, ys)):
             L.larosa_rotate_threshold_linear(g.x, g.Qt, g.W_rot, t_rot[gi], y=y, ws=ws, dev_status=st)
 
+    def batch_thr_step():  # 16 tokens per call with the threshold selection
+        for gi, (g, x, y) in enumerate(zip(groups, x_batch[16], y_batch[16])):
+            L.larosa_rotate_threshold_linear(x, g.Qt, g.W_rot, t_rot[gi], y=y, ws=ws, dev_status=st)
+
     def unrot_thr_step():
         for gi, (g, y) in enumerate(zip(groups, ys)):
             L.larosa_rotate_threshold_linear(g.x, None, g.W, t_x[gi], y=y, ws=ws, dev_status=st)
@@ -788,6 +792,7 @@ def bench_larosa(args):
         t, n = calibrate(g.x.float().abs(), g.d_in)
         t_x.append(t)
         nnz_x.append(n)
+    t_rot_list = list(t_rot)  # (t_rot is reused for a time below)
 
     g_fused = graph_of(fused_step)
     g_sparse = graph_of(sparse_only_step)
@@ -802,6 +807,7 @@ def bench_larosa(args):
     g_folded_topk = graph_of(folded_topk_step)
     g_sweep = {sp: graph_of(sparsity_step(sp)) for sp in sweep}
     g_batch = {M: graph_of(batch_step(M)) for M in batch_sizes}
+    g_batch_thr = graph_of(batch_thr_step)
     g_folded_thr = graph_of(folded_thr_step)
     g_lowrank = graph_of(lowrank_step)
 
@@ -829,6 +835,7 @@ def bench_larosa(args):
     side_steps = max(1, args.steps // 4)
     t_sweep = {sp: time_graph(gr, side_steps, args.warmup)[0] for sp, gr in g_sweep.items()}
     t_batch = {M: time_graph(gr, side_steps, args.warmup)[0] for M, gr in g_batch.items()}
+    t_batch_thr = time_graph(g_batch_thr, side_steps, args.warmup)[0]
     # rows streamed per batch step: the union of the tokens' kept rows (Q once per batch)
     batch_bytes = {}
     for M in batch_sizes:
@@ -839,6 +846,15 @@ def bench_larosa(args):
             rows = int(torch.unique(idx.flatten()).numel())
             tot += rows * g.d_out * 2 + g.d_in * g.d_in * 2 + M * (g.d_in * 6 + g.K * 8 + g.d_out * 4)
         batch_bytes[M] = tot
+    # the 16-token threshold step: Q once, the union of the kept rows
+    batch_thr_bytes = 0
+    for gi, (g, x) in enumerate(zip(groups, x_batch[16])):
+        xr = L.larosa_rotate(x, g.Qt)
+        idx, _, nnz = L.larosa_threshold(xr, t_rot_list[gi], dev_status=st)
+        kept = torch.cat([idx[m, :int(nnz[m].item())] for m in range(16)])
+        rows = int(torch.unique(kept).numel())
+        batch_thr_bytes += (rows * g.d_out * 2 + g.d_in * g.d_in * 2 + 16 * (g.d_in * 6 + g.d_out * 4)
+                            + int(nnz.sum().item()) * 8)
     n_launch = args.steps * len(groups)
     rot_us = t_rot / n_launch * 1e6
     rotsel_us = t_rotsel / n_launch * 1e6
@@ -964,6 +980,9 @@ def bench_larosa(args):
                 "rotated_threshold_tokens_per_s": args.steps / t_rot_thr * world,
                 "rotated_threshold_hbm_frac": rot_thr_bytes * args.steps / t_rot_thr / 1e9 / peak,
                 "rotated_threshold_kept_frac": sum(nnz_rot) / sum(g.d_in for g in groups),
+                # 16 tokens per call, each group's t as above (tokens/s counts every token)
+                "rotated_threshold_M16_tokens_per_s": 16 * side_steps / t_batch_thr * world,
+                "rotated_threshold_M16_hbm_frac": batch_thr_bytes * side_steps / t_batch_thr / 1e9 / peak,
                 "unrotated_threshold_tokens_per_s": args.steps / t_unrot_thr * world,
                 "unrotated_threshold_hbm_frac": unrot_thr_bytes * args.steps / t_unrot_thr / 1e9 / peak,
                 "unrotated_threshold_kept_frac": sum(nnz_x) / sum(g.d_in for g in groups),

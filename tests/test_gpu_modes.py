@@ -126,6 +126,13 @@ def check_threshold_path(x_rot, x_rot_ref, gamma, idx, val, nnz, t):
     (torch.bfloat16, 16, 512, 256, 25),
     (torch.bfloat16, 1, 1024, 1032, 0),
     (torch.bfloat16, 1, 1024, 1032, 100),
+    # several bf16 tokens: the tensor-core product with the threshold
+    # kernel's coefficient rows (everything kept, nothing kept, the 7B shape)
+    (torch.bfloat16, 2, 1024, 1032, 0),
+    (torch.bfloat16, 4, 1024, 1032, 100),
+    (torch.bfloat16, 8, 4096, 4096, 40),
+    # several fp32 tokens: the union of the kept rows, row-streamed
+    (torch.float32, 4, 256, 512, 50),
 ])
 def test_fused_threshold(L, dtype, M, d_in, d_out, drop):
     Q = sd.orthogonal(d_in, 801, device="cuda" if d_in > 4096 else "cpu").to(dtype).cpu()
