@@ -292,7 +292,10 @@ int larosa_threshold(const float *x_rot, int M, int d, float t, int32_t *idx,
  * NULL again selects the identity rotation, the TEAL/CATS-style mode).  For
  * one token one cooperative kernel as for the Top-K (no selection step: the
  * gather CTAs stream their kept rows as soon as every CTA has rotated);
- * otherwise rotation, larosa_threshold's kernel and the row-streaming sparse
+ * otherwise rotation, larosa_threshold's kernel and the sparse linear: for
+ * several bf16 tokens the dense tensor-core product with the coefficient
+ * rows the threshold kernel writes (every row of W_rot is streamed, since the
+ * kept share is known only on the device), else the row-streaming sparse
  * linear over the kept rows (for M > 1 over the union of the tokens' sets).
  * ws: at least larosa_workspace_bytes(M, d_in, d_out, d_in) bytes; x_rot,
  * idx and val ([M x d_in] each, as larosa_threshold writes them) lie at the
