@@ -90,6 +90,11 @@ cudaError_t launch_threshold(const float* x_rot, int M, int d, uint32_t t_key, i
 // y += add (n elements).
 cudaError_t launch_dropped(const float* x, const int32_t* idx, int M, int K, int d, float* x_drop,
                            int* dev_status, cudaStream_t stream);
+// The dropped part's bf16 head and tail coefficient rows, hl [2 x M x d]
+// (x with idx's K kept entries of each token zeroed; K = 0: x itself), for
+// the tensor-core factor products.  d a multiple of 8.
+cudaError_t launch_dropped_rows(const float* x, const int32_t* idx, int M, int K, int d, __nv_bfloat16* hl,
+                                int* dev_status, cudaStream_t stream);
 cudaError_t launch_add(float* y, const float* add, int n, cudaStream_t stream);
 
 // x_rot[i] = x[i] widened to fp32 (the identity rotation), n elements.

@@ -12,6 +12,7 @@
 // scan that places every kept entry, ascending in the index.  The whole
 // vector (d <= 32768 fp32) stays in shared memory; nothing but the input row
 // and the K outputs touches global memory.
+#include "coef.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
@@ -23,32 +24,19 @@ constexpr int kTopkThreads = 1024;
 constexpr int kTopkCand = 2048;
 constexpr int kTopkU = 8;  // 16-byte loads in flight per thread
 
-// The coefficient c of a kept entry (0 elsewhere) as the bf16 head and tail
-// the tensor cores multiply: head = bf16(c), tail = bf16(c - head), both
-// rounded to nearest even (about 16 significant bits of c kept in all).
-__device__ __forceinline__ void split_head_tail(float c, __nv_bfloat16* head, __nv_bfloat16* tail) {
-  const __nv_bfloat16 h = __float2bfloat16_rn(c);
-  *head = h;
-  *tail = __float2bfloat16_rn(c - __bfloat162float(h));
-}
-
 // Writes the token's dense coefficient rows hi[0, d), lo[0, d): the head and
 // tail of x where kept(key, i), zero elsewhere.  d a multiple of 8, hi and lo
-// 16-byte aligned; 8 entries (one 16-byte store to each row) per step.
+// 16-byte aligned.
 template <typename Kept>
 __device__ __forceinline__ void write_head_tail(const uint32_t* bits, int d, Kept kept,
                                                 __nv_bfloat16* hi, __nv_bfloat16* lo) {
-  for (int v = threadIdx.x; v < d / 8; v += kTopkThreads) {
-    __align__(16) __nv_bfloat16 h[8], t[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int i = 8 * v + e;
-      const uint32_t u = bits[i];
-      split_head_tail(kept(u & kKeyMask, i) ? __uint_as_float(u) : 0.f, &h[e], &t[e]);
-    }
-    reinterpret_cast<uint4*>(hi)[v] = *reinterpret_cast<const uint4*>(h);
-    reinterpret_cast<uint4*>(lo)[v] = *reinterpret_cast<const uint4*>(t);
-  }
+  write_head_tail_rows<kTopkThreads>(
+      d,
+      [&](int i) {
+        const uint32_t u = bits[i];
+        return kept(u & kKeyMask, i) ? __uint_as_float(u) : 0.f;
+      },
+      hi, lo);
 }
 
 // With hl != nullptr the kernel also writes each token's dense coefficient

@@ -737,6 +737,17 @@ def bench_larosa(args):
             L.larosa_sparse_lowrank_linear(x_rots[gi], idxs[gi], vals[gi], g.W_rot, lr_A[gi], lr_B[gi], y=y,
                                            ws=lr_ws[gi], dev_status=st)
 
+    # the same mode with 16 tokens per call (pre-rotated inputs, their Top-K lists)
+    lr_x16 = [L.larosa_rotate(x, g.Qt) for g, x in zip(groups, x_batch[16])]
+    lr_sel16 = [L.larosa_topk(xr, g.K, dev_status=st) for g, xr in zip(groups, lr_x16)]
+    lr_ws16 = [torch.zeros(L.larosa_lowrank_workspace_bytes(16, g.d_in, g.d_out, g.K, LR), dtype=torch.uint8,
+                           device=device) for g in groups]
+
+    def lowrank16_step():
+        for gi, (g, y) in enumerate(zip(groups, y_batch[16])):
+            L.larosa_sparse_lowrank_linear(lr_x16[gi], lr_sel16[gi][0], lr_sel16[gi][1], g.W_rot, lr_A[gi],
+                                           lr_B[gi], y=y, ws=lr_ws16[gi], dev_status=st)
+
     def folded_thr_step():
         for gi, (g, y) in enumerate(zip(groups, ys)):
             L.larosa_rotate_threshold_linear(x_folded[gi], None, g.W_rot, t_rot[gi], y=y, ws=ws,
@@ -810,6 +821,7 @@ def bench_larosa(args):
     g_batch_thr = graph_of(batch_thr_step)
     g_folded_thr = graph_of(folded_thr_step)
     g_lowrank = graph_of(lowrank_step)
+    g_lowrank16 = graph_of(lowrank16_step)
 
     props = torch.cuda.get_device_properties(device)
     clocks = ClockSampler(f"GPU-{props.uuid}")
@@ -832,6 +844,7 @@ def bench_larosa(args):
     t_folded_topk, _ = time_graph(g_folded_topk, args.steps, args.warmup)
     t_folded_thr, _ = time_graph(g_folded_thr, args.steps, args.warmup)
     t_lowrank, _ = time_graph(g_lowrank, args.steps, args.warmup)
+    t_lowrank16 = time_graph(g_lowrank16, max(1, args.steps // 4), args.warmup)[0]
     side_steps = max(1, args.steps // 4)
     t_sweep = {sp: time_graph(gr, side_steps, args.warmup)[0] for sp, gr in g_sweep.items()}
     t_batch = {M: time_graph(gr, side_steps, args.warmup)[0] for M, gr in g_batch.items()}
@@ -869,6 +882,11 @@ def bench_larosa(args):
     step_bytes = sum(path_bytes(g, g.K)["total"] for g in groups)
     sparse_bytes = sum(path_bytes(g, g.K, rotate=False)["total"] for g in groups)
     lowrank_bytes = sparse_bytes + sum((g.d_in + g.d_out) * LR * 2 + g.d_in * 4 for g in groups)
+    lowrank16_bytes = 0
+    for g, (idx16, _) in zip(groups, lr_sel16):
+        rows = int(torch.unique(idx16.flatten()).numel())
+        lowrank16_bytes += (rows * g.d_out * 2 + (g.d_in + g.d_out) * LR * 2
+                            + 16 * (g.d_in * 4 + g.K * 8 + g.d_out * 4))
     dense_bytes = sum(g.d_in * g.d_out * 2 + g.d_in * 2 + g.d_out * 4 for g in groups)
     unrot_topk_bytes = sum(path_bytes(g, g.K, rotate=False)["total"] for g in groups)
     rot_thr_bytes = sum(path_bytes(g, n)["total"] for g, n in zip(groups, nnz_rot))
@@ -996,6 +1014,11 @@ def bench_larosa(args):
                 # the pre-rotated input (Q not streamed)
                 "sparse_lowrank_r256_tokens_per_s": args.steps / t_lowrank * world,
                 "sparse_lowrank_r256_hbm_frac": lowrank_bytes * args.steps / t_lowrank / 1e9 / peak,
+                # 16 tokens per call (tokens/s counts every token; bytes: the union
+                # of the tokens' kept rows, both factors once, the activations)
+                "sparse_lowrank_r256_M16_tokens_per_s": 16 * max(1, args.steps // 4) / t_lowrank16 * world,
+                "sparse_lowrank_r256_M16_hbm_frac": lowrank16_bytes * max(1, args.steps // 4) / t_lowrank16
+                / 1e9 / peak,
             },
             # the fused path at the sweep's other sparsities, and with M tokens
             # per call (tokens/s counts every token; bytes: Q once plus the

@@ -315,6 +315,10 @@ def test_folded_rotation_path(L, d_prev, d, d_out):
     (torch.bfloat16, 16, 512, 256, 64, 40),
     (torch.bfloat16, 1, 4096, 4096, 256, 40),
     (torch.bfloat16, 2, 200, 24, 16, 0),
+    # several bf16 tokens with both factor products on the tensor cores
+    (torch.bfloat16, 8, 2048, 2048, 256, 40),
+    (torch.bfloat16, 3, 2048, 1032, 64, 50),
+    (torch.bfloat16, 4, 1024, 1032, 128, 100),
     # one token, one launch: every entry dropped, none dropped, ranks that are
     # not powers of two, the down projection's width, a width over 16384 (a
     # factor CTA covers at most 4096 entries of x), every entry of the down
