@@ -324,10 +324,11 @@ int larosa_rotate_threshold_linear(const void *x, const void *Qt,
  * W while factor CTAs, each over a range of x, compute partials of
  * u = dropped . A_r (reading only the dropped rows of A_r), then the
  * column-tile CTAs add the partials of their entries of u and stream the
- * rows of B_r with those coefficients into the same sums.  Otherwise: the sparse linear
- * on the kept list, the dropped part of x, u = dropped . A_r and
- * y_r = u . B_r by the row-streaming GEMV with fp32 coefficients, and
- * y += y_r.  The workspace must be zero-filled before its first use (the
+ * rows of B_r with those coefficients into the same sums.  Otherwise: the
+ * sparse linear on the kept list, then u = dropped . A_r and y_r = u . B_r
+ * -- for bf16 with 64 <= r <= d_in as tensor-core products fed with the
+ * dropped part's and u's bf16 head/tail coefficient rows, else by the
+ * row-streaming GEMV with fp32 coefficients -- and y += y_r.  The workspace must be zero-filled before its first use (the
  * one-token kernel keeps counters there, zero again after every call).
  * ws: at least larosa_lowrank_workspace_bytes(M, d_in, d_out, K, r) bytes.
  */
