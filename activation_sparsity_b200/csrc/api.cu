@@ -1,22 +1,32 @@
 // C ABI of the library: argument validation, workspace layout and the
 // sequencing of kernels for each entry point (see include/larosa.h).
 //
-//   rotation, dense baseline   rowdot (onetoken.cu), any M <= 16
+//   rotation, dense baseline   rowdot (onetoken.cu) for one token; umma_kernel
+//                              (rot_umma.cu, tcgen05) for 2-16 bf16 tokens
 //   Top-K alone                topk_kernel (topk.cu)
 //   sparse linear, M = 1       cluster gather over idx/val (onetoken.cu)
-//   sparse linear, M > 1       scatter + union (union.cu) + rowstream (rowstream.cu)
+//   sparse linear, M > 1       bf16: coefficient rows (topk.cu) + the tcgen05
+//                              product over every row, unless 2-4 tokens keep
+//                              few rows; else scatter + union (union.cu) +
+//                              rowstream (rowstream.cu)
 //   rotation + Top-K, M = 1    rotsel (onetoken.cu): its last CTA selects
 //   fused, M = 1               fused_kernel (onetoken.cu): one cooperative launch;
 //                              where it does not fit, rotsel -> list gather
-//   fused, M > 1               rowdot -> topk -> scatter/union -> rowstream
+//   fused, M > 1               rotation -> topk (writing the coefficient rows
+//                              where the tcgen05 product is taken) -> sparse linear
 //   threshold, M = 1           fused_kernel in threshold mode; where it does not
 //                              fit, rowdot -> threshold -> rowstream over the list
-//   threshold, M > 1           rowdot -> threshold (writes the coefficient rows
-//                              and the bitmap) -> union -> rowstream
-//   no Qt (identity rotation)  as above with widen in place of rowdot
-//   sparse + low rank          sparse linear on the kept list; dropped part
-//                              (lowrank.cu); two dense row-streaming GEMVs
-//                              through the factors; y += y_r
+//   threshold, M > 1           rotation -> threshold (bf16: writes the coefficient
+//                              rows for the tcgen05 product; else the coefficient
+//                              rows and the bitmap) -> union -> rowstream
+//   no Qt (identity rotation)  as above with widen in place of the rotation
+//   sparse + low rank          one token: lowrank_kernel (onetoken.cu), one
+//                              launch; several: the sparse linear, then the two
+//                              factor products (bf16: coefficient rows from
+//                              lowrank.cu and tcgen05; else the dropped part and
+//                              row-streaming GEMVs), y += y_r
+//   debug checks               check_lists_kernel (debug.cu) around the calls
+//                              that take or write kept lists, when enabled
 #include <stdio.h>
 #include <string.h>
 

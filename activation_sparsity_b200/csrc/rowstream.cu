@@ -8,7 +8,7 @@
 //   y[m][c] = sum_r coef(m, r) * W[row(r)][c]
 //
 // The LaRoSA saving comes from reading only the K kept rows of the
-// counter-rotated weight (paper abstract: activation sparsity reduces memory
+// counter-rotated weight (La RoSA abstract: activation sparsity reduces memory
 // transfers).  With the weight row-major [d_in x d_out], every kept row is
 // one contiguous run, so the kernel is a row gather that is bound by HBM
 // bandwidth.  Design:
