@@ -85,10 +85,12 @@ def test_topk_linear_bf16_weights(L, d_in, d_out, sparsity):
     assert rel_inf(y[0], oracle.sparse_linear(want_i, want_v, f64(W))) <= Y_TOL
 
 
-@pytest.mark.parametrize("M", [2, 4, 8, 16])
-def test_topk_linear_several_tokens(L, M):
+@pytest.mark.parametrize("M,sparsity", [(2, 40), (4, 40), (8, 40), (16, 40),
+                                        # few rows per token: two and four tokens stream the union
+                                        (2, 95), (4, 97)])
+def test_topk_linear_several_tokens(L, M, sparsity):
     d_in, d_out = 1024, 2048
-    K = sd.k_for_sparsity(d_in, 40)
+    K = sd.k_for_sparsity(d_in, sparsity)
     x = sd.activations(M, d_in, 1420 + M, torch.float32).cuda()
     W = sd.weights(d_in, d_out, 0.02, 1421, torch.bfloat16, device="cuda")
     y, idx, val = run(L, x, W, K)
