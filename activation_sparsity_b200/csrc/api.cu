@@ -233,7 +233,8 @@ uint32_t threshold_key(float t) {
 // 2 to 16 bf16 tokens: the union of their kept rows is most rows (84 % at
 // two tokens and 40 % sparsity, nearly all from four on), so the sparse
 // linear is the dense tcgen05 product with each token's coefficient row
-// (zero where the token did not keep the row).
+// (zero where the token did not keep the row) -- unless two to four tokens
+// keep so few rows that streaming their union is faster (umma_gemv_pays).
 bool tensor_core_gemv(int M, int d_in, int d_out, int K, int dtype, const Layout& L) {
   return dtype == LAROSA_BF16 && L.coef_hl != 0 && larosa::umma_gemv_pays(M, d_in, d_out, K);
 }
