@@ -959,20 +959,17 @@ int larosa_sparse_lowrank_linear(const float* x, const int32_t* idx, const float
       larosa::umma_gemv_applies(M, d_in, r) && larosa::umma_gemv_applies(M, r, d_out)) {
     // several bf16 tokens: both factor products on the tensor cores, fed with
     // head/tail coefficient rows of the dropped part (in the coefficient-row
-    // buffer, free again once y_s is done) and of u (in x_drop's space, which
-    // this path does not use: 2 M r bf16 <= M d_in fp32)
+    // buffer, free again once y_s is done); the first writes u directly as
+    // head/tail rows (in x_drop's space, which this path does not use:
+    // 2 M r bf16 <= M d_in fp32), the second adds y_r into y
     __nv_bfloat16* hl_x = reinterpret_cast<__nv_bfloat16*>(at(ws, LL.base.coef_hl));
     __nv_bfloat16* hl_u = reinterpret_cast<__nv_bfloat16*>(x_drop);
     cudaError_t e = larosa::launch_dropped_rows(x, idx, M, K, d_in, hl_x, dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e, "dropped-part rows kernel");
-    e = larosa::launch_umma_gemv(A_r, hl_x, u, M, d_in, r, dev_status, s);
+    e = larosa::launch_umma_gemv(A_r, hl_x, nullptr, M, d_in, r, dev_status, s, false, hl_u);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core factor kernel");
-    e = larosa::launch_dropped_rows(u, nullptr, M, 0, r, hl_u, dev_status, s);
-    if (e != cudaSuccess) return cuda_fail(e, "factor rows kernel");
-    e = larosa::launch_umma_gemv(B_r, hl_u, y_r, M, r, d_out, dev_status, s);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor-core factor kernel");
-    e = larosa::launch_add(y, y_r, M * d_out, s);
-    return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "add kernel");
+    e = larosa::launch_umma_gemv(B_r, hl_u, y, M, r, d_out, dev_status, s, true);
+    return e == cudaSuccess ? LAROSA_OK : cuda_fail(e, "tensor-core factor kernel");
   }
   // y_r = ((x - sigma(x)) . A_r) . B_r, then y = y_s + y_r
   cudaError_t e = larosa::launch_dropped(x, idx, M, K, d_in, x_drop, dev_status, s);

@@ -167,8 +167,12 @@ bool umma_gemv_applies(int M, int d_in, int d_out);
 // their union (expected share 1 - (1 - K / d_in)^M for independent
 // selections: below 0.3 for 2 tokens, 0.2 for 3-4) is faster.
 bool umma_gemv_pays(int M, int d_in, int d_out, int K);
+// accumulate: y += the product; hl_out (not null): the product written as
+// bf16 head/tail rows [2 x M x d_out] (the next product's coefficients)
+// instead of y.
 cudaError_t launch_umma_gemv(const void* W, const __nv_bfloat16* hl, float* y, int M, int d_in, int d_out,
-                             int* dev_status, cudaStream_t stream);
+                             int* dev_status, cudaStream_t stream, bool accumulate = false,
+                             __nv_bfloat16* hl_out = nullptr);
 
 // One token: x_rot = x . Q (through Qt = Q^T), then the last CTA to finish
 // writes the kept list (idx, val: the K largest |x_rot|, ties to the lower

@@ -43,6 +43,7 @@
 #include <algorithm>
 #include <cmath>
 
+#include "coef.cuh"
 #include "common.cuh"
 #include "internal.h"
 #include "tcgen05.cuh"
@@ -96,6 +97,8 @@ struct UShape {
 
 struct UParams {
   float* y;
+  __nv_bfloat16* hl_out;  // not null: the result as bf16 head/tail rows [2 x M x n_out] instead of y
+  int accumulate;         // 1: y += result
   int n_out;
   int M;
   int k_per_split;  // inputs per split, a multiple of the stage's chunk
@@ -301,7 +304,20 @@ __global__ void __launch_bounds__(kUThreads, 1)
       const int row = r0 + (e - m * (r1 - r0));
       float s = 0.f;
       for (int qq = 0; qq < R; ++qq) s += cluster.map_shared_rank(part, qq)[m * S::kCols + row];
-      if (j0 + row < p.n_out) p.y[(size_t)m * p.n_out + j0 + row] = s;
+      const int j = j0 + row;
+      if (j < p.n_out) {
+        if (p.hl_out != nullptr) {
+          // the next product's coefficients: heads in rows 0 .. M-1, tails in M .. 2M-1
+          __nv_bfloat16 h, t;
+          split_head_tail(s, &h, &t);
+          p.hl_out[(size_t)m * p.n_out + j] = h;
+          p.hl_out[(size_t)(p.M + m) * p.n_out + j] = t;
+        } else if (p.accumulate) {
+          p.y[(size_t)m * p.n_out + j] += s;
+        } else {
+          p.y[(size_t)m * p.n_out + j] = s;
+        }
+      }
     }
   }
   cluster.sync();  // no CTA leaves while another may still read its partial tile
@@ -363,12 +379,13 @@ cudaError_t umma_dev(int dev, UDev* out) {
 
 template <bool kGemv, int kNB>
 cudaError_t launch_umma(const CUtensorMap& map_a, const CUtensorMap& map_b0, const CUtensorMap& map_b1,
-                        float* y, int M, int n_in, int n_out, int R, int* dev_status, cudaStream_t stream) {
+                        float* y, int M, int n_in, int n_out, int R, int* dev_status, cudaStream_t stream,
+                        bool accumulate = false, __nv_bfloat16* hl_out = nullptr) {
   using S = UShape<kGemv, kNB>;
   const int tiles = (n_out + S::kCols - 1) / S::kCols;
   const int chunks = (n_in + S::kChunk - 1) / S::kChunk;
   const int k_per_split = ((chunks + R - 1) / R) * S::kChunk;
-  UParams p{y, n_out, M, k_per_split, n_in, dev_status, wait_limit_ns()};
+  UParams p{y, hl_out, accumulate ? 1 : 0, n_out, M, k_per_split, n_in, dev_status, wait_limit_ns()};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(R, tiles, 1);
   cfg.blockDim = dim3(kUThreads, 1, 1);
@@ -460,7 +477,7 @@ bool umma_gemv_pays(int M, int d_in, int d_out, int K) {
 constexpr int kGemvNB = 1;
 
 cudaError_t launch_umma_gemv(const void* W, const __nv_bfloat16* hl, float* y, int M, int d_in, int d_out,
-                             int* dev_status, cudaStream_t stream) {
+                             int* dev_status, cudaStream_t stream, bool accumulate, __nv_bfloat16* hl_out) {
   CUtensorMap map_w, map_hi, map_lo;
   // W: d_in rows (the reduction) of d_out columns, boxes of 64 rows x 64 columns
   if (!tc::make_map(&map_w, W, d_in, d_out, kUBox) || !tc::make_map(&map_hi, hl, M, d_in, kUTokens) ||
@@ -472,8 +489,11 @@ cudaError_t launch_umma_gemv(const void* W, const __nv_bfloat16* hl, float* y, i
   if (e == cudaSuccess) e = plan_umma<true, 2>(d_in, d_out, &R2, &t2);
   if (e != cudaSuccess) return e;
   const bool wide = kGemvNB == 2 || (kGemvNB == 0 && t2 <= t1);
-  if (wide) return launch_umma<true, 2>(map_w, map_hi, map_lo, y, M, d_in, d_out, R2, dev_status, stream);
-  return launch_umma<true, 1>(map_w, map_hi, map_lo, y, M, d_in, d_out, R1, dev_status, stream);
+  if (wide)
+    return launch_umma<true, 2>(map_w, map_hi, map_lo, y, M, d_in, d_out, R2, dev_status, stream, accumulate,
+                                hl_out);
+  return launch_umma<true, 1>(map_w, map_hi, map_lo, y, M, d_in, d_out, R1, dev_status, stream, accumulate,
+                              hl_out);
 }
 
 }  // namespace larosa
