@@ -8,7 +8,14 @@
 * The perf-only layers of the larger workloads: their rotations are signed
   row permutations of one Haar rotation per width, which must still be
   orthogonal, distinct per layer and group, and of the right shapes.
+* The reference arm (the fp64 oracle on the host cores) prints exactly one
+  JSON line with the benchmark's keys.
 """
+import json
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -79,3 +86,20 @@ def test_perf_layers_weight_scale():
     w = torch.cat([g.W_rot.double().flatten() for g in layers[0]])
     assert float(w.std()) == pytest.approx(0.02, rel=0.05)
     assert abs(float(w.mean())) < 1e-3
+
+
+def test_reference_arm_prints_one_json_line_with_the_contract_keys():
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "3"], capture_output=True, text=True, timeout=600, check=True).stdout
+    lines = [ln for ln in out.splitlines() if ln.strip()]
+    assert len(lines) == 1, lines
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["dtype"] == "f64" and d["data"] == "synthetic"
+    assert d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 3 and d["higher_is_better"] is True
+    assert d["unit"] == "tokens/s" and d["value"] > 0 and d["ms_per_step"] > 0
+    assert "llama2-7b-layer" in d["config"]["workload"]
+    cpu = d["cpu_baseline"]
+    assert cpu["kind"] == "oracle" and cpu["cores"] >= 1 and cpu["value"] == d["value"]
+    e2e = d["e2e"]
+    assert e2e["value"] == d["value"] and e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
