@@ -223,3 +223,19 @@ def test_binding_signatures_match_the_header(lib):
         assert _kind_of_c(c_ret) == _kind_of_ctypes(ret), name
     # and the binding covers every declared entry point
     assert set(protos) == set(binding._SIGNATURES)
+
+
+def test_binding_constants_match_the_header():
+    """The status codes, device bits and limits the binding names have the
+    header's values."""
+    from activation_sparsity_b200 import larosa as binding
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    values = {m.group(1): int(m.group(2), 0)
+              for m in re.finditer(r"#define\s+(LAROSA_\w+)\s+(0x[0-9a-fA-F]+|\d+)", text)}
+    values.update({m.group(1): int(m.group(2)) for m in re.finditer(r"\b(LAROSA_[A-Z_]+)\s*=\s*(\d+)", text)})
+    checked = 0
+    for name in dir(binding):
+        if name.startswith("LAROSA_") and name in values:
+            assert getattr(binding, name) == values[name], name
+            checked += 1
+    assert checked >= 12
