@@ -232,10 +232,12 @@ def test_binding_constants_match_the_header():
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
     values = {m.group(1): int(m.group(2), 0)
               for m in re.finditer(r"#define\s+(LAROSA_\w+)\s+(0x[0-9a-fA-F]+|\d+)", text)}
-    values.update({m.group(1): int(m.group(2)) for m in re.finditer(r"\b(LAROSA_[A-Z_]+)\s*=\s*(\d+)", text)})
+    values.update({m.group(1): int(m.group(2)) for m in re.finditer(r"\b(LAROSA_[A-Z0-9_]+)\s*=\s*(\d+)", text)})
+    values.update({m.group(1): int(m.group(2)) << int(m.group(3))
+                   for m in re.finditer(r"#define\s+(LAROSA_\w+)\s+\((\d+)u?\s*<<\s*(\d+)\)", text)})
     checked = 0
     for name in dir(binding):
         if name.startswith("LAROSA_") and name in values:
             assert getattr(binding, name) == values[name], name
             checked += 1
-    assert checked >= 12
+    assert checked >= 15
