@@ -18,8 +18,16 @@ rotations and kept weight rows per step) exceeds the 126 MB L2, so no flush is
 needed.  N > 1 runs N independent replicas (one process per GPU, no data-path
 collective); the reported time is the maximum over ranks.
 
-Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
-on the same workload instead (the only other path that may run it here).
+Rank 0 prints one JSON line.  Besides the headline it carries, from the same
+run: the roofline of the fused kernel (with the DRAM traffic of the committed
+ncu capture), the end-to-end rate through the Python API with host copies,
+the component kernels, the comparison modes (threshold selection, identity
+and folded rotation, sparse + low rank; the threshold and low-rank modes also
+at 16 tokens per call), the sparsity and batch sweeps, the other workloads
+(a 32-layer 7B stack, a 13B layer at 1 to 16 tokens, an 8-layer 70B slice,
+each with the dense GEMV and the folded path), a pure-read probe, clocks and
+the CPU oracle's rate.  ``--impl reference`` times the fp64 CPU oracle on the
+same workload instead (the only other path that may run it here).
 """
 from __future__ import annotations
 
