@@ -24,8 +24,8 @@ ncu capture), the end-to-end rate through the Python API with host copies,
 the component kernels, the comparison modes (threshold selection, identity
 and folded rotation, sparse + low rank; the threshold and low-rank modes also
 at 16 tokens per call), the sparsity and batch sweeps, the other workloads
-(a 32-layer 7B stack, a 13B layer at 1 to 16 tokens, an 8-layer 70B slice,
-each with the dense GEMV and the folded path), a pure-read probe, clocks and
+(a 32-layer 7B stack and an 8-layer 70B slice, each with the dense GEMV and
+the folded path; a 13B layer at 1 to 16 tokens), a pure-read probe, clocks and
 the CPU oracle's rate.  ``--impl reference`` times the fp64 CPU oracle on the
 same workload instead (the only other path that may run it here).
 """
